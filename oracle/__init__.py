@@ -1,0 +1,8 @@
+"""CPU oracle for the VC-Attention forward path.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package. The product path (``bit_fp8_attention_prep_b200``) never imports it and
+shares no code with it.
+"""
+from .vc_oracle import *  # noqa: F401,F403

@@ -1,0 +1,200 @@
+"""Pins for the oracle's V-Smooth prep and Q/K quantisation (CPU only).
+
+Brute force with exact rational arithmetic on tiny inputs, a published
+splitmix64 output, and the closed-form properties of each step.
+"""
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from bit_fp8_attention_prep_b200 import synth
+
+
+def _bf16_values(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(shape, generator=g) * scale).to(torch.bfloat16).float().numpy()
+    # keep every value on the 2^-24 fixed-point grid (|x| >= 2^-17 or 0) so that
+    # the fixed-point sums are the exact sums
+    x[np.abs(x) < 2.0 ** -16] = 0.0
+    return x
+
+
+def test_splitmix64_published_outputs():
+    # First two outputs of the splitmix64 reference implementation from state 0.
+    r = O.SplitMix64(0)
+    assert r.next() == 0xE220A8397B1DCDAF
+    assert r.next() == 0x6E789E6AA1B965F4
+
+
+def test_init_indices_distinct_in_range_and_seeded():
+    for S, k in [(256, 4), (4096, 16), (73397, 16), (5, 5)]:
+        idx = O.kmeans_init_indices(S, k, 0, 3)
+        assert len(idx) == k and len(set(idx)) == k and all(0 <= i < S for i in idx)
+    assert O.kmeans_init_indices(4096, 16, 0, 0) != O.kmeans_init_indices(4096, 16, 0, 1)
+    assert O.kmeans_init_indices(4096, 16, 0, 0) != O.kmeans_init_indices(4096, 16, 1, 0)
+    assert O.kmeans_init_indices(4096, 16, 7, 2) == O.kmeans_init_indices(4096, 16, 7, 2)
+    # fewer tokens than clusters: all tokens taken once, then repeats are allowed
+    idx = O.kmeans_init_indices(3, 8, 0, 0)
+    assert len(idx) == 8 and set(idx) == {0, 1, 2}
+
+
+def _exact_lloyd(X, k, iters, seed, bh):
+    """Lloyd's algorithm in exact rational arithmetic (brute force)."""
+    S, D = X.shape
+    C = [[Fraction(float(v)) for v in X[i]] for i in O.kmeans_init_indices(S, k, seed, bh)]
+    Xf = [[Fraction(float(v)) for v in row] for row in X]
+    hist = []
+    for t in range(iters):
+        a = []
+        for j in range(S):
+            d = [sum((Xf[j][e] - C[c][e]) ** 2 for e in range(D)) for c in range(k)]
+            a.append(min(range(k), key=lambda c: (d[c], c)))
+        hist.append(a)
+        if t < iters - 1:
+            for c in range(k):
+                mem = [j for j in range(S) if a[j] == c]
+                if mem:
+                    C[c] = [Fraction(float(np.float32(float(sum(Xf[j][e] for j in mem) / len(mem)))))
+                            for e in range(D)]
+    return hist, C
+
+
+@pytest.mark.parametrize("S,D,k,iters,seed", [(40, 3, 4, 3, 0), (64, 8, 5, 4, 1), (33, 128, 3, 3, 2)])
+def test_lloyd_matches_exact_brute_force(S, D, k, iters, seed):
+    # tight clusters so that Lloyd moves tokens between passes
+    X = _bf16_values((S, D), seed)
+    X[: S // 2] += 3.0
+    X = torch.from_numpy(X).to(torch.bfloat16).float().numpy()
+    a, C, hist, stats = O.kmeans_lloyd(X, k, iters, seed, bh=5)
+    ehist, eC = _exact_lloyd(X, k, iters, seed, bh=5)
+    for t in range(iters):
+        assert list(hist[t]) == ehist[t]
+    assert stats == {"near_ties": 0, "mismatches": 0}
+
+
+def test_lloyd_centroid_is_rounded_exact_mean():
+    X = _bf16_values((300, 128), 4)
+    a = np.arange(300) % 7
+    Xfix = np.rint(X.astype(np.float64) * 2.0 ** 24).astype(np.int64)
+    C = O.centroid_update(Xfix, a, np.zeros((8, 128), np.float32), 8)
+    for c in range(7):
+        mem = X[a == c]
+        for e in (0, 17, 127):
+            exact = sum(Fraction(float(v)) for v in mem[:, e]) / len(mem)
+            assert C[c, e] == np.float32(float(exact))
+    assert np.all(C[7] == 0)          # empty cluster keeps its centroid
+
+
+def test_lloyd_recovers_separated_mixture_labels():
+    cfg, Q, K, V = synth.make_workload("mid", B=1, H=1, S=2048)
+    X = V[0, :, 0].float().numpy()
+    a, C, hist, stats = O.kmeans_lloyd(X, 16, 4, 0, 0)
+    # each found cluster should be dominated by one generator centre: measure the
+    # purity against a nearest-centre labelling of the (outlier-free) tokens
+    norms = np.linalg.norm(X, axis=1)
+    keep = norms < np.percentile(norms, 95)
+    # tokens of the same found cluster are close together
+    spread = [np.mean(np.linalg.norm(X[keep & (a == c)] - C[c], axis=1)) for c in range(16)
+              if (keep & (a == c)).sum() > 5]
+    assert np.median(spread) < 0.3 * np.sqrt(128) * 1.5
+
+
+def test_permutation_is_stable_sort():
+    rng = np.random.default_rng(5)
+    for S, k in [(1, 1), (257, 4), (1000, 16)]:
+        a = rng.integers(0, k, S)
+        perm = O.cluster_permutation(a)
+        assert list(perm) == sorted(range(S), key=lambda j: (a[j], j))
+
+
+def test_block_means_exact_and_tail():
+    X = _bf16_values((300, 128), 6, scale=3.0)
+    perm = np.random.default_rng(6).permutation(300).astype(np.int32)
+    mu = O.block_means(X, perm)
+    assert mu.shape == (3, 128)
+    for b, (lo, hi) in enumerate([(0, 128), (128, 256), (256, 300)]):
+        rows = X[perm[lo:hi]]
+        for e in (0, 64, 127):
+            exact = sum(Fraction(float(v)) for v in rows[:, e]) / (hi - lo)
+            assert mu[b, e] == np.float32(float(exact))
+
+
+def _nearest_code_brute(v, tab, ncodes):
+    d = np.abs(tab[:ncodes] - v)
+    best = np.flatnonzero(d == d.min())
+    return best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+
+
+def test_residual_e4m3_codes_are_nearest_and_amax_maps_to_max():
+    X = _bf16_values((300, 128), 7, scale=2.0)
+    perm = np.random.default_rng(7).permutation(300).astype(np.int32)
+    mu = O.block_means(X, perm)
+    vt, s_v, amax = O.residual_e4m3(X, perm, mu)
+    assert vt.shape == (128, 384) and np.all(vt[:, 300:] == 0)
+    r = X[perm] - mu[np.arange(300) // 128]
+    assert amax == np.max(np.abs(r))
+    assert s_v == amax / np.float32(448)
+    tab = O.e4m3_table()
+    inv = np.float32(448) / amax
+    jmax, emax = np.unravel_index(np.argmax(np.abs(r)), r.shape)
+    assert vt[emax, jmax] & 0x7F == 0x7E
+    rng = np.random.default_rng(8)
+    for _ in range(300):
+        j, e = rng.integers(0, 300), rng.integers(0, 128)
+        v = float(np.float32(r[j, e] * inv))
+        want = _nearest_code_brute(abs(v), tab, 127) | (0x80 if math.copysign(1, v) < 0 else 0)
+        assert vt[e, j] == want
+
+
+def test_residual_nvfp4_brute_force_and_fp16_exactness():
+    X = _bf16_values((200, 128), 9, scale=2.0)
+    perm = np.arange(200, dtype=np.int32)[::-1].copy()
+    mu = O.block_means(X, perm)
+    packed, scales, g, amax = O.residual_nvfp4(X, perm, mu)
+    assert packed.shape == (128, 128) and scales.shape == (128, 16)
+    r = X[perm] - mu[np.arange(200) // 128]
+    assert g == amax / np.float32(2688)
+    t4, t8 = O.e2m1_table(), O.e4m3_table()
+    codes = np.empty((128, 256), np.uint8)
+    codes[:, 0::2], codes[:, 1::2] = packed & 15, packed >> 4
+    rng = np.random.default_rng(10)
+    for _ in range(200):
+        e, grp = rng.integers(0, 128), rng.integers(0, 200 // 16)
+        vals = np.zeros(16, np.float32)
+        n = min(16, 200 - 16 * grp)
+        vals[:n] = r[16 * grp:16 * grp + n, e]
+        target = float(np.float32(np.float32(np.max(np.abs(vals)) / np.float32(6)) / g))
+        assert scales[e, grp] == _nearest_code_brute(target, t8, 127)
+        den = np.float32(np.float32(t8[scales[e, grp]]) * g)
+        for i in range(16):
+            q = float(np.float32(vals[i] / den))
+            want = _nearest_code_brute(min(abs(q), 6.0), t4, 8) | (8 if math.copysign(1, q) < 0 else 0)
+            assert codes[e, 16 * grp + i] == want
+    # every e2m1 x (positive) E4M3 product is exact in fp16, so the PV operand can
+    # be dequantised exactly
+    prods = np.outer(t4[:8], t8[:127])
+    assert np.array_equal(prods.astype(np.float16).astype(np.float64), prods)
+
+
+def test_quant_blocks_scales_codes_and_zero_block():
+    X = _bf16_values((300, 128), 11)
+    X[128:256] = 0.0
+    perm = np.random.default_rng(11).permutation(300).astype(np.int32)
+    codes, scales = O.quant_blocks_e4m3(X, order=perm)
+    Xp = X[perm]
+    assert codes.shape == (384, 128) and np.all(codes[300:] == 0)
+    tab = O.e4m3_table()
+    for b, (lo, hi) in enumerate([(0, 128), (128, 256), (256, 300)]):
+        amax = np.max(np.abs(Xp[lo:hi]))
+        if amax == 0:
+            assert scales[b] == 1.0 and np.all(codes[lo:hi] == 0)
+            continue
+        assert scales[b] == amax / np.float32(448)
+        deq = tab[codes[lo:hi]] * float(scales[b])
+        # E4M3 keeps 3 mantissa bits: relative error <= 2^-4 (normals), plus the
+        # subnormal half-step
+        assert np.all(np.abs(deq - Xp[lo:hi]) <= 2.0 ** -4 * np.abs(Xp[lo:hi]) + 2.0 ** -10 * scales[b] + 1e-30)
