@@ -1,0 +1,285 @@
+// vc_api.cu -- host side of the C ABI declared in include/vc_attn.h: argument
+// validation, workspace carving, TMA descriptor encoding and kernel launches.
+// Nothing here allocates device memory or synchronises the device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+
+#include "../../include/vc_attn.h"
+#include "vc_kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+vc_status_t fail(vc_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+vc_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(VC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int nblocks(int S) { return (S + 127) / 128; }
+
+vc_status_t check_shape(const vc_shape_t* sh) {
+  if (!sh) return fail(VC_ERR_INVALID_ARG, "shape is NULL");
+  if (sh->D != 128) return fail(VC_ERR_INVALID_ARG, "D must be 128 (got %d)", sh->D);
+  if (sh->B < 1 || sh->S < 1 || sh->H < 1)
+    return fail(VC_ERR_INVALID_ARG, "B, S, H must be >= 1 (got %d, %d, %d)", sh->B, sh->S, sh->H);
+  if (sh->dtype != VC_DTYPE_F16 && sh->dtype != VC_DTYPE_BF16)
+    return fail(VC_ERR_INVALID_ARG, "dtype must be VC_DTYPE_F16 or VC_DTYPE_BF16 (got %d)", sh->dtype);
+  const long long n = (long long)sh->B * sh->H * nblocks(sh->S) * 128 * 128;
+  if (n >= (1ll << 31)) return fail(VC_ERR_INVALID_ARG, "B*H*S_pad*128 = %lld exceeds 2^31", n);
+  return VC_OK;
+}
+
+vc_status_t check_cfg(const vc_vsmooth_cfg_t* cfg) {
+  if (!cfg) return fail(VC_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->mode != VC_MODE_VSMOOTH && cfg->mode != VC_MODE_MEANONLY)
+    return fail(VC_ERR_INVALID_ARG, "mode must be VC_MODE_VSMOOTH or VC_MODE_MEANONLY (got %d)", cfg->mode);
+  if (cfg->mode == VC_MODE_VSMOOTH) {
+    if (cfg->k < 1 || cfg->k > vc::kMaxClusters)
+      return fail(VC_ERR_INVALID_ARG, "k must be in [1, %d] (got %d)", vc::kMaxClusters, cfg->k);
+    if (cfg->iters < 1 || cfg->iters > 64) return fail(VC_ERR_INVALID_ARG, "iters must be in [1, 64] (got %d)", cfg->iters);
+  }
+  if (cfg->residual_fmt != VC_RESIDUAL_E4M3 && cfg->residual_fmt != VC_RESIDUAL_NVFP4)
+    return fail(VC_ERR_INVALID_ARG, "residual_fmt must be VC_RESIDUAL_E4M3 or VC_RESIDUAL_NVFP4");
+  return VC_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace layout of vc_attn_prepare_v (every piece 256-B aligned).
+struct WsLayout {
+  size_t cent, sums, counts, assign, hist, offs, amax, total;
+};
+
+WsLayout ws_layout(const vc_shape_t* sh, const vc_vsmooth_cfg_t* cfg) {
+  const size_t BH = (size_t)sh->B * sh->H;
+  const size_t k = cfg->mode == VC_MODE_VSMOOTH ? (size_t)cfg->k : 1;
+  const size_t nch = (size_t)((sh->S + vc::kChunk - 1) / vc::kChunk);
+  WsLayout w;
+  size_t off = 0;
+  w.cent = off;   off += align256(BH * k * 128 * 4);
+  w.sums = off;   off += align256(BH * k * 128 * 8);
+  w.counts = off; off += align256(BH * k * 4);
+  w.assign = off; off += align256(BH * (size_t)sh->S);
+  w.hist = off;   off += align256(BH * nch * k * 4);
+  w.offs = off;   off += align256(BH * nch * k * 4);
+  w.amax = off;   off += align256(BH * 4);
+  w.total = off;
+  return w;
+}
+
+// Per-device one-time set-up: the device must be sm_100 and the kernels' shared
+// memory limits raised.
+std::mutex g_mu;
+int g_ready[64];  // 0 unknown, 1 ready, -1 unsupported
+
+vc_status_t ensure_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(VC_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_ready[dev] == 1) return VC_OK;
+  if (g_ready[dev] == -1) return fail(VC_ERR_UNSUPPORTED, "device %d is not an sm_100 GPU", dev);
+  int major = 0, minor = 0;
+  if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetAttribute");
+  if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetAttribute");
+  if (major != 10 || minor != 0) {
+    g_ready[dev] = -1;
+    return fail(VC_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev, major, minor);
+  }
+  if ((e = vc::prep_configure()) != cudaSuccess) return cuda_fail(e, "configuring prep kernels");
+  if ((e = vc::attn_configure()) != cudaSuccess) return cuda_fail(e, "configuring attention kernel");
+  g_ready[dev] = 1;
+  return VC_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D uint8 tensor map: rows of `inner` bytes, `rows` rows, 128 x 128 byte box,
+// 128-byte swizzle (the canonical K-major UMMA operand layout).
+vc_status_t make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(VC_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(VC_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return VC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t vc_attn_version(void) { return 100; }
+
+const char* vc_attn_last_error(void) { return g_last_error.c_str(); }
+
+size_t vc_attn_prepare_v_workspace_bytes(const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg) {
+  if (check_shape(shape) != VC_OK || check_cfg(cfg) != VC_OK) return 0;
+  return ws_layout(shape, cfg).total;
+}
+
+vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                              const vc_prepared_v_t* out, void* workspace, size_t workspace_bytes,
+                              uint8_t* assign_history, void* stream) {
+  g_last_error.clear();
+  vc_status_t st;
+  if ((st = check_shape(shape)) != VC_OK) return st;
+  if ((st = check_cfg(cfg)) != VC_OK) return st;
+  if (!v || !out || !out->perm || !out->mu || !out->v_codes || !out->s_v)
+    return fail(VC_ERR_INVALID_ARG, "v, out, out->perm, out->mu, out->v_codes and out->s_v must be non-NULL");
+  if (cfg->residual_fmt == VC_RESIDUAL_NVFP4 && !out->v_scales)
+    return fail(VC_ERR_INVALID_ARG, "out->v_scales must be non-NULL for the NVFP4 residual");
+  if (!aligned16(v) || !aligned16(out->perm) || !aligned16(out->mu) || !aligned16(out->v_codes) ||
+      !aligned16(out->s_v) || (out->v_scales && !aligned16(out->v_scales)))
+    return fail(VC_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  const WsLayout w = ws_layout(shape, cfg);
+  if (!workspace || workspace_bytes < w.total)
+    return fail(VC_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total,
+                workspace ? workspace_bytes : (size_t)0);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(VC_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if ((st = ensure_device()) != VC_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  vc::PrepPlan pl;
+  pl.B = shape->B;
+  pl.S = shape->S;
+  pl.H = shape->H;
+  pl.k = cfg->mode == VC_MODE_VSMOOTH ? cfg->k : 1;
+  pl.iters = cfg->iters;
+  pl.fmt = cfg->residual_fmt;
+  pl.mode = cfg->mode;
+  pl.seed = cfg->seed;
+  pl.nb = nblocks(shape->S);
+  pl.S_pad = pl.nb * 128;
+  pl.nchunks = (shape->S + vc::kChunk - 1) / vc::kChunk;
+  pl.cent = reinterpret_cast<float*>(ws + w.cent);
+  pl.sums = reinterpret_cast<unsigned long long*>(ws + w.sums);
+  pl.counts = reinterpret_cast<int*>(ws + w.counts);
+  pl.assign = ws + w.assign;
+  pl.hist = reinterpret_cast<int*>(ws + w.hist);
+  pl.offs = reinterpret_cast<int*>(ws + w.offs);
+  pl.amax = reinterpret_cast<unsigned int*>(ws + w.amax);
+  cudaError_t e = vc::launch_prepare_v(v, shape->dtype, pl, *out, assign_history, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "launching V-Smooth prep");
+  return VC_OK;
+}
+
+vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* shape, const int32_t* perm,
+                             const vc_qk_fp8_t* out, void* stream) {
+  g_last_error.clear();
+  vc_status_t st;
+  if ((st = check_shape(shape)) != VC_OK) return st;
+  if (!q || !k || !perm || !out || !out->q_codes || !out->q_scales || !out->k_codes || !out->k_scales)
+    return fail(VC_ERR_INVALID_ARG, "q, k, perm, out and every field of out must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(perm) || !aligned16(out->q_codes) || !aligned16(out->k_codes) ||
+      !aligned16(out->q_scales) || !aligned16(out->k_scales))
+    return fail(VC_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if ((st = ensure_device()) != VC_OK) return st;
+  cudaError_t e = vc::launch_quant_qk(q, k, shape->dtype, shape->B, shape->S, shape->H, perm, *out,
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "launching Q/K quantisation");
+  return VC_OK;
+}
+
+static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
+                                  float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream,
+                                  bool nvfp4) {
+  g_last_error.clear();
+  vc_status_t st;
+  if ((st = check_shape(shape)) != VC_OK) return st;
+  if (!qk || !pv || !o) return fail(VC_ERR_INVALID_ARG, "qk, pv and o must be non-NULL");
+  if (!qk->q_codes || !qk->q_scales || !qk->k_codes || !qk->k_scales || !pv->mu || !pv->v_codes || !pv->s_v)
+    return fail(VC_ERR_INVALID_ARG, "a required field of qk or pv is NULL");
+  if (nvfp4 && !pv->v_scales) return fail(VC_ERR_INVALID_ARG, "pv->v_scales must be non-NULL for NVFP4");
+  if (!aligned16(o) || !aligned16(qk->q_codes) || !aligned16(qk->k_codes) || !aligned16(pv->v_codes) ||
+      !aligned16(pv->mu) || (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)))
+    return fail(VC_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.0f) || !(softmax_scale < 1e30f))
+    return fail(VC_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
+  if (k_p < 0 || k_p > 8) return fail(VC_ERR_INVALID_ARG, "k_p must be in [0, 8] (got %d)", k_p);
+  if ((st = ensure_device()) != VC_OK) return st;
+  const int nb = nblocks(shape->S), S_pad = nb * 128, BH = shape->B * shape->H;
+  CUtensorMap tq, tk, tv;
+  if ((st = make_map_u8(&tq, qk->q_codes, 128, (uint64_t)BH * S_pad)) != VC_OK) return st;
+  if ((st = make_map_u8(&tk, qk->k_codes, 128, (uint64_t)BH * S_pad)) != VC_OK) return st;
+  vc::AttnParams p;
+  p.B = shape->B;
+  p.S = shape->S;
+  p.H = shape->H;
+  p.nb = nb;
+  p.S_pad = S_pad;
+  p.q_scales = qk->q_scales;
+  p.k_scales = qk->k_scales;
+  p.mu = pv->mu;
+  p.s_v = pv->s_v;
+  p.v_scales = pv->v_scales;
+  p.kappa = (float)((double)softmax_scale * 1.4426950408889634);
+  p.bias_b = 56 + 8 * k_p;
+  p.o = o;
+  p.status = dev_status;
+  p.wait_ns = 2000000000ull;
+  cudaError_t e;
+  if (!nvfp4) {
+    if ((st = make_map_u8(&tv, pv->v_codes, (uint64_t)S_pad, (uint64_t)BH * 128)) != VC_OK) return st;
+    e = vc::launch_attn_e4m3(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  } else {
+    e = vc::launch_attn_nvfp4(tq, tk, pv->v_codes, p, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return fail(VC_ERR_UNSUPPORTED, "NVFP4-V attention is not built yet");
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "launching attention");
+  return VC_OK;
+}
+
+vc_status_t vc_attn_forward(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
+                            float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, false);
+}
+
+vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
+                                   float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, true);
+}
+
+}  // extern "C"

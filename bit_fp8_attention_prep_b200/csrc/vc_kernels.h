@@ -1,0 +1,64 @@
+// vc_kernels.h -- internal launch interface between the C ABI (vc_api.cu) and
+// the kernels (vc_prep.cu, vc_attn_fwd.cu). Not installed, not part of the ABI.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "../../include/vc_attn.h"
+
+namespace vc {
+
+constexpr int kMaxClusters = 32;   // k-means clusters per (b, h)
+constexpr int kChunk = 1024;       // tokens per k-means CTA (also the sort's chunk)
+
+// Device buffers and sizes of one vc_attn_prepare_v call; the pointers are
+// carved from the caller's workspace.
+struct PrepPlan {
+  int B, S, H, k, iters, fmt, mode;
+  uint64_t seed;
+  int nb, S_pad, nchunks;
+  float* cent;                 // [BH][k][128]
+  unsigned long long* sums;    // [BH][k][128] int64 fixed-point
+  int* counts;                 // [BH][k]
+  uint8_t* assign;             // [BH][S]
+  int* hist;                   // [BH][nchunks][k]
+  int* offs;                   // [BH][nchunks][k]
+  unsigned int* amax;          // [BH] fp32 bits
+};
+
+inline size_t assign_smem_bytes(int k, bool accum) {
+  return (size_t)k * 128 * 4 + (size_t)256 * 272 + (accum ? (size_t)k * 128 * 8 : 0) + kMaxClusters * 4 + 256;
+}
+
+cudaError_t prep_configure();
+cudaError_t launch_prepare_v(const void* v, int dtype, const PrepPlan& plan, const vc_prepared_v_t& out,
+                             uint8_t* history, cudaStream_t st);
+cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int S, int H, const int32_t* perm,
+                            const vc_qk_fp8_t& out, cudaStream_t st);
+
+// Attention forward.
+struct AttnParams {
+  int B, S, H, nb, S_pad;
+  const float* q_scales;   // [BH][nb]
+  const float* k_scales;   // [BH][nb]
+  const float* mu;         // [BH][nb][128]
+  const float* s_v;        // [BH]
+  const uint8_t* v_scales; // NVFP4: [BH][128][S_pad/16]
+  float kappa;             // fl32(softmax_scale * log2 e)
+  int bias_b;              // 56 + 8 k_P
+  void* o;                 // bf16 [B][S][H][128]
+  int32_t* status;         // optional device status word
+  uint64_t wait_ns;        // bound on every in-kernel wait
+};
+
+cudaError_t attn_configure();
+cudaError_t launch_attn_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const AttnParams& p, cudaStream_t st);
+cudaError_t launch_attn_nvfp4(const CUtensorMap& tq, const CUtensorMap& tk, const uint8_t* v_codes,
+                              const AttnParams& p, cudaStream_t st);
+
+}  // namespace vc

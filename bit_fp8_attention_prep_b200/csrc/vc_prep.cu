@@ -1,0 +1,555 @@
+// vc_prep.cu -- V-Smooth prep and Q/K FP8 quantisation kernels (sm_100a).
+//
+// V-Smooth ("VC-Attention: Value Smoothing and Softmax Casting for Low-bit
+// Attention", Abstract; "Nunchux AI lanza VC-Attention kernel ...", second
+// paragraph): per (batch, head), k-means over the value tokens, a stable sort of
+// the tokens by cluster, the mean of every 128-token block of the sorted order,
+// and E4M3 / NVFP4 codes of the residual. Q/K: one E4M3 scale per 128-row block
+// ("Open VC Attention", "Описание": Q/K scales per block).
+//
+// Readings where the pages are silent: k-means init indices come from
+// splitmix64 seeded by seed ^ (0x9E3779B97F4A7C15 * (b*H + h + 1)), redrawn
+// while they repeat; assignment ties go to the lowest cluster index; centroid and
+// block-mean sums are int64 sums of llrint(x * 2^24) (exact and order-free), then
+// one double division, rounded to fp32; an empty cluster keeps its centroid; the
+// last pass's assignment is final; the residual scale is one per (b, h); a block
+// whose amax is below 2^-100 is all zero.
+//
+// Every kernel reads Q, K, V in the caller's [B, S, H, 128] layout (a token is a
+// contiguous 256-byte row for one head; rows of one head are H*256 bytes apart).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "vc_common.cuh"
+#include "vc_kernels.h"
+
+namespace vc {
+
+// --------------------------------------------------------------- k-means init
+__device__ __forceinline__ uint64_t splitmix64_next(uint64_t& state) {
+  state += 0x9E3779B97F4A7C15ull;
+  uint64_t z = state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) kmeans_init_kernel(const T* __restrict__ v, int S, int H, int k,
+                                                          uint64_t seed, float* __restrict__ cent) {
+  __shared__ int idx[kMaxClusters];
+  const int bh = blockIdx.x, b = bh / H, h = bh % H;
+  if (threadIdx.x == 0) {
+    uint64_t st = seed ^ (0x9E3779B97F4A7C15ull * (uint64_t)(bh + 1));
+    for (int i = 0; i < k; ++i) {
+      int u;
+      while (true) {
+        u = (int)(splitmix64_next(st) % (uint64_t)S);
+        bool dup = false;
+        for (int j = 0; j < i; ++j) dup |= (idx[j] == u);
+        if (!dup || i >= S) break;
+      }
+      idx[i] = u;
+    }
+  }
+  __syncthreads();
+  const int d = threadIdx.x;
+  for (int i = 0; i < k; ++i) {
+    const size_t off = (((size_t)b * S + idx[i]) * H + h) * kD + d;
+    cent[((size_t)bh * k + i) * kD + d] = to_f32<T>(v[off]);
+  }
+}
+
+// --------------------------------------------------------------- k-means assign
+// One CTA = one chunk of kChunk tokens of one (b, h), in tiles of kTile tokens.
+// A tile is staged in shared memory with coalesced 16-byte loads; each thread
+// then holds one token (128 fp32 in registers) and computes the squared fp32
+// distance to every centroid with packed f32x2 arithmetic; the nearest centroid
+// (lowest index on ties) is the assignment. When `accumulate` is set, the
+// tile's tokens are added to per-CTA int64 fixed-point sums (dimension-parallel:
+// lane l owns dimensions 4l..4l+3) that are flushed to global sums at the end.
+constexpr int kTile = 256;
+constexpr int kTileStride = 272;  // bytes per staged row (256 + 16: conflict-free 16-B reads)
+
+template <typename T, bool kAccum>
+__global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restrict__ v, int S, int H, int k,
+                                                              const float* __restrict__ cent,
+                                                              unsigned long long* __restrict__ sums,
+                                                              int* __restrict__ counts, uint8_t* __restrict__ assign,
+                                                              int* __restrict__ hist, uint8_t* __restrict__ history) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  float* negc = reinterpret_cast<float*>(smem);                                   // [k][128]
+  uint8_t* tile = smem + (size_t)k * kD * 4;                                     // [kTile][272]
+  long long* ssum = reinterpret_cast<long long*>(tile + (size_t)kTile * kTileStride);  // [k][128]
+  int* scount = reinterpret_cast<int*>(ssum + (kAccum ? (size_t)k * kD : 0));        // [k]
+  uint8_t* tassign = reinterpret_cast<uint8_t*>(scount + kMaxClusters);              // [kTile]
+
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int chunk = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t row_stride = (size_t)H * kD;  // elements between consecutive tokens of one head
+  const T* vbase = v + ((size_t)b * S * H + h) * kD;
+
+  for (int i = tid; i < k * kD; i += kTile) negc[i] = -cent[(size_t)bh * k * kD + i];
+  if (kAccum)
+    for (int i = tid; i < k * kD; i += kTile) ssum[i] = 0;
+  if (tid < kMaxClusters) scount[tid] = 0;
+
+  const int s_chunk0 = chunk * kChunk;
+  const int s_chunk1 = min(S, s_chunk0 + kChunk);
+  for (int s0 = s_chunk0; s0 < s_chunk1; s0 += kTile) {
+    const int ntok = min(kTile, s_chunk1 - s0);
+    __syncthreads();
+    // stage the tile: 16 x 16-byte pieces per token, a warp covers two tokens
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+      const int idx = i * kTile + tid, r = idx >> 4, c = idx & 15;
+      if (r < ntok) {
+        const uint4 val = *reinterpret_cast<const uint4*>(vbase + (size_t)(s0 + r) * row_stride + c * 8);
+        *reinterpret_cast<uint4*>(tile + r * kTileStride + c * 16) = val;
+      }
+    }
+    __syncthreads();
+    if (tid < ntok) {
+      float2 x[64];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        float f[8];
+        unpack8<T>(*reinterpret_cast<const uint4*>(tile + tid * kTileStride + c * 16), f);
+        x[4 * c + 0] = make_float2(f[0], f[1]);
+        x[4 * c + 1] = make_float2(f[2], f[3]);
+        x[4 * c + 2] = make_float2(f[4], f[5]);
+        x[4 * c + 3] = make_float2(f[6], f[7]);
+      }
+      float best_d = 0.0f;
+      int best = 0;
+      for (int c = 0; c < k; ++c) {
+        const float4* nc = reinterpret_cast<const float4*>(negc + c * kD);
+        float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float4 p = nc[i], q = nc[i + 1];
+          const float2 d0 = __fadd2_rn(x[2 * i + 0], make_float2(p.x, p.y));
+          const float2 d1 = __fadd2_rn(x[2 * i + 1], make_float2(p.z, p.w));
+          const float2 d2 = __fadd2_rn(x[2 * i + 2], make_float2(q.x, q.y));
+          const float2 d3 = __fadd2_rn(x[2 * i + 3], make_float2(q.z, q.w));
+          a0 = __ffma2_rn(d0, d0, a0);
+          a1 = __ffma2_rn(d1, d1, a1);
+          a2 = __ffma2_rn(d2, d2, a2);
+          a3 = __ffma2_rn(d3, d3, a3);
+        }
+        const float dist = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
+        if (c == 0 || dist < best_d) {
+          best_d = dist;
+          best = c;
+        }
+      }
+      tassign[tid] = (uint8_t)best;
+      assign[(size_t)bh * S + s0 + tid] = (uint8_t)best;
+      if (history) history[(size_t)bh * S + s0 + tid] = (uint8_t)best;
+      atomicAdd(&scount[best], 1);
+    }
+    if (kAccum) {
+      __syncthreads();
+      for (int r = warp; r < ntok; r += kTile / 32) {
+        const int c = tassign[r];
+        float f[4];
+        unpack4<T>(*reinterpret_cast<const uint2*>(tile + r * kTileStride + lane * 8), f);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const long long q = __float2ll_rn(f[e] * 16777216.0f);  // x * 2^24, exact
+          if (q != 0) atomicAdd(reinterpret_cast<unsigned long long*>(&ssum[c * kD + lane * 4 + e]),
+                                (unsigned long long)q);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (kAccum) {
+    for (int i = tid; i < k * kD; i += kTile)
+      if (ssum[i] != 0) atomicAdd(&sums[(size_t)bh * k * kD + i], (unsigned long long)ssum[i]);
+    if (tid < k && scount[tid] != 0) atomicAdd(&counts[(size_t)bh * k + tid], scount[tid]);
+  } else if (hist != nullptr && tid < k) {
+    hist[((size_t)bh * gridDim.x + chunk) * k + tid] = scount[tid];
+  }
+}
+
+// --------------------------------------------------------------- centroid update
+__global__ void __launch_bounds__(128) kmeans_update_kernel(int k, float* __restrict__ cent,
+                                                            unsigned long long* __restrict__ sums,
+                                                            int* __restrict__ counts) {
+  const int bh = blockIdx.x, d = threadIdx.x;
+  for (int c = 0; c < k; ++c) {
+    const int n = counts[(size_t)bh * k + c];
+    const size_t i = ((size_t)bh * k + c) * kD + d;
+    if (n > 0) {
+      const double s = (double)(long long)sums[i] * 5.9604644775390625e-08;  // * 2^-24, exact
+      cent[i] = __double2float_rn(__ddiv_rn(s, (double)n));
+    }
+    sums[i] = 0ull;
+  }
+  __syncthreads();
+  if (d < k) counts[(size_t)bh * k + d] = 0;
+}
+
+// --------------------------------------------------------------- stable cluster sort
+// offs[bh][chunk][c] = (tokens of clusters < c) + (tokens of cluster c in earlier chunks)
+__global__ void __launch_bounds__(32) perm_offsets_kernel(int k, int nchunks, const int* __restrict__ hist,
+                                                          int* __restrict__ offs) {
+  const int bh = blockIdx.x, c = threadIdx.x;
+  int total = 0;
+  if (c < k)
+    for (int ch = 0; ch < nchunks; ++ch) total += hist[((size_t)bh * nchunks + ch) * k + c];
+  // exclusive scan of the cluster totals across the warp
+  int incl = total;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (c >= o) incl += t;
+  }
+  int run = incl - total;
+  if (c < k)
+    for (int ch = 0; ch < nchunks; ++ch) {
+      const size_t i = ((size_t)bh * nchunks + ch) * k + c;
+      const int n = hist[i];
+      offs[i] = run;
+      run += n;
+    }
+}
+
+// One CTA = one chunk of kChunk tokens; each warp ranks its 32 tokens with
+// match_any, warps are ordered by an exclusive scan of their per-cluster counts.
+__global__ void __launch_bounds__(kChunk) perm_scatter_kernel(int S, int k, const uint8_t* __restrict__ assign,
+                                                              const int* __restrict__ offs,
+                                                              int32_t* __restrict__ perm) {
+  __shared__ int wcount[kChunk / 32][kMaxClusters];
+  const int bh = blockIdx.y, chunk = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < (kChunk / 32) * kMaxClusters; i += kChunk) (&wcount[0][0])[i] = 0;
+  __syncthreads();
+  const int s = chunk * kChunk + tid;
+  const bool valid = s < S;
+  const int a = valid ? assign[(size_t)bh * S + s] : 0xFF;
+  const unsigned peers = __match_any_sync(0xffffffffu, a);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  if (valid && rank == 0) wcount[warp][a] = __popc(peers);
+  __syncthreads();
+  if (tid < k) {
+    int run = 0;
+    for (int w = 0; w < kChunk / 32; ++w) {
+      const int n = wcount[w][tid];
+      wcount[w][tid] = run;
+      run += n;
+    }
+  }
+  __syncthreads();
+  if (valid) {
+    const int pos = offs[((size_t)bh * gridDim.x + chunk) * k + a] + wcount[warp][a] + rank;
+    perm[(size_t)bh * S + pos] = s;
+  }
+}
+
+__global__ void identity_perm_kernel(int S, int32_t* __restrict__ perm) {
+  for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < S; s += gridDim.x * blockDim.x)
+    perm[(size_t)blockIdx.y * S + s] = s;
+}
+
+// --------------------------------------------------------------- block mean + residual amax
+// One CTA (4 warps) = one 128-token block of permuted positions. Warp w walks
+// rows 32w..32w+31; lane l owns dimensions 4l..4l+3 (one coalesced 256-B row per
+// warp load). Means use the int64 fixed-point sum; the residual amax is merged
+// into amax[bh] with an integer atomicMax on the (non-negative) fp32 bits.
+template <typename T>
+__global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ v, int S, int H,
+                                                          const int32_t* __restrict__ perm,
+                                                          float* __restrict__ mu,
+                                                          unsigned int* __restrict__ amax) {
+  __shared__ long long wsum[4][kD];
+  __shared__ float smu[kD];
+  __shared__ float wmax[4];
+  const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int p0 = blk * kBlock, cnt = min(kBlock, S - p0);
+  const size_t row_stride = (size_t)H * kD;
+  const T* vbase = v + ((size_t)b * S * H + h) * kD;
+  const int32_t* pbase = perm + (size_t)bh * S + p0;
+
+  long long acc[4] = {0, 0, 0, 0};
+  for (int r = warp; r < cnt; r += 4) {
+    const int src = pbase[r];
+    float f[4];
+    unpack4<T>(*reinterpret_cast<const uint2*>(vbase + (size_t)src * row_stride + lane * 4), f);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] += __float2ll_rn(f[e] * 16777216.0f);
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) wsum[warp][lane * 4 + e] = acc[e];
+  __syncthreads();
+  {
+    const int d = tid;
+    const long long s = wsum[0][d] + wsum[1][d] + wsum[2][d] + wsum[3][d];
+    const float m = __double2float_rn(__ddiv_rn((double)s * 5.9604644775390625e-08, (double)cnt));
+    smu[d] = m;
+    mu[((size_t)bh * gridDim.x + blk) * kD + d] = m;
+  }
+  __syncthreads();
+  float mx = 0.0f;
+  for (int r = warp; r < cnt; r += 4) {
+    const int src = pbase[r];
+    float f[4];
+    unpack4<T>(*reinterpret_cast<const uint2*>(vbase + (size_t)src * row_stride + lane * 4), f);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fabsf(__fsub_rn(f[e], smu[lane * 4 + e])));
+  }
+  mx = warp_max(mx);
+  if (lane == 0) wmax[warp] = mx;
+  __syncthreads();
+  if (tid == 0) {
+    const float m = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+    atomicMax(&amax[bh], __float_as_uint(m));
+  }
+}
+
+// --------------------------------------------------------------- residual E4M3
+// One CTA = one 128-token block; thread r owns permuted row r. Codes go to a
+// transposed shared tile and leave as V^T rows (128 contiguous tokens per
+// channel), the K-major B operand of the PV product.
+template <typename T>
+__global__ void __launch_bounds__(128) residual_e4m3_kernel(const T* __restrict__ v, int S, int H, int S_pad,
+                                                            const int32_t* __restrict__ perm,
+                                                            const float* __restrict__ mu,
+                                                            const unsigned int* __restrict__ amax_bits,
+                                                            uint8_t* __restrict__ vt, float* __restrict__ s_v) {
+  __shared__ __align__(16) uint8_t ct[kD][kBlock + 16];
+  __shared__ float smu[kD];
+  const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
+  const int r = threadIdx.x;
+  const int p = blk * kBlock + r;
+  const float amax = __uint_as_float(amax_bits[bh]);
+  const bool zero = !(amax >= kTinyAmax);
+  const float inv = zero ? 0.0f : __fdiv_rn(kE4M3Max, amax);
+  if (blk == 0 && r == 0) s_v[bh] = zero ? 1.0f : __fdiv_rn(amax, kE4M3Max);
+  smu[r] = mu[((size_t)bh * gridDim.x + blk) * kD + r];
+  __syncthreads();
+  if (p < S && !zero) {
+    const T* row = v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD;
+#pragma unroll 4
+    for (int c = 0; c < 16; ++c) {
+      float f[8];
+      unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), f);
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const int d = c * 8 + e;
+        const float r0 = __fsub_rn(f[e], smu[d]), r1 = __fsub_rn(f[e + 1], smu[d + 1]);
+        const uint16_t two = cvt_e4m3x2(__fmul_rn(r0, inv), __fmul_rn(r1, inv));
+        ct[d][r] = (uint8_t)(two & 0xFF);
+        ct[d + 1][r] = (uint8_t)(two >> 8);
+      }
+    }
+  } else {
+    for (int d = 0; d < kD; ++d) ct[d][r] = 0;
+  }
+  __syncthreads();
+  uint8_t* out = vt + (size_t)bh * kD * S_pad + (size_t)blk * kBlock;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int idx = i * 128 + r, d = idx >> 3, c = idx & 7;
+    *reinterpret_cast<uint4*>(out + (size_t)d * S_pad + c * 16) = *reinterpret_cast<const uint4*>(&ct[d][c * 16]);
+  }
+}
+
+// --------------------------------------------------------------- residual NVFP4
+// Global scale g = amax / (448 * 6) per (b, h); per channel and group of 16
+// consecutive permuted tokens an E4M3 scale s = E4M3(fl32(fl32(gmax/6)/g)), and
+// E2M1 codes of r / fl32(dec(s) * g) (0 where dec(s) == 0).
+template <typename T>
+__global__ void __launch_bounds__(128) residual_nvfp4_kernel(const T* __restrict__ v, int S, int H, int S_pad,
+                                                             const int32_t* __restrict__ perm,
+                                                             const float* __restrict__ mu,
+                                                             const unsigned int* __restrict__ amax_bits,
+                                                             uint8_t* __restrict__ codes,
+                                                             uint8_t* __restrict__ scales, float* __restrict__ gsc) {
+  extern __shared__ __align__(16) float rt[];  // [128 channels][129]
+  __shared__ float smu[kD];
+  const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
+  const int t = threadIdx.x;
+  const float amax = __uint_as_float(amax_bits[bh]);
+  const bool zero = !(amax >= kTinyAmax);
+  const float g = zero ? 1.0f : __fdiv_rn(amax, kE4M3Max * kE2M1Max);
+  if (blk == 0 && t == 0) gsc[bh] = g;
+  smu[t] = mu[((size_t)bh * gridDim.x + blk) * kD + t];
+  __syncthreads();
+  {
+    const int p = blk * kBlock + t;  // thread t: permuted row t
+    if (p < S && !zero) {
+      const T* row = v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD;
+#pragma unroll 4
+      for (int c = 0; c < 16; ++c) {
+        float f[8];
+        unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) rt[(c * 8 + e) * 129 + t] = __fsub_rn(f[e], smu[c * 8 + e]);
+      }
+    } else {
+      for (int d = 0; d < kD; ++d) rt[d * 129 + t] = 0.0f;
+    }
+  }
+  __syncthreads();
+  const int d = t;  // thread t: channel t
+  const float* rr = rt + d * 129;
+  uint8_t* crow = codes + ((size_t)bh * kD + d) * (S_pad / 2) + (size_t)blk * (kBlock / 2);
+  uint8_t* srow = scales + ((size_t)bh * kD + d) * (S_pad / kGroup4) + (size_t)blk * (kBlock / kGroup4);
+#pragma unroll 1
+  for (int gi = 0; gi < kBlock / kGroup4; ++gi) {
+    float gmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kGroup4; ++i) gmax = fmaxf(gmax, fabsf(rr[gi * kGroup4 + i]));
+    const uint8_t sc = zero ? 0 : cvt_e4m3(__fdiv_rn(__fdiv_rn(gmax, kE2M1Max), g));
+    const float den = __fmul_rn(e4m3_to_f32(sc), g);
+    uint32_t w[2] = {0u, 0u};
+    if (sc != 0) {
+#pragma unroll
+      for (int i = 0; i < kGroup4; i += 2) {
+        const uint32_t byte = cvt_e2m1x2(__fdiv_rn(rr[gi * kGroup4 + i], den), __fdiv_rn(rr[gi * kGroup4 + i + 1], den));
+        w[i >> 3] |= byte << (8 * ((i >> 1) & 3));
+      }
+    }
+    *reinterpret_cast<uint2*>(crow + gi * (kGroup4 / 2)) = make_uint2(w[0], w[1]);
+    srow[gi] = sc;
+  }
+}
+
+// --------------------------------------------------------------- Q/K quantisation
+// One CTA = one 128-row block of Q (original order) or K (gathered by perm);
+// thread r owns row r: load 128 values, block amax (warp max + shared), then
+// E4M3 codes of x * (448/amax), 128 contiguous bytes per row.
+template <typename T>
+__global__ void __launch_bounds__(128) quant_qk_kernel(const T* __restrict__ q, const T* __restrict__ k, int S,
+                                                       int H, int S_pad, const int32_t* __restrict__ perm,
+                                                       uint8_t* __restrict__ qc, float* __restrict__ qs,
+                                                       uint8_t* __restrict__ kc, float* __restrict__ ks) {
+  __shared__ float wmax[4];
+  const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
+  const bool is_k = blockIdx.z == 1;
+  const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
+  const int p = blk * kBlock + r;
+  const bool valid = p < S;
+  const int nbk = gridDim.x;
+  float x[kD];
+  float mx = 0.0f;
+  if (valid) {
+    const int src = is_k ? perm[(size_t)bh * S + p] : p;
+    const T* row = (is_k ? k : q) + (((size_t)b * S + src) * H + h) * kD;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), x + c * 8);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(x[c * 8 + e]));
+    }
+  }
+  mx = warp_max(mx);
+  if (lane == 0) wmax[warp] = mx;
+  __syncthreads();
+  const float amax = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+  const bool zero = !(amax >= kTinyAmax);
+  const float inv = zero ? 0.0f : __fdiv_rn(kE4M3Max, amax);
+  if (r == 0) (is_k ? ks : qs)[(size_t)bh * nbk + blk] = zero ? 1.0f : __fdiv_rn(amax, kE4M3Max);
+  uint8_t* out = (is_k ? kc : qc) + ((size_t)bh * S_pad + p) * kD;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = c * 16 + j * 4;
+      if (valid && !zero) {
+        const uint32_t lo = cvt_e4m3x2(__fmul_rn(x[e], inv), __fmul_rn(x[e + 1], inv));
+        const uint32_t hi = cvt_e4m3x2(__fmul_rn(x[e + 2], inv), __fmul_rn(x[e + 3], inv));
+        w[j] = lo | (hi << 16);
+      } else {
+        w[j] = 0u;
+      }
+    }
+    *reinterpret_cast<uint4*>(out + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// --------------------------------------------------------------- launchers
+template <typename T>
+static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_prepared_v_t& out,
+                                      uint8_t* history, cudaStream_t st) {
+  const int S = pl.S, H = pl.H, BH = pl.B * pl.H, k = pl.k;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(pl.amax, 0, sizeof(unsigned) * BH, st)) != cudaSuccess) return e;
+  if (pl.mode == VC_MODE_VSMOOTH) {
+    if ((e = cudaMemsetAsync(pl.sums, 0, sizeof(unsigned long long) * BH * k * kD, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(pl.counts, 0, sizeof(int) * BH * k, st)) != cudaSuccess) return e;
+    kmeans_init_kernel<T><<<BH, 128, 0, st>>>(v, S, H, k, pl.seed, pl.cent);
+    const dim3 grid(pl.nchunks, BH);
+    const size_t sm_acc = assign_smem_bytes(k, true), sm_fin = assign_smem_bytes(k, false);
+    for (int it = 0; it < pl.iters; ++it) {
+      uint8_t* hist_t = history ? history + (size_t)it * BH * S : nullptr;
+      if (it + 1 < pl.iters) {
+        kmeans_assign_kernel<T, true><<<grid, kTile, sm_acc, st>>>(v, S, H, k, pl.cent, pl.sums, pl.counts,
+                                                                   pl.assign, nullptr, hist_t);
+        kmeans_update_kernel<<<BH, 128, 0, st>>>(k, pl.cent, pl.sums, pl.counts);
+      } else {
+        kmeans_assign_kernel<T, false><<<grid, kTile, sm_fin, st>>>(v, S, H, k, pl.cent, pl.sums, pl.counts,
+                                                                    pl.assign, pl.hist, hist_t);
+      }
+    }
+    perm_offsets_kernel<<<BH, 32, 0, st>>>(k, pl.nchunks, pl.hist, pl.offs);
+    perm_scatter_kernel<<<grid, kChunk, 0, st>>>(S, k, pl.assign, pl.offs, out.perm);
+  } else {
+    identity_perm_kernel<<<dim3(std::max(1, std::min(1024, (S + 255) / 256)), BH), 256, 0, st>>>(S, out.perm);
+  }
+  const dim3 gb(pl.nb, BH);
+  block_stats_kernel<T><<<gb, 128, 0, st>>>(v, S, H, out.perm, out.mu, pl.amax);
+  if (pl.fmt == VC_RESIDUAL_E4M3) {
+    residual_e4m3_kernel<T><<<gb, 128, 0, st>>>(v, S, H, pl.S_pad, out.perm, out.mu, pl.amax, out.v_codes,
+                                                out.s_v);
+  } else {
+    residual_nvfp4_kernel<T><<<gb, 128, kD * 129 * sizeof(float), st>>>(v, S, H, pl.S_pad, out.perm, out.mu,
+                                                                         pl.amax, out.v_codes, out.v_scales,
+                                                                         out.s_v);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prepare_v(const void* v, int dtype, const PrepPlan& pl, const vc_prepared_v_t& out,
+                             uint8_t* history, cudaStream_t st) {
+  if (dtype == VC_DTYPE_BF16)
+    return launch_prepare_v_t(static_cast<const __nv_bfloat16*>(v), pl, out, history, st);
+  return launch_prepare_v_t(static_cast<const __half*>(v), pl, out, history, st);
+}
+
+cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int S, int H, const int32_t* perm,
+                            const vc_qk_fp8_t& out, cudaStream_t st) {
+  const int nb = (S + kBlock - 1) / kBlock;
+  const dim3 grid(nb, B * H, 2);
+  if (dtype == VC_DTYPE_BF16)
+    quant_qk_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), S, H, nb * kBlock, perm,
+        out.q_codes, out.q_scales, out.k_codes, out.k_scales);
+  else
+    quant_qk_kernel<__half><<<grid, 128, 0, st>>>(static_cast<const __half*>(q), static_cast<const __half*>(k), S,
+                                                  H, nb * kBlock, perm, out.q_codes, out.q_scales, out.k_codes,
+                                                  out.k_scales);
+  return cudaGetLastError();
+}
+
+cudaError_t prep_configure() {
+  cudaError_t e;
+  const size_t mx = assign_smem_bytes(kMaxClusters, true);
+  for (auto f : {(const void*)kmeans_assign_kernel<__nv_bfloat16, true>,
+                 (const void*)kmeans_assign_kernel<__nv_bfloat16, false>,
+                 (const void*)kmeans_assign_kernel<__half, true>, (const void*)kmeans_assign_kernel<__half, false>})
+    if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mx)) != cudaSuccess) return e;
+  for (auto f : {(const void*)residual_nvfp4_kernel<__nv_bfloat16>, (const void*)residual_nvfp4_kernel<__half>})
+    if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kD * 129 * 4))) !=
+        cudaSuccess)
+      return e;
+  return cudaSuccess;
+}
+
+}  // namespace vc

@@ -1,0 +1,234 @@
+"""Thin Python binding of libvcattn.so (the C ABI in include/vc_attn.h).
+
+Argument marshalling only: torch provides device memory and the current CUDA
+stream; every step of the computation runs in the library's CUDA kernels. There
+is no fallback: if the library is missing or the device is not an sm_100 GPU,
+the calls raise.
+"""
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libvcattn.so")
+
+VC_OK, VC_ERR_INVALID_ARG, VC_ERR_UNSUPPORTED, VC_ERR_WORKSPACE, VC_ERR_CUDA, VC_ERR_TIMEOUT = range(6)
+STATUS_NAMES = ["VC_OK", "VC_ERR_INVALID_ARG", "VC_ERR_UNSUPPORTED", "VC_ERR_WORKSPACE", "VC_ERR_CUDA",
+                "VC_ERR_TIMEOUT"]
+VC_DTYPE_F16, VC_DTYPE_BF16 = 0, 1
+VC_RESIDUAL_E4M3, VC_RESIDUAL_NVFP4 = 0, 1
+VC_MODE_VSMOOTH, VC_MODE_MEANONLY = 0, 1
+
+# every symbol declared in include/vc_attn.h and include/vc_attn_testing.h
+ABI_SYMBOLS = [
+    "vc_attn_version", "vc_attn_last_error", "vc_attn_prepare_v_workspace_bytes", "vc_attn_prepare_v",
+    "vc_attn_quant_qk", "vc_attn_forward", "vc_attn_forward_nvfp4v",
+]
+TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
+                "vc_attn_test_bounded_wait"]
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("S", ctypes.c_int32), ("H", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("dtype", ctypes.c_int32)]
+
+
+class VSmoothCfg(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_int32), ("iters", ctypes.c_int32), ("seed", ctypes.c_uint64),
+                ("residual_fmt", ctypes.c_int32), ("mode", ctypes.c_int32)]
+
+
+class PreparedV(ctypes.Structure):
+    _fields_ = [("perm", ctypes.c_void_p), ("mu", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
+                ("v_scales", ctypes.c_void_p), ("s_v", ctypes.c_void_p)]
+
+
+class QKFP8(ctypes.Structure):
+    _fields_ = [("q_codes", ctypes.c_void_p), ("q_scales", ctypes.c_void_p), ("k_codes", ctypes.c_void_p),
+                ("k_scales", ctypes.c_void_p)]
+
+
+class VCError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{STATUS_NAMES[status] if 0 <= status < 6 else status}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def load():
+    """Load libvcattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m bit_fp8_attention_prep_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, u64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
+    P = ctypes.POINTER
+    lib.vc_attn_version.restype = i32
+    lib.vc_attn_last_error.restype = ctypes.c_char_p
+    lib.vc_attn_prepare_v_workspace_bytes.restype = sz
+    lib.vc_attn_prepare_v_workspace_bytes.argtypes = [P(Shape), P(VSmoothCfg)]
+    lib.vc_attn_prepare_v.restype = i32
+    lib.vc_attn_prepare_v.argtypes = [vp, P(Shape), P(VSmoothCfg), P(PreparedV), vp, sz, vp, vp]
+    lib.vc_attn_quant_qk.restype = i32
+    lib.vc_attn_quant_qk.argtypes = [vp, vp, P(Shape), vp, P(QKFP8), vp]
+    for name in ("vc_attn_forward", "vc_attn_forward_nvfp4v"):
+        f = getattr(lib, name)
+        f.restype = i32
+        f.argtypes = [P(QKFP8), P(PreparedV), P(Shape), ctypes.c_float, i32, vp, vp, vp]
+    lib.vc_attn_test_e4m3_round.restype = i32
+    lib.vc_attn_test_e4m3_round.argtypes = [vp, vp, i64, vp]
+    lib.vc_attn_test_e2m1_round.restype = i32
+    lib.vc_attn_test_e2m1_round.argtypes = [vp, vp, i64, vp]
+    lib.vc_attn_test_expcast.restype = i32
+    lib.vc_attn_test_expcast.argtypes = [vp, vp, vp, i32, vp, i64, i32, vp]
+    lib.vc_attn_test_bounded_wait.restype = i32
+    lib.vc_attn_test_bounded_wait.argtypes = [vp, u64, vp]
+    _lib = lib
+    return lib
+
+
+def _check(status):
+    if status != VC_OK:
+        raise VCError(status, load().vc_attn_last_error().decode())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def shape_of(x):
+    """vc_shape_t for a [B,S,H,128] or [S,H,128] FP16/BF16 tensor."""
+    if x.dim() == 3:
+        B, (S, H, D) = 1, x.shape
+    elif x.dim() == 4:
+        B, S, H, D = x.shape
+    else:
+        raise ValueError("expected [S,H,128] or [B,S,H,128]")
+    if x.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("Q, K, V must be float16 or bfloat16")
+    if not x.is_contiguous():
+        raise ValueError("Q, K, V must be contiguous")
+    return Shape(B, S, H, D, VC_DTYPE_BF16 if x.dtype == torch.bfloat16 else VC_DTYPE_F16)
+
+
+def num_blocks(S):
+    return (S + 127) // 128
+
+
+def prepare_v(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", history=False):
+    """V-Smooth prep of V (device tensor). Returns a dict of the caller-owned
+    outputs (perm, mu, v_codes, v_scales, s_v; plus the per-pass assignments
+    when ``history``)."""
+    lib = load()
+    sh = shape_of(v)
+    cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
+                     VC_MODE_MEANONLY if mode == "meanonly" else VC_MODE_VSMOOTH)
+    B, S, H = sh.B, sh.S, sh.H
+    nb = num_blocks(S)
+    Sp = nb * 128
+    dev = v.device
+    out = dict(
+        perm=torch.empty((B, H, S), dtype=torch.int32, device=dev),
+        mu=torch.empty((B, H, nb, 128), dtype=torch.float32, device=dev),
+        s_v=torch.empty((B, H), dtype=torch.float32, device=dev),
+    )
+    if fmt == "nvfp4":
+        out["v_codes"] = torch.empty((B, H, 128, Sp // 2), dtype=torch.uint8, device=dev)
+        out["v_scales"] = torch.empty((B, H, 128, Sp // 16), dtype=torch.uint8, device=dev)
+    else:
+        out["v_codes"] = torch.empty((B, H, 128, Sp), dtype=torch.uint8, device=dev)
+        out["v_scales"] = None
+    wsb = lib.vc_attn_prepare_v_workspace_bytes(ctypes.byref(sh), ctypes.byref(cfg))
+    if wsb == 0:
+        raise VCError(VC_ERR_INVALID_ARG, "invalid shape or config")
+    ws = torch.empty(wsb + 256, dtype=torch.uint8, device=dev)
+    off = (-ws.data_ptr()) % 256
+    hist = torch.empty((iters, B, H, S), dtype=torch.uint8, device=dev) if history else None
+    pv = PreparedV(_ptr(out["perm"]), _ptr(out["mu"]), _ptr(out["v_codes"]), _ptr(out["v_scales"]), _ptr(out["s_v"]))
+    _check(lib.vc_attn_prepare_v(_ptr(v), ctypes.byref(sh), ctypes.byref(cfg), ctypes.byref(pv),
+                                 ctypes.c_void_p(ws.data_ptr() + off), wsb, _ptr(hist), _stream()))
+    out["workspace"] = ws
+    out["history"] = hist
+    out["fmt"] = fmt
+    return out
+
+
+def quant_qk(q, k, perm):
+    """Per-block E4M3 quantisation of Q and of K gathered through ``perm``."""
+    lib = load()
+    sh = shape_of(q)
+    if shape_of(k).S != sh.S or k.shape != q.shape or k.dtype != q.dtype:
+        raise ValueError("q and k must have the same shape and dtype")
+    B, S, H = sh.B, sh.S, sh.H
+    nb = num_blocks(S)
+    dev = q.device
+    out = dict(
+        q_codes=torch.empty((B, H, nb * 128, 128), dtype=torch.uint8, device=dev),
+        q_scales=torch.empty((B, H, nb), dtype=torch.float32, device=dev),
+        k_codes=torch.empty((B, H, nb * 128, 128), dtype=torch.uint8, device=dev),
+        k_scales=torch.empty((B, H, nb), dtype=torch.float32, device=dev),
+    )
+    qk = QKFP8(_ptr(out["q_codes"]), _ptr(out["q_scales"]), _ptr(out["k_codes"]), _ptr(out["k_scales"]))
+    _check(lib.vc_attn_quant_qk(_ptr(q), _ptr(k), ctypes.byref(sh), _ptr(perm), ctypes.byref(qk), _stream()))
+    return out
+
+
+def forward(qk, pv, shape, softmax_scale=None, k_p=8, out=None, status=None):
+    """Fused ExpCast FP8 attention from the two prep outputs; returns BF16 O in
+    the input layout. ``shape`` is the vc_shape_t of Q (``shape_of(q)``)."""
+    lib = load()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(128)
+    dev = qk["q_codes"].device
+    if out is None:
+        out = torch.empty((shape.B, shape.S, shape.H, 128), dtype=torch.bfloat16, device=dev)
+    q_ = QKFP8(_ptr(qk["q_codes"]), _ptr(qk["q_scales"]), _ptr(qk["k_codes"]), _ptr(qk["k_scales"]))
+    p_ = PreparedV(_ptr(pv["perm"]), _ptr(pv["mu"]), _ptr(pv["v_codes"]), _ptr(pv.get("v_scales")), _ptr(pv["s_v"]))
+    fn = lib.vc_attn_forward_nvfp4v if pv.get("fmt") == "nvfp4" else lib.vc_attn_forward
+    _check(fn(ctypes.byref(q_), ctypes.byref(p_), ctypes.byref(shape), float(softmax_scale), int(k_p), _ptr(out),
+              _ptr(status), _stream()))
+    return out
+
+
+def attention(q, k, v, softmax_scale=None, k_p=8, kmeans_k=16, iters=4, seed=0, fmt="e4m3"):
+    """One call: V-Smooth prep, Q/K quantisation and the fused attention.
+    Q, K, V: [B,S,H,128] or [S,H,128] FP16/BF16 on the GPU; returns BF16 O with
+    the same layout."""
+    pv = prepare_v(v, k=kmeans_k, iters=iters, seed=seed, fmt=fmt)
+    qk = quant_qk(q, k, pv["perm"])
+    o = forward(qk, pv, shape_of(q), softmax_scale, k_p)
+    return o.view(q.shape)
+
+
+# ------------------------------------------------------------------ test hooks
+def test_e4m3_round(x):
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(load().vc_attn_test_e4m3_round(_ptr(x), _ptr(out), x.numel(), _stream()))
+    return out
+
+
+def test_e2m1_round(x):
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(load().vc_attn_test_e2m1_round(_ptr(x), _ptr(out), x.numel(), _stream()))
+    return out
+
+
+def test_expcast(t, c, M, bias_b, hot=False):
+    out = torch.empty(t.shape, dtype=torch.uint8, device=t.device)
+    _check(load().vc_attn_test_expcast(_ptr(t), _ptr(c), _ptr(M), int(bias_b), _ptr(out), t.numel(), int(hot),
+                                       _stream()))
+    return out
+
+
+def test_bounded_wait(status, limit_ns):
+    _check(load().vc_attn_test_bounded_wait(_ptr(status), int(limit_ns), _stream()))

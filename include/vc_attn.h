@@ -1,0 +1,170 @@
+/*
+ * vc_attn.h -- C ABI of the VC-Attention forward hot path on one B200 (sm_100a).
+ *
+ * The method: "VC-Attention: Value Smoothing and Softmax Casting for Low-bit
+ * Attention" (arXiv 2609.15810), Abstract -- V-Smooth reorders value tokens by
+ * online clustering, quantises only the residual after subtracting each block's
+ * mean and restores the mean from the online-softmax row sum; ExpCast-FP8 maps
+ * log-domain scores to E4M3 probability codes with one fused multiply-add.
+ * Per-(batch, head) k-means, 128-token blocks and the E4M3 / NVFP4 residual are
+ * from "Nunchux AI lanza VC-Attention kernel ..." (news summary), second
+ * paragraph. The input / output contract (FP16 or BF16 Q, K, V of shape
+ * [S,H,128] or [B,S,H,128], BF16 O) and the prep / attention split are from
+ * "Open VC Attention" (catalogue card), section "Описание".
+ *
+ * Conventions (every entry point):
+ *  - Pointers named q, k, v, o and every field of vc_prepared_v_t / vc_qk_fp8_t
+ *    are DEVICE pointers owned and allocated by the caller; the library never
+ *    allocates or frees device memory and keeps no pointer after a call returns.
+ *  - Tensors are dense and row-major in the layouts stated per field. Q, K, V and
+ *    O are [B, S, H, 128] (a [S, H, 128] tensor is B = 1). Device pointers must
+ *    be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). All work is
+ *    enqueued asynchronously on it; no call synchronises the device.
+ *  - Every call validates its arguments on the host before launching anything
+ *    and returns a vc_status_t; on error nothing has been launched and
+ *    vc_attn_last_error() gives a message (per calling thread). No call aborts,
+ *    traps or prints.
+ *  - Device-side failures (a bounded wait inside a kernel that ran out) are
+ *    reported through the optional `dev_status` int (device memory, set by the
+ *    caller to VC_OK before the call, read after the caller's own sync).
+ *  - Sizes: S >= 1, H >= 1, B >= 1, D == 128, B*H*S_pad*128 < 2^31 elements per
+ *    tensor, where nb = ceil(S/128) and S_pad = 128*nb.
+ */
+#ifndef VC_ATTN_H
+#define VC_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VC_OK = 0,
+  VC_ERR_INVALID_ARG = 1,   /* a shape, pointer, alignment or config is invalid   */
+  VC_ERR_UNSUPPORTED = 2,   /* valid but not supported by this build / device     */
+  VC_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required         */
+  VC_ERR_CUDA = 4,          /* a CUDA runtime / driver call failed                */
+  VC_ERR_TIMEOUT = 5        /* device side: a bounded wait in a kernel ran out    */
+} vc_status_t;
+
+typedef enum { VC_DTYPE_F16 = 0, VC_DTYPE_BF16 = 1 } vc_dtype_t;
+typedef enum { VC_RESIDUAL_E4M3 = 0, VC_RESIDUAL_NVFP4 = 1 } vc_residual_fmt_t;
+typedef enum {
+  VC_MODE_VSMOOTH = 0,      /* k-means + cluster sort + block means (the method)  */
+  VC_MODE_MEANONLY = 1      /* identity order, block means only (diagnostic)      */
+} vc_mode_t;
+
+/* Problem shape. D must be 128. dtype is a vc_dtype_t for Q, K and V. */
+typedef struct {
+  int32_t B, S, H, D;
+  int32_t dtype;
+} vc_shape_t;
+
+/* V-Smooth configuration. k in [1, 32] clusters, iters >= 1 assignment passes
+ * (the last pass's assignment is final), seed for the k-means init. */
+typedef struct {
+  int32_t k;
+  int32_t iters;
+  uint64_t seed;
+  int32_t residual_fmt;     /* vc_residual_fmt_t */
+  int32_t mode;             /* vc_mode_t         */
+} vc_vsmooth_cfg_t;
+
+/* Output of vc_attn_prepare_v (caller-owned device buffers):
+ *  perm     int32 [B,H,S]      original token index at each permuted position
+ *  mu       fp32  [B,H,nb,128] mean of each 128-token block (permuted order)
+ *  v_codes  E4M3:  uint8 [B,H,128,S_pad]   residual codes, V^T (token-contiguous)
+ *           NVFP4: uint8 [B,H,128,S_pad/2] two E2M1 codes per byte, even token
+ *                  in the low nibble
+ *  v_scales NVFP4 only: uint8 [B,H,128,S_pad/16] E4M3 scale per 16 tokens
+ *  s_v      fp32  [B,H]        E4M3: residual scale s_V; NVFP4: global scale g
+ * Padding columns (tokens >= S) of v_codes / v_scales are written as 0. */
+typedef struct {
+  int32_t* perm;
+  float* mu;
+  uint8_t* v_codes;
+  uint8_t* v_scales;
+  float* s_v;
+} vc_prepared_v_t;
+
+/* Output of vc_attn_quant_qk (caller-owned device buffers):
+ *  q_codes  uint8 [B,H,S_pad,128]  E4M3 codes of Q (original order)
+ *  q_scales fp32  [B,H,nb]         one scale per 128-row block of Q
+ *  k_codes  uint8 [B,H,S_pad,128]  E4M3 codes of K in permuted order
+ *  k_scales fp32  [B,H,nb]         one scale per 128-row block of permuted K
+ * Padding rows are written as 0. */
+typedef struct {
+  uint8_t* q_codes;
+  float* q_scales;
+  uint8_t* k_codes;
+  float* k_scales;
+} vc_qk_fp8_t;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int32_t vc_attn_version(void);
+
+/* Message for the last error returned on the calling thread ("" if none). */
+const char* vc_attn_last_error(void);
+
+/* Bytes of workspace vc_attn_prepare_v needs for this shape and config
+ * (0 if the arguments are invalid). */
+size_t vc_attn_prepare_v_workspace_bytes(const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg);
+
+/* V-Smooth prep ("VC-Attention ...", Abstract; "Nunchux AI lanza ...", 2nd
+ * paragraph): per (b, h), seeded k-means over the value tokens (k clusters,
+ * `iters` Lloyd assignment passes), a stable sort of the tokens by cluster id
+ * (the permutation also applied to K by vc_attn_quant_qk), subtraction of each
+ * 128-token block's mean, and quantisation of the residual to E4M3 (one scale per
+ * (b, h)) or NVFP4 (E2M1 + E4M3 scale per 16 tokens + fp32 global per (b, h)).
+ *  v               device, [B,S,H,128] of shape->dtype
+ *  out             fields as documented in vc_prepared_v_t (v_scales only NVFP4)
+ *  workspace       device, >= vc_attn_prepare_v_workspace_bytes(), 256-B aligned;
+ *                  contents on entry are ignored
+ *  assign_history  optional device uint8 [iters,B,H,S]: the assignment of every
+ *                  pass (for lock-step checking); NULL to skip
+ * Errors: VC_ERR_INVALID_ARG (shape / cfg / pointers), VC_ERR_WORKSPACE,
+ *         VC_ERR_CUDA (launch failure). */
+vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                              const vc_prepared_v_t* out, void* workspace, size_t workspace_bytes,
+                              uint8_t* assign_history, void* stream);
+
+/* Q/K FP8 quantisation ("Open VC Attention", "Описание": Q/K scales per block):
+ * per (b, h, 128-row block) scale s = amax/448 and E4M3 codes of x*(448/amax);
+ * K rows are gathered through `perm` (from vc_attn_prepare_v) first.
+ *  q, k   device, [B,S,H,128] of shape->dtype
+ *  perm   device int32 [B,H,S]
+ * Errors: VC_ERR_INVALID_ARG, VC_ERR_CUDA. */
+vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* shape,
+                             const int32_t* perm, const vc_qk_fp8_t* out, void* stream);
+
+/* Fused FP8 attention with ExpCast probabilities and the block-mean restore
+ * ("VC-Attention ...", Abstract; "Hugging Face Introduces VC-Attention",
+ * "Technical Breakthroughs and Core Innovations"), E4M3 V residual:
+ *   t = Q_codes K_codes^T (FP8 tensor cores, fp32 accumulate)
+ *   log2-domain score u = c t, c = (sQ sK) * fl32(softmax_scale * log2 e)
+ *   P code = E4M3 bit pattern of 2^(u - M + k_p), M an integer running row frame
+ *   O = (s_V * P V_codes + sum_tiles rowsum(P_tile) mu_tile) / rowsum(P)
+ *  qk, pv        outputs of the two prep calls for the same shape
+ *  softmax_scale usually 1/sqrt(128)
+ *  k_p           probability bias exponent in [0, 8] (8 recommended)
+ *  o             device bf16 [B,S,H,128], rows in original query order
+ *  dev_status    optional device int32 (see conventions)
+ * Non-causal, no mask. Errors: VC_ERR_INVALID_ARG, VC_ERR_UNSUPPORTED (device is
+ * not sm_100), VC_ERR_CUDA. */
+vc_status_t vc_attn_forward(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
+                            float softmax_scale, int32_t k_p, void* o, int32_t* dev_status,
+                            void* stream);
+
+/* As vc_attn_forward, for a V residual prepared with VC_RESIDUAL_NVFP4 (pv->v_codes
+ * packed E2M1, pv->v_scales E4M3 per 16 tokens, pv->s_v the global scale g). */
+vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv,
+                                   const vc_shape_t* shape, float softmax_scale, int32_t k_p,
+                                   void* o, int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VC_ATTN_H */

@@ -1,0 +1,90 @@
+"""The C-ABI library loads, exports every symbol its headers declare, and its
+host-side validation answers without a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_fp8_attention_prep_b200 import build, vc_attn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return vc_attn.load()
+
+
+def _declared(header):
+    text = open(os.path.join(ROOT, "include", header)).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vc_attn_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared("vc_attn.h") + _declared("vc_attn_testing.h")
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(_declared("vc_attn.h")) == set(vc_attn.ABI_SYMBOLS)
+    assert set(_declared("vc_attn_testing.h")) == set(vc_attn.TEST_SYMBOLS)
+
+
+def test_version_and_last_error(lib):
+    assert lib.vc_attn_version() == 100
+    assert lib.vc_attn_last_error() == b""
+
+
+def _shape(B=1, S=256, H=2, D=128, dt=vc_attn.VC_DTYPE_BF16):
+    return vc_attn.Shape(B, S, H, D, dt)
+
+
+def _cfg(k=4, iters=3, fmt=0, mode=0):
+    return vc_attn.VSmoothCfg(k, iters, 0, fmt, mode)
+
+
+def test_workspace_bytes_and_validation(lib):
+    ok = lib.vc_attn_prepare_v_workspace_bytes(ctypes.byref(_shape()), ctypes.byref(_cfg()))
+    assert ok > 0 and ok % 256 == 0
+    big = lib.vc_attn_prepare_v_workspace_bytes(ctypes.byref(_shape(S=73397, H=56)), ctypes.byref(_cfg(k=16)))
+    assert big > ok
+    for sh in (_shape(D=64), _shape(S=0), _shape(H=0), _shape(dt=7), _shape(S=1 << 20, H=200)):
+        assert lib.vc_attn_prepare_v_workspace_bytes(ctypes.byref(sh), ctypes.byref(_cfg())) == 0
+    for cfg in (_cfg(k=0), _cfg(k=33), _cfg(iters=0), _cfg(fmt=3), _cfg(mode=5)):
+        assert lib.vc_attn_prepare_v_workspace_bytes(ctypes.byref(_shape()), ctypes.byref(cfg)) == 0
+
+
+def test_calls_reject_bad_arguments_before_any_launch(lib):
+    sh = _shape(D=64)
+    pv = vc_attn.PreparedV(16, 16, 16, 16, 16)
+    st = lib.vc_attn_prepare_v(ctypes.c_void_p(16), ctypes.byref(sh), ctypes.byref(_cfg()), ctypes.byref(pv),
+                               ctypes.c_void_p(256), 1 << 20, None, None)
+    assert st == vc_attn.VC_ERR_INVALID_ARG
+    assert b"D must be 128" in lib.vc_attn_last_error()
+    # NULL output pointer
+    pv0 = vc_attn.PreparedV(0, 16, 16, 16, 16)
+    st = lib.vc_attn_prepare_v(ctypes.c_void_p(16), ctypes.byref(_shape()), ctypes.byref(_cfg()),
+                               ctypes.byref(pv0), ctypes.c_void_p(256), 1 << 20, None, None)
+    assert st == vc_attn.VC_ERR_INVALID_ARG
+    # misaligned input
+    st = lib.vc_attn_prepare_v(ctypes.c_void_p(18), ctypes.byref(_shape()), ctypes.byref(_cfg()),
+                               ctypes.byref(pv), ctypes.c_void_p(256), 1 << 20, None, None)
+    assert st == vc_attn.VC_ERR_INVALID_ARG and b"aligned" in lib.vc_attn_last_error()
+    # workspace too small
+    st = lib.vc_attn_prepare_v(ctypes.c_void_p(16), ctypes.byref(_shape()), ctypes.byref(_cfg()),
+                               ctypes.byref(pv), ctypes.c_void_p(256), 64, None, None)
+    assert st == vc_attn.VC_ERR_WORKSPACE
+    qk = vc_attn.QKFP8(16, 16, 16, 16)
+    st = lib.vc_attn_quant_qk(ctypes.c_void_p(16), None, ctypes.byref(_shape()), ctypes.c_void_p(16),
+                              ctypes.byref(qk), None)
+    assert st == vc_attn.VC_ERR_INVALID_ARG
+    for kp, scale in ((9, 0.088), (-1, 0.088), (8, 0.0), (8, float("nan"))):
+        st = lib.vc_attn_forward(ctypes.byref(qk), ctypes.byref(pv), ctypes.byref(_shape()), scale, kp,
+                                 ctypes.c_void_p(16), None, None)
+        assert st == vc_attn.VC_ERR_INVALID_ARG
+    for fn in (lib.vc_attn_test_e4m3_round, lib.vc_attn_test_e2m1_round):
+        assert fn(None, None, -1, None) == vc_attn.VC_ERR_INVALID_ARG
+        assert fn(None, None, 0, None) == vc_attn.VC_OK
+    assert lib.vc_attn_test_bounded_wait(None, 1000, None) == vc_attn.VC_ERR_INVALID_ARG

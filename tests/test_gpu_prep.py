@@ -1,0 +1,80 @@
+"""GPU: V-Smooth prep and Q/K quantisation are bit-exact with the oracle
+(k-means assignments compared pass by pass; near ties counted, no mismatch)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from parity_helpers import assert_prep_bit_exact, gpu_pipeline, make, oracle_head
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def va():
+    from bit_fp8_attention_prep_b200 import build, vc_attn
+    build.build()
+    vc_attn.load()
+    return vc_attn
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny", {}),
+    ("mid", dict(B=2, H=2, S=1000)),          # ragged: 7 full blocks + 104
+    ("mid", dict(B=1, H=3, S=2500)),          # several k-means chunks, ragged chunk
+])
+def test_prep_bit_exact(va, name, kw):
+    cfg, Q, K, V = make(name, **kw)
+    g = gpu_pipeline(va, Q, K, V, cfg["k"], cfg["iters"])
+    assert g["status"] == 0
+    ties = 0
+    for b in range(cfg["B"]):
+        for h in range(cfg["H"]):
+            ref = oracle_head(g, Q, K, V, b, h, cfg["k"], cfg["iters"])
+            assert_prep_bit_exact(g, ref, b, h)
+            ties += ref["stats"]["near_ties"]
+    print(f"near ties adopted: {ties}")
+
+
+def test_prep_nvfp4_bit_exact(va):
+    cfg, Q, K, V = make("mid", B=1, H=2, S=777)
+    g = gpu_pipeline(va, Q, K, V, 16, 4, fmt="nvfp4", attend=False)
+    for h in range(2):
+        ref = oracle_head(g, Q, K, V, 0, h, 16, 4, fmt="nvfp4")
+        assert_prep_bit_exact(g, ref, 0, h, fmt="nvfp4")
+
+
+@pytest.mark.parametrize("S,k", [(1, 4), (5, 16), (129, 16), (130, 1)])
+def test_prep_edge_sizes(va, S, k):
+    # fewer tokens than clusters, a single token, one token past a block, k = 1
+    cfg, Q, K, V = make("mid", B=1, H=2, S=S)
+    g = gpu_pipeline(va, Q, K, V, k, 3)
+    for h in range(2):
+        ref = oracle_head(g, Q, K, V, 0, h, k, 3)
+        assert_prep_bit_exact(g, ref, 0, h)
+
+
+def test_prep_zero_head_and_fp16(va):
+    cfg, Q, K, V = make("mid", B=1, H=2, S=300)
+    V[:, :, 1] = 0                       # an all-zero head: amax 0 -> s_V = 1, codes 0
+    Q[:, 128:256, 0] = 0                 # an all-zero Q block -> scale 1, codes 0
+    for dt in (torch.bfloat16, torch.float16):
+        Qd, Kd, Vd = Q.to(dt), K.to(dt), V.to(dt)
+        g = gpu_pipeline(va, Qd, Kd, Vd, 16, 4)
+        for h in range(2):
+            ref = oracle_head(g, Qd, Kd, Vd, 0, h, 16, 4)
+            assert_prep_bit_exact(g, ref, 0, h)
+        assert g["s_v"][0, 1] == 1.0 and not g["v_codes"][0, 1].any()
+        assert g["q_scales"][0, 0, 1] == 1.0
+
+
+def test_meanonly_mode(va):
+    cfg, Q, K, V = make("mid", B=1, H=2, S=400)
+    v = V.cuda()
+    pv = va.prepare_v(v, mode="meanonly")
+    torch.cuda.synchronize()
+    for h in range(2):
+        ref = O.prepare_v_head(V[0, :, h].float().numpy(), 16, 4, 0, h, mode="meanonly")
+        assert np.array_equal(pv["perm"][0, h].cpu().numpy(), ref["perm"])
+        assert np.array_equal(pv["mu"][0, h].cpu().numpy().view(np.uint32), ref["mu"].view(np.uint32))
+        assert np.array_equal(pv["v_codes"][0, h].cpu().numpy(), ref["v_codes"])
