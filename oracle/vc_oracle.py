@@ -39,9 +39,17 @@ Readings taken where the pages are silent (R-numbers are used in comments):
   R7  Q/K: one scale per 128-token block (Q in original order, K in permuted
       order); softmax scale enters the score multiplier, not the codes.
   R8  ExpCast: log2-domain score u = c_j * t_ij with c_j = fl32(fl32(sQ*sK) *
-      kappa), kappa = fl32(softmax_scale * log2 e); integer frame
-      M_i = ceil(max_j fl32(u_ij)); code = clip(B - 8 M_i + rne(8 c_j t_ij), 0, 126),
-      B = 56 + 8 k_P (k_P = 8 by default: P is carried scaled by 2^8).
+      kappa), kappa = fl32(softmax_scale * log2 e); the online softmax visits the
+      128-key blocks in permuted order and keeps an integer running frame per row,
+      F_i(b) = max(F_i(b-1), ceil(max_{j in block b} fl32(u_ij))), F_i(0) from
+      block 0 alone; the keys of block b are cast in the frame current after
+      block b: code = clip(B - 8 F_i(b) + rne(8 c_j t_ij), 0, 126),
+      B = 56 + 8 k_P (k_P = 8 by default: P is carried scaled by 2^8); when the
+      frame moves, what was accumulated so far is multiplied by the exact power
+      of two 2^(F_old - F_new), so key j carries dec(code_ij) 2^(F_i(b) - F_i(nb-1)).
+      ([ABS]: the mean is restored from the row sum "the online softmax already
+      maintains" -- the cast happens inside that online pass.) Where the frame
+      never moves this is the single-frame cast with M_i = ceil(max_j fl32(u_ij)).
   R9  Row sum and block restore use the cast P (the E4M3 values the PV product
       uses); O = (sum_j P_ij v~_j + sum_b r_ib mu_b) / l_i, then BF16 RNE.
   R10 A block (or head) whose amax is below 2^-100 is treated as all zero:
@@ -69,7 +77,7 @@ __all__ = [
     "SplitMix64", "kmeans_init_indices", "kmeans_lloyd", "centroid_update",
     "cluster_permutation", "block_means", "residual_e4m3", "residual_nvfp4",
     "vres_from_e4m3", "vres_from_nvfp4", "quant_blocks_e4m3", "softmax_kappa",
-    "expcast_codes", "expcast_bias", "vc_attention_rows", "vc_attention_exact_prob",
+    "expcast_codes", "expcast_bias", "expcast_online_probs", "vc_attention_rows", "vc_attention_exact_prob",
     "exact_attention_rows", "naive_v_e4m3", "prepare_v_head", "quant_qk_head",
     "padded_len", "num_blocks", "residual_energy",
 ]
@@ -411,6 +419,32 @@ def _combine(P, vres, mu, S):
     return (P @ vres + R @ np.asarray(mu, np.float64)) / l[:, None], l
 
 
+def expcast_online_probs(t, c, S, k_p=K_P_DEFAULT):
+    """R8: probabilities of one or more query rows, cast block by block in the
+    online running frame and expressed in the final frame.
+
+    t, c: (rows, S) fp32 scores and multipliers. Returns (P float64, codes
+    uint8, frames (rows, nb) float64 = F_i(b), final frame F_i(nb-1)).
+    """
+    t = np.asarray(t, np.float32)
+    c = np.asarray(c, np.float32)
+    u = c * t                                                        # fl32(c t)
+    nb = num_blocks(S)
+    bias = expcast_bias(k_p)
+    codes = np.zeros(t.shape, np.uint8)
+    frames = np.zeros((t.shape[0], nb), np.float64)
+    F = None
+    for b in range(nb):
+        cols = slice(b * BLOCK, min(b * BLOCK + BLOCK, S))
+        Fb = np.ceil(u[:, cols].max(axis=1).astype(np.float64))    # this block's frame
+        F = Fb if F is None else np.maximum(F, Fb)                   # running frame
+        frames[:, b] = F
+        codes[:, cols] = expcast_codes(t[:, cols], c[:, cols], F[:, None], bias)
+    shift = np.repeat(frames - F[:, None], BLOCK, axis=1)[:, :S]     # F(b) - F(final) <= 0
+    P = _E4M3[codes] * np.exp2(shift)                                # exact powers of two
+    return P, codes, frames, F
+
+
 def vc_attention_rows(q_codes, q_scales, k_codes, k_scales, vres, mu, S, rows,
                       softmax_scale, k_p=K_P_DEFAULT, return_codes=False):
     """VC-Attention output for query rows ``rows`` of one (b, h) slice, in fp64.
@@ -419,6 +453,8 @@ def vc_attention_rows(q_codes, q_scales, k_codes, k_scales, vres, mu, S, rows,
     k_scales: per-block fp32 scales; vres: (S, D) decoded residual values in
     permuted order; mu: (nb, D) block means. Scores t = sum_d dec(q) dec(k) are
     exact in fp64 (products of 4-bit significands) and then rounded to fp32.
+    Probabilities follow R8 (online integer frame per 128-key block), the
+    combination R9.
     """
     rows = np.asarray(rows)
     Kd = _E4M3[k_codes[:S]]
@@ -428,10 +464,7 @@ def vc_attention_rows(q_codes, q_scales, k_codes, k_scales, vres, mu, S, rows,
     sq = np.asarray(q_scales, np.float32)[rows // BLOCK]
     sk = np.asarray(k_scales, np.float32)[np.arange(S) // BLOCK]
     c = (sq[:, None] * sk[None, :]) * kappa                         # fp32, fp32
-    u = c * t                                                        # fl32(c t)
-    M = np.ceil(u.max(axis=1).astype(np.float64))                    # integer frame
-    codes = expcast_codes(t, c, M[:, None], expcast_bias(k_p))
-    P = _E4M3[codes]
+    P, codes, frames, M = expcast_online_probs(t, c, S, k_p)
     O, l = _combine(P, vres, mu, S)
     if return_codes:
         return O, codes, M, l
