@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Benchmark of the VC-Attention forward hot path on B200.
+
+One step = the whole path on one batch of synthetic input already resident in
+HBM: V-Smooth prep (k-means, cluster sort, block means, residual codes), Q/K
+per-block FP8 quantisation, and the fused ExpCast FP8 attention. The metric is
+FP8 TFLOP/s of the full call, counting the dense attention work 4*B*H*S^2*D
+("VC-Attention: Value Smoothing and Softmax Casting for Low-bit Attention",
+Abstract: low-bit tensor cores run the two matrix products).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the CPU oracle, timed on host cores
+
+Under torchrun (N > 1) every rank runs its own independent problem of the same
+size on its own GPU (weak scaling); the only collectives are a barrier and the
+max over ranks of the measured time. Rank 0 prints one JSON line.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "VC-attn FP8 TFLOP/s and % of FP8 peak at S=73397,D=128; rel-L2 vs FP64"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "minimax_h56"
+ATTN_SRC = os.path.join(ROOT, "bit_fp8_attention_prep_b200", "csrc", "vc_attn_fwd.cu")
+# DRAM bytes (read + write) of one attention launch on the default workload, from
+# the ncu capture summarised in profiles/; valid only while the kernel source
+# hashes to the recorded value (otherwise traffic is reported as null).
+ATTN_TRAFFIC = {"sha256_16": None, "bytes_per_launch": None}
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--k-p", type=int, default=8)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the SDPA comparison, accuracy, e2e and CPU-baseline legs")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+def flops_of(cfg):
+    return 4.0 * cfg["B"] * cfg["H"] * float(cfg["S"]) ** 2 * 128
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(bf16_sustained=float(p["bf16_tflops_sustained"]), bf16_burst=float(p["bf16_tflops"]),
+                    hbm=float(p["hbm_gbs"]), source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(bf16_sustained=FALLBACK_BF16_TFLOPS_SUSTAINED, bf16_burst=1590.0, hbm=FALLBACK_HBM_GBS,
+                    source="fallback")
+
+
+def src_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.dev = device_index
+
+    def start(self):
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(["nvidia-smi", "--id=" + ident, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, AttributeError, RuntimeError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- CPU oracle legs
+def oracle_sample(cfg, S_sample, rows, seed=0):
+    """Time the oracle as it stands on one (b, h) slice: V-Smooth prep and Q/K
+    quantisation of the first ``S_sample`` tokens, then ``rows`` query rows
+    against all of them. Returns (seconds for the full workload, extrapolated
+    per head and per row, the measured seconds, a description)."""
+    import numpy as np
+    import oracle as O
+    from bit_fp8_attention_prep_b200 import synth
+    Q, K, V = synth.make_qkv(1, S_sample, 1, recipe=cfg["recipe"], seed=seed)
+    q, k, v = (X[0, :, 0].float().numpy() for X in (Q, K, V))
+    t0 = time.perf_counter()
+    prep = O.prepare_v_head(v, cfg["k"], cfg["iters"], 0, 0, fmt=cfg["fmt"])
+    qc, qs, kc, ks = O.quant_qk_head(q, k, prep["perm"])
+    t1 = time.perf_counter()
+    r = np.linspace(0, S_sample - 1, rows).astype(np.int64)
+    O.vc_attention_rows(qc, qs, kc, ks, prep["vres"], prep["mu"], S_sample, r, 1.0 / math.sqrt(128))
+    t2 = time.perf_counter()
+    S, BH = cfg["S"], cfg["B"] * cfg["H"]
+    # prep and quantisation are linear in S; each output row costs O(S)
+    full = BH * ((t1 - t0) * S / S_sample + (t2 - t1) * (S / rows) * (S / S_sample))
+    desc = (f"one (b,h) slice: V-Smooth prep + Q/K quantisation of {S_sample} tokens and {rows} query rows "
+            f"of VC-attention against them; extrapolated x{BH} slices, linearly in S for prep and per row "
+            f"for attention")
+    return full, t2 - t0, desc
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        n = [i["num_threads"] for i in threadpoolctl.threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except ImportError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, cfg):
+    """--impl reference: the CPU oracle as it stands, on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    flops = flops_of(cfg)
+    # each step a bounded sample, sized so that the whole run stays within a few minutes
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    S_sample = int(min(cfg["S"], max(1024, 8192 * budget / 1.3)))   # ~1.3 s per 8192 tokens here
+    for _ in range(args.warmup):
+        oracle_sample(cfg, S_sample, 64)
+    est, meas = [], 0.0
+    for _ in range(args.steps):
+        full, took, desc = oracle_sample(cfg, S_sample, 64)
+        est.append(full)
+        meas += took
+    t_full = statistics.mean(est)
+    value = flops / t_full / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_full * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(cfg, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": desc + f"; measured {meas / max(1, args.steps):.2f} s per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(cfg, args):
+    return {"workload": cfg["name"], "B": cfg["B"], "S": cfg["S"], "H": cfg["H"], "D": 128,
+            "kmeans_k": cfg["k"], "lloyd_iters": cfg["iters"], "residual": cfg["fmt"], "k_p": args.k_p,
+            "layout": "[B,S,H,128] bf16 in, bf16 out", "non_causal": True,
+            "l2": "inputs larger than L2 (bf16 Q/K/V %.2f GB per GPU)" % (3 * cfg["B"] * cfg["S"] * cfg["H"] * 256 / 1e9),
+            "parallelism": f"independent problem per GPU x{args.gpus}"}
+
+
+# ----------------------------------------------------------------- GPU leg
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+    from bit_fp8_attention_prep_b200 import synth, vc_attn
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    B, S, H = cfg["B"], cfg["S"], cfg["H"]
+    Q, K, V = synth.make_workload(cfg["name"], seed=rank, device=dev)[1:]
+    plan = vc_attn.Plan(B, S, H, k=cfg["k"], iters=cfg["iters"], fmt=cfg["fmt"], k_p=args.k_p, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = flops_of(cfg)
+
+    for _ in range(args.warmup):
+        plan.run(Q, K, V)
+    torch.cuda.synchronize(dev)
+    if int(plan.status.item()) != 0:
+        raise RuntimeError(f"device status {int(plan.status.item())} after warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    n0 = vc_attn.launch_count()
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    for i in range(args.steps):
+        e = ev[i]
+        e[0].record(stream)
+        plan.prepare_v(V)
+        e[1].record(stream)
+        plan.quant_qk(Q, K)
+        e[2].record(stream)
+        plan.forward()
+        e[3].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    launches = vc_attn.launch_count() - n0
+    total_ms = ev[0][0].elapsed_time(ev[-1][3])
+    prep_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    qk_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    fwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    status = int(plan.status.item())
+    total_ms = max_over_ranks(total_ms)
+    ms_per_step = total_ms / args.steps
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+
+    peaks = load_peaks()
+    fp8_peak = 2.0 * peaks["bf16_sustained"]
+    attn_tflops = flops / (fwd_ms * 1e-3) / 1e12
+    traffic = None
+    if ATTN_TRAFFIC["sha256_16"] and ATTN_TRAFFIC["sha256_16"] == src_hash(ATTN_SRC) and \
+            cfg["name"] == DEFAULT_WORKLOAD:
+        traffic = ATTN_TRAFFIC["bytes_per_launch"]
+    nb = (S + 127) // 128
+    # algorithmic bytes: read bf16 V once, write codes + perm + means (prep);
+    # read bf16 Q, K once, read perm, write codes + scales (Q/K)
+    vres_bytes = 128 * nb * 128 if cfg["fmt"] == "e4m3" else 128 * nb * 128 // 2 + 128 * nb * 8
+    prep_bytes = B * H * (S * 256 + vres_bytes + S * 4 + nb * 512)
+    qk_bytes = B * H * (2 * S * 256 + S * 4 + 2 * nb * 128 * 128 + 2 * nb * 4)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": config_of(cfg, argparse.Namespace(k_p=args.k_p, gpus=world)),
+        "roofline": {"bound": "tensor", "kernel": "vc_attn_fwd_e4m3_kernel", "achieved": attn_tflops,
+                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak, "traffic": traffic,
+                     "peak_source": f"2 x {peaks['source']} sustained bf16 cuBLAS ({peaks['bf16_sustained']:.1f})"},
+        "stages_ms": {"prepare_v": prep_ms, "quant_qk": qk_ms, "forward": fwd_ms},
+        "forward_only_tflops": attn_tflops,
+        "frac_of_fp8_peak_full_call": (value / world) / fp8_peak,
+        "prep_hbm": {"algorithmic_bytes": prep_bytes, "achieved_gbs": prep_bytes / (prep_ms * 1e-3) / 1e9,
+                     "peak_gbs": peaks["hbm"], "frac": prep_bytes / (prep_ms * 1e-3) / 1e9 / peaks["hbm"]},
+        "quant_qk_hbm": {"algorithmic_bytes": qk_bytes, "achieved_gbs": qk_bytes / (qk_ms * 1e-3) / 1e9,
+                         "peak_gbs": peaks["hbm"], "frac": qk_bytes / (qk_ms * 1e-3) / 1e9 / peaks["hbm"]},
+        "gpu_launches": launches,
+        "device_status": status,
+        "clocks": clk,
+    }
+    if not args.no_extras:
+        line.update(extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_step, rank))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_step, rank):
+    import torch
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    out = {}
+    B, S, H = cfg["B"], cfg["S"], cfg["H"]
+    # accuracy on sampled rows of two heads: rel-L2 against exact attention in fp64
+    o = plan.run(Q, K, V).float()
+    rows = torch.linspace(0, S - 1, 64, device=dev).long()
+    num = den = 0.0
+    for h in (0, H - 1):
+        q = Q[0, rows, h].double()
+        k, v = K[0, :, h].double(), V[0, :, h].double()
+        p = torch.softmax((q @ k.t()) / math.sqrt(128), dim=-1)
+        ref = p @ v
+        num += float(((o[0, rows, h].double() - ref) ** 2).sum())
+        den += float((ref ** 2).sum())
+        del k, v, p
+    out["rel_l2_vs_fp64"] = math.sqrt(num / den)
+    out["accuracy_sample"] = "64 query rows x heads {0, H-1} of batch 0, exact fp64 softmax attention on the GPU"
+    # BF16 cuDNN SDPA on the same inputs, same stream
+    try:
+        qt, kt, vt = (X.transpose(1, 2) for X in (Q, K, V))
+        with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+            for _ in range(2):
+                F.scaled_dot_product_attention(qt, kt, vt)
+            n = max(2, min(args.steps, 5))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            for _ in range(n):
+                F.scaled_dot_product_attention(qt, kt, vt)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+        sdpa_ms = e0.elapsed_time(e1) / n
+        out["sdpa_bf16_cudnn"] = {"ms": sdpa_ms, "tflops": flops / (sdpa_ms * 1e-3) / 1e12,
+                                  "speedup_forward": sdpa_ms / fwd_ms, "speedup_full_call": sdpa_ms / ms_per_step}
+    except RuntimeError as exc:  # cuDNN backend not available for this shape
+        out["sdpa_bf16_cudnn"] = {"unavailable": str(exc).splitlines()[0][:200]}
+    # end to end through the public API with host buffers: H2D of Q, K, V from
+    # pinned memory, the three calls, D2H of O, all inside the timed region
+    hq, hk, hv = (X.cpu().pin_memory() for X in (Q, K, V))
+    ho = torch.empty(plan.o.shape, dtype=plan.o.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        plan.run(dq, dk, dv)
+        ho.copy_(plan.o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    n = max(2, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / n
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    out["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                  "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
+                  "d2h_bytes_per_step": plan.o.numel() * plan.o.element_size(), "ms_per_step": e2e_ms}
+    del hq, hk, hv, ho, dq, dk, dv
+    # the oracle on the host cores, rank 0 at N = 1 only
+    if world == 1 and rank == 0:
+        full, took, desc = oracle_sample(cfg, min(S, 73397), 256)
+        out["cpu_baseline"] = {"value": flops / full / 1e12, "unit": UNIT, "cores": blas_threads(),
+                               "kind": "oracle", "sample": desc + f"; measured {took:.1f} s"}
+    return out
+
+
+def main():
+    args = parse_args()
+    from bit_fp8_attention_prep_b200 import synth
+    cfg = synth.workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -7,6 +7,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -16,6 +17,7 @@
 namespace {
 
 thread_local std::string g_last_error;
+std::atomic<uint64_t> g_launches{0};  // kernels enqueued by this library since load
 
 vc_status_t fail(vc_status_t st, const char* fmt, ...) {
   char buf[512];
@@ -155,6 +157,8 @@ int32_t vc_attn_version(void) { return 100; }
 
 const char* vc_attn_last_error(void) { return g_last_error.c_str(); }
 
+uint64_t vc_attn_launch_count(void) { return g_launches.load(); }
+
 size_t vc_attn_prepare_v_workspace_bytes(const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg) {
   if (check_shape(shape) != VC_OK || check_cfg(cfg) != VC_OK) return 0;
   return ws_layout(shape, cfg).total;
@@ -201,7 +205,10 @@ vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_v
   pl.hist = reinterpret_cast<int*>(ws + w.hist);
   pl.offs = reinterpret_cast<int*>(ws + w.offs);
   pl.amax = reinterpret_cast<unsigned int*>(ws + w.amax);
-  cudaError_t e = vc::launch_prepare_v(v, shape->dtype, pl, *out, assign_history, static_cast<cudaStream_t>(stream));
+  int nl = 0;
+  cudaError_t e =
+      vc::launch_prepare_v(v, shape->dtype, pl, *out, assign_history, static_cast<cudaStream_t>(stream), &nl);
+  g_launches += (uint64_t)nl;
   if (e != cudaSuccess) return cuda_fail(e, "launching V-Smooth prep");
   return VC_OK;
 }
@@ -219,6 +226,7 @@ vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* sha
   if ((st = ensure_device()) != VC_OK) return st;
   cudaError_t e = vc::launch_quant_qk(q, k, shape->dtype, shape->B, shape->S, shape->H, perm, *out,
                                       static_cast<cudaStream_t>(stream));
+  g_launches += 1;
   if (e != cudaSuccess) return cuda_fail(e, "launching Q/K quantisation");
   return VC_OK;
 }
@@ -268,6 +276,7 @@ static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* 
     e = vc::launch_attn_nvfp4(tq, tk, pv->v_codes, p, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorNotSupported) return fail(VC_ERR_UNSUPPORTED, "NVFP4-V attention is not built yet");
   }
+  g_launches += 1;
   if (e != cudaSuccess) return cuda_fail(e, "launching attention");
   return VC_OK;
 }

@@ -35,8 +35,9 @@ inline size_t assign_smem_bytes(int k, bool accum) {
 }
 
 cudaError_t prep_configure();
+// *nlaunch receives the number of kernels enqueued (memsets not counted).
 cudaError_t launch_prepare_v(const void* v, int dtype, const PrepPlan& plan, const vc_prepared_v_t& out,
-                             uint8_t* history, cudaStream_t st);
+                             uint8_t* history, cudaStream_t st, int* nlaunch);
 cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int S, int H, const int32_t* perm,
                             const vc_qk_fp8_t& out, cudaStream_t st);
 

@@ -477,14 +477,16 @@ __global__ void __launch_bounds__(128) quant_qk_kernel(const T* __restrict__ q, 
 // --------------------------------------------------------------- launchers
 template <typename T>
 static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_prepared_v_t& out,
-                                      uint8_t* history, cudaStream_t st) {
+                                      uint8_t* history, cudaStream_t st, int* nlaunch) {
   const int S = pl.S, H = pl.H, BH = pl.B * pl.H, k = pl.k;
   cudaError_t e;
+  int n = 0;
   if ((e = cudaMemsetAsync(pl.amax, 0, sizeof(unsigned) * BH, st)) != cudaSuccess) return e;
   if (pl.mode == VC_MODE_VSMOOTH) {
     if ((e = cudaMemsetAsync(pl.sums, 0, sizeof(unsigned long long) * BH * k * kD, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(pl.counts, 0, sizeof(int) * BH * k, st)) != cudaSuccess) return e;
     kmeans_init_kernel<T><<<BH, 128, 0, st>>>(v, S, H, k, pl.seed, pl.cent);
+    ++n;
     const dim3 grid(pl.nchunks, BH);
     const size_t sm_acc = assign_smem_bytes(k, true), sm_fin = assign_smem_bytes(k, false);
     for (int it = 0; it < pl.iters; ++it) {
@@ -493,15 +495,19 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
         kmeans_assign_kernel<T, true><<<grid, kTile, sm_acc, st>>>(v, S, H, k, pl.cent, pl.sums, pl.counts,
                                                                    pl.assign, nullptr, hist_t);
         kmeans_update_kernel<<<BH, 128, 0, st>>>(k, pl.cent, pl.sums, pl.counts);
+        n += 2;
       } else {
         kmeans_assign_kernel<T, false><<<grid, kTile, sm_fin, st>>>(v, S, H, k, pl.cent, pl.sums, pl.counts,
                                                                     pl.assign, pl.hist, hist_t);
+        ++n;
       }
     }
     perm_offsets_kernel<<<BH, 32, 0, st>>>(k, pl.nchunks, pl.hist, pl.offs);
     perm_scatter_kernel<<<grid, kChunk, 0, st>>>(S, k, pl.assign, pl.offs, out.perm);
+    n += 2;
   } else {
     identity_perm_kernel<<<dim3(std::max(1, std::min(1024, (S + 255) / 256)), BH), 256, 0, st>>>(S, out.perm);
+    ++n;
   }
   const dim3 gb(pl.nb, BH);
   block_stats_kernel<T><<<gb, 128, 0, st>>>(v, S, H, out.perm, out.mu, pl.amax);
@@ -513,14 +519,15 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
                                                                          pl.amax, out.v_codes, out.v_scales,
                                                                          out.s_v);
   }
+  *nlaunch = n + 2;
   return cudaGetLastError();
 }
 
 cudaError_t launch_prepare_v(const void* v, int dtype, const PrepPlan& pl, const vc_prepared_v_t& out,
-                             uint8_t* history, cudaStream_t st) {
+                             uint8_t* history, cudaStream_t st, int* nlaunch) {
   if (dtype == VC_DTYPE_BF16)
-    return launch_prepare_v_t(static_cast<const __nv_bfloat16*>(v), pl, out, history, st);
-  return launch_prepare_v_t(static_cast<const __half*>(v), pl, out, history, st);
+    return launch_prepare_v_t(static_cast<const __nv_bfloat16*>(v), pl, out, history, st, nlaunch);
+  return launch_prepare_v_t(static_cast<const __half*>(v), pl, out, history, st, nlaunch);
 }
 
 cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int S, int H, const int32_t* perm,

@@ -45,8 +45,8 @@ def softmax_scale(d=D_HEAD):
     return 1.0 / math.sqrt(d)
 
 
-def _gen(seed, stream):
-    g = torch.Generator()
+def _gen(seed, stream, device="cpu"):
+    g = torch.Generator(device=device)
     g.manual_seed(int(seed) * 1000 + STREAM[stream])
     return g
 
@@ -58,56 +58,60 @@ def workload(name, **overrides):
     return cfg
 
 
-def make_qkv(B, S, H, recipe="mixture", seed=0, dtype=torch.bfloat16, chunk=8192, **_):
-    """Return CPU tensors Q, K, V of shape [B, S, H, 128] in ``dtype``.
+def make_qkv(B, S, H, recipe="mixture", seed=0, dtype=torch.bfloat16, chunk=8192, device="cpu", **_):
+    """Return tensors Q, K, V of shape [B, S, H, 128] in ``dtype`` on ``device``.
 
     Drawn chunk by chunk along S (fixed chunk size, so the values do not depend
-    on available memory) and converted to ``dtype`` as they are drawn.
+    on available memory) and converted to ``dtype`` as they are drawn. The values
+    depend on the device's generator: the same seed gives the same recipe but not
+    the same numbers on "cpu" and "cuda" (tests use "cpu"; the benchmark draws
+    its large workloads on the GPU).
     """
     D = D_HEAD
     shape = (B, S, H, D)
-    Q = torch.empty(shape, dtype=dtype)
-    K = torch.empty(shape, dtype=dtype)
-    V = torch.empty(shape, dtype=dtype)
-    gq, gk, gv = _gen(seed, "q"), _gen(seed, "k"), _gen(seed, "v")
+    Q = torch.empty(shape, dtype=dtype, device=device)
+    K = torch.empty(shape, dtype=dtype, device=device)
+    V = torch.empty(shape, dtype=dtype, device=device)
+    g = lambda name: _gen(seed, name, device)
+    gq, gk, gv = g("q"), g("k"), g("v")
     if recipe == "normal":
         for s0 in range(0, S, chunk):
             n = min(chunk, S - s0)
-            Q[:, s0:s0 + n] = torch.randn((B, n, H, D), generator=gq).to(dtype)
-            K[:, s0:s0 + n] = torch.randn((B, n, H, D), generator=gk).to(dtype)
-            V[:, s0:s0 + n] = torch.randn((B, n, H, D), generator=gv).to(dtype)
-        go = _gen(seed, "outliers")
+            Q[:, s0:s0 + n] = torch.randn((B, n, H, D), generator=gq, device=device).to(dtype)
+            K[:, s0:s0 + n] = torch.randn((B, n, H, D), generator=gk, device=device).to(dtype)
+            V[:, s0:s0 + n] = torch.randn((B, n, H, D), generator=gv, device=device).to(dtype)
+        go = g("outliers")
         for b in range(B):
             for h in range(H):
-                pos = torch.randperm(S, generator=go)[: min(4, S)]
+                pos = torch.randperm(S, generator=go, device=device)[: min(4, S)]
                 V[b, pos, h] = (V[b, pos, h].float() * 16.0).to(dtype)
         return Q, K, V
     if recipe != "mixture":
         raise ValueError(recipe)
-    gl = _gen(seed, "lam")
-    lam_q = torch.exp(0.5 * torch.randn((H, D), generator=gl))
-    lam_k = torch.exp(0.5 * torch.randn((H, D), generator=gl))
-    centres = 2.0 * torch.randn((B, H, 16, D), generator=_gen(seed, "centres"))
-    gc = _gen(seed, "choice")
-    hidx = torch.arange(H).view(1, 1, H)
+    gl = g("lam")
+    lam_q = torch.exp(0.5 * torch.randn((H, D), generator=gl, device=device))
+    lam_k = torch.exp(0.5 * torch.randn((H, D), generator=gl, device=device))
+    centres = 2.0 * torch.randn((B, H, 16, D), generator=g("centres"), device=device)
+    gc = g("choice")
+    hidx = torch.arange(H, device=device).view(1, 1, H)
     for s0 in range(0, S, chunk):
         n = min(chunk, S - s0)
-        Q[:, s0:s0 + n] = (torch.randn((B, n, H, D), generator=gq) * lam_q).to(dtype)
-        K[:, s0:s0 + n] = (torch.randn((B, n, H, D), generator=gk) * lam_k).to(dtype)
-        choice = torch.randint(0, 16, (B, n, H), generator=gc)
-        bidx = torch.arange(B).view(B, 1, 1)
-        v = centres[bidx, hidx, choice] + 0.3 * torch.randn((B, n, H, D), generator=gv)
+        Q[:, s0:s0 + n] = (torch.randn((B, n, H, D), generator=gq, device=device) * lam_q).to(dtype)
+        K[:, s0:s0 + n] = (torch.randn((B, n, H, D), generator=gk, device=device) * lam_k).to(dtype)
+        choice = torch.randint(0, 16, (B, n, H), generator=gc, device=device)
+        bidx = torch.arange(B, device=device).view(B, 1, 1)
+        v = centres[bidx, hidx, choice] + 0.3 * torch.randn((B, n, H, D), generator=gv, device=device)
         V[:, s0:s0 + n] = v.to(dtype)
-    go = _gen(seed, "outliers")
+    go = g("outliers")
     n_out = max(1, round(0.01 * S))
     for b in range(B):
         for h in range(H):
-            pos = torch.randperm(S, generator=go)[:n_out]
+            pos = torch.randperm(S, generator=go, device=device)[:n_out]
             V[b, pos, h] = (V[b, pos, h].float() * 20.0).to(dtype)
     return Q, K, V
 
 
-def make_workload(name, seed=0, dtype=torch.bfloat16, **overrides):
+def make_workload(name, seed=0, dtype=torch.bfloat16, device="cpu", **overrides):
     cfg = workload(name, **overrides)
-    Q, K, V = make_qkv(cfg["B"], cfg["S"], cfg["H"], recipe=cfg["recipe"], seed=seed, dtype=dtype)
+    Q, K, V = make_qkv(cfg["B"], cfg["S"], cfg["H"], recipe=cfg["recipe"], seed=seed, dtype=dtype, device=device)
     return cfg, Q, K, V

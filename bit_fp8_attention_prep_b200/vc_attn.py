@@ -23,7 +23,8 @@ VC_MODE_VSMOOTH, VC_MODE_MEANONLY = 0, 1
 
 # every symbol declared in include/vc_attn.h and include/vc_attn_testing.h
 ABI_SYMBOLS = [
-    "vc_attn_version", "vc_attn_last_error", "vc_attn_prepare_v_workspace_bytes", "vc_attn_prepare_v",
+    "vc_attn_version", "vc_attn_last_error", "vc_attn_launch_count", "vc_attn_prepare_v_workspace_bytes",
+    "vc_attn_prepare_v",
     "vc_attn_quant_qk", "vc_attn_forward", "vc_attn_forward_nvfp4v",
 ]
 TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
@@ -71,6 +72,8 @@ def load():
     P = ctypes.POINTER
     lib.vc_attn_version.restype = i32
     lib.vc_attn_last_error.restype = ctypes.c_char_p
+    lib.vc_attn_launch_count.restype = u64
+    lib.vc_attn_launch_count.argtypes = []
     lib.vc_attn_prepare_v_workspace_bytes.restype = sz
     lib.vc_attn_prepare_v_workspace_bytes.argtypes = [P(Shape), P(VSmoothCfg)]
     lib.vc_attn_prepare_v.restype = i32
@@ -208,6 +211,70 @@ def attention(q, k, v, softmax_scale=None, k_p=8, kmeans_k=16, iters=4, seed=0, 
     qk = quant_qk(q, k, pv["perm"])
     o = forward(qk, pv, shape_of(q), softmax_scale, k_p)
     return o.view(q.shape)
+
+
+class Plan:
+    """Preallocated buffers for repeated calls on one shape (the form a serving
+    loop or the benchmark uses): the prepared V, the Q/K codes, the prep
+    workspace, O and a device status word, all owned by this object.
+
+    ``run(q, k, v)`` enqueues the three calls (prepare_v, quant_qk, forward) on
+    the current stream and returns O; nothing is allocated per call.
+    """
+
+    def __init__(self, B, S, H, dtype=torch.bfloat16, k=16, iters=4, seed=0, fmt="e4m3", k_p=8,
+                 softmax_scale=None, device=None, mode="vsmooth"):
+        self.lib = load()
+        dev = torch.device(device if device is not None else "cuda")
+        self.shape = Shape(B, S, H, 128, VC_DTYPE_BF16 if dtype == torch.bfloat16 else VC_DTYPE_F16)
+        self.cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
+                              VC_MODE_MEANONLY if mode == "meanonly" else VC_MODE_VSMOOTH)
+        self.fmt, self.k_p = fmt, int(k_p)
+        self.softmax_scale = 1.0 / math.sqrt(128) if softmax_scale is None else float(softmax_scale)
+        nb = num_blocks(S)
+        Sp = nb * 128
+        e = lambda shp, dt: torch.empty(shp, dtype=dt, device=dev)
+        self.perm, self.mu, self.s_v = e((B, H, S), torch.int32), e((B, H, nb, 128), torch.float32), e((B, H), torch.float32)
+        if fmt == "nvfp4":
+            self.v_codes, self.v_scales = e((B, H, 128, Sp // 2), torch.uint8), e((B, H, 128, Sp // 16), torch.uint8)
+        else:
+            self.v_codes, self.v_scales = e((B, H, 128, Sp), torch.uint8), None
+        self.q_codes, self.k_codes = e((B, H, Sp, 128), torch.uint8), e((B, H, Sp, 128), torch.uint8)
+        self.q_scales, self.k_scales = e((B, H, nb), torch.float32), e((B, H, nb), torch.float32)
+        self.o = e((B, S, H, 128), torch.bfloat16)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.ws_bytes = self.lib.vc_attn_prepare_v_workspace_bytes(ctypes.byref(self.shape), ctypes.byref(self.cfg))
+        if self.ws_bytes == 0:
+            raise VCError(VC_ERR_INVALID_ARG, "invalid shape or config")
+        self._ws = e((self.ws_bytes + 256,), torch.uint8)
+        self.ws_ptr = ctypes.c_void_p(self._ws.data_ptr() + (-self._ws.data_ptr()) % 256)
+        self._pv = PreparedV(_ptr(self.perm), _ptr(self.mu), _ptr(self.v_codes), _ptr(self.v_scales), _ptr(self.s_v))
+        self._qk = QKFP8(_ptr(self.q_codes), _ptr(self.q_scales), _ptr(self.k_codes), _ptr(self.k_scales))
+        self._fwd = self.lib.vc_attn_forward_nvfp4v if fmt == "nvfp4" else self.lib.vc_attn_forward
+
+    def prepare_v(self, v):
+        _check(self.lib.vc_attn_prepare_v(_ptr(v), ctypes.byref(self.shape), ctypes.byref(self.cfg),
+                                          ctypes.byref(self._pv), self.ws_ptr, self.ws_bytes, None, _stream()))
+
+    def quant_qk(self, q, k):
+        _check(self.lib.vc_attn_quant_qk(_ptr(q), _ptr(k), ctypes.byref(self.shape), _ptr(self.perm),
+                                         ctypes.byref(self._qk), _stream()))
+
+    def forward(self, out=None):
+        o = self.o if out is None else out
+        _check(self._fwd(ctypes.byref(self._qk), ctypes.byref(self._pv), ctypes.byref(self.shape),
+                         self.softmax_scale, self.k_p, _ptr(o), _ptr(self.status), _stream()))
+        return o
+
+    def run(self, q, k, v, out=None):
+        self.prepare_v(v)
+        self.quant_qk(q, k)
+        return self.forward(out)
+
+
+def launch_count():
+    """Kernels the library has enqueued since it was loaded."""
+    return int(load().vc_attn_launch_count())
 
 
 # ------------------------------------------------------------------ test hooks

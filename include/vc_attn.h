@@ -109,6 +109,11 @@ int32_t vc_attn_version(void);
 /* Message for the last error returned on the calling thread ("" if none). */
 const char* vc_attn_last_error(void);
 
+/* Number of CUDA kernels this library has enqueued since it was loaded, over
+ * all threads and devices (memset nodes not counted). Monotone; for measuring
+ * how many launches a sequence of calls makes. */
+uint64_t vc_attn_launch_count(void);
+
 /* Bytes of workspace vc_attn_prepare_v needs for this shape and config
  * (0 if the arguments are invalid). */
 size_t vc_attn_prepare_v_workspace_bytes(const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg);
