@@ -36,7 +36,7 @@ ATTN_SRC = os.path.join(ROOT, "bit_fp8_attention_prep_b200", "csrc", "vc_attn_fw
 # DRAM bytes (read + write) of one attention launch on the default workload, from
 # the ncu capture summarised in profiles/; valid only while the kernel source
 # hashes to the recorded value (otherwise traffic is reported as null).
-ATTN_TRAFFIC = {"sha256_16": None, "bytes_per_launch": None}
+ATTN_TRAFFIC = {"sha256_16": "c84b739e2406d674", "bytes_per_launch": 8 * (207.309568e6 + 109.4784e6)}
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 FALLBACK_HBM_GBS = 6650.0
 
