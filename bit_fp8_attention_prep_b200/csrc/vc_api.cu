@@ -291,4 +291,50 @@ vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t*
   return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, true);
 }
 
+// ------------------------------------------------------------ fixed-scratch prep
+// vc_attn_prepare_v_noalloc: the same prep with its scratch in this file-scope
+// device array instead of a caller workspace. In host code `g_noalloc_scratch`
+// names a host-side stand-in, not device memory, so its device address is
+// looked up once per device with cudaGetSymbolAddress (with that device current)
+// and only that address is handed to the kernels.
+}  // extern "C"
+
+namespace {
+static __device__ __align__(256) uint8_t g_noalloc_scratch[VC_ATTN_NOALLOC_SCRATCH_BYTES];
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64];  // device address of g_noalloc_scratch, per device (null until set up)
+}  // namespace
+
+extern "C" {
+
+vc_status_t vc_attn_prepare_v_noalloc(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                                      const vc_prepared_v_t* out, uint8_t* assign_history, void* stream) {
+  g_last_error.clear();
+  vc_status_t st;
+  if ((st = check_shape(shape)) != VC_OK) return st;
+  if ((st = check_cfg(cfg)) != VC_OK) return st;
+  const size_t need = ws_layout(shape, cfg).total;
+  if (need > VC_ATTN_NOALLOC_SCRATCH_BYTES)
+    return fail(VC_ERR_WORKSPACE,
+                "this problem needs %zu bytes of prep scratch; the fixed scratch of vc_attn_prepare_v_noalloc "
+                "holds %zu bytes (use vc_attn_prepare_v with a caller workspace)",
+                need, (size_t)VC_ATTN_NOALLOC_SCRATCH_BYTES);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(VC_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the fixed prep scratch");
+      g_noalloc_addr[dev] = p;
+    }
+    scratch = g_noalloc_addr[dev];
+  }
+  return vc_attn_prepare_v(v, shape, cfg, out, scratch, VC_ATTN_NOALLOC_SCRATCH_BYTES, assign_history, stream);
+}
+
 }  // extern "C"

@@ -25,8 +25,9 @@ VC_MODE_VSMOOTH, VC_MODE_MEANONLY = 0, 1
 ABI_SYMBOLS = [
     "vc_attn_version", "vc_attn_last_error", "vc_attn_launch_count", "vc_attn_prepare_v_workspace_bytes",
     "vc_attn_prepare_v",
-    "vc_attn_quant_qk", "vc_attn_forward", "vc_attn_forward_nvfp4v",
+    "vc_attn_quant_qk", "vc_attn_forward", "vc_attn_forward_nvfp4v", "vc_attn_prepare_v_noalloc",
 ]
+NOALLOC_SCRATCH_BYTES = 8 << 20   # VC_ATTN_NOALLOC_SCRATCH_BYTES
 TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
                 "vc_attn_test_bounded_wait"]
 
@@ -78,6 +79,8 @@ def load():
     lib.vc_attn_prepare_v_workspace_bytes.argtypes = [P(Shape), P(VSmoothCfg)]
     lib.vc_attn_prepare_v.restype = i32
     lib.vc_attn_prepare_v.argtypes = [vp, P(Shape), P(VSmoothCfg), P(PreparedV), vp, sz, vp, vp]
+    lib.vc_attn_prepare_v_noalloc.restype = i32
+    lib.vc_attn_prepare_v_noalloc.argtypes = [vp, P(Shape), P(VSmoothCfg), P(PreparedV), vp, vp]
     lib.vc_attn_quant_qk.restype = i32
     lib.vc_attn_quant_qk.argtypes = [vp, vp, P(Shape), vp, P(QKFP8), vp]
     for name in ("vc_attn_forward", "vc_attn_forward_nvfp4v"):
@@ -163,6 +166,35 @@ def prepare_v(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", history=Fals
     out["workspace"] = ws
     out["history"] = hist
     out["fmt"] = fmt
+    return out
+
+
+def prepare_v_noalloc(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", history=False):
+    """As ``prepare_v`` but through vc_attn_prepare_v_noalloc: no workspace is
+    passed; the library's fixed device scratch is used. The outputs are still
+    allocated here (by torch), as the caller's buffers."""
+    lib = load()
+    sh = shape_of(v)
+    cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
+                     VC_MODE_MEANONLY if mode == "meanonly" else VC_MODE_VSMOOTH)
+    B, S, H = sh.B, sh.S, sh.H
+    nb = num_blocks(S)
+    Sp = nb * 128
+    dev = v.device
+    out = dict(perm=torch.empty((B, H, S), dtype=torch.int32, device=dev),
+               mu=torch.empty((B, H, nb, 128), dtype=torch.float32, device=dev),
+               s_v=torch.empty((B, H), dtype=torch.float32, device=dev), fmt=fmt)
+    if fmt == "nvfp4":
+        out["v_codes"] = torch.empty((B, H, 128, Sp // 2), dtype=torch.uint8, device=dev)
+        out["v_scales"] = torch.empty((B, H, 128, Sp // 16), dtype=torch.uint8, device=dev)
+    else:
+        out["v_codes"] = torch.empty((B, H, 128, Sp), dtype=torch.uint8, device=dev)
+        out["v_scales"] = None
+    hist = torch.empty((iters, B, H, S), dtype=torch.uint8, device=dev) if history else None
+    pv = PreparedV(_ptr(out["perm"]), _ptr(out["mu"]), _ptr(out["v_codes"]), _ptr(out["v_scales"]), _ptr(out["s_v"]))
+    _check(lib.vc_attn_prepare_v_noalloc(_ptr(v), ctypes.byref(sh), ctypes.byref(cfg), ctypes.byref(pv), _ptr(hist),
+                                         _stream()))
+    out["history"] = hist
     return out
 
 

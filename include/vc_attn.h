@@ -169,6 +169,33 @@ vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t*
                                    const vc_shape_t* shape, float softmax_scale, int32_t k_p,
                                    void* o, int32_t* dev_status, void* stream);
 
+/* Size of the fixed device scratch used by vc_attn_prepare_v_noalloc: 8 MiB. */
+#define VC_ATTN_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/* V-Smooth prep exactly as vc_attn_prepare_v, but without a caller workspace:
+ * the k-means and sort scratch lives in a fixed device array that this library
+ * owns (VC_ATTN_NOALLOC_SCRATCH_BYTES per GPU, reserved on every GPU that loads
+ * the library until the process exits). The paper has no counterpart; this is a
+ * convenience for callers that cannot allocate device memory themselves, such as
+ * a plugin that is handed only its input and output buffers by a host framework
+ * with its own memory pool, or a latency-critical loop that must not call
+ * cudaMalloc (which can synchronise the device). Inputs and outputs are still
+ * caller-owned, as for vc_attn_prepare_v; nothing is allocated or freed.
+ *  - Fits when vc_attn_prepare_v_workspace_bytes(shape, cfg) <=
+ *    VC_ATTN_NOALLOC_SCRATCH_BYTES (about 6 MB for B=1, H=56, S=73397, k=16);
+ *    larger problems return VC_ERR_WORKSPACE with a message naming both sizes
+ *    (use vc_attn_prepare_v with a workspace for them).
+ *  - The first call on a device looks up the array's device address there
+ *    (one-time set-up per device, with that device current); make that first
+ *    call before any stream capture.
+ *  - Every call on a device shares the one array, and it keeps the last call's
+ *    contents (each call clears what must start at zero). Calls whose work
+ *    overlaps on the GPU (on different streams, or from different threads
+ *    without ordering) race on it: serialise them on one stream.
+ * Arguments, outputs and other errors are those of vc_attn_prepare_v. */
+vc_status_t vc_attn_prepare_v_noalloc(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                                      const vc_prepared_v_t* out, uint8_t* assign_history, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
