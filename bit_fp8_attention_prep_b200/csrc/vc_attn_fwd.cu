@@ -10,22 +10,31 @@
 // the block row sums of P ("restores that mean from the row sum the online
 // softmax already maintains").
 //
-// One CTA = one 128-row query tile of one (b, h); it walks the (permuted) key
-// blocks j = 0 .. nb-1:
-//   warp 4 (TMA):     Q once; K_j, V^T_j and mu_j into ring buffers
-//   warp 5 (MMA):     S_j = Q K_j^T   -> TMEM (two S buffers, 128 columns each)
-//                     O  += P_{j-1} V_{j-1} -> TMEM (128 columns), issued after
-//                     QK_j so that the tensor core works while warps 0-3 cast
-//   warps 0-3:        row r = thread: tile max -> integer frame M (ceil of the
-//                     log2-domain max, running) -> ExpCast codes -> P_j in shared
-//                     memory (128-B swizzled K-major, the A operand of PV);
-//                     rescale O / l / mean accumulator by 2^(M_old - M_new) when
-//                     the frame moves; l += r_j, mean += r_j * mu_j (r_j = row
-//                     sum of the cast P over block j); epilogue
-//                     O = (s_V * O_acc + mean) / l -> BF16.
-// All operands are E4M3; the MMA is tcgen05.mma kind::f8f6f4, M=128 N=128 K=32.
+// One CTA = two 128-row query tiles (t = 0, 1) of one (b, h); both walk all key
+// blocks j = 0 .. nb-1 (permuted order), sharing every K/V tile.
+//   warps 0-3  softmax group of query tile 0 (thread = query row)
+//   warps 4-7  softmax group of query tile 1
+//   warp  8    TMA: both Q tiles once; K_j, V^T_j and mu_j into rings
+//   warp  9    MMA issuer (one thread)
+// Tensor memory (512 columns): S_t = [128t, 128t+128), O_t = [256+128t, ...).
+// Per block j and tile t the tensor core runs, in this order per tile:
+//   QK   S_t  = Q_t K_j^T                 kind::f8f6f4, M=128 N=128 K=128
+//   PV   O_t += P_t V_j                   P_t = ExpCast codes (smem), V_j = residual codes
+//   ROW  S_t[:, 0:16) = P_t 1             exact row sums r of the cast P
+//   MEAN after every 5 blocks:  O_t += R_t M    kind::f16 with bf16 operands:
+//        R_t = the blocks' row sums, M = their block means / s_V, each split into
+//        bf16 hi/lo parts (r_hi m_hi + r_hi m_lo + r_lo m_hi, three K slots a block);
+//        both operands of a tile's mean MMA live in that tile's own 128-B-swizzled
+//        smem tile (R in K chunks 0-1, M in chunks 2-3, alternating by batch), and
+//        the softmax group writes it only while no MMA of its tile is in flight
+// so O_t accumulates the whole output in residual-code units; the epilogue is
+// O = s_V O_t / l. The softmax thread of row i keeps the integer running frame
+// F (ceil of the largest log2-domain score so far); a block is cast in the frame
+// current after it; when F moves, O_t, l and the not-yet-issued row sums are
+// multiplied by the exact power of two 2^(F_old - F_new).
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "vc_common.cuh"
@@ -36,24 +45,26 @@ namespace vc {
 namespace {
 
 constexpr int kKStages = 3;
-constexpr int kVStages = 2;
-constexpr uint32_t kTileBytes = 128 * 128;  // one 128 x 128 E4M3 tile
-constexpr int kThreads = 192;
+constexpr int kVStages = 3;
+constexpr uint32_t kTileBytes = 128 * 128;  // one 128 x 128 E4M3 tile (or 128 x 64 bf16)
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr int kMeanBlocks = 5;              // key blocks per mean MMA (3 K slots each: 15 of 16)
+constexpr int kMeanChunks = 2;              // 16-slot K chunks per operand (R: 0-1, M: 2-3)
+constexpr uint32_t kOneE4M3x4 = 0x38383838u;
 
-struct __align__(1024) SmemE4M3 {
-  uint8_t q[kTileBytes];
+struct __align__(1024) SmemAttn {
+  uint8_t q[2][kTileBytes];
   uint8_t k[kKStages][kTileBytes];
   uint8_t v[kVStages][kTileBytes];
   uint8_t p[2][kTileBytes];
+  uint8_t mop[2][kTileBytes];    // bf16 operands of the mean MMA, one tile per query tile
+  uint8_t ones[2048];            // E4M3 1.0: B operand of the row-sum MMA (N=16, K=128)
   float mu[kVStages][128];
   uint64_t q_full;
   uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_empty[2];
-  uint64_t o_final;
+  uint64_t v_full[kVStages], v_empty[kVStages], mu_empty[kVStages];
+  uint64_t s_full[2], p_full[2], o_done[2], r_free[2], fin_ready[2], o_final[2];
   uint64_t mma_drain;
   uint32_t tmem_base;
   int32_t abort_flag;
@@ -63,20 +74,37 @@ __device__ __forceinline__ float exp2_int(int n) {  // 2^n for integer n <= 0, e
   return n < -126 ? 0.0f : __int_as_float((127 + n) << 23);
 }
 
-__device__ __forceinline__ bool wait_or_abort(SmemE4M3& s, uint64_t* bar, uint32_t parity, const AttnParams& P) {
+__device__ __forceinline__ bool wait_or_abort(SmemAttn& s, uint64_t* bar, uint32_t parity, const AttnParams& P) {
   if (mbar_wait(bar, parity, P.wait_ns, P.status)) return true;
   s.abort_flag = 1;
   report_status(P.status, VC_ERR_TIMEOUT);
   return false;
 }
 
+// Byte offset of 16-bit element `slot` (K index 16*chunk + slot) of row `row` in
+// a 128-B-swizzled K-major operand tile (rows of 128 B, 8-row atoms).
+__device__ __forceinline__ uint32_t sw128_off16(int row, int chunk, int slot) {
+  const int kb = chunk * 32 + slot * 2;  // byte within the unswizzled 128-B row
+  return (uint32_t)(row * 128 + ((((kb >> 4) ^ (row & 7)) & 7) << 4) + (kb & 15));
+}
+
+__device__ __forceinline__ void st_bf16(uint8_t* base, uint32_t off, __nv_bfloat16 v) {
+  *reinterpret_cast<__nv_bfloat16*>(base + off) = v;
+}
+
+// x = hi + lo with hi = bf16(x), lo = bf16(x - hi): 16 significant bits, fp32 range.
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(x);
+  lo = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     vc_attn_fwd_e4m3_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
-  SmemE4M3& s = *reinterpret_cast<SmemE4M3*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SmemAttn& s = *reinterpret_cast<SmemAttn*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, bh = blockIdx.y;
+  const int pair = blockIdx.x, bh = blockIdx.y;
   const int nkv = P.nb;
 
   if (threadIdx.x == 0) {
@@ -88,18 +116,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kVStages; ++i) {
       mbar_init(&s.v_full[i], 1);
       mbar_init(&s.v_empty[i], 1);
+      mbar_init(&s.mu_empty[i], 256);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.s_full[i], 1);
-      mbar_init(&s.s_empty[i], 128);
-      mbar_init(&s.p_full[i], 128);
-      mbar_init(&s.p_empty[i], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s.s_full[t], 1);
+      mbar_init(&s.p_full[t], 128);
+      mbar_init(&s.o_done[t], 1);
+      mbar_init(&s.r_free[t], 128);
+      mbar_init(&s.fin_ready[t], 128);
+      mbar_init(&s.o_final[t], 1);
     }
-    mbar_init(&s.o_final, 1);
     mbar_init(&s.mma_drain, 1);
     s.abort_flag = 0;
     fence_barrier_init();
   }
+  // mean-MMA operands start at zero (unused K slots stay zero); the row-sum B
+  // operand is all E4M3 1.0 (every byte 0x38, so the swizzle does not matter)
+  for (int i = threadIdx.x; i < (int)(2 * kTileBytes / 16); i += kThreads)
+    *reinterpret_cast<uint4*>(&s.mop[0][0] + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = threadIdx.x; i < 2048 / 16; i += kThreads)
+    *reinterpret_cast<uint4*>(s.ones + i * 16) = make_uint4(kOneE4M3x4, kOneE4M3x4, kOneE4M3x4, kOneE4M3x4);
+  fence_proxy_async_smem();
   if (warp == 0) {
     tmem_alloc(&s.tmem_base, kTmemCols);
     tmem_relinquish();
@@ -109,15 +146,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const int rowq = bh * P.S_pad + qt * 128;
-      mbar_arrive_expect_tx(&s.q_full, kTileBytes);
-      tma_load_2d(s.q, &tmQ, &s.q_full, 0, rowq);
+      const int rowq = bh * P.S_pad + pair * 256;
+      mbar_arrive_expect_tx(&s.q_full, 2 * kTileBytes);
+      tma_load_2d(s.q[0], &tmQ, &s.q_full, 0, rowq);
+      tma_load_2d(s.q[1], &tmQ, &s.q_full, 0, rowq + 128);  // past the head's last tile: unused rows
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < nkv && !*(volatile int32_t*)&s.abort_flag; ++j) {
         const int ks = j % kKStages;
@@ -126,14 +164,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(s.k[ks], &tmK, &s.k_full[ks], 0, bh * P.S_pad + j * 128);
         k_issued = j + 1;
         const int vs = j % kVStages;
-        if (!wait_or_abort(s, &s.v_empty[vs], ((j / kVStages) & 1) ^ 1, P)) break;
+        const uint32_t ph = ((j / kVStages) & 1) ^ 1;
+        if (!wait_or_abort(s, &s.v_empty[vs], ph, P)) break;
+        if (!wait_or_abort(s, &s.mu_empty[vs], ph, P)) break;
         mbar_arrive_expect_tx(&s.v_full[vs], kTileBytes + 512);
         tma_load_2d(s.v[vs], &tmV, &s.v_full[vs], j * 128, bh * 128);
         bulk_load(s.mu[vs], P.mu + ((size_t)bh * P.nb + j) * 128, 512, &s.v_full[vs]);
         v_issued = j + 1;
       }
-      // Copies still in flight must land before the CTA exits (normally they all
-      // have been consumed already and these waits return at once).
+      // copies still in flight must land before the CTA exits
       const uint64_t drain_ns = 100000000ull;
       mbar_wait(&s.q_full, 0, drain_ns, nullptr);
       for (int j = max(0, k_issued - kKStages); j < k_issued; ++j)
@@ -141,39 +180,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = max(0, v_issued - kVStages); j < v_issued; ++j)
         mbar_wait(&s.v_full[j % kVStages], (j / kVStages) & 1, drain_ns, nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
-      bool ok = wait_or_abort(s, &s.q_full, 0, P);
-      const uint64_t qdesc = sdesc_k_sw128(smem_u32(s.q));
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {
-          const int ks = j % kKStages, sb = j & 1;
-          if (!(ok = wait_or_abort(s, &s.k_full[ks], (j / kKStages) & 1, P))) break;
-          if (!(ok = wait_or_abort(s, &s.s_empty[sb], ((j >> 1) & 1) ^ 1, P))) break;
-          tc_fence_after();
-          const uint64_t kdesc = sdesc_k_sw128(smem_u32(s.k[ks]));
-          const uint32_t dS = tmem + (sb ? kColS1 : kColS0);
+      constexpr uint32_t id_qk = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
+      constexpr uint32_t id_row = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 16);
+      constexpr uint32_t id_mean = idesc_f32acc(kFmtBF16, kFmtBF16, 128, 128);
+      const uint64_t dq[2] = {sdesc_k_sw128(smem_u32(s.q[0])), sdesc_k_sw128(smem_u32(s.q[1]))};
+      const uint64_t dp[2] = {sdesc_k_sw128(smem_u32(s.p[0])), sdesc_k_sw128(smem_u32(s.p[1]))};
+      const uint64_t dm[2] = {sdesc_k_sw128(smem_u32(s.mop[0])), sdesc_k_sw128(smem_u32(s.mop[1]))};
+      const uint64_t dones = sdesc_k_sw128(smem_u32(s.ones));
+      bool ok = wait_or_abort(s, &s.q_full, 0, P) && wait_or_abort(s, &s.k_full[0], 0, P);
+      if (ok) {
+        tc_fence_after();
+        const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[0]));
+        for (int t = 0; t < 2; ++t) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(dS, qdesc + 2 * kk, kdesc + 2 * kk, idesc, kk > 0);
-          umma_commit(&s.s_full[sb]);
-          umma_commit(&s.k_empty[ks]);
+          for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(tmem + 128 * t, dq[t] + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
+          umma_commit(&s.s_full[t]);
         }
-        if (j >= 1) {
-          const int jj = j - 1, pb = jj & 1;
-          if (!(ok = wait_or_abort(s, &s.p_full[pb], (jj >> 1) & 1, P))) break;
-          if (!(ok = wait_or_abort(s, &s.v_full[jj % kVStages], (jj / kVStages) & 1, P))) break;
+        umma_commit(&s.k_empty[0]);
+      }
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int vs = j % kVStages;
+        const uint64_t dv = sdesc_k_sw128(smem_u32(s.v[vs]));
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!(ok = wait_or_abort(s, &s.p_full[t], j & 1, P))) break;
+          if (t == 0 && !(ok = wait_or_abort(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
           tc_fence_after();
-          const uint64_t pdesc = sdesc_k_sw128(smem_u32(s.p[pb]));
-          const uint64_t vdesc = sdesc_k_sw128(smem_u32(s.v[jj % kVStages]));
+          const uint32_t dO = tmem + 256 + 128 * t;
+          if (j >= 1 && (j - 1) % kMeanBlocks == kMeanBlocks - 1) {
+            const int ch = ((j - 1) / kMeanBlocks) % kMeanChunks;
+            umma_f16_ss(dO, dm[t] + 2 * ch, dm[t] + 2 * (kMeanChunks + ch), id_mean, 1u);
+          }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_f8f6f4_ss(tmem + kColO, pdesc + 2 * kk, vdesc + 2 * kk, idesc, (jj > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&s.p_empty[pb]);
-          umma_commit(&s.v_empty[jj % kVStages]);
-          if (jj == nkv - 1) umma_commit(&s.o_final);
+            umma_f8f6f4_ss(dO, dp[t] + 2 * kk, dv + 2 * kk, id_qk, (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(tmem + 128 * t, dp[t] + 2 * kk, dones + 2 * kk, id_row, kk > 0);
+          umma_commit(&s.o_done[t]);
         }
+        if (!ok) break;
+        umma_commit(&s.v_empty[vs]);
+        if (j + 1 < nkv) {
+          const int ks = (j + 1) % kKStages;
+          if (!(ok = wait_or_abort(s, &s.k_full[ks], ((j + 1) / kKStages) & 1, P))) break;
+          const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[ks]));
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (!(ok = wait_or_abort(s, &s.r_free[t], j & 1, P))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(tmem + 128 * t, dq[t] + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
+            umma_commit(&s.s_full[t]);
+          }
+          if (!ok) break;
+          umma_commit(&s.k_empty[ks]);
+        }
+      }
+      // the last (possibly partial) batch of block means, then the output is final
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (!(ok = wait_or_abort(s, &s.fin_ready[t], 0, P))) break;
+        tc_fence_after();
+        const int ch = ((nkv - 1) / kMeanBlocks) % kMeanChunks;
+        umma_f16_ss(tmem + 256 + 128 * t, dm[t] + 2 * ch, dm[t] + 2 * (kMeanChunks + ch), id_mean, 1u);
+        umma_commit(&s.o_final[t]);
       }
       // every MMA this thread issued has completed before TMEM is released
       umma_commit(&s.mma_drain);
@@ -181,131 +251,172 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int row = warp * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const float sQ = P.q_scales[(size_t)bh * P.nb + qt];
-    float Mrun = 0.0f, l = 0.0f;
-    float om[128];
-#pragma unroll
-    for (int d = 0; d < 128; ++d) om[d] = 0.0f;
+    const int t = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + 128 * t;
+    const uint32_t o_addr = tmem + lane_base + 256 + 128 * t;
+    const int qt = pair * 2 + t;
+    const bool q_valid = qt < P.nb;
+    const float sQ = q_valid ? P.q_scales[(size_t)bh * P.nb + qt] : 1.0f;
+    const float sV = P.s_v[bh];
+    const float inv_sV = __fdiv_rn(1.0f, sV);
+    uint8_t* const mo = s.mop[t];
+    uint8_t* const prow = s.p[t] + row * 128;
+    float F = 0.0f, l = 0.0f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1;
-      const uint32_t sph = (j >> 1) & 1;
-      if (!(ok = wait_or_abort(s, &s.s_full[sb], sph, P))) break;
+      if (!(ok = wait_or_abort(s, &s.s_full[t], j & 1, P))) break;
       tc_fence_after();
-      const uint32_t saddr = tmem + lane_base + (sb ? kColS1 : kColS0);
+      uint32_t raw[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, raw[c]);
+      tmem_ld_wait();
+      float sc[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) sc[i] = __uint_as_float(raw[i >> 5][i & 31]);
       const int valid = min(128, P.S - j * 128);
-      // pass 1: tile max of the raw scores (c > 0, so max(c t) = c max(t))
-      float tmax = -INFINITY;
+      if (valid < 128) {
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t r[32];
-        tmem_ld32(saddr + ch * 32, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (ch * 32 + i < valid) tmax = fmaxf(tmax, __uint_as_float(r[i]));
+        for (int i = 0; i < 128; ++i)
+          if (i >= valid) sc[i] = -INFINITY;
       }
+      // tile max of the raw scores (c > 0, so max(c t) = c max(t))
+      float m0 = sc[0], m1 = sc[1], m2 = sc[2], m3 = sc[3];
+#pragma unroll
+      for (int i = 4; i < 124; i += 8) {
+        m0 = fmax3(m0, sc[i + 0], sc[i + 1]);
+        m1 = fmax3(m1, sc[i + 2], sc[i + 3]);
+        m2 = fmax3(m2, sc[i + 4], sc[i + 5]);
+        m3 = fmax3(m3, sc[i + 6], sc[i + 7]);
+      }
+      m0 = fmax3(m0, sc[124], sc[125]);
+      m1 = fmax3(m1, sc[126], sc[127]);
+      const float tmax = fmaxf(fmax3(m0, m1, m2), m3);
       const float c = __fmul_rn(__fmul_rn(sQ, P.k_scales[(size_t)bh * P.nb + j]), P.kappa);
       const float Mtile = ceilf(__fmul_rn(c, tmax));
-      const float Mnew = j == 0 ? Mtile : fmaxf(Mrun, Mtile);
-      const bool resc = j > 0 && Mnew > Mrun;
-      const float alpha = resc ? exp2_int((int)(Mrun - Mnew)) : 1.0f;
-      const float bias = expcast_bias(P.bias_b, Mnew);
+      const float Fn = j == 0 ? Mtile : fmaxf(F, Mtile);
+      const bool resc = j > 0 && Fn > F;
+      const float alpha = resc ? exp2_int((int)(F - Fn)) : 1.0f;
+      const float bias = expcast_bias(P.bias_b, Fn);
       const float c8 = 8.0f * c;
-      const bool hot = fabsf(Mnew) < 1048576.0f;
-      // pass 2: codes -> P tile (swizzled), row sum of the cast P
-      if (!(ok = wait_or_abort(s, &s.p_empty[sb], sph ^ 1, P))) break;
-      uint8_t* prow = s.p[sb] + row * 128;
-      float rsum = 0.0f;
+      const bool hot = __all_sync(0xffffffffu, fabsf(Fn) < 524288.0f);
+      // ExpCast: one fma per score on the magic-biased fp32; the low byte is the code
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t r[32];
-        tmem_ld32(saddr + ch * 32, r);
-        tmem_ld_wait();
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t w[8];
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
+          const int i = cc * 32 + q4 * 4;
           float z[4];
+          if (hot) {
+            const float2 a = ffma2(make_float2(sc[i], sc[i + 1]), make_float2(c8, c8), make_float2(bias, bias));
+            const float2 b = ffma2(make_float2(sc[i + 2], sc[i + 3]), make_float2(c8, c8), make_float2(bias, bias));
+            z[0] = fmaxf(a.x, kMagic);
+            z[1] = fmaxf(a.y, kMagic);
+            z[2] = fmaxf(b.x, kMagic);
+            z[3] = fmaxf(b.y, kMagic);
+          } else {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = ch * 32 + q4 * 4 + e;
-            const float t = __uint_as_float(r[q4 * 4 + e]);
-            float zz = hot ? expcast_z(t, c8, bias) : __uint_as_float(0x4B400000u + expcast_code(t, c8, bias));
-            if (col >= valid) zz = kMagic;
-            z[e] = zz;
-            rsum += e4m3_to_f32(__float_as_uint(zz) & 0xFFu);
+            for (int e = 0; e < 4; ++e) z[e] = __uint_as_float(0x4B400000u + expcast_code(sc[i + e], c8, bias));
+          }
+          if (valid < 128) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (i + e >= valid) z[e] = kMagic;
           }
           w[q4] = pack_codes4(z[0], z[1], z[2], z[3]);
         }
-        const int c0 = (2 * ch) ^ (row & 7), c1 = (2 * ch + 1) ^ (row & 7);
+        const int c0 = (2 * cc) ^ (row & 7), c1 = (2 * cc + 1) ^ (row & 7);
         *reinterpret_cast<uint4*>(prow + c0 * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<uint4*>(prow + c1 * 16) = make_uint4(w[4], w[5], w[6], w[7]);
       }
-      tc_fence_before();
-      mbar_arrive(&s.s_empty[sb]);
       fence_proxy_async_smem();
-      // rescale the TMEM accumulator when the frame moved (after PV_{j-1} is done)
       if (__any_sync(0xffffffffu, resc)) {
-        const int jj = j - 1;
-        if (!(ok = wait_or_abort(s, &s.p_empty[jj & 1], (jj >> 1) & 1, P))) break;
-        tc_fence_after();
-        const uint32_t oaddr = tmem + lane_base + kColO;
+        // the frame moved: O_t (complete up to block j-1), l and the row sums not
+        // yet handed to a mean MMA are rescaled by the exact 2^(F_old - F_new)
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint32_t r[32];
-          tmem_ld32(oaddr + ch * 32, r);
+          tmem_ld32(o_addr + 32 * cc, r);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(oaddr + ch * 32, r);
+          tmem_st32(o_addr + 32 * cc, r);
         }
         tmem_st_wait();
+        if (resc) {
+          const int jp = j - 1, ch = (jp / kMeanBlocks) % kMeanChunks;
+          const int nslots = 3 * (jp % kMeanBlocks) + 3;
+          for (int sl = 0; sl < nslots; ++sl) {
+            __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(mo + sw128_off16(row, ch, sl));
+            *e = __float2bfloat16_rn(__bfloat162float(*e) * alpha);
+          }
+          fence_proxy_async_smem();
+        }
       }
-      // block-mean restore and row sum (same frame as O)
-      if (!(ok = wait_or_abort(s, &s.v_full[j % kVStages], (j / kVStages) & 1, P))) break;
-      const float4* mu4 = reinterpret_cast<const float4*>(s.mu[j % kVStages]);
-      l = __fmaf_rn(l, alpha, rsum);
-#pragma unroll
-      for (int d4 = 0; d4 < 32; ++d4) {
-        const float4 m = mu4[d4];
-        om[4 * d4 + 0] = __fmaf_rn(rsum, m.x, om[4 * d4 + 0] * alpha);
-        om[4 * d4 + 1] = __fmaf_rn(rsum, m.y, om[4 * d4 + 1] * alpha);
-        om[4 * d4 + 2] = __fmaf_rn(rsum, m.z, om[4 * d4 + 2] * alpha);
-        om[4 * d4 + 3] = __fmaf_rn(rsum, m.w, om[4 * d4 + 3] * alpha);
-      }
-      Mrun = Mnew;
+      l *= alpha;
+      F = Fn;
       tc_fence_before();
-      mbar_arrive(&s.p_full[sb]);
+      mbar_arrive(&s.p_full[t]);
+      // row sum of this block's cast P (tensor core), then the mean-MMA operands
+      if (!(ok = wait_or_abort(s, &s.o_done[t], j & 1, P))) break;
+      tc_fence_after();
+      const float r = __uint_as_float(tmem_ld1(s_addr));
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&s.r_free[t]);
+      l = __fadd_rn(l, r);
+      const int g = j % kMeanBlocks, ch = (j / kMeanBlocks) % kMeanChunks;
+      __nv_bfloat16 rh, rl;
+      split_bf16(r, rh, rl);
+      st_bf16(mo, sw128_off16(row, ch, 3 * g + 0), rh);
+      st_bf16(mo, sw128_off16(row, ch, 3 * g + 1), rh);
+      st_bf16(mo, sw128_off16(row, ch, 3 * g + 2), rl);
+      // thread `row` also writes channel `row` of this block's mean / s_V
+      const int vs = j % kVStages;
+      if (!(ok = wait_or_abort(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
+      const float m = __fmul_rn(s.mu[vs][row], inv_sV);
+      mbar_arrive(&s.mu_empty[vs]);
+      __nv_bfloat16 mh, ml;
+      split_bf16(m, mh, ml);
+      st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 0), mh);
+      st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 1), ml);
+      st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 2), mh);
+      const bool last = j == nkv - 1;
+      if (last)
+        for (int sl = 3 * g + 3; sl < 16; ++sl) {
+          st_bf16(mo, sw128_off16(row, ch, sl), __float2bfloat16_rn(0.0f));
+          st_bf16(mo, sw128_off16(row, kMeanChunks + ch, sl), __float2bfloat16_rn(0.0f));
+        }
+      if (g == kMeanBlocks - 1 || last) fence_proxy_async_smem();
     }
-    // epilogue: O = (s_V * O_acc + mean) / l, BF16, original query order
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(s, &s.o_final, 0, P));
     if (ok) {
+      mbar_arrive(&s.fin_ready[t]);
+      ok = __all_sync(0xffffffffu, wait_or_abort(s, &s.o_final[t], 0, P));
+    }
+    if (ok) {
+      // epilogue: O = s_V O_t / l, BF16, original query order and layout
       tc_fence_after();
       const int q = qt * 128 + row;
-      const float sV = P.s_v[bh];
-      const float rl = 1.0f / l;
+      const float scale = __fdiv_rn(sV, l);
       const int b = bh / P.H, h = bh % P.H;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(P.o) + (((size_t)b * P.S + q) * P.H + h) * 128;
-      const uint32_t oaddr = tmem + lane_base + kColO;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t r[32];
-        tmem_ld32(oaddr + ch * 32, r);
+        tmem_ld32(o_addr + 32 * cc, r);
         tmem_ld_wait();
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int d = ch * 32 + 2 * i;
-          const float a0 = __fmaf_rn(sV, __uint_as_float(r[2 * i]), om[d]) * rl;
-          const float a1 = __fmaf_rn(sV, __uint_as_float(r[2 * i + 1]), om[d + 1]) * rl;
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
+          __nv_bfloat162 b2 =
+              __floats2bfloat162_rn(__uint_as_float(r[2 * i]) * scale, __uint_as_float(r[2 * i + 1]) * scale);
           pk[i] = *reinterpret_cast<uint32_t*>(&b2);
         }
-        if (q < P.S) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+        if (q_valid && q < P.S) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
@@ -324,13 +435,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t attn_configure() {
   return cudaFuncSetAttribute(vc_attn_fwd_e4m3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)(sizeof(SmemE4M3) + 1024));
+                              (int)(sizeof(SmemAttn) + 1024));
 }
 
 cudaError_t launch_attn_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const AttnParams& p, cudaStream_t st) {
-  const dim3 grid(p.nb, p.B * p.H);
-  vc_attn_fwd_e4m3_kernel<<<grid, kThreads, sizeof(SmemE4M3) + 1024, st>>>(tq, tk, tv, p);
+  const dim3 grid((p.nb + 1) / 2, p.B * p.H);
+  vc_attn_fwd_e4m3_kernel<<<grid, kThreads, sizeof(SmemAttn) + 1024, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 

@@ -110,6 +110,27 @@ __device__ __forceinline__ uint32_t pack_codes4(float z0, float z1, float z2, fl
   return __byte_perm(lo, hi, 0x5410);       // a0, b0, c0, d0
 }
 
+// ---------------------------------------------------------------- packed fp32 math
+// Two fp32 fused multiply-adds in one instruction (sm_100 f32x2), each rounded
+// to nearest even exactly like __fmaf_rn.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t ra, rb, rc, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c.x), "f"(c.y));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+  float2 d;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
+}
+
+// max of three fp32 values in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
