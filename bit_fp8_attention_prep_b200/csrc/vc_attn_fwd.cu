@@ -12,10 +12,13 @@
 //
 // One CTA = two 128-row query tiles (t = 0, 1) of one (b, h); both walk all key
 // blocks j = 0 .. nb-1 (permuted order), sharing every K/V tile.
-//   warps 0-3  softmax group of query tile 0 (thread = query row)
-//   warps 4-7  softmax group of query tile 1
-//   warp  8    TMA: both Q tiles once; K_j, V^T_j and mu_j into rings
-//   warp  9    MMA issuer (one thread)
+//   warps 0-7   softmax group of query tile 0: two threads per query row, warps
+//               0-3 take score columns 0-63 and warps 4-7 columns 64-127 (a warp
+//               reaches the 32 tensor-memory lanes of its rank mod 4); the halves
+//               exchange their partial row maxima through shared memory
+//   warps 8-15  softmax group of query tile 1
+//   warp  16    TMA: both Q tiles once; K_j, V^T_j and mu_j into rings
+//   warp  17    MMA issuer (one thread)
 // Tensor memory (512 columns): S_t = [128t, 128t+128), O_t = [256+128t, ...).
 // Per block j and tile t the tensor core runs, in this order per tile:
 //   QK   S_t  = Q_t K_j^T                 kind::f8f6f4, M=128 N=128 K=128
@@ -47,7 +50,8 @@ namespace {
 constexpr int kKStages = 3;
 constexpr int kVStages = 3;
 constexpr uint32_t kTileBytes = 128 * 128;  // one 128 x 128 E4M3 tile (or 128 x 64 bf16)
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
+constexpr int kTmaWarp = 16, kMmaWarp = 17;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMeanBlocks = 5;              // key blocks per mean MMA (3 K slots each: 15 of 16)
 constexpr int kMeanChunks = 2;              // 16-slot K chunks per operand (R: 0-1, M: 2-3)
@@ -61,6 +65,7 @@ struct __align__(1024) SmemAttn {
   uint8_t mop[2][kTileBytes];    // bf16 operands of the mean MMA, one tile per query tile
   uint8_t ones[2048];            // E4M3 1.0: B operand of the row-sum MMA (N=16, K=128)
   float mu[kVStages][128];
+  float xmax[2][2][2][128];      // [block parity][query tile][column half][row] partial maxima
   uint64_t q_full;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages], mu_empty[kVStages];
@@ -120,10 +125,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s.s_full[t], 1);
-      mbar_init(&s.p_full[t], 128);
+      mbar_init(&s.p_full[t], 256);
       mbar_init(&s.o_done[t], 1);
-      mbar_init(&s.r_free[t], 128);
-      mbar_init(&s.fin_ready[t], 128);
+      mbar_init(&s.r_free[t], 256);
+      mbar_init(&s.fin_ready[t], 256);
       mbar_init(&s.o_final[t], 1);
     }
     mbar_init(&s.mma_drain, 1);
@@ -146,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  if (warp == 8) {
+  if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -180,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = max(0, v_issued - kVStages); j < v_issued; ++j)
         mbar_wait(&s.v_full[j % kVStages], (j / kVStages) & 1, drain_ns, nullptr);
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_qk = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
@@ -251,11 +256,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int t = warp >> 2;
+    const int t = warp >> 3;               // query tile
+    const int hf = (warp >> 2) & 1;        // score / output column half
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t s_addr = tmem + lane_base + 128 * t;
-    const uint32_t o_addr = tmem + lane_base + 256 + 128 * t;
+    const uint32_t o_addr = tmem + lane_base + 256 + 128 * t + 64 * hf;
     const int qt = pair * 2 + t;
     const bool q_valid = qt < P.nb;
     const float sQ = q_valid ? P.q_scales[(size_t)bh * P.nb + qt] : 1.0f;
@@ -264,88 +270,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* const mo = s.mop[t];
     uint8_t* const prow = s.p[t] + row * 128;
     float F = 0.0f, l = 0.0f;
-    bool ok = true;
+    bool ok = true, range_ok = true;
+    const float* const ksc = P.k_scales + (size_t)bh * P.nb;
+    float sK_next = ksc[0];
     for (int j = 0; j < nkv; ++j) {
+      const float sK = sK_next;                      // this block's K scale, loaded one block ahead
+      if (j + 1 < nkv) sK_next = ksc[j + 1];
       if (!(ok = wait_or_abort(s, &s.s_full[t], j & 1, P))) break;
       tc_fence_after();
-      uint32_t raw[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, raw[c]);
+      uint32_t raw[2][32];
+      tmem_ld32(s_addr + 64 * hf, raw[0]);
+      tmem_ld32(s_addr + 64 * hf + 32, raw[1]);
       tmem_ld_wait();
-      float sc[128];
+      float sc[64];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) sc[i] = __uint_as_float(raw[i >> 5][i & 31]);
-      const int valid = min(128, P.S - j * 128);
-      if (valid < 128) {
+      for (int i = 0; i < 64; ++i) sc[i] = __uint_as_float(raw[i >> 5][i & 31]);
+      const int valid = min(128, P.S - j * 128) - 64 * hf;   // valid columns of this half
+      if (valid < 64) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
+        for (int i = 0; i < 64; ++i)
           if (i >= valid) sc[i] = -INFINITY;
       }
-      // tile max of the raw scores (c > 0, so max(c t) = c max(t))
-      float m0 = sc[0], m1 = sc[1], m2 = sc[2], m3 = sc[3];
+      // partial max of this half's raw scores, then the full row max
+      float m0 = sc[0], m1 = sc[1];
 #pragma unroll
-      for (int i = 4; i < 124; i += 8) {
+      for (int i = 2; i < 62; i += 4) {
         m0 = fmax3(m0, sc[i + 0], sc[i + 1]);
         m1 = fmax3(m1, sc[i + 2], sc[i + 3]);
-        m2 = fmax3(m2, sc[i + 4], sc[i + 5]);
-        m3 = fmax3(m3, sc[i + 6], sc[i + 7]);
       }
-      m0 = fmax3(m0, sc[124], sc[125]);
-      m1 = fmax3(m1, sc[126], sc[127]);
-      const float tmax = fmaxf(fmax3(m0, m1, m2), m3);
-      const float c = __fmul_rn(__fmul_rn(sQ, P.k_scales[(size_t)bh * P.nb + j]), P.kappa);
+      const float mp = fmax3(m0, m1, fmaxf(sc[62], sc[63]));
+      s.xmax[j & 1][t][hf][row] = mp;
+      named_bar_sync(1 + t, 256);
+      const float tmax = fmaxf(mp, s.xmax[j & 1][t][hf ^ 1][row]);
+      // c > 0, so max(c t) = c max(t)
+      const float c = __fmul_rn(__fmul_rn(sQ, sK), P.kappa);
       const float Mtile = ceilf(__fmul_rn(c, tmax));
       const float Fn = j == 0 ? Mtile : fmaxf(F, Mtile);
       const bool resc = j > 0 && Fn > F;
       const float alpha = resc ? exp2_int((int)(F - Fn)) : 1.0f;
       const float bias = expcast_bias(P.bias_b, Fn);
       const float c8 = 8.0f * c;
-      const bool hot = __all_sync(0xffffffffu, fabsf(Fn) < 524288.0f);
-      // ExpCast: one fma per score on the magic-biased fp32; the low byte is the code
+      // The single-fma form below needs the frame's bias to be exact and the codes
+      // to stay in the fp32 binade [2^23, 2^24): |F| < 2^19 (log2-domain scores
+      // below 524288). Larger scores are reported, not computed.
+      range_ok &= fabsf(Fn) < 524288.0f;
+      // ExpCast: one fma per score on the magic-biased fp32; the low byte is the
+      // code; the clamp at the magic value is code 0 (masked tail scores are -inf)
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t w[8];
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
           const int i = cc * 32 + q4 * 4;
-          float z[4];
-          if (hot) {
-            const float2 a = ffma2(make_float2(sc[i], sc[i + 1]), make_float2(c8, c8), make_float2(bias, bias));
-            const float2 b = ffma2(make_float2(sc[i + 2], sc[i + 3]), make_float2(c8, c8), make_float2(bias, bias));
-            z[0] = fmaxf(a.x, kMagic);
-            z[1] = fmaxf(a.y, kMagic);
-            z[2] = fmaxf(b.x, kMagic);
-            z[3] = fmaxf(b.y, kMagic);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) z[e] = __uint_as_float(0x4B400000u + expcast_code(sc[i + e], c8, bias));
-          }
-          if (valid < 128) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (i + e >= valid) z[e] = kMagic;
-          }
-          w[q4] = pack_codes4(z[0], z[1], z[2], z[3]);
+          const float2 a = ffma2(make_float2(sc[i], sc[i + 1]), make_float2(c8, c8), make_float2(bias, bias));
+          const float2 b = ffma2(make_float2(sc[i + 2], sc[i + 3]), make_float2(c8, c8), make_float2(bias, bias));
+          w[q4] = pack_codes4(fmaxf(a.x, kMagic), fmaxf(a.y, kMagic), fmaxf(b.x, kMagic), fmaxf(b.y, kMagic));
         }
-        const int c0 = (2 * cc) ^ (row & 7), c1 = (2 * cc + 1) ^ (row & 7);
-        *reinterpret_cast<uint4*>(prow + c0 * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(prow + c1 * 16) = make_uint4(w[4], w[5], w[6], w[7]);
+        const int k0 = 4 * hf + 2 * cc;
+        *reinterpret_cast<uint4*>(prow + ((k0 ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(prow + (((k0 + 1) ^ (row & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
       }
       fence_proxy_async_smem();
       if (__any_sync(0xffffffffu, resc)) {
         // the frame moved: O_t (complete up to block j-1), l and the row sums not
         // yet handed to a mean MMA are rescaled by the exact 2^(F_old - F_new)
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t r[32];
           tmem_ld32(o_addr + 32 * cc, r);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
           tmem_st32(o_addr + 32 * cc, r);
+          tmem_st_wait();  // the store reads r asynchronously: done before r is reused
         }
-        tmem_st_wait();
-        if (resc) {
+        if (resc && hf == 1) {
           const int jp = j - 1, ch = (jp / kMeanBlocks) % kMeanChunks;
           const int nslots = 3 * (jp % kMeanBlocks) + 3;
           for (int sl = 0; sl < nslots; ++sl) {
@@ -359,7 +358,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       F = Fn;
       tc_fence_before();
       mbar_arrive(&s.p_full[t]);
-      // row sum of this block's cast P (tensor core), then the mean-MMA operands
+      // row sum of this block's cast P (tensor core), then the mean-MMA operands:
+      // the upper half writes the row sums of its rows, the lower half the block
+      // mean / s_V of channel `row`
       if (!(ok = wait_or_abort(s, &s.o_done[t], j & 1, P))) break;
       tc_fence_after();
       const float r = __uint_as_float(tmem_ld1(s_addr));
@@ -368,43 +369,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&s.r_free[t]);
       l = __fadd_rn(l, r);
       const int g = j % kMeanBlocks, ch = (j / kMeanBlocks) % kMeanChunks;
-      __nv_bfloat16 rh, rl;
-      split_bf16(r, rh, rl);
-      st_bf16(mo, sw128_off16(row, ch, 3 * g + 0), rh);
-      st_bf16(mo, sw128_off16(row, ch, 3 * g + 1), rh);
-      st_bf16(mo, sw128_off16(row, ch, 3 * g + 2), rl);
-      // thread `row` also writes channel `row` of this block's mean / s_V
-      const int vs = j % kVStages;
-      if (!(ok = wait_or_abort(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
-      const float m = __fmul_rn(s.mu[vs][row], inv_sV);
-      mbar_arrive(&s.mu_empty[vs]);
-      __nv_bfloat16 mh, ml;
-      split_bf16(m, mh, ml);
-      st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 0), mh);
-      st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 1), ml);
-      st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 2), mh);
       const bool last = j == nkv - 1;
-      if (last)
-        for (int sl = 3 * g + 3; sl < 16; ++sl) {
-          st_bf16(mo, sw128_off16(row, ch, sl), __float2bfloat16_rn(0.0f));
-          st_bf16(mo, sw128_off16(row, kMeanChunks + ch, sl), __float2bfloat16_rn(0.0f));
-        }
+      if (hf == 1) {
+        __nv_bfloat16 rh, rl;
+        split_bf16(r, rh, rl);
+        st_bf16(mo, sw128_off16(row, ch, 3 * g + 0), rh);
+        st_bf16(mo, sw128_off16(row, ch, 3 * g + 1), rh);
+        st_bf16(mo, sw128_off16(row, ch, 3 * g + 2), rl);
+        if (last)
+          for (int sl = 3 * g + 3; sl < 16; ++sl) st_bf16(mo, sw128_off16(row, ch, sl), __float2bfloat16_rn(0.0f));
+      } else {
+        const int vs = j % kVStages;
+        if (!(ok = wait_or_abort(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
+        const float m = __fmul_rn(s.mu[vs][row], inv_sV);
+        mbar_arrive(&s.mu_empty[vs]);
+        __nv_bfloat16 mh, ml;
+        split_bf16(m, mh, ml);
+        st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 0), mh);
+        st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 1), ml);
+        st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 2), mh);
+        if (last)
+          for (int sl = 3 * g + 3; sl < 16; ++sl)
+            st_bf16(mo, sw128_off16(row, kMeanChunks + ch, sl), __float2bfloat16_rn(0.0f));
+      }
       if (g == kMeanBlocks - 1 || last) fence_proxy_async_smem();
     }
+    if (!range_ok) report_status(P.status, VC_ERR_UNSUPPORTED);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       mbar_arrive(&s.fin_ready[t]);
       ok = __all_sync(0xffffffffu, wait_or_abort(s, &s.o_final[t], 0, P));
     }
     if (ok) {
-      // epilogue: O = s_V O_t / l, BF16, original query order and layout
+      // epilogue: O = s_V O_t / l, BF16, original query order and layout; this
+      // thread writes channels 64 hf .. 64 hf + 63 of its row
       tc_fence_after();
       const int q = qt * 128 + row;
       const float scale = __fdiv_rn(sV, l);
       const int b = bh / P.H, h = bh % P.H;
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(P.o) + (((size_t)b * P.S + q) * P.H + h) * 128;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(P.o) + (((size_t)b * P.S + q) * P.H + h) * 128 + 64 * hf;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t r[32];
         tmem_ld32(o_addr + 32 * cc, r);
         tmem_ld_wait();
