@@ -21,9 +21,10 @@
 //   warp  17    MMA issuer (one thread)
 // Tensor memory (512 columns): S_t = [128t, 128t+128), O_t = [256+128t, ...).
 // Per block j and tile t the tensor core runs, in this order per tile:
-//   QK   S_t  = Q_t K_j^T                 kind::f8f6f4, M=128 N=128 K=128
 //   PV   O_t += P_t V_j                   P_t = ExpCast codes (smem), V_j = residual codes
-//   ROW  S_t[:, 0:16) = P_t 1             exact row sums r of the cast P
+//   ROW  S_t[:, 112:128) = P_t 1          exact row sums r of the cast P
+//   QK   S_t  = Q_t K_{j+1}^T             kind::f8f6f4, M=128 K=128, as keys 0-111 (N=112)
+//        and keys 112-127 (N=16); the second part waits until r has been read
 //   MEAN after every 5 blocks:  O_t += R_t M    kind::f16 with bf16 operands:
 //        R_t = the blocks' row sums, M = their block means / s_V, each split into
 //        bf16 hi/lo parts (r_hi m_hi + r_hi m_lo + r_lo m_hi, three K slots a block);
@@ -56,6 +57,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kMeanBlocks = 5;              // key blocks per mean MMA (3 K slots each: 15 of 16)
 constexpr int kMeanChunks = 2;              // 16-slot K chunks per operand (R: 0-1, M: 2-3)
 constexpr uint32_t kOneE4M3x4 = 0x38383838u;
+constexpr uint32_t kRowCol = 112;            // score columns 112-127 also receive the row sums
+constexpr uint64_t kKeyHiOff = (112 * 128) >> 4;  // descriptor offset of K rows 112.. (14 atoms)
 
 struct __align__(1024) SmemAttn {
   uint8_t q[2][kTileBytes];
@@ -189,7 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_qk = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
-      constexpr uint32_t id_row = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 16);
+      constexpr uint32_t id_row = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 16);     // also QK_hi
+      constexpr uint32_t id_qk_lo = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, kRowCol);
       constexpr uint32_t id_mean = idesc_f32acc(kFmtBF16, kFmtBF16, 128, 128);
       const uint64_t dq[2] = {sdesc_k_sw128(smem_u32(s.q[0])), sdesc_k_sw128(smem_u32(s.q[1]))};
       const uint64_t dp[2] = {sdesc_k_sw128(smem_u32(s.p[0])), sdesc_k_sw128(smem_u32(s.p[1]))};
@@ -206,9 +210,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(&s.k_empty[0]);
       }
+      // Per block j, tile by tile: [mean batch], PV_t(j), ROW_t(j) as soon as P_t(j)
+      // is ready, then at once the scores of keys 0-111 of block j+1 (QK_lo); the
+      // last 16 keys (QK_hi) overwrite the row-sum columns 112-127, so they wait
+      // until the softmax group has read its row sums, which overlaps QK_lo.
       for (int j = 0; ok && j < nkv; ++j) {
         const int vs = j % kVStages;
+        const int ks = (j + 1) % kKStages;
         const uint64_t dv = sdesc_k_sw128(smem_u32(s.v[vs]));
+        const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[ks]));
         for (int t = 0; t < 2 && ok; ++t) {
           if (!(ok = wait_or_abort(s, &s.p_full[t], j & 1, P))) break;
           if (t == 0 && !(ok = wait_or_abort(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
@@ -222,24 +232,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < 4; ++kk)
             umma_f8f6f4_ss(dO, dp[t] + 2 * kk, dv + 2 * kk, id_qk, (j > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(tmem + 128 * t, dp[t] + 2 * kk, dones + 2 * kk, id_row, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f8f6f4_ss(tmem + 128 * t + kRowCol, dp[t] + 2 * kk, dones + 2 * kk, id_row, kk > 0);
           umma_commit(&s.o_done[t]);
-        }
-        if (!ok) break;
-        umma_commit(&s.v_empty[vs]);
-        if (j + 1 < nkv) {
-          const int ks = (j + 1) % kKStages;
-          if (!(ok = wait_or_abort(s, &s.k_full[ks], ((j + 1) / kKStages) & 1, P))) break;
-          const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[ks]));
-          for (int t = 0; t < 2 && ok; ++t) {
+          if (t == 1) umma_commit(&s.v_empty[vs]);
+          if (j + 1 < nkv) {
+            if (t == 0 && !(ok = wait_or_abort(s, &s.k_full[ks], ((j + 1) / kKStages) & 1, P))) break;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f8f6f4_ss(tmem + 128 * t, dq[t] + 2 * kk, dk + 2 * kk, id_qk_lo, kk > 0);
             if (!(ok = wait_or_abort(s, &s.r_free[t], j & 1, P))) break;
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(tmem + 128 * t, dq[t] + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f8f6f4_ss(tmem + 128 * t + kRowCol, dq[t] + 2 * kk, dk + kKeyHiOff + 2 * kk, id_row, kk > 0);
             umma_commit(&s.s_full[t]);
+            if (t == 1) umma_commit(&s.k_empty[ks]);
           }
-          if (!ok) break;
-          umma_commit(&s.k_empty[ks]);
         }
       }
       // the last (possibly partial) batch of block means, then the output is final
@@ -363,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // mean / s_V of channel `row`
       if (!(ok = wait_or_abort(s, &s.o_done[t], j & 1, P))) break;
       tc_fence_after();
-      const float r = __uint_as_float(tmem_ld1(s_addr));
+      const float r = __uint_as_float(tmem_ld1(s_addr + kRowCol));
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&s.r_free[t]);

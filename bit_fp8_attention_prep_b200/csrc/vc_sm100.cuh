@@ -45,17 +45,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete yet may be
+// suspended by the hardware for up to `hint_ns` nanoseconds (it is woken as soon
+// as the phase completes), instead of spinning and taking issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete. Returns false
 // once `limit_ns` of wall time (globaltimer) has passed, or as soon as another
-// CTA has reported an error in *abort_flag (when non-null); never spins forever.
+// CTA has reported an error in *abort_flag (when non-null); never waits forever.
+// While it waits the thread sleeps in the barrier unit (at most 50 us at a time),
+// so waiting warps do not compete with working ones for issue slots.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                           const volatile int32_t* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 256; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 50000u)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
     if (abort_flag && *abort_flag != VC_OK) return false;
   }
