@@ -279,13 +279,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* const mo = s.mop[t];
     uint8_t* const prow = s.p[t] + row * 128;
     float F = 0.0f, l = 0.0f;
-    bool ok = true, range_ok = true;
+    bool ok = true, range_ok = true, fail = false;
     const float* const ksc = P.k_scales + (size_t)bh * P.nb;
     float sK_next = ksc[0];
     for (int j = 0; j < nkv; ++j) {
       const float sK = sK_next;                      // this block's K scale, loaded one block ahead
       if (j + 1 < nkv) sK_next = ksc[j + 1];
-      if (!(ok = wait_or_abort(s, &s.s_full[t], j & 1, P))) break;
+      // A failed (timed-out) wait never breaks the loop on its own: the group
+      // leaves together at the next row-max exchange, whose barrier ORs the
+      // failures, so no thread is left waiting in that barrier.
+      fail |= !wait_or_abort(s, &s.s_full[t], j & 1, P);
       tc_fence_after();
       uint32_t raw[2][32];
       tmem_ld32(s_addr + 64 * hf, raw[0]);
@@ -309,7 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float mp = fmax3(m0, m1, fmaxf(sc[62], sc[63]));
       s.xmax[j & 1][t][hf][row] = mp;
-      named_bar_sync(1 + t, 256);
+      if (named_bar_any(1 + t, 256, fail)) {
+        ok = false;
+        break;
+      }
       const float tmax = fmaxf(mp, s.xmax[j & 1][t][hf ^ 1][row]);
       // c > 0, so max(c t) = c max(t)
       const float c = __fmul_rn(__fmul_rn(sQ, sK), P.kappa);
@@ -370,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // row sum of this block's cast P (tensor core), then the mean-MMA operands:
       // the upper half writes the row sums of its rows, the lower half the block
       // mean / s_V of channel `row`
-      if (!(ok = wait_or_abort(s, &s.o_done[t], j & 1, P))) break;
+      fail |= !wait_or_abort(s, &s.o_done[t], j & 1, P);
       tc_fence_after();
       const float r = __uint_as_float(tmem_ld1(s_addr + kRowCol));
       tmem_ld_wait();
@@ -389,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int sl = 3 * g + 3; sl < 16; ++sl) st_bf16(mo, sw128_off16(row, ch, sl), __float2bfloat16_rn(0.0f));
       } else {
         const int vs = j % kVStages;
-        if (!(ok = wait_or_abort(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
+        fail |= !wait_or_abort(s, &s.v_full[vs], (j / kVStages) & 1, P);
         const float m = __fmul_rn(s.mu[vs][row], inv_sV);
         mbar_arrive(&s.mu_empty[vs]);
         __nv_bfloat16 mh, ml;
@@ -404,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (g == kMeanBlocks - 1 || last) fence_proxy_async_smem();
     }
     if (!range_ok) report_status(P.status, VC_ERR_UNSUPPORTED);
-    ok = __all_sync(0xffffffffu, ok);
+    ok = __all_sync(0xffffffffu, ok && !fail);
     if (ok) {
       mbar_arrive(&s.fin_ready[t]);
       ok = __all_sync(0xffffffffu, wait_or_abort(s, &s.o_final[t], 0, P));
