@@ -33,6 +33,10 @@ METRIC = "VC-attn FP8 TFLOP/s and % of FP8 peak at S=73397,D=128; rel-L2 vs FP64
 UNIT = "TFLOP/s"
 DEFAULT_WORKLOAD = "minimax_h56"
 ATTN_SRC = os.path.join(ROOT, "bit_fp8_attention_prep_b200", "csrc", "vc_attn_fwd.cu")
+# the kernel the roofline line describes: one E4M3 V plane, or the two exact
+# E4M3 planes of an NVFP4 residual (the forward stage then also runs the
+# plane split, nvfp4_planes_kernel)
+ATTN_KERNEL = {"e4m3": "vc_attn_fwd_kernel<1>", "nvfp4": "vc_attn_fwd_kernel<2>"}
 # DRAM bytes (read + write) of one attention launch on the default workload, from
 # the ncu capture summarised in profiles/; valid only while the kernel source
 # hashes to the recorded value (otherwise traffic is reported as null).
@@ -284,7 +288,7 @@ def run_ours(args, cfg):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
         "config": config_of(cfg, argparse.Namespace(k_p=args.k_p, gpus=world)),
-        "roofline": {"bound": "tensor", "kernel": "vc_attn_fwd_e4m3_kernel", "achieved": attn_tflops,
+        "roofline": {"bound": "tensor", "kernel": ATTN_KERNEL[cfg["fmt"]], "achieved": attn_tflops,
                      "peak": fp8_peak, "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak, "traffic": traffic,
                      "peak_source": f"2 x {peaks['source']} sustained bf16 cuBLAS ({peaks['bf16_sustained']:.1f})"},
         "stages_ms": {"prepare_v": prep_ms, "quant_qk": qk_ms, "forward": fwd_ms},

@@ -233,22 +233,30 @@ vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* sha
 
 static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                                   float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream,
-                                  bool nvfp4) {
+                                  bool nvfp4, void* workspace, size_t workspace_bytes) {
   g_last_error.clear();
   vc_status_t st;
   if ((st = check_shape(shape)) != VC_OK) return st;
   if (!qk || !pv || !o) return fail(VC_ERR_INVALID_ARG, "qk, pv and o must be non-NULL");
   if (!qk->q_codes || !qk->q_scales || !qk->k_codes || !qk->k_scales || !pv->mu || !pv->v_codes || !pv->s_v)
     return fail(VC_ERR_INVALID_ARG, "a required field of qk or pv is NULL");
-  if (nvfp4 && !pv->v_scales) return fail(VC_ERR_INVALID_ARG, "pv->v_scales must be non-NULL for NVFP4");
+  if (nvfp4 && (!pv->v_scales || !aligned16(pv->v_scales)))
+    return fail(VC_ERR_INVALID_ARG, "pv->v_scales must be non-NULL and 16-byte aligned for NVFP4");
   if (!aligned16(o) || !aligned16(qk->q_codes) || !aligned16(qk->k_codes) || !aligned16(pv->v_codes) ||
       !aligned16(pv->mu) || (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)))
     return fail(VC_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
   if (!(softmax_scale > 0.0f) || !(softmax_scale < 1e30f))
     return fail(VC_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
   if (k_p < 0 || k_p > 8) return fail(VC_ERR_INVALID_ARG, "k_p must be in [0, 8] (got %d)", k_p);
-  if ((st = ensure_device()) != VC_OK) return st;
   const int nb = nblocks(shape->S), S_pad = nb * 128, BH = shape->B * shape->H;
+  if (nvfp4) {
+    const size_t need = (size_t)2 * BH * 128 * S_pad;
+    if (!workspace || workspace_bytes < need)
+      return fail(VC_ERR_WORKSPACE, "NVFP4-V attention needs %zu bytes of workspace (got %zu)", need,
+                  workspace ? workspace_bytes : (size_t)0);
+    if (!aligned16(workspace)) return fail(VC_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  }
+  if ((st = ensure_device()) != VC_OK) return st;
   CUtensorMap tq, tk, tv;
   if ((st = make_map_u8(&tq, qk->q_codes, 128, (uint64_t)BH * S_pad)) != VC_OK) return st;
   if ((st = make_map_u8(&tk, qk->k_codes, 128, (uint64_t)BH * S_pad)) != VC_OK) return st;
@@ -264,6 +272,7 @@ static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* 
   p.s_v = pv->s_v;
   p.v_scales = pv->v_scales;
   p.kappa = (float)((double)softmax_scale * 1.4426950408889634);
+  p.v_mul = nvfp4 ? 8.0f : 1.0f;
   p.bias_b = 56 + 8 * k_p;
   p.o = o;
   p.status = dev_status;
@@ -273,8 +282,13 @@ static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* 
     if ((st = make_map_u8(&tv, pv->v_codes, (uint64_t)S_pad, (uint64_t)BH * 128)) != VC_OK) return st;
     e = vc::launch_attn_e4m3(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
   } else {
-    e = vc::launch_attn_nvfp4(tq, tk, pv->v_codes, p, static_cast<cudaStream_t>(stream));
-    if (e == cudaErrorNotSupported) return fail(VC_ERR_UNSUPPORTED, "NVFP4-V attention is not built yet");
+    uint8_t* planes = static_cast<uint8_t*>(workspace);
+    e = vc::launch_nvfp4_planes(static_cast<const uint8_t*>(pv->v_codes), static_cast<const uint8_t*>(pv->v_scales),
+                                BH, S_pad, planes, static_cast<cudaStream_t>(stream));
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "launching the NVFP4 plane split");
+    if ((st = make_map_u8(&tv, planes, (uint64_t)S_pad, (uint64_t)2 * BH * 128)) != VC_OK) return st;
+    e = vc::launch_attn_planes(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
   }
   g_launches += 1;
   if (e != cudaSuccess) return cuda_fail(e, "launching attention");
@@ -283,12 +297,19 @@ static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* 
 
 vc_status_t vc_attn_forward(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                             float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
-  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, false);
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, false, nullptr, 0);
+}
+
+size_t vc_attn_forward_nvfp4v_workspace_bytes(const vc_shape_t* shape) {
+  if (check_shape(shape) != VC_OK) return 0;
+  return (size_t)2 * shape->B * shape->H * 128 * (size_t)(nblocks(shape->S) * 128);
 }
 
 vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
-                                   float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
-  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, true);
+                                   float softmax_scale, int32_t k_p, void* o, void* workspace,
+                                   size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, true, workspace,
+                        workspace_bytes);
 }
 
 // ------------------------------------------------------------ fixed-scratch prep

@@ -48,8 +48,12 @@
 namespace vc {
 namespace {
 
-constexpr int kKStages = 3;
-constexpr int kVStages = 3;
+// kPlanes = 1: the E4M3 residual; kPlanes = 2: the NVFP4 residual given as two
+// exact E4M3 planes (hi + lo) by the pre-pass in vc_prep.cu, with PV run over both.
+template <int kPlanes> struct Stages {
+  static constexpr int K = 3;
+  static constexpr int V = kPlanes == 1 ? 3 : 2;
+};
 constexpr uint32_t kTileBytes = 128 * 128;  // one 128 x 128 E4M3 tile (or 128 x 64 bf16)
 constexpr int kThreads = 576;
 constexpr int kTmaWarp = 16, kMmaWarp = 17;
@@ -60,10 +64,12 @@ constexpr uint32_t kOneE4M3x4 = 0x38383838u;
 constexpr uint32_t kRowCol = 112;            // score columns 112-127 also receive the row sums
 constexpr uint64_t kKeyHiOff = (112 * 128) >> 4;  // descriptor offset of K rows 112.. (14 atoms)
 
+template <int kPlanes>
 struct __align__(1024) SmemAttn {
+  static constexpr int kKStages = Stages<kPlanes>::K, kVStages = Stages<kPlanes>::V;
   uint8_t q[2][kTileBytes];
   uint8_t k[kKStages][kTileBytes];
-  uint8_t v[kVStages][kTileBytes];
+  uint8_t v[kVStages][kPlanes][kTileBytes];
   uint8_t p[2][kTileBytes];
   uint8_t mop[2][kTileBytes];    // bf16 operands of the mean MMA, one tile per query tile
   uint8_t ones[2048];            // E4M3 1.0: B operand of the row-sum MMA (N=16, K=128)
@@ -82,7 +88,8 @@ __device__ __forceinline__ float exp2_int(int n) {  // 2^n for integer n <= 0, e
   return n < -126 ? 0.0f : __int_as_float((127 + n) << 23);
 }
 
-__device__ __forceinline__ bool wait_or_abort(SmemAttn& s, uint64_t* bar, uint32_t parity, const AttnParams& P) {
+template <class Smem>
+__device__ __forceinline__ bool wait_or_abort(Smem& s, uint64_t* bar, uint32_t parity, const AttnParams& P) {
   if (mbar_wait(bar, parity, P.wait_ns, P.status)) return true;
   s.abort_flag = 1;
   report_status(P.status, VC_ERR_TIMEOUT);
@@ -106,11 +113,14 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bflo
   lo = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
 }
 
+template <int kPlanes>
 __global__ void __launch_bounds__(kThreads, 1)
-    vc_attn_fwd_e4m3_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                            const __grid_constant__ CUtensorMap tmV, const AttnParams P) {
+    vc_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const AttnParams P) {
+  using Smem = SmemAttn<kPlanes>;
+  constexpr int kKStages = Smem::kKStages, kVStages = Smem::kVStages;
   extern __shared__ uint8_t smem_raw[];
-  SmemAttn& s = *reinterpret_cast<SmemAttn*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y;
   const int nkv = P.nb;
@@ -175,8 +185,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = ((j / kVStages) & 1) ^ 1;
         if (!wait_or_abort(s, &s.v_empty[vs], ph, P)) break;
         if (!wait_or_abort(s, &s.mu_empty[vs], ph, P)) break;
-        mbar_arrive_expect_tx(&s.v_full[vs], kTileBytes + 512);
-        tma_load_2d(s.v[vs], &tmV, &s.v_full[vs], j * 128, bh * 128);
+        mbar_arrive_expect_tx(&s.v_full[vs], kPlanes * kTileBytes + 512);
+#pragma unroll
+        for (int pl = 0; pl < kPlanes; ++pl)  // plane pl of head bh: rows (pl * BH + bh) * 128
+          tma_load_2d(s.v[vs][pl], &tmV, &s.v_full[vs], j * 128, (pl * P.B * P.H + bh) * 128);
         bulk_load(s.mu[vs], P.mu + ((size_t)bh * P.nb + j) * 128, 512, &s.v_full[vs]);
         v_issued = j + 1;
       }
@@ -217,7 +229,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < nkv; ++j) {
         const int vs = j % kVStages;
         const int ks = (j + 1) % kKStages;
-        const uint64_t dv = sdesc_k_sw128(smem_u32(s.v[vs]));
         const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[ks]));
         for (int t = 0; t < 2 && ok; ++t) {
           if (!(ok = wait_or_abort(s, &s.p_full[t], j & 1, P))) break;
@@ -229,8 +240,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_f16_ss(dO, dm[t] + 2 * ch, dm[t] + 2 * (kMeanChunks + ch), id_mean, 1u);
           }
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_f8f6f4_ss(dO, dp[t] + 2 * kk, dv + 2 * kk, id_qk, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int pl = 0; pl < kPlanes; ++pl) {  // O_t += P_t V_hi (+ P_t V_lo)
+            const uint64_t dv = sdesc_k_sw128(smem_u32(s.v[vs][pl]));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f8f6f4_ss(dO, dp[t] + 2 * kk, dv + 2 * kk, id_qk, (j > 0 || pl > 0 || kk > 0) ? 1u : 0u);
+          }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_f8f6f4_ss(tmem + 128 * t + kRowCol, dp[t] + 2 * kk, dones + 2 * kk, id_row, kk > 0);
@@ -274,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qt = pair * 2 + t;
     const bool q_valid = qt < P.nb;
     const float sQ = q_valid ? P.q_scales[(size_t)bh * P.nb + qt] : 1.0f;
-    const float sV = P.s_v[bh];
+    const float sV = __fmul_rn(P.s_v[bh], P.v_mul);   // value scale of the residual codes
     const float inv_sV = __fdiv_rn(1.0f, sV);
     uint8_t* const mo = s.mop[t];
     uint8_t* const prow = s.p[t] + row * 128;
@@ -454,20 +469,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t attn_configure() {
-  return cudaFuncSetAttribute(vc_attn_fwd_e4m3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)(sizeof(SmemAttn) + 1024));
+  cudaError_t e = cudaFuncSetAttribute(vc_attn_fwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)(sizeof(SmemAttn<1>) + 1024));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(vc_attn_fwd_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)(sizeof(SmemAttn<2>) + 1024));
 }
 
 cudaError_t launch_attn_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const AttnParams& p, cudaStream_t st) {
   const dim3 grid((p.nb + 1) / 2, p.B * p.H);
-  vc_attn_fwd_e4m3_kernel<<<grid, kThreads, sizeof(SmemAttn) + 1024, st>>>(tq, tk, tv, p);
+  vc_attn_fwd_kernel<1><<<grid, kThreads, sizeof(SmemAttn<1>) + 1024, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_nvfp4(const CUtensorMap&, const CUtensorMap&, const uint8_t*, const AttnParams&,
-                              cudaStream_t) {
-  return cudaErrorNotSupported;
+cudaError_t launch_attn_planes(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tplanes,
+                               const AttnParams& p, cudaStream_t st) {
+  const dim3 grid((p.nb + 1) / 2, p.B * p.H);
+  vc_attn_fwd_kernel<2><<<grid, kThreads, sizeof(SmemAttn<2>) + 1024, st>>>(tq, tk, tplanes, p);
+  return cudaGetLastError();
 }
 
 }  // namespace vc

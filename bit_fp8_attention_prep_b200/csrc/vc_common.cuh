@@ -49,6 +49,11 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   return (code & 0x80) ? -v : v;
 }
 
+// E2M1 magnitude code (0..7) -> value {0, 0.5, 1, 1.5, 2, 3, 4, 6} (exact).
+__device__ __forceinline__ float e2m1_value(uint32_t mag) {
+  return mag < 4 ? 0.5f * (float)mag : (float)(2u << ((mag - 4) >> 1)) * ((mag & 1u) ? 1.5f : 1.0f);
+}
+
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 template <> __device__ __forceinline__ float to_f32<__half>(__half x) { return __half2float(x); }

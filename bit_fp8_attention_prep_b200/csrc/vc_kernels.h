@@ -50,6 +50,7 @@ struct AttnParams {
   const float* s_v;        // [BH]
   const uint8_t* v_scales; // NVFP4: [BH][128][S_pad/16]
   float kappa;             // fl32(softmax_scale * log2 e)
+  float v_mul;             // value scale = s_v * v_mul (1 for E4M3; 8 for the NVFP4 planes)
   int bias_b;              // 56 + 8 k_P
   void* o;                 // bf16 [B][S][H][128]
   int32_t* status;         // optional device status word
@@ -59,7 +60,12 @@ struct AttnParams {
 cudaError_t attn_configure();
 cudaError_t launch_attn_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const AttnParams& p, cudaStream_t st);
-cudaError_t launch_attn_nvfp4(const CUtensorMap& tq, const CUtensorMap& tk, const uint8_t* v_codes,
-                              const AttnParams& p, cudaStream_t st);
+// NVFP4 residual: `tplanes` maps the two E4M3 planes written by launch_nvfp4_planes.
+cudaError_t launch_attn_planes(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tplanes,
+                               const AttnParams& p, cudaStream_t st);
+// planes[pl][B*H][128][S_pad] (pl = 0 hi, 1 lo) with hi + lo = e2m1 * dec(scale16) / 8 exactly
+// (down to the E4M3 subnormal grid); padding tokens 0.
+cudaError_t launch_nvfp4_planes(const uint8_t* codes, const uint8_t* scales, int BH, int S_pad,
+                                uint8_t* planes, cudaStream_t st);
 
 }  // namespace vc

@@ -474,6 +474,67 @@ __global__ void __launch_bounds__(128) quant_qk_kernel(const T* __restrict__ q, 
   }
 }
 
+// --------------------------------------------------------------- NVFP4 -> two E4M3 planes
+// The attention kernel multiplies E4M3 probabilities with E4M3 operands only.
+// An NVFP4 residual value e2m1 * dec(s16) (times the global g) has at most 6
+// significant bits, so v = e2m1 * dec(s16) / 8 (at most 336) splits exactly into
+// hi = E4M3(v) and lo = E4M3(v - hi); the product P (hi + lo) is then P v exactly
+// wherever lo lies on the E4M3 grid (|v| >= 2^-4, i.e. down to 1/5376 of the
+// head's largest value; below that lo rounds to the 2^-9 subnormal grid).
+// One CTA = one 128-token block of one (b, h); thread d owns channel d.
+__global__ void __launch_bounds__(128) nvfp4_planes_kernel(const uint8_t* __restrict__ codes,
+                                                           const uint8_t* __restrict__ scales, int S_pad,
+                                                           size_t plane_stride, uint8_t* __restrict__ planes) {
+  const int bh = blockIdx.y, blk = blockIdx.x, d = threadIdx.x;
+  const size_t row = (size_t)bh * kD + d;
+  const uint8_t* crow = codes + row * (S_pad / 2) + (size_t)blk * (kBlock / 2);
+  const uint2 sc2 = *reinterpret_cast<const uint2*>(scales + row * (S_pad / kGroup4) + (size_t)blk * (kBlock / kGroup4));
+  uint8_t* hi = planes + row * S_pad + (size_t)blk * kBlock;
+  uint8_t* lo = hi + plane_stride;
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {  // 32 tokens (16 code bytes) at a time
+    const uint4 cw = *reinterpret_cast<const uint4*>(crow + c * 16);
+    const uint8_t* cb = reinterpret_cast<const uint8_t*>(&cw);
+    // the two scale bytes of these 32 tokens (scale byte 2c and 2c+1 of the block)
+    const uint32_t sw = ((c < 2) ? sc2.x : sc2.y) >> (16 * (c & 1));
+    const float sc_lo = e4m3_to_f32(sw & 0xFFu), sc_hi = e4m3_to_f32((sw >> 8) & 0xFFu);
+    uint32_t wh[8], wl[8];
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      float v[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const uint32_t nib = (cb[(i + e) >> 1] >> (4 * ((i + e) & 1))) & 0xFu;
+        const float mag = e2m1_value(nib & 7u);
+        v[e] = __fmul_rn(__fmul_rn((nib & 8u) ? -mag : mag, (i + e) < kGroup4 ? sc_lo : sc_hi), 0.125f);
+      }
+      const uint16_t h2 = cvt_e4m3x2(v[0], v[1]);
+      const uint16_t l2 = cvt_e4m3x2(__fsub_rn(v[0], e4m3_to_f32(h2 & 0xFF)), __fsub_rn(v[1], e4m3_to_f32(h2 >> 8)));
+      const int k = i >> 1;  // byte pair index 0..15
+      if ((k & 1) == 0) {
+        wh[k >> 1] = h2;
+        wl[k >> 1] = l2;
+      } else {
+        wh[k >> 1] |= (uint32_t)h2 << 16;
+        wl[k >> 1] |= (uint32_t)l2 << 16;
+      }
+    }
+    uint4* oh = reinterpret_cast<uint4*>(hi + c * 32);
+    uint4* ol = reinterpret_cast<uint4*>(lo + c * 32);
+    oh[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    oh[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+    ol[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+    ol[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
+  }
+}
+
+cudaError_t launch_nvfp4_planes(const uint8_t* codes, const uint8_t* scales, int BH, int S_pad, uint8_t* planes,
+                                cudaStream_t st) {
+  const dim3 grid(S_pad / kBlock, BH);
+  nvfp4_planes_kernel<<<grid, 128, 0, st>>>(codes, scales, S_pad, (size_t)BH * kD * S_pad, planes);
+  return cudaGetLastError();
+}
+
 // --------------------------------------------------------------- launchers
 template <typename T>
 static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_prepared_v_t& out,

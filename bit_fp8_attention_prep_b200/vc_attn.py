@@ -25,7 +25,8 @@ VC_MODE_VSMOOTH, VC_MODE_MEANONLY = 0, 1
 ABI_SYMBOLS = [
     "vc_attn_version", "vc_attn_last_error", "vc_attn_launch_count", "vc_attn_prepare_v_workspace_bytes",
     "vc_attn_prepare_v",
-    "vc_attn_quant_qk", "vc_attn_forward", "vc_attn_forward_nvfp4v", "vc_attn_prepare_v_noalloc",
+    "vc_attn_quant_qk", "vc_attn_forward", "vc_attn_forward_nvfp4v_workspace_bytes", "vc_attn_forward_nvfp4v",
+    "vc_attn_prepare_v_noalloc",
 ]
 NOALLOC_SCRATCH_BYTES = 8 << 20   # VC_ATTN_NOALLOC_SCRATCH_BYTES
 TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
@@ -83,10 +84,13 @@ def load():
     lib.vc_attn_prepare_v_noalloc.argtypes = [vp, P(Shape), P(VSmoothCfg), P(PreparedV), vp, vp]
     lib.vc_attn_quant_qk.restype = i32
     lib.vc_attn_quant_qk.argtypes = [vp, vp, P(Shape), vp, P(QKFP8), vp]
-    for name in ("vc_attn_forward", "vc_attn_forward_nvfp4v"):
-        f = getattr(lib, name)
-        f.restype = i32
-        f.argtypes = [P(QKFP8), P(PreparedV), P(Shape), ctypes.c_float, i32, vp, vp, vp]
+    lib.vc_attn_forward.restype = i32
+    lib.vc_attn_forward.argtypes = [P(QKFP8), P(PreparedV), P(Shape), ctypes.c_float, i32, vp, vp, vp]
+    lib.vc_attn_forward_nvfp4v_workspace_bytes.restype = sz
+    lib.vc_attn_forward_nvfp4v_workspace_bytes.argtypes = [P(Shape)]
+    lib.vc_attn_forward_nvfp4v.restype = i32
+    lib.vc_attn_forward_nvfp4v.argtypes = [P(QKFP8), P(PreparedV), P(Shape), ctypes.c_float, i32, vp, vp, sz,
+                                           vp, vp]
     lib.vc_attn_test_e4m3_round.restype = i32
     lib.vc_attn_test_e4m3_round.argtypes = [vp, vp, i64, vp]
     lib.vc_attn_test_e2m1_round.restype = i32
@@ -218,9 +222,12 @@ def quant_qk(q, k, perm):
     return out
 
 
-def forward(qk, pv, shape, softmax_scale=None, k_p=8, out=None, status=None):
+def forward(qk, pv, shape, softmax_scale=None, k_p=8, out=None, status=None, workspace=None):
     """Fused ExpCast FP8 attention from the two prep outputs; returns BF16 O in
-    the input layout. ``shape`` is the vc_shape_t of Q (``shape_of(q)``)."""
+    the input layout. ``shape`` is the vc_shape_t of Q (``shape_of(q)``).
+    For an NVFP4 ``pv`` the call needs a device workspace of
+    ``forward_nvfp4v_workspace_bytes(shape)`` bytes; one is allocated when
+    ``workspace`` is None."""
     lib = load()
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(128)
@@ -229,10 +236,22 @@ def forward(qk, pv, shape, softmax_scale=None, k_p=8, out=None, status=None):
         out = torch.empty((shape.B, shape.S, shape.H, 128), dtype=torch.bfloat16, device=dev)
     q_ = QKFP8(_ptr(qk["q_codes"]), _ptr(qk["q_scales"]), _ptr(qk["k_codes"]), _ptr(qk["k_scales"]))
     p_ = PreparedV(_ptr(pv["perm"]), _ptr(pv["mu"]), _ptr(pv["v_codes"]), _ptr(pv.get("v_scales")), _ptr(pv["s_v"]))
-    fn = lib.vc_attn_forward_nvfp4v if pv.get("fmt") == "nvfp4" else lib.vc_attn_forward
-    _check(fn(ctypes.byref(q_), ctypes.byref(p_), ctypes.byref(shape), float(softmax_scale), int(k_p), _ptr(out),
-              _ptr(status), _stream()))
+    if pv.get("fmt") == "nvfp4":
+        if workspace is None:
+            workspace = torch.empty(forward_nvfp4v_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+        _check(lib.vc_attn_forward_nvfp4v(ctypes.byref(q_), ctypes.byref(p_), ctypes.byref(shape),
+                                          float(softmax_scale), int(k_p), _ptr(out), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _ptr(status), _stream()))
+    else:
+        _check(lib.vc_attn_forward(ctypes.byref(q_), ctypes.byref(p_), ctypes.byref(shape), float(softmax_scale),
+                                   int(k_p), _ptr(out), _ptr(status), _stream()))
     return out
+
+
+def forward_nvfp4v_workspace_bytes(shape):
+    """Device bytes vc_attn_forward_nvfp4v needs for this shape (the two E4M3
+    planes of the decoded NVFP4 residual)."""
+    return int(load().vc_attn_forward_nvfp4v_workspace_bytes(ctypes.byref(shape)))
 
 
 def attention(q, k, v, softmax_scale=None, k_p=8, kmeans_k=16, iters=4, seed=0, fmt="e4m3"):
@@ -282,7 +301,11 @@ class Plan:
         self.ws_ptr = ctypes.c_void_p(self._ws.data_ptr() + (-self._ws.data_ptr()) % 256)
         self._pv = PreparedV(_ptr(self.perm), _ptr(self.mu), _ptr(self.v_codes), _ptr(self.v_scales), _ptr(self.s_v))
         self._qk = QKFP8(_ptr(self.q_codes), _ptr(self.q_scales), _ptr(self.k_codes), _ptr(self.k_scales))
-        self._fwd = self.lib.vc_attn_forward_nvfp4v if fmt == "nvfp4" else self.lib.vc_attn_forward
+        if fmt == "nvfp4":
+            self.fwd_ws_bytes = self.lib.vc_attn_forward_nvfp4v_workspace_bytes(ctypes.byref(self.shape))
+            self._fwd_ws = e((self.fwd_ws_bytes,), torch.uint8)
+        else:
+            self.fwd_ws_bytes, self._fwd_ws = 0, None
 
     def prepare_v(self, v):
         _check(self.lib.vc_attn_prepare_v(_ptr(v), ctypes.byref(self.shape), ctypes.byref(self.cfg),
@@ -294,8 +317,14 @@ class Plan:
 
     def forward(self, out=None):
         o = self.o if out is None else out
-        _check(self._fwd(ctypes.byref(self._qk), ctypes.byref(self._pv), ctypes.byref(self.shape),
-                         self.softmax_scale, self.k_p, _ptr(o), _ptr(self.status), _stream()))
+        if self.fmt == "nvfp4":
+            _check(self.lib.vc_attn_forward_nvfp4v(ctypes.byref(self._qk), ctypes.byref(self._pv),
+                                                   ctypes.byref(self.shape), self.softmax_scale, self.k_p, _ptr(o),
+                                                   _ptr(self._fwd_ws), self.fwd_ws_bytes, _ptr(self.status),
+                                                   _stream()))
+        else:
+            _check(self.lib.vc_attn_forward(ctypes.byref(self._qk), ctypes.byref(self._pv), ctypes.byref(self.shape),
+                                            self.softmax_scale, self.k_p, _ptr(o), _ptr(self.status), _stream()))
         return o
 
     def run(self, q, k, v, out=None):

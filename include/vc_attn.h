@@ -163,11 +163,30 @@ vc_status_t vc_attn_forward(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, co
                             float softmax_scale, int32_t k_p, void* o, int32_t* dev_status,
                             void* stream);
 
+/* Bytes of device workspace vc_attn_forward_nvfp4v needs: 2*B*H*128*S_pad
+ * (S_pad = S rounded up to 128). 0 for an invalid shape. */
+size_t vc_attn_forward_nvfp4v_workspace_bytes(const vc_shape_t* shape);
+
 /* As vc_attn_forward, for a V residual prepared with VC_RESIDUAL_NVFP4 (pv->v_codes
- * packed E2M1, pv->v_scales E4M3 per 16 tokens, pv->s_v the global scale g). */
+ * packed E2M1, pv->v_scales E4M3 per 16 tokens, pv->s_v the global scale g;
+ * "Hugging Face Introduces VC-Attention", "Technical Breakthroughs and Core
+ * Innovations": NVFP4 storage of the smoothed V).
+ * Each decoded value v = e2m1 * dec(scale16) / 8 is at most 6*448/8 = 336; the
+ * call writes hi = E4M3(v) and lo = E4M3(v - hi) (round to nearest even) to
+ * `workspace` (layout [2][B,H,128,S_pad] uint8), then runs the FP8 attention
+ * over both planes with value scale 8*g. hi + lo equals v exactly for
+ * v >= 1/16 and within 2^-10 below that (E4M3's subnormal step), i.e. an
+ * absolute error of at most g/128 per element before the mean restore.
+ *  workspace        device, >= vc_attn_forward_nvfp4v_workspace_bytes(shape),
+ *                   16-B aligned; caller-owned, contents undefined afterwards;
+ *                   must not be reused by other work until the call's stream
+ *                   has passed it
+ *  other arguments  as vc_attn_forward
+ * Errors: as vc_attn_forward, plus VC_ERR_WORKSPACE (NULL or too small). */
 vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv,
                                    const vc_shape_t* shape, float softmax_scale, int32_t k_p,
-                                   void* o, int32_t* dev_status, void* stream);
+                                   void* o, void* workspace, size_t workspace_bytes,
+                                   int32_t* dev_status, void* stream);
 
 /* Size of the fixed device scratch used by vc_attn_prepare_v_noalloc: 8 MiB. */
 #define VC_ATTN_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)

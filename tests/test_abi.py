@@ -88,3 +88,25 @@ def test_calls_reject_bad_arguments_before_any_launch(lib):
         assert fn(None, None, -1, None) == vc_attn.VC_ERR_INVALID_ARG
         assert fn(None, None, 0, None) == vc_attn.VC_OK
     assert lib.vc_attn_test_bounded_wait(None, 1000, None) == vc_attn.VC_ERR_INVALID_ARG
+
+
+def test_nvfp4_forward_workspace_size_and_checks(lib):
+    sz = lib.vc_attn_forward_nvfp4v_workspace_bytes
+    assert sz(ctypes.byref(_shape(B=1, S=256, H=2))) == 2 * 1 * 2 * 128 * 256
+    assert sz(ctypes.byref(_shape(B=2, S=300, H=3))) == 2 * 2 * 3 * 128 * 384  # S padded to 128
+    assert sz(ctypes.byref(_shape(D=64))) == 0
+    qk = vc_attn.QKFP8(16, 16, 16, 16)
+    pv = vc_attn.PreparedV(16, 16, 16, 16, 16)
+    need = sz(ctypes.byref(_shape()))
+    for ws, nbytes in ((None, need), (ctypes.c_void_p(256), need - 1)):
+        st = lib.vc_attn_forward_nvfp4v(ctypes.byref(qk), ctypes.byref(pv), ctypes.byref(_shape()), 0.088, 8,
+                                        ctypes.c_void_p(16), ws, nbytes, None, None)
+        assert st == vc_attn.VC_ERR_WORKSPACE
+        assert str(need).encode() in lib.vc_attn_last_error()
+    st = lib.vc_attn_forward_nvfp4v(ctypes.byref(qk), ctypes.byref(pv), ctypes.byref(_shape()), 0.088, 8,
+                                    ctypes.c_void_p(16), ctypes.c_void_p(264), need, None, None)
+    assert st == vc_attn.VC_ERR_INVALID_ARG and b"aligned" in lib.vc_attn_last_error()
+    pv_noscale = vc_attn.PreparedV(16, 16, 16, 0, 16)
+    st = lib.vc_attn_forward_nvfp4v(ctypes.byref(qk), ctypes.byref(pv_noscale), ctypes.byref(_shape()), 0.088, 8,
+                                    ctypes.c_void_p(16), ctypes.c_void_p(256), need, None, None)
+    assert st == vc_attn.VC_ERR_INVALID_ARG

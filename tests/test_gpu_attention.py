@@ -58,6 +58,39 @@ def test_attention_mid_sampled_rows(va):
     _check_all_heads(va, cfg, Q, K, V, rows=rows)
 
 
+def test_attention_nvfp4_tiny_all_rows(va):
+    cfg, Q, K, V = make("tiny")
+    _check_all_heads(va, cfg, Q, K, V, fmt="nvfp4")
+
+
+@pytest.mark.parametrize("S", [129, 700, 1000])
+def test_attention_nvfp4_ragged(va, S):
+    cfg, Q, K, V = make("mid", B=1, H=2, S=S)
+    _check_all_heads(va, cfg, Q, K, V, fmt="nvfp4")
+
+
+def test_attention_nvfp4_mid_sampled_rows_kp0(va):
+    cfg, Q, K, V = make("mid")
+    rows = np.sort(np.random.default_rng(1).choice(cfg["S"], 64, replace=False))
+    rows[0], rows[-1] = 0, cfg["S"] - 1
+    _check_all_heads(va, cfg, Q, K, V, rows=rows, fmt="nvfp4")
+    _check_all_heads(va, cfg, Q, K, V, rows=rows, fmt="nvfp4", k_p=0)
+
+
+def test_attention_nvfp4_plan_matches_one_shot_calls(va):
+    # The preallocated Plan (caller-owned plane workspace) gives the same bits as
+    # the one-shot calls (workspace allocated per call).
+    cfg, Q, K, V = make("mid", B=1, H=2, S=777)
+    q, k, v = Q.cuda(), K.cuda(), V.cuda()
+    plan = va.Plan(1, 777, 2, k=cfg["k"], iters=cfg["iters"], fmt="nvfp4")
+    o_plan = plan.run(q, k, v).clone()
+    pv = va.prepare_v(v, k=cfg["k"], iters=cfg["iters"], fmt="nvfp4")
+    o_one = va.forward(va.quant_qk(q, k, pv["perm"]), pv, va.shape_of(q), SCALE, 8)
+    torch.cuda.synchronize()
+    assert int(plan.status.item()) == 0
+    assert torch.equal(o_plan.view(torch.int16), o_one.view(torch.int16))
+
+
 def test_attention_accuracy_vs_exact_and_naive(va):
     # Reported figures: rel-L2 vs FP64 exact attention, and the error reduction of
     # V-Smooth over per-head FP8 V with the same Q/K codes and ExpCast.
