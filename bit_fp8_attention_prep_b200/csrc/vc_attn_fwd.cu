@@ -19,23 +19,31 @@
 //   warps 8-15  softmax group of query tile 1
 //   warp  16    TMA: both Q tiles once; K_j, V^T_j and mu_j into rings
 //   warp  17    MMA issuer (one thread)
-// Tensor memory (512 columns): S_t = [128t, 128t+128), O_t = [256+128t, ...).
-// Per block j and tile t the tensor core runs, in this order per tile:
-//   PV   O_t += P_t V_j                   P_t = ExpCast codes (smem), V_j = residual codes
-//   ROW  S_t[:, 112:128) = P_t 1          exact row sums r of the cast P
-//   QK   S_t  = Q_t K_{j+1}^T             kind::f8f6f4, M=128 K=128, as keys 0-111 (N=112)
-//        and keys 112-127 (N=16); the second part waits until r has been read
-//   MEAN after every 5 blocks:  O_t += R_t M    kind::f16 with bf16 operands:
-//        R_t = the blocks' row sums, M = their block means / s_V, each split into
-//        bf16 hi/lo parts (r_hi m_hi + r_hi m_lo + r_lo m_hi, three K slots a block);
-//        both operands of a tile's mean MMA live in that tile's own 128-B-swizzled
-//        smem tile (R in K chunks 0-1, M in chunks 2-3, alternating by batch), and
-//        the softmax group writes it only while no MMA of its tile is in flight
+// Tensor memory (512 columns):
+//   O_0 [0, 144)    tile 0: output channels 0-127, then 16 row-sum columns
+//   O_1 [144, 288)  tile 1: 16 row-sum columns, then output channels 0-127
+//   S_0 [288, 416)  tile 0 scores; its first 32 columns take the P codes
+//   S_1 [384, 512)  tile 1 scores; P codes in its columns 32-63
+// S_0 and S_1 share 32 columns, so the MMA issuer starts a QK product into one
+// only after the other tile's softmax group has loaded its scores (s_loaded).
+// Per block j and tile t the tensor core runs
+//   PV   O_t += P_t [V_j ; 1]     P_t (E4M3 codes) read from tensor memory,
+//        V_j^T (residual codes) with 16 rows of E4M3 1.0 appended from shared
+//        memory (N = 144): the extra columns accumulate the row sum l of the
+//        cast P exactly as PV sees it
+//   QK   S_t = Q_t K_{j+1}^T     kind::f8f6f4, M = N = K = 128
+//   MEAN after every 5 blocks:  O_t += R_t M     kind::f16 with bf16 operands:
+//        R_t = the blocks' row sums r_b (differences of successive l), M = their
+//        block means / s_V, each split into bf16 hi/lo parts (r_hi m_hi +
+//        r_hi m_lo + r_lo m_hi, three K slots a block), both operands in that
+//        tile's own 128-B-swizzled smem tile (R in K chunks 0-1, M in chunks
+//        2-3, alternating by batch); the softmax group writes it only between
+//        s_full and p_full of a block, when no MMA of its tile is in flight
 // so O_t accumulates the whole output in residual-code units; the epilogue is
 // O = s_V O_t / l. The softmax thread of row i keeps the integer running frame
 // F (ceil of the largest log2-domain score so far); a block is cast in the frame
-// current after it; when F moves, O_t, l and the not-yet-issued row sums are
-// multiplied by the exact power of two 2^(F_old - F_new).
+// current after it; when F moves, O_t (with its row-sum column) and the row sums
+// not yet handed to a mean MMA are multiplied by the exact power 2^(F_old - F_new).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stddef.h>
@@ -55,30 +63,44 @@ template <int kPlanes> struct Stages {
   static constexpr int V = kPlanes == 1 ? 3 : 2;
 };
 constexpr uint32_t kTileBytes = 128 * 128;  // one 128 x 128 E4M3 tile (or 128 x 64 bf16)
+constexpr uint32_t kOnesBytes = 16 * 128;   // 16 rows of E4M3 1.0 (K = 128 keys)
 constexpr int kThreads = 576;
 constexpr int kTmaWarp = 16, kMmaWarp = 17;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMeanBlocks = 5;              // key blocks per mean MMA (3 K slots each: 15 of 16)
 constexpr int kMeanChunks = 2;              // 16-slot K chunks per operand (R: 0-1, M: 2-3)
 constexpr uint32_t kOneE4M3x4 = 0x38383838u;
-constexpr uint32_t kRowCol = 112;            // score columns 112-127 also receive the row sums
-constexpr uint64_t kKeyHiOff = (112 * 128) >> 4;  // descriptor offset of K rows 112.. (14 atoms)
+// tensor-memory columns (see the layout above)
+__device__ __forceinline__ constexpr uint32_t col_o(int t) { return t ? 144u : 0u; }    // PV accumulator, N = 144
+__device__ __forceinline__ constexpr uint32_t col_ch(int t) { return t ? 160u : 0u; }   // output channels 0-127
+__device__ __forceinline__ constexpr uint32_t col_l(int t) { return t ? 144u : 128u; }  // first row-sum column
+__device__ __forceinline__ constexpr uint32_t col_s(int t) { return t ? 384u : 288u; }  // scores
+__device__ __forceinline__ constexpr uint32_t col_p(int t) { return t ? 416u : 288u; }  // P codes, 32 columns
+
+// One V ring stage: [16 rows of 1.0][plane 0: V^T tile][16 rows of 1.0][plane 1].
+// Tile 0's PV reads plane 0 followed by the second band (ones last), tile 1's
+// the first band followed by plane 0 (ones first), so that the row sums land
+// at the ends of the two accumulators given above.
+template <int kPlanes> struct VStage {
+  static constexpr uint32_t kPlane0 = kOnesBytes;
+  static constexpr uint32_t kOnes1 = kOnesBytes + kTileBytes;
+  static constexpr uint32_t kPlane1 = 2 * kOnesBytes + kTileBytes;
+  static constexpr uint32_t kBytes = 2 * kOnesBytes + kPlanes * kTileBytes;
+};
 
 template <int kPlanes>
 struct __align__(1024) SmemAttn {
   static constexpr int kKStages = Stages<kPlanes>::K, kVStages = Stages<kPlanes>::V;
   uint8_t q[2][kTileBytes];
   uint8_t k[kKStages][kTileBytes];
-  uint8_t v[kVStages][kPlanes][kTileBytes];
-  uint8_t p[2][kTileBytes];
+  uint8_t v[kVStages][VStage<kPlanes>::kBytes];
   uint8_t mop[2][kTileBytes];    // bf16 operands of the mean MMA, one tile per query tile
-  uint8_t ones[2048];            // E4M3 1.0: B operand of the row-sum MMA (N=16, K=128)
   float mu[kVStages][128];
   float xmax[2][2][2][128];      // [block parity][query tile][column half][row] partial maxima
   uint64_t q_full;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages], mu_empty[kVStages];
-  uint64_t s_full[2], p_full[2], o_done[2], r_free[2], fin_ready[2], o_final[2];
+  uint64_t s_full[2], s_loaded[2], p_full[2], o_done[2], fin_ready[2], o_final[2];
   uint64_t mma_drain;
   uint32_t tmem_base;
   int32_t abort_flag;
@@ -113,11 +135,32 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bflo
   lo = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
 }
 
+// Writes the three K slots of one block's row sum r (slots hi, hi, lo) into the
+// R chunk of the mean-operand tile.
+__device__ __forceinline__ void put_r(uint8_t* mo, int row, int ch, int g, float r) {
+  __nv_bfloat16 rh, rl;
+  split_bf16(r, rh, rl);
+  st_bf16(mo, sw128_off16(row, ch, 3 * g + 0), rh);
+  st_bf16(mo, sw128_off16(row, ch, 3 * g + 1), rh);
+  st_bf16(mo, sw128_off16(row, ch, 3 * g + 2), rl);
+}
+
+// Four magic-biased codes (low bytes of the fp32 patterns) into one word, a in
+// the lowest byte. b*256 + a keeps a's and b's codes (< 256) in the low 16 bits
+// (the magic's low 12 bits are zero, so nothing carries into them); the
+// multiply-adds run on the fma pipe, one byte permute merges the halves.
+__device__ __forceinline__ uint32_t pack4_imad(float a, float b, float c, float d) {
+  const uint32_t lo = __float_as_uint(b) * 256u + __float_as_uint(a);
+  const uint32_t hi = __float_as_uint(d) * 256u + __float_as_uint(c);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
 template <int kPlanes>
 __global__ void __launch_bounds__(kThreads, 1)
     vc_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnParams P) {
   using Smem = SmemAttn<kPlanes>;
+  using VS = VStage<kPlanes>;
   constexpr int kKStages = Smem::kKStages, kVStages = Smem::kVStages;
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -138,9 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s.s_full[t], 1);
+      mbar_init(&s.s_loaded[t], 1);
       mbar_init(&s.p_full[t], 256);
       mbar_init(&s.o_done[t], 1);
-      mbar_init(&s.r_free[t], 256);
       mbar_init(&s.fin_ready[t], 256);
       mbar_init(&s.o_final[t], 1);
     }
@@ -148,12 +191,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     s.abort_flag = 0;
     fence_barrier_init();
   }
-  // mean-MMA operands start at zero (unused K slots stay zero); the row-sum B
-  // operand is all E4M3 1.0 (every byte 0x38, so the swizzle does not matter)
+  // mean-MMA operands start at zero (unused K slots stay zero); the two bands of
+  // every V stage are all E4M3 1.0 (every byte 0x38, so the swizzle does not
+  // matter); the TMA never writes them
   for (int i = threadIdx.x; i < (int)(2 * kTileBytes / 16); i += kThreads)
     *reinterpret_cast<uint4*>(&s.mop[0][0] + i * 16) = make_uint4(0u, 0u, 0u, 0u);
-  for (int i = threadIdx.x; i < 2048 / 16; i += kThreads)
-    *reinterpret_cast<uint4*>(s.ones + i * 16) = make_uint4(kOneE4M3x4, kOneE4M3x4, kOneE4M3x4, kOneE4M3x4);
+  for (int i = threadIdx.x; i < (int)(kVStages * 2 * kOnesBytes / 16); i += kThreads) {
+    const int st = i / (2 * kOnesBytes / 16), r = i % (2 * kOnesBytes / 16);
+    const uint32_t off = r < (int)(kOnesBytes / 16) ? r * 16 : VS::kOnes1 + (r - kOnesBytes / 16) * 16;
+    *reinterpret_cast<uint4*>(&s.v[st][0] + off) = make_uint4(kOneE4M3x4, kOneE4M3x4, kOneE4M3x4, kOneE4M3x4);
+  }
   fence_proxy_async_smem();
   if (warp == 0) {
     tmem_alloc(&s.tmem_base, kTmemCols);
@@ -186,9 +233,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_or_abort(s, &s.v_empty[vs], ph, P)) break;
         if (!wait_or_abort(s, &s.mu_empty[vs], ph, P)) break;
         mbar_arrive_expect_tx(&s.v_full[vs], kPlanes * kTileBytes + 512);
-#pragma unroll
-        for (int pl = 0; pl < kPlanes; ++pl)  // plane pl of head bh: rows (pl * BH + bh) * 128
-          tma_load_2d(s.v[vs][pl], &tmV, &s.v_full[vs], j * 128, (pl * P.B * P.H + bh) * 128);
+        // plane pl of head bh: rows (pl * BH + bh) * 128
+        tma_load_2d(&s.v[vs][0] + VS::kPlane0, &tmV, &s.v_full[vs], j * 128, bh * 128);
+        if (kPlanes == 2)
+          tma_load_2d(&s.v[vs][0] + VS::kPlane1, &tmV, &s.v_full[vs], j * 128, (P.B * P.H + bh) * 128);
         bulk_load(s.mu[vs], P.mu + ((size_t)bh * P.nb + j) * 128, 512, &s.v_full[vs]);
         v_issued = j + 1;
       }
@@ -204,65 +252,68 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_qk = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
-      constexpr uint32_t id_row = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 16);     // also QK_hi
-      constexpr uint32_t id_qk_lo = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, kRowCol);
+      constexpr uint32_t id_pv = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 144);
+      constexpr uint32_t id_pv2 = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
       constexpr uint32_t id_mean = idesc_f32acc(kFmtBF16, kFmtBF16, 128, 128);
       const uint64_t dq[2] = {sdesc_k_sw128(smem_u32(s.q[0])), sdesc_k_sw128(smem_u32(s.q[1]))};
-      const uint64_t dp[2] = {sdesc_k_sw128(smem_u32(s.p[0])), sdesc_k_sw128(smem_u32(s.p[1]))};
       const uint64_t dm[2] = {sdesc_k_sw128(smem_u32(s.mop[0])), sdesc_k_sw128(smem_u32(s.mop[1]))};
-      const uint64_t dones = sdesc_k_sw128(smem_u32(s.ones));
+      auto qk = [&](int t, int ks) {  // S_t = Q_t K^T
+        const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[ks]));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(tmem + col_s(t), dq[t] + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
+      };
+      auto mean = [&](int t, int batch) {  // O_t += R_t M_t of one batch of blocks
+        const int ch = batch % kMeanChunks;
+        umma_f16_ss(tmem + col_ch(t), dm[t] + 2 * ch, dm[t] + 2 * (kMeanChunks + ch), id_mean, 1u);
+      };
       bool ok = wait_or_abort(s, &s.q_full, 0, P) && wait_or_abort(s, &s.k_full[0], 0, P);
       if (ok) {
         tc_fence_after();
-        const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[0]));
-        for (int t = 0; t < 2; ++t) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(tmem + 128 * t, dq[t] + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
-          umma_commit(&s.s_full[t]);
+        qk(0, 0);
+        umma_commit(&s.s_full[0]);
+        // S_1 shares columns with S_0: start it once group 0 has loaded its scores
+        ok = wait_or_abort(s, &s.s_loaded[0], 0, P);
+        if (ok) {
+          tc_fence_after();
+          qk(1, 0);
+          umma_commit(&s.s_full[1]);
+          umma_commit(&s.k_empty[0]);
         }
-        umma_commit(&s.k_empty[0]);
       }
-      // Per block j, tile by tile: [mean batch], PV_t(j), ROW_t(j) as soon as P_t(j)
-      // is ready, then at once the scores of keys 0-111 of block j+1 (QK_lo); the
-      // last 16 keys (QK_hi) overwrite the row-sum columns 112-127, so they wait
-      // until the softmax group has read its row sums, which overlaps QK_lo.
+      // Per block j, tile by tile: [mean batch], PV_t(j) as soon as P_t(j) is in
+      // tensor memory, then the scores of block j+1 (the QK product overwrites
+      // P_t(j) only after PV_t(j) has read it: MMAs of one thread run in order).
       for (int j = 0; ok && j < nkv; ++j) {
         const int vs = j % kVStages;
+        const uint32_t vb = smem_u32(&s.v[vs][0]);
         const int ks = (j + 1) % kKStages;
-        const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[ks]));
         for (int t = 0; t < 2 && ok; ++t) {
           if (!(ok = wait_or_abort(s, &s.p_full[t], j & 1, P))) break;
           if (t == 0 && !(ok = wait_or_abort(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
           tc_fence_after();
-          const uint32_t dO = tmem + 256 + 128 * t;
-          if (j >= 1 && (j - 1) % kMeanBlocks == kMeanBlocks - 1) {
-            const int ch = ((j - 1) / kMeanBlocks) % kMeanChunks;
-            umma_f16_ss(dO, dm[t] + 2 * ch, dm[t] + 2 * (kMeanChunks + ch), id_mean, 1u);
-          }
-#pragma unroll
-          for (int pl = 0; pl < kPlanes; ++pl) {  // O_t += P_t V_hi (+ P_t V_lo)
-            const uint64_t dv = sdesc_k_sw128(smem_u32(s.v[vs][pl]));
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_f8f6f4_ss(dO, dp[t] + 2 * kk, dv + 2 * kk, id_qk, (j > 0 || pl > 0 || kk > 0) ? 1u : 0u);
-          }
+          if (j >= kMeanBlocks && j % kMeanBlocks == 0) mean(t, j / kMeanBlocks - 1);
+          // O_t (+ row sums) += P_t [V ; 1]  (tile 1: [1 ; V])
+          const uint64_t dv = sdesc_k_sw128(vb + (t == 0 ? VS::kPlane0 : 0u));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_f8f6f4_ss(tmem + 128 * t + kRowCol, dp[t] + 2 * kk, dones + 2 * kk, id_row, kk > 0);
-          umma_commit(&s.o_done[t]);
+            umma_f8f6f4_ts(tmem + col_o(t), tmem + col_p(t) + 8 * kk, dv + 2 * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          if (kPlanes == 2) {
+            const uint64_t dv2 = sdesc_k_sw128(vb + VS::kPlane1);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f8f6f4_ts(tmem + col_ch(t), tmem + col_p(t) + 8 * kk, dv2 + 2 * kk, id_pv2, 1u);
+          }
           if (t == 1) umma_commit(&s.v_empty[vs]);
           if (j + 1 < nkv) {
+            // the other tile's group must have loaded the scores in the shared columns
             if (t == 0 && !(ok = wait_or_abort(s, &s.k_full[ks], ((j + 1) / kKStages) & 1, P))) break;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_f8f6f4_ss(tmem + 128 * t, dq[t] + 2 * kk, dk + 2 * kk, id_qk_lo, kk > 0);
-            if (!(ok = wait_or_abort(s, &s.r_free[t], j & 1, P))) break;
+            if (!(ok = wait_or_abort(s, &s.s_loaded[t ^ 1], (j + t) & 1, P))) break;
             tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_f8f6f4_ss(tmem + 128 * t + kRowCol, dq[t] + 2 * kk, dk + kKeyHiOff + 2 * kk, id_row, kk > 0);
+            qk(t, ks);
             umma_commit(&s.s_full[t]);
             if (t == 1) umma_commit(&s.k_empty[ks]);
+          } else {
+            umma_commit(&s.o_done[t]);
           }
         }
       }
@@ -270,8 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < 2 && ok; ++t) {
         if (!(ok = wait_or_abort(s, &s.fin_ready[t], 0, P))) break;
         tc_fence_after();
-        const int ch = ((nkv - 1) / kMeanBlocks) % kMeanChunks;
-        umma_f16_ss(tmem + 256 + 128 * t, dm[t] + 2 * ch, dm[t] + 2 * (kMeanChunks + ch), id_mean, 1u);
+        mean(t, (nkv - 1) / kMeanBlocks);
         umma_commit(&s.o_final[t]);
       }
       // every MMA this thread issued has completed before TMEM is released
@@ -284,16 +334,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hf = (warp >> 2) & 1;        // score / output column half
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + 128 * t;
-    const uint32_t o_addr = tmem + lane_base + 256 + 128 * t + 64 * hf;
+    const uint32_t s_addr = tmem + lane_base + col_s(t) + 64 * hf;
+    const uint32_t p_addr = tmem + lane_base + col_p(t) + 16 * hf;
+    const uint32_t o_addr = tmem + lane_base + col_ch(t) + 64 * hf;
+    const uint32_t l_addr = tmem + lane_base + col_l(t);
     const int qt = pair * 2 + t;
     const bool q_valid = qt < P.nb;
     const float sQ = q_valid ? P.q_scales[(size_t)bh * P.nb + qt] : 1.0f;
     const float sV = __fmul_rn(P.s_v[bh], P.v_mul);   // value scale of the residual codes
     const float inv_sV = __fdiv_rn(1.0f, sV);
     uint8_t* const mo = s.mop[t];
-    uint8_t* const prow = s.p[t] + row * 128;
-    float F = 0.0f, l = 0.0f;
+    // F: running integer frame; Lp: row-sum column after the last block's own
+    // rescale (hf == 1), so that the next read minus Lp is that block's row sum
+    float F = 0.0f, Lp = 0.0f;
     bool ok = true, range_ok = true, fail = false;
     const float* const ksc = P.k_scales + (size_t)bh * P.nb;
     float sK_next = ksc[0];
@@ -306,8 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       fail |= !wait_or_abort(s, &s.s_full[t], j & 1, P);
       tc_fence_after();
       uint32_t raw[2][32];
-      tmem_ld32(s_addr + 64 * hf, raw[0]);
-      tmem_ld32(s_addr + 64 * hf + 32, raw[1]);
+      tmem_ld32(s_addr, raw[0]);
+      tmem_ld32(s_addr + 32, raw[1]);
+      // row-sum column after PV(j-1): s_full(j) follows QK(j), issued after PV(j-1)
+      const uint32_t lraw = (hf == 1 && j > 0) ? tmem_ld1(l_addr) : 0u;
       tmem_ld_wait();
       float sc[64];
 #pragma unroll
@@ -327,10 +382,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float mp = fmax3(m0, m1, fmaxf(sc[62], sc[63]));
       s.xmax[j & 1][t][hf][row] = mp;
+      tc_fence_before();
       if (named_bar_any(1 + t, 256, fail)) {
         ok = false;
         break;
       }
+      // every thread of the group has loaded its scores: the other tile's QK may
+      // now overwrite the shared columns (and the P codes may overwrite S_t)
+      if ((warp & 7) == 0 && lane == 0) mbar_arrive(&s.s_loaded[t]);
       const float tmax = fmaxf(mp, s.xmax[j & 1][t][hf ^ 1][row]);
       // c > 0, so max(c t) = c max(t)
       const float c = __fmul_rn(__fmul_rn(sQ, sK), P.kappa);
@@ -346,24 +405,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       range_ok &= fabsf(Fn) < 524288.0f;
       // ExpCast: one fma per score on the magic-biased fp32; the low byte is the
       // code; the clamp at the magic value is code 0 (masked tail scores are -inf)
+      uint32_t w[16];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t w[8];
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const int i = cc * 32 + q4 * 4;
-          const float2 a = ffma2(make_float2(sc[i], sc[i + 1]), make_float2(c8, c8), make_float2(bias, bias));
-          const float2 b = ffma2(make_float2(sc[i + 2], sc[i + 3]), make_float2(c8, c8), make_float2(bias, bias));
-          w[q4] = pack_codes4(fmaxf(a.x, kMagic), fmaxf(a.y, kMagic), fmaxf(b.x, kMagic), fmaxf(b.y, kMagic));
-        }
-        const int k0 = 4 * hf + 2 * cc;
-        *reinterpret_cast<uint4*>(prow + ((k0 ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(prow + (((k0 + 1) ^ (row & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+      for (int q4 = 0; q4 < 16; ++q4) {
+        const int i = q4 * 4;
+        const float2 a = ffma2(make_float2(sc[i], sc[i + 1]), make_float2(c8, c8), make_float2(bias, bias));
+        const float2 b = ffma2(make_float2(sc[i + 2], sc[i + 3]), make_float2(c8, c8), make_float2(bias, bias));
+        w[q4] = pack4_imad(fmaxf(a.x, kMagic), fmaxf(a.y, kMagic), fmaxf(b.x, kMagic), fmaxf(b.y, kMagic));
       }
-      fence_proxy_async_smem();
+      tmem_st16(p_addr, w);
+      const float Lc = __uint_as_float(lraw);
       if (__any_sync(0xffffffffu, resc)) {
-        // the frame moved: O_t (complete up to block j-1), l and the row sums not
-        // yet handed to a mean MMA are rescaled by the exact 2^(F_old - F_new)
+        // the frame moved: O_t (complete up to block j-1) and its row-sum column
+        // are rescaled by the exact 2^(F_old - F_new); so are the row sums of the
+        // current batch not yet handed to a mean MMA
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
           uint32_t r[32];
@@ -374,59 +429,69 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(o_addr + 32 * cc, r);
           tmem_st_wait();  // the store reads r asynchronously: done before r is reused
         }
-        if (resc && hf == 1) {
-          const int jp = j - 1, ch = (jp / kMeanBlocks) % kMeanChunks;
-          const int nslots = 3 * (jp % kMeanBlocks) + 3;
-          for (int sl = 0; sl < nslots; ++sl) {
-            __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(mo + sw128_off16(row, ch, sl));
-            *e = __float2bfloat16_rn(__bfloat162float(*e) * alpha);
+        if (hf == 1) {
+          tmem_st1(l_addr, __float_as_uint(Lc * alpha));
+          if (resc) {
+            const int jp = j - 1, ch = (jp / kMeanBlocks) % kMeanChunks;
+            const int nslots = 3 * (jp % kMeanBlocks);
+            for (int sl = 0; sl < nslots; ++sl) {
+              __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(mo + sw128_off16(row, ch, sl));
+              *e = __float2bfloat16_rn(__bfloat162float(*e) * alpha);
+            }
           }
-          fence_proxy_async_smem();
         }
       }
-      l *= alpha;
-      F = Fn;
-      tc_fence_before();
-      mbar_arrive(&s.p_full[t]);
-      // row sum of this block's cast P (tensor core), then the mean-MMA operands:
-      // the upper half writes the row sums of its rows, the lower half the block
-      // mean / s_V of channel `row`
-      fail |= !wait_or_abort(s, &s.o_done[t], j & 1, P);
-      tc_fence_after();
-      const float r = __uint_as_float(tmem_ld1(s_addr + kRowCol));
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&s.r_free[t]);
-      l = __fadd_rn(l, r);
-      const int g = j % kMeanBlocks, ch = (j / kMeanBlocks) % kMeanChunks;
-      const bool last = j == nkv - 1;
+      // mean-MMA operands (no MMA of this tile is in flight between s_full and
+      // p_full): the upper half writes the row sum of block j-1 (the column's
+      // growth since the last block, carried into the new frame), the lower half
+      // the block mean / s_V of channel `row` for block j
       if (hf == 1) {
-        __nv_bfloat16 rh, rl;
-        split_bf16(r, rh, rl);
-        st_bf16(mo, sw128_off16(row, ch, 3 * g + 0), rh);
-        st_bf16(mo, sw128_off16(row, ch, 3 * g + 1), rh);
-        st_bf16(mo, sw128_off16(row, ch, 3 * g + 2), rl);
-        if (last)
-          for (int sl = 3 * g + 3; sl < 16; ++sl) st_bf16(mo, sw128_off16(row, ch, sl), __float2bfloat16_rn(0.0f));
+        if (j > 0) {
+          const int jp = j - 1;
+          put_r(mo, row, (jp / kMeanBlocks) % kMeanChunks, jp % kMeanBlocks, __fsub_rn(Lc, Lp) * alpha);
+        }
+        Lp = Lc * alpha;
       } else {
         const int vs = j % kVStages;
         fail |= !wait_or_abort(s, &s.v_full[vs], (j / kVStages) & 1, P);
         const float m = __fmul_rn(s.mu[vs][row], inv_sV);
         mbar_arrive(&s.mu_empty[vs]);
+        const int g = j % kMeanBlocks, ch = (j / kMeanBlocks) % kMeanChunks;
         __nv_bfloat16 mh, ml;
         split_bf16(m, mh, ml);
         st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 0), mh);
         st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 1), ml);
         st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 2), mh);
-        if (last)
+        if (j == nkv - 1)
           for (int sl = 3 * g + 3; sl < 16; ++sl)
             st_bf16(mo, sw128_off16(row, kMeanChunks + ch, sl), __float2bfloat16_rn(0.0f));
       }
-      if (g == kMeanBlocks - 1 || last) fence_proxy_async_smem();
+      // a batch is complete once the row sum of its last block is in: the mean
+      // MMA that reads it is issued right after this block's p_full
+      if (j >= kMeanBlocks && j % kMeanBlocks == 0) fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&s.p_full[t]);
+      F = Fn;
     }
     if (!range_ok) report_status(P.status, VC_ERR_UNSUPPORTED);
     ok = __all_sync(0xffffffffu, ok && !fail);
+    float l = 0.0f;
     if (ok) {
+      // after the last PV: the total row sum, and the last block's share of it
+      ok = __all_sync(0xffffffffu, wait_or_abort(s, &s.o_done[t], 0, P));
+    }
+    if (ok) {
+      tc_fence_after();
+      l = __uint_as_float(tmem_ld1(l_addr));
+      tmem_ld_wait();
+      if (hf == 1) {
+        const int jp = nkv - 1, g = jp % kMeanBlocks, ch = (jp / kMeanBlocks) % kMeanChunks;
+        put_r(mo, row, ch, g, __fsub_rn(l, Lp));
+        for (int sl = 3 * g + 3; sl < 16; ++sl) st_bf16(mo, sw128_off16(row, ch, sl), __float2bfloat16_rn(0.0f));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
       mbar_arrive(&s.fin_ready[t]);
       ok = __all_sync(0xffffffffu, wait_or_abort(s, &s.o_final[t], 0, P));
     }
