@@ -12,20 +12,19 @@
 //
 // One CTA = two 128-row query tiles (t = 0, 1) of one (b, h); both walk all key
 // blocks j = 0 .. nb-1 (permuted order), sharing every K/V tile.
-//   warps 0-7   softmax group of query tile 0: two threads per query row, warps
-//               0-3 take score columns 0-63 and warps 4-7 columns 64-127 (a warp
-//               reaches the 32 tensor-memory lanes of its rank mod 4); the halves
-//               exchange their partial row maxima through shared memory
-//   warps 8-15  softmax group of query tile 1
-//   warp  16    TMA: both Q tiles once; K_j, V^T_j and mu_j into rings
-//   warp  17    MMA issuer (one thread)
+//   warps 0-3   softmax of query tile 0: one thread per query row (warp w
+//               reaches the 32 tensor-memory lanes 32w .. 32w+31)
+//   warps 4-7   softmax of query tile 1
+//   warp  8     TMA: both Q tiles once; K_j and V^T_j into rings; it also
+//               writes the bf16 block-mean operand of the mean MMA
+//   warp  9     MMA issuer (one elected lane)
 // Tensor memory (512 columns):
 //   O_0 [0, 144)    tile 0: output channels 0-127, then 16 row-sum columns
 //   O_1 [144, 288)  tile 1: 16 row-sum columns, then output channels 0-127
 //   S_0 [288, 416)  tile 0 scores; its first 32 columns take the P codes
 //   S_1 [384, 512)  tile 1 scores; P codes in its columns 32-63
 // S_0 and S_1 share 32 columns, so the MMA issuer starts a QK product into one
-// only after the other tile's softmax group has loaded its scores (s_loaded).
+// only after the other tile's softmax warps have loaded their scores (s_loaded).
 // Per block j and tile t the tensor core runs
 //   PV   O_t += P_t [V_j ; 1]     P_t (E4M3 codes) read from tensor memory,
 //        V_j^T (residual codes) with 16 rows of E4M3 1.0 appended from shared
@@ -33,12 +32,13 @@
 //        cast P exactly as PV sees it
 //   QK   S_t = Q_t K_{j+1}^T     kind::f8f6f4, M = N = K = 128
 //   MEAN after every 5 blocks:  O_t += R_t M     kind::f16 with bf16 operands:
-//        R_t = the blocks' row sums r_b (differences of successive l), M = their
-//        block means / s_V, each split into bf16 hi/lo parts (r_hi m_hi +
-//        r_hi m_lo + r_lo m_hi, three K slots a block), both operands in that
-//        tile's own 128-B-swizzled smem tile (R in K chunks 0-1, M in chunks
-//        2-3, alternating by batch); the softmax group writes it only between
-//        s_full and p_full of a block, when no MMA of its tile is in flight
+//        R_t = the blocks' row sums r_b (growth of l from block to block), M =
+//        their block means / s_V, each split into bf16 hi/lo parts (r_hi m_hi +
+//        r_hi m_lo + r_lo m_hi, three K slots a block). R_t sits in a 128-B-
+//        swizzled smem tile of its own (K chunks 0-1, alternating by batch),
+//        written by the softmax threads only between s_full and p_full, when
+//        no MMA of their tile is in flight; M (shared by both tiles) in a
+//        double-buffered unswizzled tile written by the TMA warp
 // so O_t accumulates the whole output in residual-code units; the epilogue is
 // O = s_V O_t / l. The softmax thread of row i keeps the integer running frame
 // F (ceil of the largest log2-domain score so far); a block is cast in the frame
@@ -64,11 +64,12 @@ template <int kPlanes> struct Stages {
 };
 constexpr uint32_t kTileBytes = 128 * 128;  // one 128 x 128 E4M3 tile (or 128 x 64 bf16)
 constexpr uint32_t kOnesBytes = 16 * 128;   // 16 rows of E4M3 1.0 (K = 128 keys)
-constexpr int kThreads = 576;
-constexpr int kTmaWarp = 16, kMmaWarp = 17;
+constexpr uint32_t kMopBytes = 128 * 16 * 2;  // M operand of one batch: 128 channels x 16 bf16
+constexpr int kThreads = 320;
+constexpr int kTmaWarp = 8, kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMeanBlocks = 5;              // key blocks per mean MMA (3 K slots each: 15 of 16)
-constexpr int kMeanChunks = 2;              // 16-slot K chunks per operand (R: 0-1, M: 2-3)
+constexpr int kMeanChunks = 2;              // R: 16-slot K chunks 0 and 1, alternating by batch
 constexpr uint32_t kOneE4M3x4 = 0x38383838u;
 // tensor-memory columns (see the layout above)
 __device__ __forceinline__ constexpr uint32_t col_o(int t) { return t ? 144u : 0u; }    // PV accumulator, N = 144
@@ -94,12 +95,12 @@ struct __align__(1024) SmemAttn {
   uint8_t q[2][kTileBytes];
   uint8_t k[kKStages][kTileBytes];
   uint8_t v[kVStages][VStage<kPlanes>::kBytes];
-  uint8_t mop[2][kTileBytes];    // bf16 operands of the mean MMA, one tile per query tile
-  float mu[kVStages][128];
-  float xmax[2][2][2][128];      // [block parity][query tile][column half][row] partial maxima
+  uint8_t rop[2][kTileBytes];    // R operand of the mean MMA, one 128-B-swizzled tile per query tile
+  uint8_t mop[2][kMopBytes];     // M operand, unswizzled, one per batch parity
   uint64_t q_full;
   uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t v_full[kVStages], v_empty[kVStages], mu_empty[kVStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t m_full[2], m_empty[2];
   uint64_t s_full[2], s_loaded[2], p_full[2], o_done[2], fin_ready[2], o_final[2];
   uint64_t mma_drain;
   uint32_t tmem_base;
@@ -116,6 +117,12 @@ __device__ __forceinline__ bool wait_or_abort(Smem& s, uint64_t* bar, uint32_t p
   s.abort_flag = 1;
   report_status(P.status, VC_ERR_TIMEOUT);
   return false;
+}
+
+// wait_or_abort for a whole warp: every lane returns the same answer.
+template <class Smem>
+__device__ __forceinline__ bool wait_warp(Smem& s, uint64_t* bar, uint32_t parity, const AttnParams& P) {
+  return __all_sync(0xffffffffu, wait_or_abort(s, bar, parity, P));
 }
 
 // Byte offset of 16-bit element `slot` (K index 16*chunk + slot) of row `row` in
@@ -136,13 +143,21 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bflo
 }
 
 // Writes the three K slots of one block's row sum r (slots hi, hi, lo) into the
-// R chunk of the mean-operand tile.
-__device__ __forceinline__ void put_r(uint8_t* mo, int row, int ch, int g, float r) {
+// R operand tile.
+__device__ __forceinline__ void put_r(uint8_t* ro, int row, int ch, int g, float r) {
   __nv_bfloat16 rh, rl;
   split_bf16(r, rh, rl);
-  st_bf16(mo, sw128_off16(row, ch, 3 * g + 0), rh);
-  st_bf16(mo, sw128_off16(row, ch, 3 * g + 1), rh);
-  st_bf16(mo, sw128_off16(row, ch, 3 * g + 2), rl);
+  st_bf16(ro, sw128_off16(row, ch, 3 * g + 0), rh);
+  st_bf16(ro, sw128_off16(row, ch, 3 * g + 1), rh);
+  st_bf16(ro, sw128_off16(row, ch, 3 * g + 2), rl);
+}
+
+// M operand layout (unswizzled K-major, core matrices of 8 channels x 8 slots):
+// channel c, slots 8h .. 8h+7 are the 16 bytes at (c/8)*256 + h*128 + (c%8)*16.
+constexpr uint32_t kMopLbo = 128, kMopSbo = 256;
+
+__device__ __forceinline__ uint32_t bf16_bits(__nv_bfloat16 x) {
+  return (uint32_t)*reinterpret_cast<const uint16_t*>(&x);
 }
 
 // Four magic-biased codes (low bytes of the fp32 patterns) into one word, a in
@@ -167,6 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y;
   const int nkv = P.nb;
+  const int nbatch = (nkv + kMeanBlocks - 1) / kMeanBlocks;
 
   if (threadIdx.x == 0) {
     mbar_init(&s.q_full, 1);
@@ -177,25 +193,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kVStages; ++i) {
       mbar_init(&s.v_full[i], 1);
       mbar_init(&s.v_empty[i], 1);
-      mbar_init(&s.mu_empty[i], 256);
     }
     for (int t = 0; t < 2; ++t) {
+      mbar_init(&s.m_full[t], 1);
+      mbar_init(&s.m_empty[t], 1);
       mbar_init(&s.s_full[t], 1);
-      mbar_init(&s.s_loaded[t], 1);
-      mbar_init(&s.p_full[t], 256);
+      mbar_init(&s.s_loaded[t], 4);
+      mbar_init(&s.p_full[t], 128);
       mbar_init(&s.o_done[t], 1);
-      mbar_init(&s.fin_ready[t], 256);
+      mbar_init(&s.fin_ready[t], 128);
       mbar_init(&s.o_final[t], 1);
     }
     mbar_init(&s.mma_drain, 1);
     s.abort_flag = 0;
     fence_barrier_init();
   }
-  // mean-MMA operands start at zero (unused K slots stay zero); the two bands of
-  // every V stage are all E4M3 1.0 (every byte 0x38, so the swizzle does not
-  // matter); the TMA never writes them
+  // R operands start at zero (unused K slots stay zero); the two bands of every
+  // V stage are all E4M3 1.0 (every byte 0x38, so the swizzle does not matter);
+  // the TMA never writes them
   for (int i = threadIdx.x; i < (int)(2 * kTileBytes / 16); i += kThreads)
-    *reinterpret_cast<uint4*>(&s.mop[0][0] + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(&s.rop[0][0] + i * 16) = make_uint4(0u, 0u, 0u, 0u);
   for (int i = threadIdx.x; i < (int)(kVStages * 2 * kOnesBytes / 16); i += kThreads) {
     const int st = i / (2 * kOnesBytes / 16), r = i % (2 * kOnesBytes / 16);
     const uint32_t off = r < (int)(kOnesBytes / 16) ? r * 16 : VS::kOnes1 + (r - kOnesBytes / 16) * 16;
@@ -210,10 +227,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
+  const float sV = __fmul_rn(P.s_v[bh], P.v_mul);   // value scale of the residual codes
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp runs the loop (its values stay warp-uniform); one elected
+    // lane issues the copies. Every kMeanBlocks blocks the warp also writes the
+    // M operand of one batch: lane l takes channels l, l+32, l+64, l+96.
+    const bool leader = elect_one();
+    const float inv_sV = __fdiv_rn(1.0f, sV);
+    const float* const mu_bh = P.mu + (size_t)bh * P.nb * 128;
+    float mnext[kMeanBlocks][4];  // block means of the next batch, loaded one batch ahead
+    auto load_means = [&](int batch) {
+#pragma unroll
+      for (int g = 0; g < kMeanBlocks; ++g) {
+        const int b = batch * kMeanBlocks + g;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mnext[g][i] = b < nkv ? __ldg(mu_bh + (size_t)b * 128 + lane + 32 * i) : 0.0f;
+      }
+    };
+    load_means(0);
+    if (leader) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
@@ -221,79 +255,134 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(&s.q_full, 2 * kTileBytes);
       tma_load_2d(s.q[0], &tmQ, &s.q_full, 0, rowq);
       tma_load_2d(s.q[1], &tmQ, &s.q_full, 0, rowq + 128);  // past the head's last tile: unused rows
-      int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < nkv && !*(volatile int32_t*)&s.abort_flag; ++j) {
-        const int ks = j % kKStages;
-        if (!wait_or_abort(s, &s.k_empty[ks], ((j / kKStages) & 1) ^ 1, P)) break;
+    }
+    int k_issued = 0, v_issued = 0;
+    for (int j = 0; j < nkv && !*(volatile int32_t*)&s.abort_flag; ++j) {
+      const int ks = j % kKStages;
+      if (!wait_warp(s, &s.k_empty[ks], ((j / kKStages) & 1) ^ 1, P)) break;
+      if (leader) {
         mbar_arrive_expect_tx(&s.k_full[ks], kTileBytes);
         tma_load_2d(s.k[ks], &tmK, &s.k_full[ks], 0, bh * P.S_pad + j * 128);
-        k_issued = j + 1;
-        const int vs = j % kVStages;
-        const uint32_t ph = ((j / kVStages) & 1) ^ 1;
-        if (!wait_or_abort(s, &s.v_empty[vs], ph, P)) break;
-        if (!wait_or_abort(s, &s.mu_empty[vs], ph, P)) break;
-        mbar_arrive_expect_tx(&s.v_full[vs], kPlanes * kTileBytes + 512);
+      }
+      k_issued = j + 1;
+      const int vs = j % kVStages;
+      if (!wait_warp(s, &s.v_empty[vs], ((j / kVStages) & 1) ^ 1, P)) break;
+      if (leader) {
+        mbar_arrive_expect_tx(&s.v_full[vs], kPlanes * kTileBytes);
         // plane pl of head bh: rows (pl * BH + bh) * 128
         tma_load_2d(&s.v[vs][0] + VS::kPlane0, &tmV, &s.v_full[vs], j * 128, bh * 128);
         if (kPlanes == 2)
           tma_load_2d(&s.v[vs][0] + VS::kPlane1, &tmV, &s.v_full[vs], j * 128, (P.B * P.H + bh) * 128);
-        bulk_load(s.mu[vs], P.mu + ((size_t)bh * P.nb + j) * 128, 512, &s.v_full[vs]);
-        v_issued = j + 1;
       }
-      // copies still in flight must land before the CTA exits
-      const uint64_t drain_ns = 100000000ull;
-      mbar_wait(&s.q_full, 0, drain_ns, nullptr);
-      for (int j = max(0, k_issued - kKStages); j < k_issued; ++j)
-        mbar_wait(&s.k_full[j % kKStages], (j / kKStages) & 1, drain_ns, nullptr);
-      for (int j = max(0, v_issued - kVStages); j < v_issued; ++j)
-        mbar_wait(&s.v_full[j % kVStages], (j / kVStages) & 1, drain_ns, nullptr);
+      v_issued = j + 1;
+      if (j % kMeanBlocks == 0) {
+        // M operand of batch n = j / kMeanBlocks: slots (hi, lo, hi) of mu_b / s_V
+        // for its blocks, zero for blocks past the end and for slot 15
+        const int n = j / kMeanBlocks, mb = n & 1;
+        if (!wait_warp(s, &s.m_empty[mb], ((n >> 1) & 1) ^ 1, P)) break;
+        float cur[kMeanBlocks][4];
+#pragma unroll
+        for (int g = 0; g < kMeanBlocks; ++g)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cur[g][i] = mnext[g][i];
+        if (n + 1 < nbatch) load_means(n + 1);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = lane + 32 * i;
+          uint32_t h[8];  // 16 slots, two per word
+          uint32_t sl[16];
+#pragma unroll
+          for (int g = 0; g < kMeanBlocks; ++g) {
+            __nv_bfloat16 mh, ml;
+            split_bf16(__fmul_rn(cur[g][i], inv_sV), mh, ml);
+            sl[3 * g + 0] = bf16_bits(mh);
+            sl[3 * g + 1] = bf16_bits(ml);
+            sl[3 * g + 2] = bf16_bits(mh);
+          }
+          sl[15] = 0u;
+#pragma unroll
+          for (int k2 = 0; k2 < 8; ++k2) h[k2] = sl[2 * k2] | (sl[2 * k2 + 1] << 16);
+          uint8_t* dst = s.mop[mb] + (c >> 3) * kMopSbo + (c & 7) * 16;
+          *reinterpret_cast<uint4*>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(dst + kMopLbo) = make_uint4(h[4], h[5], h[6], h[7]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (leader) mbar_arrive(&s.m_full[mb]);
+      }
     }
+    // copies still in flight must land before the CTA exits
+    const uint64_t drain_ns = 100000000ull;
+    mbar_wait(&s.q_full, 0, drain_ns, nullptr);
+    for (int j = max(0, k_issued - kKStages); j < k_issued; ++j)
+      mbar_wait(&s.k_full[j % kKStages], (j / kKStages) & 1, drain_ns, nullptr);
+    for (int j = max(0, v_issued - kVStages); j < v_issued; ++j)
+      mbar_wait(&s.v_full[j % kVStages], (j / kVStages) & 1, drain_ns, nullptr);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t id_qk = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
-      constexpr uint32_t id_pv = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 144);
-      constexpr uint32_t id_pv2 = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
-      constexpr uint32_t id_mean = idesc_f32acc(kFmtBF16, kFmtBF16, 128, 128);
-      const uint64_t dq[2] = {sdesc_k_sw128(smem_u32(s.q[0])), sdesc_k_sw128(smem_u32(s.q[1]))};
-      const uint64_t dm[2] = {sdesc_k_sw128(smem_u32(s.mop[0])), sdesc_k_sw128(smem_u32(s.mop[1]))};
-      auto qk = [&](int t, int ks) {  // S_t = Q_t K^T
-        const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[ks]));
+    // The whole warp runs the loop so that descriptors and addresses stay
+    // warp-uniform (uniform registers feed tcgen05.mma directly); one elected
+    // lane issues the MMAs and the commits that track them.
+    const bool leader = elect_one();
+    constexpr uint32_t id_qk = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
+    constexpr uint32_t id_pv = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 144);
+    constexpr uint32_t id_pv2 = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
+    constexpr uint32_t id_mean = idesc_f32acc(kFmtBF16, kFmtBF16, 128, 128);
+    const uint64_t dq[2] = {sdesc_k_sw128(smem_u32(s.q[0])), sdesc_k_sw128(smem_u32(s.q[1]))};
+    const uint64_t dr[2] = {sdesc_k_sw128(smem_u32(s.rop[0])), sdesc_k_sw128(smem_u32(s.rop[1]))};
+    const uint64_t dmo[2] = {sdesc_k_noswz(smem_u32(s.mop[0]), kMopLbo, kMopSbo),
+                             sdesc_k_noswz(smem_u32(s.mop[1]), kMopLbo, kMopSbo)};
+    auto qk = [&](int t, int ks) {  // S_t = Q_t K^T
+      const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[ks]));
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(tmem + col_s(t), dq[t] + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
-      };
-      auto mean = [&](int t, int batch) {  // O_t += R_t M_t of one batch of blocks
-        const int ch = batch % kMeanChunks;
-        umma_f16_ss(tmem + col_ch(t), dm[t] + 2 * ch, dm[t] + 2 * (kMeanChunks + ch), id_mean, 1u);
-      };
-      bool ok = wait_or_abort(s, &s.q_full, 0, P) && wait_or_abort(s, &s.k_full[0], 0, P);
+      }
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (leader) umma_commit(bar);
+    };
+    // O_t += R_t M of one batch of blocks; tile 0 first waits for the M operand,
+    // tile 1 releases it
+    auto mean = [&](int t, int batch) -> bool {
+      const int mb = batch & 1;
+      if (t == 0) {
+        if (!wait_warp(s, &s.m_full[mb], (batch >> 1) & 1, P)) return false;
+        tc_fence_after();
+      }
+      if (leader) umma_f16_ss(tmem + col_ch(t), dr[t] + 2 * (batch % kMeanChunks), dmo[mb], id_mean, 1u);
+      if (t == 1) commit(&s.m_empty[mb]);
+      return true;
+    };
+    bool ok = wait_warp(s, &s.q_full, 0, P) && wait_warp(s, &s.k_full[0], 0, P);
+    if (ok) {
+      tc_fence_after();
+      qk(0, 0);
+      commit(&s.s_full[0]);
+      // S_1 shares columns with S_0: start it once tile 0's threads have loaded their scores
+      ok = wait_warp(s, &s.s_loaded[0], 0, P);
       if (ok) {
         tc_fence_after();
-        qk(0, 0);
-        umma_commit(&s.s_full[0]);
-        // S_1 shares columns with S_0: start it once group 0 has loaded its scores
-        ok = wait_or_abort(s, &s.s_loaded[0], 0, P);
-        if (ok) {
-          tc_fence_after();
-          qk(1, 0);
-          umma_commit(&s.s_full[1]);
-          umma_commit(&s.k_empty[0]);
-        }
+        qk(1, 0);
+        commit(&s.s_full[1]);
+        commit(&s.k_empty[0]);
       }
-      // Per block j, tile by tile: [mean batch], PV_t(j) as soon as P_t(j) is in
-      // tensor memory, then the scores of block j+1 (the QK product overwrites
-      // P_t(j) only after PV_t(j) has read it: MMAs of one thread run in order).
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int vs = j % kVStages;
-        const uint32_t vb = smem_u32(&s.v[vs][0]);
-        const int ks = (j + 1) % kKStages;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!(ok = wait_or_abort(s, &s.p_full[t], j & 1, P))) break;
-          if (t == 0 && !(ok = wait_or_abort(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
-          tc_fence_after();
-          if (j >= kMeanBlocks && j % kMeanBlocks == 0) mean(t, j / kMeanBlocks - 1);
-          // O_t (+ row sums) += P_t [V ; 1]  (tile 1: [1 ; V])
-          const uint64_t dv = sdesc_k_sw128(vb + (t == 0 ? VS::kPlane0 : 0u));
+    }
+    // Per block j, tile by tile: [mean batch], PV_t(j) as soon as P_t(j) is in
+    // tensor memory, then the scores of block j+1 (the QK product overwrites
+    // P_t(j) only after PV_t(j) has read it: MMAs of one thread run in order).
+    for (int j = 0; ok && j < nkv; ++j) {
+      const int vs = j % kVStages;
+      const uint32_t vb = smem_u32(&s.v[vs][0]);
+      const int ks = (j + 1) % kKStages;
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (!(ok = wait_warp(s, &s.p_full[t], j & 1, P))) break;
+        if (t == 0 && !(ok = wait_warp(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
+        tc_fence_after();
+        if (j >= kMeanBlocks && j % kMeanBlocks == 0 && !(ok = mean(t, j / kMeanBlocks - 1))) break;
+        // O_t (+ row sums) += P_t [V ; 1]  (tile 1: [1 ; V])
+        const uint64_t dv = sdesc_k_sw128(vb + (t == 0 ? VS::kPlane0 : 0u));
+        if (leader) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_f8f6f4_ts(tmem + col_o(t), tmem + col_p(t) + 8 * kk, dv + 2 * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
@@ -303,95 +392,85 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < 4; ++kk)
               umma_f8f6f4_ts(tmem + col_ch(t), tmem + col_p(t) + 8 * kk, dv2 + 2 * kk, id_pv2, 1u);
           }
-          if (t == 1) umma_commit(&s.v_empty[vs]);
-          if (j + 1 < nkv) {
-            // the other tile's group must have loaded the scores in the shared columns
-            if (t == 0 && !(ok = wait_or_abort(s, &s.k_full[ks], ((j + 1) / kKStages) & 1, P))) break;
-            if (!(ok = wait_or_abort(s, &s.s_loaded[t ^ 1], (j + t) & 1, P))) break;
-            tc_fence_after();
-            qk(t, ks);
-            umma_commit(&s.s_full[t]);
-            if (t == 1) umma_commit(&s.k_empty[ks]);
-          } else {
-            umma_commit(&s.o_done[t]);
-          }
+        }
+        if (t == 1) commit(&s.v_empty[vs]);
+        if (j + 1 < nkv) {
+          // the other tile's threads must have loaded the scores in the shared columns
+          if (t == 0 && !(ok = wait_warp(s, &s.k_full[ks], ((j + 1) / kKStages) & 1, P))) break;
+          if (!(ok = wait_warp(s, &s.s_loaded[t ^ 1], (j + t) & 1, P))) break;
+          tc_fence_after();
+          qk(t, ks);
+          commit(&s.s_full[t]);
+          if (t == 1) commit(&s.k_empty[ks]);
+        } else {
+          commit(&s.o_done[t]);
         }
       }
-      // the last (possibly partial) batch of block means, then the output is final
-      for (int t = 0; t < 2 && ok; ++t) {
-        if (!(ok = wait_or_abort(s, &s.fin_ready[t], 0, P))) break;
-        tc_fence_after();
-        mean(t, (nkv - 1) / kMeanBlocks);
-        umma_commit(&s.o_final[t]);
-      }
-      // every MMA this thread issued has completed before TMEM is released
-      umma_commit(&s.mma_drain);
-      mbar_wait(&s.mma_drain, 0, 100000000ull, nullptr);
     }
+    // the last (possibly partial) batch of block means, then the output is final
+    for (int t = 0; t < 2 && ok; ++t) {
+      if (!(ok = wait_warp(s, &s.fin_ready[t], 0, P))) break;
+      tc_fence_after();
+      if (!(ok = mean(t, nbatch - 1))) break;
+      commit(&s.o_final[t]);
+    }
+    // every MMA the leader issued has completed before TMEM is released
+    commit(&s.mma_drain);
+    mbar_wait(&s.mma_drain, 0, 100000000ull, nullptr);
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int t = warp >> 3;               // query tile
-    const int hf = (warp >> 2) & 1;        // score / output column half
+    const int t = warp >> 2;               // query tile
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + col_s(t) + 64 * hf;
-    const uint32_t p_addr = tmem + lane_base + col_p(t) + 16 * hf;
-    const uint32_t o_addr = tmem + lane_base + col_ch(t) + 64 * hf;
+    const uint32_t s_addr = tmem + lane_base + col_s(t);
+    const uint32_t p_addr = tmem + lane_base + col_p(t);
+    const uint32_t o_addr = tmem + lane_base + col_ch(t);
     const uint32_t l_addr = tmem + lane_base + col_l(t);
     const int qt = pair * 2 + t;
     const bool q_valid = qt < P.nb;
     const float sQ = q_valid ? P.q_scales[(size_t)bh * P.nb + qt] : 1.0f;
-    const float sV = __fmul_rn(P.s_v[bh], P.v_mul);   // value scale of the residual codes
-    const float inv_sV = __fdiv_rn(1.0f, sV);
-    uint8_t* const mo = s.mop[t];
+    uint8_t* const ro = s.rop[t];
     // F: running integer frame; Lp: row-sum column after the last block's own
-    // rescale (hf == 1), so that the next read minus Lp is that block's row sum
+    // rescale, so that the next read minus Lp is that block's row sum
     float F = 0.0f, Lp = 0.0f;
-    bool ok = true, range_ok = true, fail = false;
+    bool ok = true, range_ok = true;
     const float* const ksc = P.k_scales + (size_t)bh * P.nb;
     float sK_next = ksc[0];
     for (int j = 0; j < nkv; ++j) {
       const float sK = sK_next;                      // this block's K scale, loaded one block ahead
       if (j + 1 < nkv) sK_next = ksc[j + 1];
-      // A failed (timed-out) wait never breaks the loop on its own: the group
-      // leaves together at the next row-max exchange, whose barrier ORs the
-      // failures, so no thread is left waiting in that barrier.
-      fail |= !wait_or_abort(s, &s.s_full[t], j & 1, P);
+      if (!(ok = wait_warp(s, &s.s_full[t], j & 1, P))) break;
       tc_fence_after();
-      uint32_t raw[2][32];
-      tmem_ld32(s_addr, raw[0]);
-      tmem_ld32(s_addr + 32, raw[1]);
+      uint32_t sc[4][32];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(s_addr + 32 * cc, sc[cc]);
       // row-sum column after PV(j-1): s_full(j) follows QK(j), issued after PV(j-1)
-      const uint32_t lraw = (hf == 1 && j > 0) ? tmem_ld1(l_addr) : 0u;
+      const uint32_t lraw = j > 0 ? tmem_ld1(l_addr) : 0u;
       tmem_ld_wait();
-      float sc[64];
-#pragma unroll
-      for (int i = 0; i < 64; ++i) sc[i] = __uint_as_float(raw[i >> 5][i & 31]);
-      const int valid = min(128, P.S - j * 128) - 64 * hf;   // valid columns of this half
-      if (valid < 64) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (i >= valid) sc[i] = -INFINITY;
-      }
-      // partial max of this half's raw scores, then the full row max
-      float m0 = sc[0], m1 = sc[1];
-#pragma unroll
-      for (int i = 2; i < 62; i += 4) {
-        m0 = fmax3(m0, sc[i + 0], sc[i + 1]);
-        m1 = fmax3(m1, sc[i + 2], sc[i + 3]);
-      }
-      const float mp = fmax3(m0, m1, fmaxf(sc[62], sc[63]));
-      s.xmax[j & 1][t][hf][row] = mp;
+      // this warp's scores are in registers: the other tile's QK may now overwrite
+      // the shared columns (and the P codes may overwrite S_t)
       tc_fence_before();
-      if (named_bar_any(1 + t, 256, fail)) {
-        ok = false;
-        break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.s_loaded[t]);
+      const int valid = min(128, P.S - j * 128);
+      if (valid < 128) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i >= valid) sc[i >> 5][i & 31] = __float_as_uint(-INFINITY);
       }
-      // every thread of the group has loaded its scores: the other tile's QK may
-      // now overwrite the shared columns (and the P codes may overwrite S_t)
-      if ((warp & 7) == 0 && lane == 0) mbar_arrive(&s.s_loaded[t]);
-      const float tmax = fmaxf(mp, s.xmax[j & 1][t][hf ^ 1][row]);
-      // c > 0, so max(c t) = c max(t)
+#define SC(i) __uint_as_float(sc[(i) >> 5][(i) & 31])
+      // row max of the raw scores (c > 0, so max(c t) = c max(t))
+      float m0 = SC(0), m1 = SC(1), m2 = SC(2), m3 = SC(3);
+#pragma unroll
+      for (int i = 4; i < 124; i += 8) {
+        m0 = fmax3(m0, SC(i + 0), SC(i + 1));
+        m1 = fmax3(m1, SC(i + 2), SC(i + 3));
+        m2 = fmax3(m2, SC(i + 4), SC(i + 5));
+        m3 = fmax3(m3, SC(i + 6), SC(i + 7));
+      }
+      m0 = fmax3(m0, SC(124), SC(125));
+      m1 = fmax3(m1, SC(126), SC(127));
+      const float tmax = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
       const float c = __fmul_rn(__fmul_rn(sQ, sK), P.kappa);
       const float Mtile = ceilf(__fmul_rn(c, tmax));
       const float Fn = j == 0 ? Mtile : fmaxf(F, Mtile);
@@ -405,22 +484,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       range_ok &= fabsf(Fn) < 524288.0f;
       // ExpCast: one fma per score on the magic-biased fp32; the low byte is the
       // code; the clamp at the magic value is code 0 (masked tail scores are -inf)
-      uint32_t w[16];
+      uint32_t w[32];
 #pragma unroll
-      for (int q4 = 0; q4 < 16; ++q4) {
+      for (int q4 = 0; q4 < 32; ++q4) {
         const int i = q4 * 4;
-        const float2 a = ffma2(make_float2(sc[i], sc[i + 1]), make_float2(c8, c8), make_float2(bias, bias));
-        const float2 b = ffma2(make_float2(sc[i + 2], sc[i + 3]), make_float2(c8, c8), make_float2(bias, bias));
+        const float2 a = ffma2(make_float2(SC(i), SC(i + 1)), make_float2(c8, c8), make_float2(bias, bias));
+        const float2 b = ffma2(make_float2(SC(i + 2), SC(i + 3)), make_float2(c8, c8), make_float2(bias, bias));
         w[q4] = pack4_imad(fmaxf(a.x, kMagic), fmaxf(a.y, kMagic), fmaxf(b.x, kMagic), fmaxf(b.y, kMagic));
       }
-      tmem_st16(p_addr, w);
+#undef SC
+      tmem_st32(p_addr, w);
       const float Lc = __uint_as_float(lraw);
       if (__any_sync(0xffffffffu, resc)) {
         // the frame moved: O_t (complete up to block j-1) and its row-sum column
         // are rescaled by the exact 2^(F_old - F_new); so are the row sums of the
         // current batch not yet handed to a mean MMA
 #pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint32_t r[32];
           tmem_ld32(o_addr + 32 * cc, r);
           tmem_ld_wait();
@@ -429,43 +509,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(o_addr + 32 * cc, r);
           tmem_st_wait();  // the store reads r asynchronously: done before r is reused
         }
-        if (hf == 1) {
-          tmem_st1(l_addr, __float_as_uint(Lc * alpha));
-          if (resc) {
-            const int jp = j - 1, ch = (jp / kMeanBlocks) % kMeanChunks;
-            const int nslots = 3 * (jp % kMeanBlocks);
-            for (int sl = 0; sl < nslots; ++sl) {
-              __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(mo + sw128_off16(row, ch, sl));
-              *e = __float2bfloat16_rn(__bfloat162float(*e) * alpha);
-            }
+        tmem_st1(l_addr, __float_as_uint(Lc * alpha));
+        if (resc) {
+          const int jp = j - 1, ch = (jp / kMeanBlocks) % kMeanChunks;
+          const int nslots = 3 * (jp % kMeanBlocks);
+          for (int sl = 0; sl < nslots; ++sl) {
+            __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(ro + sw128_off16(row, ch, sl));
+            *e = __float2bfloat16_rn(__bfloat162float(*e) * alpha);
           }
         }
       }
-      // mean-MMA operands (no MMA of this tile is in flight between s_full and
-      // p_full): the upper half writes the row sum of block j-1 (the column's
-      // growth since the last block, carried into the new frame), the lower half
-      // the block mean / s_V of channel `row` for block j
-      if (hf == 1) {
-        if (j > 0) {
-          const int jp = j - 1;
-          put_r(mo, row, (jp / kMeanBlocks) % kMeanChunks, jp % kMeanBlocks, __fsub_rn(Lc, Lp) * alpha);
-        }
-        Lp = Lc * alpha;
-      } else {
-        const int vs = j % kVStages;
-        fail |= !wait_or_abort(s, &s.v_full[vs], (j / kVStages) & 1, P);
-        const float m = __fmul_rn(s.mu[vs][row], inv_sV);
-        mbar_arrive(&s.mu_empty[vs]);
-        const int g = j % kMeanBlocks, ch = (j / kMeanBlocks) % kMeanChunks;
-        __nv_bfloat16 mh, ml;
-        split_bf16(m, mh, ml);
-        st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 0), mh);
-        st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 1), ml);
-        st_bf16(mo, sw128_off16(row, kMeanChunks + ch, 3 * g + 2), mh);
-        if (j == nkv - 1)
-          for (int sl = 3 * g + 3; sl < 16; ++sl)
-            st_bf16(mo, sw128_off16(row, kMeanChunks + ch, sl), __float2bfloat16_rn(0.0f));
+      // R operand (no MMA of this tile is in flight between s_full and p_full):
+      // the row sum of block j-1 is the column's growth since the last block,
+      // carried into the new frame
+      if (j > 0) {
+        const int jp = j - 1;
+        put_r(ro, row, (jp / kMeanBlocks) % kMeanChunks, jp % kMeanBlocks, __fsub_rn(Lc, Lp) * alpha);
       }
+      Lp = Lc * alpha;
       // a batch is complete once the row sum of its last block is in: the mean
       // MMA that reads it is issued right after this block's p_full
       if (j >= kMeanBlocks && j % kMeanBlocks == 0) fence_proxy_async_smem();
@@ -475,36 +536,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       F = Fn;
     }
     if (!range_ok) report_status(P.status, VC_ERR_UNSUPPORTED);
-    ok = __all_sync(0xffffffffu, ok && !fail);
     float l = 0.0f;
-    if (ok) {
-      // after the last PV: the total row sum, and the last block's share of it
-      ok = __all_sync(0xffffffffu, wait_or_abort(s, &s.o_done[t], 0, P));
-    }
+    // after the last PV: the total row sum, and the last block's share of it
+    if (ok) ok = wait_warp(s, &s.o_done[t], 0, P);
     if (ok) {
       tc_fence_after();
       l = __uint_as_float(tmem_ld1(l_addr));
       tmem_ld_wait();
-      if (hf == 1) {
-        const int jp = nkv - 1, g = jp % kMeanBlocks, ch = (jp / kMeanBlocks) % kMeanChunks;
-        put_r(mo, row, ch, g, __fsub_rn(l, Lp));
-        for (int sl = 3 * g + 3; sl < 16; ++sl) st_bf16(mo, sw128_off16(row, ch, sl), __float2bfloat16_rn(0.0f));
-      }
+      const int jp = nkv - 1, g = jp % kMeanBlocks, ch = (jp / kMeanBlocks) % kMeanChunks;
+      put_r(ro, row, ch, g, __fsub_rn(l, Lp));
+      for (int sl = 3 * g + 3; sl < 16; ++sl) st_bf16(ro, sw128_off16(row, ch, sl), __float2bfloat16_rn(0.0f));
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&s.fin_ready[t]);
-      ok = __all_sync(0xffffffffu, wait_or_abort(s, &s.o_final[t], 0, P));
+      ok = wait_warp(s, &s.o_final[t], 0, P);
     }
     if (ok) {
-      // epilogue: O = s_V O_t / l, BF16, original query order and layout; this
-      // thread writes channels 64 hf .. 64 hf + 63 of its row
+      // epilogue: O = s_V O_t / l, BF16, original query order and layout
       tc_fence_after();
       const int q = qt * 128 + row;
       const float scale = __fdiv_rn(sV, l);
       const int b = bh / P.H, h = bh % P.H;
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(P.o) + (((size_t)b * P.S + q) * P.H + h) * 128 + 64 * hf;
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(P.o) + (((size_t)b * P.S + q) * P.H + h) * 128;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t r[32];
         tmem_ld32(o_addr + 32 * cc, r);
         tmem_ld_wait();
