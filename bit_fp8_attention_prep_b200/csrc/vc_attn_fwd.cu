@@ -21,10 +21,13 @@
 // Tensor memory (512 columns):
 //   O_0 [0, 144)    tile 0: output channels 0-127, then 16 row-sum columns
 //   O_1 [144, 288)  tile 1: 16 row-sum columns, then output channels 0-127
-//   S_0 [288, 416)  tile 0 scores; its first 32 columns take the P codes
-//   S_1 [384, 512)  tile 1 scores; P codes in its columns 32-63
-// S_0 and S_1 share 32 columns, so the MMA issuer starts a QK product into one
-// only after the other tile's softmax warps have loaded their scores (s_loaded).
+//   S_0 [288, 416)  tile 0 scores
+//   S_1 [320, 448)  tile 1 scores (shares 96 columns with S_0)
+//   P_0 [448, 480), P_1 [480, 512)   E4M3 probability codes, 4 per column
+// The QK products alternate between the tiles: each starts only after the
+// other tile's softmax warps have loaded the scores in the shared columns
+// (s_loaded). P has columns of its own, so the scores of block j+1 are computed
+// while the softmax threads still cast block j.
 // Per block j and tile t the tensor core runs
 //   PV   O_t += P_t [V_j ; 1]     P_t (E4M3 codes) read from tensor memory,
 //        V_j^T (residual codes) with 16 rows of E4M3 1.0 appended from shared
@@ -75,8 +78,8 @@ constexpr uint32_t kOneE4M3x4 = 0x38383838u;
 __device__ __forceinline__ constexpr uint32_t col_o(int t) { return t ? 144u : 0u; }    // PV accumulator, N = 144
 __device__ __forceinline__ constexpr uint32_t col_ch(int t) { return t ? 160u : 0u; }   // output channels 0-127
 __device__ __forceinline__ constexpr uint32_t col_l(int t) { return t ? 144u : 128u; }  // first row-sum column
-__device__ __forceinline__ constexpr uint32_t col_s(int t) { return t ? 384u : 288u; }  // scores
-__device__ __forceinline__ constexpr uint32_t col_p(int t) { return t ? 416u : 288u; }  // P codes, 32 columns
+__device__ __forceinline__ constexpr uint32_t col_s(int t) { return t ? 320u : 288u; }  // scores
+__device__ __forceinline__ constexpr uint32_t col_p(int t) { return t ? 480u : 448u; }  // P codes, 32 columns
 
 // One V ring stage: [16 rows of 1.0][plane 0: V^T tile][16 rows of 1.0][plane 1].
 // Tile 0's PV reads plane 0 followed by the second band (ones last), tile 1's
@@ -101,7 +104,7 @@ struct __align__(1024) SmemAttn {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t m_full[2], m_empty[2];
-  uint64_t s_full[2], s_loaded[2], p_full[2], o_done[2], fin_ready[2], o_final[2];
+  uint64_t s_full[2], s_loaded[2], p_full[2], pv_done[2], fin_ready[2], o_final[2];
   uint64_t mma_drain;
   uint32_t tmem_base;
   int32_t abort_flag;
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.s_full[t], 1);
       mbar_init(&s.s_loaded[t], 4);
       mbar_init(&s.p_full[t], 128);
-      mbar_init(&s.o_done[t], 1);
+      mbar_init(&s.pv_done[t], 1);
       mbar_init(&s.fin_ready[t], 128);
       mbar_init(&s.o_final[t], 1);
     }
@@ -368,14 +371,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         commit(&s.k_empty[0]);
       }
     }
-    // Per block j, tile by tile: [mean batch], PV_t(j) as soon as P_t(j) is in
-    // tensor memory, then the scores of block j+1 (the QK product overwrites
-    // P_t(j) only after PV_t(j) has read it: MMAs of one thread run in order).
+    // Per block j: the scores of block j+1 for tile 0 as soon as tile 1 has
+    // loaded its block-j scores (shared columns), PV_0(j) when P_0(j) is in
+    // tensor memory, the block-(j+1) scores of tile 1 once tile 0 has loaded
+    // its own, then PV_1(j). Each tile's PV accumulates its own O and P regions.
     for (int j = 0; ok && j < nkv; ++j) {
       const int vs = j % kVStages;
       const uint32_t vb = smem_u32(&s.v[vs][0]);
       const int ks = (j + 1) % kKStages;
+      const bool more = j + 1 < nkv;
       for (int t = 0; t < 2 && ok; ++t) {
+        if (more) {
+          // S_t(j+1) overwrites the shared columns the other tile has just read
+          if (t == 0 && !(ok = wait_warp(s, &s.k_full[ks], ((j + 1) / kKStages) & 1, P))) break;
+          if (!(ok = wait_warp(s, &s.s_loaded[t ^ 1], (j + t) & 1, P))) break;
+          tc_fence_after();
+          qk(t, ks);
+          commit(&s.s_full[t]);
+          if (t == 1) commit(&s.k_empty[ks]);
+        }
         if (!(ok = wait_warp(s, &s.p_full[t], j & 1, P))) break;
         if (t == 0 && !(ok = wait_warp(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
         tc_fence_after();
@@ -393,18 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_f8f6f4_ts(tmem + col_ch(t), tmem + col_p(t) + 8 * kk, dv2 + 2 * kk, id_pv2, 1u);
           }
         }
+        commit(&s.pv_done[t]);
         if (t == 1) commit(&s.v_empty[vs]);
-        if (j + 1 < nkv) {
-          // the other tile's threads must have loaded the scores in the shared columns
-          if (t == 0 && !(ok = wait_warp(s, &s.k_full[ks], ((j + 1) / kKStages) & 1, P))) break;
-          if (!(ok = wait_warp(s, &s.s_loaded[t ^ 1], (j + t) & 1, P))) break;
-          tc_fence_after();
-          qk(t, ks);
-          commit(&s.s_full[t]);
-          if (t == 1) commit(&s.k_empty[ks]);
-        } else {
-          commit(&s.o_done[t]);
-        }
       }
     }
     // the last (possibly partial) batch of block means, then the output is final
@@ -444,11 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t sc[4][32];
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) tmem_ld32(s_addr + 32 * cc, sc[cc]);
-      // row-sum column after PV(j-1): s_full(j) follows QK(j), issued after PV(j-1)
-      const uint32_t lraw = j > 0 ? tmem_ld1(l_addr) : 0u;
       tmem_ld_wait();
       // this warp's scores are in registers: the other tile's QK may now overwrite
-      // the shared columns (and the P codes may overwrite S_t)
+      // the shared columns
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.s_loaded[t]);
@@ -493,6 +495,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         w[q4] = pack4_imad(fmaxf(a.x, kMagic), fmaxf(a.y, kMagic), fmaxf(b.x, kMagic), fmaxf(b.y, kMagic));
       }
 #undef SC
+      // PV(j-1) has read P_t and added block j-1 to O_t: then the row-sum column
+      // is read, O_t may be rescaled and P_t(j) written
+      uint32_t lraw = 0u;
+      if (j > 0) {
+        if (!(ok = wait_warp(s, &s.pv_done[t], (j - 1) & 1, P))) break;
+        tc_fence_after();
+        lraw = tmem_ld1(l_addr);
+        tmem_ld_wait();
+      }
       tmem_st32(p_addr, w);
       const float Lc = __uint_as_float(lraw);
       if (__any_sync(0xffffffffu, resc)) {
@@ -538,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!range_ok) report_status(P.status, VC_ERR_UNSUPPORTED);
     float l = 0.0f;
     // after the last PV: the total row sum, and the last block's share of it
-    if (ok) ok = wait_warp(s, &s.o_done[t], 0, P);
+    if (ok) ok = wait_warp(s, &s.pv_done[t], (nkv - 1) & 1, P);
     if (ok) {
       tc_fence_after();
       l = __uint_as_float(tmem_ld1(l_addr));
