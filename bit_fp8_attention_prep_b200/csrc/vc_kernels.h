@@ -30,10 +30,6 @@ struct PrepPlan {
   unsigned int* amax;          // [BH] fp32 bits
 };
 
-inline size_t assign_smem_bytes(int k, bool accum) {
-  return (size_t)k * 128 * 4 + (size_t)256 * 272 + (accum ? (size_t)k * 128 * 8 : 0) + kMaxClusters * 4 + 256;
-}
-
 cudaError_t prep_configure();
 // *nlaunch receives the number of kernels enqueued (memsets not counted).
 cudaError_t launch_prepare_v(const void* v, int dtype, const PrepPlan& plan, const vc_prepared_v_t& out,

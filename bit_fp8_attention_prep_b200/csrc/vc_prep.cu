@@ -62,28 +62,36 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(const T* __restrict__ 
 }
 
 // --------------------------------------------------------------- k-means assign
-// One CTA = one chunk of kChunk tokens of one (b, h), in tiles of kTile tokens.
-// A tile is staged in shared memory with coalesced 16-byte loads; each thread
-// then holds one token (128 fp32 in registers) and computes the squared fp32
-// distance to every centroid with packed f32x2 arithmetic; the nearest centroid
-// (lowest index on ties) is the assignment. When `accumulate` is set, the
-// tile's tokens are added to per-CTA int64 fixed-point sums (dimension-parallel:
-// lane l owns dimensions 4l..4l+3) that are flushed to global sums at the end.
-constexpr int kTile = 256;
-constexpr int kTileStride = 272;  // bytes per staged row (256 + 16: conflict-free 16-B reads)
+// One CTA (4 warps) = one chunk of kChunk tokens of one (b, h), in tiles of
+// kTile tokens staged in shared memory with coalesced 16-byte loads.
+//  - Assignment: thread t takes token t of the tile. Its squared fp32 distances
+//    to all centroids (at most KC) live in registers as packed f32x2 partial sums
+//    (even and odd dimensions) and grow 16 dimensions at a time, the centroids
+//    read from shared memory (all lanes read the same address). The nearest
+//    centroid, lowest index on ties, is the assignment.
+//  - Accumulation (kAccum): the tile's tokens are put in cluster order (a
+//    counting sort: match_any ranks within each warp, offsets across warps), then
+//    thread d walks them in that order adding llrint(x_d * 2^24) to an int64
+//    running sum and adds the sum into the CTA's accumulator of that cluster when
+//    the cluster changes. Thread d owns column d of the accumulators, so no
+//    atomics are needed until the chunk's sums go to global memory.
+constexpr int kTile = 128;
+constexpr int kTileStride = 272;  // bytes per staged row (256 + 16)
 
-template <typename T, bool kAccum>
+template <typename T, bool kAccum, int KC>
 __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restrict__ v, int S, int H, int k,
                                                               const float* __restrict__ cent,
                                                               unsigned long long* __restrict__ sums,
                                                               int* __restrict__ counts, uint8_t* __restrict__ assign,
                                                               int* __restrict__ hist, uint8_t* __restrict__ history) {
   extern __shared__ __align__(16) uint8_t smem[];
-  float* negc = reinterpret_cast<float*>(smem);                                   // [k][128]
-  uint8_t* tile = smem + (size_t)k * kD * 4;                                     // [kTile][272]
-  long long* ssum = reinterpret_cast<long long*>(tile + (size_t)kTile * kTileStride);  // [k][128]
-  int* scount = reinterpret_cast<int*>(ssum + (kAccum ? (size_t)k * kD : 0));        // [k]
-  uint8_t* tassign = reinterpret_cast<uint8_t*>(scount + kMaxClusters);              // [kTile]
+  long long* acc = reinterpret_cast<long long*>(smem);                                  // [KC][128] (kAccum)
+  float* negc = reinterpret_cast<float*>(smem + (kAccum ? (size_t)KC * kD * 8 : 0));    // [k][128]
+  uint8_t* tile = reinterpret_cast<uint8_t*>(negc + (size_t)KC * kD);                  // [kTile][272]
+  int* scount = reinterpret_cast<int*>(tile + (size_t)kTile * kTileStride);            // [KC]
+  int* woff = scount + KC;                                                             // [4][KC]
+  uint8_t* tassign = reinterpret_cast<uint8_t*>(woff + 4 * KC);                        // [kTile]
+  uint8_t* order = tassign + kTile;                                                     // [kTile]
 
   const int bh = blockIdx.y, b = bh / H, h = bh % H;
   const int chunk = blockIdx.x;
@@ -93,8 +101,8 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
 
   for (int i = tid; i < k * kD; i += kTile) negc[i] = -cent[(size_t)bh * k * kD + i];
   if (kAccum)
-    for (int i = tid; i < k * kD; i += kTile) ssum[i] = 0;
-  if (tid < kMaxClusters) scount[tid] = 0;
+    for (int i = tid; i < KC * kD; i += kTile) acc[i] = 0;
+  if (tid < KC) scount[tid] = 0;
 
   const int s_chunk0 = chunk * kChunk;
   const int s_chunk1 = min(S, s_chunk0 + kChunk);
@@ -110,39 +118,48 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
         *reinterpret_cast<uint4*>(tile + r * kTileStride + c * 16) = val;
       }
     }
+    if (kAccum && tid < 4 * KC) woff[tid] = 0;
     __syncthreads();
-    if (tid < ntok) {
-      float2 x[64];
+    const bool valid = tid < ntok;
+    int best = 0;
+    if (valid) {
+      float2 dist[KC];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        float f[8];
-        unpack8<T>(*reinterpret_cast<const uint4*>(tile + tid * kTileStride + c * 16), f);
-        x[4 * c + 0] = make_float2(f[0], f[1]);
-        x[4 * c + 1] = make_float2(f[2], f[3]);
-        x[4 * c + 2] = make_float2(f[4], f[5]);
-        x[4 * c + 3] = make_float2(f[6], f[7]);
+      for (int c = 0; c < KC; ++c) dist[c] = make_float2(0.f, 0.f);
+#pragma unroll 1
+      for (int ch = 0; ch < 8; ++ch) {  // dimensions 16 ch .. 16 ch + 15
+        float2 x[8];
+        {
+          float f[16];
+          unpack8<T>(*reinterpret_cast<const uint4*>(tile + tid * kTileStride + ch * 32), f);
+          unpack8<T>(*reinterpret_cast<const uint4*>(tile + tid * kTileStride + ch * 32 + 16), f + 8);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[i] = make_float2(f[2 * i], f[2 * i + 1]);
+        }
+#pragma unroll
+        for (int c = 0; c < KC; ++c) {
+          if (c < k) {
+            const float4* nc = reinterpret_cast<const float4*>(negc + c * kD + ch * 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float4 p = nc[i];
+              const float2 d0 = __fadd2_rn(x[2 * i + 0], make_float2(p.x, p.y));
+              const float2 d1 = __fadd2_rn(x[2 * i + 1], make_float2(p.z, p.w));
+              dist[c] = __ffma2_rn(d0, d0, dist[c]);
+              dist[c] = __ffma2_rn(d1, d1, dist[c]);
+            }
+          }
+        }
       }
       float best_d = 0.0f;
-      int best = 0;
-      for (int c = 0; c < k; ++c) {
-        const float4* nc = reinterpret_cast<const float4*>(negc + c * kD);
-        float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float4 p = nc[i], q = nc[i + 1];
-          const float2 d0 = __fadd2_rn(x[2 * i + 0], make_float2(p.x, p.y));
-          const float2 d1 = __fadd2_rn(x[2 * i + 1], make_float2(p.z, p.w));
-          const float2 d2 = __fadd2_rn(x[2 * i + 2], make_float2(q.x, q.y));
-          const float2 d3 = __fadd2_rn(x[2 * i + 3], make_float2(q.z, q.w));
-          a0 = __ffma2_rn(d0, d0, a0);
-          a1 = __ffma2_rn(d1, d1, a1);
-          a2 = __ffma2_rn(d2, d2, a2);
-          a3 = __ffma2_rn(d3, d3, a3);
-        }
-        const float dist = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
-        if (c == 0 || dist < best_d) {
-          best_d = dist;
-          best = c;
+      for (int c = 0; c < KC; ++c) {
+        if (c < k) {
+          const float dd = dist[c].x + dist[c].y;
+          if (c == 0 || dd < best_d) {
+            best_d = dd;
+            best = c;
+          }
         }
       }
       tassign[tid] = (uint8_t)best;
@@ -151,28 +168,83 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
       atomicAdd(&scount[best], 1);
     }
     if (kAccum) {
+      // counting sort of the tile by cluster (stable is not needed for a sum)
+      const int a = valid ? best : 0xFF;
+      const unsigned peers = __match_any_sync(0xffffffffu, a);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      if (valid && rank == 0) woff[warp * KC + a] = __popc(peers);
       __syncthreads();
-      for (int r = warp; r < ntok; r += kTile / 32) {
-        const int c = tassign[r];
-        float f[4];
-        unpack4<T>(*reinterpret_cast<const uint2*>(tile + r * kTileStride + lane * 8), f);
+      if (tid < 32) {
+        int tot = 0, w0 = 0, w1 = 0, w2 = 0, w3 = 0;
+        if (tid < KC) {
+          w0 = woff[0 * KC + tid]; w1 = woff[1 * KC + tid]; w2 = woff[2 * KC + tid]; w3 = woff[3 * KC + tid];
+          tot = w0 + w1 + w2 + w3;
+        }
+        int incl = tot;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const long long q = __float2ll_rn(f[e] * 16777216.0f);  // x * 2^24, exact
-          if (q != 0) atomicAdd(reinterpret_cast<unsigned long long*>(&ssum[c * kD + lane * 4 + e]),
-                                (unsigned long long)q);
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t2 = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += t2;
+        }
+        if (tid < KC) {
+          const int base = incl - tot;
+          woff[0 * KC + tid] = base;
+          woff[1 * KC + tid] = base + w0;
+          woff[2 * KC + tid] = base + w0 + w1;
+          woff[3 * KC + tid] = base + w0 + w1 + w2;
         }
       }
+      __syncthreads();
+      if (valid) order[woff[warp * KC + best] + rank] = (uint8_t)tid;
+      __syncthreads();
+      // thread d: column d of the tile in cluster order
+      const int d = tid;
+      int cur = -1;
+      long long run = 0;
+      for (int pos = 0; pos < ntok; ++pos) {
+        const int tok = order[pos];
+        const int c = tassign[tok];
+        if (c != cur) {
+          if (cur >= 0) acc[cur * kD + d] += run;
+          cur = c;
+          run = 0;
+        }
+        const float f = to_f32<T>(*reinterpret_cast<const T*>(tile + tok * kTileStride + d * 2));
+        run += __float2ll_rn(f * 16777216.0f);  // x * 2^24, exact
+      }
+      if (cur >= 0) acc[cur * kD + d] += run;
     }
   }
   __syncthreads();
   if (kAccum) {
     for (int i = tid; i < k * kD; i += kTile)
-      if (ssum[i] != 0) atomicAdd(&sums[(size_t)bh * k * kD + i], (unsigned long long)ssum[i]);
+      if (acc[i] != 0) atomicAdd(&sums[(size_t)bh * k * kD + i], (unsigned long long)acc[i]);
     if (tid < k && scount[tid] != 0) atomicAdd(&counts[(size_t)bh * k + tid], scount[tid]);
   } else if (hist != nullptr && tid < k) {
     hist[((size_t)bh * gridDim.x + chunk) * k + tid] = scount[tid];
   }
+}
+
+template <int KC>
+constexpr size_t assign_smem(bool accum) {
+  return (accum ? (size_t)KC * kD * 8 : 0) + (size_t)KC * kD * 4 + (size_t)kTile * kTileStride + 5 * KC * 4 +
+         2 * kTile;
+}
+
+template <typename T, bool kAccum, int KC>
+static void launch_assign(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, uint8_t* hist_t) {
+  kmeans_assign_kernel<T, kAccum, KC><<<grid, kTile, assign_smem<KC>(kAccum), st>>>(
+      v, pl.S, pl.H, pl.k, pl.cent, pl.sums, pl.counts, pl.assign, kAccum ? nullptr : pl.hist, hist_t);
+}
+
+template <typename T, bool kAccum>
+static void launch_assign_k(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, uint8_t* hist_t) {
+  if (pl.k <= 8)
+    launch_assign<T, kAccum, 8>(grid, st, v, pl, hist_t);
+  else if (pl.k <= 16)
+    launch_assign<T, kAccum, 16>(grid, st, v, pl, hist_t);
+  else
+    launch_assign<T, kAccum, 32>(grid, st, v, pl, hist_t);
 }
 
 // --------------------------------------------------------------- centroid update
@@ -312,50 +384,64 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ 
 }
 
 // --------------------------------------------------------------- residual E4M3
-// One CTA = one 128-token block; thread r owns permuted row r. Codes go to a
-// transposed shared tile and leave as V^T rows (128 contiguous tokens per
-// channel), the K-major B operand of the PV product.
+// One CTA (8 warps) = one 128-token block of permuted positions. Loads as in
+// quant_qk_kernel (two gathered 256-byte rows per warp instruction); each lane
+// keeps the same 8 channels, so it subtracts 8 block means held in registers.
+// The codes go to a shared tile [token][channel] (136-byte rows: the two half
+// warps' 8-byte stores fall on disjoint banks) and leave transposed, as V^T rows
+// of 128 tokens per channel (the K-major B operand of the PV product): a lane
+// gathers the codes of one channel for 4 consecutive tokens (8 lanes read the
+// same words, so the reads are conflict-free) and stores them as one word.
+constexpr int kResStride = 136;
+
 template <typename T>
-__global__ void __launch_bounds__(128) residual_e4m3_kernel(const T* __restrict__ v, int S, int H, int S_pad,
+__global__ void __launch_bounds__(256) residual_e4m3_kernel(const T* __restrict__ v, int S, int H, int S_pad,
                                                             const int32_t* __restrict__ perm,
                                                             const float* __restrict__ mu,
                                                             const unsigned int* __restrict__ amax_bits,
                                                             uint8_t* __restrict__ vt, float* __restrict__ s_v) {
-  __shared__ __align__(16) uint8_t ct[kD][kBlock + 16];
-  __shared__ float smu[kD];
+  __shared__ __align__(16) uint8_t ct[kBlock * kResStride];
   const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
-  const int r = threadIdx.x;
-  const int p = blk * kBlock + r;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int half = lane >> 4, c = lane & 15;
   const float amax = __uint_as_float(amax_bits[bh]);
   const bool zero = !(amax >= kTinyAmax);
   const float inv = zero ? 0.0f : __fdiv_rn(kE4M3Max, amax);
-  if (blk == 0 && r == 0) s_v[bh] = zero ? 1.0f : __fdiv_rn(amax, kE4M3Max);
-  smu[r] = mu[((size_t)bh * gridDim.x + blk) * kD + r];
-  __syncthreads();
-  if (p < S && !zero) {
-    const T* row = v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD;
-#pragma unroll 4
-    for (int c = 0; c < 16; ++c) {
-      float f[8];
-      unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), f);
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const int d = c * 8 + e;
-        const float r0 = __fsub_rn(f[e], smu[d]), r1 = __fsub_rn(f[e + 1], smu[d + 1]);
-        const uint16_t two = cvt_e4m3x2(__fmul_rn(r0, inv), __fmul_rn(r1, inv));
-        ct[d][r] = (uint8_t)(two & 0xFF);
-        ct[d + 1][r] = (uint8_t)(two >> 8);
-      }
-    }
-  } else {
-    for (int d = 0; d < kD; ++d) ct[d][r] = 0;
+  if (blk == 0 && threadIdx.x == 0) s_v[bh] = zero ? 1.0f : __fdiv_rn(amax, kE4M3Max);
+  float m8[8];
+  {
+    const float4* mp = reinterpret_cast<const float4*>(mu + ((size_t)bh * gridDim.x + blk) * kD + c * 8);
+    const float4 m0 = mp[0], m1 = mp[1];
+    m8[0] = m0.x; m8[1] = m0.y; m8[2] = m0.z; m8[3] = m0.w;
+    m8[4] = m1.x; m8[5] = m1.y; m8[6] = m1.z; m8[7] = m1.w;
   }
-  __syncthreads();
-  uint8_t* out = vt + (size_t)bh * kD * S_pad + (size_t)blk * kBlock;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int idx = i * 128 + r, d = idx >> 3, c = idx & 7;
-    *reinterpret_cast<uint4*>(out + (size_t)d * S_pad + c * 16) = *reinterpret_cast<const uint4*>(&ct[d][c * 16]);
+    const int r = warp * 16 + 2 * i + half;
+    const int p = blk * kBlock + r;
+    uint2 w = make_uint2(0u, 0u);
+    if (p < S && !zero) {
+      const uint4 x = *reinterpret_cast<const uint4*>(v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD + c * 8);
+      float f[8];
+      unpack8<T>(x, f);
+      float rr[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) rr[e] = __fmul_rn(__fsub_rn(f[e], m8[e]), inv);
+      w.x = (uint32_t)cvt_e4m3x2(rr[0], rr[1]) | ((uint32_t)cvt_e4m3x2(rr[2], rr[3]) << 16);
+      w.y = (uint32_t)cvt_e4m3x2(rr[4], rr[5]) | ((uint32_t)cvt_e4m3x2(rr[6], rr[7]) << 16);
+    }
+    *reinterpret_cast<uint2*>(ct + r * kResStride + c * 8) = w;
+  }
+  __syncthreads();
+  uint8_t* const out = vt + (size_t)bh * kD * S_pad + (size_t)blk * kBlock;
+  const int m = lane & 7, q = lane >> 3;
+#pragma unroll 4
+  for (int it = 0; it < 16; ++it) {
+    const int pidx = warp * 16 + it, cg = pidx & 15, qg = pidx >> 4;
+    const int d = cg * 8 + m, t0 = qg * 16 + q * 4;
+    const uint32_t b0 = ct[(t0 + 0) * kResStride + d], b1 = ct[(t0 + 1) * kResStride + d];
+    const uint32_t b2 = ct[(t0 + 2) * kResStride + d], b3 = ct[(t0 + 3) * kResStride + d];
+    *reinterpret_cast<uint32_t*>(out + (size_t)d * S_pad + t0) = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
   }
 }
 
@@ -421,56 +507,62 @@ __global__ void __launch_bounds__(128) residual_nvfp4_kernel(const T* __restrict
 }
 
 // --------------------------------------------------------------- Q/K quantisation
-// One CTA = one 128-row block of Q (original order) or K (gathered by perm);
-// thread r owns row r: load 128 values, block amax (warp max + shared), then
-// E4M3 codes of x * (448/amax), 128 contiguous bytes per row.
+// One CTA (8 warps) = one 128-row block of Q (original order) or K (gathered by
+// perm). Warp w takes rows 16w .. 16w+15, two rows per load: lanes 0-15 read row
+// 2i and lanes 16-31 row 2i+1, 16 bytes each, so every load instruction reads two
+// whole 256-byte rows. The values stay in registers while the block amax is
+// reduced (warp shuffles, then shared memory); each lane then writes the 8 E4M3
+// codes of its 8 values (rows of 128 codes, contiguous per half warp).
 template <typename T>
-__global__ void __launch_bounds__(128) quant_qk_kernel(const T* __restrict__ q, const T* __restrict__ k, int S,
+__global__ void __launch_bounds__(256) quant_qk_kernel(const T* __restrict__ q, const T* __restrict__ k, int S,
                                                        int H, int S_pad, const int32_t* __restrict__ perm,
                                                        uint8_t* __restrict__ qc, float* __restrict__ qs,
                                                        uint8_t* __restrict__ kc, float* __restrict__ ks) {
-  __shared__ float wmax[4];
+  __shared__ float wmax[8];
   const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
   const bool is_k = blockIdx.z == 1;
-  const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
-  const int p = blk * kBlock + r;
-  const bool valid = p < S;
-  const int nbk = gridDim.x;
-  float x[kD];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int half = lane >> 4, c = lane & 15;  // row parity and 16-byte piece of the row
+  const T* const src = is_k ? k : q;
+  uint4 x[8];
   float mx = 0.0f;
-  if (valid) {
-    const int src = is_k ? perm[(size_t)bh * S + p] : p;
-    const T* row = (is_k ? k : q) + (((size_t)b * S + src) * H + h) * kD;
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), x + c * 8);
+  for (int i = 0; i < 8; ++i) {
+    const int p = blk * kBlock + warp * 16 + 2 * i + half;
+    x[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (p < S) {
+      const int row = is_k ? perm[(size_t)bh * S + p] : p;
+      x[i] = *reinterpret_cast<const uint4*>(src + (((size_t)b * S + row) * H + h) * kD + c * 8);
+      float f[8];
+      unpack8<T>(x[i], f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(x[c * 8 + e]));
+      for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
     }
   }
   mx = warp_max(mx);
   if (lane == 0) wmax[warp] = mx;
   __syncthreads();
-  const float amax = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+  float amax = wmax[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, wmax[w]);
   const bool zero = !(amax >= kTinyAmax);
   const float inv = zero ? 0.0f : __fdiv_rn(kE4M3Max, amax);
-  if (r == 0) (is_k ? ks : qs)[(size_t)bh * nbk + blk] = zero ? 1.0f : __fdiv_rn(amax, kE4M3Max);
-  uint8_t* out = (is_k ? kc : qc) + ((size_t)bh * S_pad + p) * kD;
+  const int nbk = gridDim.x;
+  if (threadIdx.x == 0) (is_k ? ks : qs)[(size_t)bh * nbk + blk] = zero ? 1.0f : __fdiv_rn(amax, kE4M3Max);
+  uint8_t* const out = (is_k ? kc : qc) + ((size_t)bh * S_pad + (size_t)blk * kBlock) * kD;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint32_t w[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = c * 16 + j * 4;
-      if (valid && !zero) {
-        const uint32_t lo = cvt_e4m3x2(__fmul_rn(x[e], inv), __fmul_rn(x[e + 1], inv));
-        const uint32_t hi = cvt_e4m3x2(__fmul_rn(x[e + 2], inv), __fmul_rn(x[e + 3], inv));
-        w[j] = lo | (hi << 16);
-      } else {
-        w[j] = 0u;
-      }
+  for (int i = 0; i < 8; ++i) {
+    const int r = warp * 16 + 2 * i + half;
+    uint2 w = make_uint2(0u, 0u);
+    if (!zero) {  // rows past S hold zeros, which code to 0
+      float f[8];
+      unpack8<T>(x[i], f);
+      w.x = (uint32_t)cvt_e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv)) |
+            ((uint32_t)cvt_e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv)) << 16);
+      w.y = (uint32_t)cvt_e4m3x2(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv)) |
+            ((uint32_t)cvt_e4m3x2(__fmul_rn(f[6], inv), __fmul_rn(f[7], inv)) << 16);
     }
-    *reinterpret_cast<uint4*>(out + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint2*>(out + (size_t)r * kD + c * 8) = w;
   }
 }
 
@@ -549,17 +641,14 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
     kmeans_init_kernel<T><<<BH, 128, 0, st>>>(v, S, H, k, pl.seed, pl.cent);
     ++n;
     const dim3 grid(pl.nchunks, BH);
-    const size_t sm_acc = assign_smem_bytes(k, true), sm_fin = assign_smem_bytes(k, false);
     for (int it = 0; it < pl.iters; ++it) {
       uint8_t* hist_t = history ? history + (size_t)it * BH * S : nullptr;
       if (it + 1 < pl.iters) {
-        kmeans_assign_kernel<T, true><<<grid, kTile, sm_acc, st>>>(v, S, H, k, pl.cent, pl.sums, pl.counts,
-                                                                   pl.assign, nullptr, hist_t);
+        launch_assign_k<T, true>(grid, st, v, pl, hist_t);
         kmeans_update_kernel<<<BH, 128, 0, st>>>(k, pl.cent, pl.sums, pl.counts);
         n += 2;
       } else {
-        kmeans_assign_kernel<T, false><<<grid, kTile, sm_fin, st>>>(v, S, H, k, pl.cent, pl.sums, pl.counts,
-                                                                    pl.assign, pl.hist, hist_t);
+        launch_assign_k<T, false>(grid, st, v, pl, hist_t);
         ++n;
       }
     }
@@ -573,7 +662,7 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
   const dim3 gb(pl.nb, BH);
   block_stats_kernel<T><<<gb, 128, 0, st>>>(v, S, H, out.perm, out.mu, pl.amax);
   if (pl.fmt == VC_RESIDUAL_E4M3) {
-    residual_e4m3_kernel<T><<<gb, 128, 0, st>>>(v, S, H, pl.S_pad, out.perm, out.mu, pl.amax, out.v_codes,
+    residual_e4m3_kernel<T><<<gb, 256, 0, st>>>(v, S, H, pl.S_pad, out.perm, out.mu, pl.amax, out.v_codes,
                                                 out.s_v);
   } else {
     residual_nvfp4_kernel<T><<<gb, 128, kD * 129 * sizeof(float), st>>>(v, S, H, pl.S_pad, out.perm, out.mu,
@@ -596,11 +685,11 @@ cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int 
   const int nb = (S + kBlock - 1) / kBlock;
   const dim3 grid(nb, B * H, 2);
   if (dtype == VC_DTYPE_BF16)
-    quant_qk_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+    quant_qk_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), S, H, nb * kBlock, perm,
         out.q_codes, out.q_scales, out.k_codes, out.k_scales);
   else
-    quant_qk_kernel<__half><<<grid, 128, 0, st>>>(static_cast<const __half*>(q), static_cast<const __half*>(k), S,
+    quant_qk_kernel<__half><<<grid, 256, 0, st>>>(static_cast<const __half*>(q), static_cast<const __half*>(k), S,
                                                   H, nb * kBlock, perm, out.q_codes, out.q_scales, out.k_codes,
                                                   out.k_scales);
   return cudaGetLastError();
@@ -608,11 +697,26 @@ cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int 
 
 cudaError_t prep_configure() {
   cudaError_t e;
-  const size_t mx = assign_smem_bytes(kMaxClusters, true);
-  for (auto f : {(const void*)kmeans_assign_kernel<__nv_bfloat16, true>,
-                 (const void*)kmeans_assign_kernel<__nv_bfloat16, false>,
-                 (const void*)kmeans_assign_kernel<__half, true>, (const void*)kmeans_assign_kernel<__half, false>})
-    if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mx)) != cudaSuccess) return e;
+  const struct {
+    const void* f;
+    size_t bytes;
+  } assign_fns[] = {
+      {(const void*)kmeans_assign_kernel<__nv_bfloat16, true, 8>, assign_smem<8>(true)},
+      {(const void*)kmeans_assign_kernel<__nv_bfloat16, true, 16>, assign_smem<16>(true)},
+      {(const void*)kmeans_assign_kernel<__nv_bfloat16, true, 32>, assign_smem<32>(true)},
+      {(const void*)kmeans_assign_kernel<__nv_bfloat16, false, 8>, assign_smem<8>(false)},
+      {(const void*)kmeans_assign_kernel<__nv_bfloat16, false, 16>, assign_smem<16>(false)},
+      {(const void*)kmeans_assign_kernel<__nv_bfloat16, false, 32>, assign_smem<32>(false)},
+      {(const void*)kmeans_assign_kernel<__half, true, 8>, assign_smem<8>(true)},
+      {(const void*)kmeans_assign_kernel<__half, true, 16>, assign_smem<16>(true)},
+      {(const void*)kmeans_assign_kernel<__half, true, 32>, assign_smem<32>(true)},
+      {(const void*)kmeans_assign_kernel<__half, false, 8>, assign_smem<8>(false)},
+      {(const void*)kmeans_assign_kernel<__half, false, 16>, assign_smem<16>(false)},
+      {(const void*)kmeans_assign_kernel<__half, false, 32>, assign_smem<32>(false)},
+  };
+  for (const auto& a : assign_fns)
+    if ((e = cudaFuncSetAttribute(a.f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)a.bytes)) != cudaSuccess)
+      return e;
   for (auto f : {(const void*)residual_nvfp4_kernel<__nv_bfloat16>, (const void*)residual_nvfp4_kernel<__half>})
     if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kD * 129 * 4))) !=
         cudaSuccess)
