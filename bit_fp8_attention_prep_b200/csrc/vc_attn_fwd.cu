@@ -17,7 +17,10 @@
 //   warps 4-7   softmax of query tile 1
 //   warp  8     TMA: both Q tiles once; K_j and V^T_j into rings; it also
 //               writes the bf16 block-mean operand of the mean MMA
-//   warp  9     MMA issuer (one elected lane)
+//   warp  9     issues the QK products of both tiles (one elected lane)
+//   warps 10-11 issue the PV (and mean) products of tile 0 and tile 1
+// The three issuing warps are independent streams into the tensor pipe, so an
+// MMA whose inputs are ready never waits behind another stream's barrier.
 // Tensor memory (512 columns):
 //   O_0 [0, 144)    tile 0: output channels 0-127, then 16 row-sum columns
 //   O_1 [144, 288)  tile 1: 16 row-sum columns, then output channels 0-127
@@ -68,8 +71,8 @@ template <int kPlanes> struct Stages {
 constexpr uint32_t kTileBytes = 128 * 128;  // one 128 x 128 E4M3 tile (or 128 x 64 bf16)
 constexpr uint32_t kOnesBytes = 16 * 128;   // 16 rows of E4M3 1.0 (K = 128 keys)
 constexpr uint32_t kMopBytes = 128 * 16 * 2;  // M operand of one batch: 128 channels x 16 bf16
-constexpr int kThreads = 320;
-constexpr int kTmaWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 384;
+constexpr int kTmaWarp = 8, kQkWarp = 9, kPvWarp0 = 10;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMeanBlocks = 5;              // key blocks per mean MMA (3 K slots each: 15 of 16)
 constexpr int kMeanChunks = 2;              // R: 16-slot K chunks 0 and 1, alternating by batch
@@ -105,7 +108,7 @@ struct __align__(1024) SmemAttn {
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t m_full[2], m_empty[2];
   uint64_t s_full[2], s_loaded[2], p_full[2], pv_done[2], fin_ready[2], o_final[2];
-  uint64_t mma_drain;
+  uint64_t mma_drain[3];
   uint32_t tmem_base;
   int32_t abort_flag;
 };
@@ -195,11 +198,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kVStages; ++i) {
       mbar_init(&s.v_full[i], 1);
-      mbar_init(&s.v_empty[i], 1);
+      mbar_init(&s.v_empty[i], 2);   // PV_0(j) and PV_1(j) both read V_j
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s.m_full[t], 1);
-      mbar_init(&s.m_empty[t], 1);
+      mbar_init(&s.m_empty[t], 2);   // both tiles' mean MMAs read it
       mbar_init(&s.s_full[t], 1);
       mbar_init(&s.s_loaded[t], 4);
       mbar_init(&s.p_full[t], 128);
@@ -207,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.fin_ready[t], 128);
       mbar_init(&s.o_final[t], 1);
     }
-    mbar_init(&s.mma_drain, 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&s.mma_drain[i], 1);
     s.abort_flag = 0;
     fence_barrier_init();
   }
@@ -321,80 +324,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&s.k_full[j % kKStages], (j / kKStages) & 1, drain_ns, nullptr);
     for (int j = max(0, v_issued - kVStages); j < v_issued; ++j)
       mbar_wait(&s.v_full[j % kVStages], (j / kVStages) & 1, drain_ns, nullptr);
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    // The whole warp runs the loop so that descriptors and addresses stay
-    // warp-uniform (uniform registers feed tcgen05.mma directly); one elected
-    // lane issues the MMAs and the commits that track them.
+  } else if (warp >= kQkWarp) {
+    // ------------------------------------------------------------ MMA issuers
+    // Each issuing warp runs its loop warp-wide so that descriptors and
+    // addresses stay warp-uniform (uniform registers feed tcgen05.mma directly);
+    // one elected lane issues the MMAs and the commits that track them.
     const bool leader = elect_one();
-    constexpr uint32_t id_qk = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
-    constexpr uint32_t id_pv = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 144);
-    constexpr uint32_t id_pv2 = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
-    constexpr uint32_t id_mean = idesc_f32acc(kFmtBF16, kFmtBF16, 128, 128);
-    const uint64_t dq[2] = {sdesc_k_sw128(smem_u32(s.q[0])), sdesc_k_sw128(smem_u32(s.q[1]))};
-    const uint64_t dr[2] = {sdesc_k_sw128(smem_u32(s.rop[0])), sdesc_k_sw128(smem_u32(s.rop[1]))};
-    const uint64_t dmo[2] = {sdesc_k_noswz(smem_u32(s.mop[0]), kMopLbo, kMopSbo),
-                             sdesc_k_noswz(smem_u32(s.mop[1]), kMopLbo, kMopSbo)};
-    auto qk = [&](int t, int ks) {  // S_t = Q_t K^T
-      const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[ks]));
-      if (leader) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(tmem + col_s(t), dq[t] + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
-      }
-    };
     auto commit = [&](uint64_t* bar) {
       if (leader) umma_commit(bar);
     };
-    // O_t += R_t M of one batch of blocks; tile 0 first waits for the M operand,
-    // tile 1 releases it
-    auto mean = [&](int t, int batch) -> bool {
-      const int mb = batch & 1;
-      if (t == 0) {
+    bool ok = true;
+    if (warp == kQkWarp) {
+      constexpr uint32_t id_qk = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
+      const uint64_t dq[2] = {sdesc_k_sw128(smem_u32(s.q[0])), sdesc_k_sw128(smem_u32(s.q[1]))};
+      auto qk = [&](int t, int ks) {  // S_t = Q_t K^T
+        const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[ks]));
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(tmem + col_s(t), dq[t] + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
+        }
+      };
+      // The QK products alternate between the tiles through the shared score
+      // columns: S_1(j) once tile 0 has loaded S_0(j), S_0(j+1) once tile 1 has
+      // loaded S_1(j).
+      ok = wait_warp(s, &s.q_full, 0, P);
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int ks = j % kKStages;
+        if (!(ok = wait_warp(s, &s.k_full[ks], (j / kKStages) & 1, P))) break;
+        if (j > 0 && !(ok = wait_warp(s, &s.s_loaded[1], (j - 1) & 1, P))) break;
+        tc_fence_after();
+        qk(0, ks);
+        commit(&s.s_full[0]);
+        if (!(ok = wait_warp(s, &s.s_loaded[0], j & 1, P))) break;
+        tc_fence_after();
+        qk(1, ks);
+        commit(&s.s_full[1]);
+        commit(&s.k_empty[ks]);
+      }
+      commit(&s.mma_drain[0]);
+      mbar_wait(&s.mma_drain[0], 0, 100000000ull, nullptr);
+    } else {
+      const int t = warp - kPvWarp0;
+      constexpr uint32_t id_pv = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 144);
+      constexpr uint32_t id_pv2 = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, 128);
+      constexpr uint32_t id_mean = idesc_f32acc(kFmtBF16, kFmtBF16, 128, 128);
+      const uint64_t dr = sdesc_k_sw128(smem_u32(s.rop[t]));
+      // O_t += R_t M of one batch of blocks (both tiles read the same M tile)
+      auto mean = [&](int batch) -> bool {
+        const int mb = batch & 1;
         if (!wait_warp(s, &s.m_full[mb], (batch >> 1) & 1, P)) return false;
         tc_fence_after();
-      }
-      if (leader) umma_f16_ss(tmem + col_ch(t), dr[t] + 2 * (batch % kMeanChunks), dmo[mb], id_mean, 1u);
-      if (t == 1) commit(&s.m_empty[mb]);
-      return true;
-    };
-    bool ok = wait_warp(s, &s.q_full, 0, P) && wait_warp(s, &s.k_full[0], 0, P);
-    if (ok) {
-      tc_fence_after();
-      qk(0, 0);
-      commit(&s.s_full[0]);
-      // S_1 shares columns with S_0: start it once tile 0's threads have loaded their scores
-      ok = wait_warp(s, &s.s_loaded[0], 0, P);
-      if (ok) {
-        tc_fence_after();
-        qk(1, 0);
-        commit(&s.s_full[1]);
-        commit(&s.k_empty[0]);
-      }
-    }
-    // Per block j: the scores of block j+1 for tile 0 as soon as tile 1 has
-    // loaded its block-j scores (shared columns), PV_0(j) when P_0(j) is in
-    // tensor memory, the block-(j+1) scores of tile 1 once tile 0 has loaded
-    // its own, then PV_1(j). Each tile's PV accumulates its own O and P regions.
-    for (int j = 0; ok && j < nkv; ++j) {
-      const int vs = j % kVStages;
-      const uint32_t vb = smem_u32(&s.v[vs][0]);
-      const int ks = (j + 1) % kKStages;
-      const bool more = j + 1 < nkv;
-      for (int t = 0; t < 2 && ok; ++t) {
-        if (more) {
-          // S_t(j+1) overwrites the shared columns the other tile has just read
-          if (t == 0 && !(ok = wait_warp(s, &s.k_full[ks], ((j + 1) / kKStages) & 1, P))) break;
-          if (!(ok = wait_warp(s, &s.s_loaded[t ^ 1], (j + t) & 1, P))) break;
-          tc_fence_after();
-          qk(t, ks);
-          commit(&s.s_full[t]);
-          if (t == 1) commit(&s.k_empty[ks]);
-        }
+        const uint64_t dmo = sdesc_k_noswz(smem_u32(s.mop[mb]), kMopLbo, kMopSbo);
+        if (leader) umma_f16_ss(tmem + col_ch(t), dr + 2 * (batch % kMeanChunks), dmo, id_mean, 1u);
+        commit(&s.m_empty[mb]);
+        return true;
+      };
+      // Per block j: [mean batch], then O_t (+ row sums) += P_t(j) [V_j ; 1]
+      // (tile 1: [1 ; V_j]) as soon as P_t(j) is in tensor memory.
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int vs = j % kVStages;
         if (!(ok = wait_warp(s, &s.p_full[t], j & 1, P))) break;
-        if (t == 0 && !(ok = wait_warp(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
+        if (!(ok = wait_warp(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
         tc_fence_after();
-        if (j >= kMeanBlocks && j % kMeanBlocks == 0 && !(ok = mean(t, j / kMeanBlocks - 1))) break;
-        // O_t (+ row sums) += P_t [V ; 1]  (tile 1: [1 ; V])
+        if (j >= kMeanBlocks && j % kMeanBlocks == 0 && !(ok = mean(j / kMeanBlocks - 1))) break;
+        const uint32_t vb = smem_u32(&s.v[vs][0]);
         const uint64_t dv = sdesc_k_sw128(vb + (t == 0 ? VS::kPlane0 : 0u));
         if (leader) {
 #pragma unroll
@@ -408,19 +401,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         commit(&s.pv_done[t]);
-        if (t == 1) commit(&s.v_empty[vs]);
+        commit(&s.v_empty[vs]);
       }
+      // the last (possibly partial) batch of block means, then the output is final
+      if (ok) ok = wait_warp(s, &s.fin_ready[t], 0, P);
+      if (ok) {
+        tc_fence_after();
+        ok = mean(nbatch - 1);
+      }
+      if (ok) commit(&s.o_final[t]);
+      // every MMA this warp issued has completed before TMEM is released
+      commit(&s.mma_drain[1 + t]);
+      mbar_wait(&s.mma_drain[1 + t], 0, 100000000ull, nullptr);
     }
-    // the last (possibly partial) batch of block means, then the output is final
-    for (int t = 0; t < 2 && ok; ++t) {
-      if (!(ok = wait_warp(s, &s.fin_ready[t], 0, P))) break;
-      tc_fence_after();
-      if (!(ok = mean(t, nbatch - 1))) break;
-      commit(&s.o_final[t]);
-    }
-    // every MMA the leader issued has completed before TMEM is released
-    commit(&s.mma_drain);
-    mbar_wait(&s.mma_drain, 0, 100000000ull, nullptr);
   } else {
     // ------------------------------------------------------------ softmax / epilogue
     const int t = warp >> 2;               // query tile

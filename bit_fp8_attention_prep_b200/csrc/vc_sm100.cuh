@@ -284,6 +284,11 @@ __device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// As tmem_ld_wait, for a value loaded earlier with work in between: passing the
+// register through the wait keeps the compiler from using it before the wait.
+__device__ __forceinline__ void tmem_ld_wait_for(uint32_t& r) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r) : : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 }  // namespace vc
