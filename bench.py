@@ -40,7 +40,7 @@ ATTN_KERNEL = {"e4m3": "vc_attn_fwd_kernel<1>", "nvfp4": "vc_attn_fwd_kernel<2>"
 # DRAM bytes (read + write) of one attention launch on the default workload, from
 # the ncu capture summarised in profiles/; valid only while the kernel source
 # hashes to the recorded value (otherwise traffic is reported as null).
-ATTN_TRAFFIC = {"sha256_16": "c84b739e2406d674", "bytes_per_launch": 8 * (207.309568e6 + 109.4784e6)}
+ATTN_TRAFFIC = {"sha256_16": "f409156f5d305706", "bytes_per_launch": 8 * (201.432064e6 + 102.87744e6)}
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 FALLBACK_HBM_GBS = 6650.0
 
@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--k-p", type=int, default=8)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the SDPA comparison, accuracy, e2e and CPU-baseline legs")
+    ap.add_argument("--extras", default="all",
+                    help="comma-separated extra legs after the timed region: accuracy, exp2, sdpa, e2e, cpu "
+                         "(default all; --no-extras = none)")
     return ap.parse_args()
 
 
@@ -302,8 +305,10 @@ def run_ours(args, cfg):
         "device_status": status,
         "clocks": clk,
     }
-    if not args.no_extras:
-        line.update(extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_step, rank))
+    legs = set() if args.no_extras else (
+        {"accuracy", "exp2", "sdpa", "e2e", "cpu"} if args.extras == "all" else set(args.extras.split(",")))
+    if legs:
+        line.update(extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_step, rank, legs))
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -311,7 +316,7 @@ def run_ours(args, cfg):
         print(json.dumps(line), flush=True)
 
 
-def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_step, rank):
+def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_step, rank, legs):
     import torch
     import torch.nn.functional as F
     from torch.nn.attention import SDPBackend, sdpa_kernel
@@ -329,10 +334,45 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
         num += float(((o[0, rows, h].double() - ref) ** 2).sum())
         den += float((ref ** 2).sum())
         del k, v, p
-    out["rel_l2_vs_fp64"] = math.sqrt(num / den)
-    out["accuracy_sample"] = "64 query rows x heads {0, H-1} of batch 0, exact fp64 softmax attention on the GPU"
+    if "accuracy" in legs:
+        out["rel_l2_vs_fp64"] = math.sqrt(num / den)
+        out["accuracy_sample"] = "64 query rows x heads {0, H-1} of batch 0, exact fp64 softmax attention on the GPU"
+    # the comparison kernel: the same fused attention with the probabilities made
+    # by exp2 on the special function unit and an E4M3 conversion instead of
+    # ExpCast (same prepared inputs, same stream)
+    if cfg["fmt"] == "e4m3" and "exp2" in legs:
+        from bit_fp8_attention_prep_b200 import vc_attn
+        qk = dict(q_codes=plan.q_codes, q_scales=plan.q_scales, k_codes=plan.k_codes, k_scales=plan.k_scales)
+        pv = dict(perm=plan.perm, mu=plan.mu, v_codes=plan.v_codes, v_scales=None, s_v=plan.s_v)
+        ox = torch.empty_like(plan.o)
+        for _ in range(2):
+            vc_attn.test_forward_exp2(qk, pv, plan.shape, plan.softmax_scale, plan.k_p, out=ox)
+        n = max(2, min(args.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(n):
+            vc_attn.test_forward_exp2(qk, pv, plan.shape, plan.softmax_scale, plan.k_p, out=ox)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_x = e0.elapsed_time(e1) / n
+        oxf = ox.float()
+        num = den = 0.0
+        for h in (0, H - 1):
+            q = Q[0, rows, h].double()
+            k, v = K[0, :, h].double(), V[0, :, h].double()
+            ref = torch.softmax((q @ k.t()) / math.sqrt(128), dim=-1) @ v
+            num += float(((oxf[0, rows, h].double() - ref) ** 2).sum())
+            den += float((ref ** 2).sum())
+            del k, v, ref
+        out["exp2_comparison"] = {"ms": ms_x, "tflops": flops / (ms_x * 1e-3) / 1e12, "expcast_speedup": ms_x / fwd_ms,
+                                  "rel_l2_vs_fp64": math.sqrt(num / den),
+                                  "what": "same fused kernel, P = E4M3(ex2.approx(c t - F + k_P)) instead of ExpCast"}
+        del ox, oxf
     # BF16 cuDNN SDPA on the same inputs, same stream
     try:
+        if "sdpa" not in legs:
+            raise StopIteration
         qt, kt, vt = (X.transpose(1, 2) for X in (Q, K, V))
         with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
             for _ in range(2):
@@ -348,42 +388,45 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
         sdpa_ms = e0.elapsed_time(e1) / n
         out["sdpa_bf16_cudnn"] = {"ms": sdpa_ms, "tflops": flops / (sdpa_ms * 1e-3) / 1e12,
                                   "speedup_forward": sdpa_ms / fwd_ms, "speedup_full_call": sdpa_ms / ms_per_step}
+    except StopIteration:
+        pass
     except RuntimeError as exc:  # cuDNN backend not available for this shape
         out["sdpa_bf16_cudnn"] = {"unavailable": str(exc).splitlines()[0][:200]}
-    # end to end through the public API with host buffers: H2D of Q, K, V from
-    # pinned memory, the three calls, D2H of O, all inside the timed region
-    hq, hk, hv = (X.cpu().pin_memory() for X in (Q, K, V))
-    ho = torch.empty(plan.o.shape, dtype=plan.o.dtype).pin_memory()
-    dq, dk, dv = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    if "e2e" in legs:
+        # end to end through the public API with host buffers: H2D of Q, K, V from
+        # pinned memory, the three calls, D2H of O, all inside the timed region
+        hq, hk, hv = (X.cpu().pin_memory() for X in (Q, K, V))
+        ho = torch.empty(plan.o.shape, dtype=plan.o.dtype).pin_memory()
+        dq, dk, dv = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        plan.run(dq, dk, dv)
-        ho.copy_(plan.o, non_blocking=True)
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            plan.run(dq, dk, dv)
+            ho.copy_(plan.o, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    n = max(2, min(args.steps, 5))
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(n):
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / n
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    out["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-                  "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
-                  "d2h_bytes_per_step": plan.o.numel() * plan.o.element_size(), "ms_per_step": e2e_ms}
-    del hq, hk, hv, ho, dq, dk, dv
+        torch.cuda.synchronize(dev)
+        n = max(2, min(args.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / n
+        if world > 1:
+            import torch.distributed as dist
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        out["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                      "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
+                      "d2h_bytes_per_step": plan.o.numel() * plan.o.element_size(), "ms_per_step": e2e_ms}
+        del hq, hk, hv, ho, dq, dk, dv
     # the oracle on the host cores, rank 0 at N = 1 only
-    if world == 1 and rank == 0:
+    if world == 1 and rank == 0 and "cpu" in legs:
         full, took, desc = oracle_sample(cfg, min(S, 73397), 256)
         out["cpu_baseline"] = {"value": flops / full / 1e12, "unit": UNIT, "cores": blas_threads(),
                                "kind": "oracle", "sample": desc + f"; measured {took:.1f} s"}

@@ -12,6 +12,7 @@
 #include <string>
 
 #include "../../include/vc_attn.h"
+#include "../../include/vc_attn_testing.h"
 #include "vc_kernels.h"
 
 namespace {
@@ -233,7 +234,7 @@ vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* sha
 
 static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                                   float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream,
-                                  bool nvfp4, void* workspace, size_t workspace_bytes) {
+                                  bool nvfp4, void* workspace, size_t workspace_bytes, bool exp2 = false) {
   g_last_error.clear();
   vc_status_t st;
   if ((st = check_shape(shape)) != VC_OK) return st;
@@ -280,7 +281,7 @@ static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* 
   cudaError_t e;
   if (!nvfp4) {
     if ((st = make_map_u8(&tv, pv->v_codes, (uint64_t)S_pad, (uint64_t)BH * 128)) != VC_OK) return st;
-    e = vc::launch_attn_e4m3(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+    e = vc::launch_attn_e4m3(tq, tk, tv, p, static_cast<cudaStream_t>(stream), exp2);
   } else {
     uint8_t* planes = static_cast<uint8_t*>(workspace);
     e = vc::launch_nvfp4_planes(static_cast<const uint8_t*>(pv->v_codes), static_cast<const uint8_t*>(pv->v_scales),
@@ -298,6 +299,11 @@ static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* 
 vc_status_t vc_attn_forward(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                             float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
   return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, false, nullptr, 0);
+}
+
+vc_status_t vc_attn_test_forward_exp2(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
+                                      float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, false, nullptr, 0, true);
 }
 
 size_t vc_attn_forward_nvfp4v_workspace_bytes(const vc_shape_t* shape) {

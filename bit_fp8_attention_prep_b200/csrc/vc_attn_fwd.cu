@@ -176,7 +176,17 @@ __device__ __forceinline__ uint32_t pack4_imad(float a, float b, float c, float 
   return __byte_perm(lo, hi, 0x5410);
 }
 
-template <int kPlanes>
+// kExp2 = true builds the comparison kernel: the same pipeline with the
+// probabilities made the conventional way, 2^(c t - F + k_P) on the special
+// function unit (ex2.approx) and then converted to E4M3 (round to nearest even,
+// saturating), instead of ExpCast's single fma per score.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int kPlanes, bool kExp2 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     vc_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnParams P) {
@@ -480,12 +490,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ExpCast: one fma per score on the magic-biased fp32; the low byte is the
       // code; the clamp at the magic value is code 0 (masked tail scores are -inf)
       uint32_t w[32];
+      if (!kExp2) {
 #pragma unroll
-      for (int q4 = 0; q4 < 32; ++q4) {
-        const int i = q4 * 4;
-        const float2 a = ffma2(make_float2(SC(i), SC(i + 1)), make_float2(c8, c8), make_float2(bias, bias));
-        const float2 b = ffma2(make_float2(SC(i + 2), SC(i + 3)), make_float2(c8, c8), make_float2(bias, bias));
-        w[q4] = pack4_imad(fmaxf(a.x, kMagic), fmaxf(a.y, kMagic), fmaxf(b.x, kMagic), fmaxf(b.y, kMagic));
+        for (int q4 = 0; q4 < 32; ++q4) {
+          const int i = q4 * 4;
+          const float2 a = ffma2(make_float2(SC(i), SC(i + 1)), make_float2(c8, c8), make_float2(bias, bias));
+          const float2 b = ffma2(make_float2(SC(i + 2), SC(i + 3)), make_float2(c8, c8), make_float2(bias, bias));
+          w[q4] = pack4_imad(fmaxf(a.x, kMagic), fmaxf(a.y, kMagic), fmaxf(b.x, kMagic), fmaxf(b.y, kMagic));
+        }
+      } else {
+        const float off = (float)((P.bias_b - 56) / 8) - Fn;  // k_P - F
+#pragma unroll
+        for (int q4 = 0; q4 < 32; ++q4) {
+          const int i = q4 * 4;
+          const uint32_t lo = cvt_e4m3x2(ex2_approx(__fmaf_rn(SC(i), c, off)), ex2_approx(__fmaf_rn(SC(i + 1), c, off)));
+          const uint32_t hi =
+              cvt_e4m3x2(ex2_approx(__fmaf_rn(SC(i + 2), c, off)), ex2_approx(__fmaf_rn(SC(i + 3), c, off)));
+          w[q4] = lo | (hi << 16);
+        }
       }
 #undef SC
       // PV(j-1) has read P_t and added block j-1 to O_t: then the row-sum column
@@ -596,14 +618,20 @@ cudaError_t attn_configure() {
   cudaError_t e = cudaFuncSetAttribute(vc_attn_fwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)(sizeof(SmemAttn<1>) + 1024));
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(vc_attn_fwd_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)(sizeof(SmemAttn<1>) + 1024));
+  if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(vc_attn_fwd_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)(sizeof(SmemAttn<2>) + 1024));
 }
 
 cudaError_t launch_attn_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const AttnParams& p, cudaStream_t st) {
+                             const AttnParams& p, cudaStream_t st, bool exp2) {
   const dim3 grid((p.nb + 1) / 2, p.B * p.H);
-  vc_attn_fwd_kernel<1><<<grid, kThreads, sizeof(SmemAttn<1>) + 1024, st>>>(tq, tk, tv, p);
+  if (exp2)
+    vc_attn_fwd_kernel<1, true><<<grid, kThreads, sizeof(SmemAttn<1>) + 1024, st>>>(tq, tk, tv, p);
+  else
+    vc_attn_fwd_kernel<1><<<grid, kThreads, sizeof(SmemAttn<1>) + 1024, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 

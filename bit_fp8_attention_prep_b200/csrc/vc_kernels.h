@@ -54,8 +54,10 @@ struct AttnParams {
 };
 
 cudaError_t attn_configure();
+// exp2 = true: the comparison kernel that makes the probabilities with ex2 +
+// E4M3 conversion instead of ExpCast (test hook only)
 cudaError_t launch_attn_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const AttnParams& p, cudaStream_t st);
+                             const AttnParams& p, cudaStream_t st, bool exp2 = false);
 // NVFP4 residual: `tplanes` maps the two E4M3 planes written by launch_nvfp4_planes.
 cudaError_t launch_attn_planes(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tplanes,
                                const AttnParams& p, cudaStream_t st);

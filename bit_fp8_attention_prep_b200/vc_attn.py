@@ -30,7 +30,7 @@ ABI_SYMBOLS = [
 ]
 NOALLOC_SCRATCH_BYTES = 8 << 20   # VC_ATTN_NOALLOC_SCRATCH_BYTES
 TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
-                "vc_attn_test_bounded_wait"]
+                "vc_attn_test_bounded_wait", "vc_attn_test_forward_exp2"]
 
 
 class Shape(ctypes.Structure):
@@ -99,6 +99,8 @@ def load():
     lib.vc_attn_test_expcast.argtypes = [vp, vp, vp, i32, vp, i64, i32, vp]
     lib.vc_attn_test_bounded_wait.restype = i32
     lib.vc_attn_test_bounded_wait.argtypes = [vp, u64, vp]
+    lib.vc_attn_test_forward_exp2.restype = i32
+    lib.vc_attn_test_forward_exp2.argtypes = [P(QKFP8), P(PreparedV), P(Shape), ctypes.c_float, i32, vp, vp, vp]
     _lib = lib
     return lib
 
@@ -355,6 +357,22 @@ def test_expcast(t, c, M, bias_b, hot=False):
     out = torch.empty(t.shape, dtype=torch.uint8, device=t.device)
     _check(load().vc_attn_test_expcast(_ptr(t), _ptr(c), _ptr(M), int(bias_b), _ptr(out), t.numel(), int(hot),
                                        _stream()))
+    return out
+
+
+def test_forward_exp2(qk, pv, shape, softmax_scale=None, k_p=8, out=None, status=None):
+    """The E4M3-V forward with exp2 + E4M3 conversion instead of ExpCast (the
+    comparison kernel of vc_attn_test_forward_exp2)."""
+    lib = load()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(128)
+    dev = qk["q_codes"].device
+    if out is None:
+        out = torch.empty((shape.B, shape.S, shape.H, 128), dtype=torch.bfloat16, device=dev)
+    q_ = QKFP8(_ptr(qk["q_codes"]), _ptr(qk["q_scales"]), _ptr(qk["k_codes"]), _ptr(qk["k_scales"]))
+    p_ = PreparedV(_ptr(pv["perm"]), _ptr(pv["mu"]), _ptr(pv["v_codes"]), _ptr(pv.get("v_scales")), _ptr(pv["s_v"]))
+    _check(lib.vc_attn_test_forward_exp2(ctypes.byref(q_), ctypes.byref(p_), ctypes.byref(shape), float(softmax_scale),
+                                         int(k_p), _ptr(out), _ptr(status), _stream()))
     return out
 
 

@@ -35,6 +35,17 @@ vc_status_t vc_attn_test_expcast(const float* t, const float* c, const float* M,
  * the kernel writes VC_ERR_TIMEOUT into *dev_status and returns; it never hangs. */
 vc_status_t vc_attn_test_bounded_wait(int32_t* dev_status, uint64_t limit_ns, void* stream);
 
+/* The fused E4M3-V attention of vc_attn_forward with one change, for
+ * comparison: each probability is made the conventional way, 2^(c t - M + k_p)
+ * on the special function unit (ex2.approx, flush-to-zero) and then converted
+ * to E4M3 (round to nearest even, saturating), instead of ExpCast's single fma
+ * on the score ("VC-Attention ...", Abstract: ExpCast replaces exactly this exp
+ * and conversion). Frame, row sums, mean restore and layouts are those of
+ * vc_attn_forward; the output differs from it by the approximation of 2^y.
+ * Arguments and errors as vc_attn_forward. */
+vc_status_t vc_attn_test_forward_exp2(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
+                                      float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -106,3 +106,26 @@ def test_attention_accuracy_vs_exact_and_naive(va):
         naive = O.vc_attention_rows(qc, qs, kc, ks, vn, np.zeros((16, 128), np.float32), 2048, rows, SCALE)
         print(f"head {h}: rel-L2 vs exact {e_gpu:.4f}, naive-V {rel_l2(naive, exact):.4f}")
         assert e_gpu < 0.1
+
+
+def test_attention_exp2_comparison_kernel(va):
+    # The comparison kernel (2^y on the special function unit, then an E4M3
+    # conversion, in place of ExpCast) runs the same pipeline: close to exact
+    # attention and to the ExpCast output, not equal to it.
+    cfg, Q, K, V = make("mid", B=1, H=2, S=700)
+    q, k, v = Q.cuda(), K.cuda(), V.cuda()
+    pv = va.prepare_v(v, k=cfg["k"], iters=cfg["iters"])
+    qk = va.quant_qk(q, k, pv["perm"])
+    sh = va.shape_of(q)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o_cast = va.forward(qk, pv, sh, SCALE, 8).float().cpu().numpy()
+    o_exp2 = va.test_forward_exp2(qk, pv, sh, SCALE, 8, status=status).float().cpu().numpy()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rows = np.arange(0, 700, 7)
+    for h in range(2):
+        exact = O.exact_attention_rows(head(Q, 0, h), head(K, 0, h), head(V, 0, h), rows, SCALE)
+        e_exp2 = rel_l2(o_exp2[0, rows, h], exact)
+        e_cast = rel_l2(o_cast[0, rows, h], exact)
+        print(f"head {h}: rel-L2 vs exact: ExpCast {e_cast:.4f}, exp2 + E4M3 {e_exp2:.4f}")
+        assert e_exp2 < 0.05 and rel_l2(o_exp2[0, rows, h], o_cast[0, rows, h]) < 0.05
