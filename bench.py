@@ -56,8 +56,11 @@ def parse_args():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the SDPA comparison, accuracy, e2e and CPU-baseline legs")
     ap.add_argument("--extras", default="all",
-                    help="comma-separated extra legs after the timed region: accuracy, exp2, sdpa, e2e, cpu "
+                    help="comma-separated extra legs after the timed region: accuracy, exp2, sdpa, e2e, cpu, ties "
                          "(default all; --no-extras = none)")
+    ap.add_argument("--sweep", choices=["nvfp4"], default=None,
+                    help="instead of the benchmark line: the NVFP4-V vs E4M3-V sweep over S (H=24), one JSON "
+                         "line per S")
     return ap.parse_args()
 
 
@@ -306,7 +309,7 @@ def run_ours(args, cfg):
         "clocks": clk,
     }
     legs = set() if args.no_extras else (
-        {"accuracy", "exp2", "sdpa", "e2e", "cpu"} if args.extras == "all" else set(args.extras.split(",")))
+        {"accuracy", "exp2", "sdpa", "e2e", "cpu", "ties"} if args.extras == "all" else set(args.extras.split(",")))
     if legs:
         line.update(extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_step, rank, legs))
     if world > 1:
@@ -425,6 +428,24 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
                       "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
                       "d2h_bytes_per_step": plan.o.numel() * plan.o.element_size(), "ms_per_step": e2e_ms}
         del hq, hk, hv, ho, dq, dk, dv
+    # k-means near ties: head 0 of this run's input through the GPU prep with its
+    # per-pass assignments recorded, then the oracle in lock-step on the host
+    if world == 1 and rank == 0 and "ties" in legs:
+        import numpy as np
+        import oracle as O
+        from bit_fp8_attention_prep_b200 import vc_attn
+        v0 = V[:, :, 0:1].contiguous()
+        pv0 = vc_attn.prepare_v(v0, k=cfg["k"], iters=cfg["iters"], fmt=cfg["fmt"], history=True)
+        torch.cuda.synchronize(dev)
+        adopt = [pv0["history"][t, 0, 0].cpu().numpy() for t in range(cfg["iters"])]
+        ref = O.prepare_v_head(v0[0, :, 0].float().cpu().numpy(), cfg["k"], cfg["iters"], 0, 0, fmt=cfg["fmt"],
+                               adopt=adopt)
+        out["kmeans_lockstep"] = {
+            "near_ties": int(ref["stats"]["near_ties"]), "mismatches": int(ref["stats"]["mismatches"]),
+            "perm_bit_exact": bool(np.array_equal(pv0["perm"][0, 0].cpu().numpy(), ref["perm"])),
+            "sample": f"head 0: {S} tokens, k={cfg['k']}, {cfg['iters']} passes; a near tie is a disagreement "
+                      f"whose relative distance gap is below 1e-6 (adopted); anything else is a mismatch"}
+        del pv0, v0
     # the oracle on the host cores, rank 0 at N = 1 only
     if world == 1 and rank == 0 and "cpu" in legs:
         full, took, desc = oracle_sample(cfg, min(S, 73397), 256)
@@ -433,9 +454,56 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
     return out
 
 
+def run_sweep(args):
+    """NVFP4-V vs E4M3-V over S (the NVFP4 sweep workloads: B=1, H=24): forward
+    FP8 TFLOP/s of each and rel-L2 against exact fp64 attention on sampled rows
+    of two heads. One JSON line per S (not the benchmark line)."""
+    import torch
+    from bit_fp8_attention_prep_b200 import synth, vc_attn
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    for S in (1024, 4096, 16384, 32768, 65536, 131072):
+        cfg = synth.workload(f"nvfp4_s{S}")
+        B, H = cfg["B"], cfg["H"]
+        Q, K, V = synth.make_workload(cfg["name"], seed=0, device=dev)[1:]
+        rows = torch.linspace(0, S - 1, 32, device=dev).long()
+        refs = {}
+        for h in (0, H - 1):
+            q = Q[0, rows, h].double()
+            k, v = K[0, :, h].double(), V[0, :, h].double()
+            refs[h] = torch.softmax((q @ k.t()) / math.sqrt(128), dim=-1) @ v
+            del k, v
+        line = {"sweep": "nvfp4_vs_e4m3", "S": S, "B": B, "H": H, "k_p": args.k_p}
+        for fmt in ("e4m3", "nvfp4"):
+            plan = vc_attn.Plan(B, S, H, k=cfg["k"], iters=cfg["iters"], fmt=fmt, k_p=args.k_p, device=dev)
+            plan.run(Q, K, V)
+            for _ in range(2):
+                plan.forward()
+            n = 5
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record()
+            for _ in range(n):
+                plan.forward()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1) / n
+            o = plan.o.float()
+            num = sum(float(((o[0, rows, h].double() - refs[h]) ** 2).sum()) for h in refs)
+            den = sum(float((refs[h] ** 2).sum()) for h in refs)
+            line[fmt] = {"forward_ms": ms, "tflops": flops_of(cfg) / (ms * 1e-3) / 1e12,
+                         "rel_l2_vs_fp64": math.sqrt(num / den), "device_status": int(plan.status.item())}
+            del plan, o
+        print(json.dumps(line), flush=True)
+        del Q, K, V, refs
+
+
 def main():
     args = parse_args()
     from bit_fp8_attention_prep_b200 import synth
+    if args.sweep:
+        run_sweep(args)
+        return
     cfg = synth.workload(args.workload)
     if args.impl == "reference":
         run_reference(args, cfg)
