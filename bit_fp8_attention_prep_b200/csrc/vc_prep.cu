@@ -70,11 +70,12 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(const T* __restrict__ 
 //    read from shared memory (all lanes read the same address). The nearest
 //    centroid, lowest index on ties, is the assignment.
 //  - Accumulation (kAccum): the tile's tokens are put in cluster order (a
-//    counting sort: match_any ranks within each warp, offsets across warps), then
-//    thread d walks them in that order adding llrint(x_d * 2^24) to an int64
-//    running sum and adds the sum into the CTA's accumulator of that cluster when
-//    the cluster changes. Thread d owns column d of the accumulators, so no
-//    atomics are needed until the chunk's sums go to global memory.
+//    counting sort: match_any ranks within each warp, offsets across warps), so
+//    cluster c owns the positions [start_c, start_{c+1}); thread d sums
+//    llrint(x_d * 2^24) over each cluster's range into an int64 register and adds
+//    it to the CTA's accumulator of that cluster. Thread d owns column d of the
+//    accumulators, so no atomics are needed until the chunk's sums go to global
+//    memory.
 constexpr int kTile = 128;
 constexpr int kTileStride = 272;  // bytes per staged row (256 + 16)
 
@@ -90,7 +91,8 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
   uint8_t* tile = reinterpret_cast<uint8_t*>(negc + (size_t)KC * kD);                  // [kTile][272]
   int* scount = reinterpret_cast<int*>(tile + (size_t)kTile * kTileStride);            // [KC]
   int* woff = scount + KC;                                                             // [4][KC]
-  uint8_t* tassign = reinterpret_cast<uint8_t*>(woff + 4 * KC);                        // [kTile]
+  int* cstart = woff + 4 * KC;                                                         // [KC + 1]
+  uint8_t* tassign = reinterpret_cast<uint8_t*>(cstart + KC + 1);                      // [kTile]
   uint8_t* order = tassign + kTile;                                                     // [kTile]
 
   const int bh = blockIdx.y, b = bh / H, h = bh % H;
@@ -192,27 +194,35 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
           woff[1 * KC + tid] = base + w0;
           woff[2 * KC + tid] = base + w0 + w1;
           woff[3 * KC + tid] = base + w0 + w1 + w2;
+          cstart[tid] = base;
+          if (tid == KC - 1) cstart[KC] = incl;
         }
       }
       __syncthreads();
       if (valid) order[woff[warp * KC + best] + rank] = (uint8_t)tid;
       __syncthreads();
-      // thread d: column d of the tile in cluster order
+      // thread d: column d of the tile, cluster by cluster
       const int d = tid;
-      int cur = -1;
-      long long run = 0;
-      for (int pos = 0; pos < ntok; ++pos) {
-        const int tok = order[pos];
-        const int c = tassign[tok];
-        if (c != cur) {
-          if (cur >= 0) acc[cur * kD + d] += run;
-          cur = c;
-          run = 0;
+      const uint8_t* col = tile + d * 2;
+      for (int c = 0; c < k; ++c) {
+        const int p0 = cstart[c], p1 = cstart[c + 1];
+        if (p0 == p1) continue;
+        long long run = 0;
+        int pos = p0;
+#pragma unroll 1
+        for (; pos + 4 <= p1; pos += 4) {
+          const int i0 = order[pos], i1 = order[pos + 1], i2 = order[pos + 2], i3 = order[pos + 3];
+          const float f0 = to_f32<T>(*reinterpret_cast<const T*>(col + i0 * kTileStride));
+          const float f1 = to_f32<T>(*reinterpret_cast<const T*>(col + i1 * kTileStride));
+          const float f2 = to_f32<T>(*reinterpret_cast<const T*>(col + i2 * kTileStride));
+          const float f3 = to_f32<T>(*reinterpret_cast<const T*>(col + i3 * kTileStride));
+          run += (__float2ll_rn(f0 * 16777216.0f) + __float2ll_rn(f1 * 16777216.0f)) +
+                 (__float2ll_rn(f2 * 16777216.0f) + __float2ll_rn(f3 * 16777216.0f));  // x * 2^24, exact
         }
-        const float f = to_f32<T>(*reinterpret_cast<const T*>(tile + tok * kTileStride + d * 2));
-        run += __float2ll_rn(f * 16777216.0f);  // x * 2^24, exact
+        for (; pos < p1; ++pos)
+          run += __float2ll_rn(to_f32<T>(*reinterpret_cast<const T*>(col + order[pos] * kTileStride)) * 16777216.0f);
+        acc[c * kD + d] += run;
       }
-      if (cur >= 0) acc[cur * kD + d] += run;
     }
   }
   __syncthreads();
@@ -227,8 +237,8 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
 
 template <int KC>
 constexpr size_t assign_smem(bool accum) {
-  return (accum ? (size_t)KC * kD * 8 : 0) + (size_t)KC * kD * 4 + (size_t)kTile * kTileStride + 5 * KC * 4 +
-         2 * kTile;
+  return (accum ? (size_t)KC * kD * 8 : 0) + (size_t)KC * kD * 4 + (size_t)kTile * kTileStride +
+         (6 * KC + 1) * 4 + 2 * kTile;
 }
 
 template <typename T, bool kAccum, int KC>
