@@ -69,6 +69,23 @@ def flops_of(cfg):
     return 4.0 * cfg["B"] * cfg["H"] * float(cfg["S"]) ** 2 * 128
 
 
+def max_over_ranks(x, world, device="cpu"):
+    """The largest of the ranks' values of x (every rank gets it); x itself when
+    there is one rank. The timed region of a multi-GPU run is the slowest rank's."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world, flops_per_rank, ms_per_step):
+    """Whole-job throughput of a weak-scaling run: every rank runs its own
+    problem of flops_per_rank, the step takes the slowest rank's time."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -230,12 +247,6 @@ def run_ours(args, cfg):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     B, S, H = cfg["B"], cfg["S"], cfg["H"]
     Q, K, V = synth.make_workload(cfg["name"], seed=rank, device=dev)[1:]
     plan = vc_attn.Plan(B, S, H, k=cfg["k"], iters=cfg["iters"], fmt=cfg["fmt"], k_p=args.k_p, device=dev)
@@ -272,9 +283,9 @@ def run_ours(args, cfg):
     qk_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     fwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
     status = int(plan.status.item())
-    total_ms = max_over_ranks(total_ms)
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = job_tflops(world, flops, ms_per_step)
 
     peaks = load_peaks()
     fp8_peak = 2.0 * peaks["bf16_sustained"]
@@ -418,13 +429,8 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1) / n
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        out["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
+        out["e2e"] = {"value": job_tflops(world, flops, e2e_ms), "unit": UNIT,
                       "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
                       "d2h_bytes_per_step": plan.o.numel() * plan.o.element_size(), "ms_per_step": e2e_ms}
         del hq, hk, hv, ho, dq, dk, dv
