@@ -105,16 +105,6 @@ __device__ __forceinline__ float expcast_z(float t, float c8, float bias) {
   return fmaxf(__fmaf_rn(t, c8, bias), kMagic);
 }
 
-// Pack the low bytes of four magic-biased floats into one 32-bit word
-// (z0 in the lowest byte).
-__device__ __forceinline__ uint32_t pack_codes4(float z0, float z1, float z2, float z3) {
-  uint32_t a = __float_as_uint(z0), b = __float_as_uint(z1);
-  uint32_t c = __float_as_uint(z2), d = __float_as_uint(z3);
-  uint32_t lo = __byte_perm(a, b, 0x0040);  // bytes: a0, b0, a0, a0
-  uint32_t hi = __byte_perm(c, d, 0x0040);  // bytes: c0, d0, ...
-  return __byte_perm(lo, hi, 0x5410);       // a0, b0, c0, d0
-}
-
 // ---------------------------------------------------------------- packed fp32 math
 // Two fp32 fused multiply-adds in one instruction (sm_100 f32x2), each rounded
 // to nearest even exactly like __fmaf_rn.
