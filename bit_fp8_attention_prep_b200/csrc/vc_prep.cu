@@ -64,20 +64,100 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(const T* __restrict__ 
 // --------------------------------------------------------------- k-means assign
 // One CTA (4 warps) = one chunk of kChunk tokens of one (b, h), in tiles of
 // kTile tokens staged in shared memory with coalesced 16-byte loads.
-//  - Assignment: thread t takes token t of the tile. Its squared fp32 distances
-//    to all centroids (at most KC) live in registers as packed f32x2 partial sums
-//    (even and odd dimensions) and grow 16 dimensions at a time, the centroids
-//    read from shared memory (all lanes read the same address). The nearest
-//    centroid, lowest index on ties, is the assignment.
+//  - Assignment. Distances are translation-invariant, so with r the
+//    coordinate-wise median of the centroids, x' = x - r and c' = c - r,
+//    |x - c|^2 = |x'|^2 + g_c where g_c = |c'|^2 - 2 x'.c'. Thread (t, half)
+//    takes tokens t and t + 64 of the tile and the centroids of its parity
+//    (c = 2i + half): one packed f32x2 FMA per two dimensions, token and
+//    centroid, against the direct form's subtract and FMA, with every centroid
+//    value read from shared memory (all lanes of a warp read the same address)
+//    feeding both tokens. The proxies go to shared memory and the token's
+//    thread takes their argmin. Their rounding is bounded: g_c is within
+//    199 u |c'|^2 + 68 u |x'|^2 of its exact value (u = 2^-24: 128-term FMA
+//    chains, the two translations, one final FMA), and the direct fp32 form
+//    sum_d (x_d - c_d)^2 within 134 u (|x'|^2 + |c'|^2). A centroid c whose
+//    g_c - 2^-15 |c'|^2 exceeds g_b + 2^-15 (|c'_b|^2 + |x'|^2) for the nearest
+//    b is farther than b exactly and also by the direct form, so it cannot be
+//    the answer. The rest (a near tie) are compared by the direct form, lowest
+//    index on ties, which is the answer the direct form over all centroids
+//    gives.
 //  - Accumulation (kAccum): the tile's tokens are put in cluster order (a
-//    counting sort: match_any ranks within each warp, offsets across warps), so
-//    cluster c owns the positions [start_c, start_{c+1}); thread d sums
-//    llrint(x_d * 2^24) over each cluster's range into an int64 register and adds
-//    it to the CTA's accumulator of that cluster. Thread d owns column d of the
+//    counting sort: match_any ranks within each warp, offsets across warps) as
+//    words holding the row's offset and its cluster. Thread d walks column d in
+//    that order, eight entries at a time (the loads and the llrint(x_d * 2^24)
+//    conversions of the eight are independent), keeps an int64 running sum and
+//    adds it to the CTA's accumulator of the cluster where the cluster changes,
+//    at the same positions for every thread. Thread d owns column d of the
 //    accumulators, so no atomics are needed until the chunk's sums go to global
 //    memory.
 constexpr int kTile = 128;
-constexpr int kTileStride = 272;  // bytes per staged row (256 + 16)
+
+// Staged tile rows. The accumulating pass pads rows to 272 bytes (its column
+// walk reads one 2-byte element of a row per thread); the final pass packs them
+// at 256 bytes and XORs the 16-byte piece index with the row's low three bits.
+// Either way, eight lanes reading the same piece of eight consecutive rows hit
+// distinct banks.
+template <bool kPad>
+__device__ __forceinline__ int tile_off(int r, int piece) {
+  return kPad ? r * 272 + piece * 16 : r * 256 + ((piece ^ (r & 7)) << 4);
+}
+template <bool kPad>
+__host__ __device__ constexpr int tile_bytes() {
+  return kTile * (kPad ? 272 : 256);
+}
+
+// 16 dimensions (16 ch .. 16 ch + 15) of staged row r, translated: x - r.
+template <typename T, bool kPad>
+__device__ __forceinline__ void load_translated(const uint8_t* tile, int r, int ch, const float* rneg,
+                                                float2* x) {
+  float f[16];
+  unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off<kPad>(r, 2 * ch)), f);
+  unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off<kPad>(r, 2 * ch + 1)), f + 8);
+  const float4* rv = reinterpret_cast<const float4*>(rneg + ch * 16);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 q = rv[i];
+    x[2 * i] = __fadd2_rn(make_float2(f[4 * i], f[4 * i + 1]), make_float2(q.x, q.y));
+    x[2 * i + 1] = __fadd2_rn(make_float2(f[4 * i + 2], f[4 * i + 3]), make_float2(q.z, q.w));
+  }
+}
+
+// Nearest centroid of staged row r among the centroids in the bit mask cand, by
+// the direct form: squared fp32 distances sum_d (x_d - c_d)^2, even and odd
+// dimensions in the two halves of a packed f32x2 accumulator, 16 dimensions at
+// a time, the halves added last; the lowest index wins ties. cg: the centroids
+// of this (b, h), fp32 [k][128].
+template <typename T, bool kPad>
+__device__ __noinline__ int nearest_direct(const uint8_t* tile, int r, const float* __restrict__ cg, uint32_t cand) {
+  int best = -1;
+  float best_d = 0.0f;
+#pragma unroll 1
+  for (; cand != 0u; cand &= cand - 1u) {
+    const int c = __ffs(cand) - 1;
+    float2 dist = make_float2(0.f, 0.f);
+#pragma unroll 1
+    for (int ch = 0; ch < 8; ++ch) {
+      float f[16];
+      unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off<kPad>(r, 2 * ch)), f);
+      unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off<kPad>(r, 2 * ch + 1)), f + 8);
+      const float4* cc = reinterpret_cast<const float4*>(cg + c * kD + ch * 16);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 p = __ldg(cc + i);
+        const float2 d0 = __fadd2_rn(make_float2(f[4 * i], f[4 * i + 1]), make_float2(-p.x, -p.y));
+        const float2 d1 = __fadd2_rn(make_float2(f[4 * i + 2], f[4 * i + 3]), make_float2(-p.z, -p.w));
+        dist = __ffma2_rn(d0, d0, dist);
+        dist = __ffma2_rn(d1, d1, dist);
+      }
+    }
+    const float dd = dist.x + dist.y;
+    if (best < 0 || dd < best_d) {
+      best_d = dd;
+      best = c;
+    }
+  }
+  return best;
+}
 
 template <typename T, bool kAccum, int KC>
 __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restrict__ v, int S, int H, int k,
@@ -85,27 +165,71 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
                                                               unsigned long long* __restrict__ sums,
                                                               int* __restrict__ counts, uint8_t* __restrict__ assign,
                                                               int* __restrict__ hist, uint8_t* __restrict__ history) {
+  constexpr bool kPad = kAccum;
+  constexpr int kHalfC = KC / 2;
+  static_assert(KC % 2 == 0, "cluster capacity must keep the staged tile 16-byte aligned");
   extern __shared__ __align__(16) uint8_t smem[];
   long long* acc = reinterpret_cast<long long*>(smem);                                  // [KC][128] (kAccum)
-  float* negc = reinterpret_cast<float*>(smem + (kAccum ? (size_t)KC * kD * 8 : 0));    // [k][128]
-  uint8_t* tile = reinterpret_cast<uint8_t*>(negc + (size_t)KC * kD);                  // [kTile][272]
-  int* scount = reinterpret_cast<int*>(tile + (size_t)kTile * kTileStride);            // [KC]
+  float* cpr = reinterpret_cast<float*>(smem + (kAccum ? (size_t)KC * kD * 8 : 0));     // [KC][128]: c - r
+  float* rneg = cpr + (size_t)KC * kD;                                                 // [128]: -r
+  float* ncs = rneg + kD;                                                              // [KC]: |c - r|^2
+  float* kns = ncs + KC;                                                               // [KC]: 2^-15 |c - r|^2
+  float* gsm = kns + KC;                                                               // [kTile][KC + 1]: g_c
+  uint8_t* tile = reinterpret_cast<uint8_t*>(gsm + kTile * (KC + 1));                   // staged rows
+  uint32_t* sent = reinterpret_cast<uint32_t*>(tile + tile_bytes<kPad>());             // [kTile]: sorted rows
+  int* scount = reinterpret_cast<int*>(sent + kTile);                                  // [KC]
   int* woff = scount + KC;                                                             // [4][KC]
-  int* cstart = woff + 4 * KC;                                                         // [KC + 1]
-  uint8_t* tassign = reinterpret_cast<uint8_t*>(cstart + KC + 1);                      // [kTile]
-  uint8_t* order = tassign + kTile;                                                     // [kTile]
 
   const int bh = blockIdx.y, b = bh / H, h = bh % H;
   const int chunk = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t row_stride = (size_t)H * kD;  // elements between consecutive tokens of one head
   const T* vbase = v + ((size_t)b * S * H + h) * kD;
+  const float* cg = cent + (size_t)bh * k * kD;
 
-  for (int i = tid; i < k * kD; i += kTile) negc[i] = -cent[(size_t)bh * k * kD + i];
+  {  // translation r = coordinate-wise lower median of the centroids; c' = c - r
+    const int d = tid;
+    float cv[KC];
+#pragma unroll
+    for (int c = 0; c < KC; ++c) cv[c] = c < k ? cg[c * kD + d] : 0.0f;
+    const int m = (k - 1) / 2;
+    float r = cv[0];
+#pragma unroll
+    for (int i = 0; i < KC; ++i) {
+      int lt = 0, le = 0;
+#pragma unroll
+      for (int j = 0; j < KC; ++j) {
+        lt += (j < k && cv[j] < cv[i]);
+        le += (j < k && cv[j] <= cv[i]);
+      }
+      if (i < k && lt <= m && m < le) r = cv[i];
+    }
+    rneg[d] = -r;
+#pragma unroll
+    for (int c = 0; c < KC; ++c)
+      if (c < k) cpr[c * kD + d] = __fsub_rn(cv[c], r);
+  }
   if (kAccum)
     for (int i = tid; i < KC * kD; i += kTile) acc[i] = 0;
   if (tid < KC) scount[tid] = 0;
+  __syncthreads();
+  for (int c = warp; c < k; c += 4) {  // |c'|^2
+    float q = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float x = cpr[c * kD + lane + 32 * j];
+      q = fmaf(x, x, q);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    if (lane == 0) {
+      ncs[c] = q;
+      kns[c] = q * 0x1p-15f;
+    }
+  }
+  __syncthreads();
 
+  const int t = tid & 63, half = tid >> 6;
   const int s_chunk0 = chunk * kChunk;
   const int s_chunk1 = min(S, s_chunk0 + kChunk);
   for (int s0 = s_chunk0; s0 < s_chunk1; s0 += kTile) {
@@ -117,54 +241,71 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
       const int idx = i * kTile + tid, r = idx >> 4, c = idx & 15;
       if (r < ntok) {
         const uint4 val = *reinterpret_cast<const uint4*>(vbase + (size_t)(s0 + r) * row_stride + c * 8);
-        *reinterpret_cast<uint4*>(tile + r * kTileStride + c * 16) = val;
+        *reinterpret_cast<uint4*>(tile + tile_off<kPad>(r, c)) = val;
       }
     }
     if (kAccum && tid < 4 * KC) woff[tid] = 0;
     __syncthreads();
+    // proxies g_c of tokens t and t + 64 (rows past ntok hold stale data; unused)
+    float2 ga[kHalfC], gb[kHalfC];
+#pragma unroll
+    for (int i = 0; i < kHalfC; ++i) ga[i] = gb[i] = make_float2(0.f, 0.f);
+    float2 xx = make_float2(0.f, 0.f);  // |x'|^2 of token tid = t + 64 half
+#pragma unroll 1
+    for (int ch = 0; ch < 8; ++ch) {
+      float2 xa[8], xb[8];
+      load_translated<T, kPad>(tile, t, ch, rneg, xa);
+      load_translated<T, kPad>(tile, t + 64, ch, rneg, xb);
+      if (half == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xx = __ffma2_rn(xa[i], xa[i], xx);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xx = __ffma2_rn(xb[i], xb[i], xx);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+#pragma unroll
+        for (int i = 0; i < kHalfC; ++i) {
+          const int c = 2 * i + half;
+          if (c < k) {
+            const float4 p = *reinterpret_cast<const float4*>(cpr + c * kD + ch * 16 + 4 * q);
+            const float2 p01 = make_float2(p.x, p.y), p23 = make_float2(p.z, p.w);
+            ga[i] = __ffma2_rn(xa[2 * q], p01, ga[i]);
+            gb[i] = __ffma2_rn(xb[2 * q], p01, gb[i]);
+            ga[i] = __ffma2_rn(xa[2 * q + 1], p23, ga[i]);
+            gb[i] = __ffma2_rn(xb[2 * q + 1], p23, gb[i]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int tok = 0; tok < 2; ++tok)
+#pragma unroll
+      for (int i = 0; i < kHalfC; ++i) {
+        const int c = 2 * i + half;
+        if (c < k) {
+          const float2 dot = tok ? gb[i] : ga[i];
+          gsm[(t + 64 * tok) * (KC + 1) + c] = fmaf(-2.0f, dot.x + dot.y, ncs[c]);
+        }
+      }
+    __syncthreads();
     const bool valid = tid < ntok;
     int best = 0;
     if (valid) {
-      float2 dist[KC];
-#pragma unroll
-      for (int c = 0; c < KC; ++c) dist[c] = make_float2(0.f, 0.f);
-#pragma unroll 1
-      for (int ch = 0; ch < 8; ++ch) {  // dimensions 16 ch .. 16 ch + 15
-        float2 x[8];
-        {
-          float f[16];
-          unpack8<T>(*reinterpret_cast<const uint4*>(tile + tid * kTileStride + ch * 32), f);
-          unpack8<T>(*reinterpret_cast<const uint4*>(tile + tid * kTileStride + ch * 32 + 16), f + 8);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) x[i] = make_float2(f[2 * i], f[2 * i + 1]);
+      const float* g = gsm + tid * (KC + 1);
+      float g_best = g[0];
+      for (int c = 1; c < k; ++c)
+        if (g[c] < g_best) {
+          g_best = g[c];
+          best = c;
         }
-#pragma unroll
-        for (int c = 0; c < KC; ++c) {
-          if (c < k) {
-            const float4* nc = reinterpret_cast<const float4*>(negc + c * kD + ch * 16);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float4 p = nc[i];
-              const float2 d0 = __fadd2_rn(x[2 * i + 0], make_float2(p.x, p.y));
-              const float2 d1 = __fadd2_rn(x[2 * i + 1], make_float2(p.z, p.w));
-              dist[c] = __ffma2_rn(d0, d0, dist[c]);
-              dist[c] = __ffma2_rn(d1, d1, dist[c]);
-            }
-          }
-        }
-      }
-      float best_d = 0.0f;
-#pragma unroll
-      for (int c = 0; c < KC; ++c) {
-        if (c < k) {
-          const float dd = dist[c].x + dist[c].y;
-          if (c == 0 || dd < best_d) {
-            best_d = dd;
-            best = c;
-          }
-        }
-      }
-      tassign[tid] = (uint8_t)best;
+      // centroids not ruled out by the rounding bound (a near tie)
+      const float lim = g_best + (kns[best] + (xx.x + xx.y) * 0x1p-15f);
+      uint32_t near = 0;
+      for (int c = 0; c < k; ++c)
+        if (c != best && !(g[c] - kns[c] > lim)) near |= 1u << c;
+      if (near != 0u) best = nearest_direct<T, kPad>(tile, tid, cg, near | (1u << best));
       assign[(size_t)bh * S + s0 + tid] = (uint8_t)best;
       if (history) history[(size_t)bh * S + s0 + tid] = (uint8_t)best;
       atomicAdd(&scount[best], 1);
@@ -194,35 +335,48 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
           woff[1 * KC + tid] = base + w0;
           woff[2 * KC + tid] = base + w0 + w1;
           woff[3 * KC + tid] = base + w0 + w1 + w2;
-          cstart[tid] = base;
-          if (tid == KC - 1) cstart[KC] = incl;
         }
       }
       __syncthreads();
-      if (valid) order[woff[warp * KC + best] + rank] = (uint8_t)tid;
+      if (valid) sent[woff[warp * KC + best] + rank] = (uint32_t)(tid * 272) | ((uint32_t)best << 16);
       __syncthreads();
-      // thread d: column d of the tile, cluster by cluster
+      // thread d: column d of the tile in cluster order; the running sum goes to
+      // the cluster's accumulator where the cluster changes (the same place for
+      // every thread)
       const int d = tid;
       const uint8_t* col = tile + d * 2;
-      for (int c = 0; c < k; ++c) {
-        const int p0 = cstart[c], p1 = cstart[c + 1];
-        if (p0 == p1) continue;
-        long long run = 0;
-        int pos = p0;
-#pragma unroll 1
-        for (; pos + 4 <= p1; pos += 4) {
-          const int i0 = order[pos], i1 = order[pos + 1], i2 = order[pos + 2], i3 = order[pos + 3];
-          const float f0 = to_f32<T>(*reinterpret_cast<const T*>(col + i0 * kTileStride));
-          const float f1 = to_f32<T>(*reinterpret_cast<const T*>(col + i1 * kTileStride));
-          const float f2 = to_f32<T>(*reinterpret_cast<const T*>(col + i2 * kTileStride));
-          const float f3 = to_f32<T>(*reinterpret_cast<const T*>(col + i3 * kTileStride));
-          run += (__float2ll_rn(f0 * 16777216.0f) + __float2ll_rn(f1 * 16777216.0f)) +
-                 (__float2ll_rn(f2 * 16777216.0f) + __float2ll_rn(f3 * 16777216.0f));  // x * 2^24, exact
+      long long run = 0;
+      int cur = (int)(sent[0] >> 16), pos = 0;
+      for (; pos + 8 <= ntok; pos += 8) {
+        const uint4 e0 = *reinterpret_cast<const uint4*>(sent + pos);
+        const uint4 e1 = *reinterpret_cast<const uint4*>(sent + pos + 4);
+        const uint32_t e[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+        long long q[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)  // x * 2^24, exact
+          q[j] = __float2ll_rn(to_f32<T>(*reinterpret_cast<const T*>(col + (e[j] & 0xffffu))) * 16777216.0f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int lab = (int)(e[j] >> 16);
+          if (lab != cur) {
+            acc[cur * kD + d] += run;
+            run = 0;
+            cur = lab;
+          }
+          run += q[j];
         }
-        for (; pos < p1; ++pos)
-          run += __float2ll_rn(to_f32<T>(*reinterpret_cast<const T*>(col + order[pos] * kTileStride)) * 16777216.0f);
-        acc[c * kD + d] += run;
       }
+      for (; pos < ntok; ++pos) {
+        const uint32_t e = sent[pos];
+        const int lab = (int)(e >> 16);
+        if (lab != cur) {
+          acc[cur * kD + d] += run;
+          run = 0;
+          cur = lab;
+        }
+        run += __float2ll_rn(to_f32<T>(*reinterpret_cast<const T*>(col + (e & 0xffffu))) * 16777216.0f);
+      }
+      acc[cur * kD + d] += run;
     }
   }
   __syncthreads();
@@ -237,8 +391,8 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
 
 template <int KC>
 constexpr size_t assign_smem(bool accum) {
-  return (accum ? (size_t)KC * kD * 8 : 0) + (size_t)KC * kD * 4 + (size_t)kTile * kTileStride +
-         (6 * KC + 1) * 4 + 2 * kTile;
+  return (accum ? (size_t)KC * kD * 8 : 0) + (size_t)KC * kD * 4 + kD * 4 + 2 * KC * 4 + kTile * (KC + 1) * 4 +
+         (accum ? tile_bytes<true>() : tile_bytes<false>()) + 4 * kTile + 5 * KC * 4;
 }
 
 template <typename T, bool kAccum, int KC>

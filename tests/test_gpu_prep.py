@@ -78,3 +78,22 @@ def test_meanonly_mode(va):
         assert np.array_equal(pv["perm"][0, h].cpu().numpy(), ref["perm"])
         assert np.array_equal(pv["mu"][0, h].cpu().numpy().view(np.uint32), ref["mu"].view(np.uint32))
         assert np.array_equal(pv["v_codes"][0, h].cpu().numpy(), ref["v_codes"])
+
+
+def test_prep_exact_ties(va):
+    # Values from three integer vectors and the midpoints of their pairs (all exact
+    # in bf16): the initial centroids repeat and many tokens are exactly as far
+    # from two centroids, so most assignments are decided by the direct-form
+    # fallback and the lowest-index rule.
+    g0 = torch.Generator().manual_seed(5)
+    base = torch.randint(-4, 5, (3, 128), generator=g0).float()
+    pool = torch.cat([base, 0.5 * (base[[0, 0, 1]] + base[[1, 2, 2]])])
+    S, H = 700, 2
+    V = pool[torch.randint(0, 6, (1, S, H), generator=g0)].to(torch.bfloat16)
+    Q = torch.randn(1, S, H, 128, generator=g0).to(torch.bfloat16)
+    K = torch.randn(1, S, H, 128, generator=g0).to(torch.bfloat16)
+    g = gpu_pipeline(va, Q, K, V, 8, 3)
+    for h in range(H):
+        ref = oracle_head(g, Q, K, V, 0, h, 8, 3)
+        assert ref["stats"]["near_ties"] == 0, ref["stats"]   # exact ties: both sides take the lowest index
+        assert_prep_bit_exact(g, ref, 0, h)
