@@ -58,6 +58,8 @@ def parse_args():
     ap.add_argument("--extras", default="all",
                     help="comma-separated extra legs after the timed region: accuracy, exp2, sdpa, e2e, cpu, ties "
                          "(default all; --no-extras = none)")
+    ap.add_argument("--head-chunk", type=int, default=4,
+                    help="heads per chunk of the host-buffer pipeline timed by the e2e leg")
     ap.add_argument("--sweep", choices=["nvfp4"], default=None,
                     help="instead of the benchmark line: the NVFP4-V vs E4M3-V sweep over S (H=24), one JSON "
                          "line per S")
@@ -334,6 +336,8 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
     import torch
     import torch.nn.functional as F
     from torch.nn.attention import SDPBackend, sdpa_kernel
+
+    from bit_fp8_attention_prep_b200 import vc_attn
     out = {}
     B, S, H = cfg["B"], cfg["S"], cfg["H"]
     # accuracy on sampled rows of two heads: rel-L2 against exact attention in fp64
@@ -355,7 +359,6 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
     # by exp2 on the special function unit and an E4M3 conversion instead of
     # ExpCast (same prepared inputs, same stream)
     if cfg["fmt"] == "e4m3" and "exp2" in legs:
-        from bit_fp8_attention_prep_b200 import vc_attn
         qk = dict(q_codes=plan.q_codes, q_scales=plan.q_scales, k_codes=plan.k_codes, k_scales=plan.k_scales)
         pv = dict(perm=plan.perm, mu=plan.mu, v_codes=plan.v_codes, v_scales=None, s_v=plan.s_v)
         ox = torch.empty_like(plan.o)
@@ -407,33 +410,49 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
     except RuntimeError as exc:  # cuDNN backend not available for this shape
         out["sdpa_bf16_cudnn"] = {"unavailable": str(exc).splitlines()[0][:200]}
     if "e2e" in legs:
-        # end to end through the public API with host buffers: H2D of Q, K, V from
-        # pinned memory, the three calls, D2H of O, all inside the timed region
+        # end to end through the public API with host buffers: vc_attn_run_host
+        # copies Q, K, V in from pinned host memory and O back, head chunk by head
+        # chunk, overlapped with the compute; everything inside the timed region
         hq, hk, hv = (X.cpu().pin_memory() for X in (Q, K, V))
         ho = torch.empty(plan.o.shape, dtype=plan.o.dtype).pin_memory()
+        hp = vc_attn.HostPlan(B, S, H, k=cfg["k"], iters=cfg["iters"], fmt=cfg["fmt"], k_p=args.k_p,
+                              head_chunk=args.head_chunk, device=dev)
+
+        def timed(step, n):
+            step()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                step()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            return max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
+
+        n = max(2, min(args.steps, 5))
+        e2e_ms = timed(lambda: hp.run(hq, hk, hv, ho), n)
+        plan.run(Q, K, V)
+        torch.cuda.synchronize(dev)
+        same = bool(torch.equal(ho.view(torch.int16), plan.o.cpu().view(torch.int16)))
+        out["e2e"] = {"value": job_tflops(world, flops, e2e_ms), "unit": UNIT,
+                      "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
+                      "d2h_bytes_per_step": plan.o.numel() * plan.o.element_size(), "ms_per_step": e2e_ms,
+                      "api": "vc_attn_run_host", "head_chunk": args.head_chunk,
+                      "status": int(hp.status.item()), "output_equals_device_path": same}
+        # the same copies done one after the other around the three device calls
         dq, dk, dv = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
 
-        def e2e_step():
+        def serial_step():
             dq.copy_(hq, non_blocking=True)
             dk.copy_(hk, non_blocking=True)
             dv.copy_(hv, non_blocking=True)
             plan.run(dq, dk, dv)
             ho.copy_(plan.o, non_blocking=True)
 
-        e2e_step()
-        torch.cuda.synchronize(dev)
-        n = max(2, min(args.steps, 5))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
-        out["e2e"] = {"value": job_tflops(world, flops, e2e_ms), "unit": UNIT,
-                      "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
-                      "d2h_bytes_per_step": plan.o.numel() * plan.o.element_size(), "ms_per_step": e2e_ms}
-        del hq, hk, hv, ho, dq, dk, dv
+        serial_ms = timed(serial_step, n)
+        out["e2e_serial_copies"] = {"value": job_tflops(world, flops, serial_ms), "unit": UNIT,
+                                    "ms_per_step": serial_ms}
+        del hq, hk, hv, ho, dq, dk, dv, hp
     # k-means near ties: head 0 of this run's input through the GPU prep with its
     # per-pass assignments recorded, then the oracle in lock-step on the host
     if world == 1 and rank == 0 and "ties" in legs:

@@ -165,10 +165,13 @@ size_t vc_attn_prepare_v_workspace_bytes(const vc_shape_t* shape, const vc_vsmoo
   return ws_layout(shape, cfg).total;
 }
 
-vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
-                              const vc_prepared_v_t* out, void* workspace, size_t workspace_bytes,
-                              uint8_t* assign_history, void* stream) {
-  g_last_error.clear();
+}  // extern "C"
+
+// vc_attn_prepare_v with the slices numbered from bh_base (the k-means seed of
+// slice i of this call is that of slice bh_base + i of the caller's problem).
+static vc_status_t prepare_v_impl(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                                  const vc_prepared_v_t* out, void* workspace, size_t workspace_bytes,
+                                  uint8_t* assign_history, void* stream, int bh_base) {
   vc_status_t st;
   if ((st = check_shape(shape)) != VC_OK) return st;
   if ((st = check_cfg(cfg)) != VC_OK) return st;
@@ -196,6 +199,7 @@ vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_v
   pl.fmt = cfg->residual_fmt;
   pl.mode = cfg->mode;
   pl.seed = cfg->seed;
+  pl.bh_base = bh_base;
   pl.nb = nblocks(shape->S);
   pl.S_pad = pl.nb * 128;
   pl.nchunks = (shape->S + vc::kChunk - 1) / vc::kChunk;
@@ -212,6 +216,15 @@ vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_v
   g_launches += (uint64_t)nl;
   if (e != cudaSuccess) return cuda_fail(e, "launching V-Smooth prep");
   return VC_OK;
+}
+
+extern "C" {
+
+vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                              const vc_prepared_v_t* out, void* workspace, size_t workspace_bytes,
+                              uint8_t* assign_history, void* stream) {
+  g_last_error.clear();
+  return prepare_v_impl(v, shape, cfg, out, workspace, workspace_bytes, assign_history, stream, 0);
 }
 
 vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* shape, const int32_t* perm,
@@ -362,6 +375,204 @@ vc_status_t vc_attn_prepare_v_noalloc(const void* v, const vc_shape_t* shape, co
     scratch = g_noalloc_addr[dev];
   }
   return vc_attn_prepare_v(v, shape, cfg, out, scratch, VC_ATTN_NOALLOC_SCRATCH_BYTES, assign_history, stream);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ host-buffer pipeline
+namespace {
+
+// Device workspace of vc_attn_run_host for chunks of at most hc heads of one
+// batch entry (every piece 256-B aligned): two slots of Q, K, V and O chunk
+// buffers, so that the copies of one chunk overlap the compute of another, then
+// one set of the chunk's prepared-V, Q/K code and prep scratch buffers (the
+// compute of the chunks is serial on the caller's stream), then the NVFP4
+// planes.
+struct RunHostLayout {
+  size_t in[2][3], out[2];
+  size_t perm, mu, v_codes, v_scales, s_v, q_codes, q_scales, k_codes, k_scales;
+  size_t prep_ws, prep_ws_bytes, planes, planes_bytes, total;
+};
+
+RunHostLayout run_host_layout(const vc_shape_t* sh, const vc_vsmooth_cfg_t* cfg, int hc) {
+  const size_t S = (size_t)sh->S, nb = (size_t)nblocks(sh->S), S_pad = nb * 128, n = (size_t)hc;
+  const size_t chunk_bytes = S * n * 128 * 2;
+  const bool nv = cfg->residual_fmt == VC_RESIDUAL_NVFP4;
+  vc_shape_t cs = *sh;
+  cs.B = 1;
+  cs.H = hc;
+  RunHostLayout L;
+  size_t off = 0;
+  for (int slot = 0; slot < 2; ++slot) {
+    for (int i = 0; i < 3; ++i) {
+      L.in[slot][i] = off;
+      off += align256(chunk_bytes);
+    }
+    L.out[slot] = off;
+    off += align256(chunk_bytes);
+  }
+  L.perm = off;     off += align256(n * S * 4);
+  L.mu = off;       off += align256(n * nb * 128 * 4);
+  L.v_codes = off;  off += align256(n * 128 * (nv ? S_pad / 2 : S_pad));
+  L.v_scales = off; off += nv ? align256(n * 128 * (S_pad / 16)) : 0;
+  L.s_v = off;      off += align256(n * 4);
+  L.q_codes = off;  off += align256(n * S_pad * 128);
+  L.q_scales = off; off += align256(n * nb * 4);
+  L.k_codes = off;  off += align256(n * S_pad * 128);
+  L.k_scales = off; off += align256(n * nb * 4);
+  L.prep_ws_bytes = ws_layout(&cs, cfg).total;
+  L.prep_ws = off;  off += align256(L.prep_ws_bytes);
+  L.planes_bytes = nv ? 2 * n * 128 * S_pad : 0;
+  L.planes = off;   off += align256(L.planes_bytes);
+  L.total = off;
+  return L;
+}
+
+// The two copy streams of a device (host to device, device to host), created on
+// first use and kept until the process exits.
+std::mutex g_copy_mu;
+cudaStream_t g_copy_streams[64][2];
+
+vc_status_t copy_streams(int dev, cudaStream_t* h2d, cudaStream_t* d2h) {
+  std::lock_guard<std::mutex> lk(g_copy_mu);
+  for (int i = 0; i < 2; ++i)
+    if (!g_copy_streams[dev][i]) {
+      cudaError_t e = cudaStreamCreateWithFlags(&g_copy_streams[dev][i], cudaStreamNonBlocking);
+      if (e != cudaSuccess) {
+        g_copy_streams[dev][i] = nullptr;
+        return cuda_fail(e, "creating a copy stream");
+      }
+    }
+  *h2d = g_copy_streams[dev][0];
+  *d2h = g_copy_streams[dev][1];
+  return VC_OK;
+}
+
+// Events of one call, destroyed when the call returns (the runtime releases an
+// event whose recorded work is still pending once that work completes).
+struct CallEvents {
+  cudaEvent_t start = nullptr, done = nullptr, in[2] = {nullptr, nullptr}, comp[2] = {nullptr, nullptr},
+              out[2] = {nullptr, nullptr};
+  cudaError_t create() {
+    cudaEvent_t* all[8] = {&start, &done, &in[0], &in[1], &comp[0], &comp[1], &out[0], &out[1]};
+    for (cudaEvent_t* e : all) {
+      cudaError_t r = cudaEventCreateWithFlags(e, cudaEventDisableTiming);
+      if (r != cudaSuccess) return r;
+    }
+    return cudaSuccess;
+  }
+  ~CallEvents() {
+    cudaEvent_t all[8] = {start, done, in[0], in[1], comp[0], comp[1], out[0], out[1]};
+    for (cudaEvent_t e : all)
+      if (e) cudaEventDestroy(e);
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+size_t vc_attn_run_host_workspace_bytes(const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                                        int32_t head_chunk) {
+  if (check_shape(shape) != VC_OK || check_cfg(cfg) != VC_OK || head_chunk < 1) return 0;
+  return run_host_layout(shape, cfg, head_chunk < shape->H ? head_chunk : shape->H).total;
+}
+
+vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const vc_shape_t* shape,
+                             const vc_vsmooth_cfg_t* cfg, float softmax_scale, int32_t k_p, void* o,
+                             int32_t head_chunk, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                             void* stream) {
+  g_last_error.clear();
+  vc_status_t st;
+  if ((st = check_shape(shape)) != VC_OK) return st;
+  if ((st = check_cfg(cfg)) != VC_OK) return st;
+  if (!q || !k || !v || !o) return fail(VC_ERR_INVALID_ARG, "q, k, v and o must be non-NULL");
+  if (head_chunk < 1) return fail(VC_ERR_INVALID_ARG, "head_chunk must be >= 1 (got %d)", head_chunk);
+  if (!(softmax_scale > 0.0f) || !(softmax_scale < 1e30f))
+    return fail(VC_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
+  if (k_p < 0 || k_p > 8) return fail(VC_ERR_INVALID_ARG, "k_p must be in [0, 8] (got %d)", k_p);
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u))
+    return fail(VC_ERR_INVALID_ARG, "dev_status must be 4-byte aligned");
+  const int B = shape->B, S = shape->S, H = shape->H;
+  const int hc = head_chunk < H ? head_chunk : H;
+  const RunHostLayout L = run_host_layout(shape, cfg, hc);
+  if (!workspace || workspace_bytes < L.total)
+    return fail(VC_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", L.total,
+                workspace ? workspace_bytes : (size_t)0);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(VC_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if ((st = ensure_device()) != VC_OK) return st;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  cudaStream_t s_in, s_out;
+  if ((st = copy_streams(dev, &s_in, &s_out)) != VC_OK) return st;
+  CallEvents ev;
+  if ((e = ev.create()) != cudaSuccess) return cuda_fail(e, "creating events");
+  const cudaStream_t cs_stream = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool nv = cfg->residual_fmt == VC_RESIDUAL_NVFP4;
+  const size_t row_bytes = (size_t)H * 256;  // one token of all heads
+  const char* hq[3] = {static_cast<const char*>(q), static_cast<const char*>(k), static_cast<const char*>(v)};
+  char* ho = static_cast<char*>(o);
+  // the copies start after the work already on the caller's stream (it may still
+  // be using the workspace)
+  if ((e = cudaEventRecord(ev.start, cs_stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((e = cudaStreamWaitEvent(s_in, ev.start, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  if ((e = cudaStreamWaitEvent(s_out, ev.start, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  int c = 0;
+  for (int b = 0; b < B; ++b)
+    for (int h0 = 0; h0 < H; h0 += hc, ++c) {
+      const int n = hc < H - h0 ? hc : H - h0, slot = c & 1;
+      const size_t host_off = ((size_t)b * S * H + h0) * 256, crow = (size_t)n * 256;
+      vc_shape_t cs = *shape;
+      cs.B = 1;
+      cs.H = n;
+      // copy in (the slot's previous chunk must have been computed)
+      if (c >= 2 && (e = cudaStreamWaitEvent(s_in, ev.comp[slot], 0)) != cudaSuccess)
+        return cuda_fail(e, "cudaStreamWaitEvent");
+      for (int i = 0; i < 3; ++i)
+        if ((e = cudaMemcpy2DAsync(ws + L.in[slot][i], crow, hq[i] + host_off, row_bytes, crow, (size_t)S,
+                                   cudaMemcpyHostToDevice, s_in)) != cudaSuccess)
+          return cuda_fail(e, "copying an input chunk to the device");
+      if ((e = cudaEventRecord(ev.in[slot], s_in)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+      // compute (the slot's previous output must have been copied out)
+      if ((e = cudaStreamWaitEvent(cs_stream, ev.in[slot], 0)) != cudaSuccess)
+        return cuda_fail(e, "cudaStreamWaitEvent");
+      if (c >= 2 && (e = cudaStreamWaitEvent(cs_stream, ev.out[slot], 0)) != cudaSuccess)
+        return cuda_fail(e, "cudaStreamWaitEvent");
+      vc_prepared_v_t pv;
+      pv.perm = reinterpret_cast<int32_t*>(ws + L.perm);
+      pv.mu = reinterpret_cast<float*>(ws + L.mu);
+      pv.v_codes = ws + L.v_codes;
+      pv.v_scales = nv ? ws + L.v_scales : nullptr;
+      pv.s_v = reinterpret_cast<float*>(ws + L.s_v);
+      vc_qk_fp8_t qk;
+      qk.q_codes = ws + L.q_codes;
+      qk.q_scales = reinterpret_cast<float*>(ws + L.q_scales);
+      qk.k_codes = ws + L.k_codes;
+      qk.k_scales = reinterpret_cast<float*>(ws + L.k_scales);
+      if ((st = prepare_v_impl(ws + L.in[slot][2], &cs, cfg, &pv, ws + L.prep_ws, L.prep_ws_bytes, nullptr,
+                               stream, b * H + h0)) != VC_OK)
+        return st;
+      if ((st = vc_attn_quant_qk(ws + L.in[slot][0], ws + L.in[slot][1], &cs, pv.perm, &qk, stream)) != VC_OK)
+        return st;
+      if ((st = forward_common(&qk, &pv, &cs, softmax_scale, k_p, ws + L.out[slot], dev_status, stream, nv,
+                               nv ? ws + L.planes : nullptr, L.planes_bytes)) != VC_OK)
+        return st;
+      if ((e = cudaEventRecord(ev.comp[slot], cs_stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+      // copy out
+      if ((e = cudaStreamWaitEvent(s_out, ev.comp[slot], 0)) != cudaSuccess)
+        return cuda_fail(e, "cudaStreamWaitEvent");
+      if ((e = cudaMemcpy2DAsync(ho + host_off, row_bytes, ws + L.out[slot], crow, crow, (size_t)S,
+                                 cudaMemcpyDeviceToHost, s_out)) != cudaSuccess)
+        return cuda_fail(e, "copying an output chunk to the host");
+      if ((e = cudaEventRecord(ev.out[slot], s_out)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    }
+  // the caller's stream passes this point once the last output chunk is on the host
+  if ((e = cudaEventRecord(ev.done, s_out)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((e = cudaStreamWaitEvent(cs_stream, ev.done, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  return VC_OK;
 }
 
 }  // extern "C"

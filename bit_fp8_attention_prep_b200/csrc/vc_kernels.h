@@ -20,6 +20,8 @@ constexpr int kChunk = 1024;       // tokens per k-means CTA (also the sort's ch
 struct PrepPlan {
   int B, S, H, k, iters, fmt, mode;
   uint64_t seed;
+  int bh_base;                 // index b*H + h of this plan's first slice in the caller's problem
+                               // (0 unless the problem is run in chunks of heads)
   int nb, S_pad, nchunks;
   float* cent;                 // [BH][k][128]
   unsigned long long* sums;    // [BH][k][128] int64 fixed-point

@@ -37,11 +37,11 @@ __device__ __forceinline__ uint64_t splitmix64_next(uint64_t& state) {
 
 template <typename T>
 __global__ void __launch_bounds__(128) kmeans_init_kernel(const T* __restrict__ v, int S, int H, int k,
-                                                          uint64_t seed, float* __restrict__ cent) {
+                                                          uint64_t seed, int bh_base, float* __restrict__ cent) {
   __shared__ int idx[kMaxClusters];
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
   if (threadIdx.x == 0) {
-    uint64_t st = seed ^ (0x9E3779B97F4A7C15ull * (uint64_t)(bh + 1));
+    uint64_t st = seed ^ (0x9E3779B97F4A7C15ull * (uint64_t)(bh_base + bh + 1));
     for (int i = 0; i < k; ++i) {
       int u;
       while (true) {
@@ -802,7 +802,7 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
   if (pl.mode == VC_MODE_VSMOOTH) {
     if ((e = cudaMemsetAsync(pl.sums, 0, sizeof(unsigned long long) * BH * k * kD, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(pl.counts, 0, sizeof(int) * BH * k, st)) != cudaSuccess) return e;
-    kmeans_init_kernel<T><<<BH, 128, 0, st>>>(v, S, H, k, pl.seed, pl.cent);
+    kmeans_init_kernel<T><<<BH, 128, 0, st>>>(v, S, H, k, pl.seed, pl.bh_base, pl.cent);
     ++n;
     const dim3 grid(pl.nchunks, BH);
     for (int it = 0; it < pl.iters; ++it) {

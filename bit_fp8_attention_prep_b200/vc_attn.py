@@ -26,7 +26,7 @@ ABI_SYMBOLS = [
     "vc_attn_version", "vc_attn_last_error", "vc_attn_launch_count", "vc_attn_prepare_v_workspace_bytes",
     "vc_attn_prepare_v",
     "vc_attn_quant_qk", "vc_attn_forward", "vc_attn_forward_nvfp4v_workspace_bytes", "vc_attn_forward_nvfp4v",
-    "vc_attn_prepare_v_noalloc",
+    "vc_attn_prepare_v_noalloc", "vc_attn_run_host_workspace_bytes", "vc_attn_run_host",
 ]
 NOALLOC_SCRATCH_BYTES = 8 << 20   # VC_ATTN_NOALLOC_SCRATCH_BYTES
 TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
@@ -91,6 +91,11 @@ def load():
     lib.vc_attn_forward_nvfp4v.restype = i32
     lib.vc_attn_forward_nvfp4v.argtypes = [P(QKFP8), P(PreparedV), P(Shape), ctypes.c_float, i32, vp, vp, sz,
                                            vp, vp]
+    lib.vc_attn_run_host_workspace_bytes.restype = sz
+    lib.vc_attn_run_host_workspace_bytes.argtypes = [P(Shape), P(VSmoothCfg), i32]
+    lib.vc_attn_run_host.restype = i32
+    lib.vc_attn_run_host.argtypes = [vp, vp, vp, P(Shape), P(VSmoothCfg), ctypes.c_float, i32, vp, i32, vp, sz,
+                                     vp, vp]
     lib.vc_attn_test_e4m3_round.restype = i32
     lib.vc_attn_test_e4m3_round.argtypes = [vp, vp, i64, vp]
     lib.vc_attn_test_e2m1_round.restype = i32
@@ -333,6 +338,45 @@ class Plan:
         self.prepare_v(v)
         self.quant_qk(q, k)
         return self.forward(out)
+
+
+class HostPlan:
+    """The whole path for Q, K, V and O in host memory (``vc_attn_run_host``):
+    the device workspace for one shape and head chunk is allocated once here;
+    ``run(q, k, v, o)`` takes CPU tensors of shape [B,S,H,128] (page-locked for
+    the copies to overlap the compute; ``o`` bf16) and enqueues the chunked
+    copies and the three calls on the current stream. ``o`` is complete once
+    the stream has passed the call."""
+
+    def __init__(self, B, S, H, dtype=torch.bfloat16, k=16, iters=4, seed=0, fmt="e4m3", k_p=8,
+                 softmax_scale=None, head_chunk=4, device=None, mode="vsmooth"):
+        self.lib = load()
+        dev = torch.device(device if device is not None else "cuda")
+        self.dtype = dtype
+        self.shape = Shape(B, S, H, 128, VC_DTYPE_BF16 if dtype == torch.bfloat16 else VC_DTYPE_F16)
+        self.cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
+                              VC_MODE_MEANONLY if mode == "meanonly" else VC_MODE_VSMOOTH)
+        self.k_p, self.head_chunk = int(k_p), int(head_chunk)
+        self.softmax_scale = 1.0 / math.sqrt(128) if softmax_scale is None else float(softmax_scale)
+        self.ws_bytes = self.lib.vc_attn_run_host_workspace_bytes(ctypes.byref(self.shape), ctypes.byref(self.cfg),
+                                                                   self.head_chunk)
+        if self.ws_bytes == 0:
+            raise VCError(VC_ERR_INVALID_ARG, "invalid shape, config or head chunk")
+        self._ws = torch.empty((self.ws_bytes + 256,), dtype=torch.uint8, device=dev)
+        self.ws_ptr = ctypes.c_void_p(self._ws.data_ptr() + (-self._ws.data_ptr()) % 256)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def run(self, q, k, v, o):
+        want = (self.shape.B, self.shape.S, self.shape.H, 128)
+        for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+            if t.device.type != "cpu" or not t.is_contiguous() or tuple(t.reshape(want).shape) != want:
+                raise ValueError(f"{name} must be a contiguous CPU tensor of shape {want}")
+        if q.dtype != self.dtype or k.dtype != self.dtype or v.dtype != self.dtype or o.dtype != torch.bfloat16:
+            raise ValueError("q, k, v must have the plan's dtype and o must be bfloat16")
+        _check(self.lib.vc_attn_run_host(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(self.shape), ctypes.byref(self.cfg),
+                                         self.softmax_scale, self.k_p, _ptr(o), self.head_chunk, self.ws_ptr,
+                                         self.ws_bytes, _ptr(self.status), _stream()))
+        return o
 
 
 def launch_count():

@@ -14,7 +14,8 @@
  *
  * Conventions (every entry point):
  *  - Pointers named q, k, v, o and every field of vc_prepared_v_t / vc_qk_fp8_t
- *    are DEVICE pointers owned and allocated by the caller; the library never
+ *    are DEVICE pointers owned and allocated by the caller (except in
+ *    vc_attn_run_host, whose q, k, v, o are host pointers); the library never
  *    allocates or frees device memory and keeps no pointer after a call returns.
  *  - Tensors are dense and row-major in the layouts stated per field. Q, K, V and
  *    O are [B, S, H, 128] (a [S, H, 128] tensor is B = 1). Device pointers must
@@ -214,6 +215,51 @@ vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t*
  * Arguments, outputs and other errors are those of vc_attn_prepare_v. */
 vc_status_t vc_attn_prepare_v_noalloc(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
                                       const vc_prepared_v_t* out, uint8_t* assign_history, void* stream);
+
+/* Bytes of device workspace vc_attn_run_host needs for this shape, config and
+ * head chunk (0 if the arguments are invalid). About 8 * S * head_chunk * 256
+ * bytes of chunk buffers plus one chunk's prep, code and scratch buffers. */
+size_t vc_attn_run_host_workspace_bytes(const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                                        int32_t head_chunk);
+
+/* The whole path -- vc_attn_prepare_v, vc_attn_quant_qk and vc_attn_forward (or
+ * vc_attn_forward_nvfp4v for cfg->residual_fmt == VC_RESIDUAL_NVFP4) -- for Q, K,
+ * V and O in HOST memory, with the host<->device copies overlapped with the
+ * compute. Every (b, h) slice of the method is independent ("VC-Attention ...",
+ * Abstract: clustering, block means and the residual scale are per value head;
+ * "Nunchux AI lanza ...", 2nd paragraph: k-means per batch and head), so the
+ * call runs the problem in chunks of `head_chunk` heads of one batch entry: the
+ * chunk's Q, K, V rows are copied to the device on one internal stream, its prep,
+ * Q/K quantisation and attention run on `stream`, and its O rows are copied back
+ * on a second internal stream, while the next chunk's inputs are already being
+ * copied in. The output is bit-identical to the three device calls on the whole
+ * problem (each chunk's k-means is seeded by the slice's index in the whole
+ * problem).
+ *  q, k, v       HOST, [B,S,H,128] of shape->dtype. Page-locked memory
+ *                (cudaHostAlloc / cudaHostRegister) lets the copies run
+ *                asynchronously; with pageable memory the call still gives the
+ *                same result, but the copies do not overlap the compute.
+ *  o             HOST, bf16 [B,S,H,128]; valid once `stream` has passed the call
+ *                (e.g. after cudaStreamSynchronize(stream))
+ *  head_chunk    heads per chunk, >= 1 (values above H mean H); smaller chunks
+ *                overlap more of the copies, larger ones keep more of the GPU
+ *                busy per launch (4 for H = 56 on a B200 over PCIe 5)
+ *  workspace     device, >= vc_attn_run_host_workspace_bytes(), 256-B aligned;
+ *                must not be reused by other work until `stream` has passed the
+ *                call
+ *  other arguments as vc_attn_forward (cfg as vc_attn_prepare_v)
+ * The host buffers must stay valid and unmodified until `stream` has passed the
+ * call. The two internal copy streams of each device are created on the first
+ * call there (not during stream capture) and live until the process exits; the
+ * call enqueues its work and returns without waiting for it.
+ * Errors: as vc_attn_prepare_v and vc_attn_forward, plus VC_ERR_INVALID_ARG for
+ * head_chunk < 1 and VC_ERR_WORKSPACE. All arguments are checked before anything
+ * is enqueued; a VC_ERR_CUDA from a failed launch or copy may leave earlier
+ * chunks enqueued. */
+vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const vc_shape_t* shape,
+                             const vc_vsmooth_cfg_t* cfg, float softmax_scale, int32_t k_p, void* o,
+                             int32_t head_chunk, void* workspace, size_t workspace_bytes,
+                             int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

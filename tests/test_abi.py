@@ -110,3 +110,28 @@ def test_nvfp4_forward_workspace_size_and_checks(lib):
     st = lib.vc_attn_forward_nvfp4v(ctypes.byref(qk), ctypes.byref(pv_noscale), ctypes.byref(_shape()), 0.088, 8,
                                     ctypes.c_void_p(16), ctypes.c_void_p(256), need, None, None)
     assert st == vc_attn.VC_ERR_INVALID_ARG
+
+
+def test_run_host_workspace_and_validation(lib):
+    sh, cfg = _shape(S=1000, H=5), _cfg(k=16, iters=4)
+    ws = [lib.vc_attn_run_host_workspace_bytes(ctypes.byref(sh), ctypes.byref(cfg), c) for c in (1, 2, 5, 9)]
+    assert all(w > 0 and w % 256 == 0 for w in ws)
+    assert ws[0] < ws[1] < ws[2] == ws[3]          # head_chunk above H means H
+    # two slots of Q, K, V, O chunk buffers are part of it
+    assert ws[1] > 8 * 1000 * 2 * 256
+    assert lib.vc_attn_run_host_workspace_bytes(ctypes.byref(sh), ctypes.byref(cfg), 0) == 0
+    assert lib.vc_attn_run_host_workspace_bytes(ctypes.byref(_shape(D=64)), ctypes.byref(cfg), 2) == 0
+    nv = lib.vc_attn_run_host_workspace_bytes(ctypes.byref(sh), ctypes.byref(_cfg(k=16, iters=4, fmt=1)), 2)
+    assert nv > ws[1]                               # plus the NVFP4 scales and planes
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    for args, code in (
+        ((p, p, p, ctypes.byref(sh), ctypes.byref(cfg), 0.088, 8, p, 0, None, 0, None, None), vc_attn.VC_ERR_INVALID_ARG),
+        ((p, p, p, ctypes.byref(sh), ctypes.byref(cfg), -1.0, 8, p, 2, None, 0, None, None), vc_attn.VC_ERR_INVALID_ARG),
+        ((p, p, p, ctypes.byref(sh), ctypes.byref(cfg), 0.088, 9, p, 2, None, 0, None, None), vc_attn.VC_ERR_INVALID_ARG),
+        ((None, p, p, ctypes.byref(sh), ctypes.byref(cfg), 0.088, 8, p, 2, None, 0, None, None), vc_attn.VC_ERR_INVALID_ARG),
+        ((p, p, p, ctypes.byref(sh), ctypes.byref(cfg), 0.088, 8, p, 2, None, 0, None, None), vc_attn.VC_ERR_WORKSPACE),
+        ((p, p, p, ctypes.byref(sh), ctypes.byref(cfg), 0.088, 8, p, 2, p, 64, None, None), vc_attn.VC_ERR_WORKSPACE),
+    ):
+        assert lib.vc_attn_run_host(*args) == code
+        assert lib.vc_attn_last_error() != b""
