@@ -383,15 +383,15 @@ vc_status_t vc_attn_prepare_v_noalloc(const void* v, const vc_shape_t* shape, co
 namespace {
 
 // Device workspace of vc_attn_run_host for chunks of at most hc heads of one
-// batch entry (every piece 256-B aligned): two slots of Q, K, V and O chunk
-// buffers, so that the copies of one chunk overlap the compute of another, then
-// one set of the chunk's prepared-V, Q/K code and prep scratch buffers (the
-// compute of the chunks is serial on the caller's stream), then the NVFP4
-// planes.
+// batch entry (every piece 256-B aligned), in two slots used by alternate
+// chunks: the chunk's Q, K, V and O buffers (the copies of one chunk overlap the
+// compute of the other), then its prepared-V, Q/K code, prep scratch and NVFP4
+// plane buffers (the two slots compute on two streams, so that one chunk's
+// last wave of attention CTAs shares the GPU with the next chunk's kernels).
 struct RunHostLayout {
   size_t in[2][3], out[2];
-  size_t perm, mu, v_codes, v_scales, s_v, q_codes, q_scales, k_codes, k_scales;
-  size_t prep_ws, prep_ws_bytes, planes, planes_bytes, total;
+  size_t perm[2], mu[2], v_codes[2], v_scales[2], s_v[2], q_codes[2], q_scales[2], k_codes[2], k_scales[2];
+  size_t prep_ws[2], prep_ws_bytes, planes[2], planes_bytes, total;
 };
 
 RunHostLayout run_host_layout(const vc_shape_t* sh, const vc_vsmooth_cfg_t* cfg, int hc) {
@@ -411,40 +411,44 @@ RunHostLayout run_host_layout(const vc_shape_t* sh, const vc_vsmooth_cfg_t* cfg,
     L.out[slot] = off;
     off += align256(chunk_bytes);
   }
-  L.perm = off;     off += align256(n * S * 4);
-  L.mu = off;       off += align256(n * nb * 128 * 4);
-  L.v_codes = off;  off += align256(n * 128 * (nv ? S_pad / 2 : S_pad));
-  L.v_scales = off; off += nv ? align256(n * 128 * (S_pad / 16)) : 0;
-  L.s_v = off;      off += align256(n * 4);
-  L.q_codes = off;  off += align256(n * S_pad * 128);
-  L.q_scales = off; off += align256(n * nb * 4);
-  L.k_codes = off;  off += align256(n * S_pad * 128);
-  L.k_scales = off; off += align256(n * nb * 4);
   L.prep_ws_bytes = ws_layout(&cs, cfg).total;
-  L.prep_ws = off;  off += align256(L.prep_ws_bytes);
   L.planes_bytes = nv ? 2 * n * 128 * S_pad : 0;
-  L.planes = off;   off += align256(L.planes_bytes);
+  for (int slot = 0; slot < 2; ++slot) {
+    L.perm[slot] = off;     off += align256(n * S * 4);
+    L.mu[slot] = off;       off += align256(n * nb * 128 * 4);
+    L.v_codes[slot] = off;  off += align256(n * 128 * (nv ? S_pad / 2 : S_pad));
+    L.v_scales[slot] = off; off += nv ? align256(n * 128 * (S_pad / 16)) : 0;
+    L.s_v[slot] = off;      off += align256(n * 4);
+    L.q_codes[slot] = off;  off += align256(n * S_pad * 128);
+    L.q_scales[slot] = off; off += align256(n * nb * 4);
+    L.k_codes[slot] = off;  off += align256(n * S_pad * 128);
+    L.k_scales[slot] = off; off += align256(n * nb * 4);
+    L.prep_ws[slot] = off;  off += align256(L.prep_ws_bytes);
+    L.planes[slot] = off;   off += align256(L.planes_bytes);
+  }
   L.total = off;
   return L;
 }
 
-// The two copy streams of a device (host to device, device to host), created on
-// first use and kept until the process exits.
+// The internal streams of a device (host to device copies, device to host
+// copies, the compute of odd chunks), created on first use and kept until the
+// process exits.
 std::mutex g_copy_mu;
-cudaStream_t g_copy_streams[64][2];
+cudaStream_t g_copy_streams[64][3];
 
-vc_status_t copy_streams(int dev, cudaStream_t* h2d, cudaStream_t* d2h) {
+vc_status_t copy_streams(int dev, cudaStream_t* h2d, cudaStream_t* d2h, cudaStream_t* odd) {
   std::lock_guard<std::mutex> lk(g_copy_mu);
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 3; ++i)
     if (!g_copy_streams[dev][i]) {
       cudaError_t e = cudaStreamCreateWithFlags(&g_copy_streams[dev][i], cudaStreamNonBlocking);
       if (e != cudaSuccess) {
         g_copy_streams[dev][i] = nullptr;
-        return cuda_fail(e, "creating a copy stream");
+        return cuda_fail(e, "creating an internal stream");
       }
     }
   *h2d = g_copy_streams[dev][0];
   *d2h = g_copy_streams[dev][1];
+  *odd = g_copy_streams[dev][2];
   return VC_OK;
 }
 
@@ -505,8 +509,8 @@ vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  cudaStream_t s_in, s_out;
-  if ((st = copy_streams(dev, &s_in, &s_out)) != VC_OK) return st;
+  cudaStream_t s_in, s_out, s_odd;
+  if ((st = copy_streams(dev, &s_in, &s_out, &s_odd)) != VC_OK) return st;
   CallEvents ev;
   if ((e = ev.create()) != cudaSuccess) return cuda_fail(e, "creating events");
   const cudaStream_t cs_stream = static_cast<cudaStream_t>(stream);
@@ -520,6 +524,8 @@ vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const 
   if ((e = cudaEventRecord(ev.start, cs_stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if ((e = cudaStreamWaitEvent(s_in, ev.start, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
   if ((e = cudaStreamWaitEvent(s_out, ev.start, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  if ((e = cudaStreamWaitEvent(s_odd, ev.start, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  const cudaStream_t comp_stream[2] = {cs_stream, s_odd};
   int c = 0;
   for (int b = 0; b < B; ++b)
     for (int h0 = 0; h0 < H; h0 += hc, ++c) {
@@ -537,30 +543,30 @@ vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const 
           return cuda_fail(e, "copying an input chunk to the device");
       if ((e = cudaEventRecord(ev.in[slot], s_in)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
       // compute (the slot's previous output must have been copied out)
-      if ((e = cudaStreamWaitEvent(cs_stream, ev.in[slot], 0)) != cudaSuccess)
-        return cuda_fail(e, "cudaStreamWaitEvent");
-      if (c >= 2 && (e = cudaStreamWaitEvent(cs_stream, ev.out[slot], 0)) != cudaSuccess)
+      const cudaStream_t cst = comp_stream[slot];
+      if ((e = cudaStreamWaitEvent(cst, ev.in[slot], 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+      if (c >= 2 && (e = cudaStreamWaitEvent(cst, ev.out[slot], 0)) != cudaSuccess)
         return cuda_fail(e, "cudaStreamWaitEvent");
       vc_prepared_v_t pv;
-      pv.perm = reinterpret_cast<int32_t*>(ws + L.perm);
-      pv.mu = reinterpret_cast<float*>(ws + L.mu);
-      pv.v_codes = ws + L.v_codes;
-      pv.v_scales = nv ? ws + L.v_scales : nullptr;
-      pv.s_v = reinterpret_cast<float*>(ws + L.s_v);
+      pv.perm = reinterpret_cast<int32_t*>(ws + L.perm[slot]);
+      pv.mu = reinterpret_cast<float*>(ws + L.mu[slot]);
+      pv.v_codes = ws + L.v_codes[slot];
+      pv.v_scales = nv ? ws + L.v_scales[slot] : nullptr;
+      pv.s_v = reinterpret_cast<float*>(ws + L.s_v[slot]);
       vc_qk_fp8_t qk;
-      qk.q_codes = ws + L.q_codes;
-      qk.q_scales = reinterpret_cast<float*>(ws + L.q_scales);
-      qk.k_codes = ws + L.k_codes;
-      qk.k_scales = reinterpret_cast<float*>(ws + L.k_scales);
-      if ((st = prepare_v_impl(ws + L.in[slot][2], &cs, cfg, &pv, ws + L.prep_ws, L.prep_ws_bytes, nullptr,
-                               stream, b * H + h0)) != VC_OK)
+      qk.q_codes = ws + L.q_codes[slot];
+      qk.q_scales = reinterpret_cast<float*>(ws + L.q_scales[slot]);
+      qk.k_codes = ws + L.k_codes[slot];
+      qk.k_scales = reinterpret_cast<float*>(ws + L.k_scales[slot]);
+      if ((st = prepare_v_impl(ws + L.in[slot][2], &cs, cfg, &pv, ws + L.prep_ws[slot], L.prep_ws_bytes, nullptr,
+                               cst, b * H + h0)) != VC_OK)
         return st;
-      if ((st = vc_attn_quant_qk(ws + L.in[slot][0], ws + L.in[slot][1], &cs, pv.perm, &qk, stream)) != VC_OK)
+      if ((st = vc_attn_quant_qk(ws + L.in[slot][0], ws + L.in[slot][1], &cs, pv.perm, &qk, cst)) != VC_OK)
         return st;
-      if ((st = forward_common(&qk, &pv, &cs, softmax_scale, k_p, ws + L.out[slot], dev_status, stream, nv,
-                               nv ? ws + L.planes : nullptr, L.planes_bytes)) != VC_OK)
+      if ((st = forward_common(&qk, &pv, &cs, softmax_scale, k_p, ws + L.out[slot], dev_status, cst, nv,
+                               nv ? ws + L.planes[slot] : nullptr, L.planes_bytes)) != VC_OK)
         return st;
-      if ((e = cudaEventRecord(ev.comp[slot], cs_stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+      if ((e = cudaEventRecord(ev.comp[slot], cst)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
       // copy out
       if ((e = cudaStreamWaitEvent(s_out, ev.comp[slot], 0)) != cudaSuccess)
         return cuda_fail(e, "cudaStreamWaitEvent");

@@ -217,8 +217,9 @@ vc_status_t vc_attn_prepare_v_noalloc(const void* v, const vc_shape_t* shape, co
                                       const vc_prepared_v_t* out, uint8_t* assign_history, void* stream);
 
 /* Bytes of device workspace vc_attn_run_host needs for this shape, config and
- * head chunk (0 if the arguments are invalid). About 8 * S * head_chunk * 256
- * bytes of chunk buffers plus one chunk's prep, code and scratch buffers. */
+ * head chunk (0 if the arguments are invalid): two slots, each with a chunk's
+ * Q, K, V and O buffers (4 * S * head_chunk * 256 bytes) and its prep, code and
+ * scratch buffers (about 3 * S * head_chunk * 128 bytes more). */
 size_t vc_attn_run_host_workspace_bytes(const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
                                         int32_t head_chunk);
 
@@ -230,8 +231,10 @@ size_t vc_attn_run_host_workspace_bytes(const vc_shape_t* shape, const vc_vsmoot
  * "Nunchux AI lanza ...", 2nd paragraph: k-means per batch and head), so the
  * call runs the problem in chunks of `head_chunk` heads of one batch entry: the
  * chunk's Q, K, V rows are copied to the device on one internal stream, its prep,
- * Q/K quantisation and attention run on `stream`, and its O rows are copied back
- * on a second internal stream, while the next chunk's inputs are already being
+ * Q/K quantisation and attention run on `stream` (even chunks) or on a second
+ * internal stream (odd chunks, so that one chunk's last wave of attention CTAs
+ * shares the GPU with the next chunk's kernels), and its O rows are copied back
+ * on a third internal stream, while the next chunks' inputs are already being
  * copied in. The output is bit-identical to the three device calls on the whole
  * problem (each chunk's k-means is seeded by the slice's index in the whole
  * problem).
@@ -249,7 +252,7 @@ size_t vc_attn_run_host_workspace_bytes(const vc_shape_t* shape, const vc_vsmoot
  *                call
  *  other arguments as vc_attn_forward (cfg as vc_attn_prepare_v)
  * The host buffers must stay valid and unmodified until `stream` has passed the
- * call. The two internal copy streams of each device are created on the first
+ * call. The three internal streams of each device are created on the first
  * call there (not during stream capture) and live until the process exits; the
  * call enqueues its work and returns without waiting for it.
  * Errors: as vc_attn_prepare_v and vc_attn_forward, plus VC_ERR_INVALID_ARG for
