@@ -492,51 +492,84 @@ __global__ void identity_perm_kernel(int S, int32_t* __restrict__ perm) {
 }
 
 // --------------------------------------------------------------- block mean + residual amax
-// One CTA (4 warps) = one 128-token block of permuted positions. Warp w walks
-// rows 32w..32w+31; lane l owns dimensions 4l..4l+3 (one coalesced 256-B row per
-// warp load). Means use the int64 fixed-point sum; the residual amax is merged
-// into amax[bh] with an integer atomicMax on the (non-negative) fp32 bits.
+// One CTA (4 warps) = one 128-token block of permuted positions, loaded as in
+// quant_qk_kernel: warp w takes rows 32w .. 32w+31, two rows per load (lanes 0-15
+// row 2i, lanes 16-31 row 2i+1, 16 bytes each), eight loads in flight at a time;
+// lane l owns dimensions 8(l%16) .. 8(l%16)+7. The amax pass reads the rows
+// again (from L1 / L2). Means use the int64 fixed-point sum; the residual amax
+// is merged into amax[bh] with an integer atomicMax on the (non-negative) fp32
+// bits.
 template <typename T>
 __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ v, int S, int H,
                                                           const int32_t* __restrict__ perm,
                                                           float* __restrict__ mu,
                                                           unsigned int* __restrict__ amax) {
-  __shared__ long long wsum[4][kD];
+  __shared__ long long wsum[8][kD];
   __shared__ float smu[kD];
   __shared__ float wmax[4];
   const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int half = lane >> 4, c = lane & 15;
   const int p0 = blk * kBlock, cnt = min(kBlock, S - p0);
   const size_t row_stride = (size_t)H * kD;
-  const T* vbase = v + ((size_t)b * S * H + h) * kD;
+  const T* vbase = v + ((size_t)b * S * H + h) * kD + c * 8;
   const int32_t* pbase = perm + (size_t)bh * S + p0;
 
-  long long acc[4] = {0, 0, 0, 0};
-  for (int r = warp; r < cnt; r += 4) {
-    const int src = pbase[r];
-    float f[4];
-    unpack4<T>(*reinterpret_cast<const uint2*>(vbase + (size_t)src * row_stride + lane * 4), f);
+  // rows warp*32 + i0*2 + 2i + half, i < 8 (rows past cnt read as 0)
+  auto load8 = [&](int i0, uint4* x) {
+    int src[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[e] += __float2ll_rn(f[e] * 16777216.0f);
+    for (int i = 0; i < 8; ++i) {
+      const int r = warp * 32 + 2 * (i0 + i) + half;
+      src[i] = r < cnt ? pbase[r] : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      x[i] = src[i] >= 0 ? *reinterpret_cast<const uint4*>(vbase + (size_t)src[i] * row_stride)
+                         : make_uint4(0u, 0u, 0u, 0u);
+  };
+  long long acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll 1
+  for (int i0 = 0; i0 < 16; i0 += 8) {
+    uint4 x[8];
+    load8(i0, x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float f[8];
+      unpack8<T>(x[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __float2ll_rn(f[e] * 16777216.0f);
+    }
   }
 #pragma unroll
-  for (int e = 0; e < 4; ++e) wsum[warp][lane * 4 + e] = acc[e];
+  for (int e = 0; e < 8; ++e) wsum[warp * 2 + half][c * 8 + e] = acc[e];
   __syncthreads();
   {
     const int d = tid;
-    const long long s = wsum[0][d] + wsum[1][d] + wsum[2][d] + wsum[3][d];
+    long long s = 0;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) s += wsum[g][d];
     const float m = __double2float_rn(__ddiv_rn((double)s * 5.9604644775390625e-08, (double)cnt));
     smu[d] = m;
     mu[((size_t)bh * gridDim.x + blk) * kD + d] = m;
   }
   __syncthreads();
-  float mx = 0.0f;
-  for (int r = warp; r < cnt; r += 4) {
-    const int src = pbase[r];
-    float f[4];
-    unpack4<T>(*reinterpret_cast<const uint2*>(vbase + (size_t)src * row_stride + lane * 4), f);
+  float m8[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fabsf(__fsub_rn(f[e], smu[lane * 4 + e])));
+  for (int e = 0; e < 8; ++e) m8[e] = smu[c * 8 + e];
+  float mx = 0.0f;
+#pragma unroll 1
+  for (int i0 = 0; i0 < 16; i0 += 8) {
+    uint4 x[8];
+    load8(i0, x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (warp * 32 + 2 * (i0 + i) + half >= cnt) continue;
+      float f[8];
+      unpack8<T>(x[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(__fsub_rn(f[e], m8[e])));
+    }
   }
   mx = warp_max(mx);
   if (lane == 0) wmax[warp] = mx;
@@ -579,15 +612,25 @@ __global__ void __launch_bounds__(256) residual_e4m3_kernel(const T* __restrict_
     m8[0] = m0.x; m8[1] = m0.y; m8[2] = m0.z; m8[3] = m0.w;
     m8[4] = m1.x; m8[5] = m1.y; m8[6] = m1.z; m8[7] = m1.w;
   }
+  // the 8 row indices, then the 8 row loads, all in flight before the first use
+  int src[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int p = blk * kBlock + warp * 16 + 2 * i + half;
+    src[i] = p < S && !zero ? perm[(size_t)bh * S + p] : -1;
+  }
+  uint4 xs[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    xs[i] = src[i] >= 0 ? *reinterpret_cast<const uint4*>(v + (((size_t)b * S + src[i]) * H + h) * kD + c * 8)
+                        : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int r = warp * 16 + 2 * i + half;
-    const int p = blk * kBlock + r;
     uint2 w = make_uint2(0u, 0u);
-    if (p < S && !zero) {
-      const uint4 x = *reinterpret_cast<const uint4*>(v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD + c * 8);
+    if (src[i] >= 0) {
       float f[8];
-      unpack8<T>(x, f);
+      unpack8<T>(xs[i], f);
       float rr[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) rr[e] = __fmul_rn(__fsub_rn(f[e], m8[e]), inv);
@@ -688,20 +731,25 @@ __global__ void __launch_bounds__(256) quant_qk_kernel(const T* __restrict__ q, 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int half = lane >> 4, c = lane & 15;  // row parity and 16-byte piece of the row
   const T* const src = is_k ? k : q;
-  uint4 x[8];
-  float mx = 0.0f;
+  // the 8 row indices, then the 8 row loads, all in flight before the first use
+  int row[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int p = blk * kBlock + warp * 16 + 2 * i + half;
-    x[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (p < S) {
-      const int row = is_k ? perm[(size_t)bh * S + p] : p;
-      x[i] = *reinterpret_cast<const uint4*>(src + (((size_t)b * S + row) * H + h) * kD + c * 8);
-      float f[8];
-      unpack8<T>(x[i], f);
+    row[i] = p < S ? (is_k ? perm[(size_t)bh * S + p] : p) : -1;
+  }
+  uint4 x[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
-    }
+  for (int i = 0; i < 8; ++i)
+    x[i] = row[i] >= 0 ? *reinterpret_cast<const uint4*>(src + (((size_t)b * S + row[i]) * H + h) * kD + c * 8)
+                       : make_uint4(0u, 0u, 0u, 0u);
+  float mx = 0.0f;  // rows past S are 0
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float f[8];
+    unpack8<T>(x[i], f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
   }
   mx = warp_max(mx);
   if (lane == 0) wmax[warp] = mx;
