@@ -509,7 +509,10 @@ def prepare_v_head(V, k, iters, seed, bh, fmt="e4m3", adopt=None, mode="vsmooth"
     -> residual quantisation ([ABS], [HF], [NUN]).
 
     mode "vsmooth" is the method; "meanonly" skips the clustering (identity
-    permutation) and keeps the block means, for the residual-energy comparison.
+    permutation) and keeps the block means, for the residual-energy comparison;
+    "naive" is the baseline the method improves on ([ABS]: low-bit V without
+    smoothing): identity order and no block means, so V itself is quantised with
+    the per-(b, h) scale.
     """
     V = np.asarray(V, np.float32)
     S = V.shape[0]
@@ -518,11 +521,11 @@ def prepare_v_head(V, k, iters, seed, bh, fmt="e4m3", adopt=None, mode="vsmooth"
         a, C, hist, stats = kmeans_lloyd(V, k, iters, seed, bh, adopt=adopt)
         out.update(assign=a, centroids=C, history=hist, stats=stats)
         perm = cluster_permutation(a)
-    elif mode == "meanonly":
+    elif mode in ("meanonly", "naive"):
         perm = np.arange(S, dtype=np.int32)
     else:
         raise ValueError(mode)
-    mu = block_means(V, perm)
+    mu = block_means(V, perm) if mode != "naive" else np.zeros((num_blocks(S), V.shape[1]), np.float32)
     out.update(perm=perm, mu=mu)
     if fmt == "e4m3":
         vt, s_v, amax = residual_e4m3(V, perm, mu)

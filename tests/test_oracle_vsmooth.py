@@ -198,3 +198,22 @@ def test_quant_blocks_scales_codes_and_zero_block():
         # E4M3 keeps 3 mantissa bits: relative error <= 2^-4 (normals), plus the
         # subnormal half-step
         assert np.all(np.abs(deq - Xp[lo:hi]) <= 2.0 ** -4 * np.abs(Xp[lo:hi]) + 2.0 ** -10 * scales[b] + 1e-30)
+
+
+def test_naive_mode_is_v_itself_with_one_scale_per_head():
+    # the baseline without smoothing: identity order, no means, and the decoded
+    # residual equals the direct per-head E4M3 quantisation of V (a separate
+    # routine), which is within half an E4M3 step of every value
+    g = torch.Generator().manual_seed(11)
+    V = (torch.randn(300, 128, generator=g) * 3 + 5).to(torch.bfloat16).float().numpy()
+    out = O.prepare_v_head(V, 16, 4, 0, 0, mode="naive")
+    assert np.array_equal(out["perm"], np.arange(300))
+    assert not out["mu"].any()
+    direct, s_v = O.naive_v_e4m3(V)
+    assert out["s_v"] == s_v == np.float32(np.abs(V).max() / 448)
+    assert np.array_equal(out["vres"], direct)
+    # E4M3: half a mantissa step (|v| / 16) for normals, half the 2^-9 step below
+    assert np.all(np.abs(direct - V) <= np.abs(V) / 16 + float(s_v) * 2.0 ** -10)
+    # with a common offset in V, the block means of V-Smooth shrink the range to code
+    vs = O.prepare_v_head(V, 16, 4, 0, 0)
+    assert vs["s_v"] < out["s_v"]
