@@ -343,7 +343,14 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
     # accuracy on sampled rows of two heads: rel-L2 against exact attention in fp64
     o = plan.run(Q, K, V).float()
     rows = torch.linspace(0, S - 1, 64, device=dev).long()
-    num = den = 0.0
+    o_naive = None
+    if "accuracy" in legs:
+        # the unsmoothed baseline: the same call with V quantised as it is (one scale per head)
+        naive = vc_attn.Plan(B, S, H, k=cfg["k"], iters=cfg["iters"], fmt=cfg["fmt"], k_p=args.k_p, device=dev,
+                             mode="naive")
+        o_naive = naive.run(Q, K, V).float()[0, rows]
+        del naive
+    num = den = num_naive = 0.0
     for h in (0, H - 1):
         q = Q[0, rows, h].double()
         k, v = K[0, :, h].double(), V[0, :, h].double()
@@ -351,10 +358,14 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
         ref = p @ v
         num += float(((o[0, rows, h].double() - ref) ** 2).sum())
         den += float((ref ** 2).sum())
+        if o_naive is not None:
+            num_naive += float(((o_naive[:, h].double() - ref) ** 2).sum())
         del k, v, p
     if "accuracy" in legs:
         out["rel_l2_vs_fp64"] = math.sqrt(num / den)
-        out["accuracy_sample"] = "64 query rows x heads {0, H-1} of batch 0, exact fp64 softmax attention on the GPU"
+        out["naive_v_rel_l2_vs_fp64"] = math.sqrt(num_naive / den)
+        out["accuracy_sample"] = ("64 query rows x heads {0, H-1} of batch 0, exact fp64 softmax attention on the "
+                                  "GPU; naive_v: the same path with V-Smooth off (V itself, one E4M3 scale per head)")
     # the comparison kernel: the same fused attention with the probabilities made
     # by exp2 on the special function unit and an E4M3 conversion instead of
     # ExpCast (same prepared inputs, same stream)

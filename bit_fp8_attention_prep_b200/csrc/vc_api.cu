@@ -11,11 +11,23 @@
 #include <mutex>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/vc_attn.h"
 #include "../../include/vc_attn_testing.h"
 #include "vc_kernels.h"
 
 namespace {
+
+// An NVTX range over the host side of an ABI call (a profiler's timeline shows
+// which call enqueued which kernels). NVTX is header-only: without a tool
+// attached a range costs a few nanoseconds.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 thread_local std::string g_last_error;
 std::atomic<uint64_t> g_launches{0};  // kernels enqueued by this library since load
@@ -52,8 +64,9 @@ vc_status_t check_shape(const vc_shape_t* sh) {
 
 vc_status_t check_cfg(const vc_vsmooth_cfg_t* cfg) {
   if (!cfg) return fail(VC_ERR_INVALID_ARG, "cfg is NULL");
-  if (cfg->mode != VC_MODE_VSMOOTH && cfg->mode != VC_MODE_MEANONLY)
-    return fail(VC_ERR_INVALID_ARG, "mode must be VC_MODE_VSMOOTH or VC_MODE_MEANONLY (got %d)", cfg->mode);
+  if (cfg->mode != VC_MODE_VSMOOTH && cfg->mode != VC_MODE_MEANONLY && cfg->mode != VC_MODE_NAIVE)
+    return fail(VC_ERR_INVALID_ARG, "mode must be VC_MODE_VSMOOTH, VC_MODE_MEANONLY or VC_MODE_NAIVE (got %d)",
+                cfg->mode);
   if (cfg->mode == VC_MODE_VSMOOTH) {
     if (cfg->k < 1 || cfg->k > vc::kMaxClusters)
       return fail(VC_ERR_INVALID_ARG, "k must be in [1, %d] (got %d)", vc::kMaxClusters, cfg->k);
@@ -223,12 +236,14 @@ extern "C" {
 vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
                               const vc_prepared_v_t* out, void* workspace, size_t workspace_bytes,
                               uint8_t* assign_history, void* stream) {
+  NvtxRange range("vc_attn_prepare_v");
   g_last_error.clear();
   return prepare_v_impl(v, shape, cfg, out, workspace, workspace_bytes, assign_history, stream, 0);
 }
 
 vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* shape, const int32_t* perm,
                              const vc_qk_fp8_t* out, void* stream) {
+  NvtxRange range("vc_attn_quant_qk");
   g_last_error.clear();
   vc_status_t st;
   if ((st = check_shape(shape)) != VC_OK) return st;
@@ -311,6 +326,7 @@ static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* 
 
 vc_status_t vc_attn_forward(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                             float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
+  NvtxRange range("vc_attn_forward");
   return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, false, nullptr, 0);
 }
 
@@ -327,6 +343,7 @@ size_t vc_attn_forward_nvfp4v_workspace_bytes(const vc_shape_t* shape) {
 vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                                    float softmax_scale, int32_t k_p, void* o, void* workspace,
                                    size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  NvtxRange range("vc_attn_forward_nvfp4v");
   return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, true, workspace,
                         workspace_bytes);
 }
@@ -349,6 +366,7 @@ extern "C" {
 
 vc_status_t vc_attn_prepare_v_noalloc(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
                                       const vc_prepared_v_t* out, uint8_t* assign_history, void* stream) {
+  NvtxRange range("vc_attn_prepare_v_noalloc");
   g_last_error.clear();
   vc_status_t st;
   if ((st = check_shape(shape)) != VC_OK) return st;
@@ -486,6 +504,7 @@ vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const 
                              const vc_vsmooth_cfg_t* cfg, float softmax_scale, int32_t k_p, void* o,
                              int32_t head_chunk, void* workspace, size_t workspace_bytes, int32_t* dev_status,
                              void* stream) {
+  NvtxRange range("vc_attn_run_host");
   g_last_error.clear();
   vc_status_t st;
   if ((st = check_shape(shape)) != VC_OK) return st;

@@ -496,12 +496,12 @@ __global__ void identity_perm_kernel(int S, int32_t* __restrict__ perm) {
 // quant_qk_kernel: warp w takes rows 32w .. 32w+31, two rows per load (lanes 0-15
 // row 2i, lanes 16-31 row 2i+1, 16 bytes each), eight loads in flight at a time;
 // lane l owns dimensions 8(l%16) .. 8(l%16)+7. The amax pass reads the rows
-// again (from L1 / L2). Means use the int64 fixed-point sum; the residual amax
-// is merged into amax[bh] with an integer atomicMax on the (non-negative) fp32
-// bits.
+// again (from L1 / L2). Means use the int64 fixed-point sum (naive mode: all
+// means are 0 and the first pass is skipped); the residual amax is merged into
+// amax[bh] with an integer atomicMax on the (non-negative) fp32 bits.
 template <typename T>
 __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ v, int S, int H,
-                                                          const int32_t* __restrict__ perm,
+                                                          const int32_t* __restrict__ perm, bool naive,
                                                           float* __restrict__ mu,
                                                           unsigned int* __restrict__ amax) {
   __shared__ long long wsum[8][kD];
@@ -530,7 +530,7 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ 
   };
   long long acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll 1
-  for (int i0 = 0; i0 < 16; i0 += 8) {
+  for (int i0 = 0; i0 < (naive ? 0 : 16); i0 += 8) {
     uint4 x[8];
     load8(i0, x);
 #pragma unroll
@@ -549,7 +549,7 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ 
     long long s = 0;
 #pragma unroll
     for (int g = 0; g < 8; ++g) s += wsum[g][d];
-    const float m = __double2float_rn(__ddiv_rn((double)s * 5.9604644775390625e-08, (double)cnt));
+    const float m = naive ? 0.0f : __double2float_rn(__ddiv_rn((double)s * 5.9604644775390625e-08, (double)cnt));
     smu[d] = m;
     mu[((size_t)bh * gridDim.x + blk) * kD + d] = m;
   }
@@ -872,7 +872,7 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
     ++n;
   }
   const dim3 gb(pl.nb, BH);
-  block_stats_kernel<T><<<gb, 128, 0, st>>>(v, S, H, out.perm, out.mu, pl.amax);
+  block_stats_kernel<T><<<gb, 128, 0, st>>>(v, S, H, out.perm, pl.mode == VC_MODE_NAIVE, out.mu, pl.amax);
   if (pl.fmt == VC_RESIDUAL_E4M3) {
     residual_e4m3_kernel<T><<<gb, 256, 0, st>>>(v, S, H, pl.S_pad, out.perm, out.mu, pl.amax, out.v_codes,
                                                 out.s_v);

@@ -19,7 +19,8 @@ STATUS_NAMES = ["VC_OK", "VC_ERR_INVALID_ARG", "VC_ERR_UNSUPPORTED", "VC_ERR_WOR
                 "VC_ERR_TIMEOUT"]
 VC_DTYPE_F16, VC_DTYPE_BF16 = 0, 1
 VC_RESIDUAL_E4M3, VC_RESIDUAL_NVFP4 = 0, 1
-VC_MODE_VSMOOTH, VC_MODE_MEANONLY = 0, 1
+VC_MODE_VSMOOTH, VC_MODE_MEANONLY, VC_MODE_NAIVE = 0, 1, 2
+_MODES = {"vsmooth": VC_MODE_VSMOOTH, "meanonly": VC_MODE_MEANONLY, "naive": VC_MODE_NAIVE}
 
 # every symbol declared in include/vc_attn.h and include/vc_attn_testing.h
 ABI_SYMBOLS = [
@@ -149,7 +150,7 @@ def prepare_v(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", history=Fals
     lib = load()
     sh = shape_of(v)
     cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
-                     VC_MODE_MEANONLY if mode == "meanonly" else VC_MODE_VSMOOTH)
+                     _MODES[mode])
     B, S, H = sh.B, sh.S, sh.H
     nb = num_blocks(S)
     Sp = nb * 128
@@ -187,7 +188,7 @@ def prepare_v_noalloc(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", hist
     lib = load()
     sh = shape_of(v)
     cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
-                     VC_MODE_MEANONLY if mode == "meanonly" else VC_MODE_VSMOOTH)
+                     _MODES[mode])
     B, S, H = sh.B, sh.S, sh.H
     nb = num_blocks(S)
     Sp = nb * 128
@@ -286,7 +287,7 @@ class Plan:
         dev = torch.device(device if device is not None else "cuda")
         self.shape = Shape(B, S, H, 128, VC_DTYPE_BF16 if dtype == torch.bfloat16 else VC_DTYPE_F16)
         self.cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
-                              VC_MODE_MEANONLY if mode == "meanonly" else VC_MODE_VSMOOTH)
+                              _MODES[mode])
         self.fmt, self.k_p = fmt, int(k_p)
         self.softmax_scale = 1.0 / math.sqrt(128) if softmax_scale is None else float(softmax_scale)
         nb = num_blocks(S)
@@ -355,7 +356,7 @@ class HostPlan:
         self.dtype = dtype
         self.shape = Shape(B, S, H, 128, VC_DTYPE_BF16 if dtype == torch.bfloat16 else VC_DTYPE_F16)
         self.cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
-                              VC_MODE_MEANONLY if mode == "meanonly" else VC_MODE_VSMOOTH)
+                              _MODES[mode])
         self.k_p, self.head_chunk = int(k_p), int(head_chunk)
         self.softmax_scale = 1.0 / math.sqrt(128) if softmax_scale is None else float(softmax_scale)
         self.ws_bytes = self.lib.vc_attn_run_host_workspace_bytes(ctypes.byref(self.shape), ctypes.byref(self.cfg),

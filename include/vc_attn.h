@@ -55,7 +55,9 @@ typedef enum { VC_DTYPE_F16 = 0, VC_DTYPE_BF16 = 1 } vc_dtype_t;
 typedef enum { VC_RESIDUAL_E4M3 = 0, VC_RESIDUAL_NVFP4 = 1 } vc_residual_fmt_t;
 typedef enum {
   VC_MODE_VSMOOTH = 0,      /* k-means + cluster sort + block means (the method)  */
-  VC_MODE_MEANONLY = 1      /* identity order, block means only (diagnostic)      */
+  VC_MODE_MEANONLY = 1,     /* identity order, block means only (diagnostic)      */
+  VC_MODE_NAIVE = 2         /* identity order, no block means: V itself at one scale
+                               per (b, h), the unsmoothed baseline (diagnostic)    */
 } vc_mode_t;
 
 /* Problem shape. D must be 128. dtype is a vc_dtype_t for Q, K and V. */
@@ -125,6 +127,9 @@ size_t vc_attn_prepare_v_workspace_bytes(const vc_shape_t* shape, const vc_vsmoo
  * (the permutation also applied to K by vc_attn_quant_qk), subtraction of each
  * 128-token block's mean, and quantisation of the residual to E4M3 (one scale per
  * (b, h)) or NVFP4 (E2M1 + E4M3 scale per 16 tokens + fp32 global per (b, h)).
+ * cfg->mode VC_MODE_MEANONLY keeps the original order (perm = identity);
+ * VC_MODE_NAIVE also writes all block means as 0, so V itself is quantised (the
+ * baseline the method improves on; vc_attn_forward then adds no mean).
  *  v               device, [B,S,H,128] of shape->dtype
  *  out             fields as documented in vc_prepared_v_t (v_scales only NVFP4)
  *  workspace       device, >= vc_attn_prepare_v_workspace_bytes(), 256-B aligned;

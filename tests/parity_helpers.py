@@ -17,10 +17,10 @@ def head(X, b, h):
     return X[b, :, h].float().numpy()
 
 
-def gpu_pipeline(va, Q, K, V, k, iters, seed=0, fmt="e4m3", k_p=8, history=True, attend=True):
+def gpu_pipeline(va, Q, K, V, k, iters, seed=0, fmt="e4m3", k_p=8, history=True, attend=True, mode="vsmooth"):
     """Q, K, V CPU tensors [B,S,H,128] -> dict of GPU outputs copied to the CPU."""
     q, kk, v = Q.cuda(), K.cuda(), V.cuda()
-    pv = va.prepare_v(v, k=k, iters=iters, seed=seed, fmt=fmt, history=history)
+    pv = va.prepare_v(v, k=k, iters=iters, seed=seed, fmt=fmt, history=history, mode=mode)
     qk = va.quant_qk(q, kk, pv["perm"])
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     o = va.forward(qk, pv, va.shape_of(q), SCALE, k_p, status=status) if attend else None

@@ -97,3 +97,19 @@ def test_prep_exact_ties(va):
         ref = oracle_head(g, Q, K, V, 0, h, 8, 3)
         assert ref["stats"]["near_ties"] == 0, ref["stats"]   # exact ties: both sides take the lowest index
         assert_prep_bit_exact(g, ref, 0, h)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "nvfp4"])
+def test_naive_mode(va, fmt):
+    # no reordering and no block means: the codes are V's own, one scale per head
+    cfg, Q, K, V = make("mid", B=1, H=2, S=400)
+    g = gpu_pipeline(va, Q, K, V, 16, 4, fmt=fmt, history=False, attend=False, mode="naive")
+    for h in range(2):
+        ref = O.prepare_v_head(V[0, :, h].float().numpy(), 16, 4, 0, h, fmt=fmt, mode="naive")
+        assert np.array_equal(g["perm"][0, h], ref["perm"])
+        assert not g["mu"][0, h].any()
+        assert np.array_equal(g["v_codes"][0, h], ref["v_codes"])
+        if fmt == "e4m3":
+            assert g["s_v"][0, h] == ref["s_v"]
+        else:
+            assert np.array_equal(g["v_scales"][0, h], ref["v_scales"]) and g["s_v"][0, h] == ref["g"]
