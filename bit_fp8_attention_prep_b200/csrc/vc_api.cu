@@ -10,6 +10,8 @@
 #include <atomic>
 #include <mutex>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -545,10 +547,24 @@ vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const 
   if ((e = cudaStreamWaitEvent(s_out, ev.start, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
   if ((e = cudaStreamWaitEvent(s_odd, ev.start, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
   const cudaStream_t comp_stream[2] = {cs_stream, s_odd};
-  int c = 0;
+  // Chunks of hc heads of one batch entry; the first and the last chunk of the
+  // call take a single head, so that the copy-in before the first compute and
+  // the copy-out after the last one (neither overlaps anything) are short.
+  std::vector<std::pair<int, int>> chunks;  // (b * H + h0, heads)
   for (int b = 0; b < B; ++b)
-    for (int h0 = 0; h0 < H; h0 += hc, ++c) {
-      const int n = hc < H - h0 ? hc : H - h0, slot = c & 1;
+    for (int h0 = 0; h0 < H; h0 += hc) chunks.emplace_back(b * H + h0, hc < H - h0 ? hc : H - h0);
+  if (chunks.front().second > 1) {
+    chunks.front().second -= 1;
+    chunks.front().first += 1;
+    chunks.insert(chunks.begin(), std::make_pair(chunks.front().first - 1, 1));
+  }
+  if (chunks.size() > 1 && chunks.back().second > 1) {
+    chunks.back().second -= 1;
+    chunks.emplace_back(chunks.back().first + chunks.back().second, 1);
+  }
+  for (int c = 0; c < (int)chunks.size(); ++c) {
+    {
+      const int b = chunks[c].first / H, h0 = chunks[c].first % H, n = chunks[c].second, slot = c & 1;
       const size_t host_off = ((size_t)b * S * H + h0) * 256, crow = (size_t)n * 256;
       vc_shape_t cs = *shape;
       cs.B = 1;
@@ -594,6 +610,7 @@ vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const 
         return cuda_fail(e, "copying an output chunk to the host");
       if ((e = cudaEventRecord(ev.out[slot], s_out)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
+  }
   // the caller's stream passes this point once the last output chunk is on the host
   if ((e = cudaEventRecord(ev.done, s_out)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if ((e = cudaStreamWaitEvent(cs_stream, ev.done, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");

@@ -240,7 +240,8 @@ size_t vc_attn_run_host_workspace_bytes(const vc_shape_t* shape, const vc_vsmoot
  * internal stream (odd chunks, so that one chunk's last wave of attention CTAs
  * shares the GPU with the next chunk's kernels), and its O rows are copied back
  * on a third internal stream, while the next chunks' inputs are already being
- * copied in. The output is bit-identical to the three device calls on the whole
+ * copied in. The first and the last chunk of the call take a single head, so
+ * that the copies that cannot overlap any compute are short. The output is bit-identical to the three device calls on the whole
  * problem (each chunk's k-means is seeded by the slice's index in the whole
  * problem).
  *  q, k, v       HOST, [B,S,H,128] of shape->dtype. Page-locked memory
