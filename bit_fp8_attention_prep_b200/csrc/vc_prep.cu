@@ -81,15 +81,20 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(const T* __restrict__ 
 //    the answer. The rest (a near tie) are compared by the direct form, lowest
 //    index on ties, which is the answer the direct form over all centroids
 //    gives.
-//  - Accumulation (kAccum): the tile's tokens are put in cluster order (a
-//    counting sort: match_any ranks within each warp, offsets across warps) as
-//    words holding the row's offset and its cluster. Thread d walks column d in
-//    that order, eight entries at a time (the loads and the llrint(x_d * 2^24)
-//    conversions of the eight are independent), keeps an int64 running sum and
-//    adds it to the CTA's accumulator of the cluster where the cluster changes,
-//    at the same positions for every thread. Thread d owns column d of the
-//    accumulators, so no atomics are needed until the chunk's sums go to global
-//    memory.
+//  - Accumulation (kAccum): sums[c] and counts[c] are running totals over the
+//    whole (b, h) of the int64 llrint(x * 2^24) and of the tokens assigned to c.
+//    The first accumulating pass adds every token to its cluster; a later
+//    ("delta") pass reads each token's previous cluster before overwriting it
+//    and, for the tokens that moved, adds x to the new cluster and subtracts it
+//    from the old one (exact integer arithmetic, so the totals equal a fresh
+//    sum). The tile's entries go into cluster order (a counting sort: match_any
+//    ranks within each warp, offsets across warps and the two signs; the order
+//    within a cluster does not matter), as words holding the row's offset, the
+//    cluster and the sign. Thread d walks column d
+//    in that order, eight entries at a time, keeps an int64 running sum and adds
+//    it to the CTA's accumulator of the cluster where the cluster changes, at the
+//    same positions for every thread; no atomics until the chunk's totals go to
+//    global memory.
 constexpr int kTile = 128;
 
 // Staged tile rows. The accumulating pass pads rows to 272 bytes (its column
@@ -161,7 +166,7 @@ __device__ __noinline__ int nearest_direct(const uint8_t* tile, int r, const flo
 
 template <typename T, bool kAccum, int KC>
 __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restrict__ v, int S, int H, int k,
-                                                              const float* __restrict__ cent,
+                                                              bool delta, const float* __restrict__ cent,
                                                               unsigned long long* __restrict__ sums,
                                                               int* __restrict__ counts, uint8_t* __restrict__ assign,
                                                               int* __restrict__ hist, uint8_t* __restrict__ history) {
@@ -176,9 +181,9 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
   float* kns = ncs + KC;                                                               // [KC]: 2^-15 |c - r|^2
   float* gsm = kns + KC;                                                               // [kTile][KC + 1]: g_c
   uint8_t* tile = reinterpret_cast<uint8_t*>(gsm + kTile * (KC + 1));                   // staged rows
-  uint32_t* sent = reinterpret_cast<uint32_t*>(tile + tile_bytes<kPad>());             // [kTile]: sorted rows
-  int* scount = reinterpret_cast<int*>(sent + kTile);                                  // [KC]
-  int* woff = scount + KC;                                                             // [4][KC]
+  uint32_t* sent = reinterpret_cast<uint32_t*>(tile + tile_bytes<kPad>());             // [2 kTile]: sorted entries
+  int* scount = reinterpret_cast<int*>(sent + 2 * kTile);                              // [KC]
+  int* woff = scount + KC;                                                             // [2][4][KC] + 1
 
   const int bh = blockIdx.y, b = bh / H, h = bh % H;
   const int chunk = blockIdx.x;
@@ -244,7 +249,8 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
         *reinterpret_cast<uint4*>(tile + tile_off<kPad>(r, c)) = val;
       }
     }
-    if (kAccum && tid < 4 * KC) woff[tid] = 0;
+    if (kAccum)
+      for (int i = tid; i < 8 * KC; i += kTile) woff[i] = 0;
     __syncthreads();
     // proxies g_c of tokens t and t + 64 (rows past ntok hold stale data; unused)
     float2 ga[kHalfC], gb[kHalfC];
@@ -291,7 +297,7 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
       }
     __syncthreads();
     const bool valid = tid < ntok;
-    int best = 0;
+    int best = 0, prev = -1;  // prev: this token's cluster in the previous pass (delta passes)
     if (valid) {
       const float* g = gsm + tid * (KC + 1);
       float g_best = g[0];
@@ -306,22 +312,38 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
       for (int c = 0; c < k; ++c)
         if (c != best && !(g[c] - kns[c] > lim)) near |= 1u << c;
       if (near != 0u) best = nearest_direct<T, kPad>(tile, tid, cg, near | (1u << best));
+      if (kAccum && delta) prev = assign[(size_t)bh * S + s0 + tid];
       assign[(size_t)bh * S + s0 + tid] = (uint8_t)best;
       if (history) history[(size_t)bh * S + s0 + tid] = (uint8_t)best;
-      atomicAdd(&scount[best], 1);
+      if (!(kAccum && delta)) {
+        atomicAdd(&scount[best], 1);
+      } else if (prev != best) {
+        atomicAdd(&scount[best], 1);
+        atomicAdd(&scount[prev], -1);
+      }
     }
     if (kAccum) {
-      // counting sort of the tile by cluster (stable is not needed for a sum)
-      const int a = valid ? best : 0xFF;
-      const unsigned peers = __match_any_sync(0xffffffffu, a);
-      const int rank = __popc(peers & ((1u << lane) - 1u));
-      if (valid && rank == 0) woff[warp * KC + a] = __popc(peers);
+      // The tile's entries: +x to the token's cluster for every token (first
+      // pass), or, in a delta pass, +x to the new and -x to the old cluster of
+      // every token that moved. Counting sort of the entries by cluster (the order
+      // within a cluster does not matter for an exact sum): per-cluster counts,
+      // their exclusive scan, then each entry takes the next slot of its cluster.
+      // ranks within each warp by match_any, for the + entries (round 0) and the
+      // - entries (round 1); woff[round][warp][c] becomes the first slot of
+      // cluster c's entries of that round and warp
+      const bool add = valid && (!delta || prev != best), sub = valid && delta && prev != best;
+      const unsigned pa = __match_any_sync(0xffffffffu, add ? best : 0xFF);
+      const unsigned ps = __match_any_sync(0xffffffffu, sub ? prev : 0xFF);
+      const int ra = __popc(pa & ((1u << lane) - 1u)), rs = __popc(ps & ((1u << lane) - 1u));
+      if (add && ra == 0) woff[(0 * 4 + warp) * KC + best] = __popc(pa);
+      if (sub && rs == 0) woff[(1 * 4 + warp) * KC + prev] = __popc(ps);
       __syncthreads();
       if (tid < 32) {
-        int tot = 0, w0 = 0, w1 = 0, w2 = 0, w3 = 0;
-        if (tid < KC) {
-          w0 = woff[0 * KC + tid]; w1 = woff[1 * KC + tid]; w2 = woff[2 * KC + tid]; w3 = woff[3 * KC + tid];
-          tot = w0 + w1 + w2 + w3;
+        int w[8], tot = 0;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          w[g] = tid < KC ? woff[g * KC + tid] : 0;
+          tot += w[g];
         }
         int incl = tot;
 #pragma unroll
@@ -330,53 +352,66 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
           if (tid >= o) incl += t2;
         }
         if (tid < KC) {
-          const int base = incl - tot;
-          woff[0 * KC + tid] = base;
-          woff[1 * KC + tid] = base + w0;
-          woff[2 * KC + tid] = base + w0 + w1;
-          woff[3 * KC + tid] = base + w0 + w1 + w2;
+          int base = incl - tot;
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            woff[g * KC + tid] = base;
+            base += w[g];
+          }
         }
+        if (tid == 31) woff[8 * KC] = incl;  // number of entries
       }
       __syncthreads();
-      if (valid) sent[woff[warp * KC + best] + rank] = (uint32_t)(tid * 272) | ((uint32_t)best << 16);
+      const uint32_t row_word = (uint32_t)(tid * 272);
+      if (add) sent[woff[(0 * 4 + warp) * KC + best] + ra] = row_word | ((uint32_t)best << 16);
+      if (sub) sent[woff[(1 * 4 + warp) * KC + prev] + rs] = row_word | ((uint32_t)prev << 16) | 0x80000000u;
       __syncthreads();
-      // thread d: column d of the tile in cluster order; the running sum goes to
-      // the cluster's accumulator where the cluster changes (the same place for
+      const int nent = woff[8 * KC];
+      // thread d: column d over the entries in cluster order; the running sum goes
+      // to the cluster's accumulator where the cluster changes (the same place for
       // every thread)
       const int d = tid;
       const uint8_t* col = tile + d * 2;
-      long long run = 0;
-      int cur = (int)(sent[0] >> 16), pos = 0;
-      for (; pos + 8 <= ntok; pos += 8) {
-        const uint4 e0 = *reinterpret_cast<const uint4*>(sent + pos);
-        const uint4 e1 = *reinterpret_cast<const uint4*>(sent + pos + 4);
-        const uint32_t e[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-        long long q[8];
+      // Within a cluster the + entries precede the - entries, so the walk keeps
+      // one unsigned running sum per (cluster, sign) segment and applies the
+      // sign where the segment ends. key = e >> 16: cluster, sign in bit 15.
+      auto flush = [&](uint32_t key, long long run) {
+        acc[(key & 0xFFu) * kD + d] += (key & 0x8000u) ? -run : run;
+      };
+      if (nent > 0) {
+        long long run = 0;
+        uint32_t cur = sent[0] >> 16;
+        int pos = 0;
+        for (; pos + 8 <= nent; pos += 8) {
+          const uint4 e0 = *reinterpret_cast<const uint4*>(sent + pos);
+          const uint4 e1 = *reinterpret_cast<const uint4*>(sent + pos + 4);
+          const uint32_t e[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+          long long q[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)  // x * 2^24, exact
-          q[j] = __float2ll_rn(to_f32<T>(*reinterpret_cast<const T*>(col + (e[j] & 0xffffu))) * 16777216.0f);
+          for (int j = 0; j < 8; ++j)  // x * 2^24, exact
+            q[j] = __float2ll_rn(to_f32<T>(*reinterpret_cast<const T*>(col + (e[j] & 0xffffu))) * 16777216.0f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int lab = (int)(e[j] >> 16);
-          if (lab != cur) {
-            acc[cur * kD + d] += run;
-            run = 0;
-            cur = lab;
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t key = e[j] >> 16;
+            if (key != cur) {
+              flush(cur, run);
+              run = 0;
+              cur = key;
+            }
+            run += q[j];
           }
-          run += q[j];
         }
-      }
-      for (; pos < ntok; ++pos) {
-        const uint32_t e = sent[pos];
-        const int lab = (int)(e >> 16);
-        if (lab != cur) {
-          acc[cur * kD + d] += run;
-          run = 0;
-          cur = lab;
+        for (; pos < nent; ++pos) {
+          const uint32_t e = sent[pos], key = e >> 16;
+          if (key != cur) {
+            flush(cur, run);
+            run = 0;
+            cur = key;
+          }
+          run += __float2ll_rn(to_f32<T>(*reinterpret_cast<const T*>(col + (e & 0xffffu))) * 16777216.0f);
         }
-        run += __float2ll_rn(to_f32<T>(*reinterpret_cast<const T*>(col + (e & 0xffffu))) * 16777216.0f);
+        flush(cur, run);
       }
-      acc[cur * kD + d] += run;
     }
   }
   __syncthreads();
@@ -392,26 +427,29 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
 template <int KC>
 constexpr size_t assign_smem(bool accum) {
   return (accum ? (size_t)KC * kD * 8 : 0) + (size_t)KC * kD * 4 + kD * 4 + 2 * KC * 4 + kTile * (KC + 1) * 4 +
-         (accum ? tile_bytes<true>() : tile_bytes<false>()) + 4 * kTile + 5 * KC * 4;
+         (accum ? tile_bytes<true>() : tile_bytes<false>()) + 8 * kTile + (9 * KC + 4) * 4;
 }
 
 template <typename T, bool kAccum, int KC>
-static void launch_assign(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, uint8_t* hist_t) {
+static void launch_assign(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, bool delta, uint8_t* hist_t) {
   kmeans_assign_kernel<T, kAccum, KC><<<grid, kTile, assign_smem<KC>(kAccum), st>>>(
-      v, pl.S, pl.H, pl.k, pl.cent, pl.sums, pl.counts, pl.assign, kAccum ? nullptr : pl.hist, hist_t);
+      v, pl.S, pl.H, pl.k, delta, pl.cent, pl.sums, pl.counts, pl.assign, kAccum ? nullptr : pl.hist, hist_t);
 }
 
 template <typename T, bool kAccum>
-static void launch_assign_k(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, uint8_t* hist_t) {
+static void launch_assign_k(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, bool delta,
+                            uint8_t* hist_t) {
   if (pl.k <= 8)
-    launch_assign<T, kAccum, 8>(grid, st, v, pl, hist_t);
+    launch_assign<T, kAccum, 8>(grid, st, v, pl, delta, hist_t);
   else if (pl.k <= 16)
-    launch_assign<T, kAccum, 16>(grid, st, v, pl, hist_t);
+    launch_assign<T, kAccum, 16>(grid, st, v, pl, delta, hist_t);
   else
-    launch_assign<T, kAccum, 32>(grid, st, v, pl, hist_t);
+    launch_assign<T, kAccum, 32>(grid, st, v, pl, delta, hist_t);
 }
 
 // --------------------------------------------------------------- centroid update
+// c = (double) sum * 2^-24 / count, rounded to fp32; an empty cluster keeps its
+// centroid. sums and counts stay as running totals for the next delta pass.
 __global__ void __launch_bounds__(128) kmeans_update_kernel(int k, float* __restrict__ cent,
                                                             unsigned long long* __restrict__ sums,
                                                             int* __restrict__ counts) {
@@ -423,10 +461,7 @@ __global__ void __launch_bounds__(128) kmeans_update_kernel(int k, float* __rest
       const double s = (double)(long long)sums[i] * 5.9604644775390625e-08;  // * 2^-24, exact
       cent[i] = __double2float_rn(__ddiv_rn(s, (double)n));
     }
-    sums[i] = 0ull;
   }
-  __syncthreads();
-  if (d < k) counts[(size_t)bh * k + d] = 0;
 }
 
 // --------------------------------------------------------------- stable cluster sort
@@ -856,11 +891,11 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
     for (int it = 0; it < pl.iters; ++it) {
       uint8_t* hist_t = history ? history + (size_t)it * BH * S : nullptr;
       if (it + 1 < pl.iters) {
-        launch_assign_k<T, true>(grid, st, v, pl, hist_t);
+        launch_assign_k<T, true>(grid, st, v, pl, it > 0, hist_t);
         kmeans_update_kernel<<<BH, 128, 0, st>>>(k, pl.cent, pl.sums, pl.counts);
         n += 2;
       } else {
-        launch_assign_k<T, false>(grid, st, v, pl, hist_t);
+        launch_assign_k<T, false>(grid, st, v, pl, false, hist_t);
         ++n;
       }
     }
