@@ -131,6 +131,33 @@ __device__ __forceinline__ bool wait_warp(Smem& s, uint64_t* bar, uint32_t parit
   return __all_sync(0xffffffffu, wait_or_abort(s, bar, parity, P));
 }
 
+// wait_warp for the TMA and MMA-issuing warps: they poll without asking to be
+// suspended, so that an issuing warp sees its barrier complete at once (it is
+// on the critical path between the two query tiles' score hand-overs). Bounded
+// like every wait: the time limit and the CTA's abort flag are checked every 64
+// polls.
+template <class Smem>
+__device__ __forceinline__ bool wait_spin_warp(Smem& s, uint64_t* bar, uint32_t parity, const AttnParams& P) {
+  bool ok = mbar_try_wait(bar, parity);
+  if (!ok) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (mbar_try_wait(bar, parity)) {
+        ok = true;
+        break;
+      }
+      if ((it & 63u) == 0u &&
+          (globaltimer_ns() - t0 > P.wait_ns || *reinterpret_cast<volatile int32_t*>(&s.abort_flag) != 0))
+        break;
+    }
+    if (!ok) {
+      s.abort_flag = 1;
+      report_status(P.status, VC_ERR_TIMEOUT);
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Byte offset of 16-bit element `slot` (K index 16*chunk + slot) of row `row` in
 // a 128-B-swizzled K-major operand tile (rows of 128 B, 8-row atoms).
 __device__ __forceinline__ uint32_t sw128_off16(int row, int chunk, int slot) {
@@ -275,14 +302,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int k_issued = 0, v_issued = 0;
     for (int j = 0; j < nkv && !*(volatile int32_t*)&s.abort_flag; ++j) {
       const int ks = j % kKStages;
-      if (!wait_warp(s, &s.k_empty[ks], ((j / kKStages) & 1) ^ 1, P)) break;
+      if (!wait_spin_warp(s, &s.k_empty[ks], ((j / kKStages) & 1) ^ 1, P)) break;
       if (leader) {
         mbar_arrive_expect_tx(&s.k_full[ks], kTileBytes);
         tma_load_2d(s.k[ks], &tmK, &s.k_full[ks], 0, bh * P.S_pad + j * 128);
       }
       k_issued = j + 1;
       const int vs = j % kVStages;
-      if (!wait_warp(s, &s.v_empty[vs], ((j / kVStages) & 1) ^ 1, P)) break;
+      if (!wait_spin_warp(s, &s.v_empty[vs], ((j / kVStages) & 1) ^ 1, P)) break;
       if (leader) {
         mbar_arrive_expect_tx(&s.v_full[vs], kPlanes * kTileBytes);
         // plane pl of head bh: rows (pl * BH + bh) * 128
@@ -295,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // M operand of batch n = j / kMeanBlocks: slots (hi, lo, hi) of mu_b / s_V
         // for its blocks, zero for blocks past the end and for slot 15
         const int n = j / kMeanBlocks, mb = n & 1;
-        if (!wait_warp(s, &s.m_empty[mb], ((n >> 1) & 1) ^ 1, P)) break;
+        if (!wait_spin_warp(s, &s.m_empty[mb], ((n >> 1) & 1) ^ 1, P)) break;
         float cur[kMeanBlocks][4];
 #pragma unroll
         for (int g = 0; g < kMeanBlocks; ++g)
@@ -357,15 +384,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The QK products alternate between the tiles through the shared score
       // columns: S_1(j) once tile 0 has loaded S_0(j), S_0(j+1) once tile 1 has
       // loaded S_1(j).
-      ok = wait_warp(s, &s.q_full, 0, P);
+      ok = wait_spin_warp(s, &s.q_full, 0, P);
       for (int j = 0; ok && j < nkv; ++j) {
         const int ks = j % kKStages;
-        if (!(ok = wait_warp(s, &s.k_full[ks], (j / kKStages) & 1, P))) break;
-        if (j > 0 && !(ok = wait_warp(s, &s.s_loaded[1], (j - 1) & 1, P))) break;
+        if (!(ok = wait_spin_warp(s, &s.k_full[ks], (j / kKStages) & 1, P))) break;
+        if (j > 0 && !(ok = wait_spin_warp(s, &s.s_loaded[1], (j - 1) & 1, P))) break;
         tc_fence_after();
         qk(0, ks);
         commit(&s.s_full[0]);
-        if (!(ok = wait_warp(s, &s.s_loaded[0], j & 1, P))) break;
+        if (!(ok = wait_spin_warp(s, &s.s_loaded[0], j & 1, P))) break;
         tc_fence_after();
         qk(1, ks);
         commit(&s.s_full[1]);
@@ -382,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O_t += R_t M of one batch of blocks (both tiles read the same M tile)
       auto mean = [&](int batch) -> bool {
         const int mb = batch & 1;
-        if (!wait_warp(s, &s.m_full[mb], (batch >> 1) & 1, P)) return false;
+        if (!wait_spin_warp(s, &s.m_full[mb], (batch >> 1) & 1, P)) return false;
         tc_fence_after();
         const uint64_t dmo = sdesc_k_noswz(smem_u32(s.mop[mb]), kMopLbo, kMopSbo);
         if (leader) umma_f16_ss(tmem + col_ch(t), dr + 2 * (batch % kMeanChunks), dmo, id_mean, 1u);
@@ -393,8 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (tile 1: [1 ; V_j]) as soon as P_t(j) is in tensor memory.
       for (int j = 0; ok && j < nkv; ++j) {
         const int vs = j % kVStages;
-        if (!(ok = wait_warp(s, &s.p_full[t], j & 1, P))) break;
-        if (!(ok = wait_warp(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
+        if (!(ok = wait_spin_warp(s, &s.p_full[t], j & 1, P))) break;
+        if (!(ok = wait_spin_warp(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
         tc_fence_after();
         if (j >= kMeanBlocks && j % kMeanBlocks == 0 && !(ok = mean(j / kMeanBlocks - 1))) break;
         const uint32_t vb = smem_u32(&s.v[vs][0]);
