@@ -83,7 +83,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Workspace layout of vc_attn_prepare_v (every piece 256-B aligned).
 struct WsLayout {
-  size_t cent, sums, counts, assign, hist, offs, amax, total;
+  size_t cent, sums, counts, assign, assign2, hist, offs, amax, total;
 };
 
 WsLayout ws_layout(const vc_shape_t* sh, const vc_vsmooth_cfg_t* cfg) {
@@ -96,6 +96,7 @@ WsLayout ws_layout(const vc_shape_t* sh, const vc_vsmooth_cfg_t* cfg) {
   w.sums = off;   off += align256(BH * k * 128 * 8);
   w.counts = off; off += align256(BH * k * 4);
   w.assign = off; off += align256(BH * (size_t)sh->S);
+  w.assign2 = off; off += cfg->mode == VC_MODE_VSMOOTH ? align256(BH * (size_t)sh->S) : 0;
   w.hist = off;   off += align256(BH * nch * k * 4);
   w.offs = off;   off += align256(BH * nch * k * 4);
   w.amax = off;   off += align256(BH * 4);
@@ -222,6 +223,7 @@ static vc_status_t prepare_v_impl(const void* v, const vc_shape_t* shape, const 
   pl.sums = reinterpret_cast<unsigned long long*>(ws + w.sums);
   pl.counts = reinterpret_cast<int*>(ws + w.counts);
   pl.assign = ws + w.assign;
+  pl.assign2 = ws + w.assign2;
   pl.hist = reinterpret_cast<int*>(ws + w.hist);
   pl.offs = reinterpret_cast<int*>(ws + w.offs);
   pl.amax = reinterpret_cast<unsigned int*>(ws + w.amax);

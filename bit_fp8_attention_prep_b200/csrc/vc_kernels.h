@@ -26,7 +26,8 @@ struct PrepPlan {
   float* cent;                 // [BH][k][128]
   unsigned long long* sums;    // [BH][k][128] int64 fixed-point
   int* counts;                 // [BH][k]
-  uint8_t* assign;             // [BH][S]
+  uint8_t* assign;             // [BH][S] labels of the even passes
+  uint8_t* assign2;            // [BH][S] labels of the odd passes
   int* hist;                   // [BH][nchunks][k]
   int* offs;                   // [BH][nchunks][k]
   unsigned int* amax;          // [BH] fp32 bits

@@ -81,43 +81,23 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(const T* __restrict__ 
 //    the answer. The rest (a near tie) are compared by the direct form, lowest
 //    index on ties, which is the answer the direct form over all centroids
 //    gives.
-//  - Accumulation (kAccum): sums[c] and counts[c] are running totals over the
-//    whole (b, h) of the int64 llrint(x * 2^24) and of the tokens assigned to c.
-//    The first accumulating pass adds every token to its cluster; a later
-//    ("delta") pass reads each token's previous cluster before overwriting it
-//    and, for the tokens that moved, adds x to the new cluster and subtracts it
-//    from the old one (exact integer arithmetic, so the totals equal a fresh
-//    sum). The tile's entries go into cluster order (a counting sort: match_any
-//    ranks within each warp, offsets across warps and the two signs; the order
-//    within a cluster does not matter), as words holding the row's offset, the
-//    cluster and the sign. Thread d walks column d
-//    in that order, eight entries at a time, keeps an int64 running sum and adds
-//    it to the CTA's accumulator of the cluster where the cluster changes, at the
-//    same positions for every thread; no atomics until the chunk's totals go to
-//    global memory.
+//  - The labels go to global memory (per pass, for the sums kernel below and
+//    the final sort), and in the last pass a per-chunk cluster histogram.
 constexpr int kTile = 128;
 
-// Staged tile rows. The accumulating pass pads rows to 272 bytes (its column
-// walk reads one 2-byte element of a row per thread); the final pass packs them
-// at 256 bytes and XORs the 16-byte piece index with the row's low three bits.
-// Either way, eight lanes reading the same piece of eight consecutive rows hit
-// distinct banks.
-template <bool kPad>
-__device__ __forceinline__ int tile_off(int r, int piece) {
-  return kPad ? r * 272 + piece * 16 : r * 256 + ((piece ^ (r & 7)) << 4);
-}
-template <bool kPad>
-__host__ __device__ constexpr int tile_bytes() {
-  return kTile * (kPad ? 272 : 256);
-}
+// Staged tile rows: 256 bytes, the 16-byte piece index XORed with the row's low
+// three bits, so that eight lanes reading the same piece of eight consecutive
+// rows hit distinct banks.
+__device__ __forceinline__ int tile_off(int r, int piece) { return r * 256 + ((piece ^ (r & 7)) << 4); }
+constexpr int kTileBytes = kTile * 256;
 
 // 16 dimensions (16 ch .. 16 ch + 15) of staged row r, translated: x - r.
-template <typename T, bool kPad>
+template <typename T>
 __device__ __forceinline__ void load_translated(const uint8_t* tile, int r, int ch, const float* rneg,
                                                 float2* x) {
   float f[16];
-  unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off<kPad>(r, 2 * ch)), f);
-  unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off<kPad>(r, 2 * ch + 1)), f + 8);
+  unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off(r, 2 * ch)), f);
+  unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off(r, 2 * ch + 1)), f + 8);
   const float4* rv = reinterpret_cast<const float4*>(rneg + ch * 16);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -132,7 +112,7 @@ __device__ __forceinline__ void load_translated(const uint8_t* tile, int r, int 
 // dimensions in the two halves of a packed f32x2 accumulator, 16 dimensions at
 // a time, the halves added last; the lowest index wins ties. cg: the centroids
 // of this (b, h), fp32 [k][128].
-template <typename T, bool kPad>
+template <typename T>
 __device__ __noinline__ int nearest_direct(const uint8_t* tile, int r, const float* __restrict__ cg, uint32_t cand) {
   int best = -1;
   float best_d = 0.0f;
@@ -143,8 +123,8 @@ __device__ __noinline__ int nearest_direct(const uint8_t* tile, int r, const flo
 #pragma unroll 1
     for (int ch = 0; ch < 8; ++ch) {
       float f[16];
-      unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off<kPad>(r, 2 * ch)), f);
-      unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off<kPad>(r, 2 * ch + 1)), f + 8);
+      unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off(r, 2 * ch)), f);
+      unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off(r, 2 * ch + 1)), f + 8);
       const float4* cc = reinterpret_cast<const float4*>(cg + c * kD + ch * 16);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -164,26 +144,21 @@ __device__ __noinline__ int nearest_direct(const uint8_t* tile, int r, const flo
   return best;
 }
 
-template <typename T, bool kAccum, int KC>
+template <typename T, int KC>
 __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restrict__ v, int S, int H, int k,
-                                                              bool delta, const float* __restrict__ cent,
-                                                              unsigned long long* __restrict__ sums,
-                                                              int* __restrict__ counts, uint8_t* __restrict__ assign,
-                                                              int* __restrict__ hist, uint8_t* __restrict__ history) {
-  constexpr bool kPad = kAccum;
+                                                              const float* __restrict__ cent,
+                                                              uint8_t* __restrict__ assign, int* __restrict__ hist,
+                                                              uint8_t* __restrict__ history) {
   constexpr int kHalfC = KC / 2;
   static_assert(KC % 2 == 0, "cluster capacity must keep the staged tile 16-byte aligned");
   extern __shared__ __align__(16) uint8_t smem[];
-  long long* acc = reinterpret_cast<long long*>(smem);                                  // [KC][128] (kAccum)
-  float* cpr = reinterpret_cast<float*>(smem + (kAccum ? (size_t)KC * kD * 8 : 0));     // [KC][128]: c - r
+  float* cpr = reinterpret_cast<float*>(smem);                                         // [KC][128]: c - r
   float* rneg = cpr + (size_t)KC * kD;                                                 // [128]: -r
   float* ncs = rneg + kD;                                                              // [KC]: |c - r|^2
   float* kns = ncs + KC;                                                               // [KC]: 2^-15 |c - r|^2
   float* gsm = kns + KC;                                                               // [kTile][KC + 1]: g_c
   uint8_t* tile = reinterpret_cast<uint8_t*>(gsm + kTile * (KC + 1));                   // staged rows
-  uint32_t* sent = reinterpret_cast<uint32_t*>(tile + tile_bytes<kPad>());             // [2 kTile]: sorted entries
-  int* scount = reinterpret_cast<int*>(sent + 2 * kTile);                              // [KC]
-  int* woff = scount + KC;                                                             // [2][4][KC] + 1
+  int* scount = reinterpret_cast<int*>(tile + kTileBytes);                     // [KC]
 
   const int bh = blockIdx.y, b = bh / H, h = bh % H;
   const int chunk = blockIdx.x;
@@ -214,8 +189,6 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
     for (int c = 0; c < KC; ++c)
       if (c < k) cpr[c * kD + d] = __fsub_rn(cv[c], r);
   }
-  if (kAccum)
-    for (int i = tid; i < KC * kD; i += kTile) acc[i] = 0;
   if (tid < KC) scount[tid] = 0;
   __syncthreads();
   for (int c = warp; c < k; c += 4) {  // |c'|^2
@@ -246,11 +219,9 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
       const int idx = i * kTile + tid, r = idx >> 4, c = idx & 15;
       if (r < ntok) {
         const uint4 val = *reinterpret_cast<const uint4*>(vbase + (size_t)(s0 + r) * row_stride + c * 8);
-        *reinterpret_cast<uint4*>(tile + tile_off<kPad>(r, c)) = val;
+        *reinterpret_cast<uint4*>(tile + tile_off(r, c)) = val;
       }
     }
-    if (kAccum)
-      for (int i = tid; i < 8 * KC; i += kTile) woff[i] = 0;
     __syncthreads();
     // proxies g_c of tokens t and t + 64 (rows past ntok hold stale data; unused)
     float2 ga[kHalfC], gb[kHalfC];
@@ -260,8 +231,8 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
 #pragma unroll 1
     for (int ch = 0; ch < 8; ++ch) {
       float2 xa[8], xb[8];
-      load_translated<T, kPad>(tile, t, ch, rneg, xa);
-      load_translated<T, kPad>(tile, t + 64, ch, rneg, xb);
+      load_translated<T>(tile, t, ch, rneg, xa);
+      load_translated<T>(tile, t + 64, ch, rneg, xb);
       if (half == 0) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) xx = __ffma2_rn(xa[i], xa[i], xx);
@@ -297,7 +268,7 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
       }
     __syncthreads();
     const bool valid = tid < ntok;
-    int best = 0, prev = -1;  // prev: this token's cluster in the previous pass (delta passes)
+    int best = 0;
     if (valid) {
       const float* g = gsm + tid * (KC + 1);
       float g_best = g[0];
@@ -311,140 +282,160 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
       uint32_t near = 0;
       for (int c = 0; c < k; ++c)
         if (c != best && !(g[c] - kns[c] > lim)) near |= 1u << c;
-      if (near != 0u) best = nearest_direct<T, kPad>(tile, tid, cg, near | (1u << best));
-      if (kAccum && delta) prev = assign[(size_t)bh * S + s0 + tid];
+      if (near != 0u) best = nearest_direct<T>(tile, tid, cg, near | (1u << best));
       assign[(size_t)bh * S + s0 + tid] = (uint8_t)best;
       if (history) history[(size_t)bh * S + s0 + tid] = (uint8_t)best;
-      if (!(kAccum && delta)) {
-        atomicAdd(&scount[best], 1);
-      } else if (prev != best) {
-        atomicAdd(&scount[best], 1);
-        atomicAdd(&scount[prev], -1);
-      }
-    }
-    if (kAccum) {
-      // The tile's entries: +x to the token's cluster for every token (first
-      // pass), or, in a delta pass, +x to the new and -x to the old cluster of
-      // every token that moved. Counting sort of the entries by cluster (the order
-      // within a cluster does not matter for an exact sum): per-cluster counts,
-      // their exclusive scan, then each entry takes the next slot of its cluster.
-      // ranks within each warp by match_any, for the + entries (round 0) and the
-      // - entries (round 1); woff[round][warp][c] becomes the first slot of
-      // cluster c's entries of that round and warp
-      const bool add = valid && (!delta || prev != best), sub = valid && delta && prev != best;
-      const unsigned pa = __match_any_sync(0xffffffffu, add ? best : 0xFF);
-      const unsigned ps = __match_any_sync(0xffffffffu, sub ? prev : 0xFF);
-      const int ra = __popc(pa & ((1u << lane) - 1u)), rs = __popc(ps & ((1u << lane) - 1u));
-      if (add && ra == 0) woff[(0 * 4 + warp) * KC + best] = __popc(pa);
-      if (sub && rs == 0) woff[(1 * 4 + warp) * KC + prev] = __popc(ps);
-      __syncthreads();
-      if (tid < 32) {
-        int w[8], tot = 0;
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          w[g] = tid < KC ? woff[g * KC + tid] : 0;
-          tot += w[g];
-        }
-        int incl = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int t2 = __shfl_up_sync(0xffffffffu, incl, o);
-          if (tid >= o) incl += t2;
-        }
-        if (tid < KC) {
-          int base = incl - tot;
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            woff[g * KC + tid] = base;
-            base += w[g];
-          }
-        }
-        if (tid == 31) woff[8 * KC] = incl;  // number of entries
-      }
-      __syncthreads();
-      const uint32_t row_word = (uint32_t)(tid * 272);
-      if (add) sent[woff[(0 * 4 + warp) * KC + best] + ra] = row_word | ((uint32_t)best << 16);
-      if (sub) sent[woff[(1 * 4 + warp) * KC + prev] + rs] = row_word | ((uint32_t)prev << 16) | 0x80000000u;
-      __syncthreads();
-      const int nent = woff[8 * KC];
-      // thread d: column d over the entries in cluster order; the running sum goes
-      // to the cluster's accumulator where the cluster changes (the same place for
-      // every thread)
-      const int d = tid;
-      const uint8_t* col = tile + d * 2;
-      // Within a cluster the + entries precede the - entries, so the walk keeps
-      // one unsigned running sum per (cluster, sign) segment and applies the
-      // sign where the segment ends. key = e >> 16: cluster, sign in bit 15.
-      auto flush = [&](uint32_t key, long long run) {
-        acc[(key & 0xFFu) * kD + d] += (key & 0x8000u) ? -run : run;
-      };
-      if (nent > 0) {
-        long long run = 0;
-        uint32_t cur = sent[0] >> 16;
-        int pos = 0;
-        for (; pos + 8 <= nent; pos += 8) {
-          const uint4 e0 = *reinterpret_cast<const uint4*>(sent + pos);
-          const uint4 e1 = *reinterpret_cast<const uint4*>(sent + pos + 4);
-          const uint32_t e[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-          long long q[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j)  // x * 2^24, exact
-            q[j] = __float2ll_rn(to_f32<T>(*reinterpret_cast<const T*>(col + (e[j] & 0xffffu))) * 16777216.0f);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t key = e[j] >> 16;
-            if (key != cur) {
-              flush(cur, run);
-              run = 0;
-              cur = key;
-            }
-            run += q[j];
-          }
-        }
-        for (; pos < nent; ++pos) {
-          const uint32_t e = sent[pos], key = e >> 16;
-          if (key != cur) {
-            flush(cur, run);
-            run = 0;
-            cur = key;
-          }
-          run += __float2ll_rn(to_f32<T>(*reinterpret_cast<const T*>(col + (e & 0xffffu))) * 16777216.0f);
-        }
-        flush(cur, run);
-      }
+      if (hist != nullptr) atomicAdd(&scount[best], 1);
     }
   }
   __syncthreads();
-  if (kAccum) {
-    for (int i = tid; i < k * kD; i += kTile)
-      if (acc[i] != 0) atomicAdd(&sums[(size_t)bh * k * kD + i], (unsigned long long)acc[i]);
-    if (tid < k && scount[tid] != 0) atomicAdd(&counts[(size_t)bh * k + tid], scount[tid]);
-  } else if (hist != nullptr && tid < k) {
-    hist[((size_t)bh * gridDim.x + chunk) * k + tid] = scount[tid];
-  }
+  if (hist != nullptr && tid < k) hist[((size_t)bh * gridDim.x + chunk) * k + tid] = scount[tid];
 }
 
 template <int KC>
-constexpr size_t assign_smem(bool accum) {
-  return (accum ? (size_t)KC * kD * 8 : 0) + (size_t)KC * kD * 4 + kD * 4 + 2 * KC * 4 + kTile * (KC + 1) * 4 +
-         (accum ? tile_bytes<true>() : tile_bytes<false>()) + 8 * kTile + (9 * KC + 4) * 4;
+constexpr size_t assign_smem() {
+  return (size_t)KC * kD * 4 + kD * 4 + 2 * KC * 4 + kTile * (KC + 1) * 4 + kTileBytes + KC * 4;
 }
 
-template <typename T, bool kAccum, int KC>
-static void launch_assign(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, bool delta, uint8_t* hist_t) {
-  kmeans_assign_kernel<T, kAccum, KC><<<grid, kTile, assign_smem<KC>(kAccum), st>>>(
-      v, pl.S, pl.H, pl.k, delta, pl.cent, pl.sums, pl.counts, pl.assign, kAccum ? nullptr : pl.hist, hist_t);
+// --------------------------------------------------------------- k-means sums
+// sums[c] and counts[c] are running totals over the whole (b, h): the int64 sum
+// of llrint(x * 2^24) over the tokens of cluster c, and their number. One CTA
+// (4 warps) = one chunk of kChunk tokens, in tiles of 128. The first pass adds
+// every token to its cluster; a later ("delta") pass compares each token's
+// cluster with the previous pass's and, for the tokens that moved, adds x to the
+// new cluster and subtracts it from the old one (exact integer arithmetic, so the
+// totals equal a fresh sum). The tile's entries go into cluster order, + before -
+// within a cluster (a counting sort: match_any ranks within each warp, offsets
+// across warps and the two signs), as words holding the token, the cluster and
+// the sign. Thread d walks dimension d of the entries' rows (the CTA reads each
+// row as one coalesced 256-byte line), eight entries in flight, keeps an int64
+// running sum and adds it to the CTA's accumulator where a (cluster, sign)
+// segment ends, at the same positions for every thread. A tile without entries
+// reads nothing; no atomics until the chunk's totals go to global memory.
+template <typename T, int KC>
+__global__ void __launch_bounds__(kTile) kmeans_sums_kernel(const T* __restrict__ v, int S, int H, int k, bool delta,
+                                                            const uint8_t* __restrict__ lab_new,
+                                                            const uint8_t* __restrict__ lab_old,
+                                                            unsigned long long* __restrict__ sums,
+                                                            int* __restrict__ counts) {
+  __shared__ long long acc[KC * kD];
+  __shared__ __align__(16) uint32_t sent[2 * kTile];
+  __shared__ int scount[KC];
+  __shared__ int woff[8 * KC + 1];  // [sign][warp][cluster], then the number of entries
+  const int bh = blockIdx.y, b = bh / H, h = bh % H, chunk = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, d = tid;
+  const size_t row_stride = (size_t)H * kD;
+  const T* vcol = v + ((size_t)b * S * H + h) * kD + d;
+  for (int i = tid; i < KC * kD; i += kTile) acc[i] = 0;
+  if (tid < KC) scount[tid] = 0;
+  const int s_chunk0 = chunk * kChunk, s_chunk1 = min(S, s_chunk0 + kChunk);
+  for (int s0 = s_chunk0; s0 < s_chunk1; s0 += kTile) {
+    const bool valid = tid < s_chunk1 - s0;
+    const int cn = valid ? lab_new[(size_t)bh * S + s0 + tid] : 0;
+    const int co = valid && delta ? lab_old[(size_t)bh * S + s0 + tid] : cn;
+    const bool add = valid && (!delta || co != cn), sub = valid && delta && co != cn;
+    __syncthreads();  // the previous tile's walk is done with sent and woff
+    for (int i = tid; i < 8 * KC; i += kTile) woff[i] = 0;
+    if (add) atomicAdd(&scount[cn], 1);
+    if (sub) atomicAdd(&scount[co], -1);
+    const unsigned pa = __match_any_sync(0xffffffffu, add ? cn : 0xFF);
+    const unsigned ps = __match_any_sync(0xffffffffu, sub ? co : 0xFF);
+    const int ra = __popc(pa & ((1u << lane) - 1u)), rs = __popc(ps & ((1u << lane) - 1u));
+    __syncthreads();
+    if (add && ra == 0) woff[(0 * 4 + warp) * KC + cn] = __popc(pa);
+    if (sub && rs == 0) woff[(1 * 4 + warp) * KC + co] = __popc(ps);
+    __syncthreads();
+    if (tid < 32) {
+      int w[8], tot = 0;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        w[g] = tid < KC ? woff[g * KC + tid] : 0;
+        tot += w[g];
+      }
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t2 = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += t2;
+      }
+      if (tid < KC) {
+        int base = incl - tot;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          woff[g * KC + tid] = base;
+          base += w[g];
+        }
+      }
+      if (tid == 31) woff[8 * KC] = incl;
+    }
+    __syncthreads();
+    if (add) sent[woff[(0 * 4 + warp) * KC + cn] + ra] = (uint32_t)tid | ((uint32_t)cn << 16);
+    if (sub) sent[woff[(1 * 4 + warp) * KC + co] + rs] = (uint32_t)tid | ((uint32_t)co << 16) | 0x80000000u;
+    __syncthreads();
+    const int nent = woff[8 * KC];
+    if (nent == 0) continue;
+    const T* tcol = vcol + (size_t)s0 * row_stride;
+    auto flush = [&](uint32_t key, long long run) {  // key = e >> 16: cluster, sign in bit 15
+      acc[(key & 0xFFu) * kD + d] += (key & 0x8000u) ? -run : run;
+    };
+    long long run = 0;
+    uint32_t cur = sent[0] >> 16;
+    int pos = 0;
+    for (; pos + 8 <= nent; pos += 8) {
+      const uint4 e0 = *reinterpret_cast<const uint4*>(sent + pos);
+      const uint4 e1 = *reinterpret_cast<const uint4*>(sent + pos + 4);
+      const uint32_t e[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+      T x[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[j] = tcol[(size_t)(e[j] & 0xFFu) * row_stride];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t key = e[j] >> 16;
+        if (key != cur) {
+          flush(cur, run);
+          run = 0;
+          cur = key;
+        }
+        run += __float2ll_rn(to_f32<T>(x[j]) * 16777216.0f);  // x * 2^24, exact
+      }
+    }
+    for (; pos < nent; ++pos) {
+      const uint32_t e = sent[pos], key = e >> 16;
+      if (key != cur) {
+        flush(cur, run);
+        run = 0;
+        cur = key;
+      }
+      run += __float2ll_rn(to_f32<T>(tcol[(size_t)(e & 0xFFu) * row_stride]) * 16777216.0f);
+    }
+    flush(cur, run);
+  }
+  __syncthreads();
+  for (int i = tid; i < k * kD; i += kTile)
+    if (acc[i] != 0) atomicAdd(&sums[(size_t)bh * k * kD + i], (unsigned long long)acc[i]);
+  if (tid < k && scount[tid] != 0) atomicAdd(&counts[(size_t)bh * k + tid], scount[tid]);
 }
 
-template <typename T, bool kAccum>
-static void launch_assign_k(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, bool delta,
-                            uint8_t* hist_t) {
+template <typename T, int KC>
+static void launch_kmeans_pass(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, int it, bool last,
+                               uint8_t* hist_t) {
+  uint8_t* lab = it & 1 ? pl.assign2 : pl.assign;
+  kmeans_assign_kernel<T, KC><<<grid, kTile, assign_smem<KC>(), st>>>(v, pl.S, pl.H, pl.k, pl.cent, lab,
+                                                                       last ? pl.hist : nullptr, hist_t);
+  if (!last)
+    kmeans_sums_kernel<T, KC><<<grid, kTile, 0, st>>>(v, pl.S, pl.H, pl.k, it > 0, lab, it & 1 ? pl.assign : pl.assign2,
+                                                      pl.sums, pl.counts);
+}
+
+template <typename T>
+static void launch_kmeans_pass_k(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, int it, bool last,
+                                 uint8_t* hist_t) {
   if (pl.k <= 8)
-    launch_assign<T, kAccum, 8>(grid, st, v, pl, delta, hist_t);
+    launch_kmeans_pass<T, 8>(grid, st, v, pl, it, last, hist_t);
   else if (pl.k <= 16)
-    launch_assign<T, kAccum, 16>(grid, st, v, pl, delta, hist_t);
+    launch_kmeans_pass<T, 16>(grid, st, v, pl, it, last, hist_t);
   else
-    launch_assign<T, kAccum, 32>(grid, st, v, pl, delta, hist_t);
+    launch_kmeans_pass<T, 32>(grid, st, v, pl, it, last, hist_t);
 }
 
 // --------------------------------------------------------------- centroid update
@@ -888,19 +879,22 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
     kmeans_init_kernel<T><<<BH, 128, 0, st>>>(v, S, H, k, pl.seed, pl.bh_base, pl.cent);
     ++n;
     const dim3 grid(pl.nchunks, BH);
+    // pass it writes its labels to assign (even) or assign2 (odd); the sums of
+    // every pass but the last feed the centroid update
     for (int it = 0; it < pl.iters; ++it) {
       uint8_t* hist_t = history ? history + (size_t)it * BH * S : nullptr;
-      if (it + 1 < pl.iters) {
-        launch_assign_k<T, true>(grid, st, v, pl, it > 0, hist_t);
+      const bool last = it + 1 == pl.iters;
+      launch_kmeans_pass_k<T>(grid, st, v, pl, it, last, hist_t);
+      if (!last) {
         kmeans_update_kernel<<<BH, 128, 0, st>>>(k, pl.cent, pl.sums, pl.counts);
-        n += 2;
+        n += 3;
       } else {
-        launch_assign_k<T, false>(grid, st, v, pl, false, hist_t);
         ++n;
       }
     }
     perm_offsets_kernel<<<BH, 32, 0, st>>>(k, pl.nchunks, pl.hist, pl.offs);
-    perm_scatter_kernel<<<grid, kChunk, 0, st>>>(S, k, pl.assign, pl.offs, out.perm);
+    perm_scatter_kernel<<<grid, kChunk, 0, st>>>(S, k, (pl.iters - 1) & 1 ? pl.assign2 : pl.assign, pl.offs,
+                                                 out.perm);
     n += 2;
   } else {
     identity_perm_kernel<<<dim3(std::max(1, std::min(1024, (S + 255) / 256)), BH), 256, 0, st>>>(S, out.perm);
@@ -948,18 +942,12 @@ cudaError_t prep_configure() {
     const void* f;
     size_t bytes;
   } assign_fns[] = {
-      {(const void*)kmeans_assign_kernel<__nv_bfloat16, true, 8>, assign_smem<8>(true)},
-      {(const void*)kmeans_assign_kernel<__nv_bfloat16, true, 16>, assign_smem<16>(true)},
-      {(const void*)kmeans_assign_kernel<__nv_bfloat16, true, 32>, assign_smem<32>(true)},
-      {(const void*)kmeans_assign_kernel<__nv_bfloat16, false, 8>, assign_smem<8>(false)},
-      {(const void*)kmeans_assign_kernel<__nv_bfloat16, false, 16>, assign_smem<16>(false)},
-      {(const void*)kmeans_assign_kernel<__nv_bfloat16, false, 32>, assign_smem<32>(false)},
-      {(const void*)kmeans_assign_kernel<__half, true, 8>, assign_smem<8>(true)},
-      {(const void*)kmeans_assign_kernel<__half, true, 16>, assign_smem<16>(true)},
-      {(const void*)kmeans_assign_kernel<__half, true, 32>, assign_smem<32>(true)},
-      {(const void*)kmeans_assign_kernel<__half, false, 8>, assign_smem<8>(false)},
-      {(const void*)kmeans_assign_kernel<__half, false, 16>, assign_smem<16>(false)},
-      {(const void*)kmeans_assign_kernel<__half, false, 32>, assign_smem<32>(false)},
+      {(const void*)kmeans_assign_kernel<__nv_bfloat16, 8>, assign_smem<8>()},
+      {(const void*)kmeans_assign_kernel<__nv_bfloat16, 16>, assign_smem<16>()},
+      {(const void*)kmeans_assign_kernel<__nv_bfloat16, 32>, assign_smem<32>()},
+      {(const void*)kmeans_assign_kernel<__half, 8>, assign_smem<8>()},
+      {(const void*)kmeans_assign_kernel<__half, 16>, assign_smem<16>()},
+      {(const void*)kmeans_assign_kernel<__half, 32>, assign_smem<32>()},
   };
   for (const auto& a : assign_fns)
     if ((e = cudaFuncSetAttribute(a.f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)a.bytes)) != cudaSuccess)

@@ -29,7 +29,7 @@ ABI_SYMBOLS = [
     "vc_attn_quant_qk", "vc_attn_forward", "vc_attn_forward_nvfp4v_workspace_bytes", "vc_attn_forward_nvfp4v",
     "vc_attn_prepare_v_noalloc", "vc_attn_run_host_workspace_bytes", "vc_attn_run_host",
 ]
-NOALLOC_SCRATCH_BYTES = 8 << 20   # VC_ATTN_NOALLOC_SCRATCH_BYTES
+NOALLOC_SCRATCH_BYTES = 12 << 20  # VC_ATTN_NOALLOC_SCRATCH_BYTES
 TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
                 "vc_attn_test_bounded_wait", "vc_attn_test_forward_exp2"]
 

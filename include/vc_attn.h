@@ -194,8 +194,8 @@ vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t*
                                    void* o, void* workspace, size_t workspace_bytes,
                                    int32_t* dev_status, void* stream);
 
-/* Size of the fixed device scratch used by vc_attn_prepare_v_noalloc: 8 MiB. */
-#define VC_ATTN_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+/* Size of the fixed device scratch used by vc_attn_prepare_v_noalloc: 12 MiB. */
+#define VC_ATTN_NOALLOC_SCRATCH_BYTES ((size_t)12 << 20)
 
 /* V-Smooth prep exactly as vc_attn_prepare_v, but without a caller workspace:
  * the k-means and sort scratch lives in a fixed device array that this library
@@ -207,7 +207,7 @@ vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t*
  * cudaMalloc (which can synchronise the device). Inputs and outputs are still
  * caller-owned, as for vc_attn_prepare_v; nothing is allocated or freed.
  *  - Fits when vc_attn_prepare_v_workspace_bytes(shape, cfg) <=
- *    VC_ATTN_NOALLOC_SCRATCH_BYTES (about 6 MB for B=1, H=56, S=73397, k=16);
+ *    VC_ATTN_NOALLOC_SCRATCH_BYTES (about 10 MB for B=1, H=56, S=73397, k=16);
  *    larger problems return VC_ERR_WORKSPACE with a message naming both sizes
  *    (use vc_attn_prepare_v with a workspace for them).
  *  - The first call on a device looks up the array's device address there

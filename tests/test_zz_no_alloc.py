@@ -50,7 +50,7 @@ def test_noalloc_prep_matches_workspace_prep_on_two_calls(va):
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(va):
-    # B=1, S=73397, H=64 with 32 clusters needs about 9 MB of prep scratch. The
+    # B=1, S=73397, H=64 with 32 clusters needs about 13 MB of prep scratch. The
     # size check comes before anything touches the device, so the data pointers
     # here are placeholders that are never dereferenced.
     lib = va.load()
