@@ -307,11 +307,12 @@ constexpr size_t assign_smem() {
 // totals equal a fresh sum). The tile's entries go into cluster order, + before -
 // within a cluster (a counting sort: match_any ranks within each warp, offsets
 // across warps and the two signs), as words holding the token, the cluster and
-// the sign. Thread d walks dimension d of the entries' rows (the CTA reads each
-// row as one coalesced 256-byte line), eight entries in flight, keeps an int64
-// running sum and adds it to the CTA's accumulator where a (cluster, sign)
-// segment ends, at the same positions for every thread. A tile without entries
-// reads nothing; no atomics until the chunk's totals go to global memory.
+// the sign. Each warp walks a contiguous quarter of the sorted entries, eight
+// entries in flight, lane l owning dimensions 4l .. 4l+3 of each entry's row (one
+// coalesced 256-byte read per warp load); it keeps int64 running sums and adds
+// them to the CTA's accumulators (shared-memory atomics: a segment can span two
+// warps) where a (cluster, sign) segment ends. A tile without entries reads
+// nothing; no global atomics until the chunk's totals go to global memory.
 template <typename T, int KC>
 __global__ void __launch_bounds__(kTile) kmeans_sums_kernel(const T* __restrict__ v, int S, int H, int k, bool delta,
                                                             const uint8_t* __restrict__ lab_new,
@@ -323,9 +324,9 @@ __global__ void __launch_bounds__(kTile) kmeans_sums_kernel(const T* __restrict_
   __shared__ int scount[KC];
   __shared__ int woff[8 * KC + 1];  // [sign][warp][cluster], then the number of entries
   const int bh = blockIdx.y, b = bh / H, h = bh % H, chunk = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, d = tid;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t row_stride = (size_t)H * kD;
-  const T* vcol = v + ((size_t)b * S * H + h) * kD + d;
+  const T* vbase4 = v + ((size_t)b * S * H + h) * kD + 4 * lane;
   for (int i = tid; i < KC * kD; i += kTile) acc[i] = 0;
   if (tid < KC) scount[tid] = 0;
   const int s_chunk0 = chunk * kChunk, s_chunk1 = min(S, s_chunk0 + kChunk);
@@ -374,39 +375,51 @@ __global__ void __launch_bounds__(kTile) kmeans_sums_kernel(const T* __restrict_
     __syncthreads();
     const int nent = woff[8 * KC];
     if (nent == 0) continue;
-    const T* tcol = vcol + (size_t)s0 * row_stride;
-    auto flush = [&](uint32_t key, long long run) {  // key = e >> 16: cluster, sign in bit 15
-      acc[(key & 0xFFu) * kD + d] += (key & 0x8000u) ? -run : run;
-    };
-    long long run = 0;
-    uint32_t cur = sent[0] >> 16;
-    int pos = 0;
-    for (; pos + 8 <= nent; pos += 8) {
-      const uint4 e0 = *reinterpret_cast<const uint4*>(sent + pos);
-      const uint4 e1 = *reinterpret_cast<const uint4*>(sent + pos + 4);
-      const uint32_t e[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-      T x[8];
+    // warp w walks entries [w n / 4, (w + 1) n / 4); lane l owns dimensions
+    // 4l .. 4l+3 of each entry's row (one coalesced 256-byte read per warp load)
+    const int e_lo = (warp * nent) >> 2, e_hi = ((warp + 1) * nent) >> 2;
+    if (e_lo == e_hi) continue;
+    const T* trow = vbase4 + (size_t)s0 * row_stride;
+    auto flush = [&](uint32_t key, const long long* run) {  // key = e >> 16: cluster, sign in bit 15
+      unsigned long long* a = reinterpret_cast<unsigned long long*>(acc + (key & 0xFFu) * kD + 4 * lane);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) x[j] = tcol[(size_t)(e[j] & 0xFFu) * row_stride];
+      for (int q = 0; q < 4; ++q) atomicAdd(a + q, (unsigned long long)((key & 0x8000u) ? -run[q] : run[q]));
+    };
+    long long run[4] = {0, 0, 0, 0};
+    uint32_t cur = sent[e_lo] >> 16;
+    int pos = e_lo;
+    for (; pos + 8 <= e_hi; pos += 8) {
+      uint32_t e[8];
+      uint2 x[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) e[j] = sent[pos + j];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[j] = *reinterpret_cast<const uint2*>(trow + (size_t)(e[j] & 0xFFu) * row_stride);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const uint32_t key = e[j] >> 16;
         if (key != cur) {
           flush(cur, run);
-          run = 0;
+          run[0] = run[1] = run[2] = run[3] = 0;
           cur = key;
         }
-        run += __float2ll_rn(to_f32<T>(x[j]) * 16777216.0f);  // x * 2^24, exact
+        float f[4];
+        unpack4<T>(x[j], f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) run[q] += __float2ll_rn(f[q] * 16777216.0f);  // x * 2^24, exact
       }
     }
-    for (; pos < nent; ++pos) {
+    for (; pos < e_hi; ++pos) {
       const uint32_t e = sent[pos], key = e >> 16;
       if (key != cur) {
         flush(cur, run);
-        run = 0;
+        run[0] = run[1] = run[2] = run[3] = 0;
         cur = key;
       }
-      run += __float2ll_rn(to_f32<T>(tcol[(size_t)(e & 0xFFu) * row_stride]) * 16777216.0f);
+      float f[4];
+      unpack4<T>(*reinterpret_cast<const uint2*>(trow + (size_t)(e & 0xFFu) * row_stride), f);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) run[q] += __float2ll_rn(f[q] * 16777216.0f);
     }
     flush(cur, run);
   }
