@@ -71,8 +71,11 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(const T* __restrict__ 
 //    (c = 2i + half): one packed f32x2 FMA per two dimensions, token and
 //    centroid, against the direct form's subtract and FMA, with every centroid
 //    value read from shared memory (all lanes of a warp read the same address)
-//    feeding both tokens. The proxies go to shared memory and the token's
-//    thread takes their argmin. Their rounding is bounded: g_c is within
+//    feeding both tokens. Each half posts its nearest centroid per token; after
+//    a barrier each half marks its centroids that the bound below cannot rule
+//    out against the merged nearest, and the token's thread combines the two
+//    (the proxies stay in registers, so 5 CTAs fit on an SM). Their rounding is
+//    bounded: g_c is within
 //    199 u |c'|^2 + 68 u |x'|^2 of its exact value (u = 2^-24: 128-term FMA
 //    chains, the two translations, one final FMA), and the direct fp32 form
 //    sum_d (x_d - c_d)^2 within 134 u (|x'|^2 + |c'|^2). A centroid c whose
@@ -145,7 +148,7 @@ __device__ __noinline__ int nearest_direct(const uint8_t* tile, int r, const flo
 }
 
 template <typename T, int KC>
-__global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restrict__ v, int S, int H, int k,
+__global__ void __launch_bounds__(kTile, 5) kmeans_assign_kernel(const T* __restrict__ v, int S, int H, int k,
                                                               const float* __restrict__ cent,
                                                               uint8_t* __restrict__ assign, int* __restrict__ hist,
                                                               uint8_t* __restrict__ history) {
@@ -156,8 +159,11 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
   float* rneg = cpr + (size_t)KC * kD;                                                 // [128]: -r
   float* ncs = rneg + kD;                                                              // [KC]: |c - r|^2
   float* kns = ncs + KC;                                                               // [KC]: 2^-15 |c - r|^2
-  float* gsm = kns + KC;                                                               // [kTile][KC + 1]: g_c
-  uint8_t* tile = reinterpret_cast<uint8_t*>(gsm + kTile * (KC + 1));                   // staged rows
+  float* pg = kns + KC;                                                                // [2][kTile]: each half's nearest g
+  float* xs = pg + 2 * kTile;                                                          // [kTile]: |x'|^2
+  uint32_t* pn = reinterpret_cast<uint32_t*>(xs + kTile);                              // [2][kTile]: near-tie bits
+  int8_t* pi = reinterpret_cast<int8_t*>(pn + 2 * kTile);                              // [2][kTile]: nearest c
+  uint8_t* tile = reinterpret_cast<uint8_t*>(pi + 2 * kTile);                          // staged rows
   int* scount = reinterpret_cast<int*>(tile + kTileBytes);                     // [KC]
 
   const int bh = blockIdx.y, b = bh / H, h = bh % H;
@@ -256,32 +262,57 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
         }
       }
     }
+    // this half's proxies of both tokens, and its nearest centroid of each
+    float g[2][kHalfC];
 #pragma unroll
-    for (int tok = 0; tok < 2; ++tok)
+    for (int tok = 0; tok < 2; ++tok) {
+      int ib = -1;  // the lowest index wins ties within the half
+      float gmin = __int_as_float(0x7f800000);
 #pragma unroll
       for (int i = 0; i < kHalfC; ++i) {
         const int c = 2 * i + half;
-        if (c < k) {
-          const float2 dot = tok ? gb[i] : ga[i];
-          gsm[(t + 64 * tok) * (KC + 1) + c] = fmaf(-2.0f, dot.x + dot.y, ncs[c]);
+        const float2 dot = tok ? gb[i] : ga[i];
+        g[tok][i] = c < k ? fmaf(-2.0f, dot.x + dot.y, ncs[c]) : __int_as_float(0x7f800000);
+        if (c < k && (ib < 0 || g[tok][i] < gmin)) {
+          gmin = g[tok][i];
+          ib = c;
         }
       }
+      pg[half * kTile + t + 64 * tok] = gmin;
+      pi[half * kTile + t + 64 * tok] = (int8_t)ib;
+    }
+    xs[tid] = xx.x + xx.y;  // token tid = t + 64 half is this thread's own
+    __syncthreads();
+    // nearest of the two halves (lowest index on equal g), then this half's
+    // centroids that the rounding bound cannot rule out (a near tie)
+    auto merged = [&](int tk, float& g_best) -> int {
+      const float a1 = pg[tk], c1 = pg[kTile + tk];
+      const int ai = pi[tk], ci = pi[kTile + tk];
+      const bool first = ci < 0 || a1 < c1 || (a1 == c1 && ai < ci) || !(c1 == c1);
+      g_best = first ? a1 : c1;
+      return first ? ai : ci;
+    };
+#pragma unroll
+    for (int tok = 0; tok < 2; ++tok) {
+      const int tk = t + 64 * tok;
+      float g_best;
+      const int bc = merged(tk, g_best);
+      const float lim = g_best + (kns[bc] + xs[tk] * 0x1p-15f);
+      uint32_t near = 0;
+#pragma unroll
+      for (int i = 0; i < kHalfC; ++i) {
+        const int c = 2 * i + half;
+        if (c < k && c != bc && !(g[tok][i] - kns[c] > lim)) near |= 1u << c;
+      }
+      pn[half * kTile + tk] = near;
+    }
     __syncthreads();
     const bool valid = tid < ntok;
     int best = 0;
     if (valid) {
-      const float* g = gsm + tid * (KC + 1);
-      float g_best = g[0];
-      for (int c = 1; c < k; ++c)
-        if (g[c] < g_best) {
-          g_best = g[c];
-          best = c;
-        }
-      // centroids not ruled out by the rounding bound (a near tie)
-      const float lim = g_best + (kns[best] + (xx.x + xx.y) * 0x1p-15f);
-      uint32_t near = 0;
-      for (int c = 0; c < k; ++c)
-        if (c != best && !(g[c] - kns[c] > lim)) near |= 1u << c;
+      float g_best;
+      best = merged(tid, g_best);
+      const uint32_t near = pn[tid] | pn[kTile + tid];
       if (near != 0u) best = nearest_direct<T>(tile, tid, cg, near | (1u << best));
       assign[(size_t)bh * S + s0 + tid] = (uint8_t)best;
       if (history) history[(size_t)bh * S + s0 + tid] = (uint8_t)best;
@@ -294,7 +325,7 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(const T* __restric
 
 template <int KC>
 constexpr size_t assign_smem() {
-  return (size_t)KC * kD * 4 + kD * 4 + 2 * KC * 4 + kTile * (KC + 1) * 4 + kTileBytes + KC * 4;
+  return (size_t)KC * kD * 4 + kD * 4 + 2 * KC * 4 + kTile * (2 * 4 + 4 + 2 * 4 + 2) + kTileBytes + KC * 4;
 }
 
 // --------------------------------------------------------------- k-means sums
