@@ -74,11 +74,11 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(const T* __restrict__ 
 //    feeding both tokens. Each half posts its nearest centroid per token; after
 //    a barrier each half marks its centroids that the bound below cannot rule
 //    out against the merged nearest, and the token's thread combines the two
-//    (the proxies stay in registers, so 5 CTAs fit on an SM). Their rounding is
-//    bounded: g_c is within
-//    199 u |c'|^2 + 68 u |x'|^2 of its exact value (u = 2^-24: 128-term FMA
-//    chains, the two translations, one final FMA), and the direct fp32 form
-//    sum_d (x_d - c_d)^2 within 134 u (|x'|^2 + |c'|^2). A centroid c whose
+//    (the proxies stay in registers, so 5 CTAs fit on an SM).
+//    The proxies' rounding is bounded: g_c is within 199 u |c'|^2 + 68 u |x'|^2
+//    of its exact value (u = 2^-24: 128-term FMA chains, the two translations,
+//    one final FMA), and the direct fp32 form sum_d (x_d - c_d)^2 within
+//    134 u (|x'|^2 + |c'|^2). A centroid c whose
 //    g_c - 2^-15 |c'|^2 exceeds g_b + 2^-15 (|c'_b|^2 + |x'|^2) for the nearest
 //    b is farther than b exactly and also by the direct form, so it cannot be
 //    the answer. The rest (a near tie) are compared by the direct form, lowest
