@@ -158,40 +158,42 @@ __device__ __forceinline__ bool wait_spin_warp(Smem& s, uint64_t* bar, uint32_t 
   return __all_sync(0xffffffffu, ok);
 }
 
-// Byte offset of 16-bit element `slot` (K index 16*chunk + slot) of row `row` in
-// a 128-B-swizzled K-major operand tile (rows of 128 B, 8-row atoms).
-__device__ __forceinline__ uint32_t sw128_off16(int row, int chunk, int slot) {
-  const int kb = chunk * 32 + slot * 2;  // byte within the unswizzled 128-B row
-  return (uint32_t)(row * 128 + ((((kb >> 4) ^ (row & 7)) & 7) << 4) + (kb & 15));
-}
-
-__device__ __forceinline__ void st_bf16(uint8_t* base, uint32_t off, __nv_bfloat16 v) {
-  *reinterpret_cast<__nv_bfloat16*>(base + off) = v;
-}
-
 // x = hi + lo with hi = bf16(x), lo = bf16(x - hi): 16 significant bits, fp32 range.
 __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
   hi = __float2bfloat16_rn(x);
   lo = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
 }
 
-// Writes the three K slots of one block's row sum r (slots hi, hi, lo) into the
-// R operand tile.
-__device__ __forceinline__ void put_r(uint8_t* ro, int row, int ch, int g, float r) {
-  __nv_bfloat16 rh, rl;
-  split_bf16(r, rh, rl);
-  st_bf16(ro, sw128_off16(row, ch, 3 * g + 0), rh);
-  st_bf16(ro, sw128_off16(row, ch, 3 * g + 1), rh);
-  st_bf16(ro, sw128_off16(row, ch, 3 * g + 2), rl);
+__device__ __forceinline__ uint32_t bf16_bits(__nv_bfloat16 x) {
+  return (uint32_t)*reinterpret_cast<const uint16_t*>(&x);
+}
+
+// Writes one batch of row sums into chunk ch of row `row` of the R operand tile:
+// r[i] for the batch's blocks i < n as the three K slots hi, hi, lo, the other
+// slots 0. A chunk's 16 slots are two 16-byte pieces of the 128-B row.
+__device__ __forceinline__ void put_r_batch(uint8_t* ro, int row, int ch, const float (&r)[kMeanBlocks], int n) {
+  uint32_t h[16];
+#pragma unroll
+  for (int i = 0; i < kMeanBlocks; ++i) {
+    __nv_bfloat16 hi, lo;
+    split_bf16(i < n ? r[i] : 0.0f, hi, lo);
+    h[3 * i] = h[3 * i + 1] = bf16_bits(hi);
+    h[3 * i + 2] = bf16_bits(lo);
+  }
+  h[15] = 0u;
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i] = h[2 * i] | (h[2 * i + 1] << 16);
+  uint8_t* base = ro + row * 128;
+  const int x = row & 7;
+  *reinterpret_cast<uint4*>(base + (((2 * ch) ^ x) & 7) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(base + (((2 * ch + 1) ^ x) & 7) * 16) = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
 // M operand layout (unswizzled K-major, core matrices of 8 channels x 8 slots):
 // channel c, slots 8h .. 8h+7 are the 16 bytes at (c/8)*256 + h*128 + (c%8)*16.
 constexpr uint32_t kMopLbo = 128, kMopSbo = 256;
 
-__device__ __forceinline__ uint32_t bf16_bits(__nv_bfloat16 x) {
-  return (uint32_t)*reinterpret_cast<const uint16_t*>(&x);
-}
 
 // Four magic-biased codes (low bytes of the fp32 patterns) into one word, a in
 // the lowest byte. b*256 + a keeps a's and b's codes (< 256) in the low 16 bits
@@ -467,6 +469,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // F: running integer frame; Lp: row-sum column after the last block's own
     // rescale, so that the next read minus Lp is that block's row sum
     float F = 0.0f, Lp = 0.0f;
+    // row sums of the current batch of blocks, in the current frame (written to
+    // the R operand when the batch is complete)
+    float rb[kMeanBlocks] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
     bool ok = true, range_ok = true;
     const float* const ksc = P.k_scales + (size_t)bh * P.nb;
     float sK_next = ksc[0];
@@ -563,26 +568,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st_wait();  // the store reads r asynchronously: done before r is reused
         }
         tmem_st1(l_addr, __float_as_uint(Lc * alpha));
-        if (resc) {
-          const int jp = j - 1, ch = (jp / kMeanBlocks) % kMeanChunks;
-          const int nslots = 3 * (jp % kMeanBlocks);
-          for (int sl = 0; sl < nslots; ++sl) {
-            __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(ro + sw128_off16(row, ch, sl));
-            *e = __float2bfloat16_rn(__bfloat162float(*e) * alpha);
-          }
-        }
       }
       // R operand (no MMA of this tile is in flight between s_full and p_full):
       // the row sum of block j-1 is the column's growth since the last block,
       // carried into the new frame
       if (j > 0) {
-        const int jp = j - 1;
-        put_r(ro, row, (jp / kMeanBlocks) % kMeanChunks, jp % kMeanBlocks, __fsub_rn(Lc, Lp) * alpha);
+        const int jp = j - 1, g = jp % kMeanBlocks;
+        const float rj = __fsub_rn(Lc, Lp) * alpha;
+#pragma unroll
+        for (int i = 0; i < kMeanBlocks; ++i) rb[i] = i == g ? rj : rb[i] * alpha;  // exact: alpha = 2^-n
+        // a batch is complete once the row sum of its last block is in: the mean
+        // MMA that reads it is issued right after this block's p_full
+        if (g == kMeanBlocks - 1) {
+          put_r_batch(ro, row, (jp / kMeanBlocks) % kMeanChunks, rb, kMeanBlocks);
+          fence_proxy_async_smem();
+        }
       }
       Lp = Lc * alpha;
-      // a batch is complete once the row sum of its last block is in: the mean
-      // MMA that reads it is issued right after this block's p_full
-      if (j >= kMeanBlocks && j % kMeanBlocks == 0) fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&s.p_full[t]);
@@ -597,8 +599,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       l = __uint_as_float(tmem_ld1(l_addr));
       tmem_ld_wait();
       const int jp = nkv - 1, g = jp % kMeanBlocks, ch = (jp / kMeanBlocks) % kMeanChunks;
-      put_r(ro, row, ch, g, __fsub_rn(l, Lp));
-      for (int sl = 3 * g + 3; sl < 16; ++sl) st_bf16(ro, sw128_off16(row, ch, sl), __float2bfloat16_rn(0.0f));
+      const float rl = __fsub_rn(l, Lp);
+#pragma unroll
+      for (int i = 0; i < kMeanBlocks; ++i)
+        if (i == g) rb[i] = rl;
+      put_r_batch(ro, row, ch, rb, g + 1);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&s.fin_ready[t]);
