@@ -49,7 +49,8 @@
 // O = s_V O_t / l. The softmax thread of row i keeps the integer running frame
 // F (ceil of the largest log2-domain score so far); a block is cast in the frame
 // current after it; when F moves, O_t (with its row-sum column) and the row sums
-// not yet handed to a mean MMA are multiplied by the exact power 2^(F_old - F_new).
+// not yet handed to a mean MMA (held in registers until their batch of 5 blocks
+// is complete) are multiplied by the exact power 2^(F_old - F_new).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stddef.h>
