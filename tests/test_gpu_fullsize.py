@@ -1,14 +1,16 @@
-"""GPU: parity at the benchmark's full size and launch configuration.
+"""GPU: parity at full size, in the launch configuration bench.py times.
 
-minimax_h56 (B=1, S=73397, H=56, D=128, the shape the headline metric is quoted
-on) is drawn on the GPU with the synthetic recipe and run through the same
-library calls and grids that bench.py times. For two heads (the first and the
-last) the oracle recomputes the prep from the same inputs: permutation, block
-means, residual codes and Q/K codes and scales must be bit-exact (k-means near
-ties adopted in lock-step and counted), and the output rows it computes one by
-one (a spread of 48 query rows, the last row included) must meet the O
-acceptance bars. The preallocated plan (the bench's path) must give the same
-output bits as the one-shot calls."""
+Each workload is drawn on the GPU with the synthetic recipe and run through the
+library calls and grids the benchmark uses:
+  minimax_h56    B=1, S=73397, H=56 (the shape the headline metric is quoted on)
+  wan            B=1, S=75600, H=40, called with [S,H,128] tensors
+  nvfp4_s131072  B=1, S=131072, H=24, NVFP4 residual (the end of the NVFP4 sweep)
+For two heads (the first and the last) the oracle recomputes the prep from the
+same inputs: permutation, block means, residual codes (and NVFP4 scales) and Q/K
+codes and scales must be bit-exact (k-means near ties adopted in lock-step and
+counted), and the output rows it computes one by one (a spread of 48 query rows,
+the last row included) must meet the O acceptance bars. The preallocated plan
+(the bench's path) must give the same output bits as the one-shot calls."""
 import numpy as np
 import pytest
 import torch
@@ -28,36 +30,39 @@ def va():
     return vc_attn
 
 
-def test_minimax_h56_sampled_heads_and_rows(va):
-    cfg, Q, K, V = synth.make_workload("minimax_h56", seed=0, device="cuda")
-    B, S, H, k, iters = cfg["B"], cfg["S"], cfg["H"], cfg["k"], cfg["iters"]
-    pv = va.prepare_v(V, k=k, iters=iters, history=True)
-    qk = va.quant_qk(Q, K, pv["perm"])
+@pytest.mark.parametrize("name", ["minimax_h56", "wan", "nvfp4_s131072"])
+def test_full_size_sampled_heads_and_rows(va, name):
+    cfg, Q, K, V = synth.make_workload(name, seed=0, device="cuda")
+    B, S, H, k, iters, fmt = cfg["B"], cfg["S"], cfg["H"], cfg["k"], cfg["iters"], cfg["fmt"]
+    if cfg["layout"] == "SHD":  # B = 1: the [S,H,128] form of the same memory
+        Qc, Kc, Vc = Q[0], K[0], V[0]
+    else:
+        Qc, Kc, Vc = Q, K, V
+    pv = va.prepare_v(Vc, k=k, iters=iters, fmt=fmt, history=True)
+    qk = va.quant_qk(Qc, Kc, pv["perm"])
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    o = va.forward(qk, pv, va.shape_of(Q), SCALE, 8, status=status)
-    plan = va.Plan(B, S, H, k=k, iters=iters)
-    o_plan = plan.run(Q, K, V)
+    o = va.forward(qk, pv, va.shape_of(Qc), SCALE, 8, status=status).reshape(B, S, H, 128)
+    plan = va.Plan(B, S, H, k=k, iters=iters, fmt=fmt)
+    o_plan = plan.run(Qc, Kc, Vc).reshape(B, S, H, 128)
     torch.cuda.synchronize()
     assert int(status.item()) == 0 and int(plan.status.item()) == 0
     assert torch.equal(o.view(torch.int16), o_plan.view(torch.int16))
 
     rows = np.unique(np.concatenate([np.linspace(0, S - 1, 47).astype(np.int64), [S - 1]]))
     ties = 0
+    cpu = lambda t, h: None if t is None else t[:, h:h + 1].cpu().numpy()
     for h in (0, H - 1):
         q, kk, v = (X[0, :, h].float().cpu().numpy() for X in (Q, K, V))
         adopt = [pv["history"][t, 0, h].cpu().numpy() for t in range(iters)]
-        ref = O.prepare_v_head(v, k, iters, 0, h, adopt=adopt)
+        ref = O.prepare_v_head(v, k, iters, 0, h, fmt=fmt, adopt=adopt)
         qc, qs, kc, ks = O.quant_qk_head(q, kk, ref["perm"])
         ref.update(q_codes=qc, q_scales=qs, k_codes=kc, k_scales=ks)
-        g = dict(perm=pv["perm"][:, h:h + 1].cpu().numpy(), mu=pv["mu"][:, h:h + 1].cpu().numpy(),
-                 v_codes=pv["v_codes"][:, h:h + 1].cpu().numpy(), s_v=pv["s_v"][:, h:h + 1].cpu().numpy(),
-                 v_scales=None, q_codes=qk["q_codes"][:, h:h + 1].cpu().numpy(),
-                 q_scales=qk["q_scales"][:, h:h + 1].cpu().numpy(),
-                 k_codes=qk["k_codes"][:, h:h + 1].cpu().numpy(),
-                 k_scales=qk["k_scales"][:, h:h + 1].cpu().numpy())
-        assert_prep_bit_exact(g, ref, 0, 0)
+        g = dict(perm=cpu(pv["perm"], h), mu=cpu(pv["mu"], h), v_codes=cpu(pv["v_codes"], h),
+                 s_v=cpu(pv["s_v"], h), v_scales=cpu(pv.get("v_scales"), h), q_codes=cpu(qk["q_codes"], h),
+                 q_scales=cpu(qk["q_scales"], h), k_codes=cpu(qk["k_codes"], h), k_scales=cpu(qk["k_scales"], h))
+        assert_prep_bit_exact(g, ref, 0, 0, fmt=fmt)
         ties += ref["stats"]["near_ties"]
         o_ref = O.vc_attention_rows(qc, qs, kc, ks, ref["vres"], ref["mu"], S, rows, SCALE, k_p=8)
         r, m = assert_o_close(o[0, rows, h].float().cpu().numpy(), o_ref)
-        print(f"head {h}: rel-L2 vs oracle {r:.2e}, max-abs {m:.2e}")
-    print(f"k-means near ties adopted: {ties}")
+        print(f"{name} head {h}: rel-L2 vs oracle {r:.2e}, max-abs {m:.2e}")
+    print(f"{name}: k-means near ties adopted: {ties}")
