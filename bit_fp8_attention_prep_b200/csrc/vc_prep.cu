@@ -657,8 +657,9 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ 
 // The codes go to a shared tile [token][channel] (136-byte rows: the two half
 // warps' 8-byte stores fall on disjoint banks) and leave transposed, as V^T rows
 // of 128 tokens per channel (the K-major B operand of the PV product): a lane
-// gathers the codes of one channel for 4 consecutive tokens (8 lanes read the
-// same words, so the reads are conflict-free) and stores them as one word.
+// reads a 4 x 4 block of codes (4 channels of 4 consecutive tokens, one word per
+// token), transposes it with byte permutes and stores 4 words, one per channel.
+// A warp reads 8 channel groups of 4 token quads, which fall on 32 distinct banks.
 constexpr int kResStride = 136;
 
 template <typename T>
@@ -711,14 +712,23 @@ __global__ void __launch_bounds__(256) residual_e4m3_kernel(const T* __restrict_
   }
   __syncthreads();
   uint8_t* const out = vt + (size_t)bh * kD * S_pad + (size_t)blk * kBlock;
-  const int m = lane & 7, q = lane >> 3;
-#pragma unroll 4
-  for (int it = 0; it < 16; ++it) {
-    const int pidx = warp * 16 + it, cg = pidx & 15, qg = pidx >> 4;
-    const int d = cg * 8 + m, t0 = qg * 16 + q * 4;
-    const uint32_t b0 = ct[(t0 + 0) * kResStride + d], b1 = ct[(t0 + 1) * kResStride + d];
-    const uint32_t b2 = ct[(t0 + 2) * kResStride + d], b3 = ct[(t0 + 3) * kResStride + d];
-    *reinterpret_cast<uint32_t*>(out + (size_t)d * S_pad + t0) = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    // a 4 x 4 block of codes: channels 4cg .. 4cg+3 of tokens 4tq .. 4tq+3
+    const int combo = warp * 4 + it;
+    const int cg = 8 * (combo & 3) + (lane & 7), tq = 4 * (combo >> 2) + (lane >> 3);
+    const uint8_t* src = ct + (4 * tq) * kResStride + 4 * cg;
+    const uint32_t r0 = *reinterpret_cast<const uint32_t*>(src);                   // token 4tq, 4 channels
+    const uint32_t r1 = *reinterpret_cast<const uint32_t*>(src + kResStride);
+    const uint32_t r2 = *reinterpret_cast<const uint32_t*>(src + 2 * kResStride);
+    const uint32_t r3 = *reinterpret_cast<const uint32_t*>(src + 3 * kResStride);
+    const uint32_t lo01 = __byte_perm(r0, r1, 0x5140), hi01 = __byte_perm(r0, r1, 0x7362);
+    const uint32_t lo23 = __byte_perm(r2, r3, 0x5140), hi23 = __byte_perm(r2, r3, 0x7362);
+    uint8_t* dst = out + (size_t)(4 * cg) * S_pad + 4 * tq;                          // 4 tokens of a channel
+    *reinterpret_cast<uint32_t*>(dst) = __byte_perm(lo01, lo23, 0x5410);
+    *reinterpret_cast<uint32_t*>(dst + S_pad) = __byte_perm(lo01, lo23, 0x7632);
+    *reinterpret_cast<uint32_t*>(dst + 2 * (size_t)S_pad) = __byte_perm(hi01, hi23, 0x5410);
+    *reinterpret_cast<uint32_t*>(dst + 3 * (size_t)S_pad) = __byte_perm(hi01, hi23, 0x7632);
   }
 }
 
