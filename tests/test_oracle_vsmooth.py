@@ -217,3 +217,65 @@ def test_naive_mode_is_v_itself_with_one_scale_per_head():
     # with a common offset in V, the block means of V-Smooth shrink the range to code
     vs = O.prepare_v_head(V, 16, 4, 0, 0)
     assert vs["s_v"] < out["s_v"]
+
+
+def test_residual_energy_block_variance_parallel_axis_and_zero_means():
+    # With the exact fp64 mean of every block of the permuted order, the energy
+    # is sum_b n_b * sum_d var_bd (numpy's population variance per block, the
+    # ragged 44-token tail included). Any other means add sum_b n_b |mu_b - m_b|^2
+    # (the parallel-axis identity), which pins the block that each permuted
+    # position is charged to; zero means give the squared Frobenius norm of V.
+    S = 300
+    rng = np.random.default_rng(5)
+    X = _bf16_values((S, 128), 21, 2.0) + np.float32(3.0)
+    perm = rng.permutation(S).astype(np.int32)
+    Xp = X.astype(np.float64)[perm]
+    blocks = [Xp[i:i + 128] for i in range(0, S, 128)]
+    assert [len(b) for b in blocks] == [128, 128, 44]
+    m = np.stack([b.mean(axis=0) for b in blocks])
+    var_sum = sum(len(b) * np.var(b, axis=0).sum() for b in blocks)
+    assert O.residual_energy(X, perm, m) == pytest.approx(var_sum, rel=1e-12)
+    mu = rng.normal(size=m.shape).astype(np.float32)
+    shift = sum(len(b) * np.sum((mu[i].astype(np.float64) - m[i]) ** 2) for i, b in enumerate(blocks))
+    assert O.residual_energy(X, perm, mu) == pytest.approx(var_sum + shift, rel=1e-12)
+    zero = np.zeros_like(mu)
+    frob = np.linalg.norm(X.astype(np.float64)) ** 2
+    assert O.residual_energy(X, perm, zero) == pytest.approx(frob, rel=1e-12)
+    assert O.residual_energy(X, np.arange(S, dtype=np.int32), zero) == pytest.approx(frob, rel=1e-12)
+
+
+def test_residual_energy_depends_on_blocks_not_order_within_them():
+    S = 300
+    rng = np.random.default_rng(6)
+    X = _bf16_values((S, 128), 22, 1.0)
+    perm = rng.permutation(S).astype(np.int32)
+    mu = O.block_means(X, perm)
+    e = O.residual_energy(X, perm, mu)
+    # shuffling positions inside each block changes nothing ...
+    p2 = perm.copy()
+    for lo in range(0, S, 128):
+        p2[lo:lo + 128] = rng.permutation(p2[lo:lo + 128])
+    assert O.residual_energy(X, p2, mu) == pytest.approx(e, rel=1e-12)
+    # ... moving a token to another block does
+    p3 = perm.copy()
+    p3[[0, 200]] = p3[[200, 0]]
+    assert O.residual_energy(X, p3, mu) != pytest.approx(e, rel=1e-9)
+
+
+def test_cluster_sort_leaves_only_within_cluster_energy():
+    # Four groups of 128 tokens each, interleaved in the original order. Sorted
+    # by group, every block is one group, so with the block means of the sorted
+    # order the energy is the within-group scatter sum_c n_c sum_d var_cd; in
+    # the original order each block mixes the groups and keeps their spread.
+    rng = np.random.default_rng(7)
+    centers = rng.normal(size=(4, 128)) * 4.0
+    lab = rng.permutation(np.repeat(np.arange(4), 128))
+    X = (centers[lab] + rng.normal(size=(512, 128))).astype(np.float32)
+    X = torch.from_numpy(X).to(torch.bfloat16).float().numpy()
+    perm = O.cluster_permutation(lab)
+    within = sum(128 * np.var(X[lab == c].astype(np.float64), axis=0).sum() for c in range(4))
+    e_sorted = O.residual_energy(X, perm, O.block_means(X, perm))
+    assert e_sorted == pytest.approx(within, rel=1e-6)
+    ident = np.arange(512, dtype=np.int32)
+    e_orig = O.residual_energy(X, ident, O.block_means(X, ident))
+    assert e_orig > 5 * e_sorted
