@@ -56,8 +56,8 @@ def parse_args():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the SDPA comparison, accuracy, e2e and CPU-baseline legs")
     ap.add_argument("--extras", default="all",
-                    help="comma-separated extra legs after the timed region: accuracy, exp2, sdpa, e2e, cpu, ties "
-                         "(default all; --no-extras = none)")
+                    help="comma-separated extra legs after the timed region: accuracy, energy, exp2, sdpa, e2e, "
+                         "cpu, ties (default all; --no-extras = none)")
     ap.add_argument("--head-chunk", type=int, default=4,
                     help="heads per chunk of the host-buffer pipeline timed by the e2e leg")
     ap.add_argument("--sweep", choices=["nvfp4"], default=None,
@@ -322,7 +322,7 @@ def run_ours(args, cfg):
         "clocks": clk,
     }
     legs = set() if args.no_extras else (
-        {"accuracy", "exp2", "sdpa", "e2e", "cpu", "ties"} if args.extras == "all" else set(args.extras.split(",")))
+        {"accuracy", "energy", "exp2", "sdpa", "e2e", "cpu", "ties"} if args.extras == "all" else set(args.extras.split(",")))
     if legs:
         line.update(extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_step, rank, legs))
     if world > 1:
@@ -366,6 +366,37 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
         out["naive_v_rel_l2_vs_fp64"] = math.sqrt(num_naive / den)
         out["accuracy_sample"] = ("64 query rows x heads {0, H-1} of batch 0, exact fp64 softmax attention on the "
                                   "GPU; naive_v: the same path with V-Smooth off (V itself, one E4M3 scale per head)")
+    if "energy" in legs:
+        # residual energy per head: in the V-Smooth order with its block means, in
+        # the original order with block means, and of V itself; the share of the
+        # energy that the token ordering removes, over the heads of batch 0
+        torch.cuda.synchronize(dev)
+        pm = vc_attn.prepare_v(V, k=cfg["k"], iters=cfg["iters"], fmt=cfg["fmt"], mode="meanonly")
+        e_vs = vc_attn.residual_energy(V, plan.perm, plan.mu)
+        e_mo = vc_attn.residual_energy(V, pm["perm"], pm["mu"])
+        e_v = vc_attn.residual_energy(V)
+        cur = torch.cuda.current_stream(dev)
+        n = max(3, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(cur)
+        for _ in range(n):
+            vc_attn.residual_energy(V, plan.perm, plan.mu)
+        e1.record(cur)
+        torch.cuda.synchronize(dev)
+        ms_e = e0.elapsed_time(e1) / n
+        nb = (S + 127) // 128
+        alg_bytes = B * H * (S * (128 * V.element_size() + 4) + nb * 128 * 4)
+        f_sort = (1.0 - e_vs / e_mo)[0].cpu().numpy()
+        out["residual_energy"] = {
+            "removed_by_sort_mean": float(f_sort.mean()), "removed_by_sort_min": float(f_sort.min()),
+            "removed_by_sort_max": float(f_sort.max()),
+            "left_of_v_sorted": float((e_vs / e_v)[0].mean()), "left_of_v_meanonly": float((e_mo / e_v)[0].mean()),
+            "kernel_ms": ms_e, "kernel_gbs": alg_bytes / (ms_e * 1e-3) / 1e9,
+            "what": "per head of batch 0: 1 - E(cluster order, block means) / E(original order, block means), "
+                    "E = fp64 sum of ||v - mu_block||^2; left_of_v_*: E / ||V||^2; kernel: one "
+                    "vc_attn_residual_energy call (V gathered through perm, 128 x 2 B + 4 B per token-head)"}
+        del pm
     # the comparison kernel: the same fused attention with the probabilities made
     # by exp2 on the special function unit and an E4M3 conversion instead of
     # ExpCast (same prepared inputs, same stream)

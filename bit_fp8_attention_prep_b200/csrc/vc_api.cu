@@ -264,6 +264,23 @@ vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* sha
   return VC_OK;
 }
 
+vc_status_t vc_attn_residual_energy(const void* v, const vc_shape_t* shape, const int32_t* perm, const float* mu,
+                                    double* energy, void* stream) {
+  NvtxRange range("vc_attn_residual_energy");
+  g_last_error.clear();
+  vc_status_t st;
+  if ((st = check_shape(shape)) != VC_OK) return st;
+  if (!v || !energy) return fail(VC_ERR_INVALID_ARG, "v and energy must be non-NULL");
+  if (!aligned16(v) || !aligned16(perm) || !aligned16(mu) || !aligned16(energy))
+    return fail(VC_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if ((st = ensure_device()) != VC_OK) return st;
+  cudaError_t e = vc::launch_residual_energy(v, shape->dtype, shape->B, shape->S, shape->H, perm, mu, energy,
+                                             static_cast<cudaStream_t>(stream));
+  g_launches += 1;
+  if (e != cudaSuccess) return cuda_fail(e, "launching the residual-energy reduction");
+  return VC_OK;
+}
+
 static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                                   float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream,
                                   bool nvfp4, void* workspace, size_t workspace_bytes, bool exp2 = false) {

@@ -39,6 +39,9 @@ cudaError_t launch_prepare_v(const void* v, int dtype, const PrepPlan& plan, con
                              uint8_t* history, cudaStream_t st, int* nlaunch);
 cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int S, int H, const int32_t* perm,
                             const vc_qk_fp8_t& out, cudaStream_t st);
+// energy[B*H] (zeroed here) = sum of ||v[perm[p]] - mu[p/128]||^2 per slice; perm / mu may be NULL
+cudaError_t launch_residual_energy(const void* v, int dtype, int B, int S, int H, const int32_t* perm,
+                                   const float* mu, double* energy, cudaStream_t st);
 
 // Attention forward.
 struct AttnParams {

@@ -919,6 +919,65 @@ cudaError_t launch_nvfp4_planes(const uint8_t* codes, const uint8_t* scales, int
   return cudaGetLastError();
 }
 
+// --------------------------------------------------------------- residual energy (diagnostic)
+// E[bh] = sum over permuted positions p < S of ||v[perm[p]] - mu[p / 128]||^2:
+// the energy the residual quantiser sees. One CTA (4 warps) = one 128-token
+// block, rows gathered as in block_stats_kernel (two 256-byte rows per warp
+// load, eight loads in flight). Each lane forms its differences, squares and
+// sums in fp64 (a 16-bit input minus an fp32 mean is exact there unless the two
+// lie some 28 binades apart, and rounded once otherwise); the CTA's sum goes to
+// energy[bh] (zeroed by the launcher) with one double atomicAdd, so only the
+// summation order varies from run to run.
+// perm == NULL reads the identity order, mu == NULL zero means.
+template <typename T>
+__global__ void __launch_bounds__(128) residual_energy_kernel(const T* __restrict__ v, int S, int H,
+                                                              const int32_t* __restrict__ perm,
+                                                              const float* __restrict__ mu,
+                                                              double* __restrict__ energy) {
+  __shared__ double wsum[4];
+  const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int half = lane >> 4, c = lane & 15;
+  const int p0 = blk * kBlock, cnt = min(kBlock, S - p0);
+  const size_t row_stride = (size_t)H * kD;
+  const T* vbase = v + ((size_t)b * S * H + h) * kD + c * 8;
+  double m8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    m8[e] = mu ? (double)mu[((size_t)bh * gridDim.x + blk) * kD + c * 8 + e] : 0.0;
+  double acc = 0.0;
+#pragma unroll 1
+  for (int i0 = 0; i0 < 16; i0 += 8) {
+    int src[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = warp * 32 + 2 * (i0 + i) + half;
+      src[i] = r < cnt ? (perm ? perm[(size_t)bh * S + p0 + r] : p0 + r) : -1;
+    }
+    uint4 x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      x[i] = src[i] >= 0 ? *reinterpret_cast<const uint4*>(vbase + (size_t)src[i] * row_stride)
+                         : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (src[i] < 0) continue;
+      float f[8];
+      unpack8<T>(x[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const double d = (double)f[e] - m8[e];
+        acc = fma(d, d, acc);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) wsum[warp] = acc;
+  __syncthreads();
+  if (tid == 0) atomicAdd(&energy[bh], (wsum[0] + wsum[1]) + (wsum[2] + wsum[3]));
+}
+
 // --------------------------------------------------------------- launchers
 template <typename T>
 static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_prepared_v_t& out,
@@ -987,6 +1046,19 @@ cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int 
     quant_qk_kernel<__half><<<grid, 256, 0, st>>>(static_cast<const __half*>(q), static_cast<const __half*>(k), S,
                                                   H, nb * kBlock, perm, out.q_codes, out.q_scales, out.k_codes,
                                                   out.k_scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_residual_energy(const void* v, int dtype, int B, int S, int H, const int32_t* perm,
+                                   const float* mu, double* energy, cudaStream_t st) {
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(energy, 0, sizeof(double) * B * H, st)) != cudaSuccess) return e;
+  const dim3 grid((S + kBlock - 1) / kBlock, B * H);
+  if (dtype == VC_DTYPE_BF16)
+    residual_energy_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(v), S, H, perm,
+                                                                mu, energy);
+  else
+    residual_energy_kernel<__half><<<grid, 128, 0, st>>>(static_cast<const __half*>(v), S, H, perm, mu, energy);
   return cudaGetLastError();
 }
 

@@ -28,6 +28,7 @@ ABI_SYMBOLS = [
     "vc_attn_prepare_v",
     "vc_attn_quant_qk", "vc_attn_forward", "vc_attn_forward_nvfp4v_workspace_bytes", "vc_attn_forward_nvfp4v",
     "vc_attn_prepare_v_noalloc", "vc_attn_run_host_workspace_bytes", "vc_attn_run_host",
+    "vc_attn_residual_energy",
 ]
 NOALLOC_SCRATCH_BYTES = 12 << 20  # VC_ATTN_NOALLOC_SCRATCH_BYTES
 TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
@@ -97,6 +98,8 @@ def load():
     lib.vc_attn_run_host.restype = i32
     lib.vc_attn_run_host.argtypes = [vp, vp, vp, P(Shape), P(VSmoothCfg), ctypes.c_float, i32, vp, i32, vp, sz,
                                      vp, vp]
+    lib.vc_attn_residual_energy.restype = i32
+    lib.vc_attn_residual_energy.argtypes = [vp, P(Shape), vp, vp, vp, vp]
     lib.vc_attn_test_e4m3_round.restype = i32
     lib.vc_attn_test_e4m3_round.argtypes = [vp, vp, i64, vp]
     lib.vc_attn_test_e2m1_round.restype = i32
@@ -228,6 +231,22 @@ def quant_qk(q, k, perm):
     qk = QKFP8(_ptr(out["q_codes"]), _ptr(out["q_scales"]), _ptr(out["k_codes"]), _ptr(out["k_scales"]))
     _check(lib.vc_attn_quant_qk(_ptr(q), _ptr(k), ctypes.byref(sh), _ptr(perm), ctypes.byref(qk), _stream()))
     return out
+
+
+def residual_energy(v, perm=None, mu=None):
+    """Per-slice fp64 energy sum ||v[perm[p]] - mu[p // 128]||^2 as a [B, H]
+    device tensor (``perm`` None: identity order; ``mu`` None: zero means)."""
+    lib = load()
+    sh = shape_of(v)
+    nb = num_blocks(sh.S)
+    for name, t, shp, dt in (("perm", perm, (sh.B, sh.H, sh.S), torch.int32),
+                             ("mu", mu, (sh.B, sh.H, nb, 128), torch.float32)):
+        if t is not None and (tuple(t.shape) != shp or t.dtype != dt or not t.is_contiguous()
+                              or t.device != v.device):
+            raise ValueError(f"{name} must be a contiguous {dt} tensor of shape {shp} on {v.device}")
+    energy = torch.empty((sh.B, sh.H), dtype=torch.float64, device=v.device)
+    _check(lib.vc_attn_residual_energy(_ptr(v), ctypes.byref(sh), _ptr(perm), _ptr(mu), _ptr(energy), _stream()))
+    return energy
 
 
 def forward(qk, pv, shape, softmax_scale=None, k_p=8, out=None, status=None, workspace=None):

@@ -151,6 +151,25 @@ vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_v
 vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* shape,
                              const int32_t* perm, const vc_qk_fp8_t* out, void* stream);
 
+/* Residual energy of V-Smooth (diagnostic; "Nunchux AI lanza ...", 2nd
+ * paragraph, reports the share of the sequence energy that the token ordering
+ * removes, averaged over Wan2.2 heads): per (b, h)
+ *   energy[b*H + h] = sum_{p < S} sum_d (v[b, perm[p], h, d] - mu[p / 128][d])^2
+ * with the differences, squares and sums in fp64 (summation order unspecified,
+ * so the last bits may vary between runs). With perm and mu from
+ * vc_attn_prepare_v in VC_MODE_VSMOOTH this is the energy left for the residual
+ * quantiser; in VC_MODE_MEANONLY, the same without the cluster sort; with
+ * mu == NULL, the energy of V itself (VC_MODE_NAIVE).
+ *  v       device, [B,S,H,128] of shape->dtype
+ *  perm    device int32 [B,H,S] (permuted position -> token), or NULL for the
+ *          identity order
+ *  mu      device fp32 [B,H,nb,128] block means of the permuted order, or NULL
+ *          for zero means
+ *  energy  device fp64 [B,H], overwritten (zeroed on `stream`, then summed into)
+ * Errors: VC_ERR_INVALID_ARG (shape, NULL v / energy, alignment), VC_ERR_CUDA. */
+vc_status_t vc_attn_residual_energy(const void* v, const vc_shape_t* shape, const int32_t* perm,
+                                    const float* mu, double* energy, void* stream);
+
 /* Fused FP8 attention with ExpCast probabilities and the block-mean restore
  * ("VC-Attention ...", Abstract; "Hugging Face Introduces VC-Attention",
  * "Technical Breakthroughs and Core Innovations"), E4M3 V residual:

@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from bit_fp8_attention_prep_b200 import build, vc_attn
 
@@ -135,3 +136,26 @@ def test_run_host_workspace_and_validation(lib):
     ):
         assert lib.vc_attn_run_host(*args) == code
         assert lib.vc_attn_last_error() != b""
+
+
+def test_residual_energy_validation(lib):
+    # argument checks run on the host before anything is launched
+    sh = _shape(S=1000, H=5)
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    odd = ctypes.c_void_p(p.value + 8)
+    for args in (
+        (p, ctypes.byref(sh), None, None, None, None),              # energy NULL
+        (None, ctypes.byref(sh), None, None, p, None),              # v NULL
+        (p, ctypes.byref(_shape(D=64)), None, None, p, None),       # D != 128
+        (p, ctypes.byref(_shape(S=0)), None, None, p, None),        # empty sequence
+        (odd, ctypes.byref(sh), None, None, p, None),               # misaligned v
+        (p, ctypes.byref(sh), odd, None, p, None),                  # misaligned perm
+    ):
+        assert lib.vc_attn_residual_energy(*args) == vc_attn.VC_ERR_INVALID_ARG
+        assert lib.vc_attn_last_error() != b""
+    v = torch.zeros(1, 300, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        vc_attn.residual_energy(v, perm=torch.zeros(1, 2, 299, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        vc_attn.residual_energy(v, mu=torch.zeros(1, 2, 3, 128, dtype=torch.float64))

@@ -113,3 +113,46 @@ def test_naive_mode(va, fmt):
             assert g["s_v"][0, h] == ref["s_v"]
         else:
             assert np.array_equal(g["v_scales"][0, h], ref["v_scales"]) and g["s_v"][0, h] == ref["g"]
+
+
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+def test_residual_energy(va, dt):
+    # fp64 residual energy per slice: in the V-Smooth order with its block means,
+    # in the original order with its block means (perm given, and perm NULL), and
+    # of V itself (mu NULL), each against the oracle's own permutation and means
+    cfg, Q, K, V = make("mid", B=2, H=3, S=1000)      # 7 full blocks + 104
+    V = V.to(dt)
+    B, S, H = 2, 1000, 3
+    v = V.cuda()
+    pv = va.prepare_v(v, history=True)
+    pm = va.prepare_v(v, mode="meanonly")
+    e_vs = va.residual_energy(v, pv["perm"], pv["mu"]).cpu().numpy()
+    e_mo = va.residual_energy(v, pm["perm"], pm["mu"]).cpu().numpy()
+    e_id = va.residual_energy(v, None, pm["mu"]).cpu().numpy()
+    e_v = va.residual_energy(v).cpu().numpy()
+    hist = pv["history"].cpu().numpy()
+    ident = np.arange(S, dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            X = V[b, :, h].float().numpy()
+            ref = O.prepare_v_head(X, 16, 4, 0, b * H + h, adopt=[hist[t, b, h] for t in range(4)])
+            assert ref["stats"]["mismatches"] == 0, ref["stats"]
+            mo = O.prepare_v_head(X, 16, 4, 0, b * H + h, mode="meanonly")
+            # fp64 sums of 128 000 non-negative terms in two orders: a few ulps apart
+            assert e_vs[b, h] == pytest.approx(O.residual_energy(X, ref["perm"], ref["mu"]), rel=1e-12)
+            assert e_mo[b, h] == pytest.approx(O.residual_energy(X, ident, mo["mu"]), rel=1e-12)
+            assert e_id[b, h] == pytest.approx(e_mo[b, h], rel=1e-12)
+            assert e_v[b, h] == pytest.approx(O.residual_energy(X, ident, np.zeros((8, 128))), rel=1e-12)
+            assert e_vs[b, h] <= e_mo[b, h] <= e_v[b, h]
+
+
+def test_residual_energy_edges(va):
+    # one token (its own block mean: energy 0) and an all-zero head
+    V = torch.zeros(1, 1, 2, 128, dtype=torch.bfloat16)
+    V[0, 0, 0] = torch.arange(128) / 16
+    v = V.cuda()
+    pv = va.prepare_v(v, k=4, iters=2)
+    e = va.residual_energy(v, pv["perm"], pv["mu"]).cpu().numpy()
+    e_v = va.residual_energy(v).cpu().numpy()
+    assert e[0, 0] == 0.0 and e[0, 1] == 0.0
+    assert e_v[0, 0] == float(np.sum((np.arange(128) / 16.0) ** 2)) and e_v[0, 1] == 0.0
