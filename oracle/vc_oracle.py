@@ -54,6 +54,12 @@ Readings taken where the pages are silent (R-numbers are used in comments):
       uses); O = (sum_j P_ij v~_j + sum_b r_ib mu_b) / l_i, then BF16 RNE.
   R10 A block (or head) whose amax is below 2^-100 is treated as all zero:
       scale 1, codes 0.
+  R11 Optional K smoothing ([ABS]: prior work smooths queries and keys; the
+      pages give no form): K minus its per-channel mean over all tokens of the
+      (b, h) slice, the mean an int64 fixed-point sum as in R4, the difference
+      taken in fp32, before the per-block quantisation of R7. Every score of a
+      query row moves by the same q.kbar, so the softmax is unchanged. Q is not
+      smoothed (its mean would shift each key's score differently).
 """
 import math
 
@@ -79,7 +85,7 @@ __all__ = [
     "vres_from_e4m3", "vres_from_nvfp4", "quant_blocks_e4m3", "softmax_kappa",
     "expcast_codes", "expcast_bias", "expcast_online_probs", "vc_attention_rows", "vc_attention_exact_prob",
     "exact_attention_rows", "naive_v_e4m3", "prepare_v_head", "quant_qk_head",
-    "padded_len", "num_blocks", "residual_energy",
+    "padded_len", "num_blocks", "residual_energy", "token_mean", "smooth_k",
 ]
 
 
@@ -543,9 +549,27 @@ def prepare_v_head(V, k, iters, seed, bh, fmt="e4m3", adopt=None, mode="vsmooth"
     return out
 
 
-def quant_qk_head(Q, K, perm):
-    """Q/K per-block E4M3 quantisation for one slice; K gathered by ``perm``."""
+def token_mean(X):
+    """R11: per-channel mean over all tokens of one slice, int64 fixed-point sum
+    of x * 2^24, one fp64 division, rounded to fp32."""
+    X = np.asarray(X, np.float32)
+    s = np.rint(X.astype(np.float64) * 2.0 ** FIX_SHIFT).astype(np.int64).sum(axis=0)
+    return ((s.astype(np.float64) * 2.0 ** -FIX_SHIFT) / X.shape[0]).astype(np.float32)
+
+
+def smooth_k(K):
+    """R11: K minus its token mean (fp32 subtraction); returns (K - kbar, kbar)."""
+    K = np.asarray(K, np.float32)
+    kbar = token_mean(K)
+    return K - kbar, kbar
+
+
+def quant_qk_head(Q, K, perm, smooth=False):
+    """Q/K per-block E4M3 quantisation for one slice; K gathered by ``perm``
+    (after the R11 smoothing when ``smooth``)."""
     qc, qs = quant_blocks_e4m3(Q)
+    if smooth:
+        K = smooth_k(K)[0]
     kc, ks = quant_blocks_e4m3(K, order=perm)
     return qc, qs, kc, ks
 

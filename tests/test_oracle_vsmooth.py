@@ -279,3 +279,51 @@ def test_cluster_sort_leaves_only_within_cluster_energy():
     ident = np.arange(512, dtype=np.int32)
     e_orig = O.residual_energy(X, ident, O.block_means(X, ident))
     assert e_orig > 5 * e_sorted
+
+
+def test_token_mean_is_the_rounded_exact_mean():
+    # on the 2^-24 grid the fixed-point sum is exact, so the mean is the exact sum
+    # divided once in fp64 and rounded to fp32: numpy's own fp64 mean, rounded
+    X = _bf16_values((1000, 128), 31, 3.0) + np.float32(2.5)
+    assert np.array_equal(O.token_mean(X), X.astype(np.float64).mean(axis=0).astype(np.float32))
+    assert np.array_equal(O.token_mean(np.full((7, 128), -1.25, np.float32)), np.full(128, -1.25, np.float32))
+
+
+def test_k_smoothing_keeps_the_softmax_and_tightens_the_k_codes():
+    # Subtracting one vector from every key moves all scores of a query row by the
+    # same amount, so exact attention is unchanged. With a per-channel offset in K
+    # the smoothed block scales are several times smaller, the decoded smoothed K
+    # is within half an E4M3 step of K - kbar, and the VC-Attention output moves
+    # closer to exact attention.
+    rng = np.random.default_rng(9)
+    S = 300
+    bf = lambda a: torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).float().numpy()
+    Q = bf(rng.normal(size=(S, 128)))
+    K = bf(rng.normal(size=(S, 128)) + rng.normal(size=128) * 6.0)
+    V = bf(rng.normal(size=(S, 128)))
+    Ks, kbar = O.smooth_k(K)
+    assert np.array_equal(Ks, K - kbar)
+    assert np.abs(O.token_mean(Ks)).max() < 1e-5
+    rows = np.arange(0, S, 7)
+    scale = 1.0 / math.sqrt(128)
+    ref = O.exact_attention_rows(Q, K, V, rows, scale)
+    exact_diff = K.astype(np.float64) - kbar.astype(np.float64)
+    assert np.allclose(O.exact_attention_rows(Q, exact_diff, V, rows, scale), ref, rtol=1e-12, atol=1e-14)
+    # the fp32 difference is rounded (to 2^-21 of |K| here): scores move by ~1e-6 at most
+    assert np.allclose(O.exact_attention_rows(Q, Ks, V, rows, scale), ref, rtol=0, atol=1e-7)
+    prep = O.prepare_v_head(V, 16, 4, 0, 0)
+    err = {}
+    for smooth in (False, True):
+        qc, qs, kc, ks = O.quant_qk_head(Q, K, prep["perm"], smooth=smooth)
+        if smooth:
+            assert np.all(ks < ks_plain / 3)
+            dec = O.e4m3_table()[kc[:S]] * np.repeat(ks, 128)[:S, None]
+            Kp = Ks[prep["perm"]]
+            step = np.repeat(ks, 128)[:S, None] * 2.0 ** -10
+            assert np.all(np.abs(dec - Kp) <= np.abs(Kp) / 16 + step)
+        else:
+            ks_plain = ks
+        o = O.vc_attention_rows(qc, qs, kc, ks, prep["vres"], prep["mu"], S, rows, scale)
+        o = o[0] if isinstance(o, tuple) else o
+        err[smooth] = np.linalg.norm(o - ref) / np.linalg.norm(ref)
+    assert err[True] < 0.7 * err[False], err
