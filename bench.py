@@ -56,8 +56,8 @@ def parse_args():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the SDPA comparison, accuracy, e2e and CPU-baseline legs")
     ap.add_argument("--extras", default="all",
-                    help="comma-separated extra legs after the timed region: accuracy, energy, exp2, sdpa, e2e, "
-                         "cpu, ties (default all; --no-extras = none)")
+                    help="comma-separated extra legs after the timed region: accuracy, energy, smoothk, exp2, "
+                         "sdpa, e2e, cpu, ties (default all; --no-extras = none)")
     ap.add_argument("--head-chunk", type=int, default=4,
                     help="heads per chunk of the host-buffer pipeline timed by the e2e leg")
     ap.add_argument("--sweep", choices=["nvfp4"], default=None,
@@ -322,7 +322,7 @@ def run_ours(args, cfg):
         "clocks": clk,
     }
     legs = set() if args.no_extras else (
-        {"accuracy", "energy", "exp2", "sdpa", "e2e", "cpu", "ties"} if args.extras == "all" else set(args.extras.split(",")))
+        {"accuracy", "energy", "smoothk", "exp2", "sdpa", "e2e", "cpu", "ties"} if args.extras == "all" else set(args.extras.split(",")))
     if legs:
         line.update(extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_step, rank, legs))
     if world > 1:
@@ -397,6 +397,43 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
                     "E = fp64 sum of ||v - mu_block||^2; left_of_v_*: E / ||V||^2; kernel: one "
                     "vc_attn_residual_energy call (V gathered through perm, 128 x 2 B + 4 B per token-head)"}
         del pm
+    if "smoothk" in legs and cfg["fmt"] == "e4m3":
+        # K smoothing on keys with a per-(head, channel) offset (the synthetic K of
+        # the workload has none): rel-L2 against exact fp64 attention with and
+        # without the token-mean subtraction, and the time of the two Q/K calls
+        gen = torch.Generator(device=dev).manual_seed(11)
+        off = torch.randn((H, 128), generator=gen, device=dev) * 6.0
+        Ko = (K.float() + off).to(K.dtype)
+        pv = dict(perm=plan.perm, mu=plan.mu, v_codes=plan.v_codes, v_scales=None, s_v=plan.s_v)
+        cur = torch.cuda.current_stream(dev)
+        res = {}
+        for sm in (False, True):
+            qk = vc_attn.quant_qk(Q, Ko, plan.perm, smooth_k=sm)
+            ok = vc_attn.forward(qk, pv, plan.shape, plan.softmax_scale, plan.k_p).float()
+            n = max(3, min(args.steps, 10))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record(cur)
+            for _ in range(n):
+                qk = vc_attn.quant_qk(Q, Ko, plan.perm, smooth_k=sm)
+            e1.record(cur)
+            torch.cuda.synchronize(dev)
+            num = den = 0.0
+            for h in (0, H - 1):
+                q = Q[0, rows, h].double()
+                k, v = Ko[0, :, h].double(), V[0, :, h].double()
+                ref = torch.softmax((q @ k.t()) / math.sqrt(128), dim=-1) @ v
+                num += float(((ok[0, rows, h].double() - ref) ** 2).sum())
+                den += float((ref ** 2).sum())
+                del k, v, ref
+            res[sm] = (math.sqrt(num / den), e0.elapsed_time(e1) / n)
+            del qk, ok
+        out["k_smoothing"] = {"rel_l2_vs_fp64_plain": res[False][0], "rel_l2_vs_fp64_smoothed": res[True][0],
+                              "quant_qk_ms_plain": res[False][1], "quant_qk_ms_smoothed": res[True][1],
+                              "what": "K + N(0, 6^2) offset per (head, channel); vc_attn_quant_qk vs "
+                                      "vc_attn_quant_qk_smoothk, same prepared V, same forward; 64 rows x heads "
+                                      "{0, H-1} against exact fp64 attention"}
+        del Ko
     # the comparison kernel: the same fused attention with the probabilities made
     # by exp2 on the special function unit and an E4M3 conversion instead of
     # ExpCast (same prepared inputs, same stream)

@@ -257,10 +257,43 @@ vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* sha
       !aligned16(out->q_scales) || !aligned16(out->k_scales))
     return fail(VC_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
   if ((st = ensure_device()) != VC_OK) return st;
-  cudaError_t e = vc::launch_quant_qk(q, k, shape->dtype, shape->B, shape->S, shape->H, perm, *out,
-                                      static_cast<cudaStream_t>(stream));
-  g_launches += 1;
+  int n = 0;
+  cudaError_t e = vc::launch_quant_qk(q, k, shape->dtype, shape->B, shape->S, shape->H, perm, *out, nullptr,
+                                      nullptr, static_cast<cudaStream_t>(stream), &n);
+  g_launches += n;
   if (e != cudaSuccess) return cuda_fail(e, "launching Q/K quantisation");
+  return VC_OK;
+}
+
+size_t vc_attn_quant_qk_smoothk_workspace_bytes(const vc_shape_t* shape) {
+  if (check_shape(shape) != VC_OK) return 0;
+  return sizeof(unsigned long long) * (size_t)shape->B * shape->H * 128;
+}
+
+vc_status_t vc_attn_quant_qk_smoothk(const void* q, const void* k, const vc_shape_t* shape, const int32_t* perm,
+                                     const vc_qk_fp8_t* out, void* workspace, size_t workspace_bytes,
+                                     float* k_mean, void* stream) {
+  NvtxRange range("vc_attn_quant_qk_smoothk");
+  g_last_error.clear();
+  vc_status_t st;
+  if ((st = check_shape(shape)) != VC_OK) return st;
+  if (!q || !k || !perm || !out || !out->q_codes || !out->q_scales || !out->k_codes || !out->k_scales)
+    return fail(VC_ERR_INVALID_ARG, "q, k, perm, out and every field of out must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(perm) || !aligned16(out->q_codes) || !aligned16(out->k_codes) ||
+      !aligned16(out->q_scales) || !aligned16(out->k_scales) || !aligned16(k_mean))
+    return fail(VC_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  const size_t need = vc_attn_quant_qk_smoothk_workspace_bytes(shape);
+  if (!workspace || workspace_bytes < need)
+    return fail(VC_ERR_WORKSPACE, "K smoothing needs %zu bytes of workspace (got %zu)", need,
+                workspace ? workspace_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(VC_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if ((st = ensure_device()) != VC_OK) return st;
+  int n = 0;
+  cudaError_t e = vc::launch_quant_qk(q, k, shape->dtype, shape->B, shape->S, shape->H, perm, *out,
+                                      static_cast<unsigned long long*>(workspace), k_mean,
+                                      static_cast<cudaStream_t>(stream), &n);
+  g_launches += n;
+  if (e != cudaSuccess) return cuda_fail(e, "launching the smoothed Q/K quantisation");
   return VC_OK;
 }
 

@@ -37,8 +37,11 @@ cudaError_t prep_configure();
 // *nlaunch receives the number of kernels enqueued (memsets not counted).
 cudaError_t launch_prepare_v(const void* v, int dtype, const PrepPlan& plan, const vc_prepared_v_t& out,
                              uint8_t* history, cudaStream_t st, int* nlaunch);
+// ksum (optional, [B*H][128] int64, zeroed here): K smoothing by the token mean,
+// written to k_mean ([B*H][128] fp32) when that is given. *nlaunch: kernels enqueued.
 cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int S, int H, const int32_t* perm,
-                            const vc_qk_fp8_t& out, cudaStream_t st);
+                            const vc_qk_fp8_t& out, unsigned long long* ksum, float* k_mean, cudaStream_t st,
+                            int* nlaunch);
 // energy[B*H] (zeroed here) = sum of ||v[perm[p]] - mu[p/128]||^2 per slice; perm / mu may be NULL
 cudaError_t launch_residual_energy(const void* v, int dtype, int B, int S, int H, const int32_t* perm,
                                    const float* mu, double* energy, cudaStream_t st);

@@ -793,6 +793,51 @@ __global__ void __launch_bounds__(128) residual_nvfp4_kernel(const T* __restrict
   }
 }
 
+// --------------------------------------------------------------- token sums (K smoothing)
+// sums[bh][d] += sum over tokens of llrint(x * 2^24), the exact, order-free
+// int64 fixed-point sum (two's complement in the unsigned atomics). One CTA
+// (4 warps) = kSumRows tokens of one (b, h); row group g = 2 warp + half takes
+// rows g, g + 8, ...: each warp load reads two whole 256-byte rows, eight loads
+// in flight; lane l owns dimensions 8 (l % 16) .. 8 (l % 16) + 7.
+constexpr int kSumRows = 1024;
+
+template <typename T>
+__global__ void __launch_bounds__(128) token_sums_kernel(const T* __restrict__ x, int S, int H,
+                                                         unsigned long long* __restrict__ sums) {
+  __shared__ long long part[8][kD];
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, half = lane >> 4, c = lane & 15;
+  const int g = warp * 2 + half;
+  const int p0 = blockIdx.x * kSumRows, cnt = min(kSumRows, S - p0);
+  const size_t rs = (size_t)H * kD;
+  const T* base = x + (((size_t)b * S + p0) * H + h) * kD + c * 8;
+  long long acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll 1
+  for (int r0 = g; r0 < cnt; r0 += 64) {
+    uint4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = r0 + 8 * j;
+      v[j] = r < cnt ? *reinterpret_cast<const uint4*>(base + (size_t)r * rs) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float f[8];
+      unpack8<T>(v[j], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __float2ll_rn(f[e] * 16777216.0f);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[g][c * 8 + e] = acc[e];
+  __syncthreads();
+  const int d = threadIdx.x;
+  long long t = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t += part[i][d];
+  atomicAdd(&sums[(size_t)bh * kD + d], (unsigned long long)t);
+}
+
 // --------------------------------------------------------------- Q/K quantisation
 // One CTA (8 warps) = one 128-row block of Q (original order) or K (gathered by
 // perm). Warp w takes rows 16w .. 16w+15, two rows per load: lanes 0-15 read row
@@ -800,14 +845,22 @@ __global__ void __launch_bounds__(128) residual_nvfp4_kernel(const T* __restrict
 // whole 256-byte rows. The values stay in registers while the block amax is
 // reduced (warp shuffles, then shared memory); each lane then writes the 8 E4M3
 // codes of its 8 values (rows of 128 codes, contiguous per half warp).
-template <typename T>
+// With ksum (K smoothing: the per-channel int64 fixed-point token sums of K),
+// the K CTAs first subtract kbar = fl32((sum * 2^-24) / S) from every valid row
+// (an fp32 subtraction; padding rows stay 0), and the first block's CTA writes
+// kbar to k_mean when that is given (a separate instantiation, so that the
+// plain one keeps its register count and occupancy).
+template <typename T, bool kSmooth>
 __global__ void __launch_bounds__(256) quant_qk_kernel(const T* __restrict__ q, const T* __restrict__ k, int S,
                                                        int H, int S_pad, const int32_t* __restrict__ perm,
+                                                       const unsigned long long* __restrict__ ksum,
                                                        uint8_t* __restrict__ qc, float* __restrict__ qs,
-                                                       uint8_t* __restrict__ kc, float* __restrict__ ks) {
+                                                       uint8_t* __restrict__ kc, float* __restrict__ ks,
+                                                       float* __restrict__ k_mean) {
   __shared__ float wmax[8];
   const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
   const bool is_k = blockIdx.z == 1;
+  const bool smooth = kSmooth && is_k;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int half = lane >> 4, c = lane & 15;  // row parity and 16-byte piece of the row
   const T* const src = is_k ? k : q;
@@ -823,11 +876,31 @@ __global__ void __launch_bounds__(256) quant_qk_kernel(const T* __restrict__ q, 
   for (int i = 0; i < 8; ++i)
     x[i] = row[i] >= 0 ? *reinterpret_cast<const uint4*>(src + (((size_t)b * S + row[i]) * H + h) * kD + c * 8)
                        : make_uint4(0u, 0u, 0u, 0u);
-  float mx = 0.0f;  // rows past S are 0
+  float kb[8];
+  if (smooth) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const long long sum = (long long)ksum[(size_t)bh * kD + c * 8 + e];
+      kb[e] = __double2float_rn(__ddiv_rn((double)sum * 5.9604644775390625e-08, (double)S));
+    }
+    if (k_mean != nullptr && blk == 0 && warp == 0 && half == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) k_mean[(size_t)bh * kD + c * 8 + e] = kb[e];
+    }
+  }
+  // the values of row i (K smoothed when asked; rows past S are 0)
+  auto values = [&](int i, float* f) {
+    unpack8<T>(x[i], f);
+    if (smooth && row[i] >= 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = __fsub_rn(f[e], kb[e]);
+    }
+  };
+  float mx = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     float f[8];
-    unpack8<T>(x[i], f);
+    values(i, f);
 #pragma unroll
     for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
   }
@@ -848,7 +921,7 @@ __global__ void __launch_bounds__(256) quant_qk_kernel(const T* __restrict__ q, 
     uint2 w = make_uint2(0u, 0u);
     if (!zero) {  // rows past S hold zeros, which code to 0
       float f[8];
-      unpack8<T>(x[i], f);
+      values(i, f);
       w.x = (uint32_t)cvt_e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv)) |
             ((uint32_t)cvt_e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv)) << 16);
       w.y = (uint32_t)cvt_e4m3x2(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv)) |
@@ -1035,17 +1108,32 @@ cudaError_t launch_prepare_v(const void* v, int dtype, const PrepPlan& pl, const
 }
 
 cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int S, int H, const int32_t* perm,
-                            const vc_qk_fp8_t& out, cudaStream_t st) {
+                            const vc_qk_fp8_t& out, unsigned long long* ksum, float* k_mean, cudaStream_t st,
+                            int* nlaunch) {
   const int nb = (S + kBlock - 1) / kBlock;
   const dim3 grid(nb, B * H, 2);
-  if (dtype == VC_DTYPE_BF16)
-    quant_qk_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), S, H, nb * kBlock, perm,
-        out.q_codes, out.q_scales, out.k_codes, out.k_scales);
+  const bool bf = dtype == VC_DTYPE_BF16;
+  int n = 1;
+  if (ksum != nullptr) {
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(ksum, 0, sizeof(unsigned long long) * B * H * kD, st)) != cudaSuccess) return e;
+    const dim3 gs((S + kSumRows - 1) / kSumRows, B * H);
+    if (bf)
+      token_sums_kernel<__nv_bfloat16><<<gs, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(k), S, H, ksum);
+    else
+      token_sums_kernel<__half><<<gs, 128, 0, st>>>(static_cast<const __half*>(k), S, H, ksum);
+    ++n;
+  }
+  auto qk = bf ? (ksum ? quant_qk_kernel<__nv_bfloat16, true> : quant_qk_kernel<__nv_bfloat16, false>)
+              : nullptr;
+  auto qh = bf ? nullptr : (ksum ? quant_qk_kernel<__half, true> : quant_qk_kernel<__half, false>);
+  if (bf)
+    qk<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), S, H,
+                             nb * kBlock, perm, ksum, out.q_codes, out.q_scales, out.k_codes, out.k_scales, k_mean);
   else
-    quant_qk_kernel<__half><<<grid, 256, 0, st>>>(static_cast<const __half*>(q), static_cast<const __half*>(k), S,
-                                                  H, nb * kBlock, perm, out.q_codes, out.q_scales, out.k_codes,
-                                                  out.k_scales);
+    qh<<<grid, 256, 0, st>>>(static_cast<const __half*>(q), static_cast<const __half*>(k), S, H, nb * kBlock, perm,
+                             ksum, out.q_codes, out.q_scales, out.k_codes, out.k_scales, k_mean);
+  *nlaunch = n;
   return cudaGetLastError();
 }
 

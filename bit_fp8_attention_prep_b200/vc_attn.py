@@ -28,7 +28,7 @@ ABI_SYMBOLS = [
     "vc_attn_prepare_v",
     "vc_attn_quant_qk", "vc_attn_forward", "vc_attn_forward_nvfp4v_workspace_bytes", "vc_attn_forward_nvfp4v",
     "vc_attn_prepare_v_noalloc", "vc_attn_run_host_workspace_bytes", "vc_attn_run_host",
-    "vc_attn_residual_energy",
+    "vc_attn_residual_energy", "vc_attn_quant_qk_smoothk_workspace_bytes", "vc_attn_quant_qk_smoothk",
 ]
 NOALLOC_SCRATCH_BYTES = 12 << 20  # VC_ATTN_NOALLOC_SCRATCH_BYTES
 TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
@@ -98,6 +98,10 @@ def load():
     lib.vc_attn_run_host.restype = i32
     lib.vc_attn_run_host.argtypes = [vp, vp, vp, P(Shape), P(VSmoothCfg), ctypes.c_float, i32, vp, i32, vp, sz,
                                      vp, vp]
+    lib.vc_attn_quant_qk_smoothk_workspace_bytes.restype = sz
+    lib.vc_attn_quant_qk_smoothk_workspace_bytes.argtypes = [P(Shape)]
+    lib.vc_attn_quant_qk_smoothk.restype = i32
+    lib.vc_attn_quant_qk_smoothk.argtypes = [vp, vp, P(Shape), vp, P(QKFP8), vp, sz, vp, vp]
     lib.vc_attn_residual_energy.restype = i32
     lib.vc_attn_residual_energy.argtypes = [vp, P(Shape), vp, vp, vp, vp]
     lib.vc_attn_test_e4m3_round.restype = i32
@@ -213,8 +217,10 @@ def prepare_v_noalloc(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", hist
     return out
 
 
-def quant_qk(q, k, perm):
-    """Per-block E4M3 quantisation of Q and of K gathered through ``perm``."""
+def quant_qk(q, k, perm, smooth_k=False):
+    """Per-block E4M3 quantisation of Q and of K gathered through ``perm``.
+    ``smooth_k``: K minus its per-channel token mean first (vc_attn_quant_qk_smoothk;
+    the mean is returned as ``k_mean``, fp32 [B, H, 128])."""
     lib = load()
     sh = shape_of(q)
     if shape_of(k).S != sh.S or k.shape != q.shape or k.dtype != q.dtype:
@@ -229,7 +235,15 @@ def quant_qk(q, k, perm):
         k_scales=torch.empty((B, H, nb), dtype=torch.float32, device=dev),
     )
     qk = QKFP8(_ptr(out["q_codes"]), _ptr(out["q_scales"]), _ptr(out["k_codes"]), _ptr(out["k_scales"]))
-    _check(lib.vc_attn_quant_qk(_ptr(q), _ptr(k), ctypes.byref(sh), _ptr(perm), ctypes.byref(qk), _stream()))
+    if not smooth_k:
+        _check(lib.vc_attn_quant_qk(_ptr(q), _ptr(k), ctypes.byref(sh), _ptr(perm), ctypes.byref(qk), _stream()))
+        return out
+    wsb = lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(sh))
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    out["k_mean"] = torch.empty((B, H, 128), dtype=torch.float32, device=dev)
+    _check(lib.vc_attn_quant_qk_smoothk(_ptr(q), _ptr(k), ctypes.byref(sh), _ptr(perm), ctypes.byref(qk), _ptr(ws),
+                                        wsb, _ptr(out["k_mean"]), _stream()))
+    out["workspace"] = ws
     return out
 
 

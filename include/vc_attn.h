@@ -151,6 +151,32 @@ vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_v
 vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* shape,
                              const int32_t* perm, const vc_qk_fp8_t* out, void* stream);
 
+/* Bytes of device workspace vc_attn_quant_qk_smoothk needs: B*H*128*8 (0 for an
+ * invalid shape). */
+size_t vc_attn_quant_qk_smoothk_workspace_bytes(const vc_shape_t* shape);
+
+/* Q/K FP8 quantisation with K smoothing ("VC-Attention ...", Abstract: prior
+ * work smooths queries and keys): as vc_attn_quant_qk, but K is first reduced by
+ * its per-channel mean over the S tokens of each (b, h),
+ *   kbar[d] = fl32((sum_t llrint(k[t][d] * 2^24) * 2^-24) / S)   (exact int64 sum,
+ *             one double division)
+ *   k'[t][d] = fl32(k[t][d] - kbar[d]),
+ * and the per-block scales and E4M3 codes of K are those of k' (gathered through
+ * perm). Every score of a query row moves by the same q . kbar, so softmax(Q K^T)
+ * is unchanged, while keys with large channel offsets quantise with much finer
+ * block scales. Q is quantised as by vc_attn_quant_qk. The outputs feed
+ * vc_attn_forward / vc_attn_forward_nvfp4v unchanged.
+ *  q, k, perm, out  as vc_attn_quant_qk
+ *  workspace        device, >= vc_attn_quant_qk_smoothk_workspace_bytes(shape),
+ *                   16-B aligned; contents on entry ignored, undefined after
+ *  k_mean           optional device fp32 [B,H,128]: receives kbar; NULL to skip
+ * The int64 sums wrap (as two's complement) only when |sum_t k[t][d]| reaches
+ * 2^39, far beyond BF16 / FP16 activations of the supported sizes.
+ * Errors: VC_ERR_INVALID_ARG, VC_ERR_WORKSPACE, VC_ERR_CUDA. */
+vc_status_t vc_attn_quant_qk_smoothk(const void* q, const void* k, const vc_shape_t* shape,
+                                     const int32_t* perm, const vc_qk_fp8_t* out, void* workspace,
+                                     size_t workspace_bytes, float* k_mean, void* stream);
+
 /* Residual energy of V-Smooth (diagnostic; "Nunchux AI lanza ...", 2nd
  * paragraph, reports the share of the sequence energy that the token ordering
  * removes, averaged over Wan2.2 heads): per (b, h)

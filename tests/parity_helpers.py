@@ -17,11 +17,12 @@ def head(X, b, h):
     return X[b, :, h].float().numpy()
 
 
-def gpu_pipeline(va, Q, K, V, k, iters, seed=0, fmt="e4m3", k_p=8, history=True, attend=True, mode="vsmooth"):
+def gpu_pipeline(va, Q, K, V, k, iters, seed=0, fmt="e4m3", k_p=8, history=True, attend=True, mode="vsmooth",
+                 smooth_k=False):
     """Q, K, V CPU tensors [B,S,H,128] -> dict of GPU outputs copied to the CPU."""
     q, kk, v = Q.cuda(), K.cuda(), V.cuda()
     pv = va.prepare_v(v, k=k, iters=iters, seed=seed, fmt=fmt, history=history, mode=mode)
-    qk = va.quant_qk(q, kk, pv["perm"])
+    qk = va.quant_qk(q, kk, pv["perm"], smooth_k=smooth_k)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     o = va.forward(qk, pv, va.shape_of(q), SCALE, k_p, status=status) if attend else None
     torch.cuda.synchronize()
@@ -29,16 +30,17 @@ def gpu_pipeline(va, Q, K, V, k, iters, seed=0, fmt="e4m3", k_p=8, history=True,
     return dict(perm=cpu(pv["perm"]), mu=cpu(pv["mu"]), v_codes=cpu(pv["v_codes"]), v_scales=cpu(pv["v_scales"]),
                 s_v=cpu(pv["s_v"]), history=cpu(pv["history"]), q_codes=cpu(qk["q_codes"]),
                 q_scales=cpu(qk["q_scales"]), k_codes=cpu(qk["k_codes"]), k_scales=cpu(qk["k_scales"]),
-                o=None if o is None else o.float().cpu().numpy(), status=int(status.item()))
+                o=None if o is None else o.float().cpu().numpy(), status=int(status.item()),
+                k_mean=cpu(qk.get("k_mean")))
 
 
-def oracle_head(g, Q, K, V, b, h, k, iters, seed=0, fmt="e4m3"):
+def oracle_head(g, Q, K, V, b, h, k, iters, seed=0, fmt="e4m3", smooth_k=False):
     """Oracle prep + quantisation for slice (b, h), in lock-step with the GPU's
     per-pass k-means assignments (near ties adopted and counted)."""
     H = V.shape[2]
     adopt = None if g.get("history") is None else [g["history"][t, b, h] for t in range(iters)]
     prep = O.prepare_v_head(head(V, b, h), k, iters, seed, b * H + h, fmt=fmt, adopt=adopt)
-    qc, qs, kc, ks = O.quant_qk_head(head(Q, b, h), head(K, b, h), prep["perm"])
+    qc, qs, kc, ks = O.quant_qk_head(head(Q, b, h), head(K, b, h), prep["perm"], smooth=smooth_k)
     prep.update(q_codes=qc, q_scales=qs, k_codes=kc, k_scales=ks)
     return prep
 

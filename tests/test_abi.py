@@ -159,3 +159,25 @@ def test_residual_energy_validation(lib):
         vc_attn.residual_energy(v, perm=torch.zeros(1, 2, 299, dtype=torch.int32))
     with pytest.raises(ValueError):
         vc_attn.residual_energy(v, mu=torch.zeros(1, 2, 3, 128, dtype=torch.float64))
+
+
+def test_quant_qk_smoothk_workspace_and_validation(lib):
+    sh = _shape(B=2, S=1000, H=5)
+    assert lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(sh)) == 2 * 5 * 128 * 8
+    assert lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(_shape(D=64))) == 0
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    qk = vc_attn.QKFP8(p, p, p, p)
+    odd = ctypes.c_void_p(p.value + 4)
+    need = 2 * 5 * 128 * 8
+    for args, code in (
+        ((p, p, ctypes.byref(sh), p, ctypes.byref(qk), None, need, None, None), vc_attn.VC_ERR_WORKSPACE),
+        ((p, p, ctypes.byref(sh), p, ctypes.byref(qk), p, need - 1, None, None), vc_attn.VC_ERR_WORKSPACE),
+        ((p, None, ctypes.byref(sh), p, ctypes.byref(qk), p, need, None, None), vc_attn.VC_ERR_INVALID_ARG),
+        ((p, p, ctypes.byref(sh), None, ctypes.byref(qk), p, need, None, None), vc_attn.VC_ERR_INVALID_ARG),
+        ((p, p, ctypes.byref(sh), p, ctypes.byref(qk), odd, need, None, None), vc_attn.VC_ERR_INVALID_ARG),
+        ((p, p, ctypes.byref(sh), p, ctypes.byref(qk), p, need, odd, None), vc_attn.VC_ERR_INVALID_ARG),
+        ((p, p, ctypes.byref(_shape(S=0)), p, ctypes.byref(qk), p, need, None, None), vc_attn.VC_ERR_INVALID_ARG),
+    ):
+        assert lib.vc_attn_quant_qk_smoothk(*args) == code
+        assert lib.vc_attn_last_error() != b""

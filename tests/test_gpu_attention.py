@@ -1,6 +1,8 @@
 """GPU: the fused ExpCast attention matches the oracle's VC-attention output
 within the acceptance bars (rel-L2 <= 2e-3, max-abs <= 1e-2), across full and
 ragged tiles, both probability biases, FP16 input and the NVFP4 residual."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -129,3 +131,28 @@ def test_attention_exp2_comparison_kernel(va):
         e_cast = rel_l2(o_cast[0, rows, h], exact)
         print(f"head {h}: rel-L2 vs exact: ExpCast {e_cast:.4f}, exp2 + E4M3 {e_exp2:.4f}")
         assert e_exp2 < 0.05 and rel_l2(o_exp2[0, rows, h], o_cast[0, rows, h]) < 0.05
+
+
+def test_forward_with_smoothed_keys(va):
+    # K smoothing end to end: prep bit-exact with the oracle, O within the parity
+    # bar of the oracle's VC-Attention on the same smoothed codes, and closer to
+    # exact fp64 attention than without smoothing
+    from test_gpu_prep import _offset_keys
+    cfg, Q, K, V = make("mid", B=1, H=2, S=1000)
+    K = _offset_keys(K, 3)
+    rows = np.arange(0, 1000, 9)
+    errs = {}
+    for smooth in (False, True):
+        g = gpu_pipeline(va, Q, K, V, 16, 4, smooth_k=smooth)
+        assert g["status"] == 0
+        num = den = 0.0
+        for h in range(2):
+            ref = oracle_head(g, Q, K, V, 0, h, 16, 4, smooth_k=smooth)
+            assert_prep_bit_exact(g, ref, 0, h)
+            if smooth:
+                assert_o_close(g["o"][0, rows, h], oracle_rows(ref, 1000, rows))
+            ex = O.exact_attention_rows(head(Q, 0, h), head(K, 0, h), head(V, 0, h), rows, SCALE)
+            num += float(((g["o"][0, rows, h] - ex) ** 2).sum())
+            den += float((ex ** 2).sum())
+        errs[smooth] = math.sqrt(num / den)
+    assert errs[True] < 0.8 * errs[False], errs

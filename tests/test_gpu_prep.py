@@ -156,3 +156,53 @@ def test_residual_energy_edges(va):
     e_v = va.residual_energy(v).cpu().numpy()
     assert e[0, 0] == 0.0 and e[0, 1] == 0.0
     assert e_v[0, 0] == float(np.sum((np.arange(128) / 16.0) ** 2)) and e_v[0, 1] == 0.0
+
+
+def _offset_keys(K, seed, size=6.0):
+    # a per-(head, channel) offset on every key, as in the keys of DiT attention
+    g = torch.Generator().manual_seed(seed)
+    off = torch.randn(K.shape[2], K.shape[3], generator=g) * size
+    return (K.float() + off).to(K.dtype)
+
+
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+def test_quant_qk_smoothk_bit_exact(va, dt):
+    # K smoothing through a random permutation: codes, scales and the token mean
+    # are bit-exact with the oracle's; Q is untouched
+    cfg, Q, K, V = make("mid", B=2, H=3, S=1000)
+    Q, K = Q.to(dt), _offset_keys(K, 3).to(dt)
+    B, S, H = 2, 1000, 3
+    rng = np.random.default_rng(4)
+    perm = np.stack([np.stack([rng.permutation(S) for _ in range(H)]) for _ in range(B)]).astype(np.int32)
+    out = va.quant_qk(Q.cuda(), K.cuda(), torch.from_numpy(perm).cuda(), smooth_k=True)
+    plain = va.quant_qk(Q.cuda(), K.cuda(), torch.from_numpy(perm).cuda())
+    torch.cuda.synchronize()
+    g = {n: t.cpu().numpy() for n, t in out.items() if n != "workspace"}
+    for b in range(B):
+        for h in range(H):
+            Kh = K[b, :, h].float().numpy()
+            qc, qs, kc, ks = O.quant_qk_head(Q[b, :, h].float().numpy(), Kh, perm[b, h], smooth=True)
+            assert np.array_equal(g["k_mean"][b, h].view(np.uint32), O.token_mean(Kh).view(np.uint32))
+            assert np.array_equal(g["k_codes"][b, h], kc)
+            assert np.array_equal(g["k_scales"][b, h].view(np.uint32), ks.view(np.uint32))
+            assert np.array_equal(g["q_codes"][b, h], qc)
+            assert np.array_equal(g["q_scales"][b, h].view(np.uint32), qs.view(np.uint32))
+    assert np.array_equal(g["q_codes"], plain["q_codes"].cpu().numpy())
+    assert (g["k_scales"] < plain["k_scales"].cpu().numpy() / 2).all()
+
+
+@pytest.mark.parametrize("S", [1, 129])
+def test_quant_qk_smoothk_edges(va, S):
+    # one token (K - kbar = 0: scale 1, codes 0) and one token past a block
+    cfg, Q, K, V = make("mid", B=1, H=2, S=S)
+    K = _offset_keys(K, 5)
+    perm = torch.arange(S, dtype=torch.int32).repeat(1, 2, 1).contiguous()
+    out = va.quant_qk(Q.cuda(), K.cuda(), perm.cuda(), smooth_k=True)
+    torch.cuda.synchronize()
+    for h in range(2):
+        Kh = K[0, :, h].float().numpy()
+        qc, qs, kc, ks = O.quant_qk_head(Q[0, :, h].float().numpy(), Kh, np.arange(S), smooth=True)
+        assert np.array_equal(out["k_codes"][0, h].cpu().numpy(), kc)
+        assert np.array_equal(out["k_scales"][0, h].cpu().numpy().view(np.uint32), ks.view(np.uint32))
+    if S == 1:
+        assert not out["k_codes"].any() and (out["k_scales"] == 1).all()
