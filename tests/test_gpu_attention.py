@@ -8,7 +8,8 @@ import pytest
 import torch
 
 import oracle as O
-from parity_helpers import (SCALE, assert_o_close, gpu_pipeline, head, make, oracle_head, oracle_rows, rel_l2)
+from parity_helpers import (SCALE, assert_o_close, assert_prep_bit_exact, gpu_pipeline, head, make, oracle_head,
+                            oracle_rows, rel_l2)
 
 pytestmark = pytest.mark.gpu
 
