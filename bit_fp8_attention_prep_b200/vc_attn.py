@@ -295,12 +295,12 @@ def forward_nvfp4v_workspace_bytes(shape):
     return int(load().vc_attn_forward_nvfp4v_workspace_bytes(ctypes.byref(shape)))
 
 
-def attention(q, k, v, softmax_scale=None, k_p=8, kmeans_k=16, iters=4, seed=0, fmt="e4m3"):
-    """One call: V-Smooth prep, Q/K quantisation and the fused attention.
-    Q, K, V: [B,S,H,128] or [S,H,128] FP16/BF16 on the GPU; returns BF16 O with
-    the same layout."""
+def attention(q, k, v, softmax_scale=None, k_p=8, kmeans_k=16, iters=4, seed=0, fmt="e4m3", smooth_k=False):
+    """One call: V-Smooth prep, Q/K quantisation (K smoothed by its token mean
+    when ``smooth_k``) and the fused attention. Q, K, V: [B,S,H,128] or [S,H,128]
+    FP16/BF16 on the GPU; returns BF16 O with the same layout."""
     pv = prepare_v(v, k=kmeans_k, iters=iters, seed=seed, fmt=fmt)
-    qk = quant_qk(q, k, pv["perm"])
+    qk = quant_qk(q, k, pv["perm"], smooth_k=smooth_k)
     o = forward(qk, pv, shape_of(q), softmax_scale, k_p)
     return o.view(q.shape)
 
@@ -311,11 +311,13 @@ class Plan:
     workspace, O and a device status word, all owned by this object.
 
     ``run(q, k, v)`` enqueues the three calls (prepare_v, quant_qk, forward) on
-    the current stream and returns O; nothing is allocated per call.
+    the current stream and returns O; nothing is allocated per call. With
+    ``smooth_k`` the Q/K call is vc_attn_quant_qk_smoothk (K minus its token mean,
+    into the preallocated ``k_mean``).
     """
 
     def __init__(self, B, S, H, dtype=torch.bfloat16, k=16, iters=4, seed=0, fmt="e4m3", k_p=8,
-                 softmax_scale=None, device=None, mode="vsmooth"):
+                 softmax_scale=None, device=None, mode="vsmooth", smooth_k=False):
         self.lib = load()
         dev = torch.device(device if device is not None else "cuda")
         self.shape = Shape(B, S, H, 128, VC_DTYPE_BF16 if dtype == torch.bfloat16 else VC_DTYPE_F16)
@@ -347,14 +349,26 @@ class Plan:
             self._fwd_ws = e((self.fwd_ws_bytes,), torch.uint8)
         else:
             self.fwd_ws_bytes, self._fwd_ws = 0, None
+        self.smooth_k = bool(smooth_k)
+        if self.smooth_k:
+            self.smooth_ws_bytes = self.lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(self.shape))
+            self._smooth_ws = e((self.smooth_ws_bytes,), torch.uint8)
+            self.k_mean = e((B, H, 128), torch.float32)
+        else:
+            self.smooth_ws_bytes, self._smooth_ws, self.k_mean = 0, None, None
 
     def prepare_v(self, v):
         _check(self.lib.vc_attn_prepare_v(_ptr(v), ctypes.byref(self.shape), ctypes.byref(self.cfg),
                                           ctypes.byref(self._pv), self.ws_ptr, self.ws_bytes, None, _stream()))
 
     def quant_qk(self, q, k):
-        _check(self.lib.vc_attn_quant_qk(_ptr(q), _ptr(k), ctypes.byref(self.shape), _ptr(self.perm),
-                                         ctypes.byref(self._qk), _stream()))
+        if self.smooth_k:
+            _check(self.lib.vc_attn_quant_qk_smoothk(_ptr(q), _ptr(k), ctypes.byref(self.shape), _ptr(self.perm),
+                                                     ctypes.byref(self._qk), _ptr(self._smooth_ws),
+                                                     self.smooth_ws_bytes, _ptr(self.k_mean), _stream()))
+        else:
+            _check(self.lib.vc_attn_quant_qk(_ptr(q), _ptr(k), ctypes.byref(self.shape), _ptr(self.perm),
+                                             ctypes.byref(self._qk), _stream()))
 
     def forward(self, out=None):
         o = self.o if out is None else out

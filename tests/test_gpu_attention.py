@@ -157,3 +157,21 @@ def test_forward_with_smoothed_keys(va):
             den += float((ex ** 2).sum())
         errs[smooth] = math.sqrt(num / den)
     assert errs[True] < 0.8 * errs[False], errs
+
+
+def test_plan_and_attention_with_smoothed_keys_match_the_calls(va):
+    # the preallocated plan and the one-call helper give the same bytes as the
+    # separate calls with K smoothing
+    from test_gpu_prep import _offset_keys
+    cfg, Q, K, V = make("mid", B=1, H=2, S=700)
+    K = _offset_keys(K, 8)
+    q, k, v = Q.cuda(), K.cuda(), V.cuda()
+    pv = va.prepare_v(v)
+    qk = va.quant_qk(q, k, pv["perm"], smooth_k=True)
+    o_calls = va.forward(qk, pv, va.shape_of(q))
+    plan = va.Plan(1, 700, 2, smooth_k=True)
+    o_plan = plan.run(q, k, v).clone()
+    o_one = va.attention(q, k, v, smooth_k=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o_plan, o_calls) and torch.equal(o_one, o_calls)
+    assert torch.equal(plan.k_mean, qk["k_mean"]) and torch.equal(plan.k_codes, qk["k_codes"])
