@@ -54,6 +54,13 @@ Readings taken where the pages are silent (R-numbers are used in comments):
       uses); O = (sum_j P_ij v~_j + sum_b r_ib mu_b) / l_i, then BF16 RNE.
   R10 A block (or head) whose amax is below 2^-100 is treated as all zero:
       scale 1, codes 0.
+  R12 Optional V residual repair ([OVC]: re-adds the quantisation residual of
+      the worst-rounded value tokens, with a budget such as 0.005): for an E4M3
+      residual, the ceil(budget * S) tokens of the slice whose decoded value
+      s_V dec(code) is farthest from the residual r it codes (squared L2 over
+      the channels, fp64; ties to the lower permuted position) get their error
+      r - s_V dec(code) back, stored in fp32. The probabilities are untouched:
+      only those tokens' values in the P V product change.
   R11 Optional K smoothing ([ABS]: prior work smooths queries and keys; the
       pages give no form): K minus its per-channel mean over all tokens of the
       (b, h) slice, the mean an int64 fixed-point sum as in R4, the difference
@@ -85,7 +92,7 @@ __all__ = [
     "vres_from_e4m3", "vres_from_nvfp4", "quant_blocks_e4m3", "softmax_kappa",
     "expcast_codes", "expcast_bias", "expcast_online_probs", "vc_attention_rows", "vc_attention_exact_prob",
     "exact_attention_rows", "naive_v_e4m3", "prepare_v_head", "quant_qk_head",
-    "padded_len", "num_blocks", "residual_energy", "token_mean", "smooth_k",
+    "padded_len", "num_blocks", "residual_energy", "token_mean", "smooth_k", "residual_repair",
 ]
 
 
@@ -350,6 +357,24 @@ def residual_nvfp4(X, perm, mu):
 def vres_from_e4m3(vt, s_v, S):
     """Decoded residual values (S, D) float64: s_V * dec(code)."""
     return float(s_v) * _E4M3[vt[:, :S]].T
+
+
+def residual_repair(X, perm, mu, vt, s_v, budget):
+    """R12: the repair of an E4M3 residual. Returns (positions, corrections,
+    repaired values): the permuted positions of the kept tokens (ascending),
+    their fp32 corrections (m, D), and the decoded residual (S, D, fp64) with the
+    corrections added at those positions."""
+    r = _residual_f32(X, perm, mu).astype(np.float64)
+    S = r.shape[0]
+    vres = vres_from_e4m3(vt, s_v, S)
+    err = np.sum((r - vres) ** 2, axis=1)
+    m = min(S, int(math.ceil(budget * S)))
+    order = np.lexsort((np.arange(S), -err))     # largest error first, then lower position
+    pos = np.sort(order[:m])
+    delta = (r[pos] - vres[pos]).astype(np.float32)
+    rep = vres.copy()
+    rep[pos] += delta.astype(np.float64)
+    return pos, delta, rep
 
 
 def vres_from_nvfp4(packed, scales, g, S):

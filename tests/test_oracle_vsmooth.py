@@ -3,6 +3,7 @@
 Brute force with exact rational arithmetic on tiny inputs, a published
 splitmix64 output, and the closed-form properties of each step.
 """
+import itertools
 import math
 from fractions import Fraction
 
@@ -327,3 +328,74 @@ def test_k_smoothing_keeps_the_softmax_and_tightens_the_k_codes():
         o = o[0] if isinstance(o, tuple) else o
         err[smooth] = np.linalg.norm(o - ref) / np.linalg.norm(ref)
     assert err[True] < 0.7 * err[False], err
+
+
+def _repair_case(S, seed, k=4):
+    g = torch.Generator().manual_seed(seed)
+    V = torch.randn(S, 128, generator=g) * 2
+    V[::17] *= 20                                  # a few outlier tokens
+    X = V.to(torch.bfloat16).float().numpy()
+    return X, O.prepare_v_head(X, k, 2, 0, 0)
+
+
+def test_residual_repair_ends_and_exactness():
+    X, prep = _repair_case(300, 41)
+    args = (X, prep["perm"], prep["mu"], prep["v_codes"], prep["s_v"])
+    pos, delta, rep = O.residual_repair(*args, 0.0)
+    assert len(pos) == 0 and np.array_equal(rep, prep["vres"])
+    # budget 1: every token gets its value back, up to the fp32 rounding of its correction
+    r = (X[prep["perm"]] - prep["mu"][np.arange(300) // 128]).astype(np.float64)
+    pos, delta, rep = O.residual_repair(*args, 1.0)
+    assert np.array_equal(pos, np.arange(300))
+    assert np.all(np.abs(rep - r) <= 2.0 ** -24 * np.abs(r - prep["vres"]))
+    # the budget is a share of the slice's tokens, rounded up
+    assert [len(O.residual_repair(*args, b)[0]) for b in (0.005, 0.01, 0.1)] == [2, 3, 30]
+
+
+def test_residual_repair_keeps_the_worst_tokens_by_brute_force():
+    # 12 tokens, two pairs of them identical (exact ties of the error). For m of
+    # 3, 9 and 11 every m-subset is tried: the kept one removes the most squared
+    # error (exactly rounded sums), and among equal errors the lower permuted
+    # positions are kept (the pairs straddle the cut at m = 9 and m = 11)
+    g = torch.Generator().manual_seed(43)
+    V = torch.randn(12, 128, generator=g) * 3
+    V[7] = V[2]
+    V[9] = V[4]
+    X = V.to(torch.bfloat16).float().numpy()
+    prep = O.prepare_v_head(X, 1, 1, 0, 0, mode="meanonly")     # identity order, one block
+    args = (X, prep["perm"], prep["mu"], prep["v_codes"], prep["s_v"])
+    vres = prep["vres"]
+    r = [[float(X[j, d]) - float(prep["mu"][0, d]) for d in range(128)] for j in range(12)]
+    err = [math.fsum((r[j][d] - vres[j, d]) ** 2 for d in range(128)) for j in range(12)]
+    assert err[2] == err[7] and err[4] == err[9]
+    for m in (3, 9, 11):
+        pos = O.residual_repair(*args, m / 12)[0].tolist()
+        best = max(itertools.combinations(range(12), m),
+                   key=lambda c: (math.fsum(err[j] for j in c), [-j for j in c]))
+        assert pos == list(best), (m, pos, best)
+    assert 2 in O.residual_repair(*args, 9 / 12)[0] and 7 not in O.residual_repair(*args, 9 / 12)[0]
+    assert 4 in O.residual_repair(*args, 11 / 12)[0] and 9 not in O.residual_repair(*args, 11 / 12)[0]
+
+
+def test_residual_repair_lowers_the_value_error_and_the_output_error():
+    X, prep = _repair_case(300, 47)
+    args = (X, prep["perm"], prep["mu"], prep["v_codes"], prep["s_v"])
+    r = (X[prep["perm"]] - prep["mu"][np.arange(300) // 128]).astype(np.float64)
+    left = []
+    for b in (0.0, 0.01, 0.05, 0.2):
+        pos, delta, rep = O.residual_repair(*args, b)
+        left.append(float(np.sum((rep - r) ** 2)))
+    assert left[0] > left[1] > left[2] > left[3]
+    g = torch.Generator().manual_seed(48)
+    Q = torch.randn(300, 128, generator=g).to(torch.bfloat16).float().numpy()
+    K = torch.randn(300, 128, generator=g).to(torch.bfloat16).float().numpy()
+    qc, qs, kc, ks = O.quant_qk_head(Q, K, prep["perm"])
+    rows = np.arange(0, 300, 5)
+    scale = 1.0 / math.sqrt(128)
+    ref = O.exact_attention_rows(Q, K, X, rows, scale)
+    e = {}
+    for b in (0.0, 0.05):
+        rep = O.residual_repair(*args, b)[2]
+        o = O.vc_attention_rows(qc, qs, kc, ks, rep, prep["mu"], 300, rows, scale)
+        e[b] = np.linalg.norm(o - ref) / np.linalg.norm(ref)
+    assert e[0.05] < e[0.0], e
