@@ -54,6 +54,14 @@ Readings taken where the pages are silent (R-numbers are used in comments):
       uses); O = (sum_j P_ij v~_j + sum_b r_ib mu_b) / l_i, then BF16 RNE.
   R10 A block (or head) whose amax is below 2^-100 is treated as all zero:
       scale 1, codes 0.
+  R13 MX-style FP4 residual (not described by the pages; the block-scaled FP4
+      operand form of the B200 tensor cores, a neighbour of the NVFP4 residual):
+      E2M1 codes with one power-of-two scale per 32 consecutive permuted tokens
+      of one channel, X = 2^e with e the smallest integer for which the group's
+      amax <= 6 * 2^e (so nothing clips; the OCP MX rule 2^(floor(log2 amax) - 2)
+      can clip a group's largest values by up to a quarter), e clamped to
+      [-127, 127] (an 8-bit biased exponent), codes E2M1(r / X) with RNE; an
+      all-zero group has e = -127 and codes 0. No per-head scale.
   R12 Optional V residual repair ([OVC]: re-adds the quantisation residual of
       the worst-rounded value tokens, with a budget such as 0.005): for an E4M3
       residual, the ceil(budget * S) tokens of the slice whose decoded value
@@ -93,6 +101,7 @@ __all__ = [
     "expcast_codes", "expcast_bias", "expcast_online_probs", "vc_attention_rows", "vc_attention_exact_prob",
     "exact_attention_rows", "naive_v_e4m3", "prepare_v_head", "quant_qk_head",
     "padded_len", "num_blocks", "residual_energy", "token_mean", "smooth_k", "residual_repair",
+    "mx_exponent", "residual_mxfp4", "vres_from_mxfp4",
 ]
 
 
@@ -377,6 +386,45 @@ def residual_repair(X, perm, mu, vt, s_v, budget):
     return pos, delta, rep
 
 
+MX_GROUP = 32
+
+
+def mx_exponent(amax):
+    """R13: smallest integer e with amax <= 6 * 2^e, clamped to [-127, 127]
+    (-127 for amax == 0). Exact: 6 * 2^e is exact in fp64."""
+    a = float(amax)
+    if not a > 0:
+        return -127
+    e = int(math.ceil(math.log2(a / E2M1_MAX)))
+    while e > -127 and E2M1_MAX * 2.0 ** (e - 1) >= a:
+        e -= 1
+    while E2M1_MAX * 2.0 ** e < a:
+        e += 1
+    return max(-127, min(127, e))
+
+
+def residual_mxfp4(X, perm, mu):
+    """R13: MX-style FP4 residual. Returns (codes (D, S_pad) uint8, one E2M1 code
+    per element, unpacked; biased exponents (D, S_pad/32) uint8 = e + 127)."""
+    r = _residual_f32(X, perm, mu)
+    S, D = r.shape
+    Sp = padded_len(S)
+    rt = np.zeros((D, Sp), np.float64)
+    rt[:, :S] = r.T
+    grp = rt.reshape(D, Sp // MX_GROUP, MX_GROUP)
+    gmax = np.max(np.abs(grp), axis=2)
+    e = np.vectorize(mx_exponent, otypes=[np.int64])(gmax)
+    scaled = grp / np.ldexp(1.0, e)[:, :, None]              # exact: a power of two
+    codes = e2m1_round(scaled.astype(np.float32)).reshape(D, Sp)
+    return codes.astype(np.uint8), (e + 127).astype(np.uint8)
+
+
+def vres_from_mxfp4(codes, e8, S):
+    """Decoded MX-style residual (S, D) float64: e2m1(code) * 2^(e8 - 127)."""
+    x = np.ldexp(1.0, np.repeat(e8.astype(np.int64) - 127, MX_GROUP, axis=1))
+    return (e2m1_table()[codes] * x)[:, :S].T
+
+
 def vres_from_nvfp4(packed, scales, g, S):
     """Decoded NVFP4 residual values (S, D) float64: e2m1 * dec(scale) * g."""
     D = packed.shape[0]
@@ -565,6 +613,9 @@ def prepare_v_head(V, k, iters, seed, bh, fmt="e4m3", adopt=None, mode="vsmooth"
     if fmt == "e4m3":
         vt, s_v, amax = residual_e4m3(V, perm, mu)
         out.update(v_codes=vt, s_v=s_v, amax=amax, vres=vres_from_e4m3(vt, s_v, S))
+    elif fmt == "mxfp4":
+        codes, e8 = residual_mxfp4(V, perm, mu)
+        out.update(v_codes=codes, v_scales=e8, vres=vres_from_mxfp4(codes, e8, S))
     elif fmt == "nvfp4":
         packed, scales, g, amax = residual_nvfp4(V, perm, mu)
         out.update(v_codes=packed, v_scales=scales, g=g, amax=amax,

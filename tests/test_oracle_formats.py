@@ -153,3 +153,60 @@ def test_expcast_piecewise_linear_error_bound(k_p):
     # subnormal codes (below the smallest normal 2^-6) sit on a linear 2^-9 grid:
     # the absolute error there stays below 2^-7.
     assert err.max() <= 2.0 ** -7
+
+
+def test_mx_exponent_is_the_smallest_non_clipping_power_of_two():
+    # brute force over every 8-bit exponent, at the boundaries 6 * 2^k, their
+    # fp64 neighbours, and random values
+    rng = np.random.default_rng(12)
+    vals = [0.0, 6.0 * 2.0 ** -127, 6.0 * 2.0 ** -130, 1e-30, 3e38]
+    for k in (-20, -3, 0, 1, 7):
+        b = 6.0 * 2.0 ** k
+        vals += [b, np.nextafter(b, 0.0), np.nextafter(b, np.inf)]
+    vals += list(np.abs(rng.normal(size=50)) * 10.0 ** rng.integers(-6, 6, size=50))
+    for a in vals:
+        want = min([k for k in range(-127, 128) if a <= 6.0 * 2.0 ** k])
+        assert O.mx_exponent(a) == want, (a, O.mx_exponent(a), want)
+
+
+def test_residual_mxfp4_nearest_codes_no_clipping_and_minimal_scale():
+    g = torch.Generator().manual_seed(13)
+    S = 300                                   # 9 full groups of 32 and a ragged one per channel
+    X = (torch.randn(S, 128, generator=g) * 2).to(torch.bfloat16).float().numpy()
+    X[::29] *= 40
+    X[:, 5] = 0                               # an all-zero channel
+    perm = np.random.default_rng(14).permutation(S).astype(np.int32)
+    mu = O.block_means(X, perm)
+    codes, e8 = O.residual_mxfp4(X, perm, mu)
+    Sp = O.padded_len(S)
+    assert codes.shape == (128, Sp) and e8.shape == (128, Sp // 32)
+    assert not codes[:, S:].any()
+    r = (X[perm] - mu[np.arange(S) // 128]).astype(np.float64)       # the residual, fp32 values
+    grid = np.array(O.e2m1_table(), np.float64)
+    dec = O.vres_from_mxfp4(codes, e8, S)
+    for d in (0, 5, 77):
+        for gi in range(Sp // 32):
+            seg = r[gi * 32: min(gi * 32 + 32, S), d]
+            if seg.size == 0:
+                continue
+            x = 2.0 ** (int(e8[d, gi]) - 127)
+            amax = np.abs(seg).max()
+            assert amax <= 6 * x                                      # nothing clips
+            assert amax == 0 and e8[d, gi] == 0 or amax > 3 * x       # a smaller power of two would clip
+            cand = np.abs(grid[None, :] * x - seg[:, None])           # every grid point
+            got = np.abs(dec[gi * 32: gi * 32 + seg.size, d] - seg)
+            assert np.all(got <= cand.min(axis=1))                    # nearest point of the scaled grid
+    assert not dec[:, 5].any()
+
+
+def test_residual_mxfp4_exact_on_the_scaled_grid():
+    # a group whose values are E2M1 values times one power of two decodes exactly
+    rng = np.random.default_rng(15)
+    grid = np.array(O.e2m1_table(), np.float32)
+    X = (grid[rng.integers(0, 16, size=(64, 128))] * np.float32(2.0 ** -9)).astype(np.float32)
+    X[0, :] = np.float32(6 * 2.0 ** -9)       # every group reaches the top of the grid
+    X[32, :] = np.float32(-6 * 2.0 ** -9)
+    perm = np.arange(64, dtype=np.int32)
+    codes, e8 = O.residual_mxfp4(X, perm, np.zeros((1, 128), np.float32))
+    assert (e8[:, :2] == 127 - 9).all() and (e8[:, 2:] == 0).all()     # the padding groups are all zero
+    assert np.array_equal(O.vres_from_mxfp4(codes, e8, 64), X.astype(np.float64))
