@@ -54,6 +54,10 @@ Readings taken where the pages are silent (R-numbers are used in comments):
       uses); O = (sum_j P_ij v~_j + sum_b r_ib mu_b) / l_i, then BF16 RNE.
   R10 A block (or head) whose amax is below 2^-100 is treated as all zero:
       scale 1, codes 0.
+  R14 Optional per-channel residual scale (SURVEY's next-4, an accuracy knob
+      beside [OVC]'s per-head V scale): s_V[d] = amax_d / 448 over the slice's
+      residual in channel d, codes E4M3(r * fl32(448 / amax_d)); a channel with
+      amax_d below 2^-100 gets scale 1 and codes 0 (R10).
   R13 MX-style FP4 residual (not described by the pages; the block-scaled FP4
       operand form of the B200 tensor cores, a neighbour of the NVFP4 residual):
       E2M1 codes with one power-of-two scale per 32 consecutive permuted tokens
@@ -101,7 +105,8 @@ __all__ = [
     "expcast_codes", "expcast_bias", "expcast_online_probs", "vc_attention_rows", "vc_attention_exact_prob",
     "exact_attention_rows", "naive_v_e4m3", "prepare_v_head", "quant_qk_head",
     "padded_len", "num_blocks", "residual_energy", "token_mean", "smooth_k", "residual_repair",
-    "mx_exponent", "residual_mxfp4", "vres_from_mxfp4",
+    "mx_exponent", "residual_mxfp4", "vres_from_mxfp4", "residual_e4m3_per_channel",
+    "vres_from_e4m3_per_channel",
 ]
 
 
@@ -331,6 +336,28 @@ def residual_e4m3(X, perm, mu):
     s_v = amax / np.float32(E4M3_MAX)
     vt[:, :S] = e4m3_round(r * inv).T
     return vt, np.float32(s_v), amax
+
+
+def residual_e4m3_per_channel(X, perm, mu):
+    """R14: the E4M3 residual with one scale per channel. Returns (V^T codes
+    (D, S_pad) uint8 with zero padding, s_V (D,) fp32, amax (D,) fp32)."""
+    r = _residual_f32(X, perm, mu)
+    S, D = r.shape
+    amax = np.max(np.abs(r), axis=0).astype(np.float32) if S else np.zeros(D, np.float32)
+    vt = np.zeros((D, padded_len(S)), np.uint8)
+    s_v = np.ones(D, np.float32)
+    for d in range(D):
+        if not amax[d] >= TINY_AMAX:
+            continue
+        inv = np.float32(E4M3_MAX) / amax[d]
+        s_v[d] = amax[d] / np.float32(E4M3_MAX)
+        vt[d, :S] = e4m3_round(r[:, d] * inv)
+    return vt, s_v, amax
+
+
+def vres_from_e4m3_per_channel(vt, s_v, S):
+    """Decoded per-channel residual (S, D) float64: s_V[d] * dec(code)."""
+    return (np.asarray(s_v, np.float64)[:, None] * _E4M3[vt[:, :S]]).T
 
 
 def residual_nvfp4(X, perm, mu):

@@ -399,3 +399,53 @@ def test_residual_repair_lowers_the_value_error_and_the_output_error():
         o = O.vc_attention_rows(qc, qs, kc, ks, rep, prep["mu"], 300, rows, scale)
         e[b] = np.linalg.norm(o - ref) / np.linalg.norm(ref)
     assert e[0.05] < e[0.0], e
+
+
+def test_residual_e4m3_per_channel_scales_codes_and_error():
+    # every channel's largest residual maps to the largest code; every code is the
+    # nearest (brute force) to r * 448 / amax_d; a zero channel gets scale 1 and
+    # codes 0; each channel's decoded error stays within its own half-step bound
+    X = _bf16_values((300, 128), 17, scale=1.0)
+    X[:, 9] = 0
+    perm = np.random.default_rng(18).permutation(300).astype(np.int32)
+    mu = O.block_means(X, perm)
+    vt, s_v, amax = O.residual_e4m3_per_channel(X, perm, mu)
+    r = X[perm] - mu[np.arange(300) // 128]
+    assert np.array_equal(amax, np.max(np.abs(r), axis=0))
+    assert s_v[9] == 1.0 and not vt[9].any() and not vt[:, 300:].any()
+    tab = O.e4m3_table()
+    for d in (0, 20, 127):
+        assert s_v[d] == amax[d] / np.float32(448)
+        j = int(np.argmax(np.abs(r[:, d])))
+        assert vt[d, j] & 0x7F == 0x7E
+        inv = np.float32(448) / amax[d]
+        for jj in range(0, 300, 7):
+            v = float(np.float32(r[jj, d] * inv))
+            want = _nearest_code_brute(abs(v), tab, 127) | (0x80 if math.copysign(1, v) < 0 else 0)
+            assert vt[d, jj] == want
+    dec = O.vres_from_e4m3_per_channel(vt, s_v, 300)
+    assert np.all(np.abs(dec - r) <= np.abs(r) / 16 + s_v[None, :] * 2.0 ** -10)
+
+
+@pytest.mark.parametrize("wide,gain", [(30.0, False), (3e4, True)])
+def test_per_channel_scale_helps_only_below_the_e4m3_normal_range(wide, gain):
+    # E4M3 keeps its relative precision over a 2^15 range below its maximum, so a
+    # head scale set by channels 30x wider costs the narrow channels nothing; only
+    # channels pushed into the subnormal codes (here 3e4x narrower) gain from
+    # their own scale
+    X = _bf16_values((300, 128), 19, scale=1.0)
+    X[:, :8] *= wide
+    X = torch.from_numpy(X).to(torch.bfloat16).float().numpy()
+    perm = np.arange(300, dtype=np.int32)
+    mu = O.block_means(X, perm)
+    r = X[perm] - mu[np.arange(300) // 128]
+    vt, s_v, _ = O.residual_e4m3_per_channel(X, perm, mu)
+    dec = O.vres_from_e4m3_per_channel(vt, s_v, 300)
+    vh, sh, _ = O.residual_e4m3(X, perm, mu)
+    head = O.vres_from_e4m3(vh, sh, 300)
+    e_ch = np.sum((dec - r)[:, 8:] ** 2)
+    e_head = np.sum((head - r)[:, 8:] ** 2)
+    if gain:
+        assert e_ch < 0.1 * e_head
+    else:
+        assert 0.8 * e_head < e_ch < 1.25 * e_head
