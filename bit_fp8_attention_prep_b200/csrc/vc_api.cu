@@ -61,6 +61,9 @@ vc_status_t check_shape(const vc_shape_t* sh) {
     return fail(VC_ERR_INVALID_ARG, "dtype must be VC_DTYPE_F16 or VC_DTYPE_BF16 (got %d)", sh->dtype);
   const long long n = (long long)sh->B * sh->H * nblocks(sh->S) * 128 * 128;
   if (n >= (1ll << 31)) return fail(VC_ERR_INVALID_ARG, "B*H*S_pad*128 = %lld exceeds 2^31", n);
+  // every kernel takes one grid row (blockIdx.y) per (b, h) slice
+  if ((long long)sh->B * sh->H > 65535)
+    return fail(VC_ERR_UNSUPPORTED, "B*H = %lld exceeds 65535 slices", (long long)sh->B * sh->H);
   return VC_OK;
 }
 

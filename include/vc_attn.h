@@ -30,7 +30,8 @@
  *    reported through the optional `dev_status` int (device memory, set by the
  *    caller to VC_OK before the call, read after the caller's own sync).
  *  - Sizes: S >= 1, H >= 1, B >= 1, D == 128, B*H*S_pad*128 < 2^31 elements per
- *    tensor, where nb = ceil(S/128) and S_pad = 128*nb.
+ *    tensor, where nb = ceil(S/128) and S_pad = 128*nb; B*H <= 65535 (else
+ *    VC_ERR_UNSUPPORTED: the kernels take one grid row per (b, h) slice).
  */
 #ifndef VC_ATTN_H
 #define VC_ATTN_H

@@ -181,3 +181,18 @@ def test_quant_qk_smoothk_workspace_and_validation(lib):
     ):
         assert lib.vc_attn_quant_qk_smoothk(*args) == code
         assert lib.vc_attn_last_error() != b""
+
+
+def test_too_many_slices_is_refused_before_any_launch(lib):
+    # B*H above 65535 fits the element limit when S <= 128 but not one grid row
+    # per slice: every entry point refuses it on the host
+    sh = _shape(B=2, S=100, H=40000)
+    cfg = _cfg(k=4, iters=2)
+    assert lib.vc_attn_prepare_v_workspace_bytes(ctypes.byref(sh), ctypes.byref(cfg)) == 0
+    assert lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(sh)) == 0
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    assert lib.vc_attn_residual_energy(p, ctypes.byref(sh), None, None, p, None) == vc_attn.VC_ERR_UNSUPPORTED
+    assert b"65535" in lib.vc_attn_last_error()
+    ok = _shape(B=1, S=100, H=65535)
+    assert lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(ok)) == 65535 * 128 * 8
