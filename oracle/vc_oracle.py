@@ -105,7 +105,7 @@ __all__ = [
     "expcast_codes", "expcast_bias", "expcast_online_probs", "vc_attention_rows", "vc_attention_exact_prob",
     "exact_attention_rows", "naive_v_e4m3", "prepare_v_head", "quant_qk_head",
     "padded_len", "num_blocks", "residual_energy", "token_mean", "smooth_k", "residual_repair",
-    "mx_exponent", "residual_mxfp4", "vres_from_mxfp4", "residual_e4m3_per_channel",
+    "residual_repair_planes", "mx_exponent", "residual_mxfp4", "vres_from_mxfp4", "residual_e4m3_per_channel",
     "vres_from_e4m3_per_channel",
 ]
 
@@ -450,6 +450,41 @@ def vres_from_mxfp4(codes, e8, S):
     """Decoded MX-style residual (S, D) float64: e2m1(code) * 2^(e8 - 127)."""
     x = np.ldexp(1.0, np.repeat(e8.astype(np.int64) - 127, MX_GROUP, axis=1))
     return (e2m1_table()[codes] * x)[:, :S].T
+
+
+def residual_repair_planes(X, perm, mu, budget):
+    """R12 in the form of two E4M3 planes at the residual's scale s_V: plane 0
+    holds the residual codes of R5; plane 1, for the kept tokens, the E4M3 codes
+    of each element's rounding error in code units, dlt = y - dec(code) with
+    y = fl32(r * fl32(448 / amax)) the value that was rounded (dlt is exact in
+    fp32), and 0 elsewhere. A token's error is sum_d fl32(dlt_d^2), added in fp32
+    channel by channel from d = 0 (a fixed order, so that any implementation
+    that follows it ranks the tokens identically); the ceil(budget * S) largest
+    are kept, ties to the lower permuted position.
+
+    Returns (positions ascending, plane 0 (D, S_pad), plane 1 (D, S_pad), s_V,
+    repaired values (S, D) fp64 = s_V (dec(plane 0) + dec(plane 1)))."""
+    r = _residual_f32(X, perm, mu)
+    S, D = r.shape
+    vt, s_v, amax = residual_e4m3(X, perm, mu)
+    lo = np.zeros_like(vt)
+    m = min(S, int(math.ceil(budget * S)))
+    if amax >= TINY_AMAX:
+        inv = np.float32(E4M3_MAX) / amax
+        y = r * inv                                                  # fp32, as R5 codes it
+        dlt = (y - _E4M3[vt[:, :S]].T.astype(np.float32)).astype(np.float32)
+        sq = dlt * dlt
+        err = np.zeros(S, np.float32)
+        for d in range(D):
+            err = err + sq[:, d]
+    else:
+        dlt = np.zeros((S, D), np.float32)
+        err = np.zeros(S, np.float32)
+    order = np.lexsort((np.arange(S), -err.astype(np.float64)))
+    pos = np.sort(order[:m])
+    lo[:, pos] = e4m3_round(dlt[pos]).T
+    rep = float(s_v) * (_E4M3[vt[:, :S]] + _E4M3[lo[:, :S]]).T
+    return pos, vt, lo, s_v, rep
 
 
 def vres_from_nvfp4(packed, scales, g, S):

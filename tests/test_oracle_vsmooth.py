@@ -449,3 +449,60 @@ def test_per_channel_scale_helps_only_below_the_e4m3_normal_range(wide, gain):
         assert e_ch < 0.1 * e_head
     else:
         assert 0.8 * e_head < e_ch < 1.25 * e_head
+
+
+def test_residual_repair_planes_selection_codes_and_agreement():
+    # Plane 0 is the residual code plane; the kept tokens are the largest by the
+    # fp32 channel-ordered error (recomputed here with scalar fp32 arithmetic);
+    # plane 1 holds the nearest E4M3 code of each kept element's error in code
+    # units and 0 elsewhere; on continuous data the kept set is the exact form's
+    # (fp64) one, and the repaired values sit within 2^-4 of the exact form's
+    # correction (plus E4M3's subnormal floor) of the residual.
+    X, prep = _repair_case(300, 51)
+    perm, mu = prep["perm"], prep["mu"]
+    pos, p0, p1, s_v, rep = O.residual_repair_planes(X, perm, mu, 0.05)
+    vt, s_ref, amax = O.residual_e4m3(X, perm, mu)
+    assert np.array_equal(p0, vt) and s_v == s_ref and len(pos) == 15
+    r = X[perm] - mu[np.arange(300) // 128]
+    inv = np.float32(448) / amax
+    tab = O.e4m3_table()
+    err = []
+    for j in range(300):
+        acc = np.float32(0)
+        for d in range(128):
+            dl = np.float32(np.float32(r[j, d] * inv) - np.float32(tab[vt[d, j]]))
+            acc = np.float32(acc + np.float32(dl * dl))
+        err.append(float(acc))
+    want = sorted(sorted(range(300), key=lambda j: (-err[j], j))[:15])
+    assert pos.tolist() == want
+    keep = np.zeros(300, bool)
+    keep[pos] = True
+    assert not p1[:, :300][:, ~keep].any() and not p1[:, 300:].any()
+    for j in pos[:4]:
+        for d in range(0, 128, 9):
+            dl = float(np.float32(np.float32(r[j, d] * inv) - np.float32(tab[vt[d, j]])))
+            want_c = _nearest_code_brute(abs(dl), tab, 127) | (0x80 if math.copysign(1, dl) < 0 else 0)
+            assert p1[d, j] == want_c or (dl == 0 and p1[d, j] & 0x7F == 0)
+    epos, delta, _ = O.residual_repair(X, perm, mu, vt, s_v, 0.05)
+    assert np.array_equal(epos, pos)
+    r64 = r.astype(np.float64)
+    assert np.all(np.abs(rep[pos] - r64[pos]) <= np.abs(delta) / 16 + float(s_v) * 2.0 ** -10)
+    assert np.sum((rep - r64) ** 2) < np.sum((prep["vres"] - r64) ** 2)
+
+
+def test_residual_repair_planes_ties_and_zero_head():
+    # identical tokens tie exactly and the lower position is kept; an all-zero
+    # slice repairs nothing
+    g = torch.Generator().manual_seed(52)
+    V = torch.randn(12, 128, generator=g) * 3
+    V[7] = V[2]
+    V[9] = V[4]
+    X = V.to(torch.bfloat16).float().numpy()
+    perm = np.arange(12, dtype=np.int32)
+    mu = np.zeros((1, 128), np.float32)
+    for m in range(1, 12):
+        pos = O.residual_repair_planes(X, perm, mu, m / 12)[0].tolist()
+        assert not (7 in pos and 2 not in pos) and not (9 in pos and 4 not in pos)
+    Z = np.zeros((40, 128), np.float32)
+    pos, p0, p1, s_v, rep = O.residual_repair_planes(Z, np.arange(40, dtype=np.int32), np.zeros((1, 128), np.float32), 0.5)
+    assert s_v == 1.0 and not p0.any() and not p1.any() and not rep.any()
