@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <cmath>
 #include <mutex>
 #include <string>
 #include <utility>
@@ -240,6 +241,43 @@ static vc_status_t prepare_v_impl(const void* v, const vc_shape_t* shape, const 
 
 extern "C" {
 
+size_t vc_attn_prepare_v_repair_workspace_bytes(const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg) {
+  if (check_shape(shape) != VC_OK || check_cfg(cfg) != VC_OK) return 0;
+  const size_t BH = (size_t)shape->B * shape->H;
+  return ws_layout(shape, cfg).total + align256(BH * (size_t)shape->S * 4) + align256(BH * 8);
+}
+
+vc_status_t vc_attn_prepare_v_repair(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                                     double budget, const vc_prepared_v_t* out, uint8_t* kept, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  NvtxRange range("vc_attn_prepare_v_repair");
+  g_last_error.clear();
+  vc_status_t st;
+  if ((st = check_shape(shape)) != VC_OK) return st;
+  if ((st = check_cfg(cfg)) != VC_OK) return st;
+  if (cfg->residual_fmt != VC_RESIDUAL_E4M3)
+    return fail(VC_ERR_UNSUPPORTED, "the residual repair is defined for the E4M3 residual only");
+  if (!(budget >= 0.0 && budget <= 1.0)) return fail(VC_ERR_INVALID_ARG, "budget must be in [0, 1]");
+  const size_t need = vc_attn_prepare_v_repair_workspace_bytes(shape, cfg);
+  if (!workspace || workspace_bytes < need)
+    return fail(VC_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                workspace ? workspace_bytes : (size_t)0);
+  const WsLayout w = ws_layout(shape, cfg);
+  if ((st = prepare_v_impl(v, shape, cfg, out, workspace, w.total, nullptr, stream, 0)) != VC_OK) return st;
+  const size_t BH = (size_t)shape->B * shape->H;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* err = reinterpret_cast<float*>(ws + w.total);
+  unsigned long long* thr = reinterpret_cast<unsigned long long*>(ws + w.total + align256(BH * (size_t)shape->S * 4));
+  const int m = (int)std::min<double>((double)shape->S, std::ceil(budget * (double)shape->S));
+  int n = 0;
+  cudaError_t e = vc::launch_repair(v, shape->dtype, shape->B, shape->S, shape->H, out->perm, out->mu,
+                                    reinterpret_cast<const unsigned int*>(ws + w.amax), out->v_codes, m, err, thr, kept,
+                                    static_cast<cudaStream_t>(stream), &n);
+  g_launches += (uint64_t)n;
+  if (e != cudaSuccess) return cuda_fail(e, "launching the residual repair");
+  return VC_OK;
+}
+
 vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
                               const vc_prepared_v_t* out, void* workspace, size_t workspace_bytes,
                               uint8_t* assign_history, void* stream) {
@@ -317,9 +355,14 @@ vc_status_t vc_attn_residual_energy(const void* v, const vc_shape_t* shape, cons
   return VC_OK;
 }
 
+// nvfp4: split pv's NVFP4 residual into two E4M3 planes in `workspace`, then the
+// two-plane kernel at value scale 8 g; two_planes: pv->v_codes already holds two
+// E4M3 planes at the residual's scale (the repaired residual); otherwise the
+// one-plane E4M3 kernel.
 static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                                   float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream,
-                                  bool nvfp4, void* workspace, size_t workspace_bytes, bool exp2 = false) {
+                                  bool nvfp4, void* workspace, size_t workspace_bytes, bool exp2 = false,
+                                  bool two_planes = false) {
   g_last_error.clear();
   vc_status_t st;
   if ((st = check_shape(shape)) != VC_OK) return st;
@@ -364,7 +407,10 @@ static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* 
   p.status = dev_status;
   p.wait_ns = 2000000000ull;
   cudaError_t e;
-  if (!nvfp4) {
+  if (two_planes) {
+    if ((st = make_map_u8(&tv, pv->v_codes, (uint64_t)S_pad, (uint64_t)2 * BH * 128)) != VC_OK) return st;
+    e = vc::launch_attn_planes(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  } else if (!nvfp4) {
     if ((st = make_map_u8(&tv, pv->v_codes, (uint64_t)S_pad, (uint64_t)BH * 128)) != VC_OK) return st;
     e = vc::launch_attn_e4m3(tq, tk, tv, p, static_cast<cudaStream_t>(stream), exp2);
   } else {
@@ -390,6 +436,12 @@ vc_status_t vc_attn_forward(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, co
 vc_status_t vc_attn_test_forward_exp2(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                                       float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
   return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, false, nullptr, 0, true);
+}
+
+vc_status_t vc_attn_forward_repair(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
+                                   float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
+  NvtxRange range("vc_attn_forward_repair");
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, false, nullptr, 0, false, true);
 }
 
 size_t vc_attn_forward_nvfp4v_workspace_bytes(const vc_shape_t* shape) {

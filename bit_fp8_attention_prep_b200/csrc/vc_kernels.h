@@ -42,6 +42,12 @@ cudaError_t launch_prepare_v(const void* v, int dtype, const PrepPlan& plan, con
 cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int S, int H, const int32_t* perm,
                             const vc_qk_fp8_t& out, unsigned long long* ksum, float* k_mean, cudaStream_t st,
                             int* nlaunch);
+// V residual repair on the two planes [2][B*H][128][S_pad] at `planes` (plane 0
+// written by the E4M3 prep, plane 1 here); m tokens kept per slice (0: plane 1
+// all zero); err [B*H][S] and thr [B*H] are scratch; kept (optional) [B*H][S].
+cudaError_t launch_repair(const void* v, int dtype, int B, int S, int H, const int32_t* perm, const float* mu,
+                          const unsigned int* amax_bits, uint8_t* planes, int m, float* err,
+                          unsigned long long* thr, uint8_t* kept, cudaStream_t st, int* nlaunch);
 // energy[B*H] (zeroed here) = sum of ||v[perm[p]] - mu[p/128]||^2 per slice; perm / mu may be NULL
 cudaError_t launch_residual_energy(const void* v, int dtype, int B, int S, int H, const int32_t* perm,
                                    const float* mu, double* energy, cudaStream_t st);

@@ -1051,6 +1051,152 @@ __global__ void __launch_bounds__(128) residual_energy_kernel(const T* __restric
   if (tid == 0) atomicAdd(&energy[bh], (wsum[0] + wsum[1]) + (wsum[2] + wsum[3]));
 }
 
+// --------------------------------------------------------------- V residual repair
+// "Open VC Attention", "Описание": the repair re-adds the quantisation residual
+// of the worst-rounded value tokens (budget e.g. 0.005). Two E4M3 planes at the
+// residual's scale s_V: plane 0 holds the residual codes (residual_e4m3_kernel),
+// plane 1, for the kept tokens, the E4M3 codes of each element's rounding error
+// in code units, dlt = y - dec(code) with y = fl32(fl32(x - mu) * fl32(448/amax))
+// the value that was rounded (exact in fp32), and 0 elsewhere; the two-plane
+// attention kernel then adds P (plane 0 + plane 1) at scale s_V.
+// A token's error is sum_d fl32(dlt_d^2), added in fp32 from d = 0 to 127; the
+// kept tokens are the m largest by the key (error, then lower position).
+
+// y - dec(code) of channel d of one token: the rounding error in code units.
+__device__ __forceinline__ float repair_dlt(float x, float m, float inv, uint32_t code) {
+  return __fsub_rn(__fmul_rn(__fsub_rn(x, m), inv), e4m3_to_f32(code));
+}
+
+// 64-bit ranking key: larger error first, then lower position (errors are >= 0,
+// so their bit patterns order like their values).
+__device__ __forceinline__ unsigned long long repair_key(float err, int p) {
+  return ((unsigned long long)__float_as_uint(err) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)p);
+}
+
+// err[bh][p] for every permuted position p < S. One CTA = one 128-token block,
+// one thread per token; the thread walks its gathered V row 16 bytes at a time
+// and reads its codes from the V^T plane (consecutive threads, consecutive bytes).
+template <typename T>
+__global__ void __launch_bounds__(128) repair_err_kernel(const T* __restrict__ v, int S, int H, int S_pad,
+                                                         const int32_t* __restrict__ perm,
+                                                         const float* __restrict__ mu,
+                                                         const unsigned int* __restrict__ amax_bits,
+                                                         const uint8_t* __restrict__ vt, float* __restrict__ err) {
+  __shared__ float smu[kD];
+  const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x, t = threadIdx.x;
+  smu[t] = mu[((size_t)bh * gridDim.x + blk) * kD + t];
+  __syncthreads();
+  const int p = blk * kBlock + t;
+  if (p >= S) return;
+  const float amax = __uint_as_float(amax_bits[bh]);
+  float e = 0.0f;
+  if (amax >= kTinyAmax) {
+    const float inv = __fdiv_rn(kE4M3Max, amax);
+    const T* row = v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD;
+    const uint8_t* code = vt + (size_t)bh * kD * S_pad + p;
+#pragma unroll 1
+    for (int c = 0; c < kD / 8; ++c) {
+      float f[8];
+      unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int d = c * 8 + i;
+        const float dl = repair_dlt(f[i], smu[d], inv, code[(size_t)d * S_pad]);
+        e = __fadd_rn(e, __fmul_rn(dl, dl));
+      }
+    }
+  }
+  err[(size_t)bh * S + p] = e;
+}
+
+// thr[bh] = the key of the m-th largest token (1 <= m <= S): a radix select over
+// the 64-bit keys, 8 bits per pass from the top, one CTA per (b, h). Each pass
+// counts the candidates (keys matching the digits chosen so far) per next digit
+// in shared memory and keeps the digit where the count from the top reaches the
+// remaining rank; keys are distinct, so exactly m keys are >= thr.
+__global__ void __launch_bounds__(256) repair_select_kernel(const float* __restrict__ err, int S, int m,
+                                                            unsigned long long* __restrict__ thr) {
+  __shared__ unsigned int hist[256];
+  __shared__ unsigned long long s_prefix;
+  __shared__ int s_left;
+  const int bh = blockIdx.x, t = threadIdx.x;
+  const float* e = err + (size_t)bh * S;
+  unsigned long long prefix = 0ull, mask = 0ull;
+  int left = m;
+#pragma unroll 1
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    hist[t] = 0u;
+    __syncthreads();
+    for (int p = t; p < S; p += 256) {
+      const unsigned long long k = repair_key(e[p], p);
+      if ((k & mask) == prefix) atomicAdd(&hist[(uint32_t)(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (t == 0) {
+      int above = 0, digit = 0;
+      for (int d = 255; d >= 0; --d) {
+        const int c = (int)hist[d];
+        if (above + c >= left) {
+          digit = d;
+          break;
+        }
+        above += c;
+      }
+      s_left = left - above;
+      s_prefix = prefix | ((unsigned long long)digit << shift);
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    left = s_left;
+    mask |= 0xFFull << shift;
+    __syncthreads();
+  }
+  if (t == 0) thr[bh] = prefix;
+}
+
+// Plane 1 (and the optional kept flags): one CTA = one 128-token block of
+// permuted positions, one thread per token; channel by channel the 128 threads
+// write 128 consecutive bytes of the V^T plane. Tokens not kept, padding tokens
+// and slices whose residual is all zero get 0.
+template <typename T>
+__global__ void __launch_bounds__(128) repair_plane_kernel(const T* __restrict__ v, int S, int H, int S_pad,
+                                                           const int32_t* __restrict__ perm,
+                                                           const float* __restrict__ mu,
+                                                           const unsigned int* __restrict__ amax_bits,
+                                                           const float* __restrict__ err,
+                                                           const unsigned long long* __restrict__ thr, bool any,
+                                                           const uint8_t* __restrict__ vt,
+                                                           uint8_t* __restrict__ plane1, uint8_t* __restrict__ kept) {
+  __shared__ float smu[kD];
+  const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x, t = threadIdx.x;
+  smu[t] = mu[((size_t)bh * gridDim.x + blk) * kD + t];
+  __syncthreads();
+  const int p = blk * kBlock + t;
+  const bool keep = any && p < S && repair_key(err[(size_t)bh * S + p], p) >= thr[bh];
+  if (kept != nullptr && p < S) kept[(size_t)bh * S + p] = keep ? 1 : 0;
+  uint8_t* out = plane1 + (size_t)bh * kD * S_pad + p;
+  const float amax = __uint_as_float(amax_bits[bh]);
+  if (!keep || !(amax >= kTinyAmax)) {
+#pragma unroll 4
+    for (int d = 0; d < kD; ++d) out[(size_t)d * S_pad] = 0;
+    return;
+  }
+  const float inv = __fdiv_rn(kE4M3Max, amax);
+  const T* row = v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD;
+  const uint8_t* code = vt + (size_t)bh * kD * S_pad + p;
+#pragma unroll 1
+  for (int c = 0; c < kD / 8; ++c) {
+    float f[8];
+    unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int d = c * 8 + i;
+      out[(size_t)d * S_pad] = cvt_e4m3(repair_dlt(f[i], smu[d], inv, code[(size_t)d * S_pad]));
+    }
+  }
+}
+
 // --------------------------------------------------------------- launchers
 template <typename T>
 static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_prepared_v_t& out,
@@ -1147,6 +1293,34 @@ cudaError_t launch_residual_energy(const void* v, int dtype, int B, int S, int H
                                                                 mu, energy);
   else
     residual_energy_kernel<__half><<<grid, 128, 0, st>>>(static_cast<const __half*>(v), S, H, perm, mu, energy);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_repair(const void* v, int dtype, int B, int S, int H, const int32_t* perm, const float* mu,
+                          const unsigned int* amax_bits, uint8_t* planes, int m, float* err,
+                          unsigned long long* thr, uint8_t* kept, cudaStream_t st, int* nlaunch) {
+  const int nb = (S + kBlock - 1) / kBlock, S_pad = nb * kBlock, BH = B * H;
+  const dim3 grid(nb, BH);
+  uint8_t* plane1 = planes + (size_t)BH * kD * S_pad;
+  const bool bf = dtype == VC_DTYPE_BF16;
+  int n = 0;
+  if (m > 0) {
+    if (bf)
+      repair_err_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(v), S, H, S_pad, perm,
+                                                             mu, amax_bits, planes, err);
+    else
+      repair_err_kernel<__half><<<grid, 128, 0, st>>>(static_cast<const __half*>(v), S, H, S_pad, perm, mu,
+                                                      amax_bits, planes, err);
+    repair_select_kernel<<<BH, 256, 0, st>>>(err, S, m, thr);
+    n += 2;
+  }
+  if (bf)
+    repair_plane_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(v), S, H, S_pad, perm,
+                                                             mu, amax_bits, err, thr, m > 0, planes, plane1, kept);
+  else
+    repair_plane_kernel<__half><<<grid, 128, 0, st>>>(static_cast<const __half*>(v), S, H, S_pad, perm, mu,
+                                                      amax_bits, err, thr, m > 0, planes, plane1, kept);
+  *nlaunch = n + 1;
   return cudaGetLastError();
 }
 

@@ -29,6 +29,7 @@ ABI_SYMBOLS = [
     "vc_attn_quant_qk", "vc_attn_forward", "vc_attn_forward_nvfp4v_workspace_bytes", "vc_attn_forward_nvfp4v",
     "vc_attn_prepare_v_noalloc", "vc_attn_run_host_workspace_bytes", "vc_attn_run_host",
     "vc_attn_residual_energy", "vc_attn_quant_qk_smoothk_workspace_bytes", "vc_attn_quant_qk_smoothk",
+    "vc_attn_prepare_v_repair_workspace_bytes", "vc_attn_prepare_v_repair", "vc_attn_forward_repair",
 ]
 NOALLOC_SCRATCH_BYTES = 12 << 20  # VC_ATTN_NOALLOC_SCRATCH_BYTES
 TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
@@ -102,6 +103,13 @@ def load():
     lib.vc_attn_quant_qk_smoothk_workspace_bytes.argtypes = [P(Shape)]
     lib.vc_attn_quant_qk_smoothk.restype = i32
     lib.vc_attn_quant_qk_smoothk.argtypes = [vp, vp, P(Shape), vp, P(QKFP8), vp, sz, vp, vp]
+    lib.vc_attn_prepare_v_repair_workspace_bytes.restype = sz
+    lib.vc_attn_prepare_v_repair_workspace_bytes.argtypes = [P(Shape), P(VSmoothCfg)]
+    lib.vc_attn_prepare_v_repair.restype = i32
+    lib.vc_attn_prepare_v_repair.argtypes = [vp, P(Shape), P(VSmoothCfg), ctypes.c_double, P(PreparedV), vp, vp,
+                                             sz, vp]
+    lib.vc_attn_forward_repair.restype = i32
+    lib.vc_attn_forward_repair.argtypes = [P(QKFP8), P(PreparedV), P(Shape), ctypes.c_float, i32, vp, vp, vp]
     lib.vc_attn_residual_energy.restype = i32
     lib.vc_attn_residual_energy.argtypes = [vp, P(Shape), vp, vp, vp, vp]
     lib.vc_attn_test_e4m3_round.restype = i32
@@ -244,6 +252,51 @@ def quant_qk(q, k, perm, smooth_k=False):
     _check(lib.vc_attn_quant_qk_smoothk(_ptr(q), _ptr(k), ctypes.byref(sh), _ptr(perm), ctypes.byref(qk), _ptr(ws),
                                         wsb, _ptr(out["k_mean"]), _stream()))
     out["workspace"] = ws
+    return out
+
+
+def prepare_v_repair(v, budget=0.005, k=16, iters=4, seed=0, mode="vsmooth"):
+    """V-Smooth prep with the V residual repair (E4M3 residual): returns the
+    prepared-V dict of ``prepare_v`` whose ``v_codes`` holds the two planes
+    [2, B, H, 128, S_pad], plus ``kept`` (uint8 [B, H, S], 1 at the repaired
+    permuted positions)."""
+    lib = load()
+    sh = shape_of(v)
+    cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_E4M3, _MODES[mode])
+    B, S, H = sh.B, sh.S, sh.H
+    nb = num_blocks(S)
+    dev = v.device
+    out = dict(perm=torch.empty((B, H, S), dtype=torch.int32, device=dev),
+               mu=torch.empty((B, H, nb, 128), dtype=torch.float32, device=dev),
+               s_v=torch.empty((B, H), dtype=torch.float32, device=dev),
+               v_codes=torch.empty((2, B, H, 128, nb * 128), dtype=torch.uint8, device=dev), v_scales=None,
+               kept=torch.empty((B, H, S), dtype=torch.uint8, device=dev), fmt="repair")
+    wsb = lib.vc_attn_prepare_v_repair_workspace_bytes(ctypes.byref(sh), ctypes.byref(cfg))
+    if wsb == 0:
+        raise VCError(VC_ERR_INVALID_ARG, "invalid shape or config")
+    ws = torch.empty(wsb + 256, dtype=torch.uint8, device=dev)
+    off = (-ws.data_ptr()) % 256
+    pv = PreparedV(_ptr(out["perm"]), _ptr(out["mu"]), _ptr(out["v_codes"]), None, _ptr(out["s_v"]))
+    _check(lib.vc_attn_prepare_v_repair(_ptr(v), ctypes.byref(sh), ctypes.byref(cfg), float(budget),
+                                        ctypes.byref(pv), _ptr(out["kept"]), ctypes.c_void_p(ws.data_ptr() + off),
+                                        wsb, _stream()))
+    out["workspace"] = ws
+    return out
+
+
+def forward_repair(qk, pv, shape, softmax_scale=None, k_p=8, out=None, status=None):
+    """Attention over the two planes of ``prepare_v_repair``; BF16 O in the input
+    layout."""
+    lib = load()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(128)
+    dev = qk["q_codes"].device
+    if out is None:
+        out = torch.empty((shape.B, shape.S, shape.H, 128), dtype=torch.bfloat16, device=dev)
+    q_ = QKFP8(_ptr(qk["q_codes"]), _ptr(qk["q_scales"]), _ptr(qk["k_codes"]), _ptr(qk["k_scales"]))
+    p_ = PreparedV(_ptr(pv["perm"]), _ptr(pv["mu"]), _ptr(pv["v_codes"]), None, _ptr(pv["s_v"]))
+    _check(lib.vc_attn_forward_repair(ctypes.byref(q_), ctypes.byref(p_), ctypes.byref(shape), float(softmax_scale),
+                                      int(k_p), _ptr(out), _ptr(status), _stream()))
     return out
 
 

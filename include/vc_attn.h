@@ -152,6 +152,45 @@ vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_v
 vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* shape,
                              const int32_t* perm, const vc_qk_fp8_t* out, void* stream);
 
+/* Bytes of workspace vc_attn_prepare_v_repair needs for this shape and config
+ * (0 if the arguments are invalid): that of vc_attn_prepare_v plus 4*B*H*S +
+ * 8*B*H bytes (each part rounded up to 256). */
+size_t vc_attn_prepare_v_repair_workspace_bytes(const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg);
+
+/* V-Smooth prep with the V residual repair ("Open VC Attention", "Описание":
+ * the repair re-adds the quantisation residual of the worst-rounded value
+ * tokens, prepared with a budget such as 0.005), for the E4M3 residual. The
+ * result is two E4M3 planes at the residual's scale s_V:
+ *   plane 0 = the residual codes of vc_attn_prepare_v;
+ *   plane 1 = for the m = min(S, ceil(budget * S)) kept tokens of each (b, h),
+ *             E4M3 codes of each element's rounding error in code units,
+ *             y - dec(code0) with y = fl32(fl32(v - mu) * fl32(448 / amax)) (the
+ *             value that was rounded); 0 for the other and the padding tokens.
+ * The kept tokens are the m largest by the error sum_d fl32(dlt_d^2), added in
+ * fp32 from d = 0 to 127, ties to the lower permuted position.
+ *  budget        share of the tokens of each (b, h) to repair, in [0, 1]
+ *  out           as vc_attn_prepare_v, except that out->v_codes points to
+ *                uint8 [2][B,H,128,S_pad] (plane 0, then plane 1)
+ *  kept          optional device uint8 [B,H,S]: 1 for the kept permuted
+ *                positions, else 0; NULL to skip
+ *  workspace     device, >= vc_attn_prepare_v_repair_workspace_bytes(),
+ *                256-B aligned
+ * The planes feed vc_attn_forward_repair. Errors: as vc_attn_prepare_v, plus
+ * VC_ERR_UNSUPPORTED for the NVFP4 residual and VC_ERR_INVALID_ARG for a budget
+ * outside [0, 1]. */
+vc_status_t vc_attn_prepare_v_repair(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                                     double budget, const vc_prepared_v_t* out, uint8_t* kept,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Attention over a repaired residual: as vc_attn_forward, with pv from
+ * vc_attn_prepare_v_repair (pv->v_codes = the two planes). O = (s_V * P (plane 0
+ * + plane 1) + sum_tiles rowsum(P_tile) mu_tile) / rowsum(P); the row sums come
+ * from P alone, so the repaired tokens are counted once. Errors: as
+ * vc_attn_forward. */
+vc_status_t vc_attn_forward_repair(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
+                                   float softmax_scale, int32_t k_p, void* o, int32_t* dev_status,
+                                   void* stream);
+
 /* Bytes of device workspace vc_attn_quant_qk_smoothk needs: B*H*128*8 (0 for an
  * invalid shape). */
 size_t vc_attn_quant_qk_smoothk_workspace_bytes(const vc_shape_t* shape);

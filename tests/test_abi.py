@@ -196,3 +196,27 @@ def test_too_many_slices_is_refused_before_any_launch(lib):
     assert b"65535" in lib.vc_attn_last_error()
     ok = _shape(B=1, S=100, H=65535)
     assert lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(ok)) == 65535 * 128 * 8
+
+
+def test_prepare_v_repair_workspace_and_validation(lib):
+    sh, cfg = _shape(S=1000, H=5), _cfg(k=16, iters=4)
+    base = lib.vc_attn_prepare_v_workspace_bytes(ctypes.byref(sh), ctypes.byref(cfg))
+    need = lib.vc_attn_prepare_v_repair_workspace_bytes(ctypes.byref(sh), ctypes.byref(cfg))
+    assert need >= base + 5 * 1000 * 4 + 5 * 8 and need % 256 == 0
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    pv = vc_attn.PreparedV(p, p, p, None, p)
+    for args, code in (
+        ((p, ctypes.byref(sh), ctypes.byref(_cfg(k=16, iters=4, fmt=1)), 0.005, ctypes.byref(pv), None, p, need, None),
+         vc_attn.VC_ERR_UNSUPPORTED),
+        ((p, ctypes.byref(sh), ctypes.byref(cfg), -0.1, ctypes.byref(pv), None, p, need, None),
+         vc_attn.VC_ERR_INVALID_ARG),
+        ((p, ctypes.byref(sh), ctypes.byref(cfg), float("nan"), ctypes.byref(pv), None, p, need, None),
+         vc_attn.VC_ERR_INVALID_ARG),
+        ((p, ctypes.byref(sh), ctypes.byref(cfg), 0.005, ctypes.byref(pv), None, p, need - 1, None),
+         vc_attn.VC_ERR_WORKSPACE),
+        ((p, ctypes.byref(sh), ctypes.byref(cfg), 0.005, ctypes.byref(pv), None, None, need, None),
+         vc_attn.VC_ERR_WORKSPACE),
+    ):
+        assert lib.vc_attn_prepare_v_repair(*args) == code
+        assert lib.vc_attn_last_error() != b""
