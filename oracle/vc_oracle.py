@@ -54,10 +54,19 @@ Readings taken where the pages are silent (R-numbers are used in comments):
       uses); O = (sum_j P_ij v~_j + sum_b r_ib mu_b) / l_i, then BF16 RNE.
   R10 A block (or head) whose amax is below 2^-100 is treated as all zero:
       scale 1, codes 0.
-  R14 Optional per-channel residual scale (SURVEY's next-4, an accuracy knob
-      beside [OVC]'s per-head V scale): s_V[d] = amax_d / 448 over the slice's
-      residual in channel d, codes E4M3(r * fl32(448 / amax_d)); a channel with
-      amax_d below 2^-100 gets scale 1 and codes 0 (R10).
+  R11 Optional K smoothing ([ABS]: prior work smooths queries and keys; the
+      pages give no form): K minus its per-channel mean over all tokens of the
+      (b, h) slice, the mean an int64 fixed-point sum as in R4, the difference
+      taken in fp32, before the per-block quantisation of R7. Every score of a
+      query row moves by the same q.kbar, so the softmax is unchanged. Q is not
+      smoothed (its mean would shift each key's score differently).
+  R12 Optional V residual repair ([OVC]: re-adds the quantisation residual of
+      the worst-rounded value tokens, with a budget such as 0.005): for an E4M3
+      residual, the ceil(budget * S) tokens of the slice whose decoded value
+      s_V dec(code) is farthest from the residual r it codes (squared L2 over
+      the channels, fp64; ties to the lower permuted position) get their error
+      r - s_V dec(code) back, stored in fp32. The probabilities are untouched:
+      only those tokens' values in the P V product change.
   R13 MX-style FP4 residual (not described by the pages; the block-scaled FP4
       operand form of the B200 tensor cores, a neighbour of the NVFP4 residual):
       E2M1 codes with one power-of-two scale per 32 consecutive permuted tokens
@@ -66,19 +75,10 @@ Readings taken where the pages are silent (R-numbers are used in comments):
       can clip a group's largest values by up to a quarter), e clamped to
       [-127, 127] (an 8-bit biased exponent), codes E2M1(r / X) with RNE; an
       all-zero group has e = -127 and codes 0. No per-head scale.
-  R12 Optional V residual repair ([OVC]: re-adds the quantisation residual of
-      the worst-rounded value tokens, with a budget such as 0.005): for an E4M3
-      residual, the ceil(budget * S) tokens of the slice whose decoded value
-      s_V dec(code) is farthest from the residual r it codes (squared L2 over
-      the channels, fp64; ties to the lower permuted position) get their error
-      r - s_V dec(code) back, stored in fp32. The probabilities are untouched:
-      only those tokens' values in the P V product change.
-  R11 Optional K smoothing ([ABS]: prior work smooths queries and keys; the
-      pages give no form): K minus its per-channel mean over all tokens of the
-      (b, h) slice, the mean an int64 fixed-point sum as in R4, the difference
-      taken in fp32, before the per-block quantisation of R7. Every score of a
-      query row moves by the same q.kbar, so the softmax is unchanged. Q is not
-      smoothed (its mean would shift each key's score differently).
+  R14 Optional per-channel residual scale (an accuracy knob beside [OVC]'s
+      per-head V scale): s_V[d] = amax_d / 448 over the slice's
+      residual in channel d, codes E4M3(r * fl32(448 / amax_d)); a channel with
+      amax_d below 2^-100 gets scale 1 and codes 0 (R10).
 """
 import math
 
