@@ -220,3 +220,29 @@ def test_prepare_v_repair_workspace_and_validation(lib):
     ):
         assert lib.vc_attn_prepare_v_repair(*args) == code
         assert lib.vc_attn_last_error() != b""
+
+
+def test_no_fallback_without_the_library_or_a_gpu(monkeypatch):
+    # the binding raises when libvcattn.so is missing ...
+    monkeypatch.setattr(vc_attn, "_lib", None)
+    monkeypatch.setattr(vc_attn, "LIB_PATH", "/nonexistent/libvcattn.so")
+    with pytest.raises(RuntimeError, match="missing"):
+        vc_attn.load()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the behaviour on a host without a GPU")
+def test_product_path_raises_on_a_host_without_gpu():
+    # ... and on a machine without a GPU the whole path raises (torch's stream
+    # lookup or the library's device check, both RuntimeError) instead of computing
+    q = torch.zeros(1, 256, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError):
+        vc_attn.attention(q, q, q)
+
+
+def test_package_never_imports_the_oracle():
+    pkg = os.path.dirname(vc_attn.__file__)
+    for root, _, files in os.walk(pkg):
+        for name in files:
+            if name.endswith(".py"):
+                src = open(os.path.join(root, name)).read()
+                assert not re.search(r"^\s*(import oracle|from oracle)", src, re.M), name
