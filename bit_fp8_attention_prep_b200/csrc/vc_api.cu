@@ -187,11 +187,9 @@ size_t vc_attn_prepare_v_workspace_bytes(const vc_shape_t* shape, const vc_vsmoo
 
 }  // extern "C"
 
-// vc_attn_prepare_v with the slices numbered from bh_base (the k-means seed of
-// slice i of this call is that of slice bh_base + i of the caller's problem).
-static vc_status_t prepare_v_impl(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
-                                  const vc_prepared_v_t* out, void* workspace, size_t workspace_bytes,
-                                  uint8_t* assign_history, void* stream, int bh_base) {
+// Shape, config and output-pointer checks shared by the prep entry points.
+static vc_status_t check_prep_args(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                                   const vc_prepared_v_t* out) {
   vc_status_t st;
   if ((st = check_shape(shape)) != VC_OK) return st;
   if ((st = check_cfg(cfg)) != VC_OK) return st;
@@ -202,6 +200,16 @@ static vc_status_t prepare_v_impl(const void* v, const vc_shape_t* shape, const 
   if (!aligned16(v) || !aligned16(out->perm) || !aligned16(out->mu) || !aligned16(out->v_codes) ||
       !aligned16(out->s_v) || (out->v_scales && !aligned16(out->v_scales)))
     return fail(VC_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  return VC_OK;
+}
+
+// vc_attn_prepare_v with the slices numbered from bh_base (the k-means seed of
+// slice i of this call is that of slice bh_base + i of the caller's problem).
+static vc_status_t prepare_v_impl(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                                  const vc_prepared_v_t* out, void* workspace, size_t workspace_bytes,
+                                  uint8_t* assign_history, void* stream, int bh_base) {
+  vc_status_t st;
+  if ((st = check_prep_args(v, shape, cfg, out)) != VC_OK) return st;
   const WsLayout w = ws_layout(shape, cfg);
   if (!workspace || workspace_bytes < w.total)
     return fail(VC_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total,
@@ -478,14 +486,16 @@ vc_status_t vc_attn_prepare_v_noalloc(const void* v, const vc_shape_t* shape, co
   NvtxRange range("vc_attn_prepare_v_noalloc");
   g_last_error.clear();
   vc_status_t st;
-  if ((st = check_shape(shape)) != VC_OK) return st;
-  if ((st = check_cfg(cfg)) != VC_OK) return st;
+  // the same checks, in the same order, as vc_attn_prepare_v, before anything
+  // touches the device: arguments, the scratch size, then the device itself
+  if ((st = check_prep_args(v, shape, cfg, out)) != VC_OK) return st;
   const size_t need = ws_layout(shape, cfg).total;
   if (need > VC_ATTN_NOALLOC_SCRATCH_BYTES)
     return fail(VC_ERR_WORKSPACE,
                 "this problem needs %zu bytes of prep scratch; the fixed scratch of vc_attn_prepare_v_noalloc "
                 "holds %zu bytes (use vc_attn_prepare_v with a caller workspace)",
                 need, (size_t)VC_ATTN_NOALLOC_SCRATCH_BYTES);
+  if ((st = ensure_device()) != VC_OK) return st;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");

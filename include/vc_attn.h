@@ -302,6 +302,9 @@ vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t*
  *    contents (each call clears what must start at zero). Calls whose work
  *    overlaps on the GPU (on different streams, or from different threads
  *    without ordering) race on it: serialise them on one stream.
+ *  - The looked-up address is kept for the life of the process: calling
+ *    cudaDeviceReset on a device after its first call here is not supported
+ *    (the array would move, and the kept address would no longer be it).
  * Arguments, outputs and other errors are those of vc_attn_prepare_v. */
 vc_status_t vc_attn_prepare_v_noalloc(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
                                       const vc_prepared_v_t* out, uint8_t* assign_history, void* stream);

@@ -246,3 +246,28 @@ def test_package_never_imports_the_oracle():
             if name.endswith(".py"):
                 src = open(os.path.join(root, name)).read()
                 assert not re.search(r"^\s*(import oracle|from oracle)", src, re.M), name
+
+
+def test_noalloc_prep_checks_arguments_before_the_device(lib):
+    # vc_attn_prepare_v_noalloc answers a bad argument exactly as vc_attn_prepare_v
+    # does, before it looks at the device or its fixed scratch: on this host there
+    # is no GPU, so any device step would give VC_ERR_CUDA or VC_ERR_UNSUPPORTED.
+    pv = vc_attn.PreparedV(16, 16, 16, 16, 16)
+    st = lib.vc_attn_prepare_v_noalloc(ctypes.c_void_p(16), ctypes.byref(_shape(D=64)), ctypes.byref(_cfg()),
+                                       ctypes.byref(pv), None, None)
+    assert st == vc_attn.VC_ERR_INVALID_ARG and b"D must be 128" in lib.vc_attn_last_error()
+    st = lib.vc_attn_prepare_v_noalloc(None, ctypes.byref(_shape()), ctypes.byref(_cfg()), ctypes.byref(pv),
+                                       None, None)
+    assert st == vc_attn.VC_ERR_INVALID_ARG and b"non-NULL" in lib.vc_attn_last_error()
+    st = lib.vc_attn_prepare_v_noalloc(ctypes.c_void_p(18), ctypes.byref(_shape()), ctypes.byref(_cfg()),
+                                       ctypes.byref(pv), None, None)
+    assert st == vc_attn.VC_ERR_INVALID_ARG and b"aligned" in lib.vc_attn_last_error()
+    pv_nv = vc_attn.PreparedV(16, 16, 16, 0, 16)   # NVFP4 without v_scales
+    st = lib.vc_attn_prepare_v_noalloc(ctypes.c_void_p(16), ctypes.byref(_shape()),
+                                       ctypes.byref(_cfg(fmt=vc_attn.VC_RESIDUAL_NVFP4)), ctypes.byref(pv_nv),
+                                       None, None)
+    assert st == vc_attn.VC_ERR_INVALID_ARG and b"v_scales" in lib.vc_attn_last_error()
+    # valid arguments: only now does the call reach the device, which this host lacks
+    st = lib.vc_attn_prepare_v_noalloc(ctypes.c_void_p(16), ctypes.byref(_shape()), ctypes.byref(_cfg()),
+                                       ctypes.byref(pv), None, None)
+    assert st in (vc_attn.VC_ERR_CUDA, vc_attn.VC_ERR_UNSUPPORTED)

@@ -1,8 +1,6 @@
 """GPU: the V residual repair. The two planes and the kept positions are
 bit-exact with the oracle's two-plane repair; O over the two planes is within the
-parity bars of the oracle's VC-Attention on the repaired values.
-
-Skipped until the repair kernels have had their first run on a B200."""
+parity bars of the oracle's VC-Attention on the repaired values."""
 import numpy as np
 import pytest
 import torch
@@ -10,7 +8,7 @@ import torch
 import oracle as O
 from parity_helpers import SCALE, assert_o_close, head, make
 
-pytestmark = [pytest.mark.gpu, pytest.mark.skip(reason="the repair kernels have not yet run on a GPU")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")

@@ -32,7 +32,15 @@ def _same(a, b):
         assert np.array_equal(x.view(np.uint8), y.view(np.uint8)), key
 
 
+def _same_nvfp4(a, b):
+    for key in ("perm", "mu", "v_codes", "v_scales", "s_v"):
+        x, y = a[key].cpu().numpy(), b[key].cpu().numpy()
+        assert np.array_equal(x.view(np.uint8), y.view(np.uint8)), key
+
+
 def test_noalloc_prep_matches_workspace_prep_on_two_calls(va):
+    # the mid case fills most of the scratch; the tiny case after it must not see
+    # its leftovers (the k-means sums, counts and histograms start at zero)
     cases = [("mid", dict(B=2, H=3, S=2500), 16, 4), ("tiny", {}, 4, 3)]
     for name, kw, k, iters in cases:
         cfg, Q, K, V = make(name, **kw)
@@ -47,6 +55,24 @@ def test_noalloc_prep_matches_workspace_prep_on_two_calls(va):
         o_got = va.forward(va.quant_qk(q, kk, got["perm"]), got, shape, SCALE)
         torch.cuda.synchronize()
         assert torch.equal(o_ref, o_got)
+
+
+def test_noalloc_prep_other_residuals_and_modes(va):
+    # the NVFP4 residual and the MEANONLY / NAIVE modes lay the scratch out
+    # differently (one cluster, no second label buffer); each runs right after a
+    # mid-size VSMOOTH call has left its contents in the array
+    cfg, Q, K, V = make("mid", B=1, H=4, S=3000)
+    v = V.cuda()
+    for fmt, mode in (("nvfp4", "vsmooth"), ("e4m3", "meanonly"), ("e4m3", "naive"), ("nvfp4", "meanonly")):
+        va.prepare_v_noalloc(v, k=16, iters=4)            # leaves VSMOOTH scratch behind
+        ref = va.prepare_v(v, k=16, iters=4, fmt=fmt, mode=mode)
+        got = va.prepare_v_noalloc(v, k=16, iters=4, fmt=fmt, mode=mode)
+        torch.cuda.synchronize()
+        if fmt == "nvfp4":
+            _same_nvfp4(got, ref)
+        else:
+            for key in ("perm", "mu", "v_codes", "s_v"):
+                assert np.array_equal(got[key].cpu().numpy().view(np.uint8), ref[key].cpu().numpy().view(np.uint8)), (fmt, mode, key)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(va):
