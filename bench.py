@@ -559,9 +559,9 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
 
 
 def run_sweep(args):
-    """NVFP4-V vs E4M3-V over S (the NVFP4 sweep workloads: B=1, H=24): forward
-    FP8 TFLOP/s of each and rel-L2 against exact fp64 attention on sampled rows
-    of two heads. One JSON line per S (not the benchmark line)."""
+    """E4M3-V, NVFP4-V and MX-style FP4 V over S (the NVFP4 sweep workloads: B=1,
+    H=24): forward FP8 TFLOP/s of each and rel-L2 against exact fp64 attention on
+    sampled rows of two heads. One JSON line per S (not the benchmark line)."""
     import torch
     from bit_fp8_attention_prep_b200 import synth, vc_attn
     dev = torch.device("cuda", 0)
@@ -577,8 +577,8 @@ def run_sweep(args):
             k, v = K[0, :, h].double(), V[0, :, h].double()
             refs[h] = torch.softmax((q @ k.t()) / math.sqrt(128), dim=-1) @ v
             del k, v
-        line = {"sweep": "nvfp4_vs_e4m3", "S": S, "B": B, "H": H, "k_p": args.k_p}
-        for fmt in ("e4m3", "nvfp4"):
+        line = {"sweep": "v_residual_formats", "S": S, "B": B, "H": H, "k_p": args.k_p}
+        for fmt in ("e4m3", "nvfp4", "mxfp4"):
             plan = vc_attn.Plan(B, S, H, k=cfg["k"], iters=cfg["iters"], fmt=fmt, k_p=args.k_p, device=dev)
             plan.run(Q, K, V)
             for _ in range(2):

@@ -78,8 +78,11 @@ vc_status_t check_cfg(const vc_vsmooth_cfg_t* cfg) {
       return fail(VC_ERR_INVALID_ARG, "k must be in [1, %d] (got %d)", vc::kMaxClusters, cfg->k);
     if (cfg->iters < 1 || cfg->iters > 64) return fail(VC_ERR_INVALID_ARG, "iters must be in [1, 64] (got %d)", cfg->iters);
   }
-  if (cfg->residual_fmt != VC_RESIDUAL_E4M3 && cfg->residual_fmt != VC_RESIDUAL_NVFP4)
-    return fail(VC_ERR_INVALID_ARG, "residual_fmt must be VC_RESIDUAL_E4M3 or VC_RESIDUAL_NVFP4");
+  if (cfg->residual_fmt != VC_RESIDUAL_E4M3 && cfg->residual_fmt != VC_RESIDUAL_NVFP4 &&
+      cfg->residual_fmt != VC_RESIDUAL_E4M3_PER_CHANNEL && cfg->residual_fmt != VC_RESIDUAL_MXFP4)
+    return fail(VC_ERR_INVALID_ARG,
+                "residual_fmt must be VC_RESIDUAL_E4M3, _NVFP4, _E4M3_PER_CHANNEL or _MXFP4 (got %d)",
+                cfg->residual_fmt);
   return VC_OK;
 }
 
@@ -103,7 +106,8 @@ WsLayout ws_layout(const vc_shape_t* sh, const vc_vsmooth_cfg_t* cfg) {
   w.assign2 = off; off += cfg->mode == VC_MODE_VSMOOTH ? align256(BH * (size_t)sh->S) : 0;
   w.hist = off;   off += align256(BH * nch * k * 4);
   w.offs = off;   off += align256(BH * nch * k * 4);
-  w.amax = off;   off += align256(BH * 4);
+  // residual amax: one per (b, h), or one per (b, h, channel)
+  w.amax = off;   off += align256(BH * 4 * (cfg->residual_fmt == VC_RESIDUAL_E4M3_PER_CHANNEL ? 128 : 1));
   w.total = off;
   return w;
 }
@@ -195,8 +199,8 @@ static vc_status_t check_prep_args(const void* v, const vc_shape_t* shape, const
   if ((st = check_cfg(cfg)) != VC_OK) return st;
   if (!v || !out || !out->perm || !out->mu || !out->v_codes || !out->s_v)
     return fail(VC_ERR_INVALID_ARG, "v, out, out->perm, out->mu, out->v_codes and out->s_v must be non-NULL");
-  if (cfg->residual_fmt == VC_RESIDUAL_NVFP4 && !out->v_scales)
-    return fail(VC_ERR_INVALID_ARG, "out->v_scales must be non-NULL for the NVFP4 residual");
+  if ((cfg->residual_fmt == VC_RESIDUAL_NVFP4 || cfg->residual_fmt == VC_RESIDUAL_MXFP4) && !out->v_scales)
+    return fail(VC_ERR_INVALID_ARG, "out->v_scales must be non-NULL for the NVFP4 and MXFP4 residuals");
   if (!aligned16(v) || !aligned16(out->perm) || !aligned16(out->mu) || !aligned16(out->v_codes) ||
       !aligned16(out->s_v) || (out->v_scales && !aligned16(out->v_scales)))
     return fail(VC_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
@@ -363,22 +367,49 @@ vc_status_t vc_attn_residual_energy(const void* v, const vc_shape_t* shape, cons
   return VC_OK;
 }
 
-// nvfp4: split pv's NVFP4 residual into two E4M3 planes in `workspace`, then the
-// two-plane kernel at value scale 8 g; two_planes: pv->v_codes already holds two
-// E4M3 planes at the residual's scale (the repaired residual); otherwise the
-// one-plane E4M3 kernel.
+// 2D tensor map over packed E2M1 codes (two per byte): rows of `inner` codes,
+// `rows` rows, 128 x 128 code box, each 16 codes widened by the TMA into a
+// 16-byte shared-memory container (the 8-bit operand footprint of
+// kind::mxf8f6f4), 128-byte swizzle. The base must be 32-byte aligned and
+// inner a multiple of 128.
+static vc_status_t make_map_e2m1(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(VC_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner / 2};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(VC_ERR_CUDA, "cuTensorMapEncodeTiled (E2M1) failed (%d)", (int)r);
+  return VC_OK;
+}
+
+// Which attention kernel a forward call runs.
+enum class FwdKind {
+  E4M3,         // one E4M3 plane, s_V per (b, h)
+  E4M3_EXP2,    // the same with ex2 + E4M3 conversion in place of ExpCast (test hook)
+  E4M3_CHANNEL, // one E4M3 plane, s_V per (b, h, channel)
+  NVFP4,        // pv's NVFP4 residual split into two E4M3 planes in `workspace`, value scale 8 g
+  TWO_PLANES,   // pv->v_codes already holds two E4M3 planes at s_V (the repaired residual)
+  MXFP4         // E2M1 codes with power-of-two scales, block-scaled PV
+};
+
 static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                                   float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream,
-                                  bool nvfp4, void* workspace, size_t workspace_bytes, bool exp2 = false,
-                                  bool two_planes = false) {
+                                  FwdKind kind, void* workspace = nullptr, size_t workspace_bytes = 0) {
+  const bool nvfp4 = kind == FwdKind::NVFP4;
   g_last_error.clear();
   vc_status_t st;
   if ((st = check_shape(shape)) != VC_OK) return st;
   if (!qk || !pv || !o) return fail(VC_ERR_INVALID_ARG, "qk, pv and o must be non-NULL");
   if (!qk->q_codes || !qk->q_scales || !qk->k_codes || !qk->k_scales || !pv->mu || !pv->v_codes || !pv->s_v)
     return fail(VC_ERR_INVALID_ARG, "a required field of qk or pv is NULL");
-  if (nvfp4 && (!pv->v_scales || !aligned16(pv->v_scales)))
-    return fail(VC_ERR_INVALID_ARG, "pv->v_scales must be non-NULL and 16-byte aligned for NVFP4");
+  if ((nvfp4 || kind == FwdKind::MXFP4) && (!pv->v_scales || !aligned16(pv->v_scales)))
+    return fail(VC_ERR_INVALID_ARG, "pv->v_scales must be non-NULL and 16-byte aligned for NVFP4 and MXFP4");
+  if (kind == FwdKind::MXFP4 && (reinterpret_cast<uintptr_t>(pv->v_codes) & 31u) != 0)
+    return fail(VC_ERR_INVALID_ARG, "pv->v_codes must be 32-byte aligned for the MXFP4 residual");
   if (!aligned16(o) || !aligned16(qk->q_codes) || !aligned16(qk->k_codes) || !aligned16(pv->v_codes) ||
       !aligned16(pv->mu) || (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)))
     return fail(VC_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
@@ -415,12 +446,19 @@ static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* 
   p.status = dev_status;
   p.wait_ns = 2000000000ull;
   cudaError_t e;
-  if (two_planes) {
+  const cudaStream_t cst = static_cast<cudaStream_t>(stream);
+  if (kind == FwdKind::TWO_PLANES) {
     if ((st = make_map_u8(&tv, pv->v_codes, (uint64_t)S_pad, (uint64_t)2 * BH * 128)) != VC_OK) return st;
-    e = vc::launch_attn_planes(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
-  } else if (!nvfp4) {
+    e = vc::launch_attn_planes(tq, tk, tv, p, cst);
+  } else if (kind == FwdKind::E4M3 || kind == FwdKind::E4M3_EXP2) {
     if ((st = make_map_u8(&tv, pv->v_codes, (uint64_t)S_pad, (uint64_t)BH * 128)) != VC_OK) return st;
-    e = vc::launch_attn_e4m3(tq, tk, tv, p, static_cast<cudaStream_t>(stream), exp2);
+    e = vc::launch_attn_e4m3(tq, tk, tv, p, cst, kind == FwdKind::E4M3_EXP2);
+  } else if (kind == FwdKind::E4M3_CHANNEL) {
+    if ((st = make_map_u8(&tv, pv->v_codes, (uint64_t)S_pad, (uint64_t)BH * 128)) != VC_OK) return st;
+    e = vc::launch_attn_channel(tq, tk, tv, p, cst);
+  } else if (kind == FwdKind::MXFP4) {
+    if ((st = make_map_e2m1(&tv, pv->v_codes, (uint64_t)S_pad, (uint64_t)BH * 128)) != VC_OK) return st;
+    e = vc::launch_attn_mx(tq, tk, tv, p, cst);
   } else {
     uint8_t* planes = static_cast<uint8_t*>(workspace);
     e = vc::launch_nvfp4_planes(static_cast<const uint8_t*>(pv->v_codes), static_cast<const uint8_t*>(pv->v_scales),
@@ -438,18 +476,31 @@ static vc_status_t forward_common(const vc_qk_fp8_t* qk, const vc_prepared_v_t* 
 vc_status_t vc_attn_forward(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                             float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
   NvtxRange range("vc_attn_forward");
-  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, false, nullptr, 0);
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, FwdKind::E4M3);
+}
+
+vc_status_t vc_attn_forward_e4m3_per_channel(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv,
+                                             const vc_shape_t* shape, float softmax_scale, int32_t k_p, void* o,
+                                             int32_t* dev_status, void* stream) {
+  NvtxRange range("vc_attn_forward_e4m3_per_channel");
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, FwdKind::E4M3_CHANNEL);
+}
+
+vc_status_t vc_attn_forward_mxfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
+                                   float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
+  NvtxRange range("vc_attn_forward_mxfp4v");
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, FwdKind::MXFP4);
 }
 
 vc_status_t vc_attn_test_forward_exp2(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                                       float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
-  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, false, nullptr, 0, true);
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, FwdKind::E4M3_EXP2);
 }
 
 vc_status_t vc_attn_forward_repair(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
                                    float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream) {
   NvtxRange range("vc_attn_forward_repair");
-  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, false, nullptr, 0, false, true);
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, FwdKind::TWO_PLANES);
 }
 
 size_t vc_attn_forward_nvfp4v_workspace_bytes(const vc_shape_t* shape) {
@@ -461,7 +512,7 @@ vc_status_t vc_attn_forward_nvfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t*
                                    float softmax_scale, int32_t k_p, void* o, void* workspace,
                                    size_t workspace_bytes, int32_t* dev_status, void* stream) {
   NvtxRange range("vc_attn_forward_nvfp4v");
-  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, true, workspace,
+  return forward_common(qk, pv, shape, softmax_scale, k_p, o, dev_status, stream, FwdKind::NVFP4, workspace,
                         workspace_bytes);
 }
 
@@ -534,7 +585,8 @@ struct RunHostLayout {
 RunHostLayout run_host_layout(const vc_shape_t* sh, const vc_vsmooth_cfg_t* cfg, int hc) {
   const size_t S = (size_t)sh->S, nb = (size_t)nblocks(sh->S), S_pad = nb * 128, n = (size_t)hc;
   const size_t chunk_bytes = S * n * 128 * 2;
-  const bool nv = cfg->residual_fmt == VC_RESIDUAL_NVFP4;
+  const int fmt = cfg->residual_fmt;
+  const bool nv = fmt == VC_RESIDUAL_NVFP4, mx = fmt == VC_RESIDUAL_MXFP4, ch = fmt == VC_RESIDUAL_E4M3_PER_CHANNEL;
   vc_shape_t cs = *sh;
   cs.B = 1;
   cs.H = hc;
@@ -553,9 +605,9 @@ RunHostLayout run_host_layout(const vc_shape_t* sh, const vc_vsmooth_cfg_t* cfg,
   for (int slot = 0; slot < 2; ++slot) {
     L.perm[slot] = off;     off += align256(n * S * 4);
     L.mu[slot] = off;       off += align256(n * nb * 128 * 4);
-    L.v_codes[slot] = off;  off += align256(n * 128 * (nv ? S_pad / 2 : S_pad));
-    L.v_scales[slot] = off; off += nv ? align256(n * 128 * (S_pad / 16)) : 0;
-    L.s_v[slot] = off;      off += align256(n * 4);
+    L.v_codes[slot] = off;  off += align256(n * 128 * (nv || mx ? S_pad / 2 : S_pad));
+    L.v_scales[slot] = off; off += nv ? align256(n * 128 * (S_pad / 16)) : mx ? align256(n * nb * 128 * 4) : 0;
+    L.s_v[slot] = off;      off += align256(n * 4 * (ch ? 128 : 1));
     L.q_codes[slot] = off;  off += align256(n * S_pad * 128);
     L.q_scales[slot] = off; off += align256(n * nb * 4);
     L.k_codes[slot] = off;  off += align256(n * S_pad * 128);
@@ -653,7 +705,11 @@ vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const 
   if ((e = ev.create()) != cudaSuccess) return cuda_fail(e, "creating events");
   const cudaStream_t cs_stream = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const bool nv = cfg->residual_fmt == VC_RESIDUAL_NVFP4;
+  const bool nv = cfg->residual_fmt == VC_RESIDUAL_NVFP4, mx = cfg->residual_fmt == VC_RESIDUAL_MXFP4;
+  const FwdKind kind = nv ? FwdKind::NVFP4
+                          : mx ? FwdKind::MXFP4
+                               : cfg->residual_fmt == VC_RESIDUAL_E4M3_PER_CHANNEL ? FwdKind::E4M3_CHANNEL
+                                                                                   : FwdKind::E4M3;
   const size_t row_bytes = (size_t)H * 256;  // one token of all heads
   const char* hq[3] = {static_cast<const char*>(q), static_cast<const char*>(k), static_cast<const char*>(v)};
   char* ho = static_cast<char*>(o);
@@ -703,7 +759,7 @@ vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const 
       pv.perm = reinterpret_cast<int32_t*>(ws + L.perm[slot]);
       pv.mu = reinterpret_cast<float*>(ws + L.mu[slot]);
       pv.v_codes = ws + L.v_codes[slot];
-      pv.v_scales = nv ? ws + L.v_scales[slot] : nullptr;
+      pv.v_scales = nv || mx ? ws + L.v_scales[slot] : nullptr;
       pv.s_v = reinterpret_cast<float*>(ws + L.s_v[slot]);
       vc_qk_fp8_t qk;
       qk.q_codes = ws + L.q_codes[slot];
@@ -715,7 +771,7 @@ vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const 
         return st;
       if ((st = vc_attn_quant_qk(ws + L.in[slot][0], ws + L.in[slot][1], &cs, pv.perm, &qk, cst)) != VC_OK)
         return st;
-      if ((st = forward_common(&qk, &pv, &cs, softmax_scale, k_p, ws + L.out[slot], dev_status, cst, nv,
+      if ((st = forward_common(&qk, &pv, &cs, softmax_scale, k_p, ws + L.out[slot], dev_status, cst, kind,
                                nv ? ws + L.planes[slot] : nullptr, L.planes_bytes)) != VC_OK)
         return st;
       if ((e = cudaEventRecord(ev.comp[slot], cst)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");

@@ -46,7 +46,14 @@
 //        no MMA of their tile is in flight; M (shared by both tiles) in a
 //        double-buffered unswizzled tile written by the TMA warp
 // so O_t accumulates the whole output in residual-code units; the epilogue is
-// O = s_V O_t / l. The softmax thread of row i keeps the integer running frame
+// O = s_V O_t / l (s_V per output channel for the per-channel residual scale).
+// The MX-style FP4 residual (kVKind = kVMx) runs PV as the block-scaled
+// kind::mxf8f6f4 product: V^T arrives as E2M1 codes (TMA widens each 16 packed
+// codes into a 16-byte smem container), its power-of-two scale per channel and
+// 32 tokens as UE8M0 bytes that the softmax threads of each tile copy into
+// tensor memory (SFB_t) next to P_t, the probabilities' scale is a constant 2^0
+// (SFA_t); the two score tiles then share all 128 of their columns, which frees
+// the 32 columns the scale factors need. The softmax thread of row i keeps the integer running frame
 // F (ceil of the largest log2-domain score so far); a block is cast in the frame
 // current after it; when F moves, O_t (with its row-sum column) and the row sums
 // not yet handed to a mean MMA (held in registers until their batch of 5 blocks
@@ -65,6 +72,10 @@ namespace {
 
 // kPlanes = 1: the E4M3 residual; kPlanes = 2: the NVFP4 residual given as two
 // exact E4M3 planes (hi + lo) by the pre-pass in vc_prep.cu, with PV run over both.
+// kVKind: how the residual codes are scaled back to values.
+constexpr int kVHead = 0;     // one scale s_V per (b, h)
+constexpr int kVChannel = 1;  // one scale per (b, h, channel): applied per output channel
+constexpr int kVMx = 2;       // MX-style FP4: a power of two per channel and 32 tokens, in the MMA
 template <int kPlanes> struct Stages {
   static constexpr int K = 3;
   static constexpr int V = kPlanes == 1 ? 3 : 2;
@@ -78,30 +89,46 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kMeanBlocks = 5;              // key blocks per mean MMA (3 K slots each: 15 of 16)
 constexpr int kMeanChunks = 2;              // R: 16-slot K chunks 0 and 1, alternating by batch
 constexpr uint32_t kOneE4M3x4 = 0x38383838u;
+// E2M1 1.0 (code 2) in the 16-byte smem container of 16 FP4 codes: the low 8
+// bytes hold the codes, two per byte, the high 8 bytes are padding
+constexpr uint32_t kOneE2M1x8 = 0x22222222u, kE2M1Pad = 0u;
+constexpr uint32_t kSfOne4 = 0x7F7F7F7Fu;   // four UE8M0 scale bytes of 2^0
+constexpr uint32_t kSfBytes = 512;          // MX exponents of one V block: 128 channels x 4 groups
+// bytes the TMA writes to shared memory for one 128 x 128 tile of E2M1 codes
+// (16-byte containers of 16 codes: the footprint of an 8-bit tile)
+constexpr uint32_t kMxTileTx = kTileBytes;
 // tensor-memory columns (see the layout above)
 __device__ __forceinline__ constexpr uint32_t col_o(int t) { return t ? 144u : 0u; }    // PV accumulator, N = 144
 __device__ __forceinline__ constexpr uint32_t col_ch(int t) { return t ? 160u : 0u; }   // output channels 0-127
 __device__ __forceinline__ constexpr uint32_t col_l(int t) { return t ? 144u : 128u; }  // first row-sum column
 __device__ __forceinline__ constexpr uint32_t col_s(int t) { return t ? 320u : 288u; }  // scores
 __device__ __forceinline__ constexpr uint32_t col_p(int t) { return t ? 480u : 448u; }  // P codes, 32 columns
+// MX-style V: both score tiles in [320, 448); the scale factors of P (constant
+// 2^0, 4 columns) and of V^T (5 of 8 columns) of each tile below them
+__device__ __forceinline__ constexpr uint32_t col_s_mx() { return 320u; }
+__device__ __forceinline__ constexpr uint32_t col_sfa(int t) { return t ? 292u : 288u; }
+__device__ __forceinline__ constexpr uint32_t col_sfb(int t) { return t ? 304u : 296u; }
 
 // One V ring stage: [16 rows of 1.0][plane 0: V^T tile][16 rows of 1.0][plane 1].
 // Tile 0's PV reads plane 0 followed by the second band (ones last), tile 1's
 // the first band followed by plane 0 (ones first), so that the row sums land
 // at the ends of the two accumulators given above.
-template <int kPlanes> struct VStage {
+// The MX-style stage appends the block's 512 exponent bytes (kSf), padded to
+// keep every stage 1024-byte aligned.
+template <int kPlanes, bool kMx = false> struct VStage {
   static constexpr uint32_t kPlane0 = kOnesBytes;
   static constexpr uint32_t kOnes1 = kOnesBytes + kTileBytes;
   static constexpr uint32_t kPlane1 = 2 * kOnesBytes + kTileBytes;
-  static constexpr uint32_t kBytes = 2 * kOnesBytes + kPlanes * kTileBytes;
+  static constexpr uint32_t kSf = 2 * kOnesBytes + kPlanes * kTileBytes;
+  static constexpr uint32_t kBytes = 2 * kOnesBytes + kPlanes * kTileBytes + (kMx ? 1024u : 0u);
 };
 
-template <int kPlanes>
+template <int kPlanes, bool kMx = false>
 struct __align__(1024) SmemAttn {
   static constexpr int kKStages = Stages<kPlanes>::K, kVStages = Stages<kPlanes>::V;
   uint8_t q[2][kTileBytes];
   uint8_t k[kKStages][kTileBytes];
-  uint8_t v[kVStages][VStage<kPlanes>::kBytes];
+  uint8_t v[kVStages][VStage<kPlanes, kMx>::kBytes];
   uint8_t rop[2][kTileBytes];    // R operand of the mean MMA, one 128-B-swizzled tile per query tile
   uint8_t mop[2][kMopBytes];     // M operand, unswizzled, one per batch parity
   uint64_t q_full;
@@ -216,12 +243,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-template <int kPlanes, bool kExp2 = false>
+template <int kPlanes, bool kExp2 = false, int kVKind = kVHead>
 __global__ void __launch_bounds__(kThreads, 1)
     vc_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnParams P) {
-  using Smem = SmemAttn<kPlanes>;
-  using VS = VStage<kPlanes>;
+  constexpr bool kMx = kVKind == kVMx;
+  static_assert(!kMx || kPlanes == 1, "the MX-style residual is one plane");
+  using Smem = SmemAttn<kPlanes, kMx>;
+  using VS = VStage<kPlanes, kMx>;
   constexpr int kKStages = Smem::kKStages, kVStages = Smem::kVStages;
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -262,7 +291,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = threadIdx.x; i < (int)(kVStages * 2 * kOnesBytes / 16); i += kThreads) {
     const int st = i / (2 * kOnesBytes / 16), r = i % (2 * kOnesBytes / 16);
     const uint32_t off = r < (int)(kOnesBytes / 16) ? r * 16 : VS::kOnes1 + (r - kOnesBytes / 16) * 16;
-    *reinterpret_cast<uint4*>(&s.v[st][0] + off) = make_uint4(kOneE4M3x4, kOneE4M3x4, kOneE4M3x4, kOneE4M3x4);
+    *reinterpret_cast<uint4*>(&s.v[st][0] + off) =
+        kMx ? make_uint4(kOneE2M1x8, kOneE2M1x8, kE2M1Pad, kE2M1Pad)   // a whole 16-byte container
+            : make_uint4(kOneE4M3x4, kOneE4M3x4, kOneE4M3x4, kOneE4M3x4);
   }
   fence_proxy_async_smem();
   if (warp == 0) {
@@ -273,7 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  const float sV = __fmul_rn(P.s_v[bh], P.v_mul);   // value scale of the residual codes
+  // value scale of the residual codes (per-channel scales are read where used;
+  // the MX-style residual carries its scales inside the product: s_v is 1)
+  const float sV = kVKind == kVChannel ? 1.0f : __fmul_rn(P.s_v[bh], P.v_mul);
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
@@ -281,7 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // lane issues the copies. Every kMeanBlocks blocks the warp also writes the
     // M operand of one batch: lane l takes channels l, l+32, l+64, l+96.
     const bool leader = elect_one();
-    const float inv_sV = __fdiv_rn(1.0f, sV);
+    float inv_sV[4];   // 1 / s_V of channels lane + 32 i
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      inv_sV[i] = __fdiv_rn(1.0f, kVKind == kVChannel ? P.s_v[(size_t)bh * 128 + lane + 32 * i] : sV);
     const float* const mu_bh = P.mu + (size_t)bh * P.nb * 128;
     float mnext[kMeanBlocks][4];  // block means of the next batch, loaded one batch ahead
     auto load_means = [&](int batch) {
@@ -314,11 +350,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int vs = j % kVStages;
       if (!wait_spin_warp(s, &s.v_empty[vs], ((j / kVStages) & 1) ^ 1, P)) break;
       if (leader) {
-        mbar_arrive_expect_tx(&s.v_full[vs], kPlanes * kTileBytes);
-        // plane pl of head bh: rows (pl * BH + bh) * 128
-        tma_load_2d(&s.v[vs][0] + VS::kPlane0, &tmV, &s.v_full[vs], j * 128, bh * 128);
-        if (kPlanes == 2)
-          tma_load_2d(&s.v[vs][0] + VS::kPlane1, &tmV, &s.v_full[vs], j * 128, (P.B * P.H + bh) * 128);
+        if (kMx) {
+          // the E2M1 tile (x in codes: 64 bytes a block in HBM) and the block's exponents
+          mbar_arrive_expect_tx(&s.v_full[vs], kMxTileTx + kSfBytes);
+          tma_load_2d(&s.v[vs][0] + VS::kPlane0, &tmV, &s.v_full[vs], j * 128, bh * 128);
+          bulk_load(&s.v[vs][0] + VS::kSf, P.v_scales + ((size_t)bh * P.nb + j) * kSfBytes, kSfBytes,
+                    &s.v_full[vs]);
+        } else {
+          mbar_arrive_expect_tx(&s.v_full[vs], kPlanes * kTileBytes);
+          // plane pl of head bh: rows (pl * BH + bh) * 128
+          tma_load_2d(&s.v[vs][0] + VS::kPlane0, &tmV, &s.v_full[vs], j * 128, bh * 128);
+          if (kPlanes == 2)
+            tma_load_2d(&s.v[vs][0] + VS::kPlane1, &tmV, &s.v_full[vs], j * 128, (P.B * P.H + bh) * 128);
+        }
       }
       v_issued = j + 1;
       if (j % kMeanBlocks == 0) {
@@ -340,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int g = 0; g < kMeanBlocks; ++g) {
             __nv_bfloat16 mh, ml;
-            split_bf16(__fmul_rn(cur[g][i], inv_sV), mh, ml);
+            split_bf16(__fmul_rn(cur[g][i], inv_sV[i]), mh, ml);
             sl[3 * g + 0] = bf16_bits(mh);
             sl[3 * g + 1] = bf16_bits(ml);
             sl[3 * g + 2] = bf16_bits(mh);
@@ -381,7 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dk = sdesc_k_sw128(smem_u32(s.k[ks]));
         if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) umma_f8f6f4_ss(tmem + col_s(t), dq[t] + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f8f6f4_ss(tmem + (kMx ? col_s_mx() : col_s(t)), dq[t] + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
         }
       };
       // The QK products alternate between the tiles through the shared score
@@ -430,9 +475,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vb = smem_u32(&s.v[vs][0]);
         const uint64_t dv = sdesc_k_sw128(vb + (t == 0 ? VS::kPlane0 : 0u));
         if (leader) {
+          if (kMx) {
+            // K group kk of the block: scale byte kk of every SFB_t cell
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_f8f6f4_ts(tmem + col_o(t), tmem + col_p(t) + 8 * kk, dv + 2 * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              umma_mx_ts(tmem + col_o(t), tmem + col_p(t) + 8 * kk, dv + 2 * kk,
+                         idesc_mx(kFmtE4M3, kFmtE2M1, 128, 144, 0, kk), tmem + col_sfa(t), tmem + col_sfb(t),
+                         (j > 0 || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f8f6f4_ts(tmem + col_o(t), tmem + col_p(t) + 8 * kk, dv + 2 * kk, id_pv,
+                             (j > 0 || kk > 0) ? 1u : 0u);
+          }
           if (kPlanes == 2) {
             const uint64_t dv2 = sdesc_k_sw128(vb + VS::kPlane1);
 #pragma unroll
@@ -459,7 +514,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = warp >> 2;               // query tile
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + col_s(t);
+    const uint32_t s_addr = tmem + lane_base + (kMx ? col_s_mx() : col_s(t));
+    const uint32_t sfb_addr = tmem + lane_base + col_sfb(t);
+    if (kMx) {
+      // the probabilities' scale factors: 2^0 for every row and K group; written
+      // once (each warp its own lane quarter), before the tile's first p_full
+      tmem_st4(tmem + lane_base + col_sfa(t), kSfOne4, kSfOne4, kSfOne4, kSfOne4);
+    }
     const uint32_t p_addr = tmem + lane_base + col_p(t);
     const uint32_t o_addr = tmem + lane_base + col_ch(t);
     const uint32_t l_addr = tmem + lane_base + col_l(t);
@@ -543,6 +604,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 #undef SC
+      // MX-style V: the scale factors of V_j^T for this tile's B operand, one
+      // cell per (lane, column c): the 4 group exponents of B row n = lane + 32 c,
+      // which is channel n (tile 0: ones rows at n >= 128) or n - 16 (tile 1:
+      // ones rows first); the ones rows and the unused cells take 2^0
+      uint32_t sfr[8];
+      if (kMx) {
+        const int vs = j % kVStages;
+        if (!(ok = wait_warp(s, &s.v_full[vs], (j / kVStages) & 1, P))) break;
+        const uint32_t* sfw = reinterpret_cast<const uint32_t*>(&s.v[vs][0] + VS::kSf);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int ch = lane + 32 * c - (t ? 16 : 0);
+          sfr[c] = (c < 5 && ch >= 0 && ch < 128) ? sfw[ch] : kSfOne4;
+        }
+      }
       // PV(j-1) has read P_t and added block j-1 to O_t: then the row-sum column
       // is read, O_t may be rescaled and P_t(j) written
       uint32_t lraw = 0u;
@@ -553,6 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
       }
       tmem_st32(p_addr, w);
+      if (kMx) tmem_st8(sfb_addr, sfr);
       const float Lc = __uint_as_float(lraw);
       if (__any_sync(0xffffffffu, resc)) {
         // the frame moved: O_t (complete up to block j-1) and its row-sum column
@@ -625,8 +702,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
+          float s0 = scale, s1 = scale;
+          if (kVKind == kVChannel) {  // s_V of the two channels over l
+            const float* sv = P.s_v + (size_t)bh * 128 + cc * 32 + 2 * i;
+            s0 = __fdiv_rn(sv[0], l);
+            s1 = __fdiv_rn(sv[1], l);
+          }
           __nv_bfloat162 b2 =
-              __floats2bfloat162_rn(__uint_as_float(r[2 * i]) * scale, __uint_as_float(r[2 * i + 1]) * scale);
+              __floats2bfloat162_rn(__uint_as_float(r[2 * i]) * s0, __uint_as_float(r[2 * i + 1]) * s1);
           pk[i] = *reinterpret_cast<uint32_t*>(&b2);
         }
         if (q_valid && q < P.S) {
@@ -651,6 +734,12 @@ cudaError_t attn_configure() {
   cudaError_t e = cudaFuncSetAttribute(vc_attn_fwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)(sizeof(SmemAttn<1>) + 1024));
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(vc_attn_fwd_kernel<1, false, kVChannel>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)(sizeof(SmemAttn<1>) + 1024));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(vc_attn_fwd_kernel<1, false, kVMx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)(sizeof(SmemAttn<1, true>) + 1024));
+  if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(vc_attn_fwd_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)(sizeof(SmemAttn<1>) + 1024));
   if (e != cudaSuccess) return e;
@@ -665,6 +754,20 @@ cudaError_t launch_attn_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const
     vc_attn_fwd_kernel<1, true><<<grid, kThreads, sizeof(SmemAttn<1>) + 1024, st>>>(tq, tk, tv, p);
   else
     vc_attn_fwd_kernel<1><<<grid, kThreads, sizeof(SmemAttn<1>) + 1024, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_channel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const AttnParams& p, cudaStream_t st) {
+  const dim3 grid((p.nb + 1) / 2, p.B * p.H);
+  vc_attn_fwd_kernel<1, false, kVChannel><<<grid, kThreads, sizeof(SmemAttn<1>) + 1024, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_mx(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv_e2m1,
+                           const AttnParams& p, cudaStream_t st) {
+  const dim3 grid((p.nb + 1) / 2, p.B * p.H);
+  vc_attn_fwd_kernel<1, false, kVMx><<<grid, kThreads, sizeof(SmemAttn<1, true>) + 1024, st>>>(tq, tk, tv_e2m1, p);
   return cudaGetLastError();
 }
 

@@ -17,6 +17,7 @@ namespace vc {
 constexpr int kD = 128;           // head dimension
 constexpr int kBlock = 128;       // 128-token blocks (also the MMA tile)
 constexpr int kGroup4 = 16;       // NVFP4: one E4M3 scale per 16 tokens
+constexpr int kMxGroup = 32;      // MX-style FP4: one power-of-two scale per 32 tokens
 constexpr float kE4M3Max = 448.0f;
 constexpr float kE2M1Max = 6.0f;
 constexpr float kTinyAmax = 7.888609052210118e-31f;  // 2^-100: below this a block is all zero

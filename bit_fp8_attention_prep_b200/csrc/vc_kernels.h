@@ -58,8 +58,8 @@ struct AttnParams {
   const float* q_scales;   // [BH][nb]
   const float* k_scales;   // [BH][nb]
   const float* mu;         // [BH][nb][128]
-  const float* s_v;        // [BH]
-  const uint8_t* v_scales; // NVFP4: [BH][128][S_pad/16]
+  const float* s_v;        // [BH] ([BH][128] for the per-channel scale)
+  const uint8_t* v_scales; // NVFP4: [BH][128][S_pad/16]; MX-style: [BH][nb][128][4]
   float kappa;             // fl32(softmax_scale * log2 e)
   float v_mul;             // value scale = s_v * v_mul (1 for E4M3; 8 for the NVFP4 planes)
   int bias_b;              // 56 + 8 k_P
@@ -73,6 +73,13 @@ cudaError_t attn_configure();
 // E4M3 conversion instead of ExpCast (test hook only)
 cudaError_t launch_attn_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const AttnParams& p, cudaStream_t st, bool exp2 = false);
+// E4M3 residual with one scale per (b, h, channel) (p.s_v is [BH][128]).
+cudaError_t launch_attn_channel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const AttnParams& p, cudaStream_t st);
+// MX-style FP4 residual: `tv_e2m1` maps the packed E2M1 codes as 16-byte smem
+// containers (128 x 128 codes a box); p.v_scales holds the exponents [BH][nb][128][4].
+cudaError_t launch_attn_mx(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv_e2m1,
+                           const AttnParams& p, cudaStream_t st);
 // NVFP4 residual: `tplanes` maps the two E4M3 planes written by launch_nvfp4_planes.
 cudaError_t launch_attn_planes(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tplanes,
                                const AttnParams& p, cudaStream_t st);

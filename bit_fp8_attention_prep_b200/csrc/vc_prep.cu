@@ -568,8 +568,9 @@ __global__ void identity_perm_kernel(int S, int32_t* __restrict__ perm) {
 // lane l owns dimensions 8(l%16) .. 8(l%16)+7. The amax pass reads the rows
 // again (from L1 / L2). Means use the int64 fixed-point sum (naive mode: all
 // means are 0 and the first pass is skipped); the residual amax is merged into
-// amax[bh] with an integer atomicMax on the (non-negative) fp32 bits.
-template <typename T>
+// amax[bh] with an integer atomicMax on the (non-negative) fp32 bits; with
+// kPerCh, one amax per channel, amax[bh * 128 + d].
+template <typename T, bool kPerCh = false>
 __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ v, int S, int H,
                                                           const int32_t* __restrict__ perm, bool naive,
                                                           float* __restrict__ mu,
@@ -627,7 +628,7 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ 
   float m8[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) m8[e] = smu[c * 8 + e];
-  float mx = 0.0f;
+  float mx8[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};  // per channel of this lane
 #pragma unroll 1
   for (int i0 = 0; i0 < 16; i0 += 8) {
     uint4 x[8];
@@ -638,15 +639,32 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ 
       float f[8];
       unpack8<T>(x[i], f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(__fsub_rn(f[e], m8[e])));
+      for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], fabsf(__fsub_rn(f[e], m8[e])));
     }
   }
-  mx = warp_max(mx);
-  if (lane == 0) wmax[warp] = mx;
-  __syncthreads();
-  if (tid == 0) {
-    const float m = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
-    atomicMax(&amax[bh], __float_as_uint(m));
+  if (!kPerCh) {
+    float mx = mx8[0];
+#pragma unroll
+    for (int e = 1; e < 8; ++e) mx = fmaxf(mx, mx8[e]);
+    mx = warp_max(mx);
+    if (lane == 0) wmax[warp] = mx;
+    __syncthreads();
+    if (tid == 0) {
+      const float m = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+      atomicMax(&amax[bh], __float_as_uint(m));
+    }
+  } else {
+    // lanes c and c + 16 hold the same channels; then the four warps
+    __shared__ float cmax[4][kD];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], __shfl_xor_sync(0xffffffffu, mx8[e], 16));
+    if (half == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cmax[warp][c * 8 + e] = mx8[e];
+    }
+    __syncthreads();
+    const float m = fmaxf(fmaxf(cmax[0][tid], cmax[1][tid]), fmaxf(cmax[2][tid], cmax[3][tid]));
+    atomicMax(&amax[(size_t)bh * kD + tid], __float_as_uint(m));
   }
 }
 
@@ -662,7 +680,9 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ 
 // A warp reads 8 channel groups of 4 token quads, which fall on 32 distinct banks.
 constexpr int kResStride = 136;
 
-template <typename T>
+// With kPerCh the scale is one per channel (amax_bits[bh * 128 + d], s_v
+// [bh][128]): a channel whose amax is below 2^-100 gets scale 1 and codes 0.
+template <typename T, bool kPerCh = false>
 __global__ void __launch_bounds__(256) residual_e4m3_kernel(const T* __restrict__ v, int S, int H, int S_pad,
                                                             const int32_t* __restrict__ perm,
                                                             const float* __restrict__ mu,
@@ -672,10 +692,26 @@ __global__ void __launch_bounds__(256) residual_e4m3_kernel(const T* __restrict_
   const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int half = lane >> 4, c = lane & 15;
-  const float amax = __uint_as_float(amax_bits[bh]);
-  const bool zero = !(amax >= kTinyAmax);
-  const float inv = zero ? 0.0f : __fdiv_rn(kE4M3Max, amax);
-  if (blk == 0 && threadIdx.x == 0) s_v[bh] = zero ? 1.0f : __fdiv_rn(amax, kE4M3Max);
+  float inv8[8];   // 448 / amax of each of this lane's 8 channels (0 for an all-zero one)
+  bool zero = false;
+  if (!kPerCh) {
+    const float amax = __uint_as_float(amax_bits[bh]);
+    zero = !(amax >= kTinyAmax);
+    const float inv = zero ? 0.0f : __fdiv_rn(kE4M3Max, amax);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) inv8[e] = inv;
+    if (blk == 0 && threadIdx.x == 0) s_v[bh] = zero ? 1.0f : __fdiv_rn(amax, kE4M3Max);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float a = __uint_as_float(amax_bits[(size_t)bh * kD + c * 8 + e]);
+      inv8[e] = a >= kTinyAmax ? __fdiv_rn(kE4M3Max, a) : 0.0f;
+    }
+    if (blk == 0 && threadIdx.x < kD) {
+      const float a = __uint_as_float(amax_bits[(size_t)bh * kD + threadIdx.x]);
+      s_v[(size_t)bh * kD + threadIdx.x] = a >= kTinyAmax ? __fdiv_rn(a, kE4M3Max) : 1.0f;
+    }
+  }
   float m8[8];
   {
     const float4* mp = reinterpret_cast<const float4*>(mu + ((size_t)bh * gridDim.x + blk) * kD + c * 8);
@@ -704,7 +740,8 @@ __global__ void __launch_bounds__(256) residual_e4m3_kernel(const T* __restrict_
       unpack8<T>(xs[i], f);
       float rr[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) rr[e] = __fmul_rn(__fsub_rn(f[e], m8[e]), inv);
+      for (int e = 0; e < 8; ++e)  // an all-zero channel codes to +0 (no -0 from a negative tiny residual)
+        rr[e] = inv8[e] != 0.0f ? __fmul_rn(__fsub_rn(f[e], m8[e]), inv8[e]) : 0.0f;
       w.x = (uint32_t)cvt_e4m3x2(rr[0], rr[1]) | ((uint32_t)cvt_e4m3x2(rr[2], rr[3]) << 16);
       w.y = (uint32_t)cvt_e4m3x2(rr[4], rr[5]) | ((uint32_t)cvt_e4m3x2(rr[6], rr[7]) << 16);
     }
@@ -791,6 +828,78 @@ __global__ void __launch_bounds__(128) residual_nvfp4_kernel(const T* __restrict
     *reinterpret_cast<uint2*>(crow + gi * (kGroup4 / 2)) = make_uint2(w[0], w[1]);
     srow[gi] = sc;
   }
+}
+
+// --------------------------------------------------------------- residual MX-style FP4
+// Per channel and group of 32 consecutive permuted tokens, the power of two
+// X = 2^e with e the smallest integer for which the group's amax <= 6 * 2^e (so
+// no value clips), e >= -127; E2M1 codes of r * 2^-e (exact scaling, then one
+// round to nearest even). From the fp32 bits of the amax, amax = f * 2^E with f
+// in [1, 2): 6 * 2^(E-2) = 1.5 * 2^E covers it iff f <= 1.5, else 6 * 2^(E-1);
+// an amax below 2^-126 (zero or subnormal) gives the clamp value -127.
+// Outputs: packed codes as the NVFP4 residual ([BH][128][S_pad/2], even token in
+// the low nibble) and the biased exponents e + 127 as [BH][nb][128][4] bytes
+// (block, channel, group of the block), so that a block's exponents are one
+// 512-byte piece with one word per channel.
+__device__ __forceinline__ int mx_exponent(float amax) {
+  const uint32_t bits = __float_as_uint(amax);
+  const int be = (int)(bits >> 23);
+  if (be == 0) return -127;
+  const int E = be - 127;
+  return max(-127, (bits & 0x7FFFFFu) <= 0x400000u ? E - 2 : E - 1);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) residual_mxfp4_kernel(const T* __restrict__ v, int S, int H, int S_pad,
+                                                             const int32_t* __restrict__ perm,
+                                                             const float* __restrict__ mu,
+                                                             uint8_t* __restrict__ codes,
+                                                             uint32_t* __restrict__ exps, float* __restrict__ s_v) {
+  extern __shared__ __align__(16) float rt[];  // [128 channels][129]
+  __shared__ float smu[kD];
+  const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x, nb = gridDim.x;
+  const int t = threadIdx.x;
+  if (blk == 0 && t == 0) s_v[bh] = 1.0f;   // no per-head scale
+  smu[t] = mu[((size_t)bh * nb + blk) * kD + t];
+  __syncthreads();
+  {
+    const int p = blk * kBlock + t;  // thread t: permuted row t
+    if (p < S) {
+      const T* row = v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD;
+#pragma unroll 4
+      for (int c = 0; c < 16; ++c) {
+        float f[8];
+        unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) rt[(c * 8 + e) * 129 + t] = __fsub_rn(f[e], smu[c * 8 + e]);
+      }
+    } else {
+      for (int d = 0; d < kD; ++d) rt[d * 129 + t] = 0.0f;
+    }
+  }
+  __syncthreads();
+  const int d = t;  // thread t: channel t
+  const float* rr = rt + d * 129;
+  uint8_t* crow = codes + ((size_t)bh * kD + d) * (S_pad / 2) + (size_t)blk * (kBlock / 2);
+  uint32_t ew = 0u;
+#pragma unroll 1
+  for (int gi = 0; gi < kBlock / kMxGroup; ++gi) {
+    float gmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMxGroup; ++i) gmax = fmaxf(gmax, fabsf(rr[gi * kMxGroup + i]));
+    const int e = mx_exponent(gmax);
+    const float sc = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, normal for e in [-127, 126]
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int i = 0; i < kMxGroup; i += 2) {
+      const uint32_t byte =
+          cvt_e2m1x2(__fmul_rn(rr[gi * kMxGroup + i], sc), __fmul_rn(rr[gi * kMxGroup + i + 1], sc));
+      w[i >> 3] |= byte << (8 * ((i >> 1) & 3));
+    }
+    *reinterpret_cast<uint4*>(crow + gi * (kMxGroup / 2)) = make_uint4(w[0], w[1], w[2], w[3]);
+    ew |= (uint32_t)(e + 127) << (8 * gi);
+  }
+  exps[((size_t)bh * nb + blk) * kD + d] = ew;
 }
 
 // --------------------------------------------------------------- token sums (K smoothing)
@@ -1233,10 +1342,20 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
     ++n;
   }
   const dim3 gb(pl.nb, BH);
-  block_stats_kernel<T><<<gb, 128, 0, st>>>(v, S, H, out.perm, pl.mode == VC_MODE_NAIVE, out.mu, pl.amax);
+  const bool naive = pl.mode == VC_MODE_NAIVE;
+  if (pl.fmt == VC_RESIDUAL_E4M3_PER_CHANNEL)
+    block_stats_kernel<T, true><<<gb, 128, 0, st>>>(v, S, H, out.perm, naive, out.mu, pl.amax);
+  else
+    block_stats_kernel<T><<<gb, 128, 0, st>>>(v, S, H, out.perm, naive, out.mu, pl.amax);
   if (pl.fmt == VC_RESIDUAL_E4M3) {
     residual_e4m3_kernel<T><<<gb, 256, 0, st>>>(v, S, H, pl.S_pad, out.perm, out.mu, pl.amax, out.v_codes,
                                                 out.s_v);
+  } else if (pl.fmt == VC_RESIDUAL_E4M3_PER_CHANNEL) {
+    residual_e4m3_kernel<T, true><<<gb, 256, 0, st>>>(v, S, H, pl.S_pad, out.perm, out.mu, pl.amax,
+                                                      out.v_codes, out.s_v);
+  } else if (pl.fmt == VC_RESIDUAL_MXFP4) {
+    residual_mxfp4_kernel<T><<<gb, 128, kD * 129 * sizeof(float), st>>>(
+        v, S, H, pl.S_pad, out.perm, out.mu, out.v_codes, reinterpret_cast<uint32_t*>(out.v_scales), out.s_v);
   } else {
     residual_nvfp4_kernel<T><<<gb, 128, kD * 129 * sizeof(float), st>>>(v, S, H, pl.S_pad, out.perm, out.mu,
                                                                          pl.amax, out.v_codes, out.v_scales,
@@ -1340,7 +1459,8 @@ cudaError_t prep_configure() {
   for (const auto& a : assign_fns)
     if ((e = cudaFuncSetAttribute(a.f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)a.bytes)) != cudaSuccess)
       return e;
-  for (auto f : {(const void*)residual_nvfp4_kernel<__nv_bfloat16>, (const void*)residual_nvfp4_kernel<__half>})
+  for (auto f : {(const void*)residual_nvfp4_kernel<__nv_bfloat16>, (const void*)residual_nvfp4_kernel<__half>,
+                 (const void*)residual_mxfp4_kernel<__nv_bfloat16>, (const void*)residual_mxfp4_kernel<__half>})
     if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kD * 129 * 4))) !=
         cudaSuccess)
       return e;

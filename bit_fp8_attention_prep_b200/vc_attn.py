@@ -18,7 +18,11 @@ VC_OK, VC_ERR_INVALID_ARG, VC_ERR_UNSUPPORTED, VC_ERR_WORKSPACE, VC_ERR_CUDA, VC
 STATUS_NAMES = ["VC_OK", "VC_ERR_INVALID_ARG", "VC_ERR_UNSUPPORTED", "VC_ERR_WORKSPACE", "VC_ERR_CUDA",
                 "VC_ERR_TIMEOUT"]
 VC_DTYPE_F16, VC_DTYPE_BF16 = 0, 1
-VC_RESIDUAL_E4M3, VC_RESIDUAL_NVFP4 = 0, 1
+VC_RESIDUAL_E4M3, VC_RESIDUAL_NVFP4, VC_RESIDUAL_E4M3_PER_CHANNEL, VC_RESIDUAL_MXFP4 = 0, 1, 2, 3
+# residual formats by name: "e4m3" (one scale per head), "nvfp4", "e4m3c" (one
+# E4M3 scale per channel), "mxfp4" (E2M1 with a power of two per 32 tokens)
+_FMTS = {"e4m3": VC_RESIDUAL_E4M3, "nvfp4": VC_RESIDUAL_NVFP4, "e4m3c": VC_RESIDUAL_E4M3_PER_CHANNEL,
+         "mxfp4": VC_RESIDUAL_MXFP4}
 VC_MODE_VSMOOTH, VC_MODE_MEANONLY, VC_MODE_NAIVE = 0, 1, 2
 _MODES = {"vsmooth": VC_MODE_VSMOOTH, "meanonly": VC_MODE_MEANONLY, "naive": VC_MODE_NAIVE}
 
@@ -30,6 +34,7 @@ ABI_SYMBOLS = [
     "vc_attn_prepare_v_noalloc", "vc_attn_run_host_workspace_bytes", "vc_attn_run_host",
     "vc_attn_residual_energy", "vc_attn_quant_qk_smoothk_workspace_bytes", "vc_attn_quant_qk_smoothk",
     "vc_attn_prepare_v_repair_workspace_bytes", "vc_attn_prepare_v_repair", "vc_attn_forward_repair",
+    "vc_attn_forward_e4m3_per_channel", "vc_attn_forward_mxfp4v",
 ]
 NOALLOC_SCRATCH_BYTES = 12 << 20  # VC_ATTN_NOALLOC_SCRATCH_BYTES
 TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
@@ -108,6 +113,9 @@ def load():
     lib.vc_attn_prepare_v_repair.restype = i32
     lib.vc_attn_prepare_v_repair.argtypes = [vp, P(Shape), P(VSmoothCfg), ctypes.c_double, P(PreparedV), vp, vp,
                                              sz, vp]
+    for name in ("vc_attn_forward_e4m3_per_channel", "vc_attn_forward_mxfp4v"):
+        getattr(lib, name).restype = i32
+        getattr(lib, name).argtypes = [P(QKFP8), P(PreparedV), P(Shape), ctypes.c_float, i32, vp, vp, vp]
     lib.vc_attn_forward_repair.restype = i32
     lib.vc_attn_forward_repair.argtypes = [P(QKFP8), P(PreparedV), P(Shape), ctypes.c_float, i32, vp, vp, vp]
     lib.vc_attn_residual_energy.restype = i32
@@ -158,29 +166,39 @@ def num_blocks(S):
     return (S + 127) // 128
 
 
+def _fmt_code(fmt):
+    if fmt not in _FMTS:
+        raise ValueError(f"fmt must be one of {sorted(_FMTS)} (got {fmt!r})")
+    return _FMTS[fmt]
+
+
+def _prepared_buffers(B, S, H, fmt, dev):
+    """The caller-owned outputs of the prep for one residual format (layouts as
+    in vc_prepared_v_t)."""
+    nb = num_blocks(S)
+    Sp = nb * 128
+    e = lambda shp, dt: torch.empty(shp, dtype=dt, device=dev)
+    out = dict(perm=e((B, H, S), torch.int32), mu=e((B, H, nb, 128), torch.float32), fmt=fmt,
+               s_v=e((B, H, 128) if fmt == "e4m3c" else (B, H), torch.float32))
+    if fmt == "nvfp4":
+        out["v_codes"], out["v_scales"] = e((B, H, 128, Sp // 2), torch.uint8), e((B, H, 128, Sp // 16), torch.uint8)
+    elif fmt == "mxfp4":
+        out["v_codes"], out["v_scales"] = e((B, H, 128, Sp // 2), torch.uint8), e((B, H, nb, 128, 4), torch.uint8)
+    else:
+        out["v_codes"], out["v_scales"] = e((B, H, 128, Sp), torch.uint8), None
+    return out
+
+
 def prepare_v(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", history=False):
     """V-Smooth prep of V (device tensor). Returns a dict of the caller-owned
     outputs (perm, mu, v_codes, v_scales, s_v; plus the per-pass assignments
     when ``history``)."""
     lib = load()
     sh = shape_of(v)
-    cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
-                     _MODES[mode])
+    cfg = VSmoothCfg(k, iters, seed, _fmt_code(fmt), _MODES[mode])
     B, S, H = sh.B, sh.S, sh.H
-    nb = num_blocks(S)
-    Sp = nb * 128
     dev = v.device
-    out = dict(
-        perm=torch.empty((B, H, S), dtype=torch.int32, device=dev),
-        mu=torch.empty((B, H, nb, 128), dtype=torch.float32, device=dev),
-        s_v=torch.empty((B, H), dtype=torch.float32, device=dev),
-    )
-    if fmt == "nvfp4":
-        out["v_codes"] = torch.empty((B, H, 128, Sp // 2), dtype=torch.uint8, device=dev)
-        out["v_scales"] = torch.empty((B, H, 128, Sp // 16), dtype=torch.uint8, device=dev)
-    else:
-        out["v_codes"] = torch.empty((B, H, 128, Sp), dtype=torch.uint8, device=dev)
-        out["v_scales"] = None
+    out = _prepared_buffers(B, S, H, fmt, dev)
     wsb = lib.vc_attn_prepare_v_workspace_bytes(ctypes.byref(sh), ctypes.byref(cfg))
     if wsb == 0:
         raise VCError(VC_ERR_INVALID_ARG, "invalid shape or config")
@@ -192,7 +210,6 @@ def prepare_v(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", history=Fals
                                  ctypes.c_void_p(ws.data_ptr() + off), wsb, _ptr(hist), _stream()))
     out["workspace"] = ws
     out["history"] = hist
-    out["fmt"] = fmt
     return out
 
 
@@ -202,21 +219,10 @@ def prepare_v_noalloc(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", hist
     allocated here (by torch), as the caller's buffers."""
     lib = load()
     sh = shape_of(v)
-    cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
-                     _MODES[mode])
+    cfg = VSmoothCfg(k, iters, seed, _fmt_code(fmt), _MODES[mode])
     B, S, H = sh.B, sh.S, sh.H
-    nb = num_blocks(S)
-    Sp = nb * 128
     dev = v.device
-    out = dict(perm=torch.empty((B, H, S), dtype=torch.int32, device=dev),
-               mu=torch.empty((B, H, nb, 128), dtype=torch.float32, device=dev),
-               s_v=torch.empty((B, H), dtype=torch.float32, device=dev), fmt=fmt)
-    if fmt == "nvfp4":
-        out["v_codes"] = torch.empty((B, H, 128, Sp // 2), dtype=torch.uint8, device=dev)
-        out["v_scales"] = torch.empty((B, H, 128, Sp // 16), dtype=torch.uint8, device=dev)
-    else:
-        out["v_codes"] = torch.empty((B, H, 128, Sp), dtype=torch.uint8, device=dev)
-        out["v_scales"] = None
+    out = _prepared_buffers(B, S, H, fmt, dev)
     hist = torch.empty((iters, B, H, S), dtype=torch.uint8, device=dev) if history else None
     pv = PreparedV(_ptr(out["perm"]), _ptr(out["mu"]), _ptr(out["v_codes"]), _ptr(out["v_scales"]), _ptr(out["s_v"]))
     _check(lib.vc_attn_prepare_v_noalloc(_ptr(v), ctypes.byref(sh), ctypes.byref(cfg), ctypes.byref(pv), _ptr(hist),
@@ -321,7 +327,8 @@ def forward(qk, pv, shape, softmax_scale=None, k_p=8, out=None, status=None, wor
     the input layout. ``shape`` is the vc_shape_t of Q (``shape_of(q)``).
     For an NVFP4 ``pv`` the call needs a device workspace of
     ``forward_nvfp4v_workspace_bytes(shape)`` bytes; one is allocated when
-    ``workspace`` is None."""
+    ``workspace`` is None. The other formats ("e4m3", "e4m3c", "mxfp4") go to
+    vc_attn_forward, vc_attn_forward_e4m3_per_channel and vc_attn_forward_mxfp4v."""
     lib = load()
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(128)
@@ -337,8 +344,10 @@ def forward(qk, pv, shape, softmax_scale=None, k_p=8, out=None, status=None, wor
                                           float(softmax_scale), int(k_p), _ptr(out), _ptr(workspace),
                                           workspace.numel() * workspace.element_size(), _ptr(status), _stream()))
     else:
-        _check(lib.vc_attn_forward(ctypes.byref(q_), ctypes.byref(p_), ctypes.byref(shape), float(softmax_scale),
-                                   int(k_p), _ptr(out), _ptr(status), _stream()))
+        fn = {"e4m3c": lib.vc_attn_forward_e4m3_per_channel, "mxfp4": lib.vc_attn_forward_mxfp4v}.get(
+            pv.get("fmt"), lib.vc_attn_forward)
+        _check(fn(ctypes.byref(q_), ctypes.byref(p_), ctypes.byref(shape), float(softmax_scale), int(k_p), _ptr(out),
+                  _ptr(status), _stream()))
     return out
 
 
@@ -374,18 +383,15 @@ class Plan:
         self.lib = load()
         dev = torch.device(device if device is not None else "cuda")
         self.shape = Shape(B, S, H, 128, VC_DTYPE_BF16 if dtype == torch.bfloat16 else VC_DTYPE_F16)
-        self.cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
-                              _MODES[mode])
+        self.cfg = VSmoothCfg(k, iters, seed, _fmt_code(fmt), _MODES[mode])
         self.fmt, self.k_p = fmt, int(k_p)
         self.softmax_scale = 1.0 / math.sqrt(128) if softmax_scale is None else float(softmax_scale)
         nb = num_blocks(S)
         Sp = nb * 128
         e = lambda shp, dt: torch.empty(shp, dtype=dt, device=dev)
-        self.perm, self.mu, self.s_v = e((B, H, S), torch.int32), e((B, H, nb, 128), torch.float32), e((B, H), torch.float32)
-        if fmt == "nvfp4":
-            self.v_codes, self.v_scales = e((B, H, 128, Sp // 2), torch.uint8), e((B, H, 128, Sp // 16), torch.uint8)
-        else:
-            self.v_codes, self.v_scales = e((B, H, 128, Sp), torch.uint8), None
+        pb = _prepared_buffers(B, S, H, fmt, dev)
+        self.perm, self.mu, self.s_v, self.v_codes, self.v_scales = (pb["perm"], pb["mu"], pb["s_v"], pb["v_codes"],
+                                                                     pb["v_scales"])
         self.q_codes, self.k_codes = e((B, H, Sp, 128), torch.uint8), e((B, H, Sp, 128), torch.uint8)
         self.q_scales, self.k_scales = e((B, H, nb), torch.float32), e((B, H, nb), torch.float32)
         self.o = e((B, S, H, 128), torch.bfloat16)
@@ -431,8 +437,10 @@ class Plan:
                                                    _ptr(self._fwd_ws), self.fwd_ws_bytes, _ptr(self.status),
                                                    _stream()))
         else:
-            _check(self.lib.vc_attn_forward(ctypes.byref(self._qk), ctypes.byref(self._pv), ctypes.byref(self.shape),
-                                            self.softmax_scale, self.k_p, _ptr(o), _ptr(self.status), _stream()))
+            fn = {"e4m3c": self.lib.vc_attn_forward_e4m3_per_channel, "mxfp4": self.lib.vc_attn_forward_mxfp4v}.get(
+                self.fmt, self.lib.vc_attn_forward)
+            _check(fn(ctypes.byref(self._qk), ctypes.byref(self._pv), ctypes.byref(self.shape), self.softmax_scale,
+                      self.k_p, _ptr(o), _ptr(self.status), _stream()))
         return o
 
     def run(self, q, k, v, out=None):
@@ -455,8 +463,7 @@ class HostPlan:
         dev = torch.device(device if device is not None else "cuda")
         self.dtype = dtype
         self.shape = Shape(B, S, H, 128, VC_DTYPE_BF16 if dtype == torch.bfloat16 else VC_DTYPE_F16)
-        self.cfg = VSmoothCfg(k, iters, seed, VC_RESIDUAL_NVFP4 if fmt == "nvfp4" else VC_RESIDUAL_E4M3,
-                              _MODES[mode])
+        self.cfg = VSmoothCfg(k, iters, seed, _fmt_code(fmt), _MODES[mode])
         self.k_p, self.head_chunk = int(k_p), int(head_chunk)
         self.softmax_scale = 1.0 / math.sqrt(128) if softmax_scale is None else float(softmax_scale)
         self.ws_bytes = self.lib.vc_attn_run_host_workspace_bytes(ctypes.byref(self.shape), ctypes.byref(self.cfg),

@@ -53,7 +53,12 @@ typedef enum {
 } vc_status_t;
 
 typedef enum { VC_DTYPE_F16 = 0, VC_DTYPE_BF16 = 1 } vc_dtype_t;
-typedef enum { VC_RESIDUAL_E4M3 = 0, VC_RESIDUAL_NVFP4 = 1 } vc_residual_fmt_t;
+typedef enum {
+  VC_RESIDUAL_E4M3 = 0,              /* E4M3 codes, one scale per (b, h)                */
+  VC_RESIDUAL_NVFP4 = 1,             /* E2M1 + E4M3 scale per 16 tokens + fp32 global   */
+  VC_RESIDUAL_E4M3_PER_CHANNEL = 2,  /* E4M3 codes, one scale per (b, h, channel)       */
+  VC_RESIDUAL_MXFP4 = 3              /* E2M1 + power-of-two scale per 32 tokens         */
+} vc_residual_fmt_t;
 typedef enum {
   VC_MODE_VSMOOTH = 0,      /* k-means + cluster sort + block means (the method)  */
   VC_MODE_MEANONLY = 1,     /* identity order, block means only (diagnostic)      */
@@ -80,12 +85,21 @@ typedef struct {
 /* Output of vc_attn_prepare_v (caller-owned device buffers):
  *  perm     int32 [B,H,S]      original token index at each permuted position
  *  mu       fp32  [B,H,nb,128] mean of each 128-token block (permuted order)
- *  v_codes  E4M3:  uint8 [B,H,128,S_pad]   residual codes, V^T (token-contiguous)
- *           NVFP4: uint8 [B,H,128,S_pad/2] two E2M1 codes per byte, even token
- *                  in the low nibble
- *  v_scales NVFP4 only: uint8 [B,H,128,S_pad/16] E4M3 scale per 16 tokens
- *  s_v      fp32  [B,H]        E4M3: residual scale s_V; NVFP4: global scale g
- * Padding columns (tokens >= S) of v_codes / v_scales are written as 0. */
+ *  v_codes  E4M3, E4M3_PER_CHANNEL: uint8 [B,H,128,S_pad] residual codes, V^T
+ *                  (token-contiguous)
+ *           NVFP4, MXFP4: uint8 [B,H,128,S_pad/2] two E2M1 codes per byte, even
+ *                  token in the low nibble (MXFP4: 32-byte aligned)
+ *  v_scales NVFP4: uint8 [B,H,128,S_pad/16] E4M3 scale per 16 tokens
+ *           MXFP4: uint8 [B,H,nb,128,4] biased exponent e + 127 of the scale 2^e
+ *                  of channel d and tokens 128 j + 32 g .. 128 j + 32 g + 31 at
+ *                  [b,h,j,d,g] (one 512-byte piece per 128-token block)
+ *           otherwise unused (may be NULL)
+ *  s_v      E4M3:  fp32 [B,H]     residual scale s_V
+ *           E4M3_PER_CHANNEL: fp32 [B,H,128] residual scale of each channel
+ *           NVFP4: fp32 [B,H]     global scale g
+ *           MXFP4: fp32 [B,H]     written as 1 (the scales are in v_scales)
+ * Padding columns (tokens >= S) of v_codes are written as 0 (MXFP4: exponent
+ * byte 0 for groups that hold only padding). */
 typedef struct {
   int32_t* perm;
   float* mu;
@@ -126,8 +140,18 @@ size_t vc_attn_prepare_v_workspace_bytes(const vc_shape_t* shape, const vc_vsmoo
  * paragraph): per (b, h), seeded k-means over the value tokens (k clusters,
  * `iters` Lloyd assignment passes), a stable sort of the tokens by cluster id
  * (the permutation also applied to K by vc_attn_quant_qk), subtraction of each
- * 128-token block's mean, and quantisation of the residual to E4M3 (one scale per
- * (b, h)) or NVFP4 (E2M1 + E4M3 scale per 16 tokens + fp32 global per (b, h)).
+ * 128-token block's mean, and quantisation of the residual (cfg->residual_fmt):
+ *  - VC_RESIDUAL_E4M3: E4M3, one scale amax/448 per (b, h) ("Open VC Attention",
+ *    "Описание": V scales per head);
+ *  - VC_RESIDUAL_NVFP4: E2M1 + E4M3 scale per 16 tokens + fp32 global per (b, h)
+ *    ("Nunchux AI lanza ...", 2nd paragraph);
+ *  - VC_RESIDUAL_E4M3_PER_CHANNEL: E4M3 with one scale amax_d/448 per (b, h,
+ *    channel d) (no passage: the per-head scale of the card, taken per channel);
+ *    a channel whose amax is below 2^-100 gets scale 1 and codes 0;
+ *  - VC_RESIDUAL_MXFP4: E2M1 codes of r * 2^-e with one power of two per
+ *    channel and 32 consecutive permuted tokens, e the smallest integer >= -127
+ *    with amax <= 6 * 2^e, so that nothing clips (no passage: the tensor cores'
+ *    block-scaled FP4 operand, a neighbour of the NVFP4 residual).
  * cfg->mode VC_MODE_MEANONLY keeps the original order (perm = identity);
  * VC_MODE_NAIVE also writes all block means as 0, so V itself is quantised (the
  * baseline the method improves on; vc_attn_forward then adds no mean).
@@ -254,6 +278,28 @@ vc_status_t vc_attn_forward(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, co
                             float softmax_scale, int32_t k_p, void* o, int32_t* dev_status,
                             void* stream);
 
+/* As vc_attn_forward, for a V residual prepared with
+ * VC_RESIDUAL_E4M3_PER_CHANNEL (pv->s_v holds one scale per (b, h, channel)):
+ * O = (s_V[d] * (P V_codes)[d] + sum_tiles rowsum(P_tile) mu_tile[d]) / rowsum(P)
+ * for each output channel d (no passage: the per-head V scale of "Open VC
+ * Attention", "Описание", taken per channel; the mean restore and the scores are
+ * those of vc_attn_forward). Errors: as vc_attn_forward. */
+vc_status_t vc_attn_forward_e4m3_per_channel(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv,
+                                             const vc_shape_t* shape, float softmax_scale, int32_t k_p, void* o,
+                                             int32_t* dev_status, void* stream);
+
+/* As vc_attn_forward, for a V residual prepared with VC_RESIDUAL_MXFP4
+ * (pv->v_codes packed E2M1 V^T, pv->v_scales the biased exponents): the P V
+ * product runs on the block-scaled FP8 x FP4 tensor-core MMA, E4M3 probability
+ * codes times E2M1 residual codes with the power of two 2^e of each channel and
+ * 32 keys applied inside the product, so the residual is read at 4.25 bits per
+ * value and no decoded copy is made (no passage: the block-scaled form of the
+ * NVFP4 residual of "Nunchux AI lanza ...", 2nd paragraph).
+ *   O = (P (e2m1 * 2^e) + sum_tiles rowsum(P_tile) mu_tile) / rowsum(P)
+ * pv->v_codes must be 32-byte aligned. Errors: as vc_attn_forward. */
+vc_status_t vc_attn_forward_mxfp4v(const vc_qk_fp8_t* qk, const vc_prepared_v_t* pv, const vc_shape_t* shape,
+                                   float softmax_scale, int32_t k_p, void* o, int32_t* dev_status, void* stream);
+
 /* Bytes of device workspace vc_attn_forward_nvfp4v needs: 2*B*H*128*S_pad
  * (S_pad = S rounded up to 128). 0 for an invalid shape. */
 size_t vc_attn_forward_nvfp4v_workspace_bytes(const vc_shape_t* shape);
@@ -317,7 +363,8 @@ size_t vc_attn_run_host_workspace_bytes(const vc_shape_t* shape, const vc_vsmoot
                                         int32_t head_chunk);
 
 /* The whole path -- vc_attn_prepare_v, vc_attn_quant_qk and vc_attn_forward (or
- * vc_attn_forward_nvfp4v for cfg->residual_fmt == VC_RESIDUAL_NVFP4) -- for Q, K,
+ * the forward call of cfg->residual_fmt: vc_attn_forward_nvfp4v,
+ * vc_attn_forward_e4m3_per_channel, vc_attn_forward_mxfp4v) -- for Q, K,
  * V and O in HOST memory, with the host<->device copies overlapped with the
  * compute. Every (b, h) slice of the method is independent ("VC-Attention ...",
  * Abstract: clustering, block means and the residual scale are per value head;

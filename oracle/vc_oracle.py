@@ -675,6 +675,9 @@ def prepare_v_head(V, k, iters, seed, bh, fmt="e4m3", adopt=None, mode="vsmooth"
     if fmt == "e4m3":
         vt, s_v, amax = residual_e4m3(V, perm, mu)
         out.update(v_codes=vt, s_v=s_v, amax=amax, vres=vres_from_e4m3(vt, s_v, S))
+    elif fmt == "e4m3c":
+        vt, s_v, amax = residual_e4m3_per_channel(V, perm, mu)
+        out.update(v_codes=vt, s_v=s_v, amax=amax, vres=vres_from_e4m3_per_channel(vt, s_v, S))
     elif fmt == "mxfp4":
         codes, e8 = residual_mxfp4(V, perm, mu)
         out.update(v_codes=codes, v_scales=e8, vres=vres_from_mxfp4(codes, e8, S))

@@ -53,7 +53,7 @@ def test_workspace_bytes_and_validation(lib):
     assert big > ok
     for sh in (_shape(D=64), _shape(S=0), _shape(H=0), _shape(dt=7), _shape(S=1 << 20, H=200)):
         assert lib.vc_attn_prepare_v_workspace_bytes(ctypes.byref(sh), ctypes.byref(_cfg())) == 0
-    for cfg in (_cfg(k=0), _cfg(k=33), _cfg(iters=0), _cfg(fmt=3), _cfg(mode=5)):
+    for cfg in (_cfg(k=0), _cfg(k=33), _cfg(iters=0), _cfg(fmt=4), _cfg(fmt=-1), _cfg(mode=5)):
         assert lib.vc_attn_prepare_v_workspace_bytes(ctypes.byref(_shape()), ctypes.byref(cfg)) == 0
 
 
