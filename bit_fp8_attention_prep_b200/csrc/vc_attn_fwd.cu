@@ -94,9 +94,10 @@ constexpr uint32_t kOneE4M3x4 = 0x38383838u;
 constexpr uint32_t kOneE2M1x8 = 0x22222222u, kE2M1Pad = 0u;
 constexpr uint32_t kSfOne4 = 0x7F7F7F7Fu;   // four UE8M0 scale bytes of 2^0
 constexpr uint32_t kSfBytes = 512;          // MX exponents of one V block: 128 channels x 4 groups
-// bytes the TMA writes to shared memory for one 128 x 128 tile of E2M1 codes
-// (16-byte containers of 16 codes: the footprint of an 8-bit tile)
-constexpr uint32_t kMxTileTx = kTileBytes;
+// transaction bytes of one 128 x 128 tile of E2M1 codes: the packed bytes read
+// (64 per row), although each 16 codes land in a 16-byte shared-memory container
+// whose upper 8 bytes the TMA leaves untouched (the MMA ignores them)
+constexpr uint32_t kMxTileTx = kTileBytes / 2;
 // tensor-memory columns (see the layout above)
 __device__ __forceinline__ constexpr uint32_t col_o(int t) { return t ? 144u : 0u; }    // PV accumulator, N = 144
 __device__ __forceinline__ constexpr uint32_t col_ch(int t) { return t ? 160u : 0u; }   // output channels 0-127

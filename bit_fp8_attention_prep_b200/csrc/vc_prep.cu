@@ -1313,7 +1313,8 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
   const int S = pl.S, H = pl.H, BH = pl.B * pl.H, k = pl.k;
   cudaError_t e;
   int n = 0;
-  if ((e = cudaMemsetAsync(pl.amax, 0, sizeof(unsigned) * BH, st)) != cudaSuccess) return e;
+  const size_t namax = (size_t)BH * (pl.fmt == VC_RESIDUAL_E4M3_PER_CHANNEL ? kD : 1);  // per (b, h) or channel
+  if ((e = cudaMemsetAsync(pl.amax, 0, sizeof(unsigned) * namax, st)) != cudaSuccess) return e;
   if (pl.mode == VC_MODE_VSMOOTH) {
     if ((e = cudaMemsetAsync(pl.sums, 0, sizeof(unsigned long long) * BH * k * kD, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(pl.counts, 0, sizeof(int) * BH * k, st)) != cudaSuccess) return e;
