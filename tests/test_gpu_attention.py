@@ -95,20 +95,34 @@ def test_attention_nvfp4_plan_matches_one_shot_calls(va):
 
 
 def test_attention_accuracy_vs_exact_and_naive(va):
-    # Reported figures: rel-L2 vs FP64 exact attention, and the error reduction of
-    # V-Smooth over per-head FP8 V with the same Q/K codes and ExpCast.
+    # V-Smooth against the unsmoothed baseline, both on the GPU (VC_MODE_NAIVE:
+    # V itself at one E4M3 scale per head) with the same Q/K codes and ExpCast,
+    # measured against exact fp64 attention. The values sit on 16 well separated
+    # centres (N(0, 6^2) per channel, spread 0.2), so each token is mostly its
+    # cluster's offset, which the block means of the sorted order carry exactly;
+    # the queries are scaled by 0.3 so that the probabilities' own FP8 error
+    # (equal in both runs) does not hide the value error. The oracle predicts a
+    # factor of about 2 on these inputs.
     cfg, Q, K, V = make("mid", B=1, H=2, S=2048)
-    g = gpu_pipeline(va, Q, K, V, 16, 4)
-    rows = np.arange(0, 2048, 8)
+    g = torch.Generator().manual_seed(5)
     for h in range(2):
-        q, k, v = head(Q, 0, h), head(K, 0, h), head(V, 0, h)
-        exact = O.exact_attention_rows(q, k, v, rows, SCALE)
-        e_gpu = rel_l2(g["o"][0, rows, h], exact)
-        qc, qs, kc, ks = O.quant_qk_head(q, k, np.arange(2048))
-        vn, _ = O.naive_v_e4m3(v)
-        naive = O.vc_attention_rows(qc, qs, kc, ks, vn, np.zeros((16, 128), np.float32), 2048, rows, SCALE)
-        print(f"head {h}: rel-L2 vs exact {e_gpu:.4f}, naive-V {rel_l2(naive, exact):.4f}")
-        assert e_gpu < 0.1
+        cent = torch.randn(16, 128, generator=g) * 6.0
+        lab = torch.randint(0, 16, (2048,), generator=g)
+        V[0, :, h] = (cent[lab] + 0.2 * torch.randn(2048, 128, generator=g)).to(torch.bfloat16)
+    Q = (Q.float() * 0.3).to(torch.bfloat16)
+    rows = np.arange(0, 2048, 8)
+    err = {}
+    for mode in ("vsmooth", "naive"):
+        gp = gpu_pipeline(va, Q, K, V, 16, 4, mode=mode, history=False)
+        assert gp["status"] == 0
+        num = den = 0.0
+        for h in range(2):
+            exact = O.exact_attention_rows(head(Q, 0, h), head(K, 0, h), head(V, 0, h), rows, SCALE)
+            num += float(((gp["o"][0, rows, h] - exact) ** 2).sum())
+            den += float((exact ** 2).sum())
+        err[mode] = math.sqrt(num / den)
+    print(f"rel-L2 vs exact fp64: V-Smooth {err['vsmooth']:.5f}, naive V {err['naive']:.5f}")
+    assert err["vsmooth"] < 0.02 and err["vsmooth"] < 0.7 * err["naive"], err
 
 
 def test_attention_exp2_comparison_kernel(va):
