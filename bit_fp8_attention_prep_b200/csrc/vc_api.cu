@@ -140,6 +140,18 @@ vc_status_t ensure_device() {
   return VC_OK;
 }
 
+// Number of SMs of the current device (cached per device; 148 if the query fails).
+int g_sms[64];
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (g_sms[dev] == 0) {
+    int n = 0;
+    g_sms[dev] = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0 ? n : 148;
+  }
+  return g_sms[dev];
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -243,6 +255,22 @@ static vc_status_t prepare_v_impl(const void* v, const vc_shape_t* shape, const 
   pl.hist = reinterpret_cast<int*>(ws + w.hist);
   pl.offs = reinterpret_cast<int*>(ws + w.offs);
   pl.amax = reinterpret_cast<unsigned int*>(ws + w.amax);
+  // BF16 V: the k-means distances run on the tensor cores, which read V through
+  // a 3D tensor map [B*S][H][128] (boxes of 128 tokens x 1 head x 64 dims)
+  pl.tc_assign = shape->dtype == VC_DTYPE_BF16;
+  pl.num_sms = device_sms();
+  if (pl.tc_assign && cfg->mode == VC_MODE_VSMOOTH) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(VC_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t dims[3] = {128, (cuuint64_t)shape->H, (cuuint64_t)shape->B * (cuuint64_t)shape->S};
+    const cuuint64_t strides[2] = {256, (cuuint64_t)shape->H * 256};
+    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(&pl.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(v), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(VC_ERR_CUDA, "cuTensorMapEncodeTiled (V for the k-means) failed (%d)", (int)r);
+  }
   int nl = 0;
   cudaError_t e =
       vc::launch_prepare_v(v, shape->dtype, pl, *out, assign_history, static_cast<cudaStream_t>(stream), &nl);

@@ -30,7 +30,10 @@ struct PrepPlan {
   uint8_t* assign2;            // [BH][S] labels of the odd passes
   int* hist;                   // [BH][nchunks][k]
   int* offs;                   // [BH][nchunks][k]
-  unsigned int* amax;          // [BH] fp32 bits
+  unsigned int* amax;          // [BH] fp32 bits ([BH][128] for the per-channel scale)
+  bool tc_assign;              // BF16 V: k-means distances on the tensor cores through tm_v
+  int num_sms;                 // streaming multiprocessors of the device (persistent grids)
+  CUtensorMap tm_v;            // V as [B*S][H][128] bf16, 128 x 1 x 64 boxes, 128-byte swizzle
 };
 
 cudaError_t prep_configure();
