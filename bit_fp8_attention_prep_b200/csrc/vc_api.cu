@@ -90,7 +90,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Workspace layout of vc_attn_prepare_v (every piece 256-B aligned).
 struct WsLayout {
-  size_t cent, sums, counts, assign, assign2, hist, offs, amax, total;
+  size_t cent, sums, counts, assign, assign2, hist, offs, amax, cops, work, total;
 };
 
 WsLayout ws_layout(const vc_shape_t* sh, const vc_vsmooth_cfg_t* cfg) {
@@ -108,6 +108,11 @@ WsLayout ws_layout(const vc_shape_t* sh, const vc_vsmooth_cfg_t* cfg) {
   w.offs = off;   off += align256(BH * nch * k * 4);
   // residual amax: one per (b, h), or one per (b, h, channel)
   w.amax = off;   off += align256(BH * 4 * (cfg->residual_fmt == VC_RESIDUAL_E4M3_PER_CHANNEL ? 128 : 1));
+  // the tensor-core k-means assignment (BF16 V): centroid operand blocks and the
+  // passes' work counters
+  const bool tc = cfg->mode == VC_MODE_VSMOOTH && sh->dtype == VC_DTYPE_BF16;
+  w.cops = off;   off += tc ? align256(BH * vc::tc_cops_bytes((int)k)) : 0;
+  w.work = off;   off += tc ? align256(sizeof(int) * (size_t)cfg->iters) : 0;
   w.total = off;
   return w;
 }
@@ -257,9 +262,11 @@ static vc_status_t prepare_v_impl(const void* v, const vc_shape_t* shape, const 
   pl.amax = reinterpret_cast<unsigned int*>(ws + w.amax);
   // BF16 V: the k-means distances run on the tensor cores, which read V through
   // a 3D tensor map [B*S][H][128] (boxes of 128 tokens x 1 head x 64 dims)
-  pl.tc_assign = shape->dtype == VC_DTYPE_BF16;
+  pl.tc_assign = shape->dtype == VC_DTYPE_BF16 && cfg->mode == VC_MODE_VSMOOTH;
   pl.num_sms = device_sms();
-  if (pl.tc_assign && cfg->mode == VC_MODE_VSMOOTH) {
+  pl.cops = ws + w.cops;
+  pl.work = reinterpret_cast<int*>(ws + w.work);
+  if (pl.tc_assign) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(VC_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     const cuuint64_t dims[3] = {128, (cuuint64_t)shape->H, (cuuint64_t)shape->B * (cuuint64_t)shape->S};

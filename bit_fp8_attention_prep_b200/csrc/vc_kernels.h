@@ -31,10 +31,16 @@ struct PrepPlan {
   int* hist;                   // [BH][nchunks][k]
   int* offs;                   // [BH][nchunks][k]
   unsigned int* amax;          // [BH] fp32 bits ([BH][128] for the per-channel scale)
+  uint8_t* cops;               // [BH] centroid operand blocks of the tensor-core assignment
+  int* work;                   // [iters] work counters of the tensor-core assignment passes
   bool tc_assign;              // BF16 V: k-means distances on the tensor cores through tm_v
   int num_sms;                 // streaming multiprocessors of the device (persistent grids)
   CUtensorMap tm_v;            // V as [B*S][H][128] bf16, 128 x 1 x 64 boxes, 128-byte swizzle
 };
+
+// Bytes of one (b, h) slice's centroid operand block of the tensor-core
+// k-means assignment for k clusters (k <= 16: 16 rows, else 32).
+constexpr size_t tc_cops_bytes(int k) { return k <= 16 ? 2 * 2 * 16 * 128 + 2 * 16 * 4 : 2 * 2 * 32 * 128 + 2 * 32 * 4; }
 
 cudaError_t prep_configure();
 // *nlaunch receives the number of kernels enqueued (memsets not counted).

@@ -332,36 +332,40 @@ constexpr size_t assign_smem() {
 }
 
 // --------------------------------------------------------------- k-means assign on the tensor cores
-// The assignment for BF16 V. A persistent CTA (10 warps, one per SM) takes a
-// contiguous range of the (b, h, chunk of kChunk tokens) work items and streams
-// their 128-token tiles through a deep pipeline, so that several tiles' loads
-// are in flight while earlier tiles are decided:
-//  - warp 8 loads each tile with TMA (two 128-byte-swizzled boxes of 64
-//    dimensions) into a ring of kTcStages stages;
-//  - warp 9 issues the tile's dot products with every centroid on the tensor
-//    cores, into one of four tensor-memory stages of 2 KC fp32 columns;
+// The assignment for BF16 V, in two kernels.
+// (1) kmeans_cops_kernel, before each pass: per (b, h) the centroid operand block
+//     of the pass: the hi and mid bf16 parts of every centroid as the MMA's B
+//     operand (two halves of 64 dimensions, rows 0..KC-1 hi, KC..2KC-1 mid, in
+//     the 128-byte-swizzled layout a 1024-byte-aligned copy reproduces), then
+//     |c|^2 (fp64 sum rounded once) and |c| for the KC centroids.
+// (2) kmeans_assign_tc_kernel: one persistent CTA (10 warps) per SM takes work
+//     items (b, h, chunk of kChunk tokens) from a global counter, so that CTAs
+//     whose tokens need the fallback below more often do not hold back the rest,
+//     and streams their 128-token tiles through a ring of stages:
+//  - warp 8 takes the items, writes each tile's descriptor next to its stage
+//    and loads the tile with TMA (two 128-byte-swizzled boxes of 64 dimensions)
+//    with the slice's centroid operand block (one bulk copy);
+//  - warp 9 issues the tile's dot products on the tensor cores into one of four
+//    tensor-memory stages of 2 KC fp32 columns;
 //  - warps 0-3 (even tiles) and 4-7 (odd tiles) take one token per thread:
 //    proxies, argmin, fallback, label, and in the last pass the cluster
 //    histogram of each chunk (zeroed by the launcher; one global atomic per
 //    cluster present in a warp's 32 tokens).
-// A range holds the items of at most a few (b, h) slices; at each new slice the
-// CTA rebuilds its centroid operands between two block-wide barriers.
 // Dots. A centroid c (fp32) is hi + mid + r with hi = bf16(c), mid = bf16(c - hi)
 // and |r_d| <= 2^-18 |c_d|, so x . c = x . hi + x . mid within 2^-18 |x| |c| (x
 // bf16; sum_d |x_d c_d| <= |x| |c|). One kind::f16 MMA chain (M = 128 tokens,
-// N = 2 KC: the hi parts, then the mid parts, K = 128 dimensions: eight
-// instructions a tile) gives both dots of every centroid in fp32; their sum is
-// the dot. Decision. g_c = |c|^2 - 2 x . c ranks the centroids as
-// |x - c|^2 = |x|^2 + g_c does. The tensor core's accumulation order and
-// rounding are not specified; measured on a B200 over mixture, outlier and
-// wide-exponent inputs, the error of its fp32 dot products stayed below 2^-20
-// of sum_d |x_d hi_d|. Each dot is allowed 2^-15 |x| |c| (the dropped part
-// 2^-18, the accumulation 2^-17: eight times the largest error measured, the
-// final add far less) and |c|^2 (an fp64 sum rounded once) with the final fma
-// 2^-19 |c|^2: with e_c = 2^-19 |c|^2 + 2^-14 |x| |c|, a centroid whose g_c - e_c
-// exceeds g_b + e_b, b the smallest proxy, is farther than b. Any other centroid
-// is a candidate. b and its candidates are then compared by the squared distance
-// sum_d (x_d - c_d)^2 in fp32 (all terms positive: the rounding of the
+// N = 2 KC, K = 128 dimensions: eight instructions a tile) gives both dots of
+// every centroid in fp32; their sum is the dot.
+// Decision. g_c = |c|^2 - 2 x . c ranks the centroids as |x - c|^2 = |x|^2 + g_c
+// does. The tensor core's accumulation order and rounding are not specified;
+// measured on a B200 over mixture, outlier and wide-exponent inputs, the error
+// of its fp32 dot products stayed below 2^-20 of sum_d |x_d hi_d|. Each dot is
+// allowed 2^-15 |x| |c| (the dropped part 2^-18, the accumulation 2^-17: eight
+// times the largest error measured, the final add far less) and |c|^2 with the
+// final fma 2^-19 |c|^2: with e_c = 2^-19 |c|^2 + 2^-14 |x| |c|, a centroid whose
+// g_c - e_c exceeds g_b + e_b, b the smallest proxy, is farther than b. Any other
+// centroid is a candidate. b and its candidates are then compared by the squared
+// distance sum_d (x_d - c_d)^2 in fp32 (all terms positive: the rounding of the
 // differences, squares and 128-term sum stays within 2^-16 of the distance
 // itself), and those still within that bound of the nearest once more in fp64
 // (differences exact, squares rounded at 2^-53), the lowest index winning ties:
@@ -371,27 +375,64 @@ constexpr int kTcTmaWarp = 8, kTcMmaWarp = 9;
 constexpr int kTcDStages = 4;                  // tensor-memory dot stages (two per token-warp group)
 constexpr uint32_t kTcStageCols = 64;          // tensor-memory columns per dot stage (N = 2 KC <= 64)
 constexpr uint32_t kTcTileBytes = kTile * 256; // 128 tokens x 128 bf16 (two 16 KB boxes)
-template <int KC> constexpr int tc_stages() { return KC == 32 ? 5 : 6; }   // tile ring depth (shared memory)
+constexpr int kTcTilesPerChunk = kChunk / kTile;
 
-template <int KC>
-struct __align__(1024) SmemAssignTc {
-  static constexpr int kStages = tc_stages<KC>();
-  uint8_t a[kStages][2][kTile * 128];  // [stage][64-dimension half] 128-B-swizzled rows of 64 bf16
-  uint8_t bsp[2][2 * KC * 128];      // [half] rows 0..KC-1: hi parts, KC..2KC-1: mid parts, same layout
-  float cf[KC][kD];                  // fp32 centroids (zero past k)
-  float cn[KC], cabs[KC];            // |c|^2 (fp64 sum rounded to fp32) and |c|
-  uint64_t a_full[kStages], a_empty[kStages], d_full[kTcDStages], d_empty[kTcDStages], drain;
-  uint32_t tmem_base;
-  int32_t abort_flag;                // a wait ran out: every role skips the remaining tiles
-};
+// Bytes of one slice's centroid operand block: [2 halves][2 KC rows][128 B], then
+// |c|^2 [KC] and |c| [KC] (fp32).
+template <int KC> __host__ __device__ constexpr uint32_t cops_bytes() { return 2 * 2 * KC * 128 + 2 * KC * 4; }
+template <int KC> __host__ __device__ constexpr int tc_stages() { return KC == 32 ? 4 : 5; }   // tile ring depth (shared memory)
 
 // Byte offset of dimension-half piece j (16 bytes, 8 dims) of row r in a
 // 128-byte-swizzled block of rows: rows of 128 B, the piece index XORed with r mod 8.
 __device__ __forceinline__ uint32_t sw128_off(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
 
-// Bounded spin on an mbarrier phase (1 s), for a whole warp; false (and the
-// CTA's abort flag set) when the time ran out or another role already gave up.
-// The waiting thread is suspended in the barrier unit (up to 20 us at a time), so
+template <int KC>
+__global__ void __launch_bounds__(128) kmeans_cops_kernel(int k, const float* __restrict__ cent,
+                                                          uint8_t* __restrict__ cops) {
+  __shared__ double wq[4][KC];
+  const int bh = blockIdx.x, d = threadIdx.x, lane = d & 31, warp = d >> 5;
+  uint8_t* blk = cops + (size_t)bh * cops_bytes<KC>();
+  const float* cg = cent + (size_t)bh * k * kD;
+#pragma unroll 4
+  for (int c = 0; c < KC; ++c) {
+    const float x = c < k ? cg[c * kD + d] : 0.0f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
+    uint8_t* half = blk + (d >> 6) * (2 * KC * 128);
+    *reinterpret_cast<__nv_bfloat16*>(half + sw128_off(c, (d & 63) >> 3) + (d & 7) * 2) = hi;
+    *reinterpret_cast<__nv_bfloat16*>(half + sw128_off(KC + c, (d & 63) >> 3) + (d & 7) * 2) = mid;
+    double q = (double)x * (double)x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    if (lane == 0) wq[warp][c] = q;
+  }
+  __syncthreads();
+  if (d < KC) {
+    const double q = (wq[0][d] + wq[1][d]) + (wq[2][d] + wq[3][d]);
+    float* nrm = reinterpret_cast<float*>(blk + 2 * 2 * KC * 128);
+    nrm[d] = __double2float_rn(q);
+    nrm[KC + d] = __double2float_rn(sqrt(q));
+  }
+}
+
+struct TcTile {
+  int bh, chunk, t, end;   // slice, chunk, tile of the chunk; end = 1 marks the end of the stream
+};
+
+template <int KC>
+struct __align__(1024) SmemAssignTc {
+  static constexpr int kStages = tc_stages<KC>();
+  uint8_t a[kStages][2][kTile * 128];      // [stage][64-dimension half] 128-B-swizzled rows of 64 bf16
+  uint8_t cop[kStages][cops_bytes<KC>() + 1024 - cops_bytes<KC>() % 1024];  // the tile's centroid operand block
+  TcTile desc[kStages];
+  uint64_t a_full[kStages], a_empty[kStages], d_full[kTcDStages], d_empty[kTcDStages], drain;
+  uint32_t tmem_base;
+  int32_t abort_flag;                      // a wait ran out: every role skips the remaining tiles
+};
+
+// Bounded wait on an mbarrier phase (1 s), for a whole warp; false (and the CTA's
+// abort flag set) when the time ran out or another role already gave up. The
+// waiting thread is suspended in the barrier unit (up to 20 us at a time), so
 // idle warps leave the issue slots to the working ones.
 template <class Smem>
 __device__ __forceinline__ bool tc_wait(Smem& s, uint64_t* bar, uint32_t parity) {
@@ -414,17 +455,19 @@ template <int KC>
 __global__ void __launch_bounds__(kTcThreads, 1) kmeans_assign_tc_kernel(const __grid_constant__ CUtensorMap tmV,
                                                                        int S, int H, int k, int nchunks, int BH,
                                                                        const float* __restrict__ cent,
+                                                                       const uint8_t* __restrict__ cops,
+                                                                       int* __restrict__ work,
                                                                        uint8_t* __restrict__ assign,
                                                                        int* __restrict__ hist,
                                                                        uint8_t* __restrict__ history) {
   static_assert(KC == 16 || KC == 32, "N of the dot MMA");
   using Smem = SmemAssignTc<KC>;
   constexpr int NS = Smem::kStages;
+  constexpr uint32_t kCopBytes = cops_bytes<KC>();
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long total = (long long)BH * nchunks;
-  const int w0 = (int)(total * blockIdx.x / gridDim.x), w1 = (int)(total * (blockIdx.x + 1) / gridDim.x);
+  const int total = BH * nchunks;
   constexpr uint32_t idesc = idesc_f32acc(kFmtBF16, kFmtBF16, 128, 2 * KC);
 
   if (tid == 0) {
@@ -449,239 +492,239 @@ __global__ void __launch_bounds__(kTcThreads, 1) kmeans_assign_tc_kernel(const _
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   const bool leader = elect_one();   // the issuing lane of the TMA and MMA warps
-  int gbase = 0;                     // tiles of this CTA before the current slice
-  static_assert(sizeof(s.bsp[0]) == 2 * KC * 64 * 2, "B operand: 2 KC rows of 64 bf16 per half");
-  for (int seg = w0; seg < w1;) {
-    const int bh = seg / nchunks, b = bh / H, h = bh % H;
-    const int c0 = seg % nchunks, c1 = min(nchunks, c0 + (w1 - seg));   // chunks [c0, c1) of slice bh
-    seg += c1 - c0;
-    const int ntiles = (min(S, c1 * kChunk) - c0 * kChunk + kTile - 1) / kTile;
-    // the slice's centroids: fp32 copy, |c|^2, the hi and mid bf16 parts in the
-    // MMA's B layout (the previous slice's MMAs have all completed: the token
-    // warps waited for every one of them before the barrier that ended it)
-    const float* cg = cent + (size_t)bh * k * kD;
-    for (int i = tid; i < KC * kD; i += kTcThreads) {
-      const int c = i / kD, d = i % kD;
-      const float x = c < k ? cg[c * kD + d] : 0.0f;
-      s.cf[c][d] = x;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-      const __nv_bfloat16 mid = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
-      *reinterpret_cast<__nv_bfloat16*>(&s.bsp[d >> 6][sw128_off(c, (d & 63) >> 3) + (d & 7) * 2]) = hi;
-      *reinterpret_cast<__nv_bfloat16*>(&s.bsp[d >> 6][sw128_off(KC + c, (d & 63) >> 3) + (d & 7) * 2]) = mid;
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    for (int c = warp; c < KC; c += kTcWarps) {  // |c|^2 in fp64, rounded once
-      double q = 0.0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const double x = (double)s.cf[c][lane + 32 * j];
-        q = fma(x, x, q);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-      if (lane == 0) {
-        s.cn[c] = __double2float_rn(q);
-        s.cabs[c] = __double2float_rn(sqrt(q));
-      }
-    }
-    __syncthreads();
+  int ntiles = 0;                    // tiles this CTA streamed (the TMA warp's count)
 
-    // tile t of the slice: chunk c0 + t / 8, rows from token t * 128 of chunk c0
-    if (warp == kTcTmaWarp) {
-      // ------------------------------------------------ TMA producer
-      for (int t = 0; t < ntiles && !*reinterpret_cast<volatile int32_t*>(&s.abort_flag); ++t) {
-        const int g = gbase + t, st = g % NS;
-        if (g >= NS && !tc_wait(s, &s.a_empty[st], ((g / NS) & 1) ^ 1)) break;
-        if (leader) {
+  if (warp == kTcTmaWarp) {
+    // ------------------------------------------------ work items, TMA producer
+    // tile g goes to stage g % NS; after the last item, two end tiles (one for
+    // each token-warp group) close the stream
+    int g = 0, ends = 0;
+    int item = 0, ntile_item = 0, ti = 0;
+    bool have = false;
+    while (ends < 2) {
+      if (*reinterpret_cast<volatile int32_t*>(&s.abort_flag)) break;
+      if (ends == 0 && (!have || ti == ntile_item)) {
+        int it = 0;
+        if (leader) it = atomicAdd(work, 1);
+        item = __shfl_sync(0xffffffffu, it, __ffs(__ballot_sync(0xffffffffu, leader)) - 1);
+        have = item < total;
+        if (have) {
+          const int chunk = item % nchunks;
+          ntile_item = (min(kChunk, S - chunk * kChunk) + kTile - 1) / kTile;
+          ti = 0;
+        }
+      }
+      const int st = g % NS;
+      if (g >= NS && !tc_wait(s, &s.a_empty[st], ((g / NS) & 1) ^ 1)) break;
+      if (leader) {
+        TcTile d;
+        if (have) {
+          d.bh = item / nchunks;
+          d.chunk = item % nchunks;
+          d.t = ti;
+          d.end = 0;
+          s.desc[st] = d;
           if (g == 0) prefetch_tmap(&tmV);
-          const int z = b * S + c0 * kChunk + t * kTile;   // rows past the tensor read as zeros
-          mbar_arrive_expect_tx(&s.a_full[st], kTcTileBytes);
+          const int b = d.bh / H, h = d.bh % H;
+          const int z = b * S + d.chunk * kChunk + ti * kTile;   // rows past the tensor read as zeros
+          mbar_arrive_expect_tx(&s.a_full[st], kTcTileBytes + kCopBytes);
           tma_load_3d(s.a[st][0], &tmV, &s.a_full[st], 0, h, z);
           tma_load_3d(s.a[st][1], &tmV, &s.a_full[st], 64, h, z);
+          bulk_load(s.cop[st], cops + (size_t)d.bh * kCopBytes, kCopBytes, &s.a_full[st]);
+        } else {
+          d.bh = d.chunk = d.t = 0;
+          d.end = 1;
+          s.desc[st] = d;
+          mbar_arrive(&s.a_full[st]);
         }
-        __syncwarp();
       }
-    } else if (warp == kTcMmaWarp) {
-      // ------------------------------------------------ dot products
-      for (int t = 0; t < ntiles && !*reinterpret_cast<volatile int32_t*>(&s.abort_flag); ++t) {
-        const int g = gbase + t, st = g % NS, ds = g % kTcDStages;
-        if (!tc_wait(s, &s.a_full[st], (g / NS) & 1)) break;
-        if (g >= kTcDStages && !tc_wait(s, &s.d_empty[ds], ((g / kTcDStages) & 1) ^ 1)) break;
-        tc_fence_after();
-        if (leader) {
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const uint64_t da = sdesc_k_sw128(smem_u32(s.a[st][half]));
-            const uint64_t db = sdesc_k_sw128(smem_u32(s.bsp[half]));
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_f16_ss(tmem + ds * kTcStageCols, da + 2 * kk, db + 2 * kk, idesc, (half | kk) != 0);
-          }
-          umma_commit(&s.d_full[ds]);
-          umma_commit(&s.a_empty[st]);
-        }
-        __syncwarp();
+      __syncwarp();
+      if (have) {
+        ++ti;
+        ++ntiles;
+      } else {
+        ++ends;
       }
-    } else {
-      // ------------------------------------------------ one token per thread
-      // group grp = warp / 4 takes the tiles g with g % 2 == grp
-      const int grp = warp >> 2;
-      const int r = tid & 127;                             // row of the tile, tensor-memory lane
-      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-      const int t0 = ((grp - gbase) % 2 + 2) % 2;          // first tile of the slice with g % 2 == grp
-#pragma unroll 1
-      for (int t = t0; t < ntiles && !*reinterpret_cast<volatile int32_t*>(&s.abort_flag); t += 2) {
-        const int g = gbase + t, st = g % NS, ds = g % kTcDStages;
-        // the tile in shared memory (for |x|^2 and the fallback) and its dots
-        if (!tc_wait(s, &s.a_full[st], (g / NS) & 1)) break;
-        if (!tc_wait(s, &s.d_full[ds], (g / kTcDStages) & 1)) break;
-        tc_fence_after();
-        uint32_t dr[32], dm[32];   // x . hi and x . mid of each centroid
-        tmem_ld32(tmem + lane_base + ds * kTcStageCols, dr);
-        tmem_ld32(tmem + lane_base + ds * kTcStageCols + KC, dm);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.d_empty[ds]);
-        const int chunk = c0 + t / (kChunk / kTile);
-        const int p = (t % (kChunk / kTile)) * kTile + r;  // token of the chunk
-        const int ntok = min(kChunk, S - chunk * kChunk);
-        const uint8_t* const arow0 = s.a[st][0];
-        const uint8_t* const arow1 = s.a[st][1];
-        auto piece = [&](int j, float* f) {                // dims 8j .. 8j+7 of row r
-          const uint8_t* base = j < 8 ? arow0 : arow1;
-          unpack8<__nv_bfloat16>(*reinterpret_cast<const uint4*>(base + sw128_off(r, j & 7)), f);
-        };
-        float xx = 0.0f;
-#pragma unroll 4
-        for (int j = 0; j < 16; ++j) {
-          float f[8];
-          piece(j, f);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) xx = fmaf(f[e], f[e], xx);
-        }
-        const float xabs = sqrtf(xx);
-        int best = 0;
-        float gb = 0.0f;
-        float gv[KC];
-#pragma unroll
-        for (int c = 0; c < KC; ++c) {
-          gv[c] = fmaf(-2.0f, __uint_as_float(dr[c]) + __uint_as_float(dm[c]), s.cn[c]);
-          if (c < k && (c == 0 || gv[c] < gb)) {
-            gb = gv[c];
-            best = c;
-          }
-        }
-        const float lim = gb + fmaf(0x1p-19f, s.cn[best], 0x1p-14f * xabs * s.cabs[best]);
-        uint32_t cand = 0u;
-#pragma unroll
-        for (int c = 0; c < KC; ++c) {
-          const float e = fmaf(0x1p-19f, s.cn[c], 0x1p-14f * xabs * s.cabs[c]);
-          if (c < k && c != best && !(gv[c] - e > lim)) cand |= 1u << c;
-        }
-        if (cand != 0u) {
-          // direct squared distances of the best proxy and its candidates: fp32
-          // first (even and odd dimensions in the two halves of a packed
-          // accumulator), fp64 for those the fp32 bound cannot separate
-          cand |= 1u << best;
-          float dd[KC];
-          float dmin = __int_as_float(0x7f800000);
-          int bmin = -1;
-#pragma unroll 1
-          for (uint32_t m = cand; m != 0u; m &= m - 1u) {
-            const int c = __ffs(m) - 1;
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 2
-            for (int j = 0; j < 16; ++j) {
-              float f[8];
-              piece(j, f);
-              const float4* cc = reinterpret_cast<const float4*>(&s.cf[c][8 * j]);
-              const float4 p0 = cc[0], p1 = cc[1];
-              const float2 d0 = __fadd2_rn(make_float2(f[0], f[1]), make_float2(-p0.x, -p0.y));
-              const float2 d1 = __fadd2_rn(make_float2(f[2], f[3]), make_float2(-p0.z, -p0.w));
-              const float2 d2 = __fadd2_rn(make_float2(f[4], f[5]), make_float2(-p1.x, -p1.y));
-              const float2 d3 = __fadd2_rn(make_float2(f[6], f[7]), make_float2(-p1.z, -p1.w));
-              acc = __ffma2_rn(d0, d0, acc);
-              acc = __ffma2_rn(d1, d1, acc);
-              acc = __ffma2_rn(d2, d2, acc);
-              acc = __ffma2_rn(d3, d3, acc);
-            }
-            const float dc = acc.x + acc.y;
-#pragma unroll
-            for (int q = 0; q < KC; ++q)
-              if (q == c) dd[q] = dc;
-            if (bmin < 0 || dc < dmin) {
-              dmin = dc;
-              bmin = c;
-            }
-          }
-          uint32_t close = 0u;   // within the fp32 bound of the nearest
-#pragma unroll
-          for (int q = 0; q < KC; ++q)
-            if (((cand >> q) & 1u) && q != bmin && !(dd[q] - 0x1p-16f * dd[q] > dmin + 0x1p-16f * dmin))
-              close |= 1u << q;
-          best = bmin;
-          if (close != 0u) {
-            close |= 1u << bmin;
-            double bd = 0.0;
-            best = -1;
-#pragma unroll 1
-            for (; close != 0u; close &= close - 1u) {
-              const int c = __ffs(close) - 1;
-              double dist = 0.0;
-#pragma unroll 1
-              for (int j = 0; j < 16; ++j) {
-                float f[8];
-                piece(j, f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  const double df = (double)f[e] - (double)s.cf[c][8 * j + e];
-                  dist = fma(df, df, dist);
-                }
-              }
-              if (best < 0 || dist < bd) {
-                bd = dist;
-                best = c;
-              }
-            }
-          }
-        }
-        const bool valid = p < ntok;
-        if (valid) {
-          const size_t o = (size_t)bh * S + (size_t)chunk * kChunk + p;
-          assign[o] = (uint8_t)best;
-          if (history) history[o] = (uint8_t)best;
-        }
-        if (hist != nullptr) {
-          // the warp's tokens of each cluster, added once by the lowest such lane
-          const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-          const uint32_t same = __match_any_sync(0xffffffffu, valid ? best : -1) & vmask;
-          if (valid && (same & ((1u << lane) - 1u)) == 0u)
-            atomicAdd(&hist[((size_t)bh * nchunks + chunk) * k + best], __popc(same));
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.a_empty[st]);
-      }
+      ++g;
     }
-    gbase += ntiles;
-    __syncthreads();
-  }
-  // every MMA (and the barrier arrivals it was to make) and every copy is
-  // complete before the CTA exits; after an abort, copies may still land
-  if (warp == kTcMmaWarp) {
+    // copies still in flight land before the CTA exits
+    for (int i = max(0, g - NS); i < g; ++i) mbar_wait(&s.a_full[i % NS], (i / NS) & 1, 100000000ull, nullptr);
+  } else if (warp == kTcMmaWarp) {
+    // ------------------------------------------------ dot products
+    for (int g = 0;; ++g) {
+      const int st = g % NS, ds = g % kTcDStages;
+      if (!tc_wait(s, &s.a_full[st], (g / NS) & 1)) break;
+      if (s.desc[st].end) break;
+      if (g >= kTcDStages && !tc_wait(s, &s.d_empty[ds], ((g / kTcDStages) & 1) ^ 1)) break;
+      tc_fence_after();
+      if (leader) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint64_t da = sdesc_k_sw128(smem_u32(s.a[st][half]));
+          const uint64_t db = sdesc_k_sw128(smem_u32(s.cop[st] + half * (2 * KC * 128)));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f16_ss(tmem + ds * kTcStageCols, da + 2 * kk, db + 2 * kk, idesc, (half | kk) != 0);
+        }
+        umma_commit(&s.d_full[ds]);
+        umma_commit(&s.a_empty[st]);
+      }
+      __syncwarp();
+    }
     if (leader) umma_commit(&s.drain);
     __syncwarp();
     mbar_wait(&s.drain, 0, 100000000ull, nullptr);
+  } else {
+    // ------------------------------------------------ one token per thread
+    // group grp = warp / 4 takes the tiles g with g % 2 == grp
+    const int grp = warp >> 2;
+    const int r = tid & 127;                             // row of the tile, tensor-memory lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+#pragma unroll 1
+    for (int g = grp;; g += 2) {
+      const int st = g % NS, ds = g % kTcDStages;
+      if (!tc_wait(s, &s.a_full[st], (g / NS) & 1)) break;
+      const TcTile d = s.desc[st];
+      if (d.end) break;
+      if (!tc_wait(s, &s.d_full[ds], (g / kTcDStages) & 1)) break;
+      tc_fence_after();
+      uint32_t dr[32], dm[32];   // x . hi and x . mid of each centroid
+      tmem_ld32(tmem + lane_base + ds * kTcStageCols, dr);
+      tmem_ld32(tmem + lane_base + ds * kTcStageCols + KC, dm);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.d_empty[ds]);
+      const int bh = d.bh, chunk = d.chunk;
+      const int p = d.t * kTile + r;                       // token of the chunk
+      const int ntok = min(kChunk, S - chunk * kChunk);
+      const float* const nrm = reinterpret_cast<const float*>(s.cop[st] + 2 * 2 * KC * 128);  // |c|^2, |c|
+      const float* const cg = cent + (size_t)bh * k * kD;
+      const uint8_t* const arow0 = s.a[st][0];
+      const uint8_t* const arow1 = s.a[st][1];
+      auto piece = [&](int j, float* f) {                // dims 8j .. 8j+7 of row r
+        const uint8_t* base = j < 8 ? arow0 : arow1;
+        unpack8<__nv_bfloat16>(*reinterpret_cast<const uint4*>(base + sw128_off(r, j & 7)), f);
+      };
+      float2 xx2 = make_float2(0.f, 0.f);
+#pragma unroll 4
+      for (int j = 0; j < 16; ++j) {
+        float f[8];
+        piece(j, f);
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) xx2 = __ffma2_rn(make_float2(f[e], f[e + 1]), make_float2(f[e], f[e + 1]), xx2);
+      }
+      const float xabs = sqrtf(xx2.x + xx2.y);
+      int best = 0;
+      float gb = 0.0f;
+      float gv[KC];
+#pragma unroll
+      for (int c = 0; c < KC; ++c) {
+        gv[c] = fmaf(-2.0f, __uint_as_float(dr[c]) + __uint_as_float(dm[c]), nrm[c]);
+        if (c < k && (c == 0 || gv[c] < gb)) {
+          gb = gv[c];
+          best = c;
+        }
+      }
+      const float xs = 0x1p-14f * xabs;
+      const float lim = gb + fmaf(0x1p-19f, nrm[best], xs * nrm[KC + best]);
+      uint32_t cand = 0u;
+#pragma unroll
+      for (int c = 0; c < KC; ++c) {
+        const float e = fmaf(0x1p-19f, nrm[c], xs * nrm[KC + c]);
+        if (c < k && c != best && !(gv[c] - e > lim)) cand |= 1u << c;
+      }
+      if (cand != 0u) {
+        // direct squared distances of the best proxy and its candidates: fp32
+        // first (even and odd dimensions in the two halves of a packed
+        // accumulator), fp64 for those the fp32 bound cannot separate
+        cand |= 1u << best;
+        float dd[KC];
+        float dmin = __int_as_float(0x7f800000);
+        int bmin = -1;
+#pragma unroll 1
+        for (uint32_t m = cand; m != 0u; m &= m - 1u) {
+          const int c = __ffs(m) - 1;
+          float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 2
+          for (int j = 0; j < 16; ++j) {
+            float f[8];
+            piece(j, f);
+            const float4* cc = reinterpret_cast<const float4*>(cg + c * kD + 8 * j);
+            const float4 p0 = __ldg(cc), p1 = __ldg(cc + 1);
+            const float2 d0 = __fadd2_rn(make_float2(f[0], f[1]), make_float2(-p0.x, -p0.y));
+            const float2 d1 = __fadd2_rn(make_float2(f[2], f[3]), make_float2(-p0.z, -p0.w));
+            const float2 d2 = __fadd2_rn(make_float2(f[4], f[5]), make_float2(-p1.x, -p1.y));
+            const float2 d3 = __fadd2_rn(make_float2(f[6], f[7]), make_float2(-p1.z, -p1.w));
+            acc = __ffma2_rn(d0, d0, acc);
+            acc = __ffma2_rn(d1, d1, acc);
+            acc = __ffma2_rn(d2, d2, acc);
+            acc = __ffma2_rn(d3, d3, acc);
+          }
+          const float dc = acc.x + acc.y;
+#pragma unroll
+          for (int q = 0; q < KC; ++q)
+            if (q == c) dd[q] = dc;
+          if (bmin < 0 || dc < dmin) {
+            dmin = dc;
+            bmin = c;
+          }
+        }
+        uint32_t close = 0u;   // within the fp32 bound of the nearest
+#pragma unroll
+        for (int q = 0; q < KC; ++q)
+          if (((cand >> q) & 1u) && q != bmin && !(dd[q] - 0x1p-16f * dd[q] > dmin + 0x1p-16f * dmin))
+            close |= 1u << q;
+        best = bmin;
+        if (close != 0u) {
+          close |= 1u << bmin;
+          double bd = 0.0;
+          best = -1;
+#pragma unroll 1
+          for (; close != 0u; close &= close - 1u) {
+            const int c = __ffs(close) - 1;
+            double dist = 0.0;
+#pragma unroll 1
+            for (int j = 0; j < 16; ++j) {
+              float f[8];
+              piece(j, f);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const double df = (double)f[e] - (double)__ldg(cg + c * kD + 8 * j + e);
+                dist = fma(df, df, dist);
+              }
+            }
+            if (best < 0 || dist < bd) {
+              bd = dist;
+              best = c;
+            }
+          }
+        }
+      }
+      const bool valid = p < ntok;
+      if (valid) {
+        const size_t o = (size_t)bh * S + (size_t)chunk * kChunk + p;
+        assign[o] = (uint8_t)best;
+        if (history) history[o] = (uint8_t)best;
+      }
+      if (hist != nullptr) {
+        // the warp's tokens of each cluster, added once by the lowest such lane
+        const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+        const uint32_t same = __match_any_sync(0xffffffffu, valid ? best : -1) & vmask;
+        if (valid && (same & ((1u << lane) - 1u)) == 0u)
+          atomicAdd(&hist[((size_t)bh * nchunks + chunk) * k + best], __popc(same));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.a_empty[st]);
+    }
   }
-  if (warp == kTcTmaWarp && *reinterpret_cast<volatile int32_t*>(&s.abort_flag))
-    for (int g = max(0, gbase - NS); g < gbase; ++g) mbar_wait(&s.a_full[g % NS], (g / NS) & 1, 100000000ull, nullptr);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTcDStages * kTcStageCols);
   }
+  (void)ntiles;
 }
 
 template <int KC>
@@ -822,38 +865,47 @@ __global__ void __launch_bounds__(kTile) kmeans_sums_kernel(const T* __restrict_
 }
 
 template <typename T, int KC>
-static void launch_kmeans_pass(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, int it, bool last,
-                               uint8_t* hist_t) {
+// Returns the number of kernels it enqueued.
+static int launch_kmeans_pass(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, int it, bool last,
+                              uint8_t* hist_t) {
   uint8_t* lab = it & 1 ? pl.assign2 : pl.assign;
   bool done = false;
+  int n = 0;
   if constexpr (std::is_same<T, __nv_bfloat16>::value && KC >= 16) {
     if (pl.tc_assign) {
-      // persistent: one CTA per SM over all (b, h, chunk) items
+      // the pass's centroid operands, then one persistent CTA per SM over all
+      // (b, h, chunk) items, taken from the pass's work counter
       const int items = pl.nchunks * pl.B * pl.H;
       const int ctas = std::max(1, std::min(items, pl.num_sms));
       if (last) cudaMemsetAsync(pl.hist, 0, sizeof(int) * (size_t)items * pl.k, st);  // summed by atomics
+      kmeans_cops_kernel<KC><<<pl.B * pl.H, 128, 0, st>>>(pl.k, pl.cent, pl.cops);
       kmeans_assign_tc_kernel<KC><<<ctas, kTcThreads, assign_tc_smem<KC>(), st>>>(
-          pl.tm_v, pl.S, pl.H, pl.k, pl.nchunks, pl.B * pl.H, pl.cent, lab, last ? pl.hist : nullptr, hist_t);
+          pl.tm_v, pl.S, pl.H, pl.k, pl.nchunks, pl.B * pl.H, pl.cent, pl.cops, pl.work + it, lab,
+          last ? pl.hist : nullptr, hist_t);
       done = true;
+      n += 2;
     }
   }
-  if (!done)
+  if (!done) {
     kmeans_assign_kernel<T, KC><<<grid, kTile, assign_smem<KC>(), st>>>(v, pl.S, pl.H, pl.k, pl.cent, lab,
                                                                          last ? pl.hist : nullptr, hist_t);
-  if (!last)
+    ++n;
+  }
+  if (!last) {
     kmeans_sums_kernel<T, KC><<<grid, kTile, 0, st>>>(v, pl.S, pl.H, pl.k, it > 0, lab, it & 1 ? pl.assign : pl.assign2,
                                                       pl.sums, pl.counts);
+    ++n;
+  }
+  return n;
 }
 
 template <typename T>
-static void launch_kmeans_pass_k(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, int it, bool last,
-                                 uint8_t* hist_t) {
+static int launch_kmeans_pass_k(dim3 grid, cudaStream_t st, const T* v, const PrepPlan& pl, int it, bool last,
+                                uint8_t* hist_t) {
   if (pl.k <= 8 && !(std::is_same<T, __nv_bfloat16>::value && pl.tc_assign))
-    launch_kmeans_pass<T, 8>(grid, st, v, pl, it, last, hist_t);
-  else if (pl.k <= 16)
-    launch_kmeans_pass<T, 16>(grid, st, v, pl, it, last, hist_t);
-  else
-    launch_kmeans_pass<T, 32>(grid, st, v, pl, it, last, hist_t);
+    return launch_kmeans_pass<T, 8>(grid, st, v, pl, it, last, hist_t);
+  if (pl.k <= 16) return launch_kmeans_pass<T, 16>(grid, st, v, pl, it, last, hist_t);
+  return launch_kmeans_pass<T, 32>(grid, st, v, pl, it, last, hist_t);
 }
 
 // --------------------------------------------------------------- centroid update
@@ -1692,6 +1744,7 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
   if (pl.mode == VC_MODE_VSMOOTH) {
     if ((e = cudaMemsetAsync(pl.sums, 0, sizeof(unsigned long long) * BH * k * kD, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(pl.counts, 0, sizeof(int) * BH * k, st)) != cudaSuccess) return e;
+    if (pl.tc_assign && (e = cudaMemsetAsync(pl.work, 0, sizeof(int) * pl.iters, st)) != cudaSuccess) return e;
     kmeans_init_kernel<T><<<BH, 128, 0, st>>>(v, S, H, k, pl.seed, pl.bh_base, pl.cent);
     ++n;
     const dim3 grid(pl.nchunks, BH);
@@ -1700,11 +1753,9 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
     for (int it = 0; it < pl.iters; ++it) {
       uint8_t* hist_t = history ? history + (size_t)it * BH * S : nullptr;
       const bool last = it + 1 == pl.iters;
-      launch_kmeans_pass_k<T>(grid, st, v, pl, it, last, hist_t);
+      n += launch_kmeans_pass_k<T>(grid, st, v, pl, it, last, hist_t);
       if (!last) {
         kmeans_update_kernel<<<BH, 128, 0, st>>>(k, pl.cent, pl.sums, pl.counts);
-        n += 3;
-      } else {
         ++n;
       }
     }
@@ -1834,6 +1885,7 @@ cudaError_t prep_configure() {
   for (const auto& a : assign_fns)
     if ((e = cudaFuncSetAttribute(a.f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)a.bytes)) != cudaSuccess)
       return e;
+  static_assert(assign_tc_smem<16>() <= 227 * 1024 && assign_tc_smem<32>() <= 227 * 1024, "shared memory per CTA");
   if ((e = cudaFuncSetAttribute(kmeans_assign_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)assign_tc_smem<16>())) != cudaSuccess)
     return e;
