@@ -1275,57 +1275,119 @@ __device__ __forceinline__ int mx_exponent(float amax) {
   return max(-127, (bits & 0x7FFFFFu) <= 0x400000u ? E - 2 : E - 1);
 }
 
+// One CTA (8 warps) = one 128-token block of permuted positions, loaded as in
+// residual_e4m3_kernel (warp w: rows 16w .. 16w+15, two rows per load; lane l
+// owns channels 8(l%16) .. 8(l%16)+7). A group of 32 tokens is warps 2g and 2g+1:
+// each lane takes the amax of its channels over its rows, the two half warps and
+// then the two warps of the group merge theirs through shared memory. The codes go
+// to a shared tile [token][channel] (one code per byte) and leave transposed as
+// in residual_e4m3_kernel (4 x 4 byte blocks and byte permutes), then packed two
+// tokens a byte.
 template <typename T>
-__global__ void __launch_bounds__(128) residual_mxfp4_kernel(const T* __restrict__ v, int S, int H, int S_pad,
+__global__ void __launch_bounds__(256) residual_mxfp4_kernel(const T* __restrict__ v, int S, int H, int S_pad,
                                                              const int32_t* __restrict__ perm,
                                                              const float* __restrict__ mu,
                                                              uint8_t* __restrict__ codes,
                                                              uint32_t* __restrict__ exps, float* __restrict__ s_v) {
-  extern __shared__ __align__(16) float rt[];  // [128 channels][129]
-  __shared__ float smu[kD];
+  __shared__ __align__(16) uint8_t ct[kBlock * kResStride];
+  __shared__ float wmx[8][kD];   // per warp: the amax of each channel over its 16 rows
   const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x, nb = gridDim.x;
-  const int t = threadIdx.x;
-  if (blk == 0 && t == 0) s_v[bh] = 1.0f;   // no per-head scale
-  smu[t] = mu[((size_t)bh * nb + blk) * kD + t];
-  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int half = lane >> 4, c = lane & 15;
+  if (blk == 0 && threadIdx.x == 0) s_v[bh] = 1.0f;   // no per-head scale
+  float m8[8];
   {
-    const int p = blk * kBlock + t;  // thread t: permuted row t
-    if (p < S) {
-      const T* row = v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD;
-#pragma unroll 4
-      for (int c = 0; c < 16; ++c) {
-        float f[8];
-        unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), f);
+    const float4* mp = reinterpret_cast<const float4*>(mu + ((size_t)bh * nb + blk) * kD + c * 8);
+    const float4 m0 = mp[0], m1 = mp[1];
+    m8[0] = m0.x; m8[1] = m0.y; m8[2] = m0.z; m8[3] = m0.w;
+    m8[4] = m1.x; m8[5] = m1.y; m8[6] = m1.z; m8[7] = m1.w;
+  }
+  int src[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) rt[(c * 8 + e) * 129 + t] = __fsub_rn(f[e], smu[c * 8 + e]);
-      }
-    } else {
-      for (int d = 0; d < kD; ++d) rt[d * 129 + t] = 0.0f;
+  for (int i = 0; i < 8; ++i) {
+    const int p = blk * kBlock + warp * 16 + 2 * i + half;
+    src[i] = p < S ? perm[(size_t)bh * S + p] : -1;
+  }
+  uint4 xs[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    xs[i] = src[i] >= 0 ? *reinterpret_cast<const uint4*>(v + (((size_t)b * S + src[i]) * H + h) * kD + c * 8)
+                        : make_uint4(0u, 0u, 0u, 0u);
+  // residuals (padding rows 0) and their per-channel amax over this lane's rows
+  float rr[8][8], mx[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mx[e] = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float f[8];
+    unpack8<T>(xs[i], f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      rr[i][e] = src[i] >= 0 ? __fsub_rn(f[e], m8[e]) : 0.0f;
+      mx[e] = fmaxf(mx[e], fabsf(rr[i][e]));
     }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 16));
+  if (half == 0) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) wmx[warp][c * 8 + e] = mx[e];
   }
   __syncthreads();
-  const int d = t;  // thread t: channel t
-  const float* rr = rt + d * 129;
-  uint8_t* crow = codes + ((size_t)bh * kD + d) * (S_pad / 2) + (size_t)blk * (kBlock / 2);
+  // this group's exponents (group g = warp / 2) and the codes of this lane's values
+  const int g = warp >> 1;
+  float sc[8];
   uint32_t ew = 0u;
-#pragma unroll 1
-  for (int gi = 0; gi < kBlock / kMxGroup; ++gi) {
-    float gmax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kMxGroup; ++i) gmax = fmaxf(gmax, fabsf(rr[gi * kMxGroup + i]));
-    const int e = mx_exponent(gmax);
-    const float sc = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, normal for e in [-127, 126]
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-    for (int i = 0; i < kMxGroup; i += 2) {
-      const uint32_t byte =
-          cvt_e2m1x2(__fmul_rn(rr[gi * kMxGroup + i], sc), __fmul_rn(rr[gi * kMxGroup + i + 1], sc));
-      w[i >> 3] |= byte << (8 * ((i >> 1) & 3));
-    }
-    *reinterpret_cast<uint4*>(crow + gi * (kMxGroup / 2)) = make_uint4(w[0], w[1], w[2], w[3]);
-    ew |= (uint32_t)(e + 127) << (8 * gi);
+  for (int e = 0; e < 8; ++e) {
+    const int ex = mx_exponent(fmaxf(wmx[2 * g][c * 8 + e], wmx[2 * g + 1][c * 8 + e]));
+    sc[e] = __uint_as_float((uint32_t)(127 - ex) << 23);   // 2^-ex, normal for ex in [-127, 126]
+    (void)ew;
   }
-  exps[((size_t)bh * nb + blk) * kD + d] = ew;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = warp * 16 + 2 * i + half;
+    uint32_t w0 = 0u, w1 = 0u;   // one code per byte, channels c*8 .. c*8+7
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      w0 |= (uint32_t)(cvt_e2m1x2(__fmul_rn(rr[i][e], sc[e]), 0.0f) & 0xFu) << (8 * e);
+      w1 |= (uint32_t)(cvt_e2m1x2(__fmul_rn(rr[i][4 + e], sc[4 + e]), 0.0f) & 0xFu) << (8 * e);
+    }
+    *reinterpret_cast<uint2*>(ct + r * kResStride + c * 8) = make_uint2(w0, w1);
+  }
+  // the block's exponent bytes: channel d, groups 0..3 in one word
+  if (threadIdx.x < kD) {
+    const int d = threadIdx.x;
+    uint32_t w = 0u;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      w |= (uint32_t)(mx_exponent(fmaxf(wmx[2 * q][d], wmx[2 * q + 1][d])) + 127) << (8 * q);
+    exps[((size_t)bh * nb + blk) * kD + d] = w;
+  }
+  __syncthreads();
+  uint8_t* const out = codes + (size_t)bh * kD * (S_pad / 2) + (size_t)blk * (kBlock / 2);
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    // a 4 x 4 block of codes: channels 4cg .. 4cg+3 of tokens 4tq .. 4tq+3
+    const int combo = warp * 4 + it;
+    const int cg = 8 * (combo & 3) + (lane & 7), tq = 4 * (combo >> 2) + (lane >> 3);
+    const uint8_t* sp = ct + (4 * tq) * kResStride + 4 * cg;
+    const uint32_t r0 = *reinterpret_cast<const uint32_t*>(sp);
+    const uint32_t r1 = *reinterpret_cast<const uint32_t*>(sp + kResStride);
+    const uint32_t r2 = *reinterpret_cast<const uint32_t*>(sp + 2 * kResStride);
+    const uint32_t r3 = *reinterpret_cast<const uint32_t*>(sp + 3 * kResStride);
+    const uint32_t lo01 = __byte_perm(r0, r1, 0x5140), hi01 = __byte_perm(r0, r1, 0x7362);
+    const uint32_t lo23 = __byte_perm(r2, r3, 0x5140), hi23 = __byte_perm(r2, r3, 0x7362);
+    // channel 4cg + q: its 4 tokens' codes, one per byte, then two per byte
+    const uint32_t ch4[4] = {__byte_perm(lo01, lo23, 0x5410), __byte_perm(lo01, lo23, 0x7632),
+                             __byte_perm(hi01, hi23, 0x5410), __byte_perm(hi01, hi23, 0x7632)};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t w = ch4[q];
+      const uint32_t packed = (w & 0xFu) | ((w >> 4) & 0xF0u) | (((w >> 16) & 0xFu) << 8) | ((w >> 12) & 0xF000u);
+      *reinterpret_cast<uint16_t*>(out + (size_t)(4 * cg + q) * (S_pad / 2) + 2 * tq) = (uint16_t)packed;
+    }
+  }
 }
 
 // --------------------------------------------------------------- token sums (K smoothing)
@@ -1780,8 +1842,8 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
     residual_e4m3_kernel<T, true><<<gb, 256, 0, st>>>(v, S, H, pl.S_pad, out.perm, out.mu, pl.amax,
                                                       out.v_codes, out.s_v);
   } else if (pl.fmt == VC_RESIDUAL_MXFP4) {
-    residual_mxfp4_kernel<T><<<gb, 128, kD * 129 * sizeof(float), st>>>(
-        v, S, H, pl.S_pad, out.perm, out.mu, out.v_codes, reinterpret_cast<uint32_t*>(out.v_scales), out.s_v);
+    residual_mxfp4_kernel<T><<<gb, 256, 0, st>>>(v, S, H, pl.S_pad, out.perm, out.mu, out.v_codes,
+                                                 reinterpret_cast<uint32_t*>(out.v_scales), out.s_v);
   } else {
     residual_nvfp4_kernel<T><<<gb, 128, kD * 129 * sizeof(float), st>>>(v, S, H, pl.S_pad, out.perm, out.mu,
                                                                          pl.amax, out.v_codes, out.v_scales,
@@ -1892,8 +1954,7 @@ cudaError_t prep_configure() {
   if ((e = cudaFuncSetAttribute(kmeans_assign_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)assign_tc_smem<32>())) != cudaSuccess)
     return e;
-  for (auto f : {(const void*)residual_nvfp4_kernel<__nv_bfloat16>, (const void*)residual_nvfp4_kernel<__half>,
-                 (const void*)residual_mxfp4_kernel<__nv_bfloat16>, (const void*)residual_mxfp4_kernel<__half>})
+  for (auto f : {(const void*)residual_nvfp4_kernel<__nv_bfloat16>, (const void*)residual_nvfp4_kernel<__half>})
     if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kD * 129 * 4))) !=
         cudaSuccess)
       return e;
