@@ -1198,61 +1198,110 @@ __global__ void __launch_bounds__(256) residual_e4m3_kernel(const T* __restrict_
 // --------------------------------------------------------------- residual NVFP4
 // Global scale g = amax / (448 * 6) per (b, h); per channel and group of 16
 // consecutive permuted tokens an E4M3 scale s = E4M3(fl32(fl32(gmax/6)/g)), and
-// E2M1 codes of r / fl32(dec(s) * g) (0 where dec(s) == 0).
+// E2M1 codes of r / fl32(dec(s) * g) (0 where dec(s) == 0). One CTA (8 warps) =
+// one 128-token block, loaded as in residual_e4m3_kernel: warp w holds rows
+// 16w .. 16w+15, which is exactly group w of the block, so a group's amax per
+// channel is a lane's max over its rows merged with the other half warp's. The
+// codes leave through a shared tile and 4 x 4 byte transposes as in
+// residual_mxfp4_kernel; the scales through a shared [channel][group] tile.
 template <typename T>
-__global__ void __launch_bounds__(128) residual_nvfp4_kernel(const T* __restrict__ v, int S, int H, int S_pad,
+__global__ void __launch_bounds__(256) residual_nvfp4_kernel(const T* __restrict__ v, int S, int H, int S_pad,
                                                              const int32_t* __restrict__ perm,
                                                              const float* __restrict__ mu,
                                                              const unsigned int* __restrict__ amax_bits,
                                                              uint8_t* __restrict__ codes,
                                                              uint8_t* __restrict__ scales, float* __restrict__ gsc) {
-  extern __shared__ __align__(16) float rt[];  // [128 channels][129]
-  __shared__ float smu[kD];
-  const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
-  const int t = threadIdx.x;
+  __shared__ __align__(16) uint8_t ct[kBlock * kResStride];
+  __shared__ __align__(8) uint8_t ssc[kD][8];   // [channel][group] scale codes of the block
+  const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x, nb = gridDim.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int half = lane >> 4, c = lane & 15;
   const float amax = __uint_as_float(amax_bits[bh]);
   const bool zero = !(amax >= kTinyAmax);
   const float g = zero ? 1.0f : __fdiv_rn(amax, kE4M3Max * kE2M1Max);
-  if (blk == 0 && t == 0) gsc[bh] = g;
-  smu[t] = mu[((size_t)bh * gridDim.x + blk) * kD + t];
-  __syncthreads();
+  if (blk == 0 && threadIdx.x == 0) gsc[bh] = g;
+  float m8[8];
   {
-    const int p = blk * kBlock + t;  // thread t: permuted row t
-    if (p < S && !zero) {
-      const T* row = v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD;
-#pragma unroll 4
-      for (int c = 0; c < 16; ++c) {
-        float f[8];
-        unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), f);
+    const float4* mp = reinterpret_cast<const float4*>(mu + ((size_t)bh * nb + blk) * kD + c * 8);
+    const float4 m0 = mp[0], m1 = mp[1];
+    m8[0] = m0.x; m8[1] = m0.y; m8[2] = m0.z; m8[3] = m0.w;
+    m8[4] = m1.x; m8[5] = m1.y; m8[6] = m1.z; m8[7] = m1.w;
+  }
+  int src[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) rt[(c * 8 + e) * 129 + t] = __fsub_rn(f[e], smu[c * 8 + e]);
-      }
-    } else {
-      for (int d = 0; d < kD; ++d) rt[d * 129 + t] = 0.0f;
+  for (int i = 0; i < 8; ++i) {
+    const int p = blk * kBlock + warp * 16 + 2 * i + half;
+    src[i] = p < S && !zero ? perm[(size_t)bh * S + p] : -1;
+  }
+  uint4 xs[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    xs[i] = src[i] >= 0 ? *reinterpret_cast<const uint4*>(v + (((size_t)b * S + src[i]) * H + h) * kD + c * 8)
+                        : make_uint4(0u, 0u, 0u, 0u);
+  float rr[8][8], mx[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mx[e] = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float f[8];
+    unpack8<T>(xs[i], f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      rr[i][e] = src[i] >= 0 ? __fsub_rn(f[e], m8[e]) : 0.0f;
+      mx[e] = fmaxf(mx[e], fabsf(rr[i][e]));
     }
   }
-  __syncthreads();
-  const int d = t;  // thread t: channel t
-  const float* rr = rt + d * 129;
-  uint8_t* crow = codes + ((size_t)bh * kD + d) * (S_pad / 2) + (size_t)blk * (kBlock / 2);
-  uint8_t* srow = scales + ((size_t)bh * kD + d) * (S_pad / kGroup4) + (size_t)blk * (kBlock / kGroup4);
-#pragma unroll 1
-  for (int gi = 0; gi < kBlock / kGroup4; ++gi) {
-    float gmax = 0.0f;
+  float den[8];
+  uint32_t scw0 = 0u, scw1 = 0u;
 #pragma unroll
-    for (int i = 0; i < kGroup4; ++i) gmax = fmaxf(gmax, fabsf(rr[gi * kGroup4 + i]));
-    const uint8_t sc = zero ? 0 : cvt_e4m3(__fdiv_rn(__fdiv_rn(gmax, kE2M1Max), g));
-    const float den = __fmul_rn(e4m3_to_f32(sc), g);
-    uint32_t w[2] = {0u, 0u};
-    if (sc != 0) {
+  for (int e = 0; e < 8; ++e) {
+    const float gmax = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 16));   // group `warp`, channel c*8+e
+    const uint32_t sc = zero ? 0u : cvt_e4m3(__fdiv_rn(__fdiv_rn(gmax, kE2M1Max), g));
+    den[e] = sc != 0u ? __fmul_rn(e4m3_to_f32(sc), g) : 0.0f;
+    if (e < 4) scw0 |= sc << (8 * e); else scw1 |= sc << (8 * (e - 4));
+  }
+  if (half == 0) {
 #pragma unroll
-      for (int i = 0; i < kGroup4; i += 2) {
-        const uint32_t byte = cvt_e2m1x2(__fdiv_rn(rr[gi * kGroup4 + i], den), __fdiv_rn(rr[gi * kGroup4 + i + 1], den));
-        w[i >> 3] |= byte << (8 * ((i >> 1) & 3));
-      }
+    for (int e = 0; e < 8; ++e) ssc[c * 8 + e][warp] = (uint8_t)(((e < 4 ? scw0 : scw1) >> (8 * (e & 3))) & 0xFFu);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = warp * 16 + 2 * i + half;
+    uint32_t w0 = 0u, w1 = 0u;   // one code per byte, channels c*8 .. c*8+7
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (den[e] != 0.0f) w0 |= (uint32_t)(cvt_e2m1x2(__fdiv_rn(rr[i][e], den[e]), 0.0f) & 0xFu) << (8 * e);
+      if (den[4 + e] != 0.0f)
+        w1 |= (uint32_t)(cvt_e2m1x2(__fdiv_rn(rr[i][4 + e], den[4 + e]), 0.0f) & 0xFu) << (8 * e);
     }
-    *reinterpret_cast<uint2*>(crow + gi * (kGroup4 / 2)) = make_uint2(w[0], w[1]);
-    srow[gi] = sc;
+    *reinterpret_cast<uint2*>(ct + r * kResStride + c * 8) = make_uint2(w0, w1);
+  }
+  __syncthreads();
+  if (threadIdx.x < kD) {
+    const int d = threadIdx.x;
+    *reinterpret_cast<uint2*>(scales + ((size_t)bh * kD + d) * (S_pad / kGroup4) + (size_t)blk * (kBlock / kGroup4)) =
+        *reinterpret_cast<const uint2*>(ssc[d]);
+  }
+  uint8_t* const out = codes + (size_t)bh * kD * (S_pad / 2) + (size_t)blk * (kBlock / 2);
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int combo = warp * 4 + it;
+    const int cg = 8 * (combo & 3) + (lane & 7), tq = 4 * (combo >> 2) + (lane >> 3);
+    const uint8_t* sp = ct + (4 * tq) * kResStride + 4 * cg;
+    const uint32_t r0 = *reinterpret_cast<const uint32_t*>(sp);
+    const uint32_t r1 = *reinterpret_cast<const uint32_t*>(sp + kResStride);
+    const uint32_t r2 = *reinterpret_cast<const uint32_t*>(sp + 2 * kResStride);
+    const uint32_t r3 = *reinterpret_cast<const uint32_t*>(sp + 3 * kResStride);
+    const uint32_t lo01 = __byte_perm(r0, r1, 0x5140), hi01 = __byte_perm(r0, r1, 0x7362);
+    const uint32_t lo23 = __byte_perm(r2, r3, 0x5140), hi23 = __byte_perm(r2, r3, 0x7362);
+    const uint32_t ch4[4] = {__byte_perm(lo01, lo23, 0x5410), __byte_perm(lo01, lo23, 0x7632),
+                             __byte_perm(hi01, hi23, 0x5410), __byte_perm(hi01, hi23, 0x7632)};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t w = ch4[q];
+      const uint32_t packed = (w & 0xFu) | ((w >> 4) & 0xF0u) | (((w >> 16) & 0xFu) << 8) | ((w >> 12) & 0xF000u);
+      *reinterpret_cast<uint16_t*>(out + (size_t)(4 * cg + q) * (S_pad / 2) + 2 * tq) = (uint16_t)packed;
+    }
   }
 }
 
@@ -1845,9 +1894,8 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
     residual_mxfp4_kernel<T><<<gb, 256, 0, st>>>(v, S, H, pl.S_pad, out.perm, out.mu, out.v_codes,
                                                  reinterpret_cast<uint32_t*>(out.v_scales), out.s_v);
   } else {
-    residual_nvfp4_kernel<T><<<gb, 128, kD * 129 * sizeof(float), st>>>(v, S, H, pl.S_pad, out.perm, out.mu,
-                                                                         pl.amax, out.v_codes, out.v_scales,
-                                                                         out.s_v);
+    residual_nvfp4_kernel<T><<<gb, 256, 0, st>>>(v, S, H, pl.S_pad, out.perm, out.mu, pl.amax, out.v_codes,
+                                                 out.v_scales, out.s_v);
   }
   *nlaunch = n + 2;
   return cudaGetLastError();
@@ -1954,10 +2002,6 @@ cudaError_t prep_configure() {
   if ((e = cudaFuncSetAttribute(kmeans_assign_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)assign_tc_smem<32>())) != cudaSuccess)
     return e;
-  for (auto f : {(const void*)residual_nvfp4_kernel<__nv_bfloat16>, (const void*)residual_nvfp4_kernel<__half>})
-    if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kD * 129 * 4))) !=
-        cudaSuccess)
-      return e;
   return cudaSuccess;
 }
 
