@@ -182,13 +182,38 @@ def oracle_sample(cfg, S_sample, rows, seed=0):
     return full, t2 - t0, desc
 
 
-def blas_threads():
-    try:
-        import threadpoolctl
-        n = [i["num_threads"] for i in threadpoolctl.threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except ImportError:
-        return os.cpu_count() or 1
+def oracle_cores():
+    """Host cores the oracle legs use: one process per core."""
+    return max(1, os.cpu_count() or 1)
+
+
+def _oracle_worker_init():
+    # one BLAS thread per process (set before the worker first imports numpy)
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"
+
+
+def _oracle_job(cfg, S_sample, rows, seed):
+    return oracle_sample(cfg, S_sample, rows, seed=seed)
+
+
+def oracle_sample_cores(cfg, S_sample, rows):
+    """The oracle as it stands on every host core: one process per core (spawned,
+    one BLAS thread each), each timing oracle_sample on its own seeded slice at
+    the same time. The workload's slices would be shared among the processes, so
+    its time is the mean per-process estimate over the process count.
+    Returns (seconds for the full workload, measured seconds per process,
+    description, processes)."""
+    n = oracle_cores()
+    if n == 1:
+        full, took, desc = oracle_sample(cfg, S_sample, rows)
+        return full, took, desc + "; 1 process", 1
+    import multiprocessing as mp
+    with mp.get_context("spawn").Pool(n, initializer=_oracle_worker_init) as pool:
+        res = pool.starmap(_oracle_job, [(cfg, S_sample, rows, seed) for seed in range(n)])
+    full = statistics.mean(r[0] for r in res) / n
+    took = statistics.mean(r[1] for r in res)
+    return full, took, res[0][2] + f"; {n} processes at once (one BLAS thread each), slices shared among them", n
 
 
 def run_reference(args, cfg):
@@ -201,10 +226,10 @@ def run_reference(args, cfg):
     budget = 150.0 / max(1, args.steps + args.warmup)
     S_sample = int(min(cfg["S"], max(1024, 8192 * budget / 1.3)))   # ~1.3 s per 8192 tokens here
     for _ in range(args.warmup):
-        oracle_sample(cfg, S_sample, 64)
+        oracle_sample_cores(cfg, S_sample, 64)
     est, meas = [], 0.0
     for _ in range(args.steps):
-        full, took, desc = oracle_sample(cfg, S_sample, 64)
+        full, took, desc, cores = oracle_sample_cores(cfg, S_sample, 64)
         est.append(full)
         meas += took
     t_full = statistics.mean(est)
@@ -214,7 +239,7 @@ def run_reference(args, cfg):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_full * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(cfg, args),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": desc + f"; measured {meas / max(1, args.steps):.2f} s per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -623,8 +648,8 @@ def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_s
         del pv0, v0
     # the oracle on the host cores, rank 0 at N = 1 only
     if world == 1 and rank == 0 and "cpu" in legs:
-        full, took, desc = oracle_sample(cfg, min(S, 73397), 256)
-        out["cpu_baseline"] = {"value": flops / full / 1e12, "unit": UNIT, "cores": blas_threads(),
+        full, took, desc, cores = oracle_sample_cores(cfg, min(S, 73397), 256)
+        out["cpu_baseline"] = {"value": flops / full / 1e12, "unit": UNIT, "cores": cores,
                                "kind": "oracle", "sample": desc + f"; measured {took:.1f} s"}
     return out
 

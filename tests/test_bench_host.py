@@ -25,6 +25,7 @@ def test_reference_line_has_the_contract_keys(monkeypatch, capsys):
         return 20.0, 0.5, f"stub over {S_sample} tokens"
 
     monkeypatch.setattr(bench, "oracle_sample", fake_sample)
+    monkeypatch.setattr(bench, "oracle_cores", lambda: 1)
     monkeypatch.delenv("RANK", raising=False)
     cfg = synth.workload("minimax_h56")
     bench.run_reference(_args(), cfg)
@@ -37,6 +38,7 @@ def test_reference_line_has_the_contract_keys(monkeypatch, capsys):
     assert line["ms_per_step"] == pytest.approx(20.0e3)
     assert line["value"] == pytest.approx(bench.flops_of(cfg) / 20.0 / 1e12)
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] == 1
     assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert line["config"]["workload"] == "minimax_h56" and line["config"]["S"] == 73397
@@ -81,3 +83,12 @@ def test_peaks_fallback(monkeypatch, tmp_path):
         {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1300.0}))
     p = bench.load_peaks()
     assert p == dict(bf16_sustained=1300.0, bf16_burst=1500.0, hbm=6000.0, source="measured")
+
+
+def test_oracle_on_several_cores_shares_the_slices(monkeypatch):
+    # two spawned processes, each timing a tiny oracle sample: the workload estimate
+    # is the mean per-process estimate over the process count
+    monkeypatch.setattr(bench, "oracle_cores", lambda: 2)
+    cfg = synth.workload("tiny")
+    full, took, desc, cores = bench.oracle_sample_cores(cfg, 256, 8)
+    assert cores == 2 and full > 0 and took > 0 and "2 processes" in desc
