@@ -40,7 +40,7 @@ ATTN_KERNEL = {"e4m3": "vc_attn_fwd_kernel<1>", "nvfp4": "vc_attn_fwd_kernel<2>"
 # DRAM bytes (read + write) of one attention launch on the default workload, from
 # the ncu capture summarised in profiles/; valid only while the kernel source
 # hashes to the recorded value (otherwise traffic is reported as null).
-ATTN_TRAFFIC = {"sha256_16": "787fd709a13f5b16", "bytes_per_launch": 8 * (200.549888e6 + 105.42976e6)}
+ATTN_TRAFFIC = {"sha256_16": "2b726db56ae51685", "bytes_per_launch": 8 * (200.098304e6 + 103.392e6)}
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 FALLBACK_HBM_GBS = 6650.0
 
