@@ -354,13 +354,61 @@ def run_ours(args, cfg):
     legs = set() if args.no_extras else (
         {"accuracy", "energy", "smoothk", "exp2", "sdpa", "e2e", "cpu", "ties", "formats", "repair"}
         if args.extras == "all" else set(args.extras.split(",")))
-    if legs:
+    if world > 1:
+        # the same problem split by heads over the ranks (strong scaling), beside
+        # the independent problem per rank that `value` reports
+        del plan
+        line["head_split"] = run_head_split(args, cfg, dev, world, rank, barrier)
+        plan = None
+    if legs and plan is not None:
         line.update(extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_step, rank, legs))
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def head_slice(X, h0, h1):
+    """Heads [h0, h1) of a [B, S, H, 128] (or [S, H, 128]) tensor, as a dense tensor."""
+    return (X[:, h0:h1] if X.dim() == 3 else X[:, :, h0:h1]).contiguous()
+
+
+def run_head_split(args, cfg, dev, world, rank, barrier):
+    """One problem (the workload drawn with seed 0 on every rank) split by heads:
+    rank r runs heads vc_attn.head_range(H, r, N) through a plan that seeds its
+    k-means as those heads of the whole problem, so the N ranks together compute
+    exactly the single-GPU result, with no exchange between them. Timed like the
+    main region (barrier and synchronize on both sides, max over ranks); the
+    value counts the whole problem's FLOPs once."""
+    import torch
+    from bit_fp8_attention_prep_b200 import synth, vc_attn
+    B, S, H = cfg["B"], cfg["S"], cfg["H"]
+    h0, h1 = vc_attn.head_range(H, rank, world)
+    Qf, Kf, Vf = synth.make_workload(cfg["name"], seed=0, device=dev)[1:]
+    Q, K, V = (head_slice(X, h0, h1) for X in (Qf, Kf, Vf))
+    del Qf, Kf, Vf
+    plan = vc_attn.Plan(B, S, h1 - h0, k=cfg["k"], iters=cfg["iters"], fmt=cfg["fmt"], k_p=args.k_p, device=dev,
+                        h_base=h0, H_total=H)
+    for _ in range(args.warmup):
+        plan.run(Q, K, V)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        plan.run(Q, K, V)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    status = int(plan.status.item())
+    del plan, Q, K, V
+    return {"value": flops_of(cfg) / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms, "scaling": "strong",
+            "heads": [list(vc_attn.head_range(H, r, world)) for r in range(world)], "device_status": status,
+            "what": "one problem split by heads over the ranks (vc_attn_prepare_v_shard seeds each shard's "
+                    "k-means as those heads of the whole problem); whole-problem FLOPs over the slowest rank"}
 
 
 def extras(args, cfg, plan, Q, K, V, dev, stream, flops, world, fwd_ms, ms_per_step, rank, legs):

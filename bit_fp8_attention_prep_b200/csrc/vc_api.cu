@@ -224,11 +224,11 @@ static vc_status_t check_prep_args(const void* v, const vc_shape_t* shape, const
   return VC_OK;
 }
 
-// vc_attn_prepare_v with the slices numbered from bh_base (the k-means seed of
-// slice i of this call is that of slice bh_base + i of the caller's problem).
+// vc_attn_prepare_v where slice (b, h) of this call is slice (seed_b0 + b,
+// seed_h0 + h) of a problem with seed_H heads (whose k-means seed it takes).
 static vc_status_t prepare_v_impl(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
                                   const vc_prepared_v_t* out, void* workspace, size_t workspace_bytes,
-                                  uint8_t* assign_history, void* stream, int bh_base) {
+                                  uint8_t* assign_history, void* stream, int seed_H, int seed_b0, int seed_h0) {
   vc_status_t st;
   if ((st = check_prep_args(v, shape, cfg, out)) != VC_OK) return st;
   const WsLayout w = ws_layout(shape, cfg);
@@ -248,7 +248,9 @@ static vc_status_t prepare_v_impl(const void* v, const vc_shape_t* shape, const 
   pl.fmt = cfg->residual_fmt;
   pl.mode = cfg->mode;
   pl.seed = cfg->seed;
-  pl.bh_base = bh_base;
+  pl.seed_H = seed_H;
+  pl.seed_b0 = seed_b0;
+  pl.seed_h0 = seed_h0;
   pl.nb = nblocks(shape->S);
   pl.S_pad = pl.nb * 128;
   pl.nchunks = (shape->S + vc::kChunk - 1) / vc::kChunk;
@@ -310,7 +312,8 @@ vc_status_t vc_attn_prepare_v_repair(const void* v, const vc_shape_t* shape, con
     return fail(VC_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
                 workspace ? workspace_bytes : (size_t)0);
   const WsLayout w = ws_layout(shape, cfg);
-  if ((st = prepare_v_impl(v, shape, cfg, out, workspace, w.total, nullptr, stream, 0)) != VC_OK) return st;
+  if ((st = prepare_v_impl(v, shape, cfg, out, workspace, w.total, nullptr, stream, shape->H, 0, 0)) != VC_OK)
+    return st;
   const size_t BH = (size_t)shape->B * shape->H;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* err = reinterpret_cast<float*>(ws + w.total);
@@ -330,7 +333,23 @@ vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_v
                               uint8_t* assign_history, void* stream) {
   NvtxRange range("vc_attn_prepare_v");
   g_last_error.clear();
-  return prepare_v_impl(v, shape, cfg, out, workspace, workspace_bytes, assign_history, stream, 0);
+  return prepare_v_impl(v, shape, cfg, out, workspace, workspace_bytes, assign_history, stream, shape ? shape->H : 0,
+                        0, 0);
+}
+
+vc_status_t vc_attn_prepare_v_shard(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                                    int32_t h_base, int32_t H_total, const vc_prepared_v_t* out, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  NvtxRange range("vc_attn_prepare_v_shard");
+  g_last_error.clear();
+  vc_status_t st;
+  if ((st = check_shape(shape)) != VC_OK) return st;
+  if (h_base < 0 || H_total < 1 || (long long)h_base + shape->H > (long long)H_total)
+    return fail(VC_ERR_INVALID_ARG, "heads [h_base, h_base + H) = [%d, %lld) must lie in [0, H_total = %d)", h_base,
+                (long long)h_base + shape->H, H_total);
+  if ((long long)shape->B * H_total > 0x7fffffffll)
+    return fail(VC_ERR_INVALID_ARG, "B * H_total exceeds the slice index range");
+  return prepare_v_impl(v, shape, cfg, out, workspace, workspace_bytes, nullptr, stream, H_total, 0, h_base);
 }
 
 vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* shape, const int32_t* perm,
@@ -802,7 +821,7 @@ vc_status_t vc_attn_run_host(const void* q, const void* k, const void* v, const 
       qk.k_codes = ws + L.k_codes[slot];
       qk.k_scales = reinterpret_cast<float*>(ws + L.k_scales[slot]);
       if ((st = prepare_v_impl(ws + L.in[slot][2], &cs, cfg, &pv, ws + L.prep_ws[slot], L.prep_ws_bytes, nullptr,
-                               cst, b * H + h0)) != VC_OK)
+                               cst, H, b, h0)) != VC_OK)
         return st;
       if ((st = vc_attn_quant_qk(ws + L.in[slot][0], ws + L.in[slot][1], &cs, pv.perm, &qk, cst)) != VC_OK)
         return st;

@@ -20,8 +20,9 @@ constexpr int kChunk = 1024;       // tokens per k-means CTA (also the sort's ch
 struct PrepPlan {
   int B, S, H, k, iters, fmt, mode;
   uint64_t seed;
-  int bh_base;                 // index b*H + h of this plan's first slice in the caller's problem
-                               // (0 unless the problem is run in chunks of heads)
+  int seed_H, seed_b0, seed_h0;  // slice (b, h) of this plan is slice (seed_b0 + b, seed_h0 + h) of a
+                                 // problem with seed_H heads (its k-means seed); H, 0, 0 unless the
+                                 // problem is run in chunks or shards of heads
   int nb, S_pad, nchunks;
   float* cent;                 // [BH][k][128]
   unsigned long long* sums;    // [BH][k][128] int64 fixed-point

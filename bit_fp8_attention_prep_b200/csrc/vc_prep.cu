@@ -40,11 +40,15 @@ __device__ __forceinline__ uint64_t splitmix64_next(uint64_t& state) {
 
 template <typename T>
 __global__ void __launch_bounds__(128) kmeans_init_kernel(const T* __restrict__ v, int S, int H, int k,
-                                                          uint64_t seed, int bh_base, float* __restrict__ cent) {
+                                                          uint64_t seed, int seed_H, int seed_b0, int seed_h0,
+                                                          float* __restrict__ cent) {
   __shared__ int idx[kMaxClusters];
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
   if (threadIdx.x == 0) {
-    uint64_t st = seed ^ (0x9E3779B97F4A7C15ull * (uint64_t)(bh_base + bh + 1));
+    // the seed of slice (b, h) of this call is that of slice (seed_b0 + b, seed_h0 + h)
+    // of the whole problem, which has seed_H heads
+    const uint64_t g = (uint64_t)(seed_b0 + b) * (uint64_t)seed_H + (uint64_t)(seed_h0 + h);
+    uint64_t st = seed ^ (0x9E3779B97F4A7C15ull * (g + 1));
     for (int i = 0; i < k; ++i) {
       int u;
       while (true) {
@@ -1856,7 +1860,7 @@ static cudaError_t launch_prepare_v_t(const T* v, const PrepPlan& pl, const vc_p
     if ((e = cudaMemsetAsync(pl.sums, 0, sizeof(unsigned long long) * BH * k * kD, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(pl.counts, 0, sizeof(int) * BH * k, st)) != cudaSuccess) return e;
     if (pl.tc_assign && (e = cudaMemsetAsync(pl.work, 0, sizeof(int) * pl.iters, st)) != cudaSuccess) return e;
-    kmeans_init_kernel<T><<<BH, 128, 0, st>>>(v, S, H, k, pl.seed, pl.bh_base, pl.cent);
+    kmeans_init_kernel<T><<<BH, 128, 0, st>>>(v, S, H, k, pl.seed, pl.seed_H, pl.seed_b0, pl.seed_h0, pl.cent);
     ++n;
     const dim3 grid(pl.nchunks, BH);
     // pass it writes its labels to assign (even) or assign2 (odd); the sums of

@@ -34,7 +34,7 @@ ABI_SYMBOLS = [
     "vc_attn_prepare_v_noalloc", "vc_attn_run_host_workspace_bytes", "vc_attn_run_host",
     "vc_attn_residual_energy", "vc_attn_quant_qk_smoothk_workspace_bytes", "vc_attn_quant_qk_smoothk",
     "vc_attn_prepare_v_repair_workspace_bytes", "vc_attn_prepare_v_repair", "vc_attn_forward_repair",
-    "vc_attn_forward_e4m3_per_channel", "vc_attn_forward_mxfp4v",
+    "vc_attn_forward_e4m3_per_channel", "vc_attn_forward_mxfp4v", "vc_attn_prepare_v_shard",
 ]
 NOALLOC_SCRATCH_BYTES = 12 << 20  # VC_ATTN_NOALLOC_SCRATCH_BYTES
 TEST_SYMBOLS = ["vc_attn_test_e4m3_round", "vc_attn_test_e2m1_round", "vc_attn_test_expcast",
@@ -88,6 +88,8 @@ def load():
     lib.vc_attn_prepare_v_workspace_bytes.argtypes = [P(Shape), P(VSmoothCfg)]
     lib.vc_attn_prepare_v.restype = i32
     lib.vc_attn_prepare_v.argtypes = [vp, P(Shape), P(VSmoothCfg), P(PreparedV), vp, sz, vp, vp]
+    lib.vc_attn_prepare_v_shard.restype = i32
+    lib.vc_attn_prepare_v_shard.argtypes = [vp, P(Shape), P(VSmoothCfg), i32, i32, P(PreparedV), vp, sz, vp]
     lib.vc_attn_prepare_v_noalloc.restype = i32
     lib.vc_attn_prepare_v_noalloc.argtypes = [vp, P(Shape), P(VSmoothCfg), P(PreparedV), vp, vp]
     lib.vc_attn_quant_qk.restype = i32
@@ -189,10 +191,27 @@ def _prepared_buffers(B, S, H, fmt, dev):
     return out
 
 
-def prepare_v(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", history=False):
+def head_range(H, rank, world):
+    """Heads [h0, h1) of rank ``rank`` when a problem of H heads is split by heads
+    over ``world`` ranks: contiguous ranges, sizes differing by at most one, that
+    tile [0, H) in rank order."""
+    if not (0 <= rank < world):
+        raise ValueError("rank must be in [0, world)")
+    return (H * rank) // world, (H * (rank + 1)) // world
+
+
+def seed_slice_index(b, h, H):
+    """Index of slice (b, h) of a problem with H heads: the k-means seed's input
+    (slice i is seeded with seed ^ (0x9E3779B97F4A7C15 * (i + 1)))."""
+    return b * H + h
+
+
+def prepare_v(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", history=False, h_base=0, H_total=None):
     """V-Smooth prep of V (device tensor). Returns a dict of the caller-owned
     outputs (perm, mu, v_codes, v_scales, s_v; plus the per-pass assignments
-    when ``history``)."""
+    when ``history``). With ``H_total``, ``v`` holds heads [h_base, h_base + H)
+    of a problem with H_total heads (vc_attn_prepare_v_shard): the outputs are
+    those heads of the whole problem's prep, bit for bit."""
     lib = load()
     sh = shape_of(v)
     cfg = VSmoothCfg(k, iters, seed, _fmt_code(fmt), _MODES[mode])
@@ -206,8 +225,14 @@ def prepare_v(v, k=16, iters=4, seed=0, fmt="e4m3", mode="vsmooth", history=Fals
     off = (-ws.data_ptr()) % 256
     hist = torch.empty((iters, B, H, S), dtype=torch.uint8, device=dev) if history else None
     pv = PreparedV(_ptr(out["perm"]), _ptr(out["mu"]), _ptr(out["v_codes"]), _ptr(out["v_scales"]), _ptr(out["s_v"]))
-    _check(lib.vc_attn_prepare_v(_ptr(v), ctypes.byref(sh), ctypes.byref(cfg), ctypes.byref(pv),
-                                 ctypes.c_void_p(ws.data_ptr() + off), wsb, _ptr(hist), _stream()))
+    if H_total is not None:
+        if history:
+            raise ValueError("the shard prep keeps no assignment history")
+        _check(lib.vc_attn_prepare_v_shard(_ptr(v), ctypes.byref(sh), ctypes.byref(cfg), int(h_base), int(H_total),
+                                           ctypes.byref(pv), ctypes.c_void_p(ws.data_ptr() + off), wsb, _stream()))
+    else:
+        _check(lib.vc_attn_prepare_v(_ptr(v), ctypes.byref(sh), ctypes.byref(cfg), ctypes.byref(pv),
+                                     ctypes.c_void_p(ws.data_ptr() + off), wsb, _ptr(hist), _stream()))
     out["workspace"] = ws
     out["history"] = hist
     return out
@@ -379,8 +404,10 @@ class Plan:
     """
 
     def __init__(self, B, S, H, dtype=torch.bfloat16, k=16, iters=4, seed=0, fmt="e4m3", k_p=8,
-                 softmax_scale=None, device=None, mode="vsmooth", smooth_k=False):
+                 softmax_scale=None, device=None, mode="vsmooth", smooth_k=False, h_base=0, H_total=None):
         self.lib = load()
+        # a shard of heads [h_base, h_base + H) of a problem with H_total heads
+        self.h_base, self.H_total = int(h_base), (None if H_total is None else int(H_total))
         dev = torch.device(device if device is not None else "cuda")
         self.shape = Shape(B, S, H, 128, VC_DTYPE_BF16 if dtype == torch.bfloat16 else VC_DTYPE_F16)
         self.cfg = VSmoothCfg(k, iters, seed, _fmt_code(fmt), _MODES[mode])
@@ -417,8 +444,13 @@ class Plan:
             self.smooth_ws_bytes, self._smooth_ws, self.k_mean = 0, None, None
 
     def prepare_v(self, v):
-        _check(self.lib.vc_attn_prepare_v(_ptr(v), ctypes.byref(self.shape), ctypes.byref(self.cfg),
-                                          ctypes.byref(self._pv), self.ws_ptr, self.ws_bytes, None, _stream()))
+        if self.H_total is not None:
+            _check(self.lib.vc_attn_prepare_v_shard(_ptr(v), ctypes.byref(self.shape), ctypes.byref(self.cfg),
+                                                    self.h_base, self.H_total, ctypes.byref(self._pv), self.ws_ptr,
+                                                    self.ws_bytes, _stream()))
+        else:
+            _check(self.lib.vc_attn_prepare_v(_ptr(v), ctypes.byref(self.shape), ctypes.byref(self.cfg),
+                                              ctypes.byref(self._pv), self.ws_ptr, self.ws_bytes, None, _stream()))
 
     def quant_qk(self, q, k):
         if self.smooth_k:

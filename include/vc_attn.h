@@ -167,6 +167,24 @@ vc_status_t vc_attn_prepare_v(const void* v, const vc_shape_t* shape, const vc_v
                               const vc_prepared_v_t* out, void* workspace, size_t workspace_bytes,
                               uint8_t* assign_history, void* stream);
 
+/* V-Smooth prep of a shard of heads of a larger problem: as vc_attn_prepare_v on
+ * v = heads [h_base, h_base + shape->H) of a [B,S,H_total,128] problem, given as a
+ * dense [B,S,shape->H,128] tensor. Every (b, h) slice of the method is independent
+ * ("VC-Attention ...", Abstract: clustering, block means and the residual scale
+ * are per value head; "Nunchux AI lanza ...", 2nd paragraph: k-means per batch and
+ * head); the only link to the rest of the problem is the k-means init, whose seed
+ * index is that of slice (b, h_base + h) of the whole problem, b*H_total + h_base + h.
+ * So the outputs are, bit for bit, the heads [h_base, h_base + shape->H) of what
+ * vc_attn_prepare_v gives for the whole problem: a problem can be split by heads over
+ * several GPUs (or calls) with no exchange at all.
+ *  h_base, H_total  0 <= h_base, h_base + shape->H <= H_total
+ *  other arguments  as vc_attn_prepare_v (no assignment history)
+ * Errors: as vc_attn_prepare_v, plus VC_ERR_INVALID_ARG for a head range outside
+ * [0, H_total). */
+vc_status_t vc_attn_prepare_v_shard(const void* v, const vc_shape_t* shape, const vc_vsmooth_cfg_t* cfg,
+                                    int32_t h_base, int32_t H_total, const vc_prepared_v_t* out, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
 /* Q/K FP8 quantisation ("Open VC Attention", "Описание": Q/K scales per block):
  * per (b, h, 128-row block) scale s = amax/448 and E4M3 codes of x*(448/amax);
  * K rows are gathered through `perm` (from vc_attn_prepare_v) first.

@@ -271,3 +271,11 @@ def test_noalloc_prep_checks_arguments_before_the_device(lib):
     st = lib.vc_attn_prepare_v_noalloc(ctypes.c_void_p(16), ctypes.byref(_shape()), ctypes.byref(_cfg()),
                                        ctypes.byref(pv), None, None)
     assert st in (vc_attn.VC_ERR_CUDA, vc_attn.VC_ERR_UNSUPPORTED)
+
+
+def test_shard_prep_rejects_head_ranges_outside_the_problem(lib):
+    pv = vc_attn.PreparedV(16, 16, 16, 16, 16)
+    for h_base, H_total in ((-1, 8), (7, 8), (0, 1), (3, 4)):   # local H = 2
+        st = lib.vc_attn_prepare_v_shard(ctypes.c_void_p(16), ctypes.byref(_shape(H=2)), ctypes.byref(_cfg()),
+                                         h_base, H_total, ctypes.byref(pv), ctypes.c_void_p(256), 1 << 20, None)
+        assert st == vc_attn.VC_ERR_INVALID_ARG and b"H_total" in lib.vc_attn_last_error()
