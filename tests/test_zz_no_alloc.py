@@ -58,17 +58,19 @@ def test_noalloc_prep_matches_workspace_prep_on_two_calls(va):
 
 
 def test_noalloc_prep_other_residuals_and_modes(va):
-    # the NVFP4 residual and the MEANONLY / NAIVE modes lay the scratch out
-    # differently (one cluster, no second label buffer); each runs right after a
-    # mid-size VSMOOTH call has left its contents in the array
+    # the NVFP4, MX-style and per-channel residuals and the MEANONLY / NAIVE modes
+    # lay the scratch out differently (one cluster, no second label buffer, an amax
+    # per channel); each runs right after a mid-size VSMOOTH call has left its
+    # contents in the array
     cfg, Q, K, V = make("mid", B=1, H=4, S=3000)
     v = V.cuda()
-    for fmt, mode in (("nvfp4", "vsmooth"), ("e4m3", "meanonly"), ("e4m3", "naive"), ("nvfp4", "meanonly")):
+    for fmt, mode in (("nvfp4", "vsmooth"), ("e4m3", "meanonly"), ("e4m3", "naive"), ("nvfp4", "meanonly"),
+                      ("e4m3c", "vsmooth"), ("mxfp4", "vsmooth")):
         va.prepare_v_noalloc(v, k=16, iters=4)            # leaves VSMOOTH scratch behind
         ref = va.prepare_v(v, k=16, iters=4, fmt=fmt, mode=mode)
         got = va.prepare_v_noalloc(v, k=16, iters=4, fmt=fmt, mode=mode)
         torch.cuda.synchronize()
-        if fmt == "nvfp4":
+        if fmt in ("nvfp4", "mxfp4"):
             _same_nvfp4(got, ref)
         else:
             for key in ("perm", "mu", "v_codes", "s_v"):
