@@ -379,7 +379,6 @@ constexpr int kTcTmaWarp = 8, kTcMmaWarp = 9;
 constexpr int kTcDStages = 4;                  // tensor-memory dot stages (two per token-warp group)
 constexpr uint32_t kTcStageCols = 64;          // tensor-memory columns per dot stage (N = 2 KC <= 64)
 constexpr uint32_t kTcTileBytes = kTile * 256; // 128 tokens x 128 bf16 (two 16 KB boxes)
-constexpr int kTcTilesPerChunk = kChunk / kTile;
 
 // Bytes of one slice's centroid operand block: [2 halves][2 KC rows][128 B], then
 // |c|^2 [KC] and |c| [KC] (fp32).
@@ -1723,40 +1722,63 @@ __device__ __forceinline__ unsigned long long repair_key(float err, int p) {
   return ((unsigned long long)__float_as_uint(err) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)p);
 }
 
-// err[bh][p] for every permuted position p < S. One CTA = one 128-token block,
-// one thread per token; the thread walks its gathered V row 16 bytes at a time
-// and reads its codes from the V^T plane (consecutive threads, consecutive bytes).
+// The tile of one 128-token block of permuted positions in shared memory: rows
+// gathered through perm with coalesced 16-byte loads (two rows per warp
+// instruction, every load of a thread issued before the first store), at
+// tile_off(r, piece). Rows past S are left unwritten.
+template <typename T>
+__device__ __forceinline__ void stage_perm_tile(uint8_t* tile, const T* __restrict__ v, int S, int H, int b, int h,
+                                                const int32_t* __restrict__ prow, int ntok) {
+  const int tid = threadIdx.x;
+  uint4 x[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int idx = i * kTile + tid, r = idx >> 4, c = idx & 15;
+    if (r < ntok) x[i] = *reinterpret_cast<const uint4*>(v + (((size_t)b * S + prow[r]) * H + h) * kD + c * 8);
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int idx = i * kTile + tid, r = idx >> 4, c = idx & 15;
+    if (r < ntok) *reinterpret_cast<uint4*>(tile + tile_off(r, c)) = x[i];
+  }
+}
+
+// err[bh][p] for every permuted position p < S. One CTA = one 128-token block:
+// the block's rows are staged in shared memory, then each thread takes one token,
+// recomputes its codes exactly as the residual kernel does (so plane 0 need not
+// be read) and sums the squared rounding errors channel by channel in order.
 template <typename T>
 __global__ void __launch_bounds__(128) repair_err_kernel(const T* __restrict__ v, int S, int H, int S_pad,
                                                          const int32_t* __restrict__ perm,
                                                          const float* __restrict__ mu,
                                                          const unsigned int* __restrict__ amax_bits,
-                                                         const uint8_t* __restrict__ vt, float* __restrict__ err) {
+                                                         float* __restrict__ err) {
   __shared__ float smu[kD];
+  extern __shared__ __align__(16) uint8_t tile[];
   const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x, t = threadIdx.x;
+  const int p0 = blk * kBlock, ntok = min(kBlock, S - p0);
   smu[t] = mu[((size_t)bh * gridDim.x + blk) * kD + t];
-  __syncthreads();
-  const int p = blk * kBlock + t;
-  if (p >= S) return;
   const float amax = __uint_as_float(amax_bits[bh]);
+  const bool zero = !(amax >= kTinyAmax);
+  if (!zero) stage_perm_tile<T>(tile, v, S, H, b, h, perm + (size_t)bh * S + p0, ntok);
+  __syncthreads();
+  if (t >= ntok) return;
   float e = 0.0f;
-  if (amax >= kTinyAmax) {
+  if (!zero) {
     const float inv = __fdiv_rn(kE4M3Max, amax);
-    const T* row = v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD;
-    const uint8_t* code = vt + (size_t)bh * kD * S_pad + p;
-#pragma unroll 1
-    for (int c = 0; c < kD / 8; ++c) {
+#pragma unroll 4
+    for (int c = 0; c < 16; ++c) {
       float f[8];
-      unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), f);
+      unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off(t, c)), f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int d = c * 8 + i;
-        const float dl = repair_dlt(f[i], smu[d], inv, code[(size_t)d * S_pad]);
+        const float y = __fmul_rn(__fsub_rn(f[i], smu[c * 8 + i]), inv);
+        const float dl = __fsub_rn(y, e4m3_to_f32(cvt_e4m3(y)));
         e = __fadd_rn(e, __fmul_rn(dl, dl));
       }
     }
   }
-  err[(size_t)bh * S + p] = e;
+  err[(size_t)bh * S + p0 + t] = e;
 }
 
 // thr[bh] = the key of the m-th largest token (1 <= m <= S): a radix select over
@@ -1806,9 +1828,10 @@ __global__ void __launch_bounds__(256) repair_select_kernel(const float* __restr
 }
 
 // Plane 1 (and the optional kept flags): one CTA = one 128-token block of
-// permuted positions, one thread per token; channel by channel the 128 threads
-// write 128 consecutive bytes of the V^T plane. Tokens not kept, padding tokens
-// and slices whose residual is all zero get 0.
+// permuted positions, its rows staged in shared memory when any is kept; one
+// thread per token, which recomputes its codes as the residual kernel does; channel
+// by channel the 128 threads write 128 consecutive bytes of the V^T plane. Tokens
+// not kept, padding tokens and slices whose residual is all zero get 0.
 template <typename T>
 __global__ void __launch_bounds__(128) repair_plane_kernel(const T* __restrict__ v, int S, int H, int S_pad,
                                                            const int32_t* __restrict__ perm,
@@ -1816,33 +1839,39 @@ __global__ void __launch_bounds__(128) repair_plane_kernel(const T* __restrict__
                                                            const unsigned int* __restrict__ amax_bits,
                                                            const float* __restrict__ err,
                                                            const unsigned long long* __restrict__ thr, bool any,
-                                                           const uint8_t* __restrict__ vt,
                                                            uint8_t* __restrict__ plane1, uint8_t* __restrict__ kept) {
   __shared__ float smu[kD];
+  __shared__ int nkeep;
+  extern __shared__ __align__(16) uint8_t tile[];
   const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x, t = threadIdx.x;
+  const int p0 = blk * kBlock, ntok = min(kBlock, S - p0), p = p0 + t;
   smu[t] = mu[((size_t)bh * gridDim.x + blk) * kD + t];
+  if (t == 0) nkeep = 0;
   __syncthreads();
-  const int p = blk * kBlock + t;
+  const float amax = __uint_as_float(amax_bits[bh]);
+  const bool zero = !(amax >= kTinyAmax);
   const bool keep = any && p < S && repair_key(err[(size_t)bh * S + p], p) >= thr[bh];
   if (kept != nullptr && p < S) kept[(size_t)bh * S + p] = keep ? 1 : 0;
+  if (keep && !zero) atomicAdd(&nkeep, 1);
+  __syncthreads();
+  const bool stage = nkeep > 0;   // uniform: the block has a kept token
+  if (stage) stage_perm_tile<T>(tile, v, S, H, b, h, perm + (size_t)bh * S + p0, ntok);
+  __syncthreads();
   uint8_t* out = plane1 + (size_t)bh * kD * S_pad + p;
-  const float amax = __uint_as_float(amax_bits[bh]);
-  if (!keep || !(amax >= kTinyAmax)) {
+  if (!keep || zero) {
 #pragma unroll 4
     for (int d = 0; d < kD; ++d) out[(size_t)d * S_pad] = 0;
     return;
   }
   const float inv = __fdiv_rn(kE4M3Max, amax);
-  const T* row = v + (((size_t)b * S + perm[(size_t)bh * S + p]) * H + h) * kD;
-  const uint8_t* code = vt + (size_t)bh * kD * S_pad + p;
-#pragma unroll 1
-  for (int c = 0; c < kD / 8; ++c) {
+#pragma unroll 4
+  for (int c = 0; c < 16; ++c) {
     float f[8];
-    unpack8<T>(*reinterpret_cast<const uint4*>(row + c * 8), f);
+    unpack8<T>(*reinterpret_cast<const uint4*>(tile + tile_off(t, c)), f);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int d = c * 8 + i;
-      out[(size_t)d * S_pad] = cvt_e4m3(repair_dlt(f[i], smu[d], inv, code[(size_t)d * S_pad]));
+      const float y = __fmul_rn(__fsub_rn(f[i], smu[c * 8 + i]), inv);
+      out[(size_t)(c * 8 + i) * S_pad] = cvt_e4m3(__fsub_rn(y, e4m3_to_f32(cvt_e4m3(y))));
     }
   }
 }
@@ -1965,20 +1994,21 @@ cudaError_t launch_repair(const void* v, int dtype, int B, int S, int H, const i
   int n = 0;
   if (m > 0) {
     if (bf)
-      repair_err_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(v), S, H, S_pad, perm,
-                                                             mu, amax_bits, planes, err);
+      repair_err_kernel<__nv_bfloat16><<<grid, 128, kTileBytes, st>>>(static_cast<const __nv_bfloat16*>(v), S, H,
+                                                                      S_pad, perm, mu, amax_bits, err);
     else
-      repair_err_kernel<__half><<<grid, 128, 0, st>>>(static_cast<const __half*>(v), S, H, S_pad, perm, mu,
-                                                      amax_bits, planes, err);
+      repair_err_kernel<__half><<<grid, 128, kTileBytes, st>>>(static_cast<const __half*>(v), S, H, S_pad, perm, mu,
+                                                               amax_bits, err);
     repair_select_kernel<<<BH, 256, 0, st>>>(err, S, m, thr);
     n += 2;
   }
   if (bf)
-    repair_plane_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(v), S, H, S_pad, perm,
-                                                             mu, amax_bits, err, thr, m > 0, planes, plane1, kept);
+    repair_plane_kernel<__nv_bfloat16><<<grid, 128, kTileBytes, st>>>(static_cast<const __nv_bfloat16*>(v), S, H,
+                                                                      S_pad, perm, mu, amax_bits, err, thr, m > 0,
+                                                                      plane1, kept);
   else
-    repair_plane_kernel<__half><<<grid, 128, 0, st>>>(static_cast<const __half*>(v), S, H, S_pad, perm, mu,
-                                                      amax_bits, err, thr, m > 0, planes, plane1, kept);
+    repair_plane_kernel<__half><<<grid, 128, kTileBytes, st>>>(static_cast<const __half*>(v), S, H, S_pad, perm, mu,
+                                                               amax_bits, err, thr, m > 0, plane1, kept);
   *nlaunch = n + 1;
   return cudaGetLastError();
 }
