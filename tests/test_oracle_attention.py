@@ -5,12 +5,14 @@
 - V-Smooth recovery: with exact probabilities and unquantised inputs, the
   block-mean split (residual through PV, mean through the block row sums)
   reproduces exact attention;
-- the ExpCast VC-attention output against a brute-force loop with exact sums.
+- the ExpCast VC-attention output against a brute-force loop with exact sums;
+- kappa against softmax_scale * log2(e) at 60 digits.
 """
 import math
 from fractions import Fraction
 
 import numpy as np
+import pytest
 import torch
 
 import oracle as O
@@ -184,3 +186,20 @@ def test_online_probs_within_piecewise_linear_bound():
     assert ratio.max() <= 1.5 / math.sqrt(2) * 2 ** (1 / 16) + 1e-12
     # the largest probability of every row sits in the top binade below 2^k_P
     assert np.all(P.max(axis=1) <= 2.0 ** 8) and np.all(P.max(axis=1) >= 2.0 ** 7 * 2 ** (-1 / 16))
+
+
+def test_softmax_kappa_is_scale_times_log2e():
+    # exp(s x) = 2^(kappa x) with kappa = s log2(e), rounded once to fp32: the
+    # oracle's fp64 product then fp32 rounding lands within half an fp32 ulp
+    # (plus 2^-53 relative) of the exact value computed at 60 digits.
+    from decimal import Decimal, getcontext
+    getcontext().prec = 60
+    log2e = 1 / Decimal(2).ln()
+    for s in (1 / math.sqrt(128), 1 / math.sqrt(64), 1.0, 0.125, 0.3):
+        s32 = Decimal(float(np.float32(s)))
+        k = O.softmax_kappa(s)
+        assert k.dtype == np.float32
+        ulp = Decimal(float(np.spacing(k)))
+        assert abs(Decimal(float(k)) - s32 * log2e) <= ulp * Decimal("0.5000001")
+        x = 7.0
+        assert 2.0 ** (float(k) * x) == pytest.approx(math.exp(float(np.float32(s)) * x), rel=1e-6)

@@ -90,18 +90,52 @@ def test_lloyd_centroid_is_rounded_exact_mean():
     assert np.all(C[7] == 0)          # empty cluster keeps its centroid
 
 
-def test_lloyd_recovers_separated_mixture_labels():
+def test_lloyd_recovers_planted_clusters():
+    # Plant 16 generator centres far apart (pairwise distance >= 8) with noise of
+    # norm < 1, and give the token at the i-th seeded init index generator i, so
+    # that every generator holds one init pick. Lloyd must then label every token
+    # with its own generator's pick after the first pass and keep that labelling,
+    # and the centroids must be the generators' exact member means (fp32-rounded).
+    S, k, D, seed, bh = 3000, 16, 128, 5, 2
+    init = O.kmeans_init_indices(S, k, seed, bh)
+    rng = np.random.default_rng(11)
+    centres = np.zeros((k, D))
+    for i in range(k):
+        centres[i, 8 * i: 8 * i + 8] = 4.0 * (1 + (i % 3))     # disjoint supports: |c_i - c_j| >= 8
+    gen = rng.integers(0, k, S)
+    gen[np.asarray(init)] = np.arange(k)
+    noise = rng.standard_normal((S, D))
+    noise *= (0.9 * rng.random(S) / np.linalg.norm(noise, axis=1))[:, None]
+    X = (centres[gen] + noise).astype(np.float32)
+    X = torch.from_numpy(X).to(torch.bfloat16).float().numpy()
+    X[np.abs(X) < 2.0 ** -16] = 0.0                   # on the fixed-point grid: exact sums
+    a, C, hist, stats = O.kmeans_lloyd(X, k, 4, seed, bh)
+    for h in hist:
+        assert np.array_equal(h, gen)
+    for i in range(k):
+        mem = X[gen == i]
+        for e in (0, 8 * i, 8 * i + 7, 127):
+            exact = sum(Fraction(float(v)) for v in mem[:, e]) / len(mem)
+            assert C[i, e] == np.float32(float(exact))
+
+
+def test_lloyd_objective_does_not_increase():
+    # Lloyd's two steps each lower sum_j |x_j - c_a(j)|^2 (exact means; here the
+    # means are rounded to fp32, so allow a relative 1e-6 per pass).
     cfg, Q, K, V = synth.make_workload("mid", B=1, H=1, S=2048)
     X = V[0, :, 0].float().numpy()
-    a, C, hist, stats = O.kmeans_lloyd(X, 16, 4, 0, 0)
-    # each found cluster should be dominated by one generator centre: measure the
-    # purity against a nearest-centre labelling of the (outlier-free) tokens
-    norms = np.linalg.norm(X, axis=1)
-    keep = norms < np.percentile(norms, 95)
-    # tokens of the same found cluster are close together
-    spread = [np.mean(np.linalg.norm(X[keep & (a == c)] - C[c], axis=1)) for c in range(16)
-              if (keep & (a == c)).sum() > 5]
-    assert np.median(spread) < 0.3 * np.sqrt(128) * 1.5
+    a, C, hist, stats = O.kmeans_lloyd(X, 16, 6, 0, 0)
+    X64 = X.astype(np.float64)
+    Cs = [X[O.kmeans_init_indices(2048, 16, 0, 0)].astype(np.float64)]
+    Xfix = np.rint(X64 * 2.0 ** 24).astype(np.int64)
+    for h in hist[:-1]:
+        Cs.append(O.centroid_update(Xfix, h, Cs[-1].astype(np.float32), 16).astype(np.float64))
+    J = [np.sum((X64 - Cs[t][h]) ** 2) for t, h in enumerate(hist)]
+    for j0, j1 in zip(J, J[1:]):
+        assert j1 <= j0 * (1 + 1e-6)
+    assert J[-1] < J[0]
+    # the final centroids are the ones the last pass assigned against
+    assert np.array_equal(Cs[-1].astype(np.float32), C)
 
 
 def test_permutation_is_stable_sort():
