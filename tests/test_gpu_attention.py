@@ -42,7 +42,10 @@ def test_attention_tiny_all_rows(va):
     _check_all_heads(va, cfg, Q, K, V)
 
 
-@pytest.mark.parametrize("S", [128, 129, 700, 1000])
+# 1 and 5: a single partial block; 128: one full block (the pair's second tile is
+# past the end); 257: an odd block count with a one-token tail; 641: one mean
+# batch in the loop and a one-block batch after it
+@pytest.mark.parametrize("S", [1, 5, 128, 129, 257, 641, 700, 1000])
 def test_attention_ragged(va, S):
     cfg, Q, K, V = make("mid", B=1, H=2, S=S)
     _check_all_heads(va, cfg, Q, K, V)
@@ -66,7 +69,7 @@ def test_attention_nvfp4_tiny_all_rows(va):
     _check_all_heads(va, cfg, Q, K, V, fmt="nvfp4")
 
 
-@pytest.mark.parametrize("S", [129, 700, 1000])
+@pytest.mark.parametrize("S", [1, 129, 257, 700, 1000])
 def test_attention_nvfp4_ragged(va, S):
     cfg, Q, K, V = make("mid", B=1, H=2, S=S)
     _check_all_heads(va, cfg, Q, K, V, fmt="nvfp4")

@@ -46,7 +46,8 @@ def _check(va, cfg, Q, K, V, fmt, rows=None, k_p=8, elementwise=True):
 
 
 @pytest.mark.parametrize("fmt", ["e4m3c", "mxfp4"])
-@pytest.mark.parametrize("name,kw", [("tiny", {}), ("mid", dict(B=1, H=2, S=1000)), ("mid", dict(B=2, H=1, S=129))])
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("mid", dict(B=1, H=2, S=1000)), ("mid", dict(B=2, H=1, S=129)),
+                                     ("mid", dict(B=1, H=1, S=5)), ("mid", dict(B=1, H=2, S=641))])
 def test_format_prep_and_output(va, fmt, name, kw):
     # full and ragged tiles (1000 = 7 blocks + 104; 129 = one block + 1 token)
     cfg, Q, K, V = make(name, **kw)
