@@ -374,7 +374,8 @@ vc_status_t vc_attn_quant_qk(const void* q, const void* k, const vc_shape_t* sha
 
 size_t vc_attn_quant_qk_smoothk_workspace_bytes(const vc_shape_t* shape) {
   if (check_shape(shape) != VC_OK) return 0;
-  return sizeof(unsigned long long) * (size_t)shape->B * shape->H * 128;
+  // the int64 token sums, then the fp32 means
+  return (sizeof(unsigned long long) + sizeof(float)) * (size_t)shape->B * shape->H * 128;
 }
 
 vc_status_t vc_attn_quant_qk_smoothk(const void* q, const void* k, const vc_shape_t* shape, const int32_t* perm,

@@ -1487,6 +1487,17 @@ __global__ void __launch_bounds__(128) token_sums_kernel(const T* __restrict__ x
   atomicAdd(&sums[(size_t)bh * kD + d], (unsigned long long)t);
 }
 
+// kbar[bh][d] = fl32((sum * 2^-24) / S) from the token sums, once per (b, h) and
+// channel (one fp64 division each); also into k_mean when that is given.
+__global__ void __launch_bounds__(128) kbar_kernel(const unsigned long long* __restrict__ sums, int S,
+                                                   float* __restrict__ kbar, float* __restrict__ k_mean) {
+  const size_t i = (size_t)blockIdx.x * kD + threadIdx.x;
+  const long long sum = (long long)sums[i];
+  const float m = __double2float_rn(__ddiv_rn((double)sum * 5.9604644775390625e-08, (double)S));
+  kbar[i] = m;
+  if (k_mean != nullptr) k_mean[i] = m;
+}
+
 // --------------------------------------------------------------- Q/K quantisation
 // One CTA (8 warps) = one 128-row block of Q (original order) or K (gathered by
 // perm). Warp w takes rows 16w .. 16w+15, two rows per load: lanes 0-15 read row
@@ -1494,18 +1505,16 @@ __global__ void __launch_bounds__(128) token_sums_kernel(const T* __restrict__ x
 // whole 256-byte rows. The values stay in registers while the block amax is
 // reduced (warp shuffles, then shared memory); each lane then writes the 8 E4M3
 // codes of its 8 values (rows of 128 codes, contiguous per half warp).
-// With ksum (K smoothing: the per-channel int64 fixed-point token sums of K),
-// the K CTAs first subtract kbar = fl32((sum * 2^-24) / S) from every valid row
-// (an fp32 subtraction; padding rows stay 0), and the first block's CTA writes
-// kbar to k_mean when that is given (a separate instantiation, so that the
-// plain one keeps its register count and occupancy).
+// With kbar (K smoothing: the per-channel token mean of K made by kbar_kernel),
+// the K CTAs first subtract kbar from every valid row (an fp32 subtraction;
+// padding rows stay 0) (a separate instantiation, so that the plain one keeps its
+// register count and occupancy).
 template <typename T, bool kSmooth>
-__global__ void __launch_bounds__(256) quant_qk_kernel(const T* __restrict__ q, const T* __restrict__ k, int S,
+__global__ void __launch_bounds__(256, 3) quant_qk_kernel(const T* __restrict__ q, const T* __restrict__ k, int S,
                                                        int H, int S_pad, const int32_t* __restrict__ perm,
-                                                       const unsigned long long* __restrict__ ksum,
+                                                       const float* __restrict__ kbar,
                                                        uint8_t* __restrict__ qc, float* __restrict__ qs,
-                                                       uint8_t* __restrict__ kc, float* __restrict__ ks,
-                                                       float* __restrict__ k_mean) {
+                                                       uint8_t* __restrict__ kc, float* __restrict__ ks) {
   __shared__ float wmax[8];
   const int bh = blockIdx.y, b = bh / H, h = bh % H, blk = blockIdx.x;
   const bool is_k = blockIdx.z == 1;
@@ -1527,15 +1536,10 @@ __global__ void __launch_bounds__(256) quant_qk_kernel(const T* __restrict__ q, 
                        : make_uint4(0u, 0u, 0u, 0u);
   float kb[8];
   if (smooth) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const long long sum = (long long)ksum[(size_t)bh * kD + c * 8 + e];
-      kb[e] = __double2float_rn(__ddiv_rn((double)sum * 5.9604644775390625e-08, (double)S));
-    }
-    if (k_mean != nullptr && blk == 0 && warp == 0 && half == 0) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) k_mean[(size_t)bh * kD + c * 8 + e] = kb[e];
-    }
+    const float4* m4 = reinterpret_cast<const float4*>(kbar + (size_t)bh * kD + c * 8);
+    const float4 m0 = __ldg(m4), m1 = __ldg(m4 + 1);
+    kb[0] = m0.x, kb[1] = m0.y, kb[2] = m0.z, kb[3] = m0.w;
+    kb[4] = m1.x, kb[5] = m1.y, kb[6] = m1.z, kb[7] = m1.w;
   }
   // the values of row i (K smoothed when asked; rows past S are 0)
   auto values = [&](int i, float* f) {
@@ -1948,6 +1952,9 @@ cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int 
   const dim3 grid(nb, B * H, 2);
   const bool bf = dtype == VC_DTYPE_BF16;
   int n = 1;
+  // K smoothing: the token sums, then the means (fp32, right after the sums in
+  // the same workspace)
+  float* const kbar = ksum != nullptr ? reinterpret_cast<float*>(ksum + (size_t)B * H * kD) : nullptr;
   if (ksum != nullptr) {
     cudaError_t e;
     if ((e = cudaMemsetAsync(ksum, 0, sizeof(unsigned long long) * B * H * kD, st)) != cudaSuccess) return e;
@@ -1956,17 +1963,18 @@ cudaError_t launch_quant_qk(const void* q, const void* k, int dtype, int B, int 
       token_sums_kernel<__nv_bfloat16><<<gs, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(k), S, H, ksum);
     else
       token_sums_kernel<__half><<<gs, 128, 0, st>>>(static_cast<const __half*>(k), S, H, ksum);
-    ++n;
+    kbar_kernel<<<B * H, kD, 0, st>>>(ksum, S, kbar, k_mean);
+    n += 2;
   }
   auto qk = bf ? (ksum ? quant_qk_kernel<__nv_bfloat16, true> : quant_qk_kernel<__nv_bfloat16, false>)
               : nullptr;
   auto qh = bf ? nullptr : (ksum ? quant_qk_kernel<__half, true> : quant_qk_kernel<__half, false>);
   if (bf)
     qk<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), S, H,
-                             nb * kBlock, perm, ksum, out.q_codes, out.q_scales, out.k_codes, out.k_scales, k_mean);
+                             nb * kBlock, perm, kbar, out.q_codes, out.q_scales, out.k_codes, out.k_scales);
   else
     qh<<<grid, 256, 0, st>>>(static_cast<const __half*>(q), static_cast<const __half*>(k), S, H, nb * kBlock, perm,
-                             ksum, out.q_codes, out.q_scales, out.k_codes, out.k_scales, k_mean);
+                             kbar, out.q_codes, out.q_scales, out.k_codes, out.k_scales);
   *nlaunch = n;
   return cudaGetLastError();
 }

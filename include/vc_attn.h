@@ -233,8 +233,8 @@ vc_status_t vc_attn_forward_repair(const vc_qk_fp8_t* qk, const vc_prepared_v_t*
                                    float softmax_scale, int32_t k_p, void* o, int32_t* dev_status,
                                    void* stream);
 
-/* Bytes of device workspace vc_attn_quant_qk_smoothk needs: B*H*128*8 (0 for an
- * invalid shape). */
+/* Bytes of device workspace vc_attn_quant_qk_smoothk needs: B*H*128*12 (the
+ * int64 token sums and the fp32 means; 0 for an invalid shape). */
 size_t vc_attn_quant_qk_smoothk_workspace_bytes(const vc_shape_t* shape);
 
 /* Q/K FP8 quantisation with K smoothing ("VC-Attention ...", Abstract: prior

@@ -163,13 +163,13 @@ def test_residual_energy_validation(lib):
 
 def test_quant_qk_smoothk_workspace_and_validation(lib):
     sh = _shape(B=2, S=1000, H=5)
-    assert lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(sh)) == 2 * 5 * 128 * 8
+    assert lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(sh)) == 2 * 5 * 128 * 12
     assert lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(_shape(D=64))) == 0
     buf = (ctypes.c_uint8 * 64)()
     p = ctypes.cast(buf, ctypes.c_void_p)
     qk = vc_attn.QKFP8(p, p, p, p)
     odd = ctypes.c_void_p(p.value + 4)
-    need = 2 * 5 * 128 * 8
+    need = 2 * 5 * 128 * 12
     for args, code in (
         ((p, p, ctypes.byref(sh), p, ctypes.byref(qk), None, need, None, None), vc_attn.VC_ERR_WORKSPACE),
         ((p, p, ctypes.byref(sh), p, ctypes.byref(qk), p, need - 1, None, None), vc_attn.VC_ERR_WORKSPACE),
@@ -195,7 +195,7 @@ def test_too_many_slices_is_refused_before_any_launch(lib):
     assert lib.vc_attn_residual_energy(p, ctypes.byref(sh), None, None, p, None) == vc_attn.VC_ERR_UNSUPPORTED
     assert b"65535" in lib.vc_attn_last_error()
     ok = _shape(B=1, S=100, H=65535)
-    assert lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(ok)) == 65535 * 128 * 8
+    assert lib.vc_attn_quant_qk_smoothk_workspace_bytes(ctypes.byref(ok)) == 65535 * 128 * 12
 
 
 def test_prepare_v_repair_workspace_and_validation(lib):
