@@ -52,6 +52,10 @@ def load():
         lib.orc_residual_e4m3.argtypes = [P, i32, i32, P, P, P, P, P]
         lib.orc_residual_nvfp4.argtypes = [P, i32, i32, P, P, P, P, P, P]
         lib.orc_vres_from_e4m3.argtypes = [P, i32, i32, i32, f32, P]
+        lib.orc_residual_e4m3_per_channel.argtypes = [P, i32, i32, P, P, P, P, P]
+        lib.orc_mx_exponent.argtypes = [ctypes.c_double]
+        lib.orc_mx_exponent.restype = i32
+        lib.orc_residual_mxfp4.argtypes = [P, i32, i32, P, P, P, P]
         lib.orc_quant_blocks_e4m3.argtypes = [P, i32, i32, P, P, P]
         lib.orc_softmax_kappa.argtypes = [f32]
         lib.orc_softmax_kappa.restype = f32
@@ -141,6 +145,29 @@ def residual_nvfp4(X, perm, mu):
     g, amax = np.empty(1, np.float32), np.empty(1, np.float32)
     load().orc_residual_nvfp4(_p(X), S, D, _p(perm), _p(mu), _p(packed), _p(scales), _p(g), _p(amax))
     return packed, scales, np.float32(g[0]), np.float32(amax[0])
+
+
+def residual_e4m3_per_channel(X, perm, mu):
+    X, perm, mu = _f32(X), _i32(perm), _f32(mu)
+    S, D = X.shape
+    vt = np.empty((D, nblocks(S) * 128), np.uint8)
+    s_v, amax = np.empty(D, np.float32), np.empty(D, np.float32)
+    load().orc_residual_e4m3_per_channel(_p(X), S, D, _p(perm), _p(mu), _p(vt), _p(s_v), _p(amax))
+    return vt, s_v, amax
+
+
+def mx_exponent(amax):
+    return int(load().orc_mx_exponent(float(amax)))
+
+
+def residual_mxfp4(X, perm, mu):
+    X, perm, mu = _f32(X), _i32(perm), _f32(mu)
+    S, D = X.shape
+    Sp = nblocks(S) * 128
+    codes = np.empty((D, Sp), np.uint8)
+    e8 = np.empty((D, Sp // 32), np.uint8)
+    load().orc_residual_mxfp4(_p(X), S, D, _p(perm), _p(mu), _p(codes), _p(e8))
+    return codes, e8
 
 
 def vres_from_e4m3(vt, s_v, S):

@@ -1,7 +1,7 @@
 // vc_oracle_ref.cpp -- the VC-Attention forward path written out plainly in C++.
 //
 // TEST INFRASTRUCTURE ONLY, like the numpy oracle beside it: a second, independent
-// CPU statement of the same definitions (readings R1-R10 of the oracle package),
+// CPU statement of the same definitions (readings R1-R10, R13 and R14 of the oracle package),
 // which the tests hold bit for bit against the numpy oracle. Only tests/, the
 // smoke test and the benchmark's CPU baseline may load it; it shares no code with
 // the CUDA library. Plain loops, one (batch, head) slice at a time, in the order
@@ -283,6 +283,63 @@ void orc_residual_nvfp4(const float* X, int S, int D, const int* perm, const flo
         const float r = p < S ? residual(X, D, perm, mu, p, d) : 0.0f;
         const uint8_t code = sdec == 0.0f ? 0 : e2m1_code(r / den);
         packed[(size_t)d * (Sp / 2) + p / 2] |= (uint8_t)((p & 1) ? code << 4 : code);
+      }
+    }
+}
+
+// R14: E4M3 residual with one scale per channel: s_v[d] = fl32(amax_d / 448), codes
+// E4M3(fl32(r fl32(448 / amax_d))); a channel below 2^-100 keeps scale 1, codes 0.
+void orc_residual_e4m3_per_channel(const float* X, int S, int D, const int* perm, const float* mu, uint8_t* vt,
+                                   float* s_v, float* amax) {
+  const int Sp = num_blocks(S) * kBlock;
+  memset(vt, 0, (size_t)D * Sp);
+  for (int d = 0; d < D; ++d) {
+    float a = 0.0f;
+    for (int p = 0; p < S; ++p) {
+      const float v = fabsf(residual(X, D, perm, mu, p, d));
+      if (v > a) a = v;
+    }
+    amax[d] = a;
+    s_v[d] = 1.0f;
+    if (!(a >= kTinyAmax)) continue;
+    const float inv = (float)kE4M3Max / a;
+    s_v[d] = a / (float)kE4M3Max;
+    for (int p = 0; p < S; ++p) vt[(size_t)d * Sp + p] = e4m3_code(residual(X, D, perm, mu, p, d) * inv);
+  }
+}
+
+// R13: the exponent of an MX group: the smallest integer e with amax <= 6 2^e,
+// clamped to [-127, 127]; -127 for an all-zero group.
+int orc_mx_exponent(double amax) {
+  if (!(amax > 0.0)) return -127;
+  int e = -127;
+  while (e < 127 && kE2M1Max * ldexp(1.0, e) < amax) ++e;
+  return e;
+}
+
+// R13: MX-style FP4 residual: per channel and group of 32 permuted tokens the
+// exponent e of the group's amax, codes E2M1(fl32(r / 2^e)) (exact division by a
+// power of two); codes (D x S_pad) one per byte, exponents (D x S_pad/32) as e + 127.
+void orc_residual_mxfp4(const float* X, int S, int D, const int* perm, const float* mu, uint8_t* codes,
+                        uint8_t* e8) {
+  const int Sp = num_blocks(S) * kBlock, ng = Sp / 32;
+  memset(codes, 0, (size_t)D * Sp);
+  for (int d = 0; d < D; ++d)
+    for (int q = 0; q < ng; ++q) {
+      double gmax = 0.0;
+      for (int i = 0; i < 32; ++i) {
+        const int p = q * 32 + i;
+        if (p < S) {
+          const double a = fabs((double)residual(X, D, perm, mu, p, d));
+          if (a > gmax) gmax = a;
+        }
+      }
+      const int e = orc_mx_exponent(gmax);
+      e8[(size_t)d * ng + q] = (uint8_t)(e + 127);
+      for (int i = 0; i < 32; ++i) {
+        const int p = q * 32 + i;
+        const double r = p < S ? (double)residual(X, D, perm, mu, p, d) : 0.0;
+        codes[(size_t)d * Sp + p] = e2m1_code((float)(r / ldexp(1.0, e)));
       }
     }
 }

@@ -76,6 +76,12 @@ def test_prep_steps_bit_exact(name, kw, h):
     pk_c, sc_c, g_c, _ = C.residual_nvfp4(V, perm, mu)
     pk_o, sc_o, g_o, _ = O.residual_nvfp4(V, perm, mu)
     assert np.array_equal(pk_c, pk_o) and np.array_equal(sc_c, sc_o) and g_c == g_o
+    vt_c, sv_c, am_c = C.residual_e4m3_per_channel(V, perm, mu)
+    vt_o, sv_o, am_o = O.residual_e4m3_per_channel(V, perm, mu)
+    assert np.array_equal(vt_c, vt_o) and np.array_equal(sv_c.view(np.uint32), sv_o.view(np.uint32))
+    cd_c, e8_c = C.residual_mxfp4(V, perm, mu)
+    cd_o, e8_o = O.residual_mxfp4(V, perm, mu)
+    assert np.array_equal(cd_c, cd_o) and np.array_equal(e8_c, e8_o)
     for X, order in ((Q, None), (K, perm)):
         cc, scc = C.quant_blocks_e4m3(X, order)
         co, sco = O.quant_blocks_e4m3(X, order)
@@ -93,6 +99,16 @@ def test_zero_slice_and_zero_block():
     cc, scc = C.quant_blocks_e4m3(X)
     co, sco = O.quant_blocks_e4m3(X)
     assert np.array_equal(cc, co) and np.array_equal(scc, sco)
+
+
+def test_mx_exponent_boundaries():
+    vals = [0.0, 6.0 * 2.0 ** -127, 6.0 * 2.0 ** -130, 6.0 * 2.0 ** 127, 6.0 * 2.0 ** 130, 1e-45, 3.0, 6.0, 6.000001,
+            12.0, 12.5, 0.75, 0.7499999]
+    for e in range(-20, 21):
+        b = 6.0 * 2.0 ** e
+        vals += [b, np.nextafter(b, 0.0), np.nextafter(b, np.inf)]
+    for v in vals:
+        assert C.mx_exponent(v) == O.mx_exponent(v), v
 
 
 def test_kappa():
