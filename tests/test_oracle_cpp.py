@@ -8,7 +8,6 @@ import math
 
 import numpy as np
 import pytest
-import torch
 
 import oracle as O
 from oracle import ref_cpp as C
