@@ -370,10 +370,12 @@ constexpr size_t assign_smem() {
 // g_c - e_c exceeds g_b + e_b, b the smallest proxy, is farther than b. Any other
 // centroid is a candidate. b and its candidates are then compared by the squared
 // distance sum_d (x_d - c_d)^2 in fp32 (all terms positive: the rounding of the
-// differences, squares and 128-term sum stays within 2^-16 of the distance
-// itself), and those still within that bound of the nearest once more in fp64
-// (differences exact, squares rounded at 2^-53), the lowest index winning ties:
-// the exact argmin but for ties below fp64 rounding.
+// differences, squares and 128-term sum, in any order, stays within 2^-16 of the
+// distance itself; the whole warp makes one such token's distances, four
+// dimensions a lane), and those still within that bound of the nearest once more
+// in fp64 by the token's own thread (differences exact, squares rounded at
+// 2^-53), the lowest index winning ties: the exact argmin but for ties below fp64
+// rounding.
 constexpr int kTcWarps = 10, kTcThreads = kTcWarps * 32;
 constexpr int kTcTmaWarp = 8, kTcMmaWarp = 9;
 constexpr int kTcDStages = 4;                  // tensor-memory dot stages (two per token-warp group)
@@ -637,50 +639,61 @@ __global__ void __launch_bounds__(kTcThreads, 1) kmeans_assign_tc_kernel(const _
         const float e = fmaf(0x1p-19f, nrm[c], xs * nrm[KC + c]);
         if (c < k && c != best && !(gv[c] - e > lim)) cand |= 1u << c;
       }
-      if (cand != 0u) {
-        // direct squared distances of the best proxy and its candidates: fp32
-        // first (even and odd dimensions in the two halves of a packed
-        // accumulator), fp64 for those the fp32 bound cannot separate
-        cand |= 1u << best;
-        float dd[KC];
-        float dmin = __int_as_float(0x7f800000);
-        int bmin = -1;
+      // Near ties: the best proxy and its candidates by their direct squared
+      // distances. The fp32 distances of a token are made by the whole warp (four
+      // dimensions a lane, the partial sums added by shuffles), one such token
+      // after another, so that a lane's near tie does not hold the other 31 lanes
+      // for its serial 128-term sums. The fp32 values only set aside the centroids
+      // clearly farther than the nearest (any order of adding the positive terms
+      // stays within 2^-16 of the distance); those still within that bound are
+      // compared in fp64 by the token's own thread, dimension after dimension, the
+      // lowest index winning ties.
+      const uint32_t cm_own = cand != 0u ? (cand | (1u << best)) : 0u;
+      uint32_t close_own = 0u;
+      int bmin_own = best;
+      {
+        const int jx = lane >> 1;                          // piece of the lane's four dimensions
+        const uint8_t* const xbase = (jx < 8 ? arow0 : arow1) + (lane & 1) * 8;
 #pragma unroll 1
-        for (uint32_t m = cand; m != 0u; m &= m - 1u) {
-          const int c = __ffs(m) - 1;
-          float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 2
-          for (int j = 0; j < 16; ++j) {
-            float f[8];
-            piece(j, f);
-            const float4* cc = reinterpret_cast<const float4*>(cg + c * kD + 8 * j);
-            const float4 p0 = __ldg(cc), p1 = __ldg(cc + 1);
-            const float2 d0 = __fadd2_rn(make_float2(f[0], f[1]), make_float2(-p0.x, -p0.y));
-            const float2 d1 = __fadd2_rn(make_float2(f[2], f[3]), make_float2(-p0.z, -p0.w));
-            const float2 d2 = __fadd2_rn(make_float2(f[4], f[5]), make_float2(-p1.x, -p1.y));
-            const float2 d3 = __fadd2_rn(make_float2(f[6], f[7]), make_float2(-p1.z, -p1.w));
-            acc = __ffma2_rn(d0, d0, acc);
-            acc = __ffma2_rn(d1, d1, acc);
-            acc = __ffma2_rn(d2, d2, acc);
-            acc = __ffma2_rn(d3, d3, acc);
+        for (uint32_t todo = __ballot_sync(0xffffffffu, cand != 0u); todo != 0u; todo &= todo - 1u) {
+          const int src = __ffs(todo) - 1;
+          const uint32_t cm = __shfl_sync(0xffffffffu, cm_own, src);
+          float xf[4];
+          unpack4<__nv_bfloat16>(*reinterpret_cast<const uint2*>(xbase + sw128_off((warp & 3) * 32 + src, jx & 7)), xf);
+          float dd[KC];
+          float dmin = __int_as_float(0x7f800000);
+          int bmin = -1;
+#pragma unroll 1
+          for (uint32_t m = cm; m != 0u; m &= m - 1u) {
+            const int c = __ffs(m) - 1;
+            const float4 cc = __ldg(reinterpret_cast<const float4*>(cg + c * kD + 4 * lane));
+            const float d0 = xf[0] - cc.x, d1 = xf[1] - cc.y, d2 = xf[2] - cc.z, d3 = xf[3] - cc.w;
+            float part = (d0 * d0 + d1 * d1) + (d2 * d2 + d3 * d3);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+#pragma unroll
+            for (int q = 0; q < KC; ++q)
+              if (q == c) dd[q] = part;
+            if (bmin < 0 || part < dmin) {
+              dmin = part;
+              bmin = c;
+            }
           }
-          const float dc = acc.x + acc.y;
+          uint32_t close = 0u;   // within the fp32 bound of the nearest
 #pragma unroll
           for (int q = 0; q < KC; ++q)
-            if (q == c) dd[q] = dc;
-          if (bmin < 0 || dc < dmin) {
-            dmin = dc;
-            bmin = c;
+            if (((cm >> q) & 1u) && q != bmin && !(dd[q] - 0x1p-16f * dd[q] > dmin + 0x1p-16f * dmin))
+              close |= 1u << q;
+          if (lane == src) {
+            bmin_own = bmin;
+            close_own = close;
           }
         }
-        uint32_t close = 0u;   // within the fp32 bound of the nearest
-#pragma unroll
-        for (int q = 0; q < KC; ++q)
-          if (((cand >> q) & 1u) && q != bmin && !(dd[q] - 0x1p-16f * dd[q] > dmin + 0x1p-16f * dmin))
-            close |= 1u << q;
-        best = bmin;
-        if (close != 0u) {
-          close |= 1u << bmin;
+      }
+      if (cand != 0u) {
+        best = bmin_own;
+        if (close_own != 0u) {
+          uint32_t close = close_own | (1u << bmin_own);
           double bd = 0.0;
           best = -1;
 #pragma unroll 1
