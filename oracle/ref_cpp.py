@@ -56,6 +56,10 @@ def load():
         lib.orc_mx_exponent.argtypes = [ctypes.c_double]
         lib.orc_mx_exponent.restype = i32
         lib.orc_residual_mxfp4.argtypes = [P, i32, i32, P, P, P, P]
+        lib.orc_residual_repair_planes.argtypes = [P, i32, i32, P, P, ctypes.c_double, P, P, P, P]
+        lib.orc_residual_repair_planes.restype = i32
+        lib.orc_residual_energy.argtypes = [P, i32, i32, P, P]
+        lib.orc_residual_energy.restype = ctypes.c_double
         lib.orc_quant_blocks_e4m3.argtypes = [P, i32, i32, P, P, P]
         lib.orc_softmax_kappa.argtypes = [f32]
         lib.orc_softmax_kappa.restype = f32
@@ -168,6 +172,26 @@ def residual_mxfp4(X, perm, mu):
     e8 = np.empty((D, Sp // 32), np.uint8)
     load().orc_residual_mxfp4(_p(X), S, D, _p(perm), _p(mu), _p(codes), _p(e8))
     return codes, e8
+
+
+def residual_repair_planes(X, perm, mu, budget):
+    """Returns (kept positions ascending, plane 0 (D, S_pad), plane 1 (D, S_pad), s_v)."""
+    X, perm, mu = _f32(X), _i32(perm), _f32(mu)
+    S, D = X.shape
+    Sp = nblocks(S) * 128
+    vt = np.empty((D, Sp), np.uint8)
+    lo = np.empty((D, Sp), np.uint8)
+    s_v = np.empty(1, np.float32)
+    pos = np.empty(max(S, 1), np.int32)
+    m = load().orc_residual_repair_planes(_p(X), S, D, _p(perm), _p(mu), float(budget), _p(vt), _p(lo), _p(s_v),
+                                         _p(pos))
+    return pos[:m].copy(), vt, lo, np.float32(s_v[0])
+
+
+def residual_energy(X, perm, mu):
+    X, perm, mu = _f32(X), _i32(perm), _f32(mu)
+    S, D = X.shape
+    return float(load().orc_residual_energy(_p(X), S, D, _p(perm), _p(mu)))
 
 
 def vres_from_e4m3(vt, s_v, S):

@@ -1,7 +1,7 @@
 // vc_oracle_ref.cpp -- the VC-Attention forward path written out plainly in C++.
 //
 // TEST INFRASTRUCTURE ONLY, like the numpy oracle beside it: a second, independent
-// CPU statement of the same definitions (readings R1-R10, R13 and R14 of the oracle package),
+// CPU statement of the same definitions (readings R1-R10 and R12-R14 of the oracle package),
 // which the tests hold bit for bit against the numpy oracle. Only tests/, the
 // smoke test and the benchmark's CPU baseline may load it; it shares no code with
 // the CUDA library. Plain loops, one (batch, head) slice at a time, in the order
@@ -25,6 +25,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <vector>
 
 namespace {
@@ -342,6 +343,59 @@ void orc_residual_mxfp4(const float* X, int S, int D, const int* perm, const flo
         codes[(size_t)d * Sp + p] = e2m1_code((float)(r / ldexp(1.0, e)));
       }
     }
+}
+
+// R12: the repair planes of an E4M3 residual. Plane 0 is the residual's codes
+// (R5); for the ceil(budget S) tokens with the largest error, plane 1 holds the
+// E4M3 codes of each element's rounding error in code units, dlt = fl32(y -
+// dec(code)) with y = fl32(r fl32(448 / amax)); a token's error is the fp32 sum
+// of fl32(dlt^2) over the channels from d = 0; ties go to the lower position.
+// pos receives the kept positions in ascending order; returns their number.
+int orc_residual_repair_planes(const float* X, int S, int D, const int* perm, const float* mu, double budget,
+                               uint8_t* vt, uint8_t* lo, float* s_v, int* pos) {
+  const int Sp = num_blocks(S) * kBlock;
+  float amax = 0.0f;
+  orc_residual_e4m3(X, S, D, perm, mu, vt, s_v, &amax);
+  memset(lo, 0, (size_t)D * Sp);
+  double mm = ceil(budget * (double)S);
+  const int m = mm < (double)S ? (int)mm : S;
+  std::vector<float> err(S, 0.0f);
+  std::vector<float> dlt((size_t)S * D, 0.0f);
+  if (amax >= kTinyAmax) {
+    const float inv = (float)kE4M3Max / amax;
+    for (int p = 0; p < S; ++p) {
+      float e = 0.0f;
+      for (int d = 0; d < D; ++d) {
+        const float y = residual(X, D, perm, mu, p, d) * inv;
+        const float dl = y - (float)e4m3_value(vt[(size_t)d * Sp + p]);
+        dlt[(size_t)p * D + d] = dl;
+        e = e + dl * dl;
+      }
+      err[p] = e;
+    }
+  }
+  std::vector<int> order(S);
+  for (int p = 0; p < S; ++p) order[p] = p;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return err[a] > err[b]; });
+  std::sort(order.begin(), order.begin() + m);
+  for (int i = 0; i < m; ++i) {
+    const int p = order[i];
+    pos[i] = p;
+    for (int d = 0; d < D; ++d) lo[(size_t)d * Sp + p] = e4m3_code(dlt[(size_t)p * D + d]);
+  }
+  return m;
+}
+
+// Residual energy of one slice: sum over permuted positions p of
+// ||x[perm[p]] - mu[p / 128]||^2 in fp64.
+double orc_residual_energy(const float* X, int S, int D, const int* perm, const float* mu) {
+  double e = 0.0;
+  for (int p = 0; p < S; ++p)
+    for (int d = 0; d < D; ++d) {
+      const double r = (double)X[(size_t)perm[p] * D + d] - (double)mu[(p / kBlock) * D + d];
+      e += r * r;
+    }
+  return e;
 }
 
 // Decoded E4M3 residual (S x D, fp64, permuted order): s_v dec(code).

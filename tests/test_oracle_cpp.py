@@ -87,6 +87,19 @@ def test_prep_steps_bit_exact(name, kw, h):
         assert np.array_equal(cc, co) and np.array_equal(scc.view(np.uint32), sco.view(np.uint32))
 
 
+@pytest.mark.parametrize("budget", [0.0, 0.005, 0.05, 1.0])
+def test_repair_planes_and_energy(budget):
+    cfg, Q, K, V = _slice("mid", B=1, H=1, S=1000)
+    ref = O.prepare_v_head(V, cfg["k"], cfg["iters"], 0, 0)
+    perm, mu = ref["perm"], ref["mu"]
+    pos_c, vt_c, lo_c, sv_c = C.residual_repair_planes(V, perm, mu, budget)
+    pos_o, vt_o, lo_o, sv_o, _ = O.residual_repair_planes(V, perm, mu, budget)
+    assert np.array_equal(pos_c, pos_o) and np.array_equal(vt_c, vt_o) and np.array_equal(lo_c, lo_o)
+    assert sv_c == sv_o
+    e_c, e_o = C.residual_energy(V, perm, mu), O.residual_energy(V, perm, mu)
+    assert abs(e_c - e_o) <= 1e-12 * e_o
+
+
 def test_zero_slice_and_zero_block():
     X = np.zeros((300, 128), np.float32)
     X[200:, 5] = 1.0          # blocks 0 and 1 all zero, block 2 not
