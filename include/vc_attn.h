@@ -46,7 +46,7 @@ extern "C" {
 typedef enum {
   VC_OK = 0,
   VC_ERR_INVALID_ARG = 1,   /* a shape, pointer, alignment or config is invalid   */
-  VC_ERR_UNSUPPORTED = 2,   /* valid but not supported by this build / device     */
+  VC_ERR_UNSUPPORTED = 2,   /* valid but not supported by the library or device  */
   VC_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required         */
   VC_ERR_CUDA = 4,          /* a CUDA runtime / driver call failed                */
   VC_ERR_TIMEOUT = 5        /* device side: a bounded wait in a kernel ran out    */
