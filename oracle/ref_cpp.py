@@ -60,6 +60,7 @@ def load():
         lib.orc_residual_repair_planes.restype = i32
         lib.orc_residual_energy.argtypes = [P, i32, i32, P, P]
         lib.orc_residual_energy.restype = ctypes.c_double
+        lib.orc_smooth_k.argtypes = [P, i32, i32, P, P]
         lib.orc_quant_blocks_e4m3.argtypes = [P, i32, i32, P, P, P]
         lib.orc_softmax_kappa.argtypes = [f32]
         lib.orc_softmax_kappa.restype = f32
@@ -210,6 +211,16 @@ def quant_blocks_e4m3(X, order=None):
     o = _i32(order) if order is not None else None
     load().orc_quant_blocks_e4m3(_p(X), S, D, _p(o), _p(codes), _p(scales))
     return codes, scales
+
+
+def smooth_k(K):
+    """Returns (K - kbar, kbar)."""
+    K = _f32(K)
+    S, D = K.shape
+    kbar = np.empty(D, np.float32)
+    xs = np.empty((S, D), np.float32)
+    load().orc_smooth_k(_p(K), S, D, _p(kbar), _p(xs))
+    return xs, kbar
 
 
 def softmax_kappa(softmax_scale):

@@ -1,7 +1,7 @@
 // vc_oracle_ref.cpp -- the VC-Attention forward path written out plainly in C++.
 //
 // TEST INFRASTRUCTURE ONLY, like the numpy oracle beside it: a second, independent
-// CPU statement of the same definitions (readings R1-R10 and R12-R14 of the oracle package),
+// CPU statement of the same definitions (readings R1-R14 of the oracle package),
 // which the tests hold bit for bit against the numpy oracle. Only tests/, the
 // smoke test and the benchmark's CPU baseline may load it; it shares no code with
 // the CUDA library. Plain loops, one (batch, head) slice at a time, in the order
@@ -425,6 +425,18 @@ void orc_quant_blocks_e4m3(const float* X, int S, int D, const int* order, uint8
     for (int p = p0; p < p1; ++p)
       for (int d = 0; d < D; ++d) codes[(size_t)p * D + d] = e4m3_code(X[(size_t)(order ? order[p] : p) * D + d] * inv);
   }
+}
+
+// R11: the per-channel token mean of one slice (int64 sum of llrint(x 2^24), one
+// fp64 division, rounded to fp32) and K - kbar in fp32 (xs: S x D, written).
+void orc_smooth_k(const float* K, int S, int D, float* kbar, float* xs) {
+  for (int d = 0; d < D; ++d) {
+    int64_t s = 0;
+    for (int j = 0; j < S; ++j) s += fix(K[(size_t)j * D + d]);
+    kbar[d] = (float)(((double)s * ldexp(1.0, -kFixShift)) / (double)S);
+  }
+  for (int j = 0; j < S; ++j)
+    for (int d = 0; d < D; ++d) xs[(size_t)j * D + d] = K[(size_t)j * D + d] - kbar[d];
 }
 
 // R8: kappa = fl32(softmax_scale log2 e).

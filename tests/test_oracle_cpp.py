@@ -22,6 +22,13 @@ def lib():
     return C.load()
 
 
+def torch_free_bf16(x):
+    """Round fp32 values to bf16 (ties to even) with integer arithmetic."""
+    b = np.asarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
+    return b.astype(np.uint32).view(np.float32)
+
+
 def _slice(name, b=0, h=0, **kw):
     cfg, Q, K, V = synth.make_workload(name, **kw)
     f = lambda X: X[b, :, h].float().numpy()
@@ -98,6 +105,20 @@ def test_repair_planes_and_energy(budget):
     assert sv_c == sv_o
     e_c, e_o = C.residual_energy(V, perm, mu), O.residual_energy(V, perm, mu)
     assert abs(e_c - e_o) <= 1e-12 * e_o
+
+
+def test_smooth_k_and_its_codes():
+    cfg, Q, K, V = _slice("mid", B=1, H=1, S=1000)
+    K = K + np.float32(3.0) * np.arange(128, dtype=np.float32)[None, :] / 128.0
+    K = np.asarray(torch_free_bf16(K))
+    xs_c, kb_c = C.smooth_k(K)
+    xs_o, kb_o = O.smooth_k(K)
+    assert np.array_equal(kb_c.view(np.uint32), kb_o.view(np.uint32))
+    assert np.array_equal(xs_c.view(np.uint32), xs_o.view(np.uint32))
+    perm = np.random.default_rng(2).permutation(1000).astype(np.int32)
+    cc, scc = C.quant_blocks_e4m3(xs_c, perm)
+    _, _, kc, ks = O.quant_qk_head(Q, K, perm, smooth=True)
+    assert np.array_equal(cc, kc) and np.array_equal(scc.view(np.uint32), ks.view(np.uint32))
 
 
 def test_zero_slice_and_zero_block():
